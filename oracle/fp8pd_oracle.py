@@ -1,0 +1,255 @@
+"""Plain CPU oracle for FP8 (E4M3) paged decode attention and KV append.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import this module:
+only the tests, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` call it. It shares no code with the
+CUDA library; it is a slow, literal restatement of what the method computes.
+
+Sources (the pages this restates):
+
+* P1 = "How do I run paged decode attention over an FP8 KV cache for a
+  quantized MoE serving path, with sliding windows, attention sinks and a
+  custom scale?" (cerinamroth.com solution page for ``fp8_paged_decode_attention``).
+* P2 = "Lecture 8 -- Inference Path: KV Cache, Decode, RoPE, GQA, Paged KV"
+  (FlashAttention Course).
+* E4M3 itself is only named by the pages; its values are those of the OCP
+  8-bit floating point format E4M3 (1 sign bit, 4 exponent bits with bias 7,
+  3 mantissa bits, subnormals, no infinities, S.1111.111 is NaN).
+
+Arithmetic is float64 except where the method fixes the precision: the
+quantizer divides in IEEE float32 (the stored code is a function of the
+float32 quotient), then rounds that quotient to the E4M3 grid exactly.
+
+Readings of the pages (each is listed with its reason in the design notes):
+
+* window W > 0 keeps the last W keys, i.e. positions t with t > (L-1) - W;
+  W = 0 keeps all keys (P1 "Expected result": ``window=W`` restricts each
+  query to the last W keys).
+* a sink is one extra logit per query head, in the same units as the scaled
+  scores, added to the softmax denominator with no value (P1 "Expected
+  result", the gpt-oss ``s_aux`` convention).
+* ``sm_scale`` multiplies q.k and replaces D**-0.5 (P1 "Expected result").
+* query head h uses KV head h // G, G = Hq / Hkv (P1 "Smallest correct
+  example", ``q.view(H_KV, H_Q // H_KV, D)``; P2 "MQA / GQA").
+* token t of sequence b lives in physical page block_table[b, t // ps] at
+  slot t % ps (P2 "Paged KV cache").
+* a K/V scale is indexed by the physical page id and the KV head; a
+  per-KV-head scale is the same array broadcast over pages.
+* empty attention (no keys, no sink) returns 0.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+E4M3_MAX = 448.0
+E4M3_NAN_CODE = 0x7F
+
+
+# ---------------------------------------------------------------------------
+# E4M3 codec
+# ---------------------------------------------------------------------------
+
+def e4m3_code_value(code: int) -> float:
+    """Value of one E4M3 code from the format's closed form (OCP E4M3).
+
+    sign s = bit 7, exponent e = bits 6..3 (bias 7), mantissa m = bits 2..0:
+      e == 0            -> (-1)^s * (m / 8) * 2^(1 - 7)      (subnormal)
+      e == 15, m == 7   -> NaN
+      otherwise         -> (-1)^s * (1 + m / 8) * 2^(e - 7)
+    """
+    s = (code >> 7) & 1
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 15 and m == 7:
+        return math.nan
+    if e == 0:
+        mag = (m / 8.0) * 2.0 ** (1 - 7)
+    else:
+        mag = (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return -mag if s else mag
+
+
+#: float64 value of every code 0..255 (NaN for 0x7F and 0xFF).
+E4M3_TABLE = np.array([e4m3_code_value(c) for c in range(256)], dtype=np.float64)
+
+#: the 127 non-negative finite values, codes 0x00..0x7E, strictly increasing.
+_E4M3_POS = E4M3_TABLE[:0x7F].copy()
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Decode uint8 E4M3 codes to float64 values."""
+    return E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
+
+
+def e4m3_encode(values) -> np.ndarray:
+    """Round real values to E4M3 codes: nearest grid value, ties to an even
+    mantissa, saturating to +-448.
+
+    The grid in the binade [2^e, 2^(e+1)) for e >= -6 has spacing 2^(e-3);
+    below 2^-6 (subnormals) the spacing is 2^-9, the same as the e = -6
+    binade, so the spacing is 2^(max(e, -6) - 3) everywhere. A value divided
+    by its spacing is exact (power of two), and rounding that quotient to the
+    nearest integer with ties to even picks the neighbour whose code has an
+    even mantissa. A result above 448 (including +-Inf) saturates to 448.
+    NaN maps to the NaN code with the input's sign; -0 keeps its sign.
+    """
+    v = np.asarray(values, dtype=np.float64)
+    flat = v.reshape(-1)
+    out = np.empty(flat.shape, dtype=np.uint8)
+    sign = np.signbit(flat)
+    a = np.abs(flat)
+    is_nan = np.isnan(flat)
+    finite = np.isfinite(a)
+
+    mag = np.full(flat.shape, E4M3_MAX)          # Inf and huge values saturate
+    af = np.where(finite & ~is_nan, a, 0.0)
+    _, ex = np.frexp(af)                          # af = f * 2^ex, f in [0.5, 1)
+    e = np.maximum(ex - 1, -6)                    # binade exponent, floored at -6
+    spacing = np.ldexp(1.0, e - 3)
+    r = np.rint(af / spacing)                     # round half to even
+    rounded = r * spacing
+    sel = finite & ~is_nan
+    mag[sel] = np.minimum(rounded[sel], E4M3_MAX)
+
+    idx = np.searchsorted(_E4M3_POS, mag)
+    idx = np.minimum(idx, 0x7E)
+    if not np.all(_E4M3_POS[idx[sel | ~finite]] == mag[sel | ~finite]):
+        raise AssertionError("e4m3_encode: rounded value is not on the grid")
+    out[:] = idx.astype(np.uint8)
+    out[is_nan] = E4M3_NAN_CODE
+    out |= (sign.astype(np.uint8) << 7)
+    return out.reshape(v.shape)
+
+
+def quantize(x, scale) -> np.ndarray:
+    """E4M3 code of x / scale, the quotient taken in IEEE float32.
+
+    ``x`` holds bf16 or float32 values (exact in float32); ``scale`` is a
+    float32 array broadcastable to ``x``. The division is float32
+    round-to-nearest (numpy float32 division; no flush to zero), then the
+    float32 quotient is rounded to E4M3 exactly by :func:`e4m3_encode`.
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    s32 = np.asarray(scale, dtype=np.float32)
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
+        quot = np.divide(x32, s32, dtype=np.float32)
+    return e4m3_encode(quot.astype(np.float64))
+
+
+# ---------------------------------------------------------------------------
+# Paged gather, attention and append
+# ---------------------------------------------------------------------------
+
+def _scale_of(scale: np.ndarray, page: np.ndarray, head: int) -> np.ndarray:
+    """Scale for (physical page, KV head): ``scale`` is [Hkv] (per KV head)
+    or [num_pages, Hkv] (per physical page and KV head)."""
+    scale = np.asarray(scale)
+    if scale.ndim == 1:
+        return np.full(np.shape(page), np.float64(scale[head]))
+    return scale[page, head].astype(np.float64)
+
+
+def gather_tokens(pages: np.ndarray, block_table_row: np.ndarray, positions: np.ndarray,
+                  head: int) -> tuple[np.ndarray, np.ndarray]:
+    """Codes of KV head ``head`` at logical token ``positions`` of one sequence.
+
+    ``pages`` is the layer's view [num_pages, ps, Hkv, D] of the pool (any
+    strides). Token t is in physical page block_table_row[t // ps], slot
+    t % ps. Returns (codes [n, D] uint8, physical page of each token [n]).
+    """
+    ps = pages.shape[1]
+    phys = np.asarray(block_table_row)[positions // ps].astype(np.int64)
+    slots = positions % ps
+    return pages[phys, slots, head, :], phys
+
+
+def attended_range(seq_len: int, window: int) -> tuple[int, int]:
+    """Keys [lo, L) a decode query at position L-1 attends to."""
+    L = int(seq_len)
+    lo = max(0, L - int(window)) if window > 0 else 0
+    return lo, L
+
+
+def paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens,
+                           window: int = 0, sinks=None, sm_scale: float | None = None,
+                           batch_heads=None) -> np.ndarray:
+    """Single-query attention over a paged E4M3 KV cache, float64.
+
+    q [B, Hq, D] (bf16 values given as floats), k_pages / v_pages
+    [num_pages, ps, Hkv, D] uint8 codes, k_scale / v_scale [Hkv] or
+    [num_pages, Hkv] float32, block_table [B, max_pages] int32,
+    seq_lens [B] = number of keys 0..L-1 visible to the query,
+    sinks [Hq] float32 or None. Returns out [B, Hq, D] float64.
+
+    For each (b, hq), with h = hq // G and keys t in [lo, L):
+      s_t  = sm_scale * sum_d q[b,hq,d] * K(t,d)
+      M    = max(max_t s_t, sink)
+      out  = sum_t exp(s_t - M) V(t) / (sum_t exp(s_t - M) + exp(sink - M))
+    where K(t,d) = decode(code) * k_scale(page(t), h). This is plain softmax
+    attention over the dequantized values (P1 "Smallest correct example"),
+    with the window, sinks and scale of P1 "Expected result".
+
+    ``batch_heads``: optional list of (b, hq) pairs; only those outputs are
+    computed (the others stay 0), for sampled checks at full size.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, D = q.shape
+    Hkv = k_pages.shape[2]
+    G = Hq // Hkv
+    if sm_scale is None:
+        sm_scale = D ** -0.5
+    sm = float(np.float32(sm_scale))
+    out = np.zeros((B, Hq, D), dtype=np.float64)
+    if batch_heads is None:
+        wanted = {(b, hq) for b in range(B) for hq in range(Hq)}
+    else:
+        wanted = {(int(b), int(hq)) for b, hq in batch_heads}
+    for b in range(B):
+        lo, L = attended_range(int(seq_lens[b]), int(window))
+        positions = np.arange(lo, L, dtype=np.int64)
+        for h in range(Hkv):
+            heads = [h * G + g for g in range(G) if (b, h * G + g) in wanted]
+            if not heads:
+                continue
+            kc, phys = gather_tokens(k_pages, block_table[b], positions, h)
+            vc, _ = gather_tokens(v_pages, block_table[b], positions, h)
+            K = e4m3_decode(kc) * _scale_of(k_scale, phys, h)[:, None]
+            V = e4m3_decode(vc) * _scale_of(v_scale, phys, h)[:, None]
+            for hq in heads:
+                s = sm * (K @ q[b, hq])
+                sink = None if sinks is None else float(sinks[hq])
+                m_keys = s.max() if s.size else -math.inf
+                M = m_keys if sink is None else max(m_keys, sink)
+                if M == -math.inf:
+                    continue                       # no keys and no finite sink: 0
+                w = np.exp(s - M)
+                den = w.sum() + (0.0 if sink is None else math.exp(sink - M))
+                if den > 0.0:
+                    out[b, hq] = (w @ V) / den
+    return out
+
+
+def kv_append(k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table, positions) -> None:
+    """Quantize one new token per sequence and store it in its page, in place.
+
+    k_new / v_new [B, Hkv, D] (bf16 values as floats), pages
+    [num_pages, ps, Hkv, D] uint8 (numpy arrays, written in place), scales
+    [Hkv] or [num_pages, Hkv] float32 (read only), positions [B].
+    Token position p of sequence b goes to page block_table[b, p // ps], slot
+    p % ps, as code = E4M3(float32(x) / scale(page, h)) (P1 "Supported scope",
+    the one-launch T=1 append; P2 "In-kernel KV cache update").
+    """
+    B, Hkv, _ = np.shape(k_new)
+    ps = k_pages.shape[1]
+    for b in range(B):
+        p = int(positions[b])
+        page = int(block_table[b][p // ps])
+        slot = p % ps
+        for h in range(Hkv):
+            ks = _scale_of(k_scale, np.array(page), h)
+            vs = _scale_of(v_scale, np.array(page), h)
+            k_pages[page, slot, h, :] = quantize(np.asarray(k_new[b][h], np.float32), np.float32(ks))
+            v_pages[page, slot, h, :] = quantize(np.asarray(v_new[b][h], np.float32), np.float32(vs))

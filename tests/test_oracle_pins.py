@@ -1,0 +1,421 @@
+"""Pins for the float64 CPU oracle, checked against things other than itself:
+the E4M3 format's published limits, a library implementation of the format
+(PyTorch ``float8_e4m3fn``), brute force, a library attention routine
+(``scaled_dot_product_attention`` in float64), closed forms and invariants.
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _anchors():
+    rows = []
+    with open(os.path.join(GOLDEN, "e4m3_anchors.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            c, v = line.split()
+            rows.append((int(c, 16), float(v)))
+    return rows
+
+
+# ---------------------------------------------------------------- E4M3 decode
+
+def test_decode_anchor_values():
+    for code, want in _anchors():
+        got = O.e4m3_decode(np.array([code]))[0]
+        if math.isnan(want):
+            assert math.isnan(got), hex(code)
+        else:
+            assert got == want, (hex(code), got, want)
+            assert math.copysign(1.0, got) == math.copysign(1.0, want), hex(code)
+
+
+def test_decode_matches_library_float8_for_all_256_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    ours = O.e4m3_decode(codes)
+    assert np.array_equal(ours, lib, equal_nan=True)
+
+
+def test_decode_structure():
+    v = O.e4m3_decode(np.arange(256, dtype=np.uint8))
+    pos = v[:0x7F]
+    assert np.all(np.diff(pos) > 0)                       # strictly increasing 0x00..0x7E
+    assert np.array_equal(v[0x80:0xFF], -pos)             # sign symmetry
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF])
+    assert np.isfinite(v).sum() == 254
+    # constant spacing inside each binade: 2^-9 for subnormals and [2^-6, 2^-5)
+    for e in range(-6, 9):
+        inb = pos[(pos >= 2.0 ** e) & (pos < 2.0 ** (e + 1))]
+        assert np.allclose(np.diff(inb), 2.0 ** (e - 3), rtol=0, atol=0)
+    sub = pos[pos < 2.0 ** -6]
+    assert np.array_equal(sub, np.arange(8) * 2.0 ** -9)
+
+
+# ---------------------------------------------------------------- E4M3 encode
+
+def test_encode_roundtrip_finite_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    v = O.e4m3_decode(codes)
+    fin = np.isfinite(v)
+    assert np.array_equal(O.e4m3_encode(v[fin]), codes[fin])
+
+
+def test_encode_midpoints_go_to_even_mantissa():
+    pos = O.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    mids = (pos[:-1] + pos[1:]) / 2
+    got = O.e4m3_encode(mids)
+    lower = np.arange(0x7E)
+    want = np.where(lower % 2 == 0, lower, lower + 1)
+    assert np.array_equal(got, want.astype(np.uint8))
+    # a hair either side of every midpoint goes to the nearer neighbour
+    eps = np.spacing(mids) * 4
+    assert np.array_equal(O.e4m3_encode(mids - eps), lower.astype(np.uint8))
+    assert np.array_equal(O.e4m3_encode(mids + eps), (lower + 1).astype(np.uint8))
+    assert np.array_equal(O.e4m3_encode(-mids), (want | 0x80).astype(np.uint8))
+
+
+def test_encode_special_values():
+    cases = [
+        (448.0, 0x7E), (449.0, 0x7E), (464.0, 0x7E), (465.0, 0x7E), (1e30, 0x7E), (math.inf, 0x7E),
+        (-math.inf, 0xFE), (-1e30, 0xFE), (0.0, 0x00), (-0.0, 0x80),
+        (2.0 ** -10, 0x00),            # tie between 0 and 2^-9 -> even (0)
+        (3 * 2.0 ** -11, 0x01),        # nearer 2^-9
+        (2.0 ** -12, 0x00),
+        (-(2.0 ** -9), 0x81),
+    ]
+    got = O.e4m3_encode(np.array([x for x, _ in cases]))
+    assert [int(g) for g in got] == [c for _, c in cases]
+    n = O.e4m3_encode(np.array([math.nan, -math.nan]))
+    assert n[0] == 0x7F and n[1] == 0xFF
+
+
+def test_encode_matches_brute_force_nearest():
+    rng = np.random.default_rng(11)
+    x = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 1e-1, 1.0, 30.0, 150.0)])
+    x = x[np.abs(x) < 448]
+    grid = O.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    got = O.e4m3_encode(x)
+    for xi, gi in zip(x[:5000], got[:5000]):
+        a = abs(xi)
+        d = np.abs(grid - a)
+        best = np.flatnonzero(d == d.min())
+        code = best[0] if len(best) == 1 else [c for c in best if c % 2 == 0][0]
+        if xi < 0 or (xi == 0 and math.copysign(1, xi) < 0):
+            code |= 0x80
+        assert gi == code, (xi, gi, code)
+
+
+def test_encode_matches_library_float8_for_float32_inputs():
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.standard_normal(200000) * s for s in (1e-4, 1e-2, 1.0, 100.0)])
+    x = x.astype(np.float32)
+    x = x[np.abs(x) <= 464]
+    lib = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(x.astype(np.float64)), lib)
+
+
+def test_quantize_all_bf16_inputs_match_library_path():
+    """Every bf16 bit pattern, several scales: float32 division, then E4M3.
+    The library path (torch float32 division, float8 cast) agrees wherever the
+    quotient is <= 464; above that the library gives NaN where E4M3
+    quantization saturates to +-448."""
+    bits = np.arange(65536, dtype=np.uint32) << 16
+    x = bits.view(np.float32)
+    for scale in (1.0, 0.5, 4.0 / 448, 3.0 / 448, 1e-3, 2.0 ** -20, 1e6, 37.0 / 448):
+        s = np.float32(scale)
+        ours = O.quantize(x, s)
+        xt = torch.from_numpy(x.copy())
+        quot = (xt / torch.tensor(s)).numpy()
+        lib = torch.from_numpy(quot).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        ok = np.isfinite(quot) & (np.abs(quot) <= 464)
+        assert np.array_equal(ours[ok], lib[ok]), scale
+        big = np.isfinite(quot) & (np.abs(quot) > 464) | np.isinf(quot)
+        assert np.all((ours[big] & 0x7F) == 0x7E)
+        assert np.all((ours[np.isnan(quot)] & 0x7F) == 0x7F)
+
+
+def test_quantize_divides_in_float32():
+    """The code is a function of the float32 quotient: aim x / s just below a
+    midpoint whose lower neighbour has an odd mantissa. In float64 the quotient
+    rounds down; in float32 it rounds onto the midpoint, which then goes to the
+    even (upper) code. The oracle must give the float32 answer."""
+    pos = O.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    rng = np.random.default_rng(3)
+    found = 0
+    for c in range(9, 0x7D, 2):                      # odd lower neighbour
+        m = (pos[c] + pos[c + 1]) / 2
+        for s in rng.uniform(0.001, 0.05, 400).astype(np.float32):
+            x = np.float32(m * float(s))
+            q64 = float(x) / float(s)
+            q32 = float(np.float32(x) / s)
+            if q32 == m and q64 < m:
+                assert O.e4m3_encode(np.array([q64]))[0] == c
+                assert O.quantize(np.array([x]), s)[0] == c + 1
+                found += 1
+                break
+    assert found > 20
+
+
+# ---------------------------------------------------------------- attention
+
+def _dense_case(rng, B=2, Hq=8, Hkv=2, D=16, ps=16, L=(37, 50), scale_mode="page",
+                permute=True, extra_pages=3):
+    lens = np.array([L[b % len(L)] for b in range(B)])
+    npg = (lens + ps - 1) // ps
+    total = int(npg.sum()) + extra_pages
+    perm = rng.permutation(total) if permute else np.arange(total)
+    table = np.full((B, npg.max()), -1, np.int32)
+    off = 0
+    for b in range(B):
+        table[b, :npg[b]] = perm[off:off + npg[b]]
+        off += npg[b]
+    k = rng.integers(0, 256, size=(total, ps, Hkv, D)).astype(np.uint8)
+    v = rng.integers(0, 256, size=(total, ps, Hkv, D)).astype(np.uint8)
+    k[(k & 0x7F) == 0x7F] = 0x10                                 # no NaN codes
+    v[(v & 0x7F) == 0x7F] = 0x21
+    if scale_mode == "page":
+        ks = rng.uniform(0.001, 0.02, size=(total, Hkv)).astype(np.float32)
+        vs = rng.uniform(0.001, 0.02, size=(total, Hkv)).astype(np.float32)
+    else:
+        ks = rng.uniform(0.001, 0.02, size=Hkv).astype(np.float32)
+        vs = rng.uniform(0.001, 0.02, size=Hkv).astype(np.float32)
+    q = torch.randn(B, Hq, D, generator=torch.Generator().manual_seed(int(rng.integers(1 << 30))))
+    q = q.to(torch.bfloat16).double().numpy()
+    return dict(q=q, k=k, v=v, ks=ks, vs=vs, table=table, lens=lens)
+
+
+def _sdpa_reference(c, window, sinks, sm_scale):
+    """Library attention (torch SDPA, float64) over the dequantized keys,
+    with KV heads repeated G times, the window as an additive mask, and a
+    sink as one extra key with a zero value and logit = sink."""
+    q, k, v, ks, vs, table, lens = (c[n] for n in ("q", "k", "v", "ks", "vs", "table", "lens"))
+    B, Hq, D = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    ps = k.shape[1]
+    out = np.zeros((B, Hq, D))
+    for b in range(B):
+        L = int(lens[b])
+        t = np.arange(L)
+        phys = table[b][t // ps]
+        K = np.zeros((Hq, L + 1, D))
+        V = np.zeros((Hq, L + 1, D))
+        for hq in range(Hq):
+            h = hq // G
+            kscale = ks[phys, h] if ks.ndim == 2 else np.full(L, ks[h])
+            vscale = vs[phys, h] if vs.ndim == 2 else np.full(L, vs[h])
+            K[hq, :L] = torch.from_numpy(k[phys, t % ps, h]).view(torch.float8_e4m3fn).double().numpy() \
+                * kscale[:, None]
+            V[hq, :L] = torch.from_numpy(v[phys, t % ps, h]).view(torch.float8_e4m3fn).double().numpy() \
+                * vscale[:, None]
+        mask = np.zeros((Hq, 1, L + 1))
+        if window > 0:
+            mask[:, :, :max(0, L - window)] = -np.inf
+        mask[:, :, L] = -np.inf if sinks is None else sinks[:, None]
+        o = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[b][:, None, :]), torch.from_numpy(K), torch.from_numpy(V),
+            attn_mask=torch.from_numpy(mask), scale=float(np.float32(sm_scale)))
+        out[b] = o[:, 0, :].numpy()
+    return out
+
+
+def _run(c, **kw):
+    return O.paged_decode_attention(c["q"], c["k"], c["v"], c["ks"], c["vs"], c["table"],
+                                    c["lens"], **kw)
+
+
+@pytest.mark.parametrize("window,with_sinks,scale_mode",
+                         [(0, False, "page"), (0, True, "head"), (20, False, "head"), (7, True, "page")])
+def test_attention_matches_library_sdpa(window, with_sinks, scale_mode):
+    rng = np.random.default_rng(100 + window)
+    c = _dense_case(rng, scale_mode=scale_mode)
+    sinks = rng.standard_normal(8).astype(np.float32) if with_sinks else None
+    sm = 0.3
+    got = _run(c, window=window, sinks=sinks, sm_scale=sm)
+    want = _sdpa_reference(c, window, sinks, sm)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_paged_equals_contiguous():
+    rng = np.random.default_rng(7)
+    c = _dense_case(rng, B=1, L=(53,), permute=True, extra_pages=0)
+    # contiguous copy: logical page i stored at physical page i
+    ps = c["k"].shape[1]
+    n = c["table"].shape[1]
+    k2 = c["k"][c["table"][0]]
+    v2 = c["v"][c["table"][0]]
+    ks2 = c["ks"][c["table"][0]]
+    vs2 = c["vs"][c["table"][0]]
+    c2 = dict(c, k=k2, v=v2, ks=ks2, vs=vs2, table=np.arange(n, dtype=np.int32)[None])
+    a = _run(c, window=0)
+    b = _run(c2, window=0)
+    assert np.array_equal(a, b)
+    assert ps == 16
+
+
+def test_gqa_equals_repeated_kv_heads():
+    rng = np.random.default_rng(8)
+    c = _dense_case(rng, Hq=8, Hkv=2)
+    G = 4
+    rep = dict(c, k=np.repeat(c["k"], G, axis=2), v=np.repeat(c["v"], G, axis=2),
+               ks=np.repeat(c["ks"], G, axis=1), vs=np.repeat(c["vs"], G, axis=1))
+    assert np.array_equal(_run(c, window=0), _run(rep, window=0))
+
+
+def test_minus_inf_sink_equals_no_sink_and_infinite_window_equals_full():
+    rng = np.random.default_rng(9)
+    c = _dense_case(rng)
+    base = _run(c, window=0)
+    assert np.array_equal(_run(c, window=0, sinks=np.full(8, -np.inf, np.float32)), base)
+    assert np.array_equal(_run(c, window=int(c["lens"].max())), base)
+    assert np.array_equal(_run(c, window=10 ** 6), base)
+
+
+def test_closed_forms_zero_query_and_single_key():
+    rng = np.random.default_rng(10)
+    c = _dense_case(rng, scale_mode="head")
+    c0 = dict(c, q=np.zeros_like(c["q"]))
+    ps = c["k"].shape[1]
+    G = 4
+    for window, sinks in ((0, None), (9, np.linspace(-1, 1, 8).astype(np.float32))):
+        got = _run(c0, window=window, sinks=sinks)
+        for b in range(2):
+            L = int(c["lens"][b])
+            lo = max(0, L - window) if window else 0
+            t = np.arange(lo, L)
+            phys = c["table"][b][t // ps]
+            for hq in range(8):
+                h = hq // G
+                V = O.e4m3_decode(c["v"][phys, t % ps, h]) * float(c["vs"][h])
+                den = len(t) + (0.0 if sinks is None else math.exp(float(sinks[hq])))
+                assert np.allclose(got[b, hq], V.sum(0) / den, rtol=1e-13, atol=1e-15)
+    c1 = dict(c, lens=np.array([1, 1]))
+    got = _run(c1, window=0)
+    for b in range(2):
+        p = c["table"][b][0]
+        for hq in range(8):
+            assert np.array_equal(got[b, hq], O.e4m3_decode(c["v"][p, 0, hq // G]) * float(c["vs"][hq // G]))
+
+
+def test_empty_sequence_gives_zero():
+    rng = np.random.default_rng(12)
+    c = dict(_dense_case(rng), lens=np.array([0, 0]))
+    assert np.array_equal(_run(c, window=0), np.zeros((2, 8, 16)))
+    assert np.array_equal(_run(c, window=0, sinks=np.ones(8, np.float32)), np.zeros((2, 8, 16)))
+
+
+def test_brute_force_tiny_inputs():
+    """Naive softmax without max subtraction, in pure Python, on tiny inputs."""
+    rng = np.random.default_rng(13)
+    for trial in range(20):
+        D = int(rng.integers(1, 9))
+        L = int(rng.integers(1, 9))
+        c = _dense_case(rng, B=1, Hq=2, Hkv=1, D=D, ps=16, L=(L,), scale_mode="page")
+        window = int(rng.integers(0, L + 2))
+        sinks = rng.standard_normal(2).astype(np.float32) if trial % 2 else None
+        sm = float(np.float32(rng.uniform(0.05, 0.5)))
+        got = _run(c, window=window, sinks=sinks, sm_scale=sm)
+        for hq in range(2):
+            lo = max(0, L - window) if window else 0
+            num = [0.0] * D
+            den = 0.0 if sinks is None else math.exp(float(sinks[hq]))
+            for t in range(lo, L):
+                p = int(c["table"][0][t // 16])
+                kv = [e4m3(int(c["k"][p, t % 16, 0, d])) * float(c["ks"][p, 0]) for d in range(D)]
+                vv = [e4m3(int(c["v"][p, t % 16, 0, d])) * float(c["vs"][p, 0]) for d in range(D)]
+                s = sm * sum(float(c["q"][0, hq, d]) * kv[d] for d in range(D))
+                w = math.exp(s)
+                den += w
+                for d in range(D):
+                    num[d] += w * vv[d]
+            want = [x / den for x in num] if den > 0 else [0.0] * D
+            assert np.allclose(got[0, hq], want, rtol=1e-12, atol=1e-14)
+
+
+def e4m3(code: int) -> float:
+    """Tiny independent E4M3 reading through the library float8 type."""
+    return float(torch.tensor([code], dtype=torch.uint8).view(torch.float8_e4m3fn).double()[0])
+
+
+def test_page1_worked_example_shape():
+    """The paged oracle reproduces plain softmax attention over dequantized
+    K/V for the worked example's shape (16-token blocks, GQA 2:1, 40 tokens,
+    block table [2, 0, 1]); per-(page, head) scales from the oracle quantizer."""
+    spec = {}
+    with open(os.path.join(GOLDEN, "page1_worked_example.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                k, *v = line.split()
+                spec[k] = v
+    BT, HKV, HQ, D, T = (int(spec[k][0]) for k in
+                         ("block_tokens", "n_kv_heads", "n_q_heads", "head_dim", "live_tokens"))
+    table = np.array([[int(x) for x in spec["block_table"]]], np.int32)
+    n_blk = (T + BT - 1) // BT
+    g = torch.Generator().manual_seed(0)
+    kt = torch.randn(n_blk * BT, HKV, D, generator=g).numpy().astype(np.float32)
+    vt = torch.randn(n_blk * BT, HKV, D, generator=g).numpy().astype(np.float32)
+    kp = np.zeros((n_blk, BT, HKV, D), np.uint8)
+    vp = np.zeros_like(kp)
+    ks = np.zeros((n_blk, HKV), np.float32)
+    vs = np.zeros_like(ks)
+    for i in range(n_blk):
+        r = table[0, i]
+        blk_k, blk_v = kt[i * BT:(i + 1) * BT], vt[i * BT:(i + 1) * BT]
+        ks[r] = np.abs(blk_k).max(axis=(0, 2)) / np.float32(448)
+        vs[r] = np.abs(blk_v).max(axis=(0, 2)) / np.float32(448)
+        kp[r] = O.quantize(blk_k, ks[r][None, :, None])
+        vp[r] = O.quantize(blk_v, vs[r][None, :, None])
+    q = torch.randn(1, HQ, D, generator=g).to(torch.bfloat16).double().numpy()
+    out = O.paged_decode_attention(q, kp, vp, ks, vs, table, np.array([T]), window=0)
+    # plain attention over the dequantized values, in logical order
+    kd = np.concatenate([O.e4m3_decode(kp[table[0, i]]) * ks[table[0, i]][None, :, None]
+                         for i in range(n_blk)])[:T].transpose(1, 0, 2)
+    vd = np.concatenate([O.e4m3_decode(vp[table[0, i]]) * vs[table[0, i]][None, :, None]
+                         for i in range(n_blk)])[:T].transpose(1, 0, 2)
+    qq = q[0].reshape(HKV, HQ // HKV, D)
+    w = torch.softmax(torch.einsum("hgd,htd->hgt", torch.from_numpy(qq), torch.from_numpy(kd)) * D ** -0.5,
+                      dim=-1)
+    want = torch.einsum("hgt,htd->hgd", w, torch.from_numpy(vd)).reshape(1, HQ, D).numpy()
+    assert np.allclose(out, want, rtol=1e-12, atol=1e-12)
+    # the dequantized values are within E4M3 rounding of the originals
+    assert np.all(np.abs(kd.transpose(1, 0, 2) - kt[:T]) <= np.abs(kt[:T]) / 16 + 2.0 ** -10)
+    assert float(spec["tolerance"][0]) == 1e-2
+
+
+# ---------------------------------------------------------------- append
+
+def test_append_writes_only_the_new_slot():
+    rng = np.random.default_rng(14)
+    num_pages, ps, Hkv, D, B = 12, 16, 2, 32, 3
+    kp = rng.integers(0, 256, (num_pages, ps, Hkv, D)).astype(np.uint8)
+    vp = rng.integers(0, 256, (num_pages, ps, Hkv, D)).astype(np.uint8)
+    k0, v0 = kp.copy(), vp.copy()
+    table = rng.permutation(num_pages)[:B * 4].reshape(B, 4).astype(np.int32)
+    pos = np.array([0, 17, 63])
+    ks = rng.uniform(0.005, 0.02, (num_pages, Hkv)).astype(np.float32)
+    vs = rng.uniform(0.005, 0.02, Hkv).astype(np.float32)
+    kn = torch.randn(B, Hkv, D).to(torch.bfloat16).float().numpy()
+    vn = torch.randn(B, Hkv, D).to(torch.bfloat16).float().numpy()
+    O.kv_append(kn, vn, kp, vp, ks, vs, table, pos)
+    touched = np.zeros((num_pages, ps), bool)
+    for b in range(B):
+        p, s = table[b, pos[b] // ps], pos[b] % ps
+        touched[p, s] = True
+        for h in range(Hkv):
+            want_k = torch.from_numpy(kn[b, h] / ks[p, h]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            want_v = torch.from_numpy(vn[b, h] / vs[h]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            assert np.array_equal(kp[p, s, h], want_k)
+            assert np.array_equal(vp[p, s, h], want_v)
+    assert np.array_equal(kp[~touched], k0[~touched])
+    assert np.array_equal(vp[~touched], v0[~touched])
