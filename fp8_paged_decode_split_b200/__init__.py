@@ -1,0 +1,228 @@
+"""FP8 (E4M3) paged split-KV decode attention for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over the C ABI in ``include/fp8pd.h``: it turns torch
+tensors into descriptors (pointer, dtype, shape, strides) and calls the
+library on the current CUDA stream. Every step of the computation runs in
+the library's CUDA kernels; there is no Python or CPU fallback. If the
+library is missing, importing this package raises ``ImportError``.
+
+Entry points (same names as the C ABI):
+
+* :func:`fp8_paged_decode_attention` -- decode attention over a paged E4M3
+  KV cache with GQA, an optional sliding window, optional sink logits and a
+  caller softmax scale.
+* :func:`fp8_kv_append` -- quantize one new bf16 K/V token per sequence to
+  E4M3 and store it in its page.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "fp8_paged_decode_attention", "fp8_kv_append", "fp8pd_plan", "fp8pd_reserve_workspace",
+    "fp8pd_check_errors", "fp8pd_set_option", "fp8pd_get_option", "fp8pd_last_run_info",
+    "fp8pd_timing_enable", "fp8pd_timing_collect", "Fp8pdError", "lib", "LIB_PATH",
+    "FLAG_PAGE_OOB", "FLAG_SEQLEN_OOB", "FLAG_POS_OOB", "OPT_NUM_SPLITS", "OPT_VARIANT",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libfp8pd.so")
+
+DTYPE_U8, DTYPE_I32, DTYPE_F32, DTYPE_BF16 = 1, 2, 3, 4
+FLAG_PAGE_OOB, FLAG_SEQLEN_OOB, FLAG_POS_OOB = 1, 2, 4
+OPT_NUM_SPLITS, OPT_VARIANT = 1, 2
+_DTYPES = {torch.uint8: DTYPE_U8, torch.int32: DTYPE_I32, torch.float32: DTYPE_F32,
+           torch.bfloat16: DTYPE_BF16}
+
+
+class Tensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+class Scales(ctypes.Structure):
+    _fields_ = [("k_scale", Tensor), ("v_scale", Tensor)]
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("num_splits", ctypes.c_int32), ("head_groups", ctypes.c_int32),
+                ("grid_blocks", ctypes.c_int32), ("combine", ctypes.c_int32),
+                ("workspace_bytes", ctypes.c_uint64)]
+
+
+class RunInfo(ctypes.Structure):
+    _fields_ = [("variant", ctypes.c_int32), ("num_splits", ctypes.c_int32),
+                ("head_groups", ctypes.c_int32), ("grid_blocks", ctypes.c_int32),
+                ("combine", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("calls", ctypes.c_int64), ("appends", ctypes.c_int64)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m fp8_paged_decode_split_b200._build` "
+            "(nvcc, sm_100a). There is no fallback implementation.")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER
+    T = P(Tensor)
+    i32, f32, vp = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p
+    lib.fp8_paged_decode_attention.argtypes = [T, T, T, T, T, T, T, i32, T, f32, T, vp]
+    lib.fp8_kv_append.argtypes = [T, T, T, T, P(Scales), T, T, vp]
+    lib.fp8pd_plan.argtypes = [T, T, T, i32, P(PlanInfo)]
+    lib.fp8pd_reserve_workspace.argtypes = [ctypes.c_uint64]
+    lib.fp8pd_check_errors.argtypes = [vp, P(ctypes.c_uint32)]
+    lib.fp8pd_set_option.argtypes = [i32, ctypes.c_int64]
+    lib.fp8pd_get_option.argtypes = [i32]
+    lib.fp8pd_get_option.restype = ctypes.c_int64
+    lib.fp8pd_last_run_info.argtypes = [P(RunInfo)]
+    lib.fp8pd_timing_enable.argtypes = [i32]
+    lib.fp8pd_timing_collect.argtypes = [P(ctypes.c_double), P(ctypes.c_double), P(i32), P(i32)]
+    lib.fp8pd_status_string.argtypes = [i32]
+    lib.fp8pd_status_string.restype = ctypes.c_char_p
+    lib.fp8pd_last_cuda_error.restype = i32
+    lib.fp8pd_version.restype = i32
+    for name in ("fp8_paged_decode_attention", "fp8_kv_append", "fp8pd_plan",
+                 "fp8pd_reserve_workspace", "fp8pd_check_errors", "fp8pd_set_option",
+                 "fp8pd_last_run_info", "fp8pd_timing_enable", "fp8pd_timing_collect"):
+        getattr(lib, name).restype = i32
+    return lib
+
+
+lib = _load()
+
+
+class Fp8pdError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = lib.fp8pd_status_string(status).decode()
+        if status == -9:
+            msg += f" (cudaError {lib.fp8pd_last_cuda_error()})"
+        super().__init__(f"{where}: status {status}: {msg}")
+        self.status = status
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise Fp8pdError(status, where)
+
+
+def describe(t: torch.Tensor | None) -> Tensor | None:
+    """Descriptor of a torch tensor (no copy; the tensor must outlive the call)."""
+    if t is None:
+        return None
+    if t.dim() > 4:
+        raise ValueError("at most 4 dimensions")
+    d = Tensor()
+    d.data = t.data_ptr()
+    d.dtype = _DTYPES.get(t.dtype, 0)
+    d.ndim = t.dim()
+    for i, (s, st) in enumerate(zip(t.shape, t.stride())):
+        d.shape[i] = s
+        d.stride[i] = st
+    return d
+
+
+def _same_device(*ts) -> None:
+    """All tensors on one CUDA device, or all on the host (which the library
+    then refuses during validation, before any CUDA call)."""
+    devs = {t.device for t in ts if t is not None}
+    if len(devs) > 1:
+        raise ValueError(f"tensors on different devices: {sorted(map(str, devs))}")
+
+
+def _ref(d: Tensor | None):
+    return ctypes.byref(d) if d is not None else None
+
+
+def _stream(stream, like: torch.Tensor | None = None) -> int:
+    if stream is None:
+        if like is not None and like.device.type != "cuda":
+            return 0  # host tensors: the library refuses them before any CUDA call
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def fp8_paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens,
+                               window: int = 0, sinks=None, sm_scale: float | None = None,
+                               out=None, stream=None) -> torch.Tensor:
+    """Decode attention over a paged E4M3 KV cache (see include/fp8pd.h).
+
+    q [B, Hq, D] bf16; k_pages / v_pages [num_pages, ps, Hkv, D] uint8 views
+    (any page stride that is a multiple of 16 bytes); k_scale / v_scale
+    float32 [Hkv] or [num_pages, Hkv]; block_table int32 [B, max_pages];
+    seq_lens int32 [B] (keys visible to the query); sinks float32 [Hq] or
+    None; sm_scale defaults to D ** -0.5. Returns out [B, Hq, D] float32.
+    """
+    if sm_scale is None:
+        sm_scale = q.shape[-1] ** -0.5
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    _same_device(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens, sinks, out)
+    ds = [describe(t) for t in (q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens)]
+    ds_sinks, ds_out = describe(sinks), describe(out)
+    st = lib.fp8_paged_decode_attention(*[_ref(d) for d in ds], int(window), _ref(ds_sinks),
+                                        float(sm_scale), _ref(ds_out), _stream(stream, q))
+    _check(st, "fp8_paged_decode_attention")
+    return out
+
+
+def fp8_kv_append(k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table, positions,
+                  stream=None) -> None:
+    """Quantize k_new / v_new [B, Hkv, D] bf16 to E4M3 and write them at
+    positions[b] of each sequence's pages (see include/fp8pd.h)."""
+    _same_device(k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table, positions)
+    sc = Scales()
+    sc.k_scale = describe(k_scale)
+    sc.v_scale = describe(v_scale)
+    ds = [describe(t) for t in (k_new, v_new, k_pages, v_pages)]
+    dt, dp = describe(block_table), describe(positions)
+    st = lib.fp8_kv_append(*[_ref(d) for d in ds], ctypes.byref(sc), _ref(dt), _ref(dp),
+                           _stream(stream, k_new))
+    _check(st, "fp8_kv_append")
+
+
+def fp8pd_plan(q, k_pages, block_table, window: int = 0) -> dict:
+    info = PlanInfo()
+    dq, dk, dt = describe(q), describe(k_pages), describe(block_table)
+    _check(lib.fp8pd_plan(_ref(dq), _ref(dk), _ref(dt), int(window), ctypes.byref(info)),
+           "fp8pd_plan")
+    return {f: getattr(info, f) for f, _ in PlanInfo._fields_}
+
+
+def fp8pd_reserve_workspace(nbytes: int) -> None:
+    _check(lib.fp8pd_reserve_workspace(int(nbytes)), "fp8pd_reserve_workspace")
+
+
+def fp8pd_check_errors(stream=None) -> int:
+    flags = ctypes.c_uint32(0)
+    _check(lib.fp8pd_check_errors(_stream(stream), ctypes.byref(flags)), "fp8pd_check_errors")
+    return int(flags.value)
+
+
+def fp8pd_set_option(option: int, value: int) -> None:
+    _check(lib.fp8pd_set_option(int(option), int(value)), "fp8pd_set_option")
+
+
+def fp8pd_get_option(option: int) -> int:
+    return int(lib.fp8pd_get_option(int(option)))
+
+
+def fp8pd_last_run_info() -> dict:
+    info = RunInfo()
+    _check(lib.fp8pd_last_run_info(ctypes.byref(info)), "fp8pd_last_run_info")
+    return {f: getattr(info, f) for f, _ in RunInfo._fields_}
+
+
+def fp8pd_timing_enable(on: bool) -> None:
+    _check(lib.fp8pd_timing_enable(1 if on else 0), "fp8pd_timing_enable")
+
+
+def fp8pd_timing_collect() -> dict:
+    a, b = ctypes.c_double(), ctypes.c_double()
+    na, nb = ctypes.c_int32(), ctypes.c_int32()
+    _check(lib.fp8pd_timing_collect(ctypes.byref(a), ctypes.byref(b), ctypes.byref(na),
+                                    ctypes.byref(nb)), "fp8pd_timing_collect")
+    return {"split_ms": a.value, "combine_ms": b.value, "split_launches": na.value,
+            "combine_launches": nb.value}

@@ -1,0 +1,546 @@
+// Host side of the C ABI declared in include/fp8pd.h: argument validation
+// (nothing is launched unless every check passes), split planning, the
+// per-device split workspace, options, run info and optional kernel timing.
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/fp8pd.h"
+#include "fp8pd_internal.h"
+
+using fp8pd::AppendParams;
+using fp8pd::DecodeParams;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+thread_local int32_t t_last_cuda_error = 0;
+thread_local fp8pd_run_info t_run_info = {};
+std::atomic<int64_t> g_calls{0}, g_appends{0};
+std::atomic<int64_t> g_opt_num_splits{0}, g_opt_variant{0};
+
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::mutex g_ws_mutex;
+Workspace g_ws[kMaxDevices];
+
+struct EventPair {
+  cudaEvent_t a = nullptr, b = nullptr;
+  int kind = 0;  // 0 = split kernel, 1 = combine kernel
+};
+std::mutex g_timing_mutex;
+std::atomic<int> g_timing_on{0};
+std::vector<EventPair> g_timing_pool;  // events of the current device(s)
+size_t g_timing_used = 0;
+
+int fail_cuda(cudaError_t e) {
+  t_last_cuda_error = static_cast<int32_t>(e);
+  return FP8PD_ERR_CUDA;
+}
+
+bool is_capturing(cudaStream_t s) {
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &st) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return st != cudaStreamCaptureStatusNone;
+}
+
+// ---- descriptor checks -------------------------------------------------------
+int check(const fp8pd_tensor* t, int32_t dtype, int32_t ndim) {
+  if (!t || !t->data) return FP8PD_ERR_NULL;
+  if (t->dtype != dtype) return FP8PD_ERR_DTYPE;
+  if (t->ndim != ndim) return FP8PD_ERR_SHAPE;
+  for (int i = 0; i < ndim; ++i)
+    if (t->shape[i] < 0) return FP8PD_ERR_SHAPE;
+  return FP8PD_OK;
+}
+
+bool fits_i32(int64_t v) { return v >= 0 && v <= INT32_MAX; }
+
+// Scale descriptor -> (page stride, head stride) in elements.
+int scale_strides(const fp8pd_tensor* s, int64_t num_pages, int64_t hkv, int64_t* sp, int64_t* sh) {
+  if (!s || !s->data) return FP8PD_ERR_NULL;
+  if (s->dtype != FP8PD_DTYPE_F32) return FP8PD_ERR_DTYPE;
+  if (s->ndim == 1) {
+    if (s->shape[0] != hkv) return FP8PD_ERR_SHAPE;
+    *sp = 0;
+    *sh = s->stride[0];
+    return FP8PD_OK;
+  }
+  if (s->ndim == 2) {
+    if (s->shape[0] != num_pages || s->shape[1] != hkv) return FP8PD_ERR_SHAPE;
+    *sp = s->stride[0];
+    *sh = s->stride[1];
+    return FP8PD_OK;
+  }
+  return FP8PD_ERR_SHAPE;
+}
+
+// Pool view [num_pages, ps, Hkv, D] of uint8 codes.
+int check_pool(const fp8pd_tensor* t, bool aligned) {
+  int r = check(t, FP8PD_DTYPE_U8, 4);
+  if (r) return r;
+  if (t->stride[3] != 1) return FP8PD_ERR_ALIGN;
+  if (aligned) {
+    if (reinterpret_cast<uintptr_t>(t->data) % 16) return FP8PD_ERR_ALIGN;
+    for (int i = 0; i < 3; ++i)
+      if (t->stride[i] % 16 || t->stride[i] < 0) return FP8PD_ERR_ALIGN;
+  }
+  return FP8PD_OK;
+}
+
+bool same_pool_shape(const fp8pd_tensor* a, const fp8pd_tensor* b) {
+  for (int i = 0; i < 4; ++i)
+    if (a->shape[i] != b->shape[i]) return false;
+  return true;
+}
+
+struct Plan {
+  int num_splits = 1;
+  int head_groups = 1;
+  int grid_blocks = 0;
+  int combine = 0;
+  size_t workspace = 0;
+};
+
+int current_device(int* dev) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (*dev < 0 || *dev >= kMaxDevices) return FP8PD_ERR_TOO_LARGE;
+  return FP8PD_OK;
+}
+
+// Splits per (sequence, KV head, head group): enough thread blocks to fill
+// whole waves of the device, each split keeping >= 256 keys of work.
+int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, Plan* plan) {
+  const int G = Hq / Hkv;
+  plan->head_groups = (G + fp8pd::kHeadsPerGroup - 1) / fp8pd::kHeadsPerGroup;
+  const int64_t units = static_cast<int64_t>(B) * Hkv * plan->head_groups;
+  int64_t pages = max_pages;
+  if (window > 0) pages = std::min<int64_t>(pages, (window + ps - 1) / ps + 1);
+  const int64_t min_pages = std::max(1, 256 / ps);
+  const int64_t s_max = std::max<int64_t>(1, (pages + min_pages - 1) / min_pages);
+  int64_t S = 1;
+  const int64_t forced = g_opt_num_splits.load();
+  if (forced > 0) {
+    S = std::min<int64_t>(forced, std::max<int64_t>(1, pages));
+  } else if (units > 0) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+      int v = 0;
+      if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) sms = v;
+    }
+    cudaGetLastError();
+    const int64_t slots = static_cast<int64_t>(sms) * fp8pd::decode_mma_blocks_per_sm(D);
+    double best_eff = -1.0;
+    int64_t best = 1;
+    for (int64_t s = 1; s <= s_max && s <= 1024; ++s) {
+      const double waves = static_cast<double>(units * s) / static_cast<double>(slots);
+      const double eff = waves / std::ceil(waves);
+      if (eff >= 0.9) {
+        best = s;
+        best_eff = eff;
+        break;
+      }
+      if (eff > best_eff + 1e-9) {
+        best_eff = eff;
+        best = s;
+      }
+    }
+    S = best;
+  }
+  if (S > 65535) S = 65535;
+  plan->num_splits = static_cast<int>(S);
+  plan->grid_blocks = static_cast<int>(std::min<int64_t>(INT32_MAX, units * S));
+  plan->combine = S > 1 ? 1 : 0;
+  plan->workspace = S > 1 ? static_cast<size_t>(B) * Hq * S * (D + 2) * sizeof(float) : 0;
+  return FP8PD_OK;
+}
+
+struct DecodeArgs {
+  int B, Hq, Hkv, D, ps, num_pages, max_pages;
+};
+
+int validate_decode(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_tensor* v_pages,
+                    const fp8pd_tensor* k_scale, const fp8pd_tensor* v_scale,
+                    const fp8pd_tensor* block_table, const fp8pd_tensor* seq_lens, int32_t window,
+                    const fp8pd_tensor* sinks, float sm_scale, const fp8pd_tensor* out,
+                    DecodeParams* p, DecodeArgs* a) {
+  int r;
+  if ((r = check(q, FP8PD_DTYPE_BF16, 3))) return r;
+  if ((r = check_pool(k_pages, true))) return r;
+  if ((r = check_pool(v_pages, true))) return r;
+  if (!same_pool_shape(k_pages, v_pages)) return FP8PD_ERR_SHAPE;
+  if ((r = check(block_table, FP8PD_DTYPE_I32, 2))) return r;
+  if ((r = check(seq_lens, FP8PD_DTYPE_I32, 1))) return r;
+  if ((r = check(out, FP8PD_DTYPE_F32, 3))) return r;
+  const int64_t B = q->shape[0], Hq = q->shape[1], D = q->shape[2];
+  const int64_t P = k_pages->shape[0], ps = k_pages->shape[1], Hkv = k_pages->shape[2];
+  if (k_pages->shape[3] != D) return FP8PD_ERR_SHAPE;
+  if (block_table->shape[0] != B || seq_lens->shape[0] != B) return FP8PD_ERR_SHAPE;
+  if (out->shape[0] != B || out->shape[1] != Hq || out->shape[2] != D) return FP8PD_ERR_SHAPE;
+  if (!(D == 64 || D == 128 || D == 256 || D == 512)) return FP8PD_ERR_UNSUPPORTED;
+  if (ps < 16 || ps > 256 || ps % 16) return FP8PD_ERR_UNSUPPORTED;
+  if (Hkv < 1 || Hq < Hkv || Hq % Hkv) return FP8PD_ERR_UNSUPPORTED;
+  if (out->stride[2] != 1 || reinterpret_cast<uintptr_t>(out->data) % 16 || out->stride[0] % 4 ||
+      out->stride[1] % 4)
+    return FP8PD_ERR_ALIGN;
+  if (window < 0) return FP8PD_ERR_ARG;
+  if (!(std::isfinite(sm_scale) && sm_scale > 0.f)) return FP8PD_ERR_ARG;
+  int64_t ks_sp, ks_sh, vs_sp, vs_sh;
+  if ((r = scale_strides(k_scale, P, Hkv, &ks_sp, &ks_sh))) return r;
+  if ((r = scale_strides(v_scale, P, Hkv, &vs_sp, &vs_sh))) return r;
+  if (sinks) {
+    if ((r = check(sinks, FP8PD_DTYPE_F32, 1))) return r;
+    if (sinks->shape[0] != Hq) return FP8PD_ERR_SHAPE;
+  }
+  const int64_t max_pages = block_table->shape[1];
+  if (!fits_i32(B) || B > 65535 || !fits_i32(P) || !fits_i32(max_pages) ||
+      max_pages * ps > INT32_MAX || Hkv * ((Hq / Hkv + 7) / 8) > 65535 || !fits_i32(Hq))
+    return FP8PD_ERR_TOO_LARGE;
+
+  std::memset(p, 0, sizeof(*p));
+  p->q = static_cast<const uint16_t*>(q->data);
+  p->q_sb = q->stride[0];
+  p->q_sh = q->stride[1];
+  p->q_sd = q->stride[2];
+  p->k = static_cast<const uint8_t*>(k_pages->data);
+  p->v = static_cast<const uint8_t*>(v_pages->data);
+  p->k_sp = k_pages->stride[0];
+  p->k_st = k_pages->stride[1];
+  p->k_sh = k_pages->stride[2];
+  p->v_sp = v_pages->stride[0];
+  p->v_st = v_pages->stride[1];
+  p->v_sh = v_pages->stride[2];
+  p->ks = static_cast<const float*>(k_scale->data);
+  p->vs = static_cast<const float*>(v_scale->data);
+  p->ks_sp = ks_sp;
+  p->ks_sh = ks_sh;
+  p->vs_sp = vs_sp;
+  p->vs_sh = vs_sh;
+  p->table = static_cast<const int32_t*>(block_table->data);
+  p->tab_sb = block_table->stride[0];
+  p->tab_sp = block_table->stride[1];
+  p->lens = static_cast<const int32_t*>(seq_lens->data);
+  p->lens_s = seq_lens->stride[0];
+  p->sinks = sinks ? static_cast<const float*>(sinks->data) : nullptr;
+  p->sinks_s = sinks ? sinks->stride[0] : 0;
+  p->out = static_cast<float*>(out->data);
+  p->o_sb = out->stride[0];
+  p->o_sh = out->stride[1];
+  p->B = static_cast<int>(B);
+  p->Hq = static_cast<int>(Hq);
+  p->Hkv = static_cast<int>(Hkv);
+  p->G = static_cast<int>(Hq / Hkv);
+  p->D = static_cast<int>(D);
+  p->ps = static_cast<int>(ps);
+  p->num_pages = static_cast<int>(P);
+  p->max_pages = static_cast<int>(max_pages);
+  p->window = window;
+  p->sm_scale_log2 = sm_scale * 1.4426950408889634f;
+  a->B = p->B;
+  a->Hq = p->Hq;
+  a->Hkv = p->Hkv;
+  a->D = p->D;
+  a->ps = p->ps;
+  a->num_pages = p->num_pages;
+  a->max_pages = p->max_pages;
+  return FP8PD_OK;
+}
+
+// Returns a workspace of >= bytes on the current device, growing it unless
+// the stream is capturing.
+int get_workspace(size_t bytes, cudaStream_t s, void** out) {
+  int dev;
+  int r = current_device(&dev);
+  if (r) return r;
+  std::lock_guard<std::mutex> lock(g_ws_mutex);
+  Workspace& w = g_ws[dev];
+  if (w.bytes < bytes) {
+    if (is_capturing(s)) return FP8PD_ERR_CAPTURE_WORKSPACE;
+    if (w.ptr) {
+      cudaError_t e = cudaFree(w.ptr);  // synchronizes the device first
+      w.ptr = nullptr;
+      w.bytes = 0;
+      if (e != cudaSuccess) return fail_cuda(e);
+    }
+    size_t grow = std::max(bytes, static_cast<size_t>(1) << 20);
+    cudaError_t e = cudaMalloc(&w.ptr, grow);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      w.ptr = nullptr;
+      return FP8PD_ERR_WORKSPACE;
+    }
+    w.bytes = grow;
+  }
+  *out = w.ptr;
+  return FP8PD_OK;
+}
+
+EventPair* timing_slot(int kind) {
+  if (!g_timing_on.load()) return nullptr;
+  std::lock_guard<std::mutex> lock(g_timing_mutex);
+  if (g_timing_used == g_timing_pool.size()) {
+    EventPair ep;
+    if (cudaEventCreate(&ep.a) != cudaSuccess || cudaEventCreate(&ep.b) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_timing_pool.push_back(ep);
+  }
+  EventPair* ep = &g_timing_pool[g_timing_used++];
+  ep->kind = kind;
+  return ep;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_pages,
+                               const fp8pd_tensor* v_pages, const fp8pd_tensor* k_scale,
+                               const fp8pd_tensor* v_scale, const fp8pd_tensor* block_table,
+                               const fp8pd_tensor* seq_lens, int32_t window,
+                               const fp8pd_tensor* sinks, float sm_scale, fp8pd_tensor* out,
+                               fp8pd_stream_t stream) {
+  DecodeParams p;
+  DecodeArgs a;
+  int r = validate_decode(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens, window,
+                          sinks, sm_scale, out, &p, &a);
+  if (r) return r;
+  if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
+  const int64_t variant = g_opt_variant.load();
+  if (variant == 2) return FP8PD_ERR_UNSUPPORTED;  // CUDA-core variant not built in this library
+  Plan plan;
+  make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  p.num_splits = plan.num_splits;
+  p.head_groups = plan.head_groups;
+  if (plan.combine) {
+    void* ws = nullptr;
+    r = get_workspace(plan.workspace, s, &ws);
+    if (r) return r;
+    p.part_o = static_cast<float*>(ws);
+    p.part_ml = p.part_o + static_cast<size_t>(a.B) * a.Hq * plan.num_splits * a.D;
+  }
+  EventPair* ev = timing_slot(0);
+  if (ev) cudaEventRecord(ev->a, s);
+  cudaError_t e = fp8pd::launch_decode_mma(p, a.D, s);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (ev) cudaEventRecord(ev->b, s);
+  if (plan.combine) {
+    EventPair* ev2 = timing_slot(1);
+    if (ev2) cudaEventRecord(ev2->a, s);
+    e = fp8pd::launch_combine(p, s);
+    if (e != cudaSuccess) return fail_cuda(e);
+    if (ev2) cudaEventRecord(ev2->b, s);
+  }
+  ++g_calls;
+  t_run_info.variant = 1;
+  t_run_info.num_splits = plan.num_splits;
+  t_run_info.head_groups = plan.head_groups;
+  t_run_info.grid_blocks = plan.grid_blocks;
+  t_run_info.combine = plan.combine;
+  t_run_info.head_dim = a.D;
+  return FP8PD_OK;
+}
+
+int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_tensor* block_table,
+               int32_t window, fp8pd_plan_info* info) {
+  int r;
+  if (!info) return FP8PD_ERR_NULL;
+  if ((r = check(q, FP8PD_DTYPE_BF16, 3))) return r;
+  if ((r = check_pool(k_pages, true))) return r;
+  if ((r = check(block_table, FP8PD_DTYPE_I32, 2))) return r;
+  const int64_t B = q->shape[0], Hq = q->shape[1], D = q->shape[2];
+  const int64_t ps = k_pages->shape[1], Hkv = k_pages->shape[2];
+  if (!(D == 64 || D == 128 || D == 256 || D == 512) || k_pages->shape[3] != D)
+    return FP8PD_ERR_UNSUPPORTED;
+  if (ps < 16 || ps > 256 || ps % 16 || Hkv < 1 || Hq % Hkv) return FP8PD_ERR_UNSUPPORTED;
+  if (window < 0) return FP8PD_ERR_ARG;
+  if (!fits_i32(B) || !fits_i32(block_table->shape[1])) return FP8PD_ERR_TOO_LARGE;
+  Plan plan;
+  make_plan(static_cast<int>(B), static_cast<int>(Hq), static_cast<int>(Hkv), static_cast<int>(D),
+            static_cast<int>(ps), static_cast<int>(block_table->shape[1]), window, &plan);
+  info->num_splits = plan.num_splits;
+  info->head_groups = plan.head_groups;
+  info->grid_blocks = plan.grid_blocks;
+  info->combine = plan.combine;
+  info->workspace_bytes = plan.workspace;
+  return FP8PD_OK;
+}
+
+int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_tensor* k_pages,
+                  fp8pd_tensor* v_pages, const fp8pd_scales* scales,
+                  const fp8pd_tensor* block_table, const fp8pd_tensor* positions,
+                  fp8pd_stream_t stream) {
+  int r;
+  if (!scales) return FP8PD_ERR_NULL;
+  if ((r = check(k_new, FP8PD_DTYPE_BF16, 3))) return r;
+  if ((r = check(v_new, FP8PD_DTYPE_BF16, 3))) return r;
+  if ((r = check_pool(k_pages, false))) return r;
+  if ((r = check_pool(v_pages, false))) return r;
+  if (!same_pool_shape(k_pages, v_pages)) return FP8PD_ERR_SHAPE;
+  if ((r = check(block_table, FP8PD_DTYPE_I32, 2))) return r;
+  if ((r = check(positions, FP8PD_DTYPE_I32, 1))) return r;
+  const int64_t B = k_new->shape[0], Hkv = k_new->shape[1], D = k_new->shape[2];
+  const int64_t P = k_pages->shape[0], ps = k_pages->shape[1];
+  for (int i = 0; i < 3; ++i)
+    if (v_new->shape[i] != k_new->shape[i]) return FP8PD_ERR_SHAPE;
+  if (k_pages->shape[2] != Hkv || k_pages->shape[3] != D) return FP8PD_ERR_SHAPE;
+  if (block_table->shape[0] != B || positions->shape[0] != B) return FP8PD_ERR_SHAPE;
+  if (ps < 1) return FP8PD_ERR_UNSUPPORTED;
+  int64_t ks_sp, ks_sh, vs_sp, vs_sh;
+  if ((r = scale_strides(&scales->k_scale, P, Hkv, &ks_sp, &ks_sh))) return r;
+  if ((r = scale_strides(&scales->v_scale, P, Hkv, &vs_sp, &vs_sh))) return r;
+  const int64_t max_pages = block_table->shape[1];
+  if (!fits_i32(B) || !fits_i32(P) || !fits_i32(Hkv) || !fits_i32(D) || !fits_i32(max_pages) ||
+      max_pages * ps > INT32_MAX || B * Hkv * ((D + 1) / 2) > (int64_t(1) << 40))
+    return FP8PD_ERR_TOO_LARGE;
+  if (B == 0 || Hkv == 0 || D == 0) return FP8PD_OK;
+  AppendParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.kn = static_cast<const uint16_t*>(k_new->data);
+  p.vn = static_cast<const uint16_t*>(v_new->data);
+  p.kn_sb = k_new->stride[0];
+  p.kn_sh = k_new->stride[1];
+  p.kn_sd = k_new->stride[2];
+  p.vn_sb = v_new->stride[0];
+  p.vn_sh = v_new->stride[1];
+  p.vn_sd = v_new->stride[2];
+  p.k = static_cast<uint8_t*>(k_pages->data);
+  p.v = static_cast<uint8_t*>(v_pages->data);
+  p.k_sp = k_pages->stride[0];
+  p.k_st = k_pages->stride[1];
+  p.k_sh = k_pages->stride[2];
+  p.v_sp = v_pages->stride[0];
+  p.v_st = v_pages->stride[1];
+  p.v_sh = v_pages->stride[2];
+  p.ks = static_cast<const float*>(scales->k_scale.data);
+  p.vs = static_cast<const float*>(scales->v_scale.data);
+  p.ks_sp = ks_sp;
+  p.ks_sh = ks_sh;
+  p.vs_sp = vs_sp;
+  p.vs_sh = vs_sh;
+  p.table = static_cast<const int32_t*>(block_table->data);
+  p.tab_sb = block_table->stride[0];
+  p.tab_sp = block_table->stride[1];
+  p.pos = static_cast<const int32_t*>(positions->data);
+  p.pos_s = positions->stride[0];
+  p.B = static_cast<int>(B);
+  p.Hkv = static_cast<int>(Hkv);
+  p.D = static_cast<int>(D);
+  p.ps = static_cast<int>(ps);
+  p.num_pages = static_cast<int>(P);
+  p.max_pages = static_cast<int>(max_pages);
+  cudaError_t e = fp8pd::launch_append(p, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e);
+  ++g_appends;
+  return FP8PD_OK;
+}
+
+int fp8pd_reserve_workspace(uint64_t bytes) {
+  void* ws = nullptr;
+  return get_workspace(static_cast<size_t>(bytes), nullptr, &ws);
+}
+
+int fp8pd_check_errors(fp8pd_stream_t stream, uint32_t* flags) {
+  uint32_t v = 0;
+  cudaError_t e = fp8pd::read_and_clear_error_word(&v, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (flags) *flags = v;
+  return FP8PD_OK;
+}
+
+int fp8pd_set_option(int32_t option, int64_t value) {
+  switch (option) {
+    case FP8PD_OPT_NUM_SPLITS:
+      if (value < 0 || value > 65535) return FP8PD_ERR_ARG;
+      g_opt_num_splits = value;
+      return FP8PD_OK;
+    case FP8PD_OPT_VARIANT:
+      if (value < 0 || value > 2) return FP8PD_ERR_ARG;
+      g_opt_variant = value;
+      return FP8PD_OK;
+    default:
+      return FP8PD_ERR_ARG;
+  }
+}
+
+int64_t fp8pd_get_option(int32_t option) {
+  switch (option) {
+    case FP8PD_OPT_NUM_SPLITS: return g_opt_num_splits.load();
+    case FP8PD_OPT_VARIANT: return g_opt_variant.load();
+    default: return -1;
+  }
+}
+
+int fp8pd_last_run_info(fp8pd_run_info* info) {
+  if (!info) return FP8PD_ERR_NULL;
+  *info = t_run_info;
+  info->calls = g_calls.load();
+  info->appends = g_appends.load();
+  return FP8PD_OK;
+}
+
+int fp8pd_timing_enable(int32_t on) {
+  g_timing_on = on ? 1 : 0;
+  return FP8PD_OK;
+}
+
+int fp8pd_timing_collect(double* split_ms, double* combine_ms, int32_t* split_launches,
+                         int32_t* combine_launches) {
+  std::lock_guard<std::mutex> lock(g_timing_mutex);
+  double t[2] = {0.0, 0.0};
+  int32_t n[2] = {0, 0};
+  for (size_t i = 0; i < g_timing_used; ++i) {
+    EventPair& ep = g_timing_pool[i];
+    cudaError_t e = cudaEventSynchronize(ep.b);
+    if (e != cudaSuccess) return fail_cuda(e);
+    float ms = 0.f;
+    e = cudaEventElapsedTime(&ms, ep.a, ep.b);
+    if (e != cudaSuccess) return fail_cuda(e);
+    t[ep.kind] += ms;
+    n[ep.kind] += 1;
+  }
+  g_timing_used = 0;
+  if (split_ms) *split_ms = t[0];
+  if (combine_ms) *combine_ms = t[1];
+  if (split_launches) *split_launches = n[0];
+  if (combine_launches) *combine_launches = n[1];
+  return FP8PD_OK;
+}
+
+const char* fp8pd_status_string(int32_t status) {
+  switch (status) {
+    case FP8PD_OK: return "ok";
+    case FP8PD_ERR_NULL: return "a required descriptor or pointer is NULL";
+    case FP8PD_ERR_DTYPE: return "wrong element type";
+    case FP8PD_ERR_SHAPE: return "inconsistent or unsupported shape";
+    case FP8PD_ERR_ALIGN: return "misaligned pointer or stride (16-byte pool rule, contiguous inner dim)";
+    case FP8PD_ERR_UNSUPPORTED: return "unsupported configuration (head dim, page size, head ratio)";
+    case FP8PD_ERR_ARG: return "bad scalar argument";
+    case FP8PD_ERR_WORKSPACE: return "split workspace allocation failed";
+    case FP8PD_ERR_CAPTURE_WORKSPACE: return "split workspace too small during stream capture";
+    case FP8PD_ERR_CUDA: return "CUDA runtime error";
+    case FP8PD_ERR_TOO_LARGE: return "size exceeds a documented limit";
+    default: return "unknown status";
+  }
+}
+
+int32_t fp8pd_last_cuda_error(void) { return t_last_cuda_error; }
+
+int32_t fp8pd_version(void) { return FP8PD_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// Internal declarations shared by the host API and the kernels of the FP8
+// paged decode attention library (not part of the public ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fp8pd {
+
+// Everything the split kernel needs, resolved from the public descriptors.
+// Strides of the pools are in bytes; of scales, tables, q and out in elements.
+struct DecodeParams {
+  const uint16_t* q;          // bf16 bits [B, Hq, D]
+  int64_t q_sb, q_sh, q_sd;
+  const uint8_t* k;           // pool views [num_pages, ps, Hkv, D]
+  const uint8_t* v;
+  int64_t k_sp, k_st, k_sh;
+  int64_t v_sp, v_st, v_sh;
+  const float* ks;            // scale(page, h) = ks[page * ks_sp + h * ks_sh]
+  const float* vs;
+  int64_t ks_sp, ks_sh, vs_sp, vs_sh;
+  const int32_t* table;       // [B, max_pages]
+  int64_t tab_sb, tab_sp;
+  const int32_t* lens;        // [B]
+  int64_t lens_s;
+  const float* sinks;         // [Hq] or nullptr
+  int64_t sinks_s;
+  float* out;                 // [B, Hq, D], d contiguous
+  int64_t o_sb, o_sh;
+  float* part_o;              // [B * Hq * S, D] split numerators (S > 1)
+  float* part_ml;             // [B * Hq * S, 2] split (max, sum) in log2 units
+  int B, Hq, Hkv, G, D, ps, num_pages, max_pages, window, num_splits, head_groups;
+  float sm_scale_log2;        // sm_scale * log2(e)
+};
+
+struct AppendParams {
+  const uint16_t* kn;         // bf16 bits [B, Hkv, D]
+  const uint16_t* vn;
+  int64_t kn_sb, kn_sh, kn_sd, vn_sb, vn_sh, vn_sd;
+  uint8_t* k;
+  uint8_t* v;
+  int64_t k_sp, k_st, k_sh, v_sp, v_st, v_sh;
+  const float* ks;
+  const float* vs;
+  int64_t ks_sp, ks_sh, vs_sp, vs_sh;
+  const int32_t* table;
+  int64_t tab_sb, tab_sp;
+  const int32_t* pos;
+  int64_t pos_s;
+  int B, Hkv, D, ps, num_pages, max_pages;
+};
+
+// Launchers (defined with the kernels). Return a cudaError_t of the launch.
+cudaError_t launch_decode_mma(const DecodeParams& p, int D, cudaStream_t s);
+cudaError_t launch_combine(const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+
+// Thread blocks of the tensor-core split kernel one SM holds for head dim D.
+int decode_mma_blocks_per_sm(int D);
+// Dynamic shared memory of the tensor-core split kernel for head dim D.
+int decode_mma_smem_bytes(int D);
+
+// Device error word (one per device): read and cleared by the host API.
+cudaError_t read_and_clear_error_word(uint32_t* value, cudaStream_t s);
+
+constexpr int kHeadsPerGroup = 8;   // query heads one thread block serves (MMA N)
+constexpr int kTileTokens = 16;     // tokens per MMA row tile
+
+}  // namespace fp8pd

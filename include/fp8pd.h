@@ -1,0 +1,251 @@
+/*
+ * fp8pd.h -- C ABI of the FP8 (E4M3) paged split-KV decode attention library
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Two operations, both from the "FP8 paged attention for MoE serving"
+ * solution page (cerinamroth.com, "How do I run paged decode attention over
+ * an FP8 KV cache ... with sliding windows, attention sinks and a custom
+ * scale?"):
+ *
+ *   fp8_paged_decode_attention  one decode query per sequence attending over
+ *                               a paged E4M3 KV cache, with grouped-query
+ *                               heads, an optional sliding window, optional
+ *                               per-head sink logits and a caller softmax
+ *                               scale (sections "Expected result" and
+ *                               "Supported scope").
+ *   fp8_kv_append               quantize one new token per sequence to E4M3
+ *                               and store it in its page (section "Supported
+ *                               scope", the one-launch T=1 append; the
+ *                               "Lecture 8 -- Inference Path" page, "In-kernel
+ *                               KV cache update").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every buffer is caller-owned device memory described by fp8pd_tensor
+ *   (pointer, dtype, shape, strides in ELEMENTS). The library never frees or
+ *   keeps a caller pointer past the call.
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *   default stream) and return a status: 0 = success, negative = the call
+ *   was refused and NOTHING was launched (validation happens on the host
+ *   before any launch). FP8PD_ERR_CUDA means a CUDA call failed; the CUDA
+ *   error is available from fp8pd_last_cuda_error().
+ * - Problems only visible on the device never trap: the kernel skips the
+ *   offending work and sets a bit in the device error word, read and
+ *   cleared by fp8pd_check_errors(). A sequence length outside
+ *   [0, max_pages * page_size] makes that sequence's output 0; a 16-token
+ *   tile whose block-table entry is outside [0, num_pages) is left out of
+ *   the softmax; an append position outside the block table, or whose page
+ *   is outside the pool, is not written.
+ * - The library is thread-safe; per-device state (split workspace) is
+ *   guarded by a mutex. The split workspace is reused by every call on the
+ *   device, so calls that overlap on the GPU (different streams, no
+ *   ordering) must not both need it; calls on one stream are ordered.
+ */
+#ifndef FP8PD_H_
+#define FP8PD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FP8PD_VERSION 1
+
+/* A CUDA stream handle (identical to cudaStream_t / CUstream). */
+typedef struct CUstream_st* fp8pd_stream_t;
+
+/* Element types. */
+enum {
+  FP8PD_DTYPE_U8 = 1,   /* uint8: E4M3 codes (pools) */
+  FP8PD_DTYPE_I32 = 2,  /* int32: block tables, lengths, positions */
+  FP8PD_DTYPE_F32 = 3,  /* float32: scales, sinks, output */
+  FP8PD_DTYPE_BF16 = 4  /* bfloat16: q, new K/V */
+};
+
+/* A strided view of device memory. `data` points at element [0,..,0];
+ * element (i0,..,i{n-1}) lives at data + sum_k i_k * stride[k] elements.
+ * Unused trailing entries of shape/stride are ignored. */
+typedef struct fp8pd_tensor {
+  void* data;
+  int32_t dtype;
+  int32_t ndim;
+  int64_t shape[4];
+  int64_t stride[4];
+} fp8pd_tensor;
+
+/* K and V scales for fp8_kv_append (read only). Each is float32 of shape
+ * [Hkv] (one scale per KV head) or [num_pages, Hkv] (one per physical page
+ * and KV head, indexed by the page id found in the block table). */
+typedef struct fp8pd_scales {
+  fp8pd_tensor k_scale;
+  fp8pd_tensor v_scale;
+} fp8pd_scales;
+
+/* Status codes. */
+enum {
+  FP8PD_OK = 0,
+  FP8PD_ERR_NULL = -1,              /* a required descriptor or pointer is NULL */
+  FP8PD_ERR_DTYPE = -2,             /* wrong element type */
+  FP8PD_ERR_SHAPE = -3,             /* inconsistent or unsupported shape */
+  FP8PD_ERR_ALIGN = -4,             /* pool base / strides not multiples of 16 bytes, or
+                                       inner dimension not contiguous */
+  FP8PD_ERR_UNSUPPORTED = -5,       /* head_dim not in {64,128,256,512}, page size not a
+                                       multiple of 16, Hq not a multiple of Hkv, ... */
+  FP8PD_ERR_ARG = -6,               /* bad scalar: window < 0, sm_scale not finite and > 0,
+                                       unknown option */
+  FP8PD_ERR_WORKSPACE = -7,         /* the split workspace could not be allocated */
+  FP8PD_ERR_CAPTURE_WORKSPACE = -8, /* the stream is capturing and the split workspace is
+                                       smaller than the call needs (reserve it first) */
+  FP8PD_ERR_CUDA = -9,              /* a CUDA runtime call failed */
+  FP8PD_ERR_TOO_LARGE = -10         /* a size exceeds a documented limit */
+};
+
+/* Bits of the device error word. */
+enum {
+  FP8PD_FLAG_PAGE_OOB = 1u,    /* block-table entry outside [0, num_pages): tile skipped */
+  FP8PD_FLAG_SEQLEN_OOB = 2u,  /* seq_lens[b] < 0 or > max_pages * page_size: sequence skipped */
+  FP8PD_FLAG_POS_OOB = 4u      /* append position < 0 or >= max_pages * page_size: not written */
+};
+
+/*
+ * fp8_paged_decode_attention -- decode attention over a paged E4M3 KV cache.
+ *
+ * Defines (for each sequence b and query head hq, h = hq / (Hq / Hkv)):
+ *   keys t in [lo, L), L = seq_lens[b], lo = window > 0 ? max(0, L - window) : 0
+ *   K(t, d) = e4m3(k_pages[page(t), t % ps, h, d]) * k_scale(page(t), h)
+ *   V(t, d) likewise, page(t) = block_table[b, t / ps]
+ *   s_t = sm_scale * sum_d q[b, hq, d] * K(t, d)
+ *   M = max(max_t s_t, sink[hq]);  den = sum_t exp(s_t - M) + exp(sink[hq] - M)
+ *   out[b, hq, :] = sum_t exp(s_t - M) * V(t, :) / den     (0 if there is nothing to attend)
+ * The window keeps the last `window` keys; a sink is a logit in the scaled
+ * space that enters the denominator only (the solution page's "Expected
+ * result": `window=W` keeps the last W keys, sinks are [H_q] fp32 with no
+ * value, `sm_scale` replaces D**-0.5). Query head hq reads KV head
+ * hq / (Hq/Hkv) ("Smallest correct example", q.view(H_KV, H_Q // H_KV, D)).
+ * E4M3 codes 0x7F / 0xFF (NaN) decode as +-480: finite inputs never
+ * produce them.
+ *
+ * Arguments (shapes; all device memory):
+ *   q            bf16 [B, Hq, D], any strides.
+ *   k_pages,     uint8 [num_pages, ps, Hkv, D] E4M3 codes; stride[3] must be 1;
+ *   v_pages      base pointer and strides 0..2 must be multiples of 16 bytes
+ *                (a page stride wider than one layer's page is allowed: several
+ *                layers may share one pool -- the solution page's per-layer row
+ *                strides; the 16-byte rule follows DeepGEMM PR #459's paged
+ *                accessor). D in {64, 128, 256, 512}; ps a multiple of 16, <= 256.
+ *   k_scale,     float32 [Hkv] or [num_pages, Hkv], any strides (0 = broadcast).
+ *   v_scale
+ *   block_table  int32 [B, max_pages]: physical page of each logical page.
+ *                Entries past the attended range are never read.
+ *   seq_lens     int32 [B]: number of keys visible to the query (positions 0..L-1).
+ *   window       >= 0; 0 = full attention.
+ *   sinks        float32 [Hq] or NULL.
+ *   sm_scale     finite, > 0.
+ *   out          float32 [B, Hq, D]; stride[2] must be 1, rows 16-byte aligned.
+ *   stream       CUDA stream.
+ * Launches one split kernel, plus one combine kernel when the planner splits
+ * the keys of a sequence over several thread blocks. The split partials live
+ * in a library-owned per-device workspace: it grows on demand outside stream
+ * capture; under capture a call that would need to grow it fails with
+ * FP8PD_ERR_CAPTURE_WORKSPACE (call fp8pd_reserve_workspace, or run the call
+ * once eagerly, before capturing).
+ */
+int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_pages,
+                               const fp8pd_tensor* v_pages, const fp8pd_tensor* k_scale,
+                               const fp8pd_tensor* v_scale, const fp8pd_tensor* block_table,
+                               const fp8pd_tensor* seq_lens, int32_t window,
+                               const fp8pd_tensor* sinks, float sm_scale, fp8pd_tensor* out,
+                               fp8pd_stream_t stream);
+
+/*
+ * fp8_kv_append -- quantize one new token per sequence and store it.
+ *
+ * For each b and KV head h, with p = positions[b], page = block_table[b, p / ps]:
+ *   k_pages[page, p % ps, h, d] = E4M3_RNE_SAT( float(k_new[b, h, d]) / k_scale(page, h) )
+ * and the same for V. The division is IEEE float32 round-to-nearest; the
+ * rounding to E4M3 is round-to-nearest-even, saturating to +-448 (a NaN
+ * input gives the NaN code). Scales are read only. Nothing else in the
+ * pools is written. The new token is then visible to an attention call with
+ * seq_lens[b] = p + 1 (the "Lecture 8" page's kv-cache update before the
+ * decode attention).
+ *
+ * Arguments:
+ *   k_new, v_new  bf16 [B, Hkv, D], any strides.
+ *   k_pages,      uint8 [num_pages, ps, Hkv, D], as for the attention
+ *   v_pages       (stride[3] must be 1; no alignment rule).
+ *   scales        k_scale / v_scale as for the attention.
+ *   block_table   int32 [B, max_pages]; stride[0] may be 0 (every b uses one row,
+ *                 e.g. to write many tokens of one sequence in one call).
+ *   positions     int32 [B].
+ * One kernel launch; no workspace. Two entries that name the same slot race.
+ */
+int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_tensor* k_pages,
+                  fp8pd_tensor* v_pages, const fp8pd_scales* scales,
+                  const fp8pd_tensor* block_table, const fp8pd_tensor* positions,
+                  fp8pd_stream_t stream);
+
+/* What a call with these arguments would launch, without launching it. */
+typedef struct fp8pd_plan_info {
+  int32_t num_splits;        /* thread blocks per (sequence, KV head, head group) */
+  int32_t head_groups;       /* ceil(G / 8) query-head groups per KV head */
+  int32_t grid_blocks;       /* split-kernel thread blocks */
+  int32_t combine;           /* 1 if a combine kernel follows */
+  uint64_t workspace_bytes;  /* split workspace the call needs (0 if no combine) */
+} fp8pd_plan_info;
+
+/* Plans a decode-attention call (same argument rules; nothing launched). */
+int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages,
+               const fp8pd_tensor* block_table, int32_t window, fp8pd_plan_info* info);
+
+/* Grows the current device's split workspace to at least `bytes` (never
+ * shrinks). Must not be called while a stream of the device is capturing. */
+int fp8pd_reserve_workspace(uint64_t bytes);
+
+/* Waits for `stream`, returns the current device's error word in *flags (may
+ * be NULL) and clears it. */
+int fp8pd_check_errors(fp8pd_stream_t stream, uint32_t* flags);
+
+/* Options (process-wide). */
+enum {
+  FP8PD_OPT_NUM_SPLITS = 1,  /* 0 = planner chooses (default); n > 0 forces n splits */
+  FP8PD_OPT_VARIANT = 2      /* 0 = auto; 1 = tensor-core (mma) split kernel;
+                                2 = CUDA-core (f32 FMA) split kernel */
+};
+int fp8pd_set_option(int32_t option, int64_t value);
+int64_t fp8pd_get_option(int32_t option);
+
+/* What the last attention call on this host thread launched. */
+typedef struct fp8pd_run_info {
+  int32_t variant;           /* 1 = tensor-core, 2 = CUDA-core */
+  int32_t num_splits;
+  int32_t head_groups;
+  int32_t grid_blocks;
+  int32_t combine;
+  int32_t head_dim;
+  int64_t calls;             /* attention calls made by this process */
+  int64_t appends;           /* append calls made by this process */
+} fp8pd_run_info;
+int fp8pd_last_run_info(fp8pd_run_info* info);
+
+/* Device timing of the library's own kernels (for benchmarks): while
+ * enabled, each attention call records CUDA events around its split kernel
+ * and its combine kernel on the call's stream. fp8pd_timing_collect waits
+ * for those events, returns the summed milliseconds and launch counts since
+ * the last collect, and resets them. Enabling allocates events; do not
+ * enable during stream capture. */
+int fp8pd_timing_enable(int32_t on);
+int fp8pd_timing_collect(double* split_ms, double* combine_ms, int32_t* split_launches,
+                         int32_t* combine_launches);
+
+/* Human-readable status text (static storage). */
+const char* fp8pd_status_string(int32_t status);
+/* cudaError_t of the last failed CUDA call on this host thread (0 if none). */
+int32_t fp8pd_last_cuda_error(void);
+int32_t fp8pd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP8PD_H_ */

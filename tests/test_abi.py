@@ -1,0 +1,162 @@
+"""CPU-only checks of the C ABI: the library loads, exports every function
+include/fp8pd.h declares, refuses bad arguments with the documented status
+before touching CUDA, and plans splits as documented."""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def F():
+    from fp8_paged_decode_split_b200 import _build
+    _build.build()
+    import fp8_paged_decode_split_b200 as F
+    return F
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "fp8pd.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b((?:fp8_|fp8pd_)\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("fp8_paged_decode_attention", "fp8_kv_append", "fp8pd_check_errors",
+                     "fp8pd_reserve_workspace", "fp8pd_plan", "fp8pd_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_function(F):
+    lib = ctypes.CDLL(F.LIB_PATH)
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(F):
+    assert F.lib.fp8pd_version() == 1
+    for code in range(0, -11, -1):
+        assert F.lib.fp8pd_status_string(code).decode() != "unknown status"
+    assert F.lib.fp8pd_status_string(-99).decode() == "unknown status"
+
+
+def _args(**over):
+    a = dict(
+        q=torch.zeros(2, 8, 128, dtype=torch.bfloat16),
+        k=torch.zeros(6, 16, 2, 128, dtype=torch.uint8),
+        v=torch.zeros(6, 16, 2, 128, dtype=torch.uint8),
+        ks=torch.ones(2), vs=torch.ones(6, 2),
+        table=torch.zeros(2, 3, dtype=torch.int32), lens=torch.zeros(2, dtype=torch.int32),
+        window=0, sinks=None, sm_scale=0.1, out=torch.zeros(2, 8, 128),
+    )
+    a.update(over)
+    return a
+
+
+def _call(F, a):
+    try:
+        F.fp8_paged_decode_attention(a["q"], a["k"], a["v"], a["ks"], a["vs"], a["table"], a["lens"],
+                                     window=a["window"], sinks=a["sinks"], sm_scale=a["sm_scale"],
+                                     out=a["out"], stream=0)
+    except F.Fp8pdError as e:
+        return e.status
+    return 0
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q=torch.zeros(2, 8, 128)), -2),                                    # q not bf16
+    (dict(q=torch.zeros(2, 8, 96, dtype=torch.bfloat16),
+          out=torch.zeros(2, 8, 96)), -3),                                   # pool D != q D
+    (dict(k=torch.zeros(6, 16, 2, 96, dtype=torch.uint8), v=torch.zeros(6, 16, 2, 96, dtype=torch.uint8),
+          q=torch.zeros(2, 8, 96, dtype=torch.bfloat16), out=torch.zeros(2, 8, 96)), -5),  # D=96
+    (dict(k=torch.zeros(6, 8, 2, 128, dtype=torch.uint8), v=torch.zeros(6, 8, 2, 128, dtype=torch.uint8)), -5),
+    (dict(q=torch.zeros(2, 6, 128, dtype=torch.bfloat16), out=torch.zeros(2, 6, 128),
+          k=torch.zeros(6, 16, 4, 128, dtype=torch.uint8), v=torch.zeros(6, 16, 4, 128, dtype=torch.uint8),
+          ks=torch.ones(4), vs=torch.ones(4)), -5),                           # Hq % Hkv
+    (dict(window=-1), -6),
+    (dict(sm_scale=0.0), -6),
+    (dict(sm_scale=float("nan")), -6),
+    (dict(ks=torch.ones(3)), -3),
+    (dict(vs=torch.ones(5, 2)), -3),
+    (dict(sinks=torch.zeros(7)), -3),
+    (dict(table=torch.zeros(3, 3, dtype=torch.int32)), -3),
+    (dict(lens=torch.zeros(2, dtype=torch.int64)), -2),
+    (dict(out=torch.zeros(2, 8, 128, dtype=torch.bfloat16)), -2),
+    (dict(out=torch.zeros(2, 8, 256)[:, :, ::2]), -4),                       # out not contiguous in d
+    (dict(k=torch.zeros(6, 16, 2, 136, dtype=torch.uint8)[..., :128]), -4),  # strides not 16 B multiples
+    (dict(k=torch.zeros(6 * 16 * 2 * 128 + 8, dtype=torch.uint8)[8:].view(6, 16, 2, 128)), -4),  # base
+])
+def test_validation_refuses_before_any_launch(F, over, status):
+    assert _call(F, _args(**over)) == status
+
+
+def test_null_descriptors(F):
+    st = F.lib.fp8_paged_decode_attention(None, None, None, None, None, None, None, 0, None, 1.0,
+                                          None, None)
+    assert st == -1
+    st = F.lib.fp8_kv_append(None, None, None, None, None, None, None, None)
+    assert st == -1
+
+
+def test_append_validation(F):
+    kn = torch.zeros(2, 2, 64, dtype=torch.bfloat16)
+    kp = torch.zeros(4, 16, 2, 64, dtype=torch.uint8)
+    ks = torch.ones(2)
+    tbl = torch.zeros(2, 2, dtype=torch.int32)
+    pos = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(F.Fp8pdError) as e:
+        F.fp8_kv_append(kn.float(), kn, kp, kp, ks, ks, tbl, pos, stream=0)
+    assert e.value.status == -2
+    with pytest.raises(F.Fp8pdError) as e:
+        F.fp8_kv_append(kn, kn, kp, kp, torch.ones(3), ks, tbl, pos, stream=0)
+    assert e.value.status == -3
+    with pytest.raises(F.Fp8pdError) as e:
+        F.fp8_kv_append(kn, kn, kp, kp, ks, ks, tbl, torch.zeros(3, dtype=torch.int32), stream=0)
+    assert e.value.status == -3
+
+
+def test_options_roundtrip(F):
+    F.fp8pd_set_option(F.OPT_NUM_SPLITS, 7)
+    assert F.fp8pd_get_option(F.OPT_NUM_SPLITS) == 7
+    F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
+    with pytest.raises(F.Fp8pdError):
+        F.fp8pd_set_option(99, 1)
+    with pytest.raises(F.Fp8pdError):
+        F.fp8pd_set_option(F.OPT_NUM_SPLITS, -1)
+
+
+def _plan(F, B, Hq, Hkv, D, ps, max_pages, window=0):
+    q = torch.zeros(B, Hq, D, dtype=torch.bfloat16)
+    k = torch.zeros(1, ps, Hkv, D, dtype=torch.uint8).expand(2, ps, Hkv, D)
+    k = torch.as_strided(torch.zeros(ps * Hkv * D, dtype=torch.uint8), (2, ps, Hkv, D), (0, Hkv * D, D, 1))
+    t = torch.as_strided(torch.zeros(1, dtype=torch.int32), (B, max_pages), (0, 0))
+    return F.fp8pd_plan(q, k, t, window)
+
+
+def test_planner_fills_the_device_with_enough_work_per_split(F):
+    # long context, one sequence: many splits, each >= 256 keys
+    p = _plan(F, 1, 64, 8, 128, 64, 2049)
+    assert p["num_splits"] > 16 and p["combine"] == 1
+    assert 2049 / p["num_splits"] >= 4
+    assert p["workspace_bytes"] == 1 * 64 * p["num_splits"] * (128 + 2) * 4
+    # short window: one split, no combine, no workspace
+    p = _plan(F, 64, 64, 8, 64, 16, 513, window=128)
+    assert p["num_splits"] == 1 and p["combine"] == 0 and p["workspace_bytes"] == 0
+    # head groups of at most 8 query heads
+    assert _plan(F, 2, 32, 2, 128, 16, 10)["head_groups"] == 2
+    assert _plan(F, 2, 24, 2, 128, 16, 10)["head_groups"] == 2
+    assert _plan(F, 2, 8, 8, 128, 16, 10)["head_groups"] == 1
+    # forced split count, capped by the pages there are
+    F.fp8pd_set_option(F.OPT_NUM_SPLITS, 5)
+    try:
+        assert _plan(F, 4, 32, 8, 128, 16, 100)["num_splits"] == 5
+        assert _plan(F, 4, 32, 8, 128, 16, 3)["num_splits"] == 3
+    finally:
+        F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
