@@ -1,0 +1,460 @@
+"""Benchmark: FP8 paged decode attention, achieved HBM GB/s and us/step.
+
+One step = the decode hot path for one layer of a synthetic serving batch:
+``fp8_kv_append`` of one new token per sequence, then
+``fp8_paged_decode_attention`` over the updated paged E4M3 cache (split
+kernel + combine). Inputs are resident in HBM when the timed region starts;
+L2 is flushed (a 256 MiB write) between timed steps, outside each step's
+events. ``value`` = algorithmic bytes (attended K/V once per KV head + q +
+the block-table entries read) / device time, summed over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own copy of
+the workload on its GPU (independent sequences: no data-path collective);
+time is the max over ranks, throughput the sum (weak scaling).
+``--impl reference`` times the float64 CPU oracle on the same workload (rank
+0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "FP8 paged decode attention: achieved HBM GB/s and µs/step on 1 B200"
+DEFAULT_CONFIG = "llama"
+WORKLOAD_TEXT = {
+    "llama": "Llama-3-8B-like layer: B=32 Hq=32 Hkv=8 D=128 page=16 seq_len~U[512,4096] "
+             "per-(page,head) scales, +1 appended token/seq",
+    "tiny": "tiny: B=1 Hq=8 Hkv=2 D=64 page=16 L=256",
+    "gptoss_full": "gpt-oss-like: B=64 Hq=64 Hkv=8 D=64 page=16 L=8192 sinks, full attention",
+    "gptoss_w128": "gpt-oss-like: B=64 Hq=64 Hkv=8 D=64 page=16 L=8192 sinks, window=128",
+    "mixed": "mixed pool: B=16 page=32 L~U[2048,16384]; sliding D=256 W=1024 + full D=512",
+    "long_b1": "long context: B=1 Hq=64 Hkv=8 D=128 page=64 L=131072 +append",
+    "long_b8": "long context: B=8 Hq=64 Hkv=8 D=128 page=64 L=131072 +append",
+}
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def _peaks() -> dict:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def _kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("fp8pd_kernels.cu", "fp8pd_internal.h"):
+        with open(os.path.join(ROOT, "fp8_paged_decode_split_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(config: str):
+    """DRAM bytes per split-kernel launch from the committed ncu summary, if
+    it was taken on the current kernel source and this workload."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            d = json.load(f)
+        e = d.get(config)
+        if e and e.get("kernel_hash") == _kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: torch.device):
+        try:
+            self.index = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.index = str(device.index or 0)
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+            os.remove(self.path)
+        except Exception:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class Step:
+    """One decode step of the workload through the library's public API."""
+
+    def __init__(self, F, case: W.Case):
+        self.F = F
+        self.case = case
+
+    def run(self, stream=None):
+        F, c = self.F, self.case
+        for layer in c.layers:
+            if c.spec.append:
+                F.fp8_kv_append(layer.k_new, layer.v_new, layer.k_pages, layer.v_pages,
+                                layer.k_scale, layer.v_scale, layer.block_table, c.positions,
+                                stream=stream)
+            F.fp8_paged_decode_attention(layer.q, layer.k_pages, layer.v_pages, layer.k_scale,
+                                         layer.v_scale, layer.block_table, c.attend_lens,
+                                         window=layer.window, sinks=layer.sinks,
+                                         sm_scale=layer.sm_scale, out=layer.out, stream=stream)
+
+
+def _step_bytes(case: W.Case) -> int:
+    return sum(W.algorithmic_bytes(case, i) for i in range(len(case.layers)))
+
+
+def run_ours(args) -> dict | None:
+    import fp8_paged_decode_split_b200 as F
+    world, rank, local = _dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    case = W.make_case(args.config, dev)
+    for layer in case.layers:
+        layer.out = torch.empty(layer.q.shape, dtype=torch.float32, device=dev)
+    step = Step(F, case)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    nbytes = _step_bytes(case)
+
+    for _ in range(args.warmup):
+        step.run()
+        flush.fill_(1)
+    torch.cuda.synchronize(dev)
+    if F.fp8pd_check_errors() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    # ---- device-timed region: inputs resident, per-step events, L2 flushed between
+    info0 = F.fp8pd_last_run_info()
+    F.fp8pd_timing_enable(True)
+    F.fp8pd_timing_collect()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev) as clocks:
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step.run()
+            ev[i][1].record(stream)
+            flush.fill_(i & 0xFF)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    kt = F.fp8pd_timing_collect()
+    F.fp8pd_timing_enable(False)
+    info1 = F.fp8pd_last_run_info()
+    launches = int(info1["kernel_launches"] - info0["kernel_launches"])
+    if F.fp8pd_check_errors() != 0:
+        raise RuntimeError("device error word set during the timed region")
+
+    # ---- end to end through the public API with host buffers -----------------
+    e2e = run_e2e(F, case, dev, flush, args)
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e["ms"]], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+        torch.distributed.destroy_process_group()
+    else:
+        e2e_ms = e2e["ms"]
+    if rank != 0:
+        return None
+
+    ms_per_step = total_ms / args.steps
+    gbs = world * nbytes / (ms_per_step * 1e-3) / 1e9
+    peaks = _peaks()
+    split_ms = kt["split_ms"] / max(1, kt["split_launches"])
+    layer_bytes = nbytes / max(1, len(case.layers))
+    achieved = layer_bytes / (split_ms * 1e-3) / 1e9 if split_ms > 0 else None
+    traffic = _traffic(args.config)
+    line = {
+        "metric": METRIC,
+        "value": round(gbs, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 6),
+        "us_per_step": round(ms_per_step * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3 cache; f16 tensor-core MMA, f32 accumulate",
+        "data": "synthetic (seeded), no dataset",
+        "config": {"workload": WORKLOAD_TEXT.get(args.config, args.config),
+                   "name": args.config,
+                   "bytes_per_step": nbytes,
+                   "l2": "flushed between timed steps (256 MiB write, outside the step events)",
+                   "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
+        "roofline": {"bound": "hbm", "kernel": "decode_mma_kernel (split)",
+                     "achieved": round(achieved, 2) if achieved else None,
+                     "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
+                     "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4) if achieved else None,
+                     "traffic": traffic,
+                     "split_us_per_launch": round(split_ms * 1e3, 3),
+                     "combine_us_per_launch": round(kt["combine_ms"] * 1e3 / kt["combine_launches"], 3)
+                     if kt["combine_launches"] else None},
+        "gpu_launches": launches,
+        "e2e": {"value": round(world * nbytes / (e2e_ms / e2e["steps"] * 1e-3) / 1e9, 2),
+                "unit": "GB/s", "ms_per_step": round(e2e_ms / e2e["steps"], 6),
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+        "clocks": clocks.summary(),
+        "plan": {k: info1[k] for k in ("num_splits", "head_groups", "grid_blocks", "combine")},
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case, budget_s=args.cpu_seconds)
+    return line
+
+
+def run_e2e(F, case: W.Case, dev, flush, args) -> dict:
+    """Per step: pinned host -> device copies of the step's inputs (q, the new
+    K/V token, lengths, positions, block table), the step, and a device ->
+    host copy of the outputs; timed with events on the step's stream."""
+    stream = torch.cuda.current_stream(dev)
+    host_in, dev_in, host_out = [], [], []
+    for layer in case.layers:
+        tensors = [layer.q, layer.block_table]
+        if case.spec.append:
+            tensors += [layer.k_new, layer.v_new]
+        for t in tensors:
+            host_in.append(t.detach().cpu().pin_memory())
+            dev_in.append(t)
+        host_out.append(torch.empty(layer.q.shape, dtype=torch.float32).pin_memory())
+    for t in [case.attend_lens] + ([case.positions] if case.spec.append else []):
+        host_in.append(t.cpu().pin_memory())
+        dev_in.append(t)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    step = Step(F, case)
+    steps = max(3, min(args.steps, 20))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps + 2):
+        timed = i >= 2
+        if timed:
+            ev[i - 2][0].record(stream)
+        for h, d in zip(host_in, dev_in):
+            d.copy_(h, non_blocking=True)
+        step.run()
+        for h, layer in zip(host_out, case.layers):
+            h.copy_(layer.out, non_blocking=True)
+        if timed:
+            ev[i - 2][1].record(stream)
+        flush.fill_(3)
+    torch.cuda.synchronize(dev)
+    ms = sum(a.elapsed_time(b) for a, b in ev)
+    return {"ms": ms, "steps": steps, "h2d": int(h2d), "d2h": int(d2h)}
+
+
+def _oracle_step(case_np: dict, lens, positions, append: bool):
+    import oracle as O
+    for L in case_np["layers"]:
+        if append:
+            O.kv_append(L["k_new"], L["v_new"], L["k_pages"], L["v_pages"], L["k_scale"],
+                        L["v_scale"], L["block_table"], positions)
+        O.paged_decode_attention(L["q"], L["k_pages"], L["v_pages"], L["k_scale"], L["v_scale"],
+                                 L["block_table"], lens, window=L["window"], sinks=L["sinks"],
+                                 sm_scale=L["sm_scale"])
+
+
+def _case_to_numpy(case: W.Case, seqs) -> tuple[dict, np.ndarray, np.ndarray | None, int]:
+    """Host copy of the sequences ``seqs`` of a case (their pages only)."""
+    out = {"layers": []}
+    ps = case.spec.ps
+    lens = case.attend_lens.cpu().numpy()[seqs]
+    pos = case.positions.cpu().numpy()[seqs] if case.positions is not None else None
+    nbytes = 0
+    for li, layer in enumerate(case.layers):
+        tbl = layer.block_table.cpu().numpy()[seqs]
+        npg = (lens + ps - 1) // ps
+        ids = np.concatenate([tbl[i, :npg[i]] for i in range(len(seqs))]).astype(np.int64)
+        new_tbl = np.full_like(tbl, -1)
+        off = 0
+        for i in range(len(seqs)):
+            new_tbl[i, :npg[i]] = np.arange(off, off + npg[i])
+            off += npg[i]
+        idx = torch.as_tensor(ids, device=layer.k_pages.device)
+        f = lambda t: t.detach().float().cpu().numpy().astype(np.float64)  # noqa: E731
+        per_page = layer.k_scale.dim() == 2
+        d = {"q": f(layer.q[list(seqs)]),
+             "k_pages": layer.k_pages[idx].cpu().numpy(), "v_pages": layer.v_pages[idx].cpu().numpy(),
+             "k_scale": (layer.k_scale[idx] if per_page else layer.k_scale).cpu().numpy(),
+             "v_scale": (layer.v_scale[idx] if per_page else layer.v_scale).cpu().numpy(),
+             "block_table": new_tbl, "window": layer.window, "sm_scale": layer.sm_scale,
+             "sinks": layer.sinks.cpu().numpy() if layer.sinks is not None else None,
+             "k_new": f(layer.k_new[list(seqs)]) if layer.k_new is not None else None,
+             "v_new": f(layer.v_new[list(seqs)]) if layer.v_new is not None else None}
+        out["layers"].append(d)
+        for b in range(len(seqs)):
+            Lb = int(lens[b])
+            lo = max(0, Lb - layer.window) if layer.window > 0 else 0
+            n = Lb - lo
+            nbytes += 2 * n * layer.spec.Hkv * layer.spec.D
+            if n > 0:
+                nbytes += 4 * ((Lb - 1) // ps - lo // ps + 1)
+        nbytes += 2 * d["q"].size
+    return out, lens, pos, nbytes
+
+
+def cpu_baseline(case: W.Case, budget_s: float = 10.0) -> dict:
+    """The oracle as it stands, timed on this host on a bounded sample of the
+    workload: whole steps over the first sequences of the batch, repeated
+    until about ``budget_s`` seconds, single BLAS thread."""
+    from threadpoolctl import threadpool_limits
+    B = case.spec.B
+    total = _step_bytes(case)
+    nseq = max(1, min(B, int(B * 160e6 / max(1, total))))   # ~1 s of oracle work per step
+    seqs = list(range(nseq))
+    case_np, lens, pos, nbytes = _case_to_numpy(case, seqs)
+    reps, t_total = 0, 0.0
+    with threadpool_limits(1):
+        while t_total < budget_s and reps < 1000:
+            t0 = time.perf_counter()
+            _oracle_step(case_np, lens, pos, case.spec.append)
+            t_total += time.perf_counter() - t0
+            reps += 1
+    return {"value": round(nbytes * reps / t_total / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{reps} full step(s) over {nseq}/{B} sequences "
+                      f"({nbytes / 1e6:.1f} MB/step algorithmic), float64 numpy, 1 thread",
+            "seconds": round(t_total, 2)}
+
+
+def run_reference(args) -> dict | None:
+    """The float64 CPU oracle on this host: each step is one bounded sample of
+    the workload (rank 0 only)."""
+    world, rank, _ = _dist_env()
+    if rank != 0:
+        return None
+    from threadpoolctl import threadpool_limits
+    case = W.make_case(args.config, "cpu")
+    B = case.spec.B
+    # bounded sample per step: as many whole sequences as fit in ~1.5 s
+    seqs = list(range(B))
+    case_np, lens, pos, nbytes = _case_to_numpy(case, seqs)
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        _oracle_step(case_np, lens, pos, case.spec.append)
+        one = time.perf_counter() - t0
+        if one > 1.5 and B > 1:
+            keep = max(1, int(B * 1.5 / one))
+            seqs = list(range(keep))
+            case_np, lens, pos, nbytes = _case_to_numpy(case, seqs)
+        for _ in range(args.warmup):
+            _oracle_step(case_np, lens, pos, case.spec.append)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            _oracle_step(case_np, lens, pos, case.spec.append)
+        total = time.perf_counter() - t0
+    gbs = nbytes * args.steps / total / 1e9
+    sample = f"{len(seqs)}/{B} sequences per step ({nbytes / 1e6:.1f} MB algorithmic), float64 numpy"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded), no dataset",
+        "config": {"workload": WORKLOAD_TEXT.get(args.config, args.config), "name": args.config},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(W.SPECS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -57,7 +57,8 @@ class RunInfo(ctypes.Structure):
     _fields_ = [("variant", ctypes.c_int32), ("num_splits", ctypes.c_int32),
                 ("head_groups", ctypes.c_int32), ("grid_blocks", ctypes.c_int32),
                 ("combine", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("calls", ctypes.c_int64), ("appends", ctypes.c_int64)]
+                ("calls", ctypes.c_int64), ("appends", ctypes.c_int64),
+                ("kernel_launches", ctypes.c_int64)]
 
 
 def _load() -> ctypes.CDLL:

@@ -23,7 +23,7 @@ constexpr int kMaxDevices = 64;
 
 thread_local int32_t t_last_cuda_error = 0;
 thread_local fp8pd_run_info t_run_info = {};
-std::atomic<int64_t> g_calls{0}, g_appends{0};
+std::atomic<int64_t> g_calls{0}, g_appends{0}, g_launches{0};
 std::atomic<int64_t> g_opt_num_splits{0}, g_opt_variant{0};
 
 struct Workspace {
@@ -338,12 +338,14 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
   if (ev) cudaEventRecord(ev->a, s);
   cudaError_t e = fp8pd::launch_decode_mma(p, a.D, s);
   if (e != cudaSuccess) return fail_cuda(e);
+  ++g_launches;
   if (ev) cudaEventRecord(ev->b, s);
   if (plan.combine) {
     EventPair* ev2 = timing_slot(1);
     if (ev2) cudaEventRecord(ev2->a, s);
     e = fp8pd::launch_combine(p, s);
     if (e != cudaSuccess) return fail_cuda(e);
+    ++g_launches;
     if (ev2) cudaEventRecord(ev2->b, s);
   }
   ++g_calls;
@@ -447,6 +449,7 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
   cudaError_t e = fp8pd::launch_append(p, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e);
   ++g_appends;
+  ++g_launches;
   return FP8PD_OK;
 }
 
@@ -491,6 +494,7 @@ int fp8pd_last_run_info(fp8pd_run_info* info) {
   *info = t_run_info;
   info->calls = g_calls.load();
   info->appends = g_appends.load();
+  info->kernel_launches = g_launches.load();
   return FP8PD_OK;
 }
 

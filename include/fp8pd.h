@@ -226,6 +226,7 @@ typedef struct fp8pd_run_info {
   int32_t head_dim;
   int64_t calls;             /* attention calls made by this process */
   int64_t appends;           /* append calls made by this process */
+  int64_t kernel_launches;   /* kernels this library launched in this process */
 } fp8pd_run_info;
 int fp8pd_last_run_info(fp8pd_run_info* info);
 
