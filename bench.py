@@ -176,6 +176,8 @@ def _step_bytes(case: W.Case) -> int:
 
 def run_ours(args) -> dict | None:
     import fp8_paged_decode_split_b200 as F
+    F.fp8pd_set_option(F.OPT_K_DECODE, 1 if args.k_decode == "cvt" else 0)
+    F.fp8pd_set_option(F.OPT_NUM_SPLITS, args.splits)
     world, rank, local = _dist_env()
     if world > 1:
         import torch.distributed as dist
@@ -197,11 +199,27 @@ def run_ours(args) -> dict | None:
     torch.cuda.synchronize(dev)
     if F.fp8pd_check_errors() != 0:
         raise RuntimeError("device error word set during warm-up")
+    info0 = F.fp8pd_last_run_info()
+    step.run()
+    plan_info = F.fp8pd_last_run_info()
+    launches_per_step = int(plan_info["kernel_launches"] - info0["kernel_launches"])
+    torch.cuda.synchronize(dev)
+
+    # ---- the step as a CUDA graph (how a serving loop replays decode steps) --
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        step.run()
+    stream.wait_stream(side)
+    with torch.cuda.graph(graph):
+        step.run()
+    for _ in range(args.warmup):
+        graph.replay()
+        flush.fill_(1)
+    torch.cuda.synchronize(dev)
 
     # ---- device-timed region: inputs resident, per-step events, L2 flushed between
-    info0 = F.fp8pd_last_run_info()
-    F.fp8pd_timing_enable(True)
-    F.fp8pd_timing_collect()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     if world > 1:
@@ -210,19 +228,34 @@ def run_ours(args) -> dict | None:
     with ClockSampler(dev) as clocks:
         for i in range(args.steps):
             ev[i][0].record(stream)
-            step.run()
+            graph.replay()
             ev[i][1].record(stream)
             flush.fill_(i & 0xFF)
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    launches = launches_per_step * args.steps
+
+    # ---- per-kernel durations: the same steps eagerly, the library's events
+    # around each of its kernels on the launching stream, L2 flushed between
+    F.fp8pd_timing_enable(True)
+    F.fp8pd_timing_collect()
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        ev2[i][0].record(stream)
+        step.run()
+        ev2[i][1].record(stream)
+        flush.fill_(i & 0xFF)
+    torch.cuda.synchronize(dev)
+    eager_ms = sum(a.elapsed_time(b) for a, b in ev2)
     kt = F.fp8pd_timing_collect()
     F.fp8pd_timing_enable(False)
-    info1 = F.fp8pd_last_run_info()
-    launches = int(info1["kernel_launches"] - info0["kernel_launches"])
     if F.fp8pd_check_errors() != 0:
         raise RuntimeError("device error word set during the timed region")
+    del graph
 
     # ---- end to end through the public API with host buffers -----------------
     e2e = run_e2e(F, case, dev, flush, args)
@@ -240,9 +273,10 @@ def run_ours(args) -> dict | None:
     ms_per_step = total_ms / args.steps
     gbs = world * nbytes / (ms_per_step * 1e-3) / 1e9
     peaks = _peaks()
-    split_ms = kt["split_ms"] / max(1, kt["split_launches"])
+    att_ms = kt["attention_ms"] / max(1, kt["attention_launches"])
+    app_ms = kt["append_ms"] / kt["append_launches"] if kt["append_launches"] else None
     layer_bytes = nbytes / max(1, len(case.layers))
-    achieved = layer_bytes / (split_ms * 1e-3) / 1e9 if split_ms > 0 else None
+    achieved = layer_bytes / (att_ms * 1e-3) / 1e9 if att_ms > 0 else None
     traffic = _traffic(args.config)
     line = {
         "metric": METRIC,
@@ -260,24 +294,26 @@ def run_ours(args) -> dict | None:
         "data": "synthetic (seeded), no dataset",
         "config": {"workload": WORKLOAD_TEXT.get(args.config, args.config),
                    "name": args.config,
-                   "bytes_per_step": nbytes,
+                   "bytes_per_step": nbytes, "k_decode": args.k_decode,
                    "l2": "flushed between timed steps (256 MiB write, outside the step events)",
                    "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
-        "roofline": {"bound": "hbm", "kernel": "decode_mma_kernel (split)",
+        "timing": "device time of CUDA-graph replays of the step (per-step events); "
+                  "eager time and per-kernel events from an eager pass of the same steps",
+        "eager_ms_per_step": round(eager_ms / args.steps, 6),
+        "roofline": {"bound": "hbm", "kernel": "decode_mma_kernel (split-KV attention, one launch)",
                      "achieved": round(achieved, 2) if achieved else None,
                      "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
                      "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4) if achieved else None,
                      "traffic": traffic,
-                     "split_us_per_launch": round(split_ms * 1e3, 3),
-                     "combine_us_per_launch": round(kt["combine_ms"] * 1e3 / kt["combine_launches"], 3)
-                     if kt["combine_launches"] else None},
+                     "us_per_launch": round(att_ms * 1e3, 3),
+                     "append_us_per_launch": round(app_ms * 1e3, 3) if app_ms else None},
         "gpu_launches": launches,
         "e2e": {"value": round(world * nbytes / (e2e_ms / e2e["steps"] * 1e-3) / 1e9, 2),
                 "unit": "GB/s", "ms_per_step": round(e2e_ms / e2e["steps"], 6),
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
         "clocks": clocks.summary(),
-        "plan": {k: info1[k] for k in ("num_splits", "head_groups", "grid_blocks", "combine")},
+        "plan": {k: plan_info[k] for k in ("num_splits", "head_groups", "grid_blocks", "combine")},
     }
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case, budget_s=args.cpu_seconds)
@@ -448,6 +484,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--k-decode", default="bits", choices=["bits", "cvt"],
+                    help="E4M3 -> f16 decode of K: bit assembly or hardware cvt")
+    ap.add_argument("--splits", type=int, default=0, help="force a split count (0 = planner)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

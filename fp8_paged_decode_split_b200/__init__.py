@@ -26,14 +26,15 @@ __all__ = [
     "fp8_paged_decode_attention", "fp8_kv_append", "fp8pd_plan", "fp8pd_reserve_workspace",
     "fp8pd_check_errors", "fp8pd_set_option", "fp8pd_get_option", "fp8pd_last_run_info",
     "fp8pd_timing_enable", "fp8pd_timing_collect", "Fp8pdError", "lib", "LIB_PATH",
-    "FLAG_PAGE_OOB", "FLAG_SEQLEN_OOB", "FLAG_POS_OOB", "OPT_NUM_SPLITS", "OPT_VARIANT",
+    "FLAG_PAGE_OOB", "FLAG_SEQLEN_OOB", "FLAG_POS_OOB", "FLAG_INTERNAL", "OPT_NUM_SPLITS",
+    "OPT_VARIANT", "OPT_K_DECODE",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libfp8pd.so")
 
 DTYPE_U8, DTYPE_I32, DTYPE_F32, DTYPE_BF16 = 1, 2, 3, 4
-FLAG_PAGE_OOB, FLAG_SEQLEN_OOB, FLAG_POS_OOB = 1, 2, 4
-OPT_NUM_SPLITS, OPT_VARIANT = 1, 2
+FLAG_PAGE_OOB, FLAG_SEQLEN_OOB, FLAG_POS_OOB, FLAG_INTERNAL = 1, 2, 4, 8
+OPT_NUM_SPLITS, OPT_VARIANT, OPT_K_DECODE = 1, 2, 3
 _DTYPES = {torch.uint8: DTYPE_U8, torch.int32: DTYPE_I32, torch.float32: DTYPE_F32,
            torch.bfloat16: DTYPE_BF16}
 
@@ -80,7 +81,7 @@ def _load() -> ctypes.CDLL:
     lib.fp8pd_get_option.restype = ctypes.c_int64
     lib.fp8pd_last_run_info.argtypes = [P(RunInfo)]
     lib.fp8pd_timing_enable.argtypes = [i32]
-    lib.fp8pd_timing_collect.argtypes = [P(ctypes.c_double), P(ctypes.c_double), P(i32), P(i32)]
+    lib.fp8pd_timing_collect.argtypes = [P(ctypes.c_double), P(i32), P(ctypes.c_double), P(i32)]
     lib.fp8pd_status_string.argtypes = [i32]
     lib.fp8pd_status_string.restype = ctypes.c_char_p
     lib.fp8pd_last_cuda_error.restype = i32
@@ -223,7 +224,7 @@ def fp8pd_timing_enable(on: bool) -> None:
 def fp8pd_timing_collect() -> dict:
     a, b = ctypes.c_double(), ctypes.c_double()
     na, nb = ctypes.c_int32(), ctypes.c_int32()
-    _check(lib.fp8pd_timing_collect(ctypes.byref(a), ctypes.byref(b), ctypes.byref(na),
+    _check(lib.fp8pd_timing_collect(ctypes.byref(a), ctypes.byref(na), ctypes.byref(b),
                                     ctypes.byref(nb)), "fp8pd_timing_collect")
-    return {"split_ms": a.value, "combine_ms": b.value, "split_launches": na.value,
-            "combine_launches": nb.value}
+    return {"attention_ms": a.value, "attention_launches": na.value, "append_ms": b.value,
+            "append_launches": nb.value}

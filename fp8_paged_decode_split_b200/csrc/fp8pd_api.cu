@@ -24,7 +24,7 @@ constexpr int kMaxDevices = 64;
 thread_local int32_t t_last_cuda_error = 0;
 thread_local fp8pd_run_info t_run_info = {};
 std::atomic<int64_t> g_calls{0}, g_appends{0}, g_launches{0};
-std::atomic<int64_t> g_opt_num_splits{0}, g_opt_variant{0};
+std::atomic<int64_t> g_opt_num_splits{0}, g_opt_variant{0}, g_opt_k_decode{0};
 
 struct Workspace {
   void* ptr = nullptr;
@@ -35,7 +35,7 @@ Workspace g_ws[kMaxDevices];
 
 struct EventPair {
   cudaEvent_t a = nullptr, b = nullptr;
-  int kind = 0;  // 0 = split kernel, 1 = combine kernel
+  int kind = 0;  // 0 = attention kernel, 1 = append kernel
 };
 std::mutex g_timing_mutex;
 std::atomic<int> g_timing_on{0};
@@ -111,6 +111,8 @@ struct Plan {
   int head_groups = 1;
   int grid_blocks = 0;
   int combine = 0;
+  size_t counters_bytes = 0;  // ticket counters (first in the workspace; all zero between calls)
+  size_t ml_bytes = 0;        // split (max, sum) pairs
   size_t workspace = 0;
 };
 
@@ -122,19 +124,25 @@ int current_device(int* dev) {
 }
 
 // Splits per (sequence, KV head, head group): enough thread blocks to fill
-// whole waves of the device, each split keeping >= 256 keys of work.
+// whole waves of the device, each split keeping >= 256 keys of work, no split
+// covering more than kMaxSplitPages pages, at most kMaxSplits splits.
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
 int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, Plan* plan) {
   const int G = Hq / Hkv;
   plan->head_groups = (G + fp8pd::kHeadsPerGroup - 1) / fp8pd::kHeadsPerGroup;
   const int64_t units = static_cast<int64_t>(B) * Hkv * plan->head_groups;
   int64_t pages = max_pages;
   if (window > 0) pages = std::min<int64_t>(pages, (window + ps - 1) / ps + 1);
+  pages = std::max<int64_t>(pages, 1);
+  const int64_t s_min = (pages + fp8pd::kMaxSplitPages - 1) / fp8pd::kMaxSplitPages;
   const int64_t min_pages = std::max(1, 256 / ps);
-  const int64_t s_max = std::max<int64_t>(1, (pages + min_pages - 1) / min_pages);
+  const int64_t s_max = std::min<int64_t>(
+      fp8pd::kMaxSplits, std::max<int64_t>(s_min, (pages + min_pages - 1) / min_pages));
   int64_t S = 1;
   const int64_t forced = g_opt_num_splits.load();
   if (forced > 0) {
-    S = std::min<int64_t>(forced, std::max<int64_t>(1, pages));
+    S = std::min<int64_t>(forced, std::min<int64_t>(pages, fp8pd::kMaxSplits));
   } else if (units > 0) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) {
@@ -145,7 +153,7 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
     const int64_t slots = static_cast<int64_t>(sms) * fp8pd::decode_mma_blocks_per_sm(D);
     double best_eff = -1.0;
     int64_t best = 1;
-    for (int64_t s = 1; s <= s_max && s <= 1024; ++s) {
+    for (int64_t s = 1; s <= s_max; ++s) {
       const double waves = static_cast<double>(units * s) / static_cast<double>(slots);
       const double eff = waves / std::ceil(waves);
       if (eff >= 0.9) {
@@ -160,11 +168,16 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
     }
     S = best;
   }
-  if (S > 65535) S = 65535;
+  S = std::max<int64_t>(S, s_min);
+  if (S > fp8pd::kMaxSplits) return FP8PD_ERR_TOO_LARGE;  // > 65,536 attended pages per sequence
   plan->num_splits = static_cast<int>(S);
   plan->grid_blocks = static_cast<int>(std::min<int64_t>(INT32_MAX, units * S));
   plan->combine = S > 1 ? 1 : 0;
-  plan->workspace = S > 1 ? static_cast<size_t>(B) * Hq * S * (D + 2) * sizeof(float) : 0;
+  plan->counters_bytes = S > 1 ? align256(static_cast<size_t>(units) * sizeof(int)) : 0;
+  plan->ml_bytes = S > 1 ? align256(static_cast<size_t>(B) * Hq * S * 2 * sizeof(float)) : 0;
+  plan->workspace = S > 1 ? plan->counters_bytes + plan->ml_bytes +
+                                static_cast<size_t>(B) * Hq * S * D * sizeof(float)
+                          : 0;
   return FP8PD_OK;
 }
 
@@ -282,6 +295,14 @@ int get_workspace(size_t bytes, cudaStream_t s, void** out) {
       w.ptr = nullptr;
       return FP8PD_ERR_WORKSPACE;
     }
+    // The ticket counters at the start of the workspace must read zero
+    // between calls; each call's merging blocks put them back to zero.
+    e = cudaMemset(w.ptr, 0, grow);
+    if (e != cudaSuccess) {
+      cudaFree(w.ptr);
+      w.ptr = nullptr;
+      return fail_cuda(e);
+    }
     w.bytes = grow;
   }
   *out = w.ptr;
@@ -323,7 +344,8 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
   const int64_t variant = g_opt_variant.load();
   if (variant == 2) return FP8PD_ERR_UNSUPPORTED;  // CUDA-core variant not built in this library
   Plan plan;
-  make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
+  r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
+  if (r) return r;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   p.num_splits = plan.num_splits;
   p.head_groups = plan.head_groups;
@@ -331,23 +353,17 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
     void* ws = nullptr;
     r = get_workspace(plan.workspace, s, &ws);
     if (r) return r;
-    p.part_o = static_cast<float*>(ws);
-    p.part_ml = p.part_o + static_cast<size_t>(a.B) * a.Hq * plan.num_splits * a.D;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    p.counters = reinterpret_cast<int*>(base);
+    p.part_ml = reinterpret_cast<float*>(base + plan.counters_bytes);
+    p.part_o = reinterpret_cast<float*>(base + plan.counters_bytes + plan.ml_bytes);
   }
   EventPair* ev = timing_slot(0);
   if (ev) cudaEventRecord(ev->a, s);
-  cudaError_t e = fp8pd::launch_decode_mma(p, a.D, s);
+  cudaError_t e = fp8pd::launch_decode_mma(p, a.D, g_opt_k_decode.load() == 1, s);
   if (e != cudaSuccess) return fail_cuda(e);
   ++g_launches;
   if (ev) cudaEventRecord(ev->b, s);
-  if (plan.combine) {
-    EventPair* ev2 = timing_slot(1);
-    if (ev2) cudaEventRecord(ev2->a, s);
-    e = fp8pd::launch_combine(p, s);
-    if (e != cudaSuccess) return fail_cuda(e);
-    ++g_launches;
-    if (ev2) cudaEventRecord(ev2->b, s);
-  }
   ++g_calls;
   t_run_info.variant = 1;
   t_run_info.num_splits = plan.num_splits;
@@ -373,8 +389,9 @@ int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_t
   if (window < 0) return FP8PD_ERR_ARG;
   if (!fits_i32(B) || !fits_i32(block_table->shape[1])) return FP8PD_ERR_TOO_LARGE;
   Plan plan;
-  make_plan(static_cast<int>(B), static_cast<int>(Hq), static_cast<int>(Hkv), static_cast<int>(D),
-            static_cast<int>(ps), static_cast<int>(block_table->shape[1]), window, &plan);
+  r = make_plan(static_cast<int>(B), static_cast<int>(Hq), static_cast<int>(Hkv), static_cast<int>(D),
+                static_cast<int>(ps), static_cast<int>(block_table->shape[1]), window, &plan);
+  if (r) return r;
   info->num_splits = plan.num_splits;
   info->head_groups = plan.head_groups;
   info->grid_blocks = plan.grid_blocks;
@@ -446,8 +463,11 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
   p.ps = static_cast<int>(ps);
   p.num_pages = static_cast<int>(P);
   p.max_pages = static_cast<int>(max_pages);
+  EventPair* ev = timing_slot(1);
+  if (ev) cudaEventRecord(ev->a, reinterpret_cast<cudaStream_t>(stream));
   cudaError_t e = fp8pd::launch_append(p, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e);
+  if (ev) cudaEventRecord(ev->b, reinterpret_cast<cudaStream_t>(stream));
   ++g_appends;
   ++g_launches;
   return FP8PD_OK;
@@ -476,6 +496,10 @@ int fp8pd_set_option(int32_t option, int64_t value) {
       if (value < 0 || value > 2) return FP8PD_ERR_ARG;
       g_opt_variant = value;
       return FP8PD_OK;
+    case FP8PD_OPT_K_DECODE:
+      if (value < 0 || value > 1) return FP8PD_ERR_ARG;
+      g_opt_k_decode = value;
+      return FP8PD_OK;
     default:
       return FP8PD_ERR_ARG;
   }
@@ -485,6 +509,7 @@ int64_t fp8pd_get_option(int32_t option) {
   switch (option) {
     case FP8PD_OPT_NUM_SPLITS: return g_opt_num_splits.load();
     case FP8PD_OPT_VARIANT: return g_opt_variant.load();
+    case FP8PD_OPT_K_DECODE: return g_opt_k_decode.load();
     default: return -1;
   }
 }
@@ -503,8 +528,8 @@ int fp8pd_timing_enable(int32_t on) {
   return FP8PD_OK;
 }
 
-int fp8pd_timing_collect(double* split_ms, double* combine_ms, int32_t* split_launches,
-                         int32_t* combine_launches) {
+int fp8pd_timing_collect(double* attention_ms, int32_t* attention_launches, double* append_ms,
+                         int32_t* append_launches) {
   std::lock_guard<std::mutex> lock(g_timing_mutex);
   double t[2] = {0.0, 0.0};
   int32_t n[2] = {0, 0};
@@ -519,10 +544,10 @@ int fp8pd_timing_collect(double* split_ms, double* combine_ms, int32_t* split_la
     n[ep.kind] += 1;
   }
   g_timing_used = 0;
-  if (split_ms) *split_ms = t[0];
-  if (combine_ms) *combine_ms = t[1];
-  if (split_launches) *split_launches = n[0];
-  if (combine_launches) *combine_launches = n[1];
+  if (attention_ms) *attention_ms = t[0];
+  if (attention_launches) *attention_launches = n[0];
+  if (append_ms) *append_ms = t[1];
+  if (append_launches) *append_launches = n[1];
   return FP8PD_OK;
 }
 

@@ -29,6 +29,7 @@ struct DecodeParams {
   int64_t o_sb, o_sh;
   float* part_o;              // [B * Hq * S, D] split numerators (S > 1)
   float* part_ml;             // [B * Hq * S, 2] split (max, sum) in log2 units
+  int* counters;              // [B * Hkv * head_groups] tickets, zero between calls
   int B, Hq, Hkv, G, D, ps, num_pages, max_pages, window, num_splits, head_groups;
   float sm_scale_log2;        // sm_scale * log2(e)
 };
@@ -51,8 +52,7 @@ struct AppendParams {
 };
 
 // Launchers (defined with the kernels). Return a cudaError_t of the launch.
-cudaError_t launch_decode_mma(const DecodeParams& p, int D, cudaStream_t s);
-cudaError_t launch_combine(const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_decode_mma(const DecodeParams& p, int D, bool k_cvt, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 
 // Thread blocks of the tensor-core split kernel one SM holds for head dim D.
@@ -65,5 +65,7 @@ cudaError_t read_and_clear_error_word(uint32_t* value, cudaStream_t s);
 
 constexpr int kHeadsPerGroup = 8;   // query heads one thread block serves (MMA N)
 constexpr int kTileTokens = 16;     // tokens per MMA row tile
+constexpr int kMaxSplitPages = 256; // pages one split may cover (their ids live in smem)
+constexpr int kMaxSplits = 256;     // splits per (sequence, KV head, head group)
 
 }  // namespace fp8pd

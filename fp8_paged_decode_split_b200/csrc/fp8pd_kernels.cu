@@ -14,7 +14,9 @@
 //   split round robin; each warp streams its tiles HBM -> shared memory with
 //   16-byte cp.async into a private multi-stage ring (no block-wide barrier
 //   in the main loop) and keeps its own online-softmax state. The warps are
-//   merged once at the end.
+//   merged once at the end; when the keys are split over several blocks the
+//   last block of a (sequence, KV head, head group) to finish merges the
+//   splits (a ticket counter, never a wait), so one launch does the call.
 // * QK and PV are tensor-core contractions (mma.sync m16n8k16, f16 inputs,
 //   f32 accumulate): rows = 16 tokens (QK) or 16 head-dim entries (PV),
 //   columns = the 8 packed query heads. E4M3 -> f16 is exact, so K and V
@@ -165,10 +167,38 @@ __device__ __forceinline__ uint32_t v_off(int row, int chunk) {
   }
 }
 
+// Hardware E4M3 -> f16 conversion of bytes (0,1) or (2,3) of a word
+// (cvt.rn.f16x2.e4m3x2; exact). Used by the K path when selected.
+__device__ __forceinline__ uint32_t e4m3x2_lo16_to_f16x2(uint32_t w) {
+  uint32_t r;
+  asm("{\n.reg .b16 lo, hi;\nmov.b32 {lo, hi}, %1;\ncvt.rn.f16x2.e4m3x2 %0, lo;\n}\n"
+      : "=r"(r) : "r"(w));
+  return r;
+}
+__device__ __forceinline__ uint32_t e4m3x2_hi16_to_f16x2(uint32_t w) {
+  uint32_t r;
+  asm("{\n.reg .b16 lo, hi;\nmov.b32 {lo, hi}, %1;\ncvt.rn.f16x2.e4m3x2 %0, hi;\n}\n"
+      : "=r"(r) : "r"(w));
+  return r;
+}
+
+__device__ __forceinline__ float4 ldcg4(const float* p) {
+  float4 v;
+  asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];\n"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ float2 ldcg2(const float* p) {
+  float2 v;
+  asm volatile("ld.global.cg.v2.f32 {%0,%1}, [%2];\n" : "=f"(v.x), "=f"(v.y) : "l"(p));
+  return v;
+}
+
 template <int D>
 struct Cfg {
   static constexpr int NW = 4;                                        // warps per block
-  static constexpr int NS = (D == 64) ? 8 : (D == 128) ? 4 : 2;       // ring stages per warp
+  static constexpr int NS = (D == 64) ? 6 : (D == 128) ? 3 : 2;       // ring stages per warp
   static constexpr int TILE = kTileTokens * D;                        // bytes of a K or V tile
   static constexpr int STAGE = 2 * TILE;
   static constexpr int WARP_BYTES = NS * STAGE;
@@ -177,14 +207,19 @@ struct Cfg {
   static constexpr int QFRAG_BYTES = Q_IN_SMEM ? (D / 16) * 32 * 8 : 0;
   static constexpr int PROW = 24;                                     // halves per P row
   static constexpr int PBUF_BYTES = NW * 2 * 8 * PROW * 2;
-  static constexpr int MISC_FLOATS = 8 + NW * 8 * 2;
-  static constexpr int SMEM = PIPE_BYTES + QFRAG_BYTES + PBUF_BYTES + MISC_FLOATS * 4;
-  static constexpr int MIN_BLOCKS = (D == 512) ? 1 : (D == 256) ? 2 : 3;
+  static constexpr int PAGE_BYTES = kMaxSplitPages * 12;              // page id, k / v scale
+  static constexpr int MISC_FLOATS = 8 + NW * 8 * 2 + 4;
+  static constexpr int SMEM = PIPE_BYTES + QFRAG_BYTES + PBUF_BYTES + PAGE_BYTES + MISC_FLOATS * 4;
+  static constexpr int MIN_BLOCKS = (D == 512) ? 1 : (D == 256) ? 2 : 4;
   static_assert(NW * 8 * D * 4 <= PIPE_BYTES, "merge scratch must fit in the ring");
   static_assert(8 * D * 4 <= PIPE_BYTES, "q staging must fit in the ring");
+  static_assert(8 * kMaxSplits * 4 <= PIPE_BYTES, "combine weights must fit in the ring");
 };
 
-template <int D>
+// One thread block: (split, KV head x head group, sequence). KCVT selects the
+// K decode: false = bit assembly (byte pairs (0,2)/(1,3)), true = hardware
+// cvt (byte pairs (0,1)/(2,3)); the q fragments follow the same pairing.
+template <int D, bool KCVT>
 __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     decode_mma_kernel(const DecodeParams p) {
   using C = Cfg<D>;
@@ -193,7 +228,10 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   uint8_t* pipe = smem;
   uint2* qfrag_s = reinterpret_cast<uint2*>(smem + C::PIPE_BYTES);
   __half* pbuf = reinterpret_cast<__half*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES);
-  float* misc = reinterpret_cast<float*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES + C::PBUF_BYTES);
+  int32_t* s_pid = reinterpret_cast<int32_t*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES + C::PBUF_BYTES);
+  float* s_ks = reinterpret_cast<float*>(s_pid + kMaxSplitPages);
+  float* s_vs = s_ks + kMaxSplitPages;
+  float* misc = s_vs + kMaxSplitPages;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, grp = lane >> 2, qd = lane & 3;
@@ -214,14 +252,34 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   const int n_pages = (L > lo) ? (L - 1) / p.ps - first_page + 1 : 0;
   const int chunk = (n_pages + p.num_splits - 1) / p.num_splits;
   const int pg0 = first_page + split * chunk;
-  const int pg1 = min(first_page + n_pages, pg0 + chunk);
+  int pg1 = min(first_page + n_pages, pg0 + chunk);
+  if (pg1 - pg0 > kMaxSplitPages) {  // the planner never does this; refuse rather than overflow
+    if (tid == 0) raise_flag(FP8PD_FLAG_INTERNAL);
+    pg1 = pg0;
+  }
   const int t0 = max(lo, pg0 * p.ps);
   const int t1 = min(L, pg1 * p.ps);
   const int tile_first = t0 / kTileTokens;
   const int n_tiles = (t1 > t0) ? (t1 + kTileTokens - 1) / kTileTokens - tile_first : 0;
   const int32_t* trow = p.table + (int64_t)b * p.tab_sb;
 
-  // ---- q of the head group, max |q|, V reference scale ----------------------
+  // ---- pages of the split, their scales; q of the head group ---------------
+  float vmax = 0.f;
+  for (int i = tid; i < pg1 - pg0; i += 128) {
+    const int page = __ldg(trow + (int64_t)(pg0 + i) * p.tab_sp);
+    const bool ok = (unsigned)page < (unsigned)p.num_pages;
+    float ks = 0.f, vs = 0.f;
+    if (ok) {
+      ks = __ldg(p.ks + (int64_t)page * p.ks_sp + (int64_t)kvh * p.ks_sh);
+      vs = __ldg(p.vs + (int64_t)page * p.vs_sp + (int64_t)kvh * p.vs_sh);
+    } else if (hg == 0) {
+      raise_flag(FP8PD_FLAG_PAGE_OOB);
+    }
+    s_pid[i] = ok ? page : -1;
+    s_ks[i] = ks;
+    s_vs[i] = vs;
+    vmax = fmaxf(vmax, fabsf(vs));
+  }
   float* qs = reinterpret_cast<float*>(pipe);  // [8][D] staging
   float qmax = 0.f;
   for (int i = tid; i < 8 * D; i += 128) {
@@ -233,15 +291,6 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     qs[i] = x;
     qmax = fmaxf(qmax, fabsf(x));
   }
-  float vmax = 0.f;
-  const bool vs_per_page = p.vs_sp != 0;
-  if (vs_per_page) {
-    for (int pg = pg0 + tid; pg < pg1; pg += 128) {
-      const int page = __ldg(trow + (int64_t)pg * p.tab_sp);
-      if ((unsigned)page < (unsigned)p.num_pages)
-        vmax = fmaxf(vmax, fabsf(__ldg(p.vs + (int64_t)page * p.vs_sp + (int64_t)kvh * p.vs_sh)));
-    }
-  }
   qmax = warp_max(qmax);
   vmax = warp_max(vmax);
   if (lane == 0) {
@@ -250,8 +299,9 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   }
   __syncthreads();
   qmax = fmaxf(fmaxf(misc[0], misc[1]), fmaxf(misc[2], misc[3]));
-  float vref = vs_per_page ? fmaxf(fmaxf(misc[4], misc[5]), fmaxf(misc[6], misc[7]))
-                           : fabsf(__ldg(p.vs + (int64_t)kvh * p.vs_sh));
+  // V reference scale: the split's largest |v_scale|, so every P * v_scale /
+  // vref stays <= 1 and its f16 hi/lo split keeps full relative precision.
+  float vref = fmaxf(fmaxf(misc[4], misc[5]), fmaxf(misc[6], misc[7]));
   if (!(vref > 0.f) || !isfinite(vref)) vref = 1.f;
   const float inv_vref = 1.f / vref;
   // q' = q * 2^(15 - e) puts max|q'| in [2^14, 2^15): exact in f16 for every
@@ -265,16 +315,22 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   const float score_base = p.sm_scale_log2 * 256.f / qmul;
 
   // B fragments of q (column n = query head grp of the group). The k16 block
-  // (jj, i) covers head-dim entries 64jj + 16q + 4i + {0..3} of lane quad q;
-  // k = 2q -> +0, 2q+1 -> +2, 2q+8 -> +1, 2q+9 -> +3, matching the byte pairs
-  // (0,2) and (1,3) the K words are decoded into.
+  // (jj, i) covers head-dim entries 64jj + 16q + 4i + {0..3} of lane quad q.
+  // Bit-assembly K pairs bytes (0,2) and (1,3): k = 2q -> +0, 2q+1 -> +2,
+  // 2q+8 -> +1, 2q+9 -> +3. Hardware-cvt K pairs (0,1) and (2,3).
   uint32_t qf[C::Q_IN_SMEM ? 1 : KB][2];
 #pragma unroll
   for (int kb = 0; kb < KB; ++kb) {
     const int jj = kb >> 2, i = kb & 3;
     const float* qrow = qs + grp * D + 64 * jj + 16 * qd + 4 * i;
-    const uint32_t r0 = pack_f16x2(qrow[0] * qmul, qrow[2] * qmul);
-    const uint32_t r1 = pack_f16x2(qrow[1] * qmul, qrow[3] * qmul);
+    uint32_t r0, r1;
+    if constexpr (KCVT) {
+      r0 = pack_f16x2(qrow[0] * qmul, qrow[1] * qmul);
+      r1 = pack_f16x2(qrow[2] * qmul, qrow[3] * qmul);
+    } else {
+      r0 = pack_f16x2(qrow[0] * qmul, qrow[2] * qmul);
+      r1 = pack_f16x2(qrow[1] * qmul, qrow[3] * qmul);
+    }
     if constexpr (C::Q_IN_SMEM) {
       if (warp == 0) qfrag_s[kb * 32 + lane] = make_uint2(r0, r1);
     } else {
@@ -289,15 +345,17 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   __half* p_hi = pbuf + warp * (2 * 8 * C::PROW);
   __half* p_lo = p_hi + 8 * C::PROW;
   const int my_tiles = (n_tiles > warp) ? (n_tiles - warp + C::NW - 1) / C::NW : 0;
+  const uint8_t* kbase = p.k + (int64_t)kvh * p.k_sh;
+  const uint8_t* vbase = p.v + (int64_t)kvh * p.v_sh;
 
   auto issue = [&](int j, int stage) {
     const int tok0 = (tile_first + warp + C::NW * j) * kTileTokens;
     const int lp = tok0 / p.ps;
-    const int page = __ldg(trow + (int64_t)lp * p.tab_sp);
-    if ((unsigned)page >= (unsigned)p.num_pages) return;
+    const int page = s_pid[lp - pg0];
+    if (page < 0) return;
     const int slot0 = tok0 - lp * p.ps;
-    const uint8_t* gk = p.k + (int64_t)page * p.k_sp + (int64_t)slot0 * p.k_st + (int64_t)kvh * p.k_sh;
-    const uint8_t* gv = p.v + (int64_t)page * p.v_sp + (int64_t)slot0 * p.v_st + (int64_t)kvh * p.v_sh;
+    const uint8_t* gk = kbase + (int64_t)page * p.k_sp + (int64_t)slot0 * p.k_st;
+    const uint8_t* gv = vbase + (int64_t)page * p.v_sp + (int64_t)slot0 * p.v_st;
     const uint32_t sk = wpipe + stage * C::STAGE;
     const uint32_t sv = sk + C::TILE;
     constexpr int CPR = D / 16;
@@ -336,20 +394,15 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       cp_async_commit();
     }
     const int tok0 = (tile_first + warp + C::NW * j) * kTileTokens;
-    const int lp = tok0 / p.ps;
-    const int page = __ldg(trow + (int64_t)lp * p.tab_sp);
-    const bool page_ok = (unsigned)page < (unsigned)p.num_pages;
-    if (!page_ok && lane == 0) raise_flag(FP8PD_FLAG_PAGE_OOB);
-    float kfac = 0.f, vsr = 0.f;
-    if (page_ok) {
-      kfac = score_base * __ldg(p.ks + (int64_t)page * p.ks_sp + (int64_t)kvh * p.ks_sh);
-      vsr = __ldg(p.vs + (int64_t)page * p.vs_sp + (int64_t)kvh * p.vs_sh) * inv_vref;
-    }
+    const int li = tok0 / p.ps - pg0;
+    const bool page_ok = s_pid[li] >= 0;
+    const float kfac = score_base * s_ks[li];
+    const float vsr = s_vs[li] * inv_vref;
     const uint32_t sk = wpipe + (j % C::NS) * C::STAGE;
     const uint32_t sv = sk + C::TILE;
 
-    // -- S[token][head] = K q'^T -------------------------------------------
-    float S[4] = {0.f, 0.f, 0.f, 0.f};
+    // -- S[token][head] = K q'^T (two independent accumulator chains) --------
+    float Sa[4] = {0.f, 0.f, 0.f, 0.f}, Sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int jj = 0; jj < D / 64; ++jj) {
       const uint4 ka = lds128(sk + k_off<D>(grp, 4 * jj + qd));
@@ -367,8 +420,22 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
           b0 = qf[jj * 4 + i][0];
           b1 = qf[jj * 4 + i][1];
         }
-        mma16816(S, e4m3x2_b02_to_f16x2(wa[i]), e4m3x2_b02_to_f16x2(wb[i]),
-                 e4m3x2_b13_to_f16x2(wa[i]), e4m3x2_b13_to_f16x2(wb[i]), b0, b1);
+        uint32_t a0, a1, a2, a3;
+        if constexpr (KCVT) {
+          a0 = e4m3x2_lo16_to_f16x2(wa[i]);
+          a1 = e4m3x2_lo16_to_f16x2(wb[i]);
+          a2 = e4m3x2_hi16_to_f16x2(wa[i]);
+          a3 = e4m3x2_hi16_to_f16x2(wb[i]);
+        } else {
+          a0 = e4m3x2_b02_to_f16x2(wa[i]);
+          a1 = e4m3x2_b02_to_f16x2(wb[i]);
+          a2 = e4m3x2_b13_to_f16x2(wa[i]);
+          a3 = e4m3x2_b13_to_f16x2(wb[i]);
+        }
+        if (i & 1)
+          mma16816(Sb, a0, a1, a2, a3, b0, b1);
+        else
+          mma16816(Sa, a0, a1, a2, a3, b0, b1);
       }
     }
 
@@ -376,10 +443,11 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     const int ta = tok0 + grp, tb = ta + 8;
     const bool va = page_ok && ta >= t0 && ta < t1;
     const bool vb = page_ok && tb >= t0 && tb < t1;
-    const float s00 = va ? S[0] * kfac : -CUDART_INF_F;  // token grp,   head 2qd
-    const float s01 = va ? S[1] * kfac : -CUDART_INF_F;  // token grp,   head 2qd+1
-    const float s10 = vb ? S[2] * kfac : -CUDART_INF_F;  // token grp+8, head 2qd
-    const float s11 = vb ? S[3] * kfac : -CUDART_INF_F;  // token grp+8, head 2qd+1
+    // a masked row may hold stale or NaN-decoded bytes: select, never multiply
+    const float s00 = va ? (Sa[0] + Sb[0]) * kfac : -CUDART_INF_F;  // token grp,   head 2qd
+    const float s01 = va ? (Sa[1] + Sb[1]) * kfac : -CUDART_INF_F;  // token grp,   head 2qd+1
+    const float s10 = vb ? (Sa[2] + Sb[2]) * kfac : -CUDART_INF_F;  // token grp+8, head 2qd
+    const float s11 = vb ? (Sa[3] + Sb[3]) * kfac : -CUDART_INF_F;  // token grp+8, head 2qd+1
     float tm0 = fmaxf(s00, s10), tm1 = fmaxf(s01, s11);
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
@@ -485,6 +553,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
 
   const float fold = 256.f * vref;  // f16 offset of the decoded V, and the V reference scale
   constexpr float kLog2e = 1.4426950408889634f;
+  const int S = p.num_splits;
   for (int it = tid; it < 8 * (D / 4); it += 128) {
     const int n = it / (D / 4);
     const int d = (it - n * (D / 4)) * 4;
@@ -508,7 +577,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       }
     }
     const int head = head0 + n;
-    if (p.num_splits == 1) {
+    if (S == 1) {
       const float sl = p.sinks ? p.sinks[(int64_t)head * p.sinks_s] * kLog2e : -CUDART_INF_F;
       const float M2 = fmaxf(M, sl);
       float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -522,64 +591,74 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       }
       *reinterpret_cast<float4*>(p.out + (int64_t)b * p.o_sb + (int64_t)head * p.o_sh + d) = r;
     } else {
-      const int64_t row = ((int64_t)b * p.Hq + head) * p.num_splits + split;
+      const int64_t row = ((int64_t)b * p.Hq + head) * S + split;
       *reinterpret_cast<float4*>(p.part_o + row * D + d) =
           make_float4(acc.x * fold, acc.y * fold, acc.z * fold, acc.w * fold);
-      if (d == 0) {
-        p.part_ml[row * 2 + 0] = M;
-        p.part_ml[row * 2 + 1] = l;
-      }
+      if (d == 0) *reinterpret_cast<float2*>(p.part_ml + row * 2) = make_float2(M, l);
     }
   }
-}
+  if (S == 1) return;
 
-// ---------------------------------------------------------------------------
-// Log-sum-exp combine of the splits of one (sequence, query head) row, with
-// the sink entering the denominator once. One warp per row.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
-  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= p.B * p.Hq) return;
-  const int b = row / p.Hq, head = row - b * p.Hq;
-  const int S = p.num_splits;
-  const float* ml = p.part_ml + (int64_t)row * S * 2;
-  constexpr float kLog2e = 1.4426950408889634f;
-  float M = -CUDART_INF_F;
-  for (int s = lane; s < S; s += 32) M = fmaxf(M, ml[2 * s]);
-  M = warp_max(M);
-  const float sl = p.sinks ? p.sinks[(int64_t)head * p.sinks_s] * kLog2e : -CUDART_INF_F;
-  const float M2 = fmaxf(M, sl);
-  float den = 0.f;
-  if (M2 != -CUDART_INF_F) {
-    for (int s = lane; s < S; s += 32) {
-      const float ms = ml[2 * s];
-      if (ms != -CUDART_INF_F) den += ml[2 * s + 1] * exp2f(ms - M2);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    if (p.sinks) den += exp2f(sl - M2);
+  // ---- the last block of this (sequence, KV head, head group) combines ------
+  // Every block publishes its partials, then takes a ticket; the block that
+  // draws the last ticket merges all S partials (log-sum-exp, sink added once)
+  // and resets the counter for the next call. No block ever waits for another.
+  __threadfence();
+  __syncthreads();
+  int* last_flag = reinterpret_cast<int*>(misc + 8 + C::NW * 8 * 2);
+  const int64_t unit = (int64_t)b * gridDim.y + blockIdx.y;
+  if (tid == 0) {
+    const int prev = atomicAdd(p.counters + unit, 1);
+    *last_flag = (prev == S - 1);
   }
-  const float inv = (M2 != -CUDART_INF_F && den > 0.f) ? 1.f / den : 0.f;
-  float* out = p.out + (int64_t)b * p.o_sb + (int64_t)head * p.o_sh;
-  const float* po = p.part_o + (int64_t)row * S * p.D;
-  for (int d = lane * 4; d < p.D; d += 128) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (inv != 0.f) {
-      for (int s = 0; s < S; ++s) {
-        const float ms = ml[2 * s];
-        if (ms == -CUDART_INF_F) continue;
-        const float w = exp2f(ms - M2);
-        const float4 o = *reinterpret_cast<const float4*>(po + (int64_t)s * p.D + d);
-        acc.x += w * o.x;
-        acc.y += w * o.y;
-        acc.z += w * o.z;
-        acc.w += w * o.w;
+  __syncthreads();
+  if (!*last_flag) return;
+  __threadfence();
+
+  float* wts = reinterpret_cast<float*>(pipe);  // [8][S] split weights / den
+  for (int n = warp; n < nheads; n += C::NW) {
+    const int head = head0 + n;
+    const float* pml = p.part_ml + ((int64_t)b * p.Hq + head) * S * 2;
+    float M = -CUDART_INF_F;
+    for (int s = lane; s < S; s += 32) M = fmaxf(M, ldcg2(pml + 2 * s).x);
+    M = warp_max(M);
+    const float sl = p.sinks ? p.sinks[(int64_t)head * p.sinks_s] * kLog2e : -CUDART_INF_F;
+    const float M2 = fmaxf(M, sl);
+    float den = 0.f;
+    if (M2 != -CUDART_INF_F) {
+      for (int s = lane; s < S; s += 32) {
+        const float2 ml2 = ldcg2(pml + 2 * s);
+        if (ml2.x != -CUDART_INF_F) den += ml2.y * exp2f(ml2.x - M2);
       }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+      if (p.sinks) den += exp2f(sl - M2);
     }
-    *reinterpret_cast<float4*>(out + d) =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    const float inv = (M2 != -CUDART_INF_F && den > 0.f) ? 1.f / den : 0.f;
+    for (int s = lane; s < S; s += 32) {
+      const float ms = ldcg2(pml + 2 * s).x;
+      wts[n * kMaxSplits + s] = (inv == 0.f || ms == -CUDART_INF_F) ? 0.f : exp2f(ms - M2) * inv;
+    }
   }
+  __syncthreads();
+  for (int it = tid; it < nheads * (D / 4); it += 128) {
+    const int n = it / (D / 4);
+    const int d = (it - n * (D / 4)) * 4;
+    const int head = head0 + n;
+    const float* po = p.part_o + ((int64_t)b * p.Hq + head) * S * D + d;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < S; ++s) {
+      const float w = wts[n * kMaxSplits + s];
+      if (w == 0.f) continue;
+      const float4 o = ldcg4(po + (int64_t)s * D);
+      acc.x += w * o.x;
+      acc.y += w * o.y;
+      acc.z += w * o.z;
+      acc.w += w * o.w;
+    }
+    *reinterpret_cast<float4*>(p.out + (int64_t)b * p.o_sb + (int64_t)head * p.o_sh + d) = acc;
+  }
+  if (tid == 0) p.counters[unit] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -639,7 +718,7 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
 // ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool KCVT>
 static cudaError_t launch_decode_mma_d(const DecodeParams& p, cudaStream_t s) {
   // The shared-memory opt-in is a per-device function attribute: set it once
   // per device (an idempotent call, so a race only repeats it).
@@ -650,21 +729,22 @@ static cudaError_t launch_decode_mma_d(const DecodeParams& p, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
   if (!bit || !(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(decode_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(decode_mma_kernel<D, KCVT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
   const dim3 grid(p.num_splits, p.Hkv * p.head_groups, p.B);
-  decode_mma_kernel<D><<<grid, 128, smem, s>>>(p);
+  decode_mma_kernel<D, KCVT><<<grid, 128, smem, s>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode_mma(const DecodeParams& p, int D, cudaStream_t s) {
+cudaError_t launch_decode_mma(const DecodeParams& p, int D, bool k_cvt, cudaStream_t s) {
   switch (D) {
-    case 64: return launch_decode_mma_d<64>(p, s);
-    case 128: return launch_decode_mma_d<128>(p, s);
-    case 256: return launch_decode_mma_d<256>(p, s);
-    case 512: return launch_decode_mma_d<512>(p, s);
+    case 64: return k_cvt ? launch_decode_mma_d<64, true>(p, s) : launch_decode_mma_d<64, false>(p, s);
+    case 128: return k_cvt ? launch_decode_mma_d<128, true>(p, s) : launch_decode_mma_d<128, false>(p, s);
+    case 256: return k_cvt ? launch_decode_mma_d<256, true>(p, s) : launch_decode_mma_d<256, false>(p, s);
+    case 512: return k_cvt ? launch_decode_mma_d<512, true>(p, s) : launch_decode_mma_d<512, false>(p, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -681,18 +761,20 @@ int decode_mma_smem_bytes(int D) {
 
 template <int D>
 static int blocks_per_sm_d() {
-  static int cached = -1;
-  if (cached >= 0) return cached;
+  static std::atomic<int> cached{-1};
+  int c = cached.load();
+  if (c >= 0) return c;
   int n = 0;
-  if (cudaFuncSetAttribute(decode_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(decode_mma_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cfg<D>::SMEM) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_mma_kernel<D>, 128, Cfg<D>::SMEM) !=
-          cudaSuccess) {
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_mma_kernel<D, false>, 128,
+                                                    Cfg<D>::SMEM) != cudaSuccess) {
     cudaGetLastError();
-    n = Cfg<D>::MIN_BLOCKS;
+    return Cfg<D>::MIN_BLOCKS;  // no device: do not cache the guess
   }
-  cached = n > 0 ? n : 1;
-  return cached;
+  c = n > 0 ? n : 1;
+  cached.store(c);
+  return c;
 }
 
 int decode_mma_blocks_per_sm(int D) {
@@ -703,12 +785,6 @@ int decode_mma_blocks_per_sm(int D) {
     case 512: return blocks_per_sm_d<512>();
     default: return 1;
   }
-}
-
-cudaError_t launch_combine(const DecodeParams& p, cudaStream_t s) {
-  const int rows = p.B * p.Hq;
-  combine_kernel<<<(rows + 3) / 4, 128, 0, s>>>(p);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {

@@ -99,14 +99,17 @@ enum {
   FP8PD_ERR_CAPTURE_WORKSPACE = -8, /* the stream is capturing and the split workspace is
                                        smaller than the call needs (reserve it first) */
   FP8PD_ERR_CUDA = -9,              /* a CUDA runtime call failed */
-  FP8PD_ERR_TOO_LARGE = -10         /* a size exceeds a documented limit */
+  FP8PD_ERR_TOO_LARGE = -10         /* a size exceeds a documented limit (e.g. more than
+                                       65,536 attended pages in one sequence) */
 };
 
 /* Bits of the device error word. */
 enum {
   FP8PD_FLAG_PAGE_OOB = 1u,    /* block-table entry outside [0, num_pages): tile skipped */
   FP8PD_FLAG_SEQLEN_OOB = 2u,  /* seq_lens[b] < 0 or > max_pages * page_size: sequence skipped */
-  FP8PD_FLAG_POS_OOB = 4u      /* append position < 0 or >= max_pages * page_size: not written */
+  FP8PD_FLAG_POS_OOB = 4u,     /* append position < 0 or >= max_pages * page_size: not written */
+  FP8PD_FLAG_INTERNAL = 8u     /* a split covered more pages than the kernel holds (a planner
+                                  bug): that split is left out */
 };
 
 /*
@@ -145,8 +148,9 @@ enum {
  *   sm_scale     finite, > 0.
  *   out          float32 [B, Hq, D]; stride[2] must be 1, rows 16-byte aligned.
  *   stream       CUDA stream.
- * Launches one split kernel, plus one combine kernel when the planner splits
- * the keys of a sequence over several thread blocks. The split partials live
+ * Launches one kernel. When the planner splits the keys of a sequence over
+ * several thread blocks, the last block of each (sequence, KV head) merges
+ * the splits. The split partials and the blocks' ticket counters live
  * in a library-owned per-device workspace: it grows on demand outside stream
  * capture; under capture a call that would need to grow it fails with
  * FP8PD_ERR_CAPTURE_WORKSPACE (call fp8pd_reserve_workspace, or run the call
@@ -191,8 +195,8 @@ typedef struct fp8pd_plan_info {
   int32_t num_splits;        /* thread blocks per (sequence, KV head, head group) */
   int32_t head_groups;       /* ceil(G / 8) query-head groups per KV head */
   int32_t grid_blocks;       /* split-kernel thread blocks */
-  int32_t combine;           /* 1 if a combine kernel follows */
-  uint64_t workspace_bytes;  /* split workspace the call needs (0 if no combine) */
+  int32_t combine;           /* 1 if the keys are split (the last block merges the splits) */
+  uint64_t workspace_bytes;  /* split workspace the call needs (0 if not split) */
 } fp8pd_plan_info;
 
 /* Plans a decode-attention call (same argument rules; nothing launched). */
@@ -209,9 +213,13 @@ int fp8pd_check_errors(fp8pd_stream_t stream, uint32_t* flags);
 
 /* Options (process-wide). */
 enum {
-  FP8PD_OPT_NUM_SPLITS = 1,  /* 0 = planner chooses (default); n > 0 forces n splits */
-  FP8PD_OPT_VARIANT = 2      /* 0 = auto; 1 = tensor-core (mma) split kernel;
+  FP8PD_OPT_NUM_SPLITS = 1,  /* 0 = planner chooses (default); n > 0 asks for n splits (raised
+                                so that no split covers more than 256 pages, capped at 256
+                                splits and at the number of pages) */
+  FP8PD_OPT_VARIANT = 2,     /* 0 = auto; 1 = tensor-core (mma) split kernel;
                                 2 = CUDA-core (f32 FMA) split kernel */
+  FP8PD_OPT_K_DECODE = 3     /* E4M3 -> f16 decode of K: 0 = bit assembly (default),
+                                1 = hardware cvt.rn.f16x2.e4m3x2 */
 };
 int fp8pd_set_option(int32_t option, int64_t value);
 int64_t fp8pd_get_option(int32_t option);
@@ -231,14 +239,14 @@ typedef struct fp8pd_run_info {
 int fp8pd_last_run_info(fp8pd_run_info* info);
 
 /* Device timing of the library's own kernels (for benchmarks): while
- * enabled, each attention call records CUDA events around its split kernel
- * and its combine kernel on the call's stream. fp8pd_timing_collect waits
- * for those events, returns the summed milliseconds and launch counts since
- * the last collect, and resets them. Enabling allocates events; do not
- * enable during stream capture. */
+ * enabled, each attention call records CUDA events around its kernel, and
+ * each append call around its kernel, on the call's stream (eager calls only;
+ * do not enable while a stream is capturing). fp8pd_timing_collect waits for
+ * those events, returns the summed milliseconds and launch counts since the
+ * last collect, and resets them. Enabling allocates events lazily. */
 int fp8pd_timing_enable(int32_t on);
-int fp8pd_timing_collect(double* split_ms, double* combine_ms, int32_t* split_launches,
-                         int32_t* combine_launches);
+int fp8pd_timing_collect(double* attention_ms, int32_t* attention_launches, double* append_ms,
+                         int32_t* append_launches);
 
 /* Human-readable status text (static storage). */
 const char* fp8pd_status_string(int32_t status);

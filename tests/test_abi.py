@@ -145,7 +145,18 @@ def test_planner_fills_the_device_with_enough_work_per_split(F):
     p = _plan(F, 1, 64, 8, 128, 64, 2049)
     assert p["num_splits"] > 16 and p["combine"] == 1
     assert 2049 / p["num_splits"] >= 4
-    assert p["workspace_bytes"] == 1 * 64 * p["num_splits"] * (128 + 2) * 4
+    S = p["num_splits"]
+    assert p["workspace_bytes"] >= 1 * 64 * S * (128 + 2) * 4 + 8 * 4
+    assert p["workspace_bytes"] <= 1 * 64 * S * (128 + 2) * 4 + 8 * 4 + 512
+    # no split may cover more than 256 pages: 131,072 keys on 16-token pages
+    p = _plan(F, 64, 64, 8, 64, 16, 8193)
+    assert p["num_splits"] >= 33 and 8193 / p["num_splits"] <= 256
+    assert p["num_splits"] <= 256
+    # more than 256 x 256 attended pages in one sequence is refused
+    with pytest.raises(F.Fp8pdError) as e:
+        _plan(F, 1, 8, 8, 128, 16, 256 * 256 + 1)
+    assert e.value.status == -10
+    assert _plan(F, 1, 8, 8, 128, 16, 256 * 256 + 1, window=4096)["num_splits"] >= 1
     # short window: one split, no combine, no workspace
     p = _plan(F, 64, 64, 8, 64, 16, 513, window=128)
     assert p["num_splits"] == 1 and p["combine"] == 0 and p["workspace_bytes"] == 0
@@ -158,5 +169,8 @@ def test_planner_fills_the_device_with_enough_work_per_split(F):
     try:
         assert _plan(F, 4, 32, 8, 128, 16, 100)["num_splits"] == 5
         assert _plan(F, 4, 32, 8, 128, 16, 3)["num_splits"] == 3
+        assert _plan(F, 4, 32, 8, 128, 16, 2000)["num_splits"] == 8    # raised: <= 256 pages each
+        F.fp8pd_set_option(F.OPT_NUM_SPLITS, 1000)
+        assert _plan(F, 4, 32, 8, 128, 16, 5000)["num_splits"] == 256  # capped
     finally:
         F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
