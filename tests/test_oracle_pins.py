@@ -420,6 +420,5 @@ def test_append_writes_only_the_new_slot():
                 small = np.abs(quot) <= 464          # the library cast agrees up to here
                 assert np.array_equal(got[small], lib[small])
                 assert np.all((got[~small] & 0x7F) == 0x7E)   # beyond it E4M3 saturates
-                assert (~small).any() or b > 0 or h > 0 or True
     assert np.array_equal(kp[~touched], k0[~touched])
     assert np.array_equal(vp[~touched], v0[~touched])
