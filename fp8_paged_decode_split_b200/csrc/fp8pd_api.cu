@@ -24,7 +24,7 @@ constexpr int kMaxDevices = 64;
 thread_local int32_t t_last_cuda_error = 0;
 thread_local fp8pd_run_info t_run_info = {};
 std::atomic<int64_t> g_calls{0}, g_appends{0}, g_launches{0};
-std::atomic<int64_t> g_opt_num_splits{0}, g_opt_variant{0}, g_opt_k_decode{0};
+std::atomic<int64_t> g_opt_num_splits{0}, g_opt_variant{0}, g_opt_k_decode{1};
 
 struct Workspace {
   void* ptr = nullptr;
@@ -108,6 +108,7 @@ bool same_pool_shape(const fp8pd_tensor* a, const fp8pd_tensor* b) {
 
 struct Plan {
   int num_splits = 1;
+  int chunk_pages = 1;
   int head_groups = 1;
   int grid_blocks = 0;
   int combine = 0;
@@ -123,9 +124,12 @@ int current_device(int* dev) {
   return FP8PD_OK;
 }
 
-// Splits per (sequence, KV head, head group): enough thread blocks to fill
-// whole waves of the device, each split keeping >= 256 keys of work, no split
-// covering more than kMaxSplitPages pages, at most kMaxSplits splits.
+// Splits per (sequence, KV head, head group). Split s covers pages
+// [s * chunk, (s+1) * chunk) of a sequence's attended range, so every block
+// has the same amount of work whatever the sequence lengths (blocks past the
+// end of a short sequence finish at once). The count fills whole waves of the
+// device with >= 512 keys per split, never more than 16,384 keys per split
+// (the kernel's per-warp tile list) nor more than kMaxSplits splits.
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, Plan* plan) {
@@ -135,10 +139,12 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
   int64_t pages = max_pages;
   if (window > 0) pages = std::min<int64_t>(pages, (window + ps - 1) / ps + 1);
   pages = std::max<int64_t>(pages, 1);
-  const int64_t s_min = (pages + fp8pd::kMaxSplitPages - 1) / fp8pd::kMaxSplitPages;
-  const int64_t min_pages = std::max(1, 256 / ps);
+  const int64_t max_chunk = std::max<int64_t>(1, fp8pd::kMaxSplitTokens / ps);
+  const int64_t s_min = (pages + max_chunk - 1) / max_chunk;
+  if (s_min > fp8pd::kMaxSplits) return FP8PD_ERR_TOO_LARGE;  // > 4 Mi keys in one sequence
+  const int64_t min_chunk = std::max(1, 512 / ps);
   const int64_t s_max = std::min<int64_t>(
-      fp8pd::kMaxSplits, std::max<int64_t>(s_min, (pages + min_pages - 1) / min_pages));
+      fp8pd::kMaxSplits, std::max<int64_t>(s_min, (pages + min_chunk - 1) / min_chunk));
   int64_t S = 1;
   const int64_t forced = g_opt_num_splits.load();
   if (forced > 0) {
@@ -156,7 +162,7 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
     for (int64_t s = 1; s <= s_max; ++s) {
       const double waves = static_cast<double>(units * s) / static_cast<double>(slots);
       const double eff = waves / std::ceil(waves);
-      if (eff >= 0.9) {
+      if (eff >= 0.85) {
         best = s;
         best_eff = eff;
         break;
@@ -169,8 +175,10 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
     S = best;
   }
   S = std::max<int64_t>(S, s_min);
-  if (S > fp8pd::kMaxSplits) return FP8PD_ERR_TOO_LARGE;  // > 65,536 attended pages per sequence
+  const int64_t chunk = (pages + S - 1) / S;
+  S = (pages + chunk - 1) / chunk;
   plan->num_splits = static_cast<int>(S);
+  plan->chunk_pages = static_cast<int>(chunk);
   plan->grid_blocks = static_cast<int>(std::min<int64_t>(INT32_MAX, units * S));
   plan->combine = S > 1 ? 1 : 0;
   plan->counters_bytes = S > 1 ? align256(static_cast<size_t>(units) * sizeof(int)) : 0;
@@ -348,6 +356,7 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
   if (r) return r;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   p.num_splits = plan.num_splits;
+  p.chunk_pages = plan.chunk_pages;
   p.head_groups = plan.head_groups;
   if (plan.combine) {
     void* ws = nullptr;

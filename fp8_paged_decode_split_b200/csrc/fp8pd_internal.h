@@ -31,6 +31,7 @@ struct DecodeParams {
   float* part_ml;             // [B * Hq * S, 2] split (max, sum) in log2 units
   int* counters;              // [B * Hkv * head_groups] tickets, zero between calls
   int B, Hq, Hkv, G, D, ps, num_pages, max_pages, window, num_splits, head_groups;
+  int chunk_pages;            // pages per split (the last split of a sequence may have fewer)
   float sm_scale_log2;        // sm_scale * log2(e)
 };
 
@@ -65,7 +66,8 @@ cudaError_t read_and_clear_error_word(uint32_t* value, cudaStream_t s);
 
 constexpr int kHeadsPerGroup = 8;   // query heads one thread block serves (MMA N)
 constexpr int kTileTokens = 16;     // tokens per MMA row tile
-constexpr int kMaxSplitPages = 256; // pages one split may cover (their ids live in smem)
+constexpr int kMaxWarpTiles = 256;  // 16-token tiles one warp takes in a split (ids in smem)
+constexpr int kMaxSplitTokens = kMaxWarpTiles * 4 * kTileTokens;  // 16,384 keys per split
 constexpr int kMaxSplits = 256;     // splits per (sequence, KV head, head group)
 
 }  // namespace fp8pd

@@ -195,24 +195,34 @@ __device__ __forceinline__ float2 ldcg2(const float* p) {
   return v;
 }
 
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src) : "memory");
+}
+
 template <int D>
 struct Cfg {
   static constexpr int NW = 4;                                        // warps per block
   static constexpr int NS = (D == 64) ? 6 : (D == 128) ? 3 : 2;       // ring stages per warp
   static constexpr int TILE = kTileTokens * D;                        // bytes of a K or V tile
-  static constexpr int STAGE = 2 * TILE;
+  static constexpr int STAGE = 2 * TILE + 16;                         // K, V, then k / v scale
   static constexpr int WARP_BYTES = NS * STAGE;
-  static constexpr int PIPE_BYTES = NW * WARP_BYTES;
+  static constexpr int PIPE_BYTES = (NW * WARP_BYTES + 127) / 128 * 128;
   static constexpr bool Q_IN_SMEM = (D > 256);                        // q fragments in smem
   static constexpr int QFRAG_BYTES = Q_IN_SMEM ? (D / 16) * 32 * 8 : 0;
   static constexpr int PROW = 24;                                     // halves per P row
   static constexpr int PBUF_BYTES = NW * 2 * 8 * PROW * 2;
-  static constexpr int PAGE_BYTES = kMaxSplitPages * 12;              // page id, k / v scale
-  static constexpr int MISC_FLOATS = 8 + NW * 8 * 2 + 4;
-  static constexpr int SMEM = PIPE_BYTES + QFRAG_BYTES + PBUF_BYTES + PAGE_BYTES + MISC_FLOATS * 4;
+  static constexpr int PID_BYTES = NW * kMaxWarpTiles * 4;            // each warp's page ids
+  static constexpr int MISC_FLOATS = NW * 8 * 2 + 4;
+  static constexpr int SMEM =
+      PIPE_BYTES + QFRAG_BYTES + PBUF_BYTES + PID_BYTES + MISC_FLOATS * 4;
   static constexpr int MIN_BLOCKS = (D == 512) ? 1 : (D == 256) ? 2 : 4;
   static_assert(NW * 8 * D * 4 <= PIPE_BYTES, "merge scratch must fit in the ring");
-  static_assert(8 * D * 4 <= PIPE_BYTES, "q staging must fit in the ring");
   static_assert(8 * kMaxSplits * 4 <= PIPE_BYTES, "combine weights must fit in the ring");
 };
 
@@ -229,9 +239,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   uint2* qfrag_s = reinterpret_cast<uint2*>(smem + C::PIPE_BYTES);
   __half* pbuf = reinterpret_cast<__half*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES);
   int32_t* s_pid = reinterpret_cast<int32_t*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES + C::PBUF_BYTES);
-  float* s_ks = reinterpret_cast<float*>(s_pid + kMaxSplitPages);
-  float* s_vs = s_ks + kMaxSplitPages;
-  float* misc = s_vs + kMaxSplitPages;
+  float* misc = reinterpret_cast<float*>(s_pid + C::NW * kMaxWarpTiles);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, grp = lane >> 2, qd = lane & 3;
@@ -242,6 +250,9 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   const int nheads = min(8, p.G - hg * 8);
 
   // ---- the keys this block attends: [t0, t1) ------------------------------
+  // Split s of a sequence covers pages [first + s * chunk, first + (s+1) * chunk)
+  // of its attended range: equal-sized work per block whatever the length,
+  // and the blocks past the end of a short sequence have nothing to do.
   int L = __ldg(p.lens + (int64_t)b * p.lens_s);
   if (L < 0 || L > p.max_pages * p.ps) {
     if (tid == 0 && split == 0 && blockIdx.y == 0) raise_flag(FP8PD_FLAG_SEQLEN_OOB);
@@ -250,110 +261,99 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   const int lo = p.window > 0 ? max(0, L - p.window) : 0;
   const int first_page = lo / p.ps;
   const int n_pages = (L > lo) ? (L - 1) / p.ps - first_page + 1 : 0;
-  const int chunk = (n_pages + p.num_splits - 1) / p.num_splits;
-  const int pg0 = first_page + split * chunk;
-  int pg1 = min(first_page + n_pages, pg0 + chunk);
-  if (pg1 - pg0 > kMaxSplitPages) {  // the planner never does this; refuse rather than overflow
-    if (tid == 0) raise_flag(FP8PD_FLAG_INTERNAL);
-    pg1 = pg0;
-  }
+  const int pg0 = first_page + split * p.chunk_pages;
+  const int pg1 = min(first_page + n_pages, pg0 + p.chunk_pages);
   const int t0 = max(lo, pg0 * p.ps);
   const int t1 = min(L, pg1 * p.ps);
   const int tile_first = t0 / kTileTokens;
   const int n_tiles = (t1 > t0) ? (t1 + kTileTokens - 1) / kTileTokens - tile_first : 0;
+  int my_tiles = (n_tiles > warp) ? (n_tiles - warp + C::NW - 1) / C::NW : 0;
+  if (my_tiles > kMaxWarpTiles) {  // the planner never does this; refuse rather than overflow
+    if (lane == 0) raise_flag(FP8PD_FLAG_INTERNAL);
+    my_tiles = 0;
+  }
   const int32_t* trow = p.table + (int64_t)b * p.tab_sb;
 
-  // ---- pages of the split, their scales; q of the head group ---------------
-  float vmax = 0.f;
-  for (int i = tid; i < pg1 - pg0; i += 128) {
-    const int page = __ldg(trow + (int64_t)(pg0 + i) * p.tab_sp);
-    const bool ok = (unsigned)page < (unsigned)p.num_pages;
-    float ks = 0.f, vs = 0.f;
-    if (ok) {
-      ks = __ldg(p.ks + (int64_t)page * p.ks_sp + (int64_t)kvh * p.ks_sh);
-      vs = __ldg(p.vs + (int64_t)page * p.vs_sp + (int64_t)kvh * p.vs_sh);
-    } else if (hg == 0) {
-      raise_flag(FP8PD_FLAG_PAGE_OOB);
+  // ---- warp-local setup: this warp's page ids, q fragments ------------------
+  int32_t* wpid = s_pid + warp * kMaxWarpTiles;
+  for (int j = lane; j < my_tiles; j += 32) {
+    const int lp = (tile_first + warp + C::NW * j) * kTileTokens / p.ps;
+    int page = __ldg(trow + (int64_t)lp * p.tab_sp);
+    if ((unsigned)page >= (unsigned)p.num_pages) {
+      if (hg == 0) raise_flag(FP8PD_FLAG_PAGE_OOB);
+      page = -1;
     }
-    s_pid[i] = ok ? page : -1;
-    s_ks[i] = ks;
-    s_vs[i] = vs;
-    vmax = fmaxf(vmax, fabsf(vs));
+    wpid[j] = page;
   }
-  float* qs = reinterpret_cast<float*>(pipe);  // [8][D] staging
+  // Lane (g, q) holds query head g of the group at head-dim entries
+  // 64jj + 16q + {0..15}; the k16 block (jj, i) covers entries
+  // 64jj + 16q + 4i + {0..3}. Bit-assembly K pairs bytes (0,2) and (1,3):
+  // k = 2q -> +0, 2q+1 -> +2, 2q+8 -> +1, 2q+9 -> +3; hardware-cvt K pairs
+  // (0,1) and (2,3).
+  const bool q_head_ok = grp < nheads;
+  const uint16_t* qrow = p.q + (int64_t)b * p.q_sb + (int64_t)(head0 + (q_head_ok ? grp : 0)) * p.q_sh;
   float qmax = 0.f;
-  for (int i = tid; i < 8 * D; i += 128) {
-    const int n = i / D, d = i - n * D;
-    float x = 0.f;
-    if (n < nheads)
-      x = bf16_bits_to_float(p.q[(int64_t)b * p.q_sb + (int64_t)(head0 + n) * p.q_sh +
-                                 (int64_t)d * p.q_sd]);
-    qs[i] = x;
-    qmax = fmaxf(qmax, fabsf(x));
+  if (q_head_ok) {
+#pragma unroll 4
+    for (int e = 0; e < D / 4; ++e) {
+      const int d = 64 * (e >> 4) + 16 * qd + (e & 15);
+      qmax = fmaxf(qmax, fabsf(bf16_bits_to_float(__ldg(qrow + (int64_t)d * p.q_sd))));
+    }
   }
   qmax = warp_max(qmax);
-  vmax = warp_max(vmax);
-  if (lane == 0) {
-    misc[warp] = qmax;
-    misc[4 + warp] = vmax;
-  }
-  __syncthreads();
-  qmax = fmaxf(fmaxf(misc[0], misc[1]), fmaxf(misc[2], misc[3]));
-  // V reference scale: the split's largest |v_scale|, so every P * v_scale /
-  // vref stays <= 1 and its f16 hi/lo split keeps full relative precision.
-  float vref = fmaxf(fmaxf(misc[4], misc[5]), fmaxf(misc[6], misc[7]));
-  if (!(vref > 0.f) || !isfinite(vref)) vref = 1.f;
-  const float inv_vref = 1.f / vref;
   // q' = q * 2^(15 - e) puts max|q'| in [2^14, 2^15): exact in f16 for every
   // element above max|q| * 2^-28 (bf16 has 8 significant bits).
   int qe = 0;
   if (qmax > 0.f && isfinite(qmax)) frexpf(qmax, &qe);
   qe = max(qe, -111);
   const float qmul = ldexpf(1.f, 15 - qe);
-  // kfac(page) = sm_scale * log2(e) * 2^8 / qmul * k_scale(page): the 2^8
-  // undoes the f16 offset of the decoded K.
+  // kfac = sm_scale * log2(e) * 2^8 / qmul * k_scale(page): the 2^8 undoes
+  // the f16 offset of the decoded K.
   const float score_base = p.sm_scale_log2 * 256.f / qmul;
-
-  // B fragments of q (column n = query head grp of the group). The k16 block
-  // (jj, i) covers head-dim entries 64jj + 16q + 4i + {0..3} of lane quad q.
-  // Bit-assembly K pairs bytes (0,2) and (1,3): k = 2q -> +0, 2q+1 -> +2,
-  // 2q+8 -> +1, 2q+9 -> +3. Hardware-cvt K pairs (0,1) and (2,3).
+  auto qval = [&](int d) -> float {
+    return q_head_ok ? bf16_bits_to_float(__ldg(qrow + (int64_t)d * p.q_sd)) * qmul : 0.f;
+  };
   uint32_t qf[C::Q_IN_SMEM ? 1 : KB][2];
 #pragma unroll
   for (int kb = 0; kb < KB; ++kb) {
-    const int jj = kb >> 2, i = kb & 3;
-    const float* qrow = qs + grp * D + 64 * jj + 16 * qd + 4 * i;
+    if constexpr (C::Q_IN_SMEM) {
+      if ((kb & 3) != warp) continue;  // the four warps share the work
+    }
+    const int d = 64 * (kb >> 2) + 16 * qd + 4 * (kb & 3);
     uint32_t r0, r1;
     if constexpr (KCVT) {
-      r0 = pack_f16x2(qrow[0] * qmul, qrow[1] * qmul);
-      r1 = pack_f16x2(qrow[2] * qmul, qrow[3] * qmul);
+      r0 = pack_f16x2(qval(d + 0), qval(d + 1));
+      r1 = pack_f16x2(qval(d + 2), qval(d + 3));
     } else {
-      r0 = pack_f16x2(qrow[0] * qmul, qrow[2] * qmul);
-      r1 = pack_f16x2(qrow[1] * qmul, qrow[3] * qmul);
+      r0 = pack_f16x2(qval(d + 0), qval(d + 2));
+      r1 = pack_f16x2(qval(d + 1), qval(d + 3));
     }
     if constexpr (C::Q_IN_SMEM) {
-      if (warp == 0) qfrag_s[kb * 32 + lane] = make_uint2(r0, r1);
+      qfrag_s[kb * 32 + lane] = make_uint2(r0, r1);
     } else {
       qf[kb][0] = r0;
       qf[kb][1] = r1;
     }
   }
-  __syncthreads();  // q staging (in the ring) is dead from here on
+  if constexpr (C::Q_IN_SMEM) __syncthreads();
+  __syncwarp();
 
   // ---- per-warp pipeline over 16-token tiles --------------------------------
   const uint32_t wpipe = smem_u32(pipe + warp * C::WARP_BYTES);
   __half* p_hi = pbuf + warp * (2 * 8 * C::PROW);
   __half* p_lo = p_hi + 8 * C::PROW;
-  const int my_tiles = (n_tiles > warp) ? (n_tiles - warp + C::NW - 1) / C::NW : 0;
   const uint8_t* kbase = p.k + (int64_t)kvh * p.k_sh;
   const uint8_t* vbase = p.v + (int64_t)kvh * p.v_sh;
+  const float* ksbase = p.ks + (int64_t)kvh * p.ks_sh;
+  const float* vsbase = p.vs + (int64_t)kvh * p.vs_sh;
 
+  // Copies tile j of this warp into ring stage `stage`: K and V rows (16-byte
+  // cp.async per lane), then the page's k and v scales (4 bytes each).
   auto issue = [&](int j, int stage) {
-    const int tok0 = (tile_first + warp + C::NW * j) * kTileTokens;
-    const int lp = tok0 / p.ps;
-    const int page = s_pid[lp - pg0];
+    const int page = wpid[j];
     if (page < 0) return;
-    const int slot0 = tok0 - lp * p.ps;
+    const int tok0 = (tile_first + warp + C::NW * j) * kTileTokens;
+    const int slot0 = tok0 - (tok0 / p.ps) * p.ps;
     const uint8_t* gk = kbase + (int64_t)page * p.k_sp + (int64_t)slot0 * p.k_st;
     const uint8_t* gv = vbase + (int64_t)page * p.v_sp + (int64_t)slot0 * p.v_st;
     const uint32_t sk = wpipe + stage * C::STAGE;
@@ -366,6 +366,8 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       cp_async16(sk + k_off<D>(r, c), gk + (int64_t)r * p.k_st + c * 16);
       cp_async16(sv + v_off<D>(r, c), gv + (int64_t)r * p.v_st + c * 16);
     }
+    if (lane == 0) cp_async4(sv + C::TILE, ksbase + (int64_t)page * p.ks_sp);
+    if (lane == 1) cp_async4(sv + C::TILE + 4, vsbase + (int64_t)page * p.vs_sp);
   };
 
   float O[D / 32][2][4];
@@ -377,6 +379,9 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       for (int c = 0; c < 4; ++c) O[jb][h][c] = 0.f;
   float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F;  // running max, heads 2qd / 2qd+1 (log2 units)
   float l0 = 0.f, l1 = 0.f;                      // this lane's share of the running sums
+  // Running V reference scale: the largest |v_scale| seen so far. O holds
+  // sum P * v_scale / vref, so every f16 P operand stays <= 1 in magnitude.
+  float vref = 0.f;
 
 #pragma unroll 1
   for (int s = 0; s < C::NS - 1; ++s) {
@@ -394,12 +399,14 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       cp_async_commit();
     }
     const int tok0 = (tile_first + warp + C::NW * j) * kTileTokens;
-    const int li = tok0 / p.ps - pg0;
-    const bool page_ok = s_pid[li] >= 0;
-    const float kfac = score_base * s_ks[li];
-    const float vsr = s_vs[li] * inv_vref;
+    const bool page_ok = wpid[j] >= 0;
     const uint32_t sk = wpipe + (j % C::NS) * C::STAGE;
     const uint32_t sv = sk + C::TILE;
+    float kfac = 0.f, vs = 0.f;
+    if (page_ok) {
+      kfac = score_base * __uint_as_float(lds32(sv + C::TILE));
+      vs = __uint_as_float(lds32(sv + C::TILE + 4));
+    }
 
     // -- S[token][head] = K q'^T (two independent accumulator chains) --------
     float Sa[4] = {0.f, 0.f, 0.f, 0.f}, Sb[4] = {0.f, 0.f, 0.f, 0.f};
@@ -455,32 +462,38 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, o));
     }
     const float mn0 = fmaxf(m0, tm0), mn1 = fmaxf(m1, tm1);
-    if (__any_sync(0xffffffffu, (mn0 > m0) || (mn1 > m1))) {
-      const float c0 = (mn0 > m0) ? exp2f(m0 - mn0) : 1.f;  // exp2(-inf) = 0 for a first max
-      const float c1 = (mn1 > m1) ? exp2f(m1 - mn1) : 1.f;
+    const float vabs = fabsf(vs);
+    const bool grow_v = vabs > vref;  // warp-uniform: one scale per tile
+    if (grow_v || __any_sync(0xffffffffu, (mn0 > m0) || (mn1 > m1))) {
+      const float c0 = (mn0 > m0) ? fast_exp2(m0 - mn0) : 1.f;  // exp2(-inf) = 0 for a first max
+      const float c1 = (mn1 > m1) ? fast_exp2(m1 - mn1) : 1.f;
+      const float fv = grow_v ? vref / vabs : 1.f;
       l0 *= c0;
       l1 *= c1;
+      const float o0 = c0 * fv, o1 = c1 * fv;
 #pragma unroll
       for (int jb = 0; jb < D / 32; ++jb)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          O[jb][h][0] *= c0;
-          O[jb][h][1] *= c1;
-          O[jb][h][2] *= c0;
-          O[jb][h][3] *= c1;
+          O[jb][h][0] *= o0;
+          O[jb][h][1] *= o1;
+          O[jb][h][2] *= o0;
+          O[jb][h][3] *= o1;
         }
       m0 = mn0;
       m1 = mn1;
+      if (grow_v) vref = vabs;
     }
     const float mb0 = (m0 == -CUDART_INF_F) ? 0.f : m0;
     const float mb1 = (m1 == -CUDART_INF_F) ? 0.f : m1;
-    const float p00 = exp2f(s00 - mb0), p01 = exp2f(s01 - mb1);
-    const float p10 = exp2f(s10 - mb0), p11 = exp2f(s11 - mb1);
+    const float p00 = fast_exp2(s00 - mb0), p01 = fast_exp2(s01 - mb1);
+    const float p10 = fast_exp2(s10 - mb0), p11 = fast_exp2(s11 - mb1);
     l0 += p00 + p10;
     l1 += p01 + p11;
 
-    // -- P (times the page's V scale ratio) as f16 hi + lo, transposed via smem
+    // -- P * v_scale / vref as f16 hi + lo, transposed through shared memory
     {
+      const float vsr = (vref > 0.f) ? vs / vref : 0.f;
       const float w00 = p00 * vsr, w01 = p01 * vsr, w10 = p10 * vsr, w11 = p11 * vsr;
       const __half h00 = __float2half_rn(w00), h01 = __float2half_rn(w01);
       const __half h10 = __float2half_rn(w10), h11 = __float2half_rn(w11);
@@ -533,15 +546,16 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     l1 += __shfl_xor_sync(0xffffffffu, l1, o);
   }
   __syncthreads();  // every warp is done with its ring
-  float* Os = reinterpret_cast<float*>(pipe);  // [NW][8][D]
-  float* ml = misc + 8;                        // [NW][8][2]
+  float* Os = reinterpret_cast<float*>(pipe);  // [NW][8][D], already times 2^8 * vref
+  float* ml = misc;                            // [NW][8][2]
+  const float fold = 256.f * vref;             // f16 offset of the decoded V, V reference scale
 #pragma unroll
   for (int jb = 0; jb < D / 32; ++jb) {
     const int d = 32 * jb + 4 * grp;
-    *reinterpret_cast<float4*>(Os + (warp * 8 + 2 * qd) * D + d) =
-        make_float4(O[jb][0][0], O[jb][0][2], O[jb][1][0], O[jb][1][2]);
-    *reinterpret_cast<float4*>(Os + (warp * 8 + 2 * qd + 1) * D + d) =
-        make_float4(O[jb][0][1], O[jb][0][3], O[jb][1][1], O[jb][1][3]);
+    *reinterpret_cast<float4*>(Os + (warp * 8 + 2 * qd) * D + d) = make_float4(
+        O[jb][0][0] * fold, O[jb][0][2] * fold, O[jb][1][0] * fold, O[jb][1][2] * fold);
+    *reinterpret_cast<float4*>(Os + (warp * 8 + 2 * qd + 1) * D + d) = make_float4(
+        O[jb][0][1] * fold, O[jb][0][3] * fold, O[jb][1][1] * fold, O[jb][1][3] * fold);
   }
   if (grp == 0) {
     ml[(warp * 8 + 2 * qd) * 2 + 0] = m0;
@@ -551,7 +565,6 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   }
   __syncthreads();
 
-  const float fold = 256.f * vref;  // f16 offset of the decoded V, and the V reference scale
   constexpr float kLog2e = 1.4426950408889634f;
   const int S = p.num_splits;
   for (int it = tid; it < 8 * (D / 4); it += 128) {
@@ -567,7 +580,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
 #pragma unroll
       for (int w = 0; w < C::NW; ++w) {
         const float mw = ml[(w * 8 + n) * 2];
-        const float f = (mw == -CUDART_INF_F) ? 0.f : exp2f(mw - M);
+        const float f = (mw == -CUDART_INF_F) ? 0.f : fast_exp2(mw - M);
         const float4 o = *reinterpret_cast<const float4*>(Os + (w * 8 + n) * D + d);
         acc.x += f * o.x;
         acc.y += f * o.y;
@@ -582,18 +595,17 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       const float M2 = fmaxf(M, sl);
       float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
       if (M2 != -CUDART_INF_F) {
-        const float a = (M == -CUDART_INF_F) ? 0.f : exp2f(M - M2);
-        const float den = l * a + (p.sinks ? exp2f(sl - M2) : 0.f);
+        const float a = (M == -CUDART_INF_F) ? 0.f : fast_exp2(M - M2);
+        const float den = l * a + (p.sinks ? fast_exp2(sl - M2) : 0.f);
         if (den > 0.f) {
-          const float f = a * fold / den;
+          const float f = a / den;
           r = make_float4(acc.x * f, acc.y * f, acc.z * f, acc.w * f);
         }
       }
       *reinterpret_cast<float4*>(p.out + (int64_t)b * p.o_sb + (int64_t)head * p.o_sh + d) = r;
     } else {
       const int64_t row = ((int64_t)b * p.Hq + head) * S + split;
-      *reinterpret_cast<float4*>(p.part_o + row * D + d) =
-          make_float4(acc.x * fold, acc.y * fold, acc.z * fold, acc.w * fold);
+      *reinterpret_cast<float4*>(p.part_o + row * D + d) = acc;
       if (d == 0) *reinterpret_cast<float2*>(p.part_ml + row * 2) = make_float2(M, l);
     }
   }
@@ -605,7 +617,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   // and resets the counter for the next call. No block ever waits for another.
   __threadfence();
   __syncthreads();
-  int* last_flag = reinterpret_cast<int*>(misc + 8 + C::NW * 8 * 2);
+  int* last_flag = reinterpret_cast<int*>(misc + C::NW * 8 * 2);
   const int64_t unit = (int64_t)b * gridDim.y + blockIdx.y;
   if (tid == 0) {
     const int prev = atomicAdd(p.counters + unit, 1);
@@ -615,7 +627,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   if (!*last_flag) return;
   __threadfence();
 
-  float* wts = reinterpret_cast<float*>(pipe);  // [8][S] split weights / den
+  float* wts = reinterpret_cast<float*>(pipe);  // [8][kMaxSplits] split weight / den
   for (int n = warp; n < nheads; n += C::NW) {
     const int head = head0 + n;
     const float* pml = p.part_ml + ((int64_t)b * p.Hq + head) * S * 2;
@@ -628,28 +640,31 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     if (M2 != -CUDART_INF_F) {
       for (int s = lane; s < S; s += 32) {
         const float2 ml2 = ldcg2(pml + 2 * s);
-        if (ml2.x != -CUDART_INF_F) den += ml2.y * exp2f(ml2.x - M2);
+        if (ml2.x != -CUDART_INF_F) den += ml2.y * fast_exp2(ml2.x - M2);
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-      if (p.sinks) den += exp2f(sl - M2);
+      if (p.sinks) den += fast_exp2(sl - M2);
     }
     const float inv = (M2 != -CUDART_INF_F && den > 0.f) ? 1.f / den : 0.f;
     for (int s = lane; s < S; s += 32) {
       const float ms = ldcg2(pml + 2 * s).x;
-      wts[n * kMaxSplits + s] = (inv == 0.f || ms == -CUDART_INF_F) ? 0.f : exp2f(ms - M2) * inv;
+      wts[n * kMaxSplits + s] = (inv == 0.f || ms == -CUDART_INF_F) ? 0.f : fast_exp2(ms - M2) * inv;
     }
   }
   __syncthreads();
+  // Every split wrote its row (zeros for an empty one), so the weighted sum
+  // needs no branch and its loads can all be in flight at once.
   for (int it = tid; it < nheads * (D / 4); it += 128) {
     const int n = it / (D / 4);
     const int d = (it - n * (D / 4)) * 4;
     const int head = head0 + n;
     const float* po = p.part_o + ((int64_t)b * p.Hq + head) * S * D + d;
+    const float* wn = wts + n * kMaxSplits;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
     for (int s = 0; s < S; ++s) {
-      const float w = wts[n * kMaxSplits + s];
-      if (w == 0.f) continue;
+      const float w = wn[s];
       const float4 o = ldcg4(po + (int64_t)s * D);
       acc.x += w * o.x;
       acc.y += w * o.y;

@@ -148,15 +148,15 @@ def test_planner_fills_the_device_with_enough_work_per_split(F):
     S = p["num_splits"]
     assert p["workspace_bytes"] >= 1 * 64 * S * (128 + 2) * 4 + 8 * 4
     assert p["workspace_bytes"] <= 1 * 64 * S * (128 + 2) * 4 + 8 * 4 + 512
-    # no split may cover more than 256 pages: 131,072 keys on 16-token pages
-    p = _plan(F, 64, 64, 8, 64, 16, 8193)
-    assert p["num_splits"] >= 33 and 8193 / p["num_splits"] <= 256
+    # no split may cover more than 16,384 keys: 1 Mi keys on 16-token pages
+    p = _plan(F, 64, 64, 8, 64, 16, 65537)
+    assert p["num_splits"] >= 65 and 65537 * 16 / p["num_splits"] <= 16384 + 16
     assert p["num_splits"] <= 256
-    # more than 256 x 256 attended pages in one sequence is refused
+    # more than 256 splits of 16,384 keys in one sequence is refused
     with pytest.raises(F.Fp8pdError) as e:
-        _plan(F, 1, 8, 8, 128, 16, 256 * 256 + 1)
+        _plan(F, 1, 8, 8, 128, 16, 256 * 1024 + 1)
     assert e.value.status == -10
-    assert _plan(F, 1, 8, 8, 128, 16, 256 * 256 + 1, window=4096)["num_splits"] >= 1
+    assert _plan(F, 1, 8, 8, 128, 16, 256 * 1024 + 1, window=4096)["num_splits"] >= 1
     # short window: one split, no combine, no workspace
     p = _plan(F, 64, 64, 8, 64, 16, 513, window=128)
     assert p["num_splits"] == 1 and p["combine"] == 0 and p["workspace_bytes"] == 0
@@ -169,8 +169,8 @@ def test_planner_fills_the_device_with_enough_work_per_split(F):
     try:
         assert _plan(F, 4, 32, 8, 128, 16, 100)["num_splits"] == 5
         assert _plan(F, 4, 32, 8, 128, 16, 3)["num_splits"] == 3
-        assert _plan(F, 4, 32, 8, 128, 16, 2000)["num_splits"] == 8    # raised: <= 256 pages each
+        assert _plan(F, 4, 32, 8, 128, 16, 6000)["num_splits"] == 6    # raised: <= 16,384 keys each
         F.fp8pd_set_option(F.OPT_NUM_SPLITS, 1000)
-        assert _plan(F, 4, 32, 8, 128, 16, 5000)["num_splits"] == 256  # capped
+        assert 240 <= _plan(F, 4, 32, 8, 128, 16, 5000)["num_splits"] <= 256  # capped
     finally:
         F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
