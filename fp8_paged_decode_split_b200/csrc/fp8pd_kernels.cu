@@ -307,9 +307,10 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   if (qmax > 0.f && isfinite(qmax)) frexpf(qmax, &qe);
   qe = max(qe, -111);
   const float qmul = ldexpf(1.f, 15 - qe);
-  // kfac = sm_scale * log2(e) * 2^8 / qmul * k_scale(page): the 2^8 undoes
-  // the f16 offset of the decoded K.
-  const float score_base = p.sm_scale_log2 * 256.f / qmul;
+  // kfac = sm_scale * log2(e) / qmul * k_scale(page), times 2^8 when K is
+  // decoded by bit assembly (which yields value * 2^-8); the hardware cvt
+  // yields the value itself.
+  const float score_base = p.sm_scale_log2 * (KCVT ? 1.f : 256.f) / qmul;
   auto qval = [&](int d) -> float {
     return q_head_ok ? bf16_bits_to_float(__ldg(qrow + (int64_t)d * p.q_sd)) * qmul : 0.f;
   };

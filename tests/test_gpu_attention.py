@@ -25,6 +25,14 @@ def F(cuda_device):
     return F
 
 
+@pytest.fixture(params=[1, 0], ids=["kcvt", "kbits"])
+def kdecode(F, request):
+    """Run a test with each E4M3 -> f16 decode of K (hardware cvt, bit assembly)."""
+    F.fp8pd_set_option(F.OPT_K_DECODE, request.param)
+    yield request.param
+    F.fp8pd_set_option(F.OPT_K_DECODE, 1)
+
+
 @pytest.fixture
 def splits(F):
     """Force a split count for one test; restore the planner afterwards."""
@@ -46,7 +54,7 @@ def _check_layer(F, case, li=0, lens=None, where=""):
 
 # --------------------------------------------------------------- workloads
 
-def test_tiny_config_full_size(F, cuda_device):
+def test_tiny_config_full_size(F, cuda_device, kdecode):
     case = W.make_case("tiny", cuda_device)
     _check_layer(F, case, where="tiny")
 
@@ -70,12 +78,12 @@ def test_llama_like_reduced_with_append(F, cuda_device, splits, nsplit):
 
 
 @pytest.mark.parametrize("name", ["gptoss_w128", "gptoss_full"])
-def test_gptoss_like_reduced_sinks(F, cuda_device, name):
+def test_gptoss_like_reduced_sinks(F, cuda_device, name, kdecode):
     case = W.make_case(name, cuda_device, B=3, seq_len=1000)
     _check_layer(F, case, where=name)
 
 
-def test_mixed_pool_two_geometries(F, cuda_device):
+def test_mixed_pool_two_geometries(F, cuda_device, kdecode):
     """A sliding layer (D=256, window) and a full layer (D=512) read one pool
     with a 65,536-byte page stride; N(0,2) values with 1% x20 outliers."""
     case = W.make_case("mixed", cuda_device, B=3, seq_len=(300, 1500))
@@ -97,7 +105,7 @@ def test_long_context_reduced_split(F, cuda_device, splits, nsplit):
 
 @pytest.mark.parametrize("D", [64, 128, 256, 512])
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (8, 2), (12, 4), (16, 1), (24, 2)])
-def test_head_dims_and_group_sizes(F, cuda_device, D, Hq, Hkv):
+def test_head_dims_and_group_sizes(F, cuda_device, D, Hq, Hkv, kdecode):
     spec = W.Spec("shape", B=2, ps=16, layers=(W.LayerSpec(Hq, Hkv, D, 0, 0.7 / math.sqrt(D)),),
                   seq_len=(17, 161), scale_mode="page", sinks=True, seed=D + Hq)
     _check_layer(F, W.make_case(spec, cuda_device), where=f"D={D} Hq={Hq} Hkv={Hkv}")
@@ -154,7 +162,7 @@ def test_zero_query_gives_mean_of_values(F, cuda_device):
 
 
 @pytest.mark.parametrize("qscale", [1e-6, 1e-3, 30.0, 3000.0])
-def test_query_magnitudes(F, cuda_device, qscale):
+def test_query_magnitudes(F, cuda_device, qscale, kdecode):
     case = _small(cuda_device)
     layer = case.layers[0]
     q = (layer.q.float() * qscale).to(torch.bfloat16)
@@ -163,7 +171,7 @@ def test_query_magnitudes(F, cuda_device, qscale):
     assert_attention_close(got, oracle_attention(lc, case.attend_lens), f"qscale={qscale}")
 
 
-def test_extreme_scales_and_subnormal_codes(F, cuda_device):
+def test_extreme_scales_and_subnormal_codes(F, cuda_device, kdecode):
     """Scales far from 1 and caches made of E4M3 subnormal codes only."""
     case = _small(cuda_device)
     layer = case.layers[0]
