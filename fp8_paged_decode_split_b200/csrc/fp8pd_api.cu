@@ -24,7 +24,7 @@ constexpr int kMaxDevices = 64;
 thread_local int32_t t_last_cuda_error = 0;
 thread_local fp8pd_run_info t_run_info = {};
 std::atomic<int64_t> g_calls{0}, g_appends{0}, g_launches{0};
-std::atomic<int64_t> g_opt_num_splits{0}, g_opt_variant{0}, g_opt_k_decode{1};
+std::atomic<int64_t> g_opt_num_splits{0}, g_opt_variant{0}, g_opt_k_decode{1}, g_opt_v_decode{1};
 
 struct Workspace {
   void* ptr = nullptr;
@@ -112,8 +112,12 @@ struct Plan {
   int head_groups = 1;
   int grid_blocks = 0;
   int combine = 0;
+  int num_groups = 1;
   size_t counters_bytes = 0;  // ticket counters (first in the workspace; all zero between calls)
   size_t ml_bytes = 0;        // split (max, sum) pairs
+  size_t o_bytes = 0;         // split numerators
+  size_t grp_ml_bytes = 0;    // merged groups of splits
+  size_t grp_o_bytes = 0;
   size_t workspace = 0;
 };
 
@@ -150,6 +154,8 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
   if (forced > 0) {
     S = std::min<int64_t>(forced, std::min<int64_t>(pages, fp8pd::kMaxSplits));
   } else if (units > 0) {
+    // At least 1.25 waves of blocks: with equal-sized splits the hardware
+    // scheduler then evens out ragged lengths; fewer would leave SMs idle.
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) {
       int v = 0;
@@ -157,22 +163,8 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
     }
     cudaGetLastError();
     const int64_t slots = static_cast<int64_t>(sms) * fp8pd::decode_mma_blocks_per_sm(D);
-    double best_eff = -1.0;
-    int64_t best = 1;
-    for (int64_t s = 1; s <= s_max; ++s) {
-      const double waves = static_cast<double>(units * s) / static_cast<double>(slots);
-      const double eff = waves / std::ceil(waves);
-      if (eff >= 0.85) {
-        best = s;
-        best_eff = eff;
-        break;
-      }
-      if (eff > best_eff + 1e-9) {
-        best_eff = eff;
-        best = s;
-      }
-    }
-    S = best;
+    S = std::min<int64_t>(s_max, (5 * slots + 4 * units - 1) / (4 * units));
+    S = std::max<int64_t>(S, 1);
   }
   S = std::max<int64_t>(S, s_min);
   const int64_t chunk = (pages + S - 1) / S;
@@ -181,11 +173,16 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
   plan->chunk_pages = static_cast<int>(chunk);
   plan->grid_blocks = static_cast<int>(std::min<int64_t>(INT32_MAX, units * S));
   plan->combine = S > 1 ? 1 : 0;
-  plan->counters_bytes = S > 1 ? align256(static_cast<size_t>(units) * sizeof(int)) : 0;
-  plan->ml_bytes = S > 1 ? align256(static_cast<size_t>(B) * Hq * S * 2 * sizeof(float)) : 0;
-  plan->workspace = S > 1 ? plan->counters_bytes + plan->ml_bytes +
-                                static_cast<size_t>(B) * Hq * S * D * sizeof(float)
-                          : 0;
+  const int64_t NG = (S + 7) / 8;
+  plan->num_groups = static_cast<int>(NG);
+  const size_t rows = static_cast<size_t>(B) * Hq;
+  plan->counters_bytes = S > 1 ? align256(static_cast<size_t>(units) * (1 + NG) * sizeof(int)) : 0;
+  plan->ml_bytes = S > 1 ? align256(rows * S * 2 * sizeof(float)) : 0;
+  plan->o_bytes = S > 1 ? align256(rows * S * D * sizeof(float)) : 0;
+  plan->grp_ml_bytes = NG > 1 ? align256(rows * NG * 2 * sizeof(float)) : 0;
+  plan->grp_o_bytes = NG > 1 ? align256(rows * NG * D * sizeof(float)) : 0;
+  plan->workspace = plan->counters_bytes + plan->ml_bytes + plan->o_bytes + plan->grp_ml_bytes +
+                    plan->grp_o_bytes;
   return FP8PD_OK;
 }
 
@@ -227,7 +224,7 @@ int validate_decode(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp
     if (sinks->shape[0] != Hq) return FP8PD_ERR_SHAPE;
   }
   const int64_t max_pages = block_table->shape[1];
-  if (!fits_i32(B) || B > 65535 || !fits_i32(P) || !fits_i32(max_pages) ||
+  if (!fits_i32(B) || B > 65535 || P > fp8pd::kMaxPages || !fits_i32(max_pages) ||
       max_pages * ps > INT32_MAX || Hkv * ((Hq / Hkv + 7) / 8) > 65535 || !fits_i32(Hq))
     return FP8PD_ERR_TOO_LARGE;
 
@@ -357,6 +354,7 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   p.num_splits = plan.num_splits;
   p.chunk_pages = plan.chunk_pages;
+  p.num_groups = plan.num_groups;
   p.head_groups = plan.head_groups;
   if (plan.combine) {
     void* ws = nullptr;
@@ -364,12 +362,19 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
     if (r) return r;
     uint8_t* base = static_cast<uint8_t*>(ws);
     p.counters = reinterpret_cast<int*>(base);
-    p.part_ml = reinterpret_cast<float*>(base + plan.counters_bytes);
-    p.part_o = reinterpret_cast<float*>(base + plan.counters_bytes + plan.ml_bytes);
+    base += plan.counters_bytes;
+    p.part_ml = reinterpret_cast<float*>(base);
+    base += plan.ml_bytes;
+    p.part_o = reinterpret_cast<float*>(base);
+    base += plan.o_bytes;
+    p.grp_ml = reinterpret_cast<float*>(base);
+    base += plan.grp_ml_bytes;
+    p.grp_o = reinterpret_cast<float*>(base);
   }
   EventPair* ev = timing_slot(0);
   if (ev) cudaEventRecord(ev->a, s);
-  cudaError_t e = fp8pd::launch_decode_mma(p, a.D, g_opt_k_decode.load() == 1, s);
+  cudaError_t e =
+      fp8pd::launch_decode_mma(p, a.D, g_opt_k_decode.load() == 1, g_opt_v_decode.load() == 1, s);
   if (e != cudaSuccess) return fail_cuda(e);
   ++g_launches;
   if (ev) cudaEventRecord(ev->b, s);
@@ -509,6 +514,10 @@ int fp8pd_set_option(int32_t option, int64_t value) {
       if (value < 0 || value > 1) return FP8PD_ERR_ARG;
       g_opt_k_decode = value;
       return FP8PD_OK;
+    case FP8PD_OPT_V_DECODE:
+      if (value < 0 || value > 1) return FP8PD_ERR_ARG;
+      g_opt_v_decode = value;
+      return FP8PD_OK;
     default:
       return FP8PD_ERR_ARG;
   }
@@ -519,6 +528,7 @@ int64_t fp8pd_get_option(int32_t option) {
     case FP8PD_OPT_NUM_SPLITS: return g_opt_num_splits.load();
     case FP8PD_OPT_VARIANT: return g_opt_variant.load();
     case FP8PD_OPT_K_DECODE: return g_opt_k_decode.load();
+    case FP8PD_OPT_V_DECODE: return g_opt_v_decode.load();
     default: return -1;
   }
 }

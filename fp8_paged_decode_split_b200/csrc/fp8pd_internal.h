@@ -29,9 +29,12 @@ struct DecodeParams {
   int64_t o_sb, o_sh;
   float* part_o;              // [B * Hq * S, D] split numerators (S > 1)
   float* part_ml;             // [B * Hq * S, 2] split (max, sum) in log2 units
-  int* counters;              // [B * Hkv * head_groups] tickets, zero between calls
+  int* counters;              // [B * Hkv * head_groups][1 + num_groups] tickets, zero between calls
+  float* grp_o;               // [B * Hq * num_groups, D] merged groups of splits
+  float* grp_ml;              // [B * Hq * num_groups, 2]
   int B, Hq, Hkv, G, D, ps, num_pages, max_pages, window, num_splits, head_groups;
   int chunk_pages;            // pages per split (the last split of a sequence may have fewer)
+  int num_groups;             // ceil(num_splits / 8): groups of the two-level split merge
   float sm_scale_log2;        // sm_scale * log2(e)
 };
 
@@ -53,7 +56,7 @@ struct AppendParams {
 };
 
 // Launchers (defined with the kernels). Return a cudaError_t of the launch.
-cudaError_t launch_decode_mma(const DecodeParams& p, int D, bool k_cvt, cudaStream_t s);
+cudaError_t launch_decode_mma(const DecodeParams& p, int D, bool k_cvt, bool v_cvt, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 
 // Thread blocks of the tensor-core split kernel one SM holds for head dim D.
@@ -69,5 +72,6 @@ constexpr int kTileTokens = 16;     // tokens per MMA row tile
 constexpr int kMaxWarpTiles = 256;  // 16-token tiles one warp takes in a split (ids in smem)
 constexpr int kMaxSplitTokens = kMaxWarpTiles * 4 * kTileTokens;  // 16,384 keys per split
 constexpr int kMaxSplits = 256;     // splits per (sequence, KV head, head group)
+constexpr int kMaxPages = (1 << 27) - 1;  // pool pages (tile lists pack page << 4)
 
 }  // namespace fp8pd

@@ -205,6 +205,20 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src) : "memory");
 }
 
+// Transposes an 8x8 matrix of 16-bit elements held one row pair per lane
+// (lane = 4 * row + col / 2), the layout of an MMA accumulator fragment.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
+  return d;
+}
+
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+constexpr int kMergeFan = 8;  // splits merged per group in the two-level merge
+
 template <int D>
 struct Cfg {
   static constexpr int NW = 4;                                        // warps per block
@@ -215,21 +229,75 @@ struct Cfg {
   static constexpr int PIPE_BYTES = (NW * WARP_BYTES + 127) / 128 * 128;
   static constexpr bool Q_IN_SMEM = (D > 256);                        // q fragments in smem
   static constexpr int QFRAG_BYTES = Q_IN_SMEM ? (D / 16) * 32 * 8 : 0;
-  static constexpr int PROW = 24;                                     // halves per P row
-  static constexpr int PBUF_BYTES = NW * 2 * 8 * PROW * 2;
-  static constexpr int PID_BYTES = NW * kMaxWarpTiles * 4;            // each warp's page ids
+  static constexpr int LIST_BYTES = NW * kMaxWarpTiles * 4;           // each warp's tile list
   static constexpr int MISC_FLOATS = NW * 8 * 2 + 4;
-  static constexpr int SMEM =
-      PIPE_BYTES + QFRAG_BYTES + PBUF_BYTES + PID_BYTES + MISC_FLOATS * 4;
+  static constexpr int SMEM = PIPE_BYTES + QFRAG_BYTES + LIST_BYTES + MISC_FLOATS * 4;
   static constexpr int MIN_BLOCKS = (D == 512) ? 1 : (D == 256) ? 2 : 4;
   static_assert(NW * 8 * D * 4 <= PIPE_BYTES, "merge scratch must fit in the ring");
-  static_assert(8 * kMaxSplits * 4 <= PIPE_BYTES, "combine weights must fit in the ring");
+  static_assert(8 * 32 * 4 <= PIPE_BYTES, "merge weights must fit in the ring");
 };
 
-// One thread block: (split, KV head x head group, sequence). KCVT selects the
-// K decode: false = bit assembly (byte pairs (0,2)/(1,3)), true = hardware
-// cvt (byte pairs (0,1)/(2,3)); the q fragments follow the same pairing.
-template <int D, bool KCVT>
+// Merges K partial rows (max m, sum l, numerator O, all in log2 units) of one
+// (sequence, head group): for head n they are rows row0(n) + s, s < K, of
+// (ml, o). With `final`, the sink enters the denominator once and the result
+// (numerator / denominator) goes to `out`; otherwise the merged (m, l, O) goes
+// to row dst_row(n) of (dst_ml, dst_o). Called by one whole block.
+template <int D, int NW>
+__device__ void merge_partials(const float* ml, const float* o, int64_t row0, int64_t head_rows,
+                               int K, int nheads, bool final, const DecodeParams& p, int b,
+                               int head0, float* dst_ml, float* dst_o, int64_t dst_row0,
+                               int64_t dst_head_rows, float* wts) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int n = warp; n < nheads; n += NW) {
+    const int head = head0 + n;
+    const float* pml = ml + (row0 + n * head_rows) * 2;
+    const float2 me = lane < K ? ldcg2(pml + 2 * lane) : make_float2(-CUDART_INF_F, 0.f);
+    const float M = warp_max(me.x);
+    const float sl = (final && p.sinks) ? p.sinks[(int64_t)head * p.sinks_s] * kLog2e : -CUDART_INF_F;
+    const float M2 = fmaxf(M, sl);
+    const float w = (M2 == -CUDART_INF_F || me.x == -CUDART_INF_F) ? 0.f : fast_exp2(me.x - M2);
+    float l = w * me.y;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    if (final) {
+      const float den = l + ((p.sinks && M2 != -CUDART_INF_F) ? fast_exp2(sl - M2) : 0.f);
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      if (lane < K) wts[n * 32 + lane] = w * inv;
+    } else {
+      if (lane < K) wts[n * 32 + lane] = w;
+      if (lane == 0)
+        *reinterpret_cast<float2*>(dst_ml + (dst_row0 + n * dst_head_rows) * 2) = make_float2(M, l);
+    }
+  }
+  __syncthreads();
+  for (int it = tid; it < nheads * (D / 4); it += NW * 32) {
+    const int n = it / (D / 4);
+    const int d = (it - n * (D / 4)) * 4;
+    const float* po = o + (row0 + n * head_rows) * D + d;
+    const float* wn = wts + n * 32;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int s = 0; s < K; ++s) {
+      const float ws = wn[s];
+      const float4 v = ldcg4(po + (int64_t)s * D);
+      acc.x += ws * v.x;
+      acc.y += ws * v.y;
+      acc.z += ws * v.z;
+      acc.w += ws * v.w;
+    }
+    if (final)
+      *reinterpret_cast<float4*>(p.out + (int64_t)b * p.o_sb + (int64_t)(head0 + n) * p.o_sh + d) = acc;
+    else
+      *reinterpret_cast<float4*>(dst_o + (dst_row0 + n * dst_head_rows) * D + d) = acc;
+  }
+}
+
+// One thread block: (split, KV head x head group, sequence). KCVT / VCVT
+// select the E4M3 -> f16 decode of K / V: false = bit assembly (value * 2^-8),
+// true = hardware cvt.rn.f16x2.e4m3x2 (the value itself). The q fragments
+// follow the K byte pairing.
+template <int D, bool KCVT, bool VCVT>
 __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     decode_mma_kernel(const DecodeParams p) {
   using C = Cfg<D>;
@@ -237,9 +305,8 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* pipe = smem;
   uint2* qfrag_s = reinterpret_cast<uint2*>(smem + C::PIPE_BYTES);
-  __half* pbuf = reinterpret_cast<__half*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES);
-  int32_t* s_pid = reinterpret_cast<int32_t*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES + C::PBUF_BYTES);
-  float* misc = reinterpret_cast<float*>(s_pid + C::NW * kMaxWarpTiles);
+  int32_t* s_list = reinterpret_cast<int32_t*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES);
+  float* misc = reinterpret_cast<float*>(s_list + C::NW * kMaxWarpTiles);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, grp = lane >> 2, qd = lane & 3;
@@ -274,16 +341,23 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   }
   const int32_t* trow = p.table + (int64_t)b * p.tab_sb;
 
-  // ---- warp-local setup: this warp's page ids, q fragments ------------------
-  int32_t* wpid = s_pid + warp * kMaxWarpTiles;
+  // ---- warp-local setup: this warp's tile list, q fragments -----------------
+  // Tile j of warp w starts at token 16 * (tile_first + w + 4j); its list
+  // entry packs the physical page and the tile's index inside the page as
+  // (page << 4) | index, or -1 when the block-table entry is out of range.
+  int32_t* wlist = s_list + warp * kMaxWarpTiles;
+#pragma unroll 4
   for (int j = lane; j < my_tiles; j += 32) {
-    const int lp = (tile_first + warp + C::NW * j) * kTileTokens / p.ps;
-    int page = __ldg(trow + (int64_t)lp * p.tab_sp);
-    if ((unsigned)page >= (unsigned)p.num_pages) {
-      if (hg == 0) raise_flag(FP8PD_FLAG_PAGE_OOB);
-      page = -1;
+    const int tok = (tile_first + warp + C::NW * j) * kTileTokens;
+    const int lp = tok / p.ps;
+    const int page = __ldg(trow + (int64_t)lp * p.tab_sp);
+    int e = -1;
+    if ((unsigned)page < (unsigned)p.num_pages) {
+      e = (page << 4) | ((tok - lp * p.ps) / kTileTokens);
+    } else if (hg == 0) {
+      raise_flag(FP8PD_FLAG_PAGE_OOB);
     }
-    wpid[j] = page;
+    wlist[j] = e;
   }
   // Lane (g, q) holds query head g of the group at head-dim entries
   // 64jj + 16q + {0..15}; the k16 block (jj, i) covers entries
@@ -294,7 +368,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   const uint16_t* qrow = p.q + (int64_t)b * p.q_sb + (int64_t)(head0 + (q_head_ok ? grp : 0)) * p.q_sh;
   float qmax = 0.f;
   if (q_head_ok) {
-#pragma unroll 4
+#pragma unroll 8
     for (int e = 0; e < D / 4; ++e) {
       const int d = 64 * (e >> 4) + 16 * qd + (e & 15);
       qmax = fmaxf(qmax, fabsf(bf16_bits_to_float(__ldg(qrow + (int64_t)d * p.q_sd))));
@@ -341,22 +415,21 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
 
   // ---- per-warp pipeline over 16-token tiles --------------------------------
   const uint32_t wpipe = smem_u32(pipe + warp * C::WARP_BYTES);
-  __half* p_hi = pbuf + warp * (2 * 8 * C::PROW);
-  __half* p_lo = p_hi + 8 * C::PROW;
   const uint8_t* kbase = p.k + (int64_t)kvh * p.k_sh;
   const uint8_t* vbase = p.v + (int64_t)kvh * p.v_sh;
   const float* ksbase = p.ks + (int64_t)kvh * p.ks_sh;
   const float* vsbase = p.vs + (int64_t)kvh * p.vs_sh;
+  const int64_t k_tile_st = (int64_t)kTileTokens * p.k_st;
+  const int64_t v_tile_st = (int64_t)kTileTokens * p.v_st;
 
   // Copies tile j of this warp into ring stage `stage`: K and V rows (16-byte
   // cp.async per lane), then the page's k and v scales (4 bytes each).
   auto issue = [&](int j, int stage) {
-    const int page = wpid[j];
-    if (page < 0) return;
-    const int tok0 = (tile_first + warp + C::NW * j) * kTileTokens;
-    const int slot0 = tok0 - (tok0 / p.ps) * p.ps;
-    const uint8_t* gk = kbase + (int64_t)page * p.k_sp + (int64_t)slot0 * p.k_st;
-    const uint8_t* gv = vbase + (int64_t)page * p.v_sp + (int64_t)slot0 * p.v_st;
+    const int e = wlist[j];
+    if (e < 0) return;
+    const int page = e >> 4, tip = e & 15;
+    const uint8_t* gk = kbase + (int64_t)page * p.k_sp + tip * k_tile_st;
+    const uint8_t* gv = vbase + (int64_t)page * p.v_sp + tip * v_tile_st;
     const uint32_t sk = wpipe + stage * C::STAGE;
     const uint32_t sv = sk + C::TILE;
     constexpr int CPR = D / 16;
@@ -382,7 +455,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   float l0 = 0.f, l1 = 0.f;                      // this lane's share of the running sums
   // Running V reference scale: the largest |v_scale| seen so far. O holds
   // sum P * v_scale / vref, so every f16 P operand stays <= 1 in magnitude.
-  float vref = 0.f;
+  float vref = 0.f, inv_vref = 0.f;
 
 #pragma unroll 1
   for (int s = 0; s < C::NS - 1; ++s) {
@@ -400,7 +473,8 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       cp_async_commit();
     }
     const int tok0 = (tile_first + warp + C::NW * j) * kTileTokens;
-    const bool page_ok = wpid[j] >= 0;
+    const bool page_ok = wlist[j] >= 0;
+    const bool full = page_ok && tok0 >= t0 && tok0 + kTileTokens <= t1;  // warp-uniform
     const uint32_t sk = wpipe + (j % C::NS) * C::STAGE;
     const uint32_t sv = sk + C::TILE;
     float kfac = 0.f, vs = 0.f;
@@ -448,10 +522,10 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     }
 
     // -- masked scores (log2 units), online softmax ------------------------
+    // A masked row may hold stale or NaN-decoded bytes: select, never multiply.
     const int ta = tok0 + grp, tb = ta + 8;
-    const bool va = page_ok && ta >= t0 && ta < t1;
-    const bool vb = page_ok && tb >= t0 && tb < t1;
-    // a masked row may hold stale or NaN-decoded bytes: select, never multiply
+    const bool va = full || (page_ok && ta >= t0 && ta < t1);
+    const bool vb = full || (page_ok && tb >= t0 && tb < t1);
     const float s00 = va ? (Sa[0] + Sb[0]) * kfac : -CUDART_INF_F;  // token grp,   head 2qd
     const float s01 = va ? (Sa[1] + Sb[1]) * kfac : -CUDART_INF_F;  // token grp,   head 2qd+1
     const float s10 = vb ? (Sa[2] + Sb[2]) * kfac : -CUDART_INF_F;  // token grp+8, head 2qd
@@ -483,7 +557,10 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
         }
       m0 = mn0;
       m1 = mn1;
-      if (grow_v) vref = vabs;
+      if (grow_v) {
+        vref = vabs;
+        inv_vref = 1.f / vabs;
+      }
     }
     const float mb0 = (m0 == -CUDART_INF_F) ? 0.f : m0;
     const float mb1 = (m1 == -CUDART_INF_F) ? 0.f : m1;
@@ -492,48 +569,69 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     l0 += p00 + p10;
     l1 += p01 + p11;
 
-    // -- P * v_scale / vref as f16 hi + lo, transposed through shared memory
-    {
-      const float vsr = (vref > 0.f) ? vs / vref : 0.f;
-      const float w00 = p00 * vsr, w01 = p01 * vsr, w10 = p10 * vsr, w11 = p11 * vsr;
-      const __half h00 = __float2half_rn(w00), h01 = __float2half_rn(w01);
-      const __half h10 = __float2half_rn(w10), h11 = __float2half_rn(w11);
-      const int r0 = (2 * qd) * C::PROW, r1 = r0 + C::PROW;
-      p_hi[r0 + grp] = h00;
-      p_hi[r0 + grp + 8] = h10;
-      p_hi[r1 + grp] = h01;
-      p_hi[r1 + grp + 8] = h11;
-      p_lo[r0 + grp] = __float2half_rn(w00 - __half2float(h00));
-      p_lo[r0 + grp + 8] = __float2half_rn(w10 - __half2float(h10));
-      p_lo[r1 + grp] = __float2half_rn(w01 - __half2float(h01));
-      p_lo[r1 + grp + 8] = __float2half_rn(w11 - __half2float(h11));
-    }
-    __syncwarp();
-    const uint32_t* phw = reinterpret_cast<const uint32_t*>(p_hi + grp * C::PROW);
-    const uint32_t* plw = reinterpret_cast<const uint32_t*>(p_lo + grp * C::PROW);
-    const uint32_t bh0 = phw[qd], bh1 = phw[qd + 4];  // tokens (2qd, 2qd+1), (2qd+8, 2qd+9)
-    const uint32_t bl0 = plw[qd], bl1 = plw[qd + 4];
+    // -- P * v_scale / vref as f16 hi + lo; the B fragments of the PV MMA are
+    // the transposes of the score fragment's 8x8 blocks (movmatrix).
+    const float vsr = vs * inv_vref;
+    const float w00 = p00 * vsr, w01 = p01 * vsr, w10 = p10 * vsr, w11 = p11 * vsr;
+    const uint32_t ha = pack_f16x2(w00, w01), hb = pack_f16x2(w10, w11);
+    const float2 fa = unpack_f16x2(ha), fb = unpack_f16x2(hb);
+    const uint32_t la = pack_f16x2(w00 - fa.x, w01 - fa.y), lb = pack_f16x2(w10 - fb.x, w11 - fb.y);
+    const uint32_t bh0 = movmatrix_trans(ha), bh1 = movmatrix_trans(hb);  // tokens 2qd.., 2qd+8..
+    const uint32_t bl0 = movmatrix_trans(la), bl1 = movmatrix_trans(lb);
 
     // -- O^T[d][head] += V^T P ---------------------------------------------
     // Block jb covers d in [32jb, 32jb+32). Lane (g, q) reads bytes 4g..4g+3
     // of the block from tokens 2q, 2q+1, 2q+8, 2q+9; M tile (jb, h) row g is
-    // d = 32jb + 4g + 2h, row g+8 is d + 1.
+    // d = 32jb + 4g + 2h, row g+8 is d + 1. With the hardware cvt a masked
+    // row is zeroed first (a NaN byte times P = 0 would still be NaN).
+    uint32_t vm0 = ~0u, vm1 = ~0u, vm2 = ~0u, vm3 = ~0u;
+    if (VCVT && !full) {
+      const int r = tok0 + 2 * qd;
+      vm0 = (page_ok && r >= t0 && r < t1) ? ~0u : 0u;
+      vm1 = (page_ok && r + 1 >= t0 && r + 1 < t1) ? ~0u : 0u;
+      vm2 = (page_ok && r + 8 >= t0 && r + 8 < t1) ? ~0u : 0u;
+      vm3 = (page_ok && r + 9 >= t0 && r + 9 < t1) ? ~0u : 0u;
+    }
 #pragma unroll
     for (int jb = 0; jb < D / 32; ++jb) {
       const int c = 2 * jb + (grp >> 2);
       const uint32_t cb = (grp & 3) * 4;
-      const uint32_t w0 = lds32(sv + v_off<D>(2 * qd, c) + cb);
-      const uint32_t w1 = lds32(sv + v_off<D>(2 * qd + 1, c) + cb);
-      const uint32_t w2 = lds32(sv + v_off<D>(2 * qd + 8, c) + cb);
-      const uint32_t w3 = lds32(sv + v_off<D>(2 * qd + 9, c) + cb);
-      const uint32_t za = prmt(w0, w1, 0x5410), zb = prmt(w0, w1, 0x7632);
-      const uint32_t zc = prmt(w2, w3, 0x5410), zd = prmt(w2, w3, 0x7632);
-      const uint32_t a0 = e4m3x2_b02_to_f16x2(za), a1 = e4m3x2_b13_to_f16x2(za);
-      const uint32_t a2 = e4m3x2_b02_to_f16x2(zc), a3 = e4m3x2_b13_to_f16x2(zc);
+      uint32_t w0 = lds32(sv + v_off<D>(2 * qd, c) + cb);
+      uint32_t w1 = lds32(sv + v_off<D>(2 * qd + 1, c) + cb);
+      uint32_t w2 = lds32(sv + v_off<D>(2 * qd + 8, c) + cb);
+      uint32_t w3 = lds32(sv + v_off<D>(2 * qd + 9, c) + cb);
+      uint32_t a0, a1, a2, a3, e0, e1, e2, e3;
+      if constexpr (VCVT) {
+        w0 &= vm0;
+        w1 &= vm1;
+        w2 &= vm2;
+        w3 &= vm3;
+        // [w0.c, w1.c, w0.c+1, w1.c+1]: each 16-bit half is one column's token pair
+        const uint32_t za = prmt(w0, w1, 0x5140), zb = prmt(w0, w1, 0x7362);
+        const uint32_t zc = prmt(w2, w3, 0x5140), zd = prmt(w2, w3, 0x7362);
+        a0 = e4m3x2_lo16_to_f16x2(za);
+        a1 = e4m3x2_hi16_to_f16x2(za);
+        a2 = e4m3x2_lo16_to_f16x2(zc);
+        a3 = e4m3x2_hi16_to_f16x2(zc);
+        e0 = e4m3x2_lo16_to_f16x2(zb);
+        e1 = e4m3x2_hi16_to_f16x2(zb);
+        e2 = e4m3x2_lo16_to_f16x2(zd);
+        e3 = e4m3x2_hi16_to_f16x2(zd);
+      } else {
+        // [w0.c, w0.c+1, w1.c, w1.c+1]: bytes (0,2) and (1,3) are token pairs
+        const uint32_t za = prmt(w0, w1, 0x5410), zb = prmt(w0, w1, 0x7632);
+        const uint32_t zc = prmt(w2, w3, 0x5410), zd = prmt(w2, w3, 0x7632);
+        a0 = e4m3x2_b02_to_f16x2(za);
+        a1 = e4m3x2_b13_to_f16x2(za);
+        a2 = e4m3x2_b02_to_f16x2(zc);
+        a3 = e4m3x2_b13_to_f16x2(zc);
+        e0 = e4m3x2_b02_to_f16x2(zb);
+        e1 = e4m3x2_b13_to_f16x2(zb);
+        e2 = e4m3x2_b02_to_f16x2(zd);
+        e3 = e4m3x2_b13_to_f16x2(zd);
+      }
       mma16816(O[jb][0], a0, a1, a2, a3, bh0, bh1);
       mma16816(O[jb][0], a0, a1, a2, a3, bl0, bl1);
-      const uint32_t e0 = e4m3x2_b02_to_f16x2(zb), e1 = e4m3x2_b13_to_f16x2(zb);
-      const uint32_t e2 = e4m3x2_b02_to_f16x2(zd), e3 = e4m3x2_b13_to_f16x2(zd);
       mma16816(O[jb][1], e0, e1, e2, e3, bh0, bh1);
       mma16816(O[jb][1], e0, e1, e2, e3, bl0, bl1);
     }
@@ -547,9 +645,10 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     l1 += __shfl_xor_sync(0xffffffffu, l1, o);
   }
   __syncthreads();  // every warp is done with its ring
-  float* Os = reinterpret_cast<float*>(pipe);  // [NW][8][D], already times 2^8 * vref
+  float* Os = reinterpret_cast<float*>(pipe);  // [NW][8][D], already times fold
   float* ml = misc;                            // [NW][8][2]
-  const float fold = 256.f * vref;             // f16 offset of the decoded V, V reference scale
+  // f16 offset of the decoded V (bit assembly only), times the V reference scale
+  const float fold = (VCVT ? 1.f : 256.f) * vref;
 #pragma unroll
   for (int jb = 0; jb < D / 32; ++jb) {
     const int d = 32 * jb + 4 * grp;
@@ -612,69 +711,45 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   }
   if (S == 1) return;
 
-  // ---- the last block of this (sequence, KV head, head group) combines ------
-  // Every block publishes its partials, then takes a ticket; the block that
-  // draws the last ticket merges all S partials (log-sum-exp, sink added once)
-  // and resets the counter for the next call. No block ever waits for another.
+  // ---- two-level merge by the last blocks to finish --------------------------
+  // Splits form groups of kMergeFan. Every block publishes its partial, then
+  // takes a ticket of its group; the block drawing the group's last ticket
+  // merges the group (or, with a single group, produces the output). With
+  // several groups, each group merger then takes a ticket of the (sequence,
+  // KV head, head group) and the last one merges the group partials, adding
+  // the sink once. Mergers reset their counters; no block ever waits.
   __threadfence();
   __syncthreads();
-  int* last_flag = reinterpret_cast<int*>(misc + C::NW * 8 * 2);
+  int* flag = reinterpret_cast<int*>(misc + C::NW * 8 * 2);
+  const int NG = p.num_groups;
   const int64_t unit = (int64_t)b * gridDim.y + blockIdx.y;
-  if (tid == 0) {
-    const int prev = atomicAdd(p.counters + unit, 1);
-    *last_flag = (prev == S - 1);
-  }
+  int* ucnt = p.counters + unit * (1 + NG);
+  const int g = split / kMergeFan;
+  const int gsize = min(kMergeFan, S - g * kMergeFan);
+  if (tid == 0) *flag = (atomicAdd(ucnt + 1 + g, 1) == gsize - 1);
   __syncthreads();
-  if (!*last_flag) return;
+  if (!*flag) return;
   __threadfence();
-
-  float* wts = reinterpret_cast<float*>(pipe);  // [8][kMaxSplits] split weight / den
-  for (int n = warp; n < nheads; n += C::NW) {
-    const int head = head0 + n;
-    const float* pml = p.part_ml + ((int64_t)b * p.Hq + head) * S * 2;
-    float M = -CUDART_INF_F;
-    for (int s = lane; s < S; s += 32) M = fmaxf(M, ldcg2(pml + 2 * s).x);
-    M = warp_max(M);
-    const float sl = p.sinks ? p.sinks[(int64_t)head * p.sinks_s] * kLog2e : -CUDART_INF_F;
-    const float M2 = fmaxf(M, sl);
-    float den = 0.f;
-    if (M2 != -CUDART_INF_F) {
-      for (int s = lane; s < S; s += 32) {
-        const float2 ml2 = ldcg2(pml + 2 * s);
-        if (ml2.x != -CUDART_INF_F) den += ml2.y * fast_exp2(ml2.x - M2);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-      if (p.sinks) den += fast_exp2(sl - M2);
-    }
-    const float inv = (M2 != -CUDART_INF_F && den > 0.f) ? 1.f / den : 0.f;
-    for (int s = lane; s < S; s += 32) {
-      const float ms = ldcg2(pml + 2 * s).x;
-      wts[n * kMaxSplits + s] = (inv == 0.f || ms == -CUDART_INF_F) ? 0.f : fast_exp2(ms - M2) * inv;
-    }
+  float* wts = reinterpret_cast<float*>(pipe);  // [8][32] merge weights
+  const int64_t row_b = (int64_t)b * p.Hq + head0;
+  if (NG == 1) {
+    merge_partials<D, C::NW>(p.part_ml, p.part_o, row_b * S, S, S, nheads, true, p, b, head0,
+                             nullptr, nullptr, 0, 0, wts);
+    if (tid == 0) ucnt[1] = 0;
+    return;
   }
+  merge_partials<D, C::NW>(p.part_ml, p.part_o, row_b * S + g * kMergeFan, S, gsize, nheads, false,
+                           p, b, head0, p.grp_ml, p.grp_o, row_b * NG + g, NG, wts);
+  if (tid == 0) ucnt[1 + g] = 0;
+  __threadfence();
   __syncthreads();
-  // Every split wrote its row (zeros for an empty one), so the weighted sum
-  // needs no branch and its loads can all be in flight at once.
-  for (int it = tid; it < nheads * (D / 4); it += 128) {
-    const int n = it / (D / 4);
-    const int d = (it - n * (D / 4)) * 4;
-    const int head = head0 + n;
-    const float* po = p.part_o + ((int64_t)b * p.Hq + head) * S * D + d;
-    const float* wn = wts + n * kMaxSplits;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-    for (int s = 0; s < S; ++s) {
-      const float w = wn[s];
-      const float4 o = ldcg4(po + (int64_t)s * D);
-      acc.x += w * o.x;
-      acc.y += w * o.y;
-      acc.z += w * o.z;
-      acc.w += w * o.w;
-    }
-    *reinterpret_cast<float4*>(p.out + (int64_t)b * p.o_sb + (int64_t)head * p.o_sh + d) = acc;
-  }
-  if (tid == 0) p.counters[unit] = 0;
+  if (tid == 0) *flag = (atomicAdd(ucnt, 1) == NG - 1);
+  __syncthreads();
+  if (!*flag) return;
+  __threadfence();
+  merge_partials<D, C::NW>(p.grp_ml, p.grp_o, row_b * NG, NG, NG, nheads, true, p, b, head0,
+                           nullptr, nullptr, 0, 0, wts);
+  if (tid == 0) ucnt[0] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -734,7 +809,7 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
 // ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
-template <int D, bool KCVT>
+template <int D, bool KCVT, bool VCVT>
 static cudaError_t launch_decode_mma_d(const DecodeParams& p, cudaStream_t s) {
   // The shared-memory opt-in is a per-device function attribute: set it once
   // per device (an idempotent call, so a race only repeats it).
@@ -745,22 +820,29 @@ static cudaError_t launch_decode_mma_d(const DecodeParams& p, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
   if (!bit || !(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(decode_mma_kernel<D, KCVT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem);
+    e = cudaFuncSetAttribute(decode_mma_kernel<D, KCVT, VCVT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
   const dim3 grid(p.num_splits, p.Hkv * p.head_groups, p.B);
-  decode_mma_kernel<D, KCVT><<<grid, 128, smem, s>>>(p);
+  decode_mma_kernel<D, KCVT, VCVT><<<grid, 128, smem, s>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode_mma(const DecodeParams& p, int D, bool k_cvt, cudaStream_t s) {
+template <int D>
+static cudaError_t launch_decode_mma_kv(const DecodeParams& p, bool k_cvt, bool v_cvt,
+                                       cudaStream_t s) {
+  if (k_cvt) return v_cvt ? launch_decode_mma_d<D, true, true>(p, s) : launch_decode_mma_d<D, true, false>(p, s);
+  return v_cvt ? launch_decode_mma_d<D, false, true>(p, s) : launch_decode_mma_d<D, false, false>(p, s);
+}
+
+cudaError_t launch_decode_mma(const DecodeParams& p, int D, bool k_cvt, bool v_cvt, cudaStream_t s) {
   switch (D) {
-    case 64: return k_cvt ? launch_decode_mma_d<64, true>(p, s) : launch_decode_mma_d<64, false>(p, s);
-    case 128: return k_cvt ? launch_decode_mma_d<128, true>(p, s) : launch_decode_mma_d<128, false>(p, s);
-    case 256: return k_cvt ? launch_decode_mma_d<256, true>(p, s) : launch_decode_mma_d<256, false>(p, s);
-    case 512: return k_cvt ? launch_decode_mma_d<512, true>(p, s) : launch_decode_mma_d<512, false>(p, s);
+    case 64: return launch_decode_mma_kv<64>(p, k_cvt, v_cvt, s);
+    case 128: return launch_decode_mma_kv<128>(p, k_cvt, v_cvt, s);
+    case 256: return launch_decode_mma_kv<256>(p, k_cvt, v_cvt, s);
+    case 512: return launch_decode_mma_kv<512>(p, k_cvt, v_cvt, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -781,9 +863,9 @@ static int blocks_per_sm_d() {
   int c = cached.load();
   if (c >= 0) return c;
   int n = 0;
-  if (cudaFuncSetAttribute(decode_mma_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Cfg<D>::SMEM) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_mma_kernel<D, false>, 128,
+  if (cudaFuncSetAttribute(decode_mma_kernel<D, true, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_mma_kernel<D, true, true>, 128,
                                                     Cfg<D>::SMEM) != cudaSuccess) {
     cudaGetLastError();
     return Cfg<D>::MIN_BLOCKS;  // no device: do not cache the guess

@@ -137,7 +137,8 @@ enum {
  *                (a page stride wider than one layer's page is allowed: several
  *                layers may share one pool -- the solution page's per-layer row
  *                strides; the 16-byte rule follows DeepGEMM PR #459's paged
- *                accessor). D in {64, 128, 256, 512}; ps a multiple of 16, <= 256.
+ *                accessor). D in {64, 128, 256, 512}; ps a multiple of 16, <= 256;
+ *                num_pages < 2^27.
  *   k_scale,     float32 [Hkv] or [num_pages, Hkv], any strides (0 = broadcast).
  *   v_scale
  *   block_table  int32 [B, max_pages]: physical page of each logical page.
@@ -218,8 +219,9 @@ enum {
                                 splits and at the number of pages) */
   FP8PD_OPT_VARIANT = 2,     /* 0 = auto; 1 = tensor-core (mma) split kernel;
                                 2 = CUDA-core (f32 FMA) split kernel */
-  FP8PD_OPT_K_DECODE = 3     /* E4M3 -> f16 decode of K: 0 = bit assembly,
+  FP8PD_OPT_K_DECODE = 3,    /* E4M3 -> f16 decode of K: 0 = bit assembly,
                                 1 = hardware cvt.rn.f16x2.e4m3x2 (default) */
+  FP8PD_OPT_V_DECODE = 4     /* the same for V (default 1) */
 };
 int fp8pd_set_option(int32_t option, int64_t value);
 int64_t fp8pd_get_option(int32_t option);

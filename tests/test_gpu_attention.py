@@ -25,12 +25,24 @@ def F(cuda_device):
     return F
 
 
-@pytest.fixture(params=[1, 0], ids=["kcvt", "kbits"])
+@pytest.fixture(params=[(1, 1), (0, 0)], ids=["cvt", "bits"])
 def kdecode(F, request):
-    """Run a test with each E4M3 -> f16 decode of K (hardware cvt, bit assembly)."""
-    F.fp8pd_set_option(F.OPT_K_DECODE, request.param)
+    """Run a test with each E4M3 -> f16 decode of K and V (hardware cvt, bit
+    assembly)."""
+    F.fp8pd_set_option(F.OPT_K_DECODE, request.param[0])
+    F.fp8pd_set_option(F.OPT_V_DECODE, request.param[1])
     yield request.param
     F.fp8pd_set_option(F.OPT_K_DECODE, 1)
+    F.fp8pd_set_option(F.OPT_V_DECODE, 1)
+
+
+@pytest.fixture(params=[(1, 0), (0, 1)], ids=["kcvt-vbits", "kbits-vcvt"])
+def mixed_decode(F, request):
+    F.fp8pd_set_option(F.OPT_K_DECODE, request.param[0])
+    F.fp8pd_set_option(F.OPT_V_DECODE, request.param[1])
+    yield request.param
+    F.fp8pd_set_option(F.OPT_K_DECODE, 1)
+    F.fp8pd_set_option(F.OPT_V_DECODE, 1)
 
 
 @pytest.fixture
@@ -99,6 +111,37 @@ def test_long_context_reduced_split(F, cuda_device, splits, nsplit):
     _check_layer(F, case, where=f"long splits={nsplit}")
     if nsplit == 40:
         assert F.fp8pd_last_run_info()["combine"] == 1
+
+
+def test_mixed_decodes(F, cuda_device, mixed_decode):
+    case = W.make_case("llama", cuda_device, B=3, seq_len=(40, 400))
+    _check_layer(F, case, where=f"decode {mixed_decode}")
+
+
+@pytest.mark.parametrize("window", [0, 37])
+def test_nan_codes_outside_the_attended_keys_are_ignored(F, cuda_device, kdecode, window):
+    """Slots past the last key, and keys before the window, hold E4M3 NaN
+    codes: they are never attended, so the output stays finite and equal to
+    the oracle's (which never reads them)."""
+    case = _small(cuda_device, sinks=True)
+    layer = case.layers[0]
+    lc = W.LayerCase(**{**layer.__dict__, "window": window})
+    ps = layer.k_pages.shape[1]
+    lens = case.attend_lens.cpu().numpy()
+    tbl = layer.block_table.cpu().numpy()
+    for b, L in enumerate(lens):
+        last = tbl[b, (L - 1) // ps]
+        s = L % ps
+        if s:
+            layer.k_pages[last, s:] = 0x7F
+            layer.v_pages[last, s:] = 0xFF
+        if window:
+            lo = max(0, L - window)
+            first = tbl[b, lo // ps]
+            if lo % ps:
+                layer.k_pages[first, : lo % ps] = 0xFF
+                layer.v_pages[first, : lo % ps] = 0x7F
+    _check_layer(F, W.Case(**{**case.__dict__, "layers": [lc]}), where=f"nan codes w={window}")
 
 
 # --------------------------------------------------------------- shapes
