@@ -2,7 +2,9 @@
 // (nothing is launched unless every check passes), split planning, the
 // per-device split workspace, options, run info and optional kernel timing.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <atomic>
@@ -132,7 +134,7 @@ int current_device(int* dev) {
 // [s * chunk, (s+1) * chunk) of a sequence's attended range, so every block
 // has the same amount of work whatever the sequence lengths (blocks past the
 // end of a short sequence finish at once). The count fills whole waves of the
-// device with >= 512 keys per split, never more than 16,384 keys per split
+// device with >= 512 keys per split, never more than 8,192 keys per split
 // (the kernel's per-warp tile list) nor more than kMaxSplits splits.
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
@@ -145,7 +147,7 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
   pages = std::max<int64_t>(pages, 1);
   const int64_t max_chunk = std::max<int64_t>(1, fp8pd::kMaxSplitTokens / ps);
   const int64_t s_min = (pages + max_chunk - 1) / max_chunk;
-  if (s_min > fp8pd::kMaxSplits) return FP8PD_ERR_TOO_LARGE;  // > 4 Mi keys in one sequence
+  if (s_min > fp8pd::kMaxSplits) return FP8PD_ERR_TOO_LARGE;  // > 2 Mi keys in one sequence
   const int64_t min_chunk = std::max(1, 512 / ps);
   const int64_t s_max = std::min<int64_t>(
       fp8pd::kMaxSplits, std::max<int64_t>(s_min, (pages + min_chunk - 1) / min_chunk));
@@ -162,7 +164,7 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
       if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) sms = v;
     }
     cudaGetLastError();
-    const int64_t slots = static_cast<int64_t>(sms) * fp8pd::decode_mma_blocks_per_sm(D);
+    const int64_t slots = static_cast<int64_t>(sms) * fp8pd::decode_blocks_per_sm(D);
     S = std::min<int64_t>(s_max, (5 * slots + 4 * units - 1) / (4 * units));
     S = std::max<int64_t>(S, 1);
   }
@@ -183,6 +185,87 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
   plan->grp_o_bytes = NG > 1 ? align256(rows * NG * D * sizeof(float)) : 0;
   plan->workspace = plan->counters_bytes + plan->ml_bytes + plan->o_bytes + plan->grp_ml_bytes +
                     plan->grp_o_bytes;
+  return FP8PD_OK;
+}
+
+// ---- TMA tensor maps over pool views ---------------------------------------
+// A pool view [num_pages, ps, Hkv, D] (byte strides sp, st, sh, 1) is described
+// to the TMA as 5 dims, innermost first: head-dim bytes within a 128-byte
+// block (min(D, 128)), slot (stride st), 128-byte block (stride 128, D / 128
+// of them), KV head (stride sh), page (stride sp). One box = one 16-token tile
+// of one KV head, laid out in shared memory as [block][slot][bytes] with the
+// 128-byte swizzle (64-byte for D = 64).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+struct MapKey {
+  const void* base;
+  int64_t shape[4];
+  int64_t stride[4];
+  bool operator==(const MapKey& o) const {
+    return base == o.base && std::memcmp(shape, o.shape, sizeof(shape)) == 0 &&
+           std::memcmp(stride, o.stride, sizeof(stride)) == 0;
+  }
+};
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+};
+std::mutex g_map_mutex;
+std::vector<MapEntry> g_maps;  // small most-recently-used cache
+
+int make_pool_map(const fp8pd_tensor* pool, CUtensorMap* out) {
+  MapKey key{pool->data, {}, {}};
+  for (int i = 0; i < 4; ++i) {
+    key.shape[i] = pool->shape[i];
+    key.stride[i] = pool->stride[i];
+  }
+  {
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    for (size_t i = 0; i < g_maps.size(); ++i)
+      if (g_maps[i].key == key) {
+        *out = g_maps[i].map;
+        if (i) std::swap(g_maps[i], g_maps[0]);
+        return FP8PD_OK;
+      }
+  }
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (!enc) return fail_cuda(cudaErrorNotSupported);
+  const int64_t P = pool->shape[0], ps = pool->shape[1], Hkv = pool->shape[2], D = pool->shape[3];
+  const cuuint64_t x = D < 128 ? D : 128;
+  const cuuint64_t nblk = D < 128 ? 1 : D / 128;
+  const cuuint64_t dims[5] = {x, static_cast<cuuint64_t>(ps), nblk, static_cast<cuuint64_t>(Hkv),
+                              static_cast<cuuint64_t>(P)};
+  const cuuint64_t strides[4] = {static_cast<cuuint64_t>(pool->stride[1]), 128,
+                                 static_cast<cuuint64_t>(pool->stride[2]),
+                                 static_cast<cuuint64_t>(pool->stride[0])};
+  const cuuint32_t box[5] = {static_cast<cuuint32_t>(x), static_cast<cuuint32_t>(fp8pd::kTileTokens),
+                             static_cast<cuuint32_t>(nblk), 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUtensorMap map;
+  const CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, pool->data, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         D == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail_cuda(cudaErrorInvalidValue);
+  {
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    g_maps.insert(g_maps.begin(), MapEntry{key, map});
+    if (g_maps.size() > 32) g_maps.pop_back();
+  }
+  *out = map;
   return FP8PD_OK;
 }
 
@@ -371,10 +454,13 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
     base += plan.grp_ml_bytes;
     p.grp_o = reinterpret_cast<float*>(base);
   }
+  CUtensorMap tmk, tmv;
+  if ((r = make_pool_map(k_pages, &tmk))) return r;
+  if ((r = make_pool_map(v_pages, &tmv))) return r;
   EventPair* ev = timing_slot(0);
   if (ev) cudaEventRecord(ev->a, s);
-  cudaError_t e =
-      fp8pd::launch_decode_mma(p, a.D, g_opt_k_decode.load() == 1, g_opt_v_decode.load() == 1, s);
+  cudaError_t e = fp8pd::launch_decode(p, tmk, tmv, g_opt_k_decode.load() == 1,
+                                       g_opt_v_decode.load() == 1, s);
   if (e != cudaSuccess) return fail_cuda(e);
   ++g_launches;
   if (ev) cudaEventRecord(ev->b, s);

@@ -2,6 +2,7 @@
 // paged decode attention library (not part of the public ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -56,21 +57,23 @@ struct AppendParams {
 };
 
 // Launchers (defined with the kernels). Return a cudaError_t of the launch.
-cudaError_t launch_decode_mma(const DecodeParams& p, int D, bool k_cvt, bool v_cvt, cudaStream_t s);
+// tmk / tmv: tensor maps over the K / V pool views (see make_pool_map).
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                          bool k_cvt, bool v_cvt, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 
-// Thread blocks of the tensor-core split kernel one SM holds for head dim D.
-int decode_mma_blocks_per_sm(int D);
-// Dynamic shared memory of the tensor-core split kernel for head dim D.
-int decode_mma_smem_bytes(int D);
+// Thread blocks of the split kernel one SM holds for head dim D.
+int decode_blocks_per_sm(int D);
+// Dynamic shared memory of the split kernel for head dim D.
+int decode_smem_bytes(int D);
 
 // Device error word (one per device): read and cleared by the host API.
 cudaError_t read_and_clear_error_word(uint32_t* value, cudaStream_t s);
 
 constexpr int kHeadsPerGroup = 8;   // query heads one thread block serves (MMA N)
 constexpr int kTileTokens = 16;     // tokens per MMA row tile
-constexpr int kMaxWarpTiles = 256;  // 16-token tiles one warp takes in a split (ids in smem)
-constexpr int kMaxSplitTokens = kMaxWarpTiles * 4 * kTileTokens;  // 16,384 keys per split
+constexpr int kMaxWarpTiles = 128;  // 16-token tiles one warp takes in a split (list in smem)
+constexpr int kMaxSplitTokens = kMaxWarpTiles * 4 * kTileTokens;  // 8,192 keys per split
 constexpr int kMaxSplits = 256;     // splits per (sequence, KV head, head group)
 constexpr int kMaxPages = (1 << 27) - 1;  // pool pages (tile lists pack page << 4)
 

@@ -12,8 +12,10 @@
 // * One thread block = one (sequence b, KV head h, group of <= 8 query
 //   heads, split of the key range). Its 4 warps take 16-token tiles of the
 //   split round robin; each warp streams its tiles HBM -> shared memory with
-//   16-byte cp.async into a private multi-stage ring (no block-wide barrier
-//   in the main loop) and keeps its own online-softmax state. The warps are
+//   TMA (one cp.async.bulk.tensor per K or V tile, issued by one lane, no
+//   multicast) into a private multi-stage ring completed on mbarriers (no
+//   block-wide barrier in the main loop) and keeps its own online-softmax
+//   state. The warps are
 //   merged once at the end; when the keys are split over several blocks the
 //   last block of a (sequence, KV head, head group) to finish merges the
 //   splits (a ticket counter, never a wait), so one launch does the call.
@@ -23,12 +25,12 @@
 //   enter the MMA without rounding; q enters exactly as f16 after a
 //   power-of-two rescale; P enters as an f16 hi + lo pair (two MMAs), which
 //   keeps it to about 22 significant bits.
-// * The MMA k index may map to any head-dim (QK) or token (PV) order as
-//   long as both operands agree; the orders below are chosen so that every
-//   operand word comes from one 32-bit shared-memory word or one byte
-//   permute, and the shared-memory layouts are XOR-swizzled so that those
-//   loads are free of bank conflicts.
+// * Operands leave shared memory through ldmatrix (K as stored, V
+//   transposed: a pair of E4M3 bytes is one 16-bit matrix element), which
+//   with the TMA's 128-byte swizzle reads every 8-row column without bank
+//   conflicts and needs one address per lane per 32 columns.
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
@@ -87,24 +89,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ uint4 lds128(uint32_t a) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(a));
-  return v;
-}
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(a));
@@ -136,37 +120,6 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// ---------------------------------------------------------------------------
-// Tile layouts in shared memory: a 16-token K (or V) tile of one KV head is
-// 16 rows of D bytes, stored in 16-byte chunks with an XOR swizzle on the
-// chunk index inside each 128-byte line.
-//  K: lane (g, q) of a warp reads 16 bytes at (row g, chunk 4j + q); rows g
-//     and g+1 share a read phase, so odd rows flip chunk bit 2.
-//  V: lane (g, q) reads 4 bytes at (row 2q + e, byte 32j + 4g); the four
-//     rows 2q + e of one read must land in different 32-byte groups, so
-//     chunk bits 1..2 are flipped by row bits 1..2.
-// D = 64 packs two rows per 128-byte line; its K rows already split the line
-// and its V swizzle works on the line index.
-// ---------------------------------------------------------------------------
-template <int D>
-__device__ __forceinline__ uint32_t k_off(int row, int chunk) {
-  if constexpr (D == 64) {
-    return row * 64 + chunk * 16;
-  } else {
-    return row * D + ((chunk ^ ((row & 1) << 2)) << 4);
-  }
-}
-template <int D>
-__device__ __forceinline__ uint32_t v_off(int row, int chunk) {
-  if constexpr (D == 64) {
-    const int line = row >> 1;
-    const int cil = ((row & 1) << 2) | chunk;
-    return line * 128 + ((cil ^ ((line & 3) << 1)) << 4);
-  } else {
-    return row * D + ((chunk ^ (row & 6)) << 4);
-  }
-}
-
 // Hardware E4M3 -> f16 conversion of bytes (0,1) or (2,3) of a word
 // (cvt.rn.f16x2.e4m3x2; exact). Used by the K path when selected.
 __device__ __forceinline__ uint32_t e4m3x2_lo16_to_f16x2(uint32_t w) {
@@ -195,14 +148,75 @@ __device__ __forceinline__ float2 ldcg2(const float* p) {
   return v;
 }
 
+// ---------------------------------------------------------------------------
+// Asynchronous tile copies (TMA) and their mbarriers.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+// Waits for phase `parity` of the barrier; gives up (returns false) after a
+// bounded number of polls so that a lost copy can never hang the GPU.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+#pragma unroll 1
+  for (int it = 0; it < (1 << 22); ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+// 5-D tiled TMA load (no multicast) into this block's shared memory.
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0,
+                                            int c1, int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Four 8x8 matrices of 16-bit elements (here: pairs of E4M3 bytes); lane l
+// supplies the address of row l % 8 of matrix l / 8.
+__device__ __forceinline__ uint4 ldsm_x4(uint32_t addr) {
+  uint4 r;
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(addr));
+  return r;
+}
+__device__ __forceinline__ uint4 ldsm_x4_trans(uint32_t addr) {
+  uint4 r;
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(addr));
+  return r;
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src) : "memory");
 }
 
 // Transposes an 8x8 matrix of 16-bit elements held one row pair per lane
@@ -219,29 +233,49 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
 
 constexpr int kMergeFan = 8;  // splits merged per group in the two-level merge
 
+// ---------------------------------------------------------------------------
+// Shared-memory tile layout. The TMA writes one 16-token tile of one KV head
+// as [D/128 column blocks][16 rows][128 bytes] (D >= 128, 128-byte swizzle:
+// 16-byte chunk c of row r sits at chunk c ^ (r % 8)) or [16 rows][64 bytes]
+// (D = 64, 64-byte swizzle: chunk c of row r at c ^ ((r / 2) % 4)). Every
+// ldmatrix then reads 8 rows of one 16-byte column with no bank conflict.
+// tile_off(r, b) = byte offset of row r, byte column b (b a multiple of 16).
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ uint32_t tile_off(int r, int b) {
+  if constexpr (D == 64) {
+    return r * 64 + ((((b >> 4) ^ ((r >> 1) & 3))) << 4);
+  } else {
+    return (b >> 7) * 2048 + r * 128 + (((((b & 127) >> 4) ^ (r & 7))) << 4);
+  }
+}
+
 template <int D>
 struct Cfg {
   static constexpr int NW = 4;                                        // warps per block
   static constexpr int NS = (D == 64) ? 6 : (D == 128) ? 3 : 2;       // ring stages per warp
   static constexpr int TILE = kTileTokens * D;                        // bytes of a K or V tile
-  static constexpr int STAGE = 2 * TILE + 16;                         // K, V, then k / v scale
+  static constexpr int STAGE = 2 * TILE;
   static constexpr int WARP_BYTES = NS * STAGE;
-  static constexpr int PIPE_BYTES = (NW * WARP_BYTES + 127) / 128 * 128;
+  static constexpr int PIPE_BYTES = NW * WARP_BYTES;                  // multiple of 1024
   static constexpr bool Q_IN_SMEM = (D > 256);                        // q fragments in smem
   static constexpr int QFRAG_BYTES = Q_IN_SMEM ? (D / 16) * 32 * 8 : 0;
-  static constexpr int LIST_BYTES = NW * kMaxWarpTiles * 4;           // each warp's tile list
+  static constexpr int LIST_BYTES = NW * kMaxWarpTiles * 12;          // tile entry, k / v scale
+  static constexpr int BAR_BYTES = NW * NS * 8;
   static constexpr int MISC_FLOATS = NW * 8 * 2 + 4;
-  static constexpr int SMEM = PIPE_BYTES + QFRAG_BYTES + LIST_BYTES + MISC_FLOATS * 4;
+  static constexpr int SMEM = 1024 /* alignment slack */ + PIPE_BYTES + QFRAG_BYTES + LIST_BYTES +
+                              BAR_BYTES + MISC_FLOATS * 4;
   static constexpr int MIN_BLOCKS = (D == 512) ? 1 : (D == 256) ? 2 : 4;
+  static_assert(PIPE_BYTES % 1024 == 0, "tiles must stay 1024-byte aligned for the swizzle");
   static_assert(NW * 8 * D * 4 <= PIPE_BYTES, "merge scratch must fit in the ring");
   static_assert(8 * 32 * 4 <= PIPE_BYTES, "merge weights must fit in the ring");
 };
 
 // Merges K partial rows (max m, sum l, numerator O, all in log2 units) of one
-// (sequence, head group): for head n they are rows row0(n) + s, s < K, of
-// (ml, o). With `final`, the sink enters the denominator once and the result
-// (numerator / denominator) goes to `out`; otherwise the merged (m, l, O) goes
-// to row dst_row(n) of (dst_ml, dst_o). Called by one whole block.
+// (sequence, head group): for head n they are rows row0 + n * head_rows + s,
+// s < K, of (ml, o). With `final`, the sink enters the denominator once and
+// numerator / denominator goes to `out`; otherwise the merged (m, l, O) goes to
+// row dst_row0 + n * dst_head_rows of (dst_ml, dst_o). Called by the whole block.
 template <int D, int NW>
 __device__ void merge_partials(const float* ml, const float* o, int64_t row0, int64_t head_rows,
                                int K, int nheads, bool final, const DecodeParams& p, int b,
@@ -296,17 +330,25 @@ __device__ void merge_partials(const float* ml, const float* o, int64_t row0, in
 // One thread block: (split, KV head x head group, sequence). KCVT / VCVT
 // select the E4M3 -> f16 decode of K / V: false = bit assembly (value * 2^-8),
 // true = hardware cvt.rn.f16x2.e4m3x2 (the value itself). The q fragments
-// follow the K byte pairing.
+// follow the K byte pairing. tmk / tmv: 5-D tensor maps over the K / V pool
+// views, dims (head-dim bytes within a 128-byte block, slot, 128-byte block,
+// KV head, page), box (min(D,128), 16, max(1, D/128), 1, 1).
 template <int D, bool KCVT, bool VCVT>
 __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
-    decode_mma_kernel(const DecodeParams p) {
+    decode_tma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv) {
   using C = Cfg<D>;
   constexpr int KB = D / 16;  // k16 blocks of the QK contraction
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned base for the swizzled tiles
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* pipe = smem;
   uint2* qfrag_s = reinterpret_cast<uint2*>(smem + C::PIPE_BYTES);
-  int32_t* s_list = reinterpret_cast<int32_t*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES);
-  float* misc = reinterpret_cast<float*>(s_list + C::NW * kMaxWarpTiles);
+  int32_t* s_ent = reinterpret_cast<int32_t*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES);
+  float* s_ks = reinterpret_cast<float*>(s_ent + C::NW * kMaxWarpTiles);
+  float* s_vs = s_ks + C::NW * kMaxWarpTiles;
+  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_vs + C::NW * kMaxWarpTiles);
+  float* misc = reinterpret_cast<float*>(s_bar + C::NW * C::NS);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, grp = lane >> 2, qd = lane & 3;
@@ -315,6 +357,16 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   const int hg = blockIdx.y - kvh * p.head_groups;
   const int head0 = kvh * p.G + hg * 8;
   const int nheads = min(8, p.G - hg * 8);
+
+  const uint32_t wbar = smem_u32(s_bar + warp * C::NS);
+  if (lane == 0) {
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+#pragma unroll
+    for (int s = 0; s < C::NS; ++s) mbar_init(wbar + 8 * s, 1);
+    fence_barrier_init();
+    fence_proxy_async();
+  }
 
   // ---- the keys this block attends: [t0, t1) ------------------------------
   // Split s of a sequence covers pages [first + s * chunk, first + (s+1) * chunk)
@@ -342,35 +394,44 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   const int32_t* trow = p.table + (int64_t)b * p.tab_sb;
 
   // ---- warp-local setup: this warp's tile list, q fragments -----------------
-  // Tile j of warp w starts at token 16 * (tile_first + w + 4j); its list
-  // entry packs the physical page and the tile's index inside the page as
-  // (page << 4) | index, or -1 when the block-table entry is out of range.
-  int32_t* wlist = s_list + warp * kMaxWarpTiles;
-#pragma unroll 4
+  // Tile j of warp w starts at token 16 * (tile_first + w + 4j). Its entry is
+  // (page << 4) | (tile index inside the page), or -1 for a block-table entry
+  // outside the pool; the page's k and v scales sit beside it.
+  int32_t* went = s_ent + warp * kMaxWarpTiles;
+  float* wks = s_ks + warp * kMaxWarpTiles;
+  float* wvs = s_vs + warp * kMaxWarpTiles;
+  const float* ksbase = p.ks + (int64_t)kvh * p.ks_sh;
+  const float* vsbase = p.vs + (int64_t)kvh * p.vs_sh;
+#pragma unroll 2
   for (int j = lane; j < my_tiles; j += 32) {
     const int tok = (tile_first + warp + C::NW * j) * kTileTokens;
     const int lp = tok / p.ps;
     const int page = __ldg(trow + (int64_t)lp * p.tab_sp);
     int e = -1;
+    float ks = 0.f, vs = 0.f;
     if ((unsigned)page < (unsigned)p.num_pages) {
       e = (page << 4) | ((tok - lp * p.ps) / kTileTokens);
+      ks = __ldg(ksbase + (int64_t)page * p.ks_sp);
+      vs = __ldg(vsbase + (int64_t)page * p.vs_sp);
     } else if (hg == 0) {
       raise_flag(FP8PD_FLAG_PAGE_OOB);
     }
-    wlist[j] = e;
+    went[j] = e;
+    wks[j] = ks;
+    wvs[j] = vs;
   }
-  // Lane (g, q) holds query head g of the group at head-dim entries
-  // 64jj + 16q + {0..15}; the k16 block (jj, i) covers entries
-  // 64jj + 16q + 4i + {0..3}. Bit-assembly K pairs bytes (0,2) and (1,3):
-  // k = 2q -> +0, 2q+1 -> +2, 2q+8 -> +1, 2q+9 -> +3; hardware-cvt K pairs
-  // (0,1) and (2,3).
+  // Lane (g, q) holds query head g of the group; the k16 block kb covers
+  // head-dim entries 16kb + 4q + {0..3} of lane quad q. Hardware-cvt K pairs
+  // bytes (0,1) and (2,3): k = 2q -> +0, 2q+1 -> +1, 2q+8 -> +2, 2q+9 -> +3;
+  // bit-assembly K pairs (0,2) and (1,3): k = 2q -> +0, 2q+1 -> +2, 2q+8 -> +1,
+  // 2q+9 -> +3.
   const bool q_head_ok = grp < nheads;
   const uint16_t* qrow = p.q + (int64_t)b * p.q_sb + (int64_t)(head0 + (q_head_ok ? grp : 0)) * p.q_sh;
   float qmax = 0.f;
   if (q_head_ok) {
 #pragma unroll 8
     for (int e = 0; e < D / 4; ++e) {
-      const int d = 64 * (e >> 4) + 16 * qd + (e & 15);
+      const int d = 16 * (e >> 2) + 4 * qd + (e & 3);
       qmax = fmaxf(qmax, fabsf(bf16_bits_to_float(__ldg(qrow + (int64_t)d * p.q_sd))));
     }
   }
@@ -394,7 +455,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     if constexpr (C::Q_IN_SMEM) {
       if ((kb & 3) != warp) continue;  // the four warps share the work
     }
-    const int d = 64 * (kb >> 2) + 16 * qd + 4 * (kb & 3);
+    const int d = 16 * kb + 4 * qd;
     uint32_t r0, r1;
     if constexpr (KCVT) {
       r0 = pack_f16x2(qval(d + 0), qval(d + 1));
@@ -415,33 +476,46 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
 
   // ---- per-warp pipeline over 16-token tiles --------------------------------
   const uint32_t wpipe = smem_u32(pipe + warp * C::WARP_BYTES);
-  const uint8_t* kbase = p.k + (int64_t)kvh * p.k_sh;
-  const uint8_t* vbase = p.v + (int64_t)kvh * p.v_sh;
-  const float* ksbase = p.ks + (int64_t)kvh * p.ks_sh;
-  const float* vsbase = p.vs + (int64_t)kvh * p.vs_sh;
-  const int64_t k_tile_st = (int64_t)kTileTokens * p.k_st;
-  const int64_t v_tile_st = (int64_t)kTileTokens * p.v_st;
-
-  // Copies tile j of this warp into ring stage `stage`: K and V rows (16-byte
-  // cp.async per lane), then the page's k and v scales (4 bytes each).
-  auto issue = [&](int j, int stage) {
-    const int e = wlist[j];
-    if (e < 0) return;
-    const int page = e >> 4, tip = e & 15;
-    const uint8_t* gk = kbase + (int64_t)page * p.k_sp + tip * k_tile_st;
-    const uint8_t* gv = vbase + (int64_t)page * p.v_sp + tip * v_tile_st;
-    const uint32_t sk = wpipe + stage * C::STAGE;
-    const uint32_t sv = sk + C::TILE;
-    constexpr int CPR = D / 16;
+  // Per-lane ldmatrix row offsets inside a tile. K (no transpose): matrix
+  // i = lane / 8 is rows (lane % 8) + 8 * (i % 2) at byte column 16 * (i / 2)
+  // of each 32-byte block; V (transposed): rows (lane % 8) + 8 * (i / 2) at
+  // byte column 16 * (i % 2). The swizzle makes the offset of 32-byte block kc
+  // depend on kc % 4 (D >= 128) or kc (D = 64), so four offsets per operand.
+  uint32_t koff[4], voff[4];
+  {
+    const int i = lane >> 3;
+    const int rk = (lane & 7) + 8 * (i & 1), hk = i >> 1;
+    const int rv = (lane & 7) + 8 * (i >> 1), hv = i & 1;
 #pragma unroll
-    for (int it = 0; it < (kTileTokens * CPR) / 32; ++it) {
-      const int idx = it * 32 + lane;
-      const int r = idx / CPR, c = idx - r * CPR;
-      cp_async16(sk + k_off<D>(r, c), gk + (int64_t)r * p.k_st + c * 16);
-      cp_async16(sv + v_off<D>(r, c), gv + (int64_t)r * p.v_st + c * 16);
+    for (int kc = 0; kc < 4; ++kc) {
+      koff[kc] = tile_off<D>(rk, 32 * kc + 16 * hk);
+      voff[kc] = tile_off<D>(rv, 32 * kc + 16 * hv);
     }
-    if (lane == 0) cp_async4(sv + C::TILE, ksbase + (int64_t)page * p.ks_sp);
-    if (lane == 1) cp_async4(sv + C::TILE + 4, vsbase + (int64_t)page * p.vs_sp);
+  }
+  auto blk_off = [&](const uint32_t (&off)[4], int kc) -> uint32_t {
+    // 32-byte block kc: blocks 4.. of a 128-byte line group repeat the
+    // offsets of blocks 0..3 one 2048-byte column block further (D >= 128)
+    if constexpr (D == 64) return off[kc];
+    else return off[kc & 3] + (kc >> 2) * 2048;
+  };
+
+  // Lane 0 issues tile j of this warp into ring stage `stage`: one TMA for
+  // K, one for V, both completing on the stage's barrier. A tile whose page
+  // is out of range is not copied; its barrier phase still completes.
+  auto issue = [&](int j, int stage) {
+    if (lane != 0) return;
+    const uint32_t bar = wbar + 8 * stage;
+    const int e = went[j];
+    if (e < 0) {
+      mbar_arrive(bar);
+      return;
+    }
+    const int page = e >> 4, slot0 = (e & 15) * kTileTokens;
+    const uint32_t sk = wpipe + stage * C::STAGE;
+    fence_proxy_async();  // this warp's earlier reads of the stage come first
+    mbar_arrive_expect_tx(bar, 2 * C::TILE);
+    tma_load_5d(sk, &tmk, bar, 0, slot0, 0, kvh, page);
+    tma_load_5d(sk + C::TILE, &tmv, bar, 0, slot0, 0, kvh, page);
   };
 
   float O[D / 32][2][4];
@@ -456,65 +530,71 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   // Running V reference scale: the largest |v_scale| seen so far. O holds
   // sum P * v_scale / vref, so every f16 P operand stays <= 1 in magnitude.
   float vref = 0.f, inv_vref = 0.f;
+  bool ok_all = true;
 
 #pragma unroll 1
-  for (int s = 0; s < C::NS - 1; ++s) {
+  for (int s = 0; s < C::NS - 1; ++s)
     if (s < my_tiles) issue(s, s);
-    cp_async_commit();
-  }
+  __syncwarp();
 
+  int stage = 0;
+  uint32_t phase = 0;
+  int tok0 = (tile_first + warp) * kTileTokens;
 #pragma unroll 1
-  for (int j = 0; j < my_tiles; ++j) {
-    cp_async_wait<C::NS - 2>();
+  for (int j = 0; j < my_tiles; ++j, tok0 += C::NW * kTileTokens) {
+    if (!mbar_wait(wbar + 8 * stage, phase)) {
+      if (lane == 0) raise_flag(FP8PD_FLAG_TIMEOUT);
+      ok_all = false;
+      break;
+    }
     __syncwarp();
     {
       const int nj = j + C::NS - 1;
-      if (nj < my_tiles) issue(nj, nj % C::NS);
-      cp_async_commit();
+      if (nj < my_tiles) issue(nj, stage == 0 ? C::NS - 1 : stage - 1);
     }
-    const int tok0 = (tile_first + warp + C::NW * j) * kTileTokens;
-    const bool page_ok = wlist[j] >= 0;
+    const bool page_ok = went[j] >= 0;
     const bool full = page_ok && tok0 >= t0 && tok0 + kTileTokens <= t1;  // warp-uniform
-    const uint32_t sk = wpipe + (j % C::NS) * C::STAGE;
+    const uint32_t sk = wpipe + stage * C::STAGE;
     const uint32_t sv = sk + C::TILE;
-    float kfac = 0.f, vs = 0.f;
-    if (page_ok) {
-      kfac = score_base * __uint_as_float(lds32(sv + C::TILE));
-      vs = __uint_as_float(lds32(sv + C::TILE + 4));
+    const float kfac = score_base * wks[j];
+    const float vs = wvs[j];
+    if (++stage == C::NS) {
+      stage = 0;
+      phase ^= 1;
     }
 
     // -- S[token][head] = K q'^T (two independent accumulator chains) --------
     float Sa[4] = {0.f, 0.f, 0.f, 0.f}, Sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int jj = 0; jj < D / 64; ++jj) {
-      const uint4 ka = lds128(sk + k_off<D>(grp, 4 * jj + qd));
-      const uint4 kb = lds128(sk + k_off<D>(grp + 8, 4 * jj + qd));
-      const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
-      const uint32_t wb[4] = {kb.x, kb.y, kb.z, kb.w};
+    for (int kc = 0; kc < D / 32; ++kc) {
+      // rows g / g+8, bytes 32kc + 4q.. (regs 0 / 1) and 32kc + 16 + 4q.. (2 / 3)
+      const uint4 kw = ldsm_x4(sk + blk_off(koff, kc));
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int half = 0; half < 2; ++half) {
+        const int kb = 2 * kc + half;
+        const uint32_t wa = half ? kw.z : kw.x, wb = half ? kw.w : kw.y;
         uint32_t b0, b1;
         if constexpr (C::Q_IN_SMEM) {
-          const uint2 f = qfrag_s[(jj * 4 + i) * 32 + lane];
+          const uint2 f = qfrag_s[kb * 32 + lane];
           b0 = f.x;
           b1 = f.y;
         } else {
-          b0 = qf[jj * 4 + i][0];
-          b1 = qf[jj * 4 + i][1];
+          b0 = qf[kb][0];
+          b1 = qf[kb][1];
         }
         uint32_t a0, a1, a2, a3;
         if constexpr (KCVT) {
-          a0 = e4m3x2_lo16_to_f16x2(wa[i]);
-          a1 = e4m3x2_lo16_to_f16x2(wb[i]);
-          a2 = e4m3x2_hi16_to_f16x2(wa[i]);
-          a3 = e4m3x2_hi16_to_f16x2(wb[i]);
+          a0 = e4m3x2_lo16_to_f16x2(wa);
+          a1 = e4m3x2_lo16_to_f16x2(wb);
+          a2 = e4m3x2_hi16_to_f16x2(wa);
+          a3 = e4m3x2_hi16_to_f16x2(wb);
         } else {
-          a0 = e4m3x2_b02_to_f16x2(wa[i]);
-          a1 = e4m3x2_b02_to_f16x2(wb[i]);
-          a2 = e4m3x2_b13_to_f16x2(wa[i]);
-          a3 = e4m3x2_b13_to_f16x2(wb[i]);
+          a0 = e4m3x2_b02_to_f16x2(wa);
+          a1 = e4m3x2_b02_to_f16x2(wb);
+          a2 = e4m3x2_b13_to_f16x2(wa);
+          a3 = e4m3x2_b13_to_f16x2(wb);
         }
-        if (i & 1)
+        if (half)
           mma16816(Sb, a0, a1, a2, a3, b0, b1);
         else
           mma16816(Sa, a0, a1, a2, a3, b0, b1);
@@ -580,55 +660,45 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     const uint32_t bl0 = movmatrix_trans(la), bl1 = movmatrix_trans(lb);
 
     // -- O^T[d][head] += V^T P ---------------------------------------------
-    // Block jb covers d in [32jb, 32jb+32). Lane (g, q) reads bytes 4g..4g+3
-    // of the block from tokens 2q, 2q+1, 2q+8, 2q+9; M tile (jb, h) row g is
-    // d = 32jb + 4g + 2h, row g+8 is d + 1. With the hardware cvt a masked
-    // row is zeroed first (a NaN byte times P = 0 would still be NaN).
-    uint32_t vm0 = ~0u, vm1 = ~0u, vm2 = ~0u, vm3 = ~0u;
+    // ldmatrix.trans of the 32-byte block jb gives lane (g, q) the bytes
+    // (d, d+1), d = 32jb + 2g, of tokens 2q and 2q+1 (reg 0), the same for
+    // d + 16 (reg 1), and for tokens 2q+8, 2q+9 (regs 2, 3). M tile (jb, 0)
+    // rows g / g+8 are d / d+1; M tile (jb, 1) adds 16.
+    uint32_t vmask_lo = ~0u, vmask_hi = ~0u;
     if (VCVT && !full) {
+      // with the hardware cvt a masked row must be zeroed (a NaN byte times
+      // P = 0 would still be NaN); bytes 0-1 / 2-3 are tokens 2q / 2q+1
       const int r = tok0 + 2 * qd;
-      vm0 = (page_ok && r >= t0 && r < t1) ? ~0u : 0u;
-      vm1 = (page_ok && r + 1 >= t0 && r + 1 < t1) ? ~0u : 0u;
-      vm2 = (page_ok && r + 8 >= t0 && r + 8 < t1) ? ~0u : 0u;
-      vm3 = (page_ok && r + 9 >= t0 && r + 9 < t1) ? ~0u : 0u;
+      auto in = [&](int t) { return page_ok && t >= t0 && t < t1; };
+      vmask_lo = (in(r) ? 0x0000FFFFu : 0u) | (in(r + 1) ? 0xFFFF0000u : 0u);
+      vmask_hi = (in(r + 8) ? 0x0000FFFFu : 0u) | (in(r + 9) ? 0xFFFF0000u : 0u);
     }
 #pragma unroll
     for (int jb = 0; jb < D / 32; ++jb) {
-      const int c = 2 * jb + (grp >> 2);
-      const uint32_t cb = (grp & 3) * 4;
-      uint32_t w0 = lds32(sv + v_off<D>(2 * qd, c) + cb);
-      uint32_t w1 = lds32(sv + v_off<D>(2 * qd + 1, c) + cb);
-      uint32_t w2 = lds32(sv + v_off<D>(2 * qd + 8, c) + cb);
-      uint32_t w3 = lds32(sv + v_off<D>(2 * qd + 9, c) + cb);
+      const uint4 vw = ldsm_x4_trans(sv + blk_off(voff, jb));
       uint32_t a0, a1, a2, a3, e0, e1, e2, e3;
       if constexpr (VCVT) {
-        w0 &= vm0;
-        w1 &= vm1;
-        w2 &= vm2;
-        w3 &= vm3;
-        // [w0.c, w1.c, w0.c+1, w1.c+1]: each 16-bit half is one column's token pair
-        const uint32_t za = prmt(w0, w1, 0x5140), zb = prmt(w0, w1, 0x7362);
-        const uint32_t zc = prmt(w2, w3, 0x5140), zd = prmt(w2, w3, 0x7362);
-        a0 = e4m3x2_lo16_to_f16x2(za);
-        a1 = e4m3x2_hi16_to_f16x2(za);
-        a2 = e4m3x2_lo16_to_f16x2(zc);
-        a3 = e4m3x2_hi16_to_f16x2(zc);
-        e0 = e4m3x2_lo16_to_f16x2(zb);
-        e1 = e4m3x2_hi16_to_f16x2(zb);
-        e2 = e4m3x2_lo16_to_f16x2(zd);
-        e3 = e4m3x2_hi16_to_f16x2(zd);
+        // [t.d, t'.d, t.d+1, t'.d+1]: each 16-bit half is one column's token pair
+        const uint32_t z0 = prmt(vw.x & vmask_lo, 0, 0x3120), z1 = prmt(vw.y & vmask_lo, 0, 0x3120);
+        const uint32_t z2 = prmt(vw.z & vmask_hi, 0, 0x3120), z3 = prmt(vw.w & vmask_hi, 0, 0x3120);
+        a0 = e4m3x2_lo16_to_f16x2(z0);
+        a1 = e4m3x2_hi16_to_f16x2(z0);
+        a2 = e4m3x2_lo16_to_f16x2(z2);
+        a3 = e4m3x2_hi16_to_f16x2(z2);
+        e0 = e4m3x2_lo16_to_f16x2(z1);
+        e1 = e4m3x2_hi16_to_f16x2(z1);
+        e2 = e4m3x2_lo16_to_f16x2(z3);
+        e3 = e4m3x2_hi16_to_f16x2(z3);
       } else {
-        // [w0.c, w0.c+1, w1.c, w1.c+1]: bytes (0,2) and (1,3) are token pairs
-        const uint32_t za = prmt(w0, w1, 0x5410), zb = prmt(w0, w1, 0x7632);
-        const uint32_t zc = prmt(w2, w3, 0x5410), zd = prmt(w2, w3, 0x7632);
-        a0 = e4m3x2_b02_to_f16x2(za);
-        a1 = e4m3x2_b13_to_f16x2(za);
-        a2 = e4m3x2_b02_to_f16x2(zc);
-        a3 = e4m3x2_b13_to_f16x2(zc);
-        e0 = e4m3x2_b02_to_f16x2(zb);
-        e1 = e4m3x2_b13_to_f16x2(zb);
-        e2 = e4m3x2_b02_to_f16x2(zd);
-        e3 = e4m3x2_b13_to_f16x2(zd);
+        // [t.d, t.d+1, t'.d, t'.d+1]: bytes (0,2) and (1,3) are token pairs
+        a0 = e4m3x2_b02_to_f16x2(vw.x);
+        a1 = e4m3x2_b13_to_f16x2(vw.x);
+        a2 = e4m3x2_b02_to_f16x2(vw.z);
+        a3 = e4m3x2_b13_to_f16x2(vw.z);
+        e0 = e4m3x2_b02_to_f16x2(vw.y);
+        e1 = e4m3x2_b13_to_f16x2(vw.y);
+        e2 = e4m3x2_b02_to_f16x2(vw.w);
+        e3 = e4m3x2_b13_to_f16x2(vw.w);
       }
       mma16816(O[jb][0], a0, a1, a2, a3, bh0, bh1);
       mma16816(O[jb][0], a0, a1, a2, a3, bl0, bl1);
@@ -636,7 +706,13 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       mma16816(O[jb][1], e0, e1, e2, e3, bl0, bl1);
     }
   }
-  cp_async_wait<0>();
+  if (!ok_all) {
+    // A copy never completed: leave this warp's result out (its flag is set)
+    // and wait, again bounded, for whatever this warp still has in flight.
+    for (int s = 0; s < C::NS; ++s) mbar_wait(wbar + 8 * s, phase ^ (s < stage ? 1u : 0u));
+    m0 = m1 = -CUDART_INF_F;
+    l0 = l1 = 0.f;
+  }
 
   // ---- merge the warps ------------------------------------------------------
 #pragma unroll
@@ -648,14 +724,17 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   float* Os = reinterpret_cast<float*>(pipe);  // [NW][8][D], already times fold
   float* ml = misc;                            // [NW][8][2]
   // f16 offset of the decoded V (bit assembly only), times the V reference scale
-  const float fold = (VCVT ? 1.f : 256.f) * vref;
+  const float fold = ok_all ? (VCVT ? 1.f : 256.f) * vref : 0.f;
 #pragma unroll
   for (int jb = 0; jb < D / 32; ++jb) {
-    const int d = 32 * jb + 4 * grp;
-    *reinterpret_cast<float4*>(Os + (warp * 8 + 2 * qd) * D + d) = make_float4(
-        O[jb][0][0] * fold, O[jb][0][2] * fold, O[jb][1][0] * fold, O[jb][1][2] * fold);
-    *reinterpret_cast<float4*>(Os + (warp * 8 + 2 * qd + 1) * D + d) = make_float4(
-        O[jb][0][1] * fold, O[jb][0][3] * fold, O[jb][1][1] * fold, O[jb][1][3] * fold);
+    const int d = 32 * jb + 2 * grp;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      *reinterpret_cast<float2*>(Os + (warp * 8 + 2 * qd) * D + d + 16 * h) =
+          make_float2(O[jb][h][0] * fold, O[jb][h][2] * fold);
+      *reinterpret_cast<float2*>(Os + (warp * 8 + 2 * qd + 1) * D + d + 16 * h) =
+          make_float2(O[jb][h][1] * fold, O[jb][h][3] * fold);
+    }
   }
   if (grp == 0) {
     ml[(warp * 8 + 2 * qd) * 2 + 0] = m0;
@@ -810,7 +889,8 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
 // Launchers
 // ---------------------------------------------------------------------------
 template <int D, bool KCVT, bool VCVT>
-static cudaError_t launch_decode_mma_d(const DecodeParams& p, cudaStream_t s) {
+static cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap& tmk,
+                                   const CUtensorMap& tmv, cudaStream_t s) {
   // The shared-memory opt-in is a per-device function attribute: set it once
   // per device (an idempotent call, so a race only repeats it).
   static std::atomic<uint64_t> configured{0};
@@ -820,40 +900,34 @@ static cudaError_t launch_decode_mma_d(const DecodeParams& p, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
   if (!bit || !(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(decode_mma_kernel<D, KCVT, VCVT>,
+    e = cudaFuncSetAttribute(decode_tma_kernel<D, KCVT, VCVT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
   const dim3 grid(p.num_splits, p.Hkv * p.head_groups, p.B);
-  decode_mma_kernel<D, KCVT, VCVT><<<grid, 128, smem, s>>>(p);
+  decode_tma_kernel<D, KCVT, VCVT><<<grid, 128, smem, s>>>(p, tmk, tmv);
   return cudaGetLastError();
 }
 
 template <int D>
-static cudaError_t launch_decode_mma_kv(const DecodeParams& p, bool k_cvt, bool v_cvt,
-                                       cudaStream_t s) {
-  if (k_cvt) return v_cvt ? launch_decode_mma_d<D, true, true>(p, s) : launch_decode_mma_d<D, true, false>(p, s);
-  return v_cvt ? launch_decode_mma_d<D, false, true>(p, s) : launch_decode_mma_d<D, false, false>(p, s);
+static cudaError_t launch_decode_kv(const DecodeParams& p, const CUtensorMap& tmk,
+                                   const CUtensorMap& tmv, bool k_cvt, bool v_cvt, cudaStream_t s) {
+  if (k_cvt)
+    return v_cvt ? launch_decode_d<D, true, true>(p, tmk, tmv, s)
+                 : launch_decode_d<D, true, false>(p, tmk, tmv, s);
+  return v_cvt ? launch_decode_d<D, false, true>(p, tmk, tmv, s)
+               : launch_decode_d<D, false, false>(p, tmk, tmv, s);
 }
 
-cudaError_t launch_decode_mma(const DecodeParams& p, int D, bool k_cvt, bool v_cvt, cudaStream_t s) {
-  switch (D) {
-    case 64: return launch_decode_mma_kv<64>(p, k_cvt, v_cvt, s);
-    case 128: return launch_decode_mma_kv<128>(p, k_cvt, v_cvt, s);
-    case 256: return launch_decode_mma_kv<256>(p, k_cvt, v_cvt, s);
-    case 512: return launch_decode_mma_kv<512>(p, k_cvt, v_cvt, s);
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                          bool k_cvt, bool v_cvt, cudaStream_t s) {
+  switch (p.D) {
+    case 64: return launch_decode_kv<64>(p, tmk, tmv, k_cvt, v_cvt, s);
+    case 128: return launch_decode_kv<128>(p, tmk, tmv, k_cvt, v_cvt, s);
+    case 256: return launch_decode_kv<256>(p, tmk, tmv, k_cvt, v_cvt, s);
+    case 512: return launch_decode_kv<512>(p, tmk, tmv, k_cvt, v_cvt, s);
     default: return cudaErrorInvalidValue;
-  }
-}
-
-int decode_mma_smem_bytes(int D) {
-  switch (D) {
-    case 64: return Cfg<64>::SMEM;
-    case 128: return Cfg<128>::SMEM;
-    case 256: return Cfg<256>::SMEM;
-    case 512: return Cfg<512>::SMEM;
-    default: return 0;
   }
 }
 
@@ -863,9 +937,9 @@ static int blocks_per_sm_d() {
   int c = cached.load();
   if (c >= 0) return c;
   int n = 0;
-  if (cudaFuncSetAttribute(decode_mma_kernel<D, true, true>,
+  if (cudaFuncSetAttribute(decode_tma_kernel<D, true, true>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_mma_kernel<D, true, true>, 128,
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tma_kernel<D, true, true>, 128,
                                                     Cfg<D>::SMEM) != cudaSuccess) {
     cudaGetLastError();
     return Cfg<D>::MIN_BLOCKS;  // no device: do not cache the guess
@@ -875,13 +949,23 @@ static int blocks_per_sm_d() {
   return c;
 }
 
-int decode_mma_blocks_per_sm(int D) {
+int decode_blocks_per_sm(int D) {
   switch (D) {
     case 64: return blocks_per_sm_d<64>();
     case 128: return blocks_per_sm_d<128>();
     case 256: return blocks_per_sm_d<256>();
     case 512: return blocks_per_sm_d<512>();
     default: return 1;
+  }
+}
+
+int decode_smem_bytes(int D) {
+  switch (D) {
+    case 64: return Cfg<64>::SMEM;
+    case 128: return Cfg<128>::SMEM;
+    case 256: return Cfg<256>::SMEM;
+    case 512: return Cfg<512>::SMEM;
+    default: return 0;
   }
 }
 

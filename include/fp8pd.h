@@ -100,7 +100,7 @@ enum {
                                        smaller than the call needs (reserve it first) */
   FP8PD_ERR_CUDA = -9,              /* a CUDA runtime call failed */
   FP8PD_ERR_TOO_LARGE = -10         /* a size exceeds a documented limit (e.g. more than
-                                       4,194,304 attended keys in one sequence) */
+                                       2,097,152 attended keys in one sequence) */
 };
 
 /* Bits of the device error word. */
@@ -108,8 +108,10 @@ enum {
   FP8PD_FLAG_PAGE_OOB = 1u,    /* block-table entry outside [0, num_pages): tile skipped */
   FP8PD_FLAG_SEQLEN_OOB = 2u,  /* seq_lens[b] < 0 or > max_pages * page_size: sequence skipped */
   FP8PD_FLAG_POS_OOB = 4u,     /* append position < 0 or >= max_pages * page_size: not written */
-  FP8PD_FLAG_INTERNAL = 8u     /* a split covered more keys than the kernel holds (a planner
+  FP8PD_FLAG_INTERNAL = 8u,    /* a split covered more keys than the kernel holds (a planner
                                   bug): that split is left out */
+  FP8PD_FLAG_TIMEOUT = 16u     /* a tile copy did not complete within the kernel's bounded wait:
+                                  that warp's keys are left out */
 };
 
 /*
@@ -215,7 +217,7 @@ int fp8pd_check_errors(fp8pd_stream_t stream, uint32_t* flags);
 /* Options (process-wide). */
 enum {
   FP8PD_OPT_NUM_SPLITS = 1,  /* 0 = planner chooses (default); n > 0 asks for n splits (raised
-                                so that no split covers more than 16,384 keys, capped at 256
+                                so that no split covers more than 8,192 keys, capped at 256
                                 splits and at the number of pages) */
   FP8PD_OPT_VARIANT = 2,     /* 0 = auto; 1 = tensor-core (mma) split kernel;
                                 2 = CUDA-core (f32 FMA) split kernel */

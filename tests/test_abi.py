@@ -149,15 +149,15 @@ def test_planner_fills_the_device_with_enough_work_per_split(F):
     assert p["workspace_bytes"] >= 1 * 64 * S * (128 + 2) * 4 + 8 * 4
     NG = (S + 7) // 8
     assert p["workspace_bytes"] <= 64 * (S + NG) * (128 + 2) * 4 + 8 * (1 + NG) * 4 + 5 * 256
-    # no split may cover more than 16,384 keys: 1 Mi keys on 16-token pages
+    # no split may cover more than 8,192 keys: 1 Mi keys on 16-token pages
     p = _plan(F, 64, 64, 8, 64, 16, 65537)
-    assert p["num_splits"] >= 65 and 65537 * 16 / p["num_splits"] <= 16384 + 16
+    assert p["num_splits"] >= 129 and 65537 * 16 / p["num_splits"] <= 8192 + 16
     assert p["num_splits"] <= 256
-    # more than 256 splits of 16,384 keys in one sequence is refused
+    # more than 256 splits of 8,192 keys in one sequence is refused
     with pytest.raises(F.Fp8pdError) as e:
-        _plan(F, 1, 8, 8, 128, 16, 256 * 1024 + 1)
+        _plan(F, 1, 8, 8, 128, 16, 256 * 512 + 1)
     assert e.value.status == -10
-    assert _plan(F, 1, 8, 8, 128, 16, 256 * 1024 + 1, window=4096)["num_splits"] >= 1
+    assert _plan(F, 1, 8, 8, 128, 16, 256 * 512 + 1, window=4096)["num_splits"] >= 1
     # short window: one split, no combine, no workspace
     p = _plan(F, 64, 64, 8, 64, 16, 513, window=128)
     assert p["num_splits"] == 1 and p["combine"] == 0 and p["workspace_bytes"] == 0
@@ -170,7 +170,7 @@ def test_planner_fills_the_device_with_enough_work_per_split(F):
     try:
         assert _plan(F, 4, 32, 8, 128, 16, 100)["num_splits"] == 5
         assert _plan(F, 4, 32, 8, 128, 16, 3)["num_splits"] == 3
-        assert _plan(F, 4, 32, 8, 128, 16, 6000)["num_splits"] == 6    # raised: <= 16,384 keys each
+        assert _plan(F, 4, 32, 8, 128, 16, 6000)["num_splits"] == 12   # raised: <= 8,192 keys each
         F.fp8pd_set_option(F.OPT_NUM_SPLITS, 1000)
         assert 240 <= _plan(F, 4, 32, 8, 128, 16, 5000)["num_splits"] <= 256  # capped
     finally:
