@@ -133,9 +133,9 @@ int current_device(int* dev) {
 // Splits per (sequence, KV head, head group). Split s covers pages
 // [s * chunk, (s+1) * chunk) of a sequence's attended range, so every block
 // has the same amount of work whatever the sequence lengths (blocks past the
-// end of a short sequence finish at once). The count fills whole waves of the
-// device with >= 512 keys per split, never more than 8,192 keys per split
-// (the kernel's per-warp tile list) nor more than kMaxSplits splits.
+// end of a short sequence finish at once). The count aims at just under two
+// waves of the device, with >= 512 keys per split, never more than 8,192 keys
+// per split (the kernel's per-warp tile list) nor more than kMaxSplits splits.
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, Plan* plan) {
@@ -156,8 +156,9 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
   if (forced > 0) {
     S = std::min<int64_t>(forced, std::min<int64_t>(pages, fp8pd::kMaxSplits));
   } else if (units > 0) {
-    // At least 1.25 waves of blocks: with equal-sized splits the hardware
-    // scheduler then evens out ragged lengths; fewer would leave SMs idle.
+    // Just under two waves of blocks: equal-sized splits fill whole waves
+    // for uniform lengths (a partial extra wave would cost a whole split),
+    // and the second wave lets the scheduler even out ragged lengths.
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) {
       int v = 0;
@@ -165,7 +166,7 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
     }
     cudaGetLastError();
     const int64_t slots = static_cast<int64_t>(sms) * fp8pd::decode_blocks_per_sm(D);
-    S = std::min<int64_t>(s_max, (5 * slots + 4 * units - 1) / (4 * units));
+    S = std::min<int64_t>(s_max, (2 * slots) / units);
     S = std::max<int64_t>(S, 1);
   }
   S = std::max<int64_t>(S, s_min);

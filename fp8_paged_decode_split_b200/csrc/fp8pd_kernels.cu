@@ -161,14 +161,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
-// Waits for phase `parity` of the barrier; gives up (returns false) after a
-// bounded number of polls so that a lost copy can never hang the GPU.
+// Waits for phase `parity` of the barrier. Each poll lets the warp sleep in
+// the barrier for up to 20 us (the suspend-time hint) instead of spinning;
+// after 2^17 polls (about 2.6 s) it gives up and returns false, so a lost copy
+// can never hang the GPU.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 #pragma unroll 1
-  for (int it = 0; it < (1 << 22); ++it) {
+  for (int it = 0; it < (1 << 17); ++it) {
     uint32_t ok;
     asm volatile(
-        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 20000;\n"
         "selp.u32 %0, 1, 0, p;\n}\n"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
