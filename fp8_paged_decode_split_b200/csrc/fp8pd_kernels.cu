@@ -235,6 +235,18 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
 
 constexpr int kMergeFan = 8;  // splits merged per group in the two-level merge
 
+// Pipeline depth (ring stages per warp) and blocks per SM the register budget
+// targets; compile-time settings, overridable for tuning builds.
+#ifndef FP8PD_NS_D64
+#define FP8PD_NS_D64 6
+#endif
+#ifndef FP8PD_NS_D128
+#define FP8PD_NS_D128 3
+#endif
+#ifndef FP8PD_MIN_BLOCKS_D128
+#define FP8PD_MIN_BLOCKS_D128 4
+#endif
+
 // ---------------------------------------------------------------------------
 // Shared-memory tile layout. The TMA writes one 16-token tile of one KV head
 // as [D/128 column blocks][16 rows][128 bytes] (D >= 128, 128-byte swizzle:
@@ -255,7 +267,7 @@ __device__ __forceinline__ uint32_t tile_off(int r, int b) {
 template <int D>
 struct Cfg {
   static constexpr int NW = 4;                                        // warps per block
-  static constexpr int NS = (D == 64) ? 6 : (D == 128) ? 3 : 2;       // ring stages per warp
+  static constexpr int NS = (D == 64) ? FP8PD_NS_D64 : (D == 128) ? FP8PD_NS_D128 : 2;  // ring stages per warp
   static constexpr int TILE = kTileTokens * D;                        // bytes of a K or V tile
   static constexpr int STAGE = 2 * TILE;
   static constexpr int WARP_BYTES = NS * STAGE;
@@ -267,7 +279,7 @@ struct Cfg {
   static constexpr int MISC_FLOATS = NW * 8 * 2 + 4;
   static constexpr int SMEM = 1024 /* alignment slack */ + PIPE_BYTES + QFRAG_BYTES + LIST_BYTES +
                               BAR_BYTES + MISC_FLOATS * 4;
-  static constexpr int MIN_BLOCKS = (D == 512) ? 1 : (D == 256) ? 2 : 4;
+  static constexpr int MIN_BLOCKS = (D == 512) ? 1 : (D == 256) ? 2 : FP8PD_MIN_BLOCKS_D128;
   static_assert(PIPE_BYTES % 1024 == 0, "tiles must stay 1024-byte aligned for the swizzle");
   static_assert(NW * 8 * D * 4 <= PIPE_BYTES, "merge scratch must fit in the ring");
   static_assert(8 * 32 * 4 <= PIPE_BYTES, "merge weights must fit in the ring");
@@ -395,30 +407,63 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   }
   const int32_t* trow = p.table + (int64_t)b * p.tab_sb;
 
-  // ---- warp-local setup: this warp's tile list, q fragments -----------------
+  // ---- warp-local setup: tile list, first copies, scales, q fragments -------
   // Tile j of warp w starts at token 16 * (tile_first + w + 4j). Its entry is
   // (page << 4) | (tile index inside the page), or -1 for a block-table entry
-  // outside the pool; the page's k and v scales sit beside it.
+  // outside the pool; the page's k and v scales sit beside it. The page ids
+  // come first so the first tile copies are in flight while the scales and
+  // the q fragments load.
   int32_t* went = s_ent + warp * kMaxWarpTiles;
   float* wks = s_ks + warp * kMaxWarpTiles;
   float* wvs = s_vs + warp * kMaxWarpTiles;
-  const float* ksbase = p.ks + (int64_t)kvh * p.ks_sh;
-  const float* vsbase = p.vs + (int64_t)kvh * p.vs_sh;
 #pragma unroll 2
   for (int j = lane; j < my_tiles; j += 32) {
     const int tok = (tile_first + warp + C::NW * j) * kTileTokens;
     const int lp = tok / p.ps;
     const int page = __ldg(trow + (int64_t)lp * p.tab_sp);
     int e = -1;
-    float ks = 0.f, vs = 0.f;
     if ((unsigned)page < (unsigned)p.num_pages) {
       e = (page << 4) | ((tok - lp * p.ps) / kTileTokens);
-      ks = __ldg(ksbase + (int64_t)page * p.ks_sp);
-      vs = __ldg(vsbase + (int64_t)page * p.vs_sp);
     } else if (hg == 0) {
       raise_flag(FP8PD_FLAG_PAGE_OOB);
     }
     went[j] = e;
+  }
+  __syncwarp();
+
+  const uint32_t wpipe = smem_u32(pipe + warp * C::WARP_BYTES);
+  // Lane 0 issues tile j of this warp into ring stage `stage`: one TMA for
+  // K, one for V, both completing on the stage's barrier. A tile whose page
+  // is out of range is not copied; its barrier phase still completes.
+  auto issue = [&](int j, int stage) {
+    if (lane != 0) return;
+    const uint32_t bar = wbar + 8 * stage;
+    const int e = went[j];
+    if (e < 0) {
+      mbar_arrive(bar);
+      return;
+    }
+    const int page = e >> 4, slot0 = (e & 15) * kTileTokens;
+    const uint32_t sk = wpipe + stage * C::STAGE;
+    fence_proxy_async();  // this warp's earlier reads of the stage come first
+    mbar_arrive_expect_tx(bar, 2 * C::TILE);
+    tma_load_5d(sk, &tmk, bar, 0, slot0, 0, kvh, page);
+    tma_load_5d(sk + C::TILE, &tmv, bar, 0, slot0, 0, kvh, page);
+  };
+#pragma unroll 1
+  for (int s = 0; s < C::NS - 1; ++s)
+    if (s < my_tiles) issue(s, s);
+
+  const float* ksbase = p.ks + (int64_t)kvh * p.ks_sh;
+  const float* vsbase = p.vs + (int64_t)kvh * p.vs_sh;
+#pragma unroll 2
+  for (int j = lane; j < my_tiles; j += 32) {
+    const int e = went[j];
+    float ks = 0.f, vs = 0.f;
+    if (e >= 0) {
+      ks = __ldg(ksbase + (int64_t)(e >> 4) * p.ks_sp);
+      vs = __ldg(vsbase + (int64_t)(e >> 4) * p.vs_sp);
+    }
     wks[j] = ks;
     wvs[j] = vs;
   }
@@ -477,7 +522,6 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   __syncwarp();
 
   // ---- per-warp pipeline over 16-token tiles --------------------------------
-  const uint32_t wpipe = smem_u32(pipe + warp * C::WARP_BYTES);
   // Per-lane ldmatrix row offsets inside a tile. K (no transpose): matrix
   // i = lane / 8 is rows (lane % 8) + 8 * (i % 2) at byte column 16 * (i / 2)
   // of each 32-byte block; V (transposed): rows (lane % 8) + 8 * (i / 2) at
@@ -501,25 +545,6 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     else return off[kc & 3] + (kc >> 2) * 2048;
   };
 
-  // Lane 0 issues tile j of this warp into ring stage `stage`: one TMA for
-  // K, one for V, both completing on the stage's barrier. A tile whose page
-  // is out of range is not copied; its barrier phase still completes.
-  auto issue = [&](int j, int stage) {
-    if (lane != 0) return;
-    const uint32_t bar = wbar + 8 * stage;
-    const int e = went[j];
-    if (e < 0) {
-      mbar_arrive(bar);
-      return;
-    }
-    const int page = e >> 4, slot0 = (e & 15) * kTileTokens;
-    const uint32_t sk = wpipe + stage * C::STAGE;
-    fence_proxy_async();  // this warp's earlier reads of the stage come first
-    mbar_arrive_expect_tx(bar, 2 * C::TILE);
-    tma_load_5d(sk, &tmk, bar, 0, slot0, 0, kvh, page);
-    tma_load_5d(sk + C::TILE, &tmv, bar, 0, slot0, 0, kvh, page);
-  };
-
   float O[D / 32][2][4];
 #pragma unroll
   for (int jb = 0; jb < D / 32; ++jb)
@@ -533,11 +558,6 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   // sum P * v_scale / vref, so every f16 P operand stays <= 1 in magnitude.
   float vref = 0.f, inv_vref = 0.f;
   bool ok_all = true;
-
-#pragma unroll 1
-  for (int s = 0; s < C::NS - 1; ++s)
-    if (s < my_tiles) issue(s, s);
-  __syncwarp();
 
   int stage = 0;
   uint32_t phase = 0;
