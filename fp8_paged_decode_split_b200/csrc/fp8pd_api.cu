@@ -351,6 +351,10 @@ int validate_decode(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp
   p->max_pages = static_cast<int>(max_pages);
   p->window = window;
   p->sm_scale_log2 = sm_scale * 1.4426950408889634f;
+  p->q_vec = (q->stride[2] == 1 && q->stride[1] % 4 == 0 && q->stride[0] % 4 == 0 &&
+              reinterpret_cast<uintptr_t>(q->data) % 8 == 0)
+                 ? 1
+                 : 0;
   a->B = p->B;
   a->Hq = p->Hq;
   a->Hkv = p->Hkv;

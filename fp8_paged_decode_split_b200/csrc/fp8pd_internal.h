@@ -36,6 +36,7 @@ struct DecodeParams {
   int B, Hq, Hkv, G, D, ps, num_pages, max_pages, window, num_splits, head_groups;
   int chunk_pages;            // pages per split (the last split of a sequence may have fewer)
   int num_groups;             // ceil(num_splits / 8): groups of the two-level split merge
+  int q_vec;                  // 1: q rows are contiguous and 8-byte aligned (vector loads)
   float sm_scale_log2;        // sm_scale * log2(e)
 };
 

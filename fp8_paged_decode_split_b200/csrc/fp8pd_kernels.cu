@@ -372,6 +372,33 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   const int head0 = kvh * p.G + hg * 8;
   const int nheads = min(8, p.G - hg * 8);
 
+  // q of this lane's query head (grp): entries 16kb + 4q + {0..3} of every
+  // k16 block kb, loaded before anything else so that their latency overlaps
+  // the rest of the setup (one 8-byte load per block when q is contiguous).
+  const bool q_head_ok = grp < nheads;
+  const uint16_t* qrow = p.q + (int64_t)b * p.q_sb + (int64_t)(head0 + (q_head_ok ? grp : 0)) * p.q_sh;
+  constexpr int QR = C::Q_IN_SMEM ? 1 : KB;
+  uint2 qraw[QR];
+  if constexpr (!C::Q_IN_SMEM) {
+#pragma unroll
+    for (int kb = 0; kb < KB; ++kb) {
+      const int d = 16 * kb + 4 * qd;
+      uint2 v = make_uint2(0u, 0u);
+      if (q_head_ok) {
+        if (p.q_vec) {
+          v = __ldg(reinterpret_cast<const uint2*>(qrow + d));
+        } else {
+          const uint32_t e0 = __ldg(qrow + (int64_t)(d + 0) * p.q_sd);
+          const uint32_t e1 = __ldg(qrow + (int64_t)(d + 1) * p.q_sd);
+          const uint32_t e2 = __ldg(qrow + (int64_t)(d + 2) * p.q_sd);
+          const uint32_t e3 = __ldg(qrow + (int64_t)(d + 3) * p.q_sd);
+          v = make_uint2(e0 | (e1 << 16), e2 | (e3 << 16));
+        }
+      }
+      qraw[kb] = v;
+    }
+  }
+
   const uint32_t wbar = smem_u32(s_bar + warp * C::NS);
   if (lane == 0) {
     prefetch_tensormap(&tmk);
@@ -472,14 +499,23 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   // bytes (0,1) and (2,3): k = 2q -> +0, 2q+1 -> +1, 2q+8 -> +2, 2q+9 -> +3;
   // bit-assembly K pairs (0,2) and (1,3): k = 2q -> +0, 2q+1 -> +2, 2q+8 -> +1,
   // 2q+9 -> +3.
-  const bool q_head_ok = grp < nheads;
-  const uint16_t* qrow = p.q + (int64_t)b * p.q_sb + (int64_t)(head0 + (q_head_ok ? grp : 0)) * p.q_sh;
   float qmax = 0.f;
-  if (q_head_ok) {
+  if constexpr (C::Q_IN_SMEM) {
+    if (q_head_ok) {
 #pragma unroll 8
-    for (int e = 0; e < D / 4; ++e) {
-      const int d = 16 * (e >> 2) + 4 * qd + (e & 3);
-      qmax = fmaxf(qmax, fabsf(bf16_bits_to_float(__ldg(qrow + (int64_t)d * p.q_sd))));
+      for (int e = 0; e < D / 4; ++e) {
+        const int d = 16 * (e >> 2) + 4 * qd + (e & 3);
+        qmax = fmaxf(qmax, fabsf(bf16_bits_to_float(__ldg(qrow + (int64_t)d * p.q_sd))));
+      }
+    }
+  } else {
+#pragma unroll
+    for (int kb = 0; kb < KB; ++kb) {
+      const uint2 v = qraw[kb];
+      qmax = fmaxf(qmax, fmaxf(fmaxf(fabsf(__uint_as_float(v.x << 16)),
+                                     fabsf(__uint_as_float(v.x & 0xFFFF0000u))),
+                               fmaxf(fabsf(__uint_as_float(v.y << 16)),
+                                     fabsf(__uint_as_float(v.y & 0xFFFF0000u)))));
     }
   }
   qmax = warp_max(qmax);
@@ -493,23 +529,34 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   // decoded by bit assembly (which yields value * 2^-8); the hardware cvt
   // yields the value itself.
   const float score_base = p.sm_scale_log2 * (KCVT ? 1.f : 256.f) / qmul;
-  auto qval = [&](int d) -> float {
-    return q_head_ok ? bf16_bits_to_float(__ldg(qrow + (int64_t)d * p.q_sd)) * qmul : 0.f;
-  };
   uint32_t qf[C::Q_IN_SMEM ? 1 : KB][2];
 #pragma unroll
   for (int kb = 0; kb < KB; ++kb) {
+    float x0, x1, x2, x3;
     if constexpr (C::Q_IN_SMEM) {
       if ((kb & 3) != warp) continue;  // the four warps share the work
+      const int d = 16 * kb + 4 * qd;
+      auto qv = [&](int dd) -> float {
+        return q_head_ok ? bf16_bits_to_float(__ldg(qrow + (int64_t)dd * p.q_sd)) : 0.f;
+      };
+      x0 = qv(d);
+      x1 = qv(d + 1);
+      x2 = qv(d + 2);
+      x3 = qv(d + 3);
+    } else {
+      const uint2 v = qraw[kb];
+      x0 = __uint_as_float(v.x << 16);
+      x1 = __uint_as_float(v.x & 0xFFFF0000u);
+      x2 = __uint_as_float(v.y << 16);
+      x3 = __uint_as_float(v.y & 0xFFFF0000u);
     }
-    const int d = 16 * kb + 4 * qd;
     uint32_t r0, r1;
     if constexpr (KCVT) {
-      r0 = pack_f16x2(qval(d + 0), qval(d + 1));
-      r1 = pack_f16x2(qval(d + 2), qval(d + 3));
+      r0 = pack_f16x2(x0 * qmul, x1 * qmul);
+      r1 = pack_f16x2(x2 * qmul, x3 * qmul);
     } else {
-      r0 = pack_f16x2(qval(d + 0), qval(d + 2));
-      r1 = pack_f16x2(qval(d + 1), qval(d + 3));
+      r0 = pack_f16x2(x0 * qmul, x2 * qmul);
+      r1 = pack_f16x2(x1 * qmul, x3 * qmul);
     }
     if constexpr (C::Q_IN_SMEM) {
       qfrag_s[kb * 32 + lane] = make_uint2(r0, r1);
