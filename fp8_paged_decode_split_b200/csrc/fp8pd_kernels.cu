@@ -366,9 +366,11 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, grp = lane >> 2, qd = lane & 3;
-  const int split = blockIdx.x, b = blockIdx.z;
-  const int kvh = blockIdx.y / p.head_groups;
-  const int hg = blockIdx.y - kvh * p.head_groups;
+  // grid (KV head x head group, sequence, split): all first splits dispatch
+  // before any second split, so the longest blocks start first
+  const int split = blockIdx.z, b = blockIdx.y;
+  const int kvh = blockIdx.x / p.head_groups;
+  const int hg = blockIdx.x - kvh * p.head_groups;
   const int head0 = kvh * p.G + hg * 8;
   const int nheads = min(8, p.G - hg * 8);
 
@@ -409,13 +411,53 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     fence_proxy_async();
   }
 
+  const int32_t* trow = p.table + (int64_t)b * p.tab_sb;
+  const uint32_t wpipe = smem_u32(pipe + warp * C::WARP_BYTES);
+  // Lane 0 copies the tile with entry e (see below) into ring stage `stage`:
+  // one TMA for K, one for V, both completing on the stage's barrier. A tile
+  // whose page is out of range is not copied; its barrier phase still
+  // completes.
+  auto issue = [&](int e, int stage) {
+    if (lane != 0) return;
+    const uint32_t bar = wbar + 8 * stage;
+    if (e < 0) {
+      mbar_arrive(bar);
+      return;
+    }
+    const int page = e >> 4, slot0 = (e & 15) * kTileTokens;
+    const uint32_t sk = wpipe + stage * C::STAGE;
+    fence_proxy_async();  // this warp's earlier reads of the stage come first
+    mbar_arrive_expect_tx(bar, 2 * C::TILE);
+    tma_load_5d(sk, &tmk, bar, 0, slot0, 0, kvh, page);
+    tma_load_5d(sk + C::TILE, &tmv, bar, 0, slot0, 0, kvh, page);
+  };
+  // Without a window a split starts at page split * chunk whatever the
+  // sequence length, so the first tiles of each warp are copied before the
+  // length is known. Copies past the end of a short sequence are drained
+  // before the block exits; a page id outside the pool is never copied.
+  const bool spec = p.window == 0;
+  if (spec) {
+    const int tf = split * p.chunk_pages * (p.ps / kTileTokens);
+    int e = -1;
+    if (lane < C::NS - 1) {
+      const int tok = (tf + warp + C::NW * lane) * kTileTokens;
+      const int lp = tok / p.ps;
+      if (lp < p.max_pages) {
+        const int page = __ldg(trow + (int64_t)lp * p.tab_sp);
+        if ((unsigned)page < (unsigned)p.num_pages) e = (page << 4) | ((tok - lp * p.ps) / kTileTokens);
+      }
+    }
+#pragma unroll
+    for (int s = 0; s < C::NS - 1; ++s) issue(__shfl_sync(0xffffffffu, e, s), s);
+  }
+
   // ---- the keys this block attends: [t0, t1) ------------------------------
   // Split s of a sequence covers pages [first + s * chunk, first + (s+1) * chunk)
   // of its attended range: equal-sized work per block whatever the length,
   // and the blocks past the end of a short sequence have nothing to do.
   int L = __ldg(p.lens + (int64_t)b * p.lens_s);
   if (L < 0 || L > p.max_pages * p.ps) {
-    if (tid == 0 && split == 0 && blockIdx.y == 0) raise_flag(FP8PD_FLAG_SEQLEN_OOB);
+    if (tid == 0 && split == 0 && blockIdx.x == 0) raise_flag(FP8PD_FLAG_SEQLEN_OOB);
     L = 0;
   }
   const int lo = p.window > 0 ? max(0, L - p.window) : 0;
@@ -432,7 +474,6 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     if (lane == 0) raise_flag(FP8PD_FLAG_INTERNAL);
     my_tiles = 0;
   }
-  const int32_t* trow = p.table + (int64_t)b * p.tab_sb;
 
   // ---- warp-local setup: tile list, first copies, scales, q fragments -------
   // Tile j of warp w starts at token 16 * (tile_first + w + 4j). Its entry is
@@ -458,28 +499,11 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   }
   __syncwarp();
 
-  const uint32_t wpipe = smem_u32(pipe + warp * C::WARP_BYTES);
-  // Lane 0 issues tile j of this warp into ring stage `stage`: one TMA for
-  // K, one for V, both completing on the stage's barrier. A tile whose page
-  // is out of range is not copied; its barrier phase still completes.
-  auto issue = [&](int j, int stage) {
-    if (lane != 0) return;
-    const uint32_t bar = wbar + 8 * stage;
-    const int e = went[j];
-    if (e < 0) {
-      mbar_arrive(bar);
-      return;
-    }
-    const int page = e >> 4, slot0 = (e & 15) * kTileTokens;
-    const uint32_t sk = wpipe + stage * C::STAGE;
-    fence_proxy_async();  // this warp's earlier reads of the stage come first
-    mbar_arrive_expect_tx(bar, 2 * C::TILE);
-    tma_load_5d(sk, &tmk, bar, 0, slot0, 0, kvh, page);
-    tma_load_5d(sk + C::TILE, &tmv, bar, 0, slot0, 0, kvh, page);
-  };
+  if (!spec) {
 #pragma unroll 1
-  for (int s = 0; s < C::NS - 1; ++s)
-    if (s < my_tiles) issue(s, s);
+    for (int s = 0; s < C::NS - 1; ++s)
+      if (s < my_tiles) issue(went[s], s);
+  }
 
   const float* ksbase = p.ks + (int64_t)kvh * p.ks_sh;
   const float* vsbase = p.vs + (int64_t)kvh * p.vs_sh;
@@ -619,7 +643,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     __syncwarp();
     {
       const int nj = j + C::NS - 1;
-      if (nj < my_tiles) issue(nj, stage == 0 ? C::NS - 1 : stage - 1);
+      if (nj < my_tiles) issue(went[nj], stage == 0 ? C::NS - 1 : stage - 1);
     }
     const bool page_ok = went[j] >= 0;
     const bool full = page_ok && tok0 >= t0 && tok0 + kTileTokens <= t1;  // warp-uniform
@@ -783,6 +807,10 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     l0 = l1 = 0.f;
   }
 
+  // speculative copies past this warp's last tile (first use of their stage)
+  if (spec)
+    for (int j = my_tiles; j < C::NS - 1; ++j) mbar_wait(wbar + 8 * j, 0);
+
   // ---- merge the warps ------------------------------------------------------
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
@@ -870,7 +898,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   __syncthreads();
   int* flag = reinterpret_cast<int*>(misc + C::NW * 8 * 2);
   const int NG = p.num_groups;
-  const int64_t unit = (int64_t)b * gridDim.y + blockIdx.y;
+  const int64_t unit = (int64_t)b * gridDim.x + blockIdx.x;
   int* ucnt = p.counters + unit * (1 + NG);
   const int g = split / kMergeFan;
   const int gsize = min(kMergeFan, S - g * kMergeFan);
@@ -974,7 +1002,7 @@ static cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap& tmk
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  const dim3 grid(p.num_splits, p.Hkv * p.head_groups, p.B);
+  const dim3 grid(p.Hkv * p.head_groups, p.B, p.num_splits);
   decode_tma_kernel<D, KCVT, VCVT><<<grid, 128, smem, s>>>(p, tmk, tmv);
   return cudaGetLastError();
 }
