@@ -65,7 +65,7 @@ class RunInfo(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m fp8_paged_decode_split_b200._build` "
+            f"{LIB_PATH} is missing: build it with `python fp8_paged_decode_split_b200/_build.py` "
             "(nvcc, sm_100a). There is no fallback implementation.")
     lib = ctypes.CDLL(LIB_PATH)
     P = ctypes.POINTER

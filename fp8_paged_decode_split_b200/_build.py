@@ -1,6 +1,6 @@
 """Builds the in-tree CUDA library ``_lib/libfp8pd.so`` for sm_100a with nvcc.
 
-``python -m fp8_paged_decode_split_b200._build [--force] [-v]``
+``python fp8_paged_decode_split_b200/_build.py [--force] [-v]``
 """
 
 from __future__ import annotations

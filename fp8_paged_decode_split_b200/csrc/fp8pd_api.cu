@@ -115,7 +115,7 @@ struct Plan {
   int grid_blocks = 0;
   int combine = 0;
   int num_groups = 1;
-  size_t counters_bytes = 0;  // ticket counters (first in the workspace; all zero between calls)
+  size_t counters_bytes = 0;  // ticket counters (counter area of the workspace)
   size_t ml_bytes = 0;        // split (max, sum) pairs
   size_t o_bytes = 0;         // split numerators
   size_t grp_ml_bytes = 0;    // merged groups of splits
@@ -365,15 +365,32 @@ int validate_decode(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp
   return FP8PD_OK;
 }
 
-// Returns a workspace of >= bytes on the current device, growing it unless
-// the stream is capturing.
-int get_workspace(size_t bytes, cudaStream_t s, void** out) {
+// The split workspace of a device has two areas. The counter area holds
+// only ticket counters: every call's merging blocks put the counters they
+// used back to zero, so it reads zero between calls whatever the shapes of
+// earlier calls. The partial area holds the split partials, whose layout
+// changes with the call's shape. Keeping the two apart matters: if the
+// counters sat at the start of one shared area, a call with few counters
+// would write partials over bytes that a later call with more counters
+// reads as tickets, and that later call's merges would misfire.
+//
+// The capacity T of the partial area fixes the counter area at
+// align256(T / 64 + 256) bytes. A split call (S >= 2 splits, D >= 64) has at
+// most units * S tickets and at least units * S * 66 floats of partials, so
+// every call whose plan fits in T bytes (fp8pd_plan's workspace_bytes) also
+// fits in the counter area: fp8pd_reserve_workspace(T) covers it.
+size_t counter_area(size_t T) { return align256(T / 64 + 256); }
+
+// Returns the counter and partial areas for a call needing `counters` and
+// `partials` bytes, growing the workspace (zero-filled) unless the stream is
+// capturing.
+int get_workspace(size_t counters, size_t partials, cudaStream_t s, void** ctr, void** part) {
   int dev;
   int r = current_device(&dev);
   if (r) return r;
   std::lock_guard<std::mutex> lock(g_ws_mutex);
   Workspace& w = g_ws[dev];
-  if (w.bytes < bytes) {
+  if (w.bytes < partials || counter_area(w.bytes) < counters) {
     if (is_capturing(s)) return FP8PD_ERR_CAPTURE_WORKSPACE;
     if (w.ptr) {
       cudaError_t e = cudaFree(w.ptr);  // synchronizes the device first
@@ -381,24 +398,25 @@ int get_workspace(size_t bytes, cudaStream_t s, void** out) {
       w.bytes = 0;
       if (e != cudaSuccess) return fail_cuda(e);
     }
-    size_t grow = std::max(bytes, static_cast<size_t>(1) << 20);
-    cudaError_t e = cudaMalloc(&w.ptr, grow);
+    size_t T = std::max({partials, static_cast<size_t>(1) << 20, w.bytes});
+    while (counter_area(T) < counters) T *= 2;
+    const size_t total = counter_area(T) + T;
+    cudaError_t e = cudaMalloc(&w.ptr, total);
     if (e != cudaSuccess) {
       cudaGetLastError();
       w.ptr = nullptr;
       return FP8PD_ERR_WORKSPACE;
     }
-    // The ticket counters at the start of the workspace must read zero
-    // between calls; each call's merging blocks put them back to zero.
-    e = cudaMemset(w.ptr, 0, grow);
+    e = cudaMemset(w.ptr, 0, total);
     if (e != cudaSuccess) {
       cudaFree(w.ptr);
       w.ptr = nullptr;
       return fail_cuda(e);
     }
-    w.bytes = grow;
+    w.bytes = T;
   }
-  *out = w.ptr;
+  *ctr = w.ptr;
+  *part = static_cast<uint8_t*>(w.ptr) + counter_area(w.bytes);
   return FP8PD_OK;
 }
 
@@ -445,12 +463,11 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
   p.num_groups = plan.num_groups;
   p.head_groups = plan.head_groups;
   if (plan.combine) {
-    void* ws = nullptr;
-    r = get_workspace(plan.workspace, s, &ws);
+    void *ctr = nullptr, *part = nullptr;
+    r = get_workspace(plan.counters_bytes, plan.workspace - plan.counters_bytes, s, &ctr, &part);
     if (r) return r;
-    uint8_t* base = static_cast<uint8_t*>(ws);
-    p.counters = reinterpret_cast<int*>(base);
-    base += plan.counters_bytes;
+    p.counters = static_cast<int*>(ctr);
+    uint8_t* base = static_cast<uint8_t*>(part);
     p.part_ml = reinterpret_cast<float*>(base);
     base += plan.ml_bytes;
     p.part_o = reinterpret_cast<float*>(base);
@@ -579,8 +596,8 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
 }
 
 int fp8pd_reserve_workspace(uint64_t bytes) {
-  void* ws = nullptr;
-  return get_workspace(static_cast<size_t>(bytes), nullptr, &ws);
+  void *ctr = nullptr, *part = nullptr;
+  return get_workspace(0, static_cast<size_t>(bytes), nullptr, &ctr, &part);
 }
 
 int fp8pd_check_errors(fp8pd_stream_t stream, uint32_t* flags) {

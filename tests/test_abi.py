@@ -14,8 +14,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def F():
-    from fp8_paged_decode_split_b200 import _build
-    _build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import fp8_paged_decode_split_b200 as F
     return F
 

@@ -315,6 +315,21 @@ def test_bad_lengths_and_page_ids_are_flagged(F, cuda_device):
     assert F.fp8pd_check_errors() == 0
 
 
+def test_workspace_reuse_across_call_shapes(F, cuda_device):
+    """Split calls of different shapes share the device's workspace: a call
+    with few ticket counters and a later one with more must both be right
+    (the later call's counters must not sit where the earlier call wrote its
+    split partials)."""
+    small = W.Spec("few-units", B=3, ps=16, layers=(W.LayerSpec(16, 4, 128, 0, None),),
+                   seq_len=(300, 600), scale_mode="head", seed=16)
+    for spec in (small, W.spec_with("llama", B=6, seq_len=(40, 700)), small,
+                 W.spec_with("long_b1", seq_len=20000), W.spec_with("llama", B=6, seq_len=(40, 700))):
+        case = W.make_case(spec, cuda_device)
+        assert F.fp8pd_plan(case.layers[0].q, case.layers[0].k_pages, case.layers[0].block_table,
+                            case.layers[0].window)["combine"] == 1
+        _check_layer(F, case, where=spec.name)
+
+
 # --------------------------------------------------------------- graphs
 
 def test_cuda_graph_capture_and_replay(F, cuda_device, splits):
