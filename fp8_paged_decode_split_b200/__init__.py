@@ -23,7 +23,8 @@ import os
 import torch
 
 __all__ = [
-    "fp8_paged_decode_attention", "fp8_kv_append", "fp8pd_plan", "fp8pd_reserve_workspace",
+    "fp8_paged_decode_attention", "fp8_paged_decode_attention_noalloc", "fp8_kv_append",
+    "fp8pd_plan", "fp8pd_reserve_workspace",
     "fp8pd_check_errors", "fp8pd_set_option", "fp8pd_get_option", "fp8pd_last_run_info",
     "fp8pd_timing_enable", "fp8pd_timing_collect", "Fp8pdError", "lib", "LIB_PATH",
     "FLAG_PAGE_OOB", "FLAG_SEQLEN_OOB", "FLAG_POS_OOB", "FLAG_INTERNAL", "OPT_NUM_SPLITS",
@@ -72,6 +73,7 @@ def _load() -> ctypes.CDLL:
     T = P(Tensor)
     i32, f32, vp = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p
     lib.fp8_paged_decode_attention.argtypes = [T, T, T, T, T, T, T, i32, T, f32, T, vp]
+    lib.fp8_paged_decode_attention_noalloc.argtypes = [T, T, T, T, T, T, T, i32, T, f32, T, vp]
     lib.fp8_kv_append.argtypes = [T, T, T, T, P(Scales), T, T, vp]
     lib.fp8pd_plan.argtypes = [T, T, T, i32, P(PlanInfo)]
     lib.fp8pd_reserve_workspace.argtypes = [ctypes.c_uint64]
@@ -86,7 +88,8 @@ def _load() -> ctypes.CDLL:
     lib.fp8pd_status_string.restype = ctypes.c_char_p
     lib.fp8pd_last_cuda_error.restype = i32
     lib.fp8pd_version.restype = i32
-    for name in ("fp8_paged_decode_attention", "fp8_kv_append", "fp8pd_plan",
+    for name in ("fp8_paged_decode_attention", "fp8_paged_decode_attention_noalloc",
+                 "fp8_kv_append", "fp8pd_plan",
                  "fp8pd_reserve_workspace", "fp8pd_check_errors", "fp8pd_set_option",
                  "fp8pd_last_run_info", "fp8pd_timing_enable", "fp8pd_timing_collect"):
         getattr(lib, name).restype = i32
@@ -167,6 +170,30 @@ def fp8_paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_tabl
     st = lib.fp8_paged_decode_attention(*[_ref(d) for d in ds], int(window), _ref(ds_sinks),
                                         float(sm_scale), _ref(ds_out), _stream(stream, q))
     _check(st, "fp8_paged_decode_attention")
+    return out
+
+
+def fp8_paged_decode_attention_noalloc(q, k_pages, v_pages, k_scale, v_scale, block_table,
+                                       seq_lens, window: int = 0, sinks=None,
+                                       sm_scale: float | None = None, out=None,
+                                       stream=None) -> torch.Tensor:
+    """Same as :func:`fp8_paged_decode_attention`, for callers that cannot
+    allocate device memory during the call: the split scratch is a fixed
+    8 MiB array inside the library instead of an allocated workspace, so the
+    library allocates nothing (``out`` must then be supplied by such a caller;
+    when it is None this wrapper creates it with torch). Calls on one device
+    share that array and must not overlap on the GPU."""
+    if sm_scale is None:
+        sm_scale = q.shape[-1] ** -0.5
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    _same_device(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens, sinks, out)
+    ds = [describe(t) for t in (q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens)]
+    ds_sinks, ds_out = describe(sinks), describe(out)
+    st = lib.fp8_paged_decode_attention_noalloc(*[_ref(d) for d in ds], int(window),
+                                                _ref(ds_sinks), float(sm_scale), _ref(ds_out),
+                                                _stream(stream, q))
+    _check(st, "fp8_paged_decode_attention_noalloc")
     return out
 
 

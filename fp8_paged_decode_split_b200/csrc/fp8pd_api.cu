@@ -700,3 +700,98 @@ int32_t fp8pd_last_cuda_error(void) { return t_last_cuda_error; }
 int32_t fp8pd_version(void) { return FP8PD_VERSION; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode attention that allocates nothing.
+//
+// Some callers cannot allocate device memory at the point where they run
+// attention: an allocator-free runtime, a custom memory manager that owns all
+// of the device's memory, or code that must never call cudaMalloc because it
+// would synchronize the device. fp8_paged_decode_attention keeps its split
+// scratch in a workspace it allocates on first need; this entry point uses a
+// fixed array inside the library's own device image instead, so no call
+// allocates. Every GPU that loads the library holds the array until exit.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device. Host code only
+// sees a stand-in for the array's name, so the address is looked up once per
+// device, with that device current, and cached.
+int noalloc_scratch(void** out) {
+  int dev;
+  int r = current_device(&dev);
+  if (r) return r;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return fail_cuda(e);
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FP8PD_OK;
+}
+
+}  // namespace
+
+extern "C" int fp8_paged_decode_attention_noalloc(
+    const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_tensor* v_pages,
+    const fp8pd_tensor* k_scale, const fp8pd_tensor* v_scale, const fp8pd_tensor* block_table,
+    const fp8pd_tensor* seq_lens, int32_t window, const fp8pd_tensor* sinks, float sm_scale,
+    fp8pd_tensor* out, fp8pd_stream_t stream) {
+  DecodeParams p;
+  DecodeArgs a;
+  int r = validate_decode(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens, window,
+                          sinks, sm_scale, out, &p, &a);
+  if (r) return r;
+  if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
+  if (g_opt_variant.load() == 2) return FP8PD_ERR_UNSUPPORTED;
+  Plan plan;
+  r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
+  if (r) return r;
+  if (plan.workspace > kNoAllocScratchBytes) return FP8PD_ERR_TOO_LARGE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  p.num_splits = plan.num_splits;
+  p.chunk_pages = plan.chunk_pages;
+  p.num_groups = plan.num_groups;
+  p.head_groups = plan.head_groups;
+  if (plan.combine) {
+    void* ws = nullptr;
+    r = noalloc_scratch(&ws);
+    if (r) return r;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    // The ticket counters must read zero when the kernel starts; the array
+    // keeps whatever the previous call left, so clear them on the stream.
+    cudaError_t e = cudaMemsetAsync(base, 0, plan.counters_bytes, s);
+    if (e != cudaSuccess) return fail_cuda(e);
+    p.counters = reinterpret_cast<int*>(base);
+    base += plan.counters_bytes;
+    p.part_ml = reinterpret_cast<float*>(base);
+    base += plan.ml_bytes;
+    p.part_o = reinterpret_cast<float*>(base);
+    base += plan.o_bytes;
+    p.grp_ml = reinterpret_cast<float*>(base);
+    base += plan.grp_ml_bytes;
+    p.grp_o = reinterpret_cast<float*>(base);
+  }
+  CUtensorMap tmk, tmv;
+  if ((r = make_pool_map(k_pages, &tmk))) return r;
+  if ((r = make_pool_map(v_pages, &tmv))) return r;
+  const cudaError_t e = fp8pd::launch_decode(p, tmk, tmv, g_opt_k_decode.load() == 1,
+                                             g_opt_v_decode.load() == 1, s);
+  if (e != cudaSuccess) return fail_cuda(e);
+  ++g_launches;
+  ++g_calls;
+  t_run_info.variant = 1;
+  t_run_info.num_splits = plan.num_splits;
+  t_run_info.head_groups = plan.head_groups;
+  t_run_info.grid_blocks = plan.grid_blocks;
+  t_run_info.combine = plan.combine;
+  t_run_info.head_dim = a.D;
+  return FP8PD_OK;
+}

@@ -193,6 +193,33 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
                   const fp8pd_tensor* block_table, const fp8pd_tensor* positions,
                   fp8pd_stream_t stream);
 
+/*
+ * fp8_paged_decode_attention_noalloc -- the same operation, allocating nothing.
+ *
+ * This entry point has no counterpart in the method's description; it is for
+ * callers that cannot allocate device memory where they run attention (an
+ * allocator-free runtime, a memory manager that owns all of the device's
+ * memory, or code that must not call cudaMalloc because it synchronizes the
+ * device). Arguments, results and errors are those of
+ * fp8_paged_decode_attention. The split scratch is a fixed 8 MiB array inside
+ * the library's device image (every GPU that loads the library holds it until
+ * the process exits) instead of the allocated workspace; a call whose plan
+ * needs more returns FP8PD_ERR_TOO_LARGE and launches nothing. No call
+ * allocates or frees memory: the first call on a device looks up the array's
+ * device address once (cudaGetSymbolAddress), so make that first call before
+ * any stream capture. Each call clears the array's ticket counters with an
+ * asynchronous memset on `stream`. All calls on a device share the array, and
+ * the array keeps the last call's contents: calls that overlap on the GPU
+ * (different streams without ordering) race and give wrong results.
+ */
+int fp8_paged_decode_attention_noalloc(const fp8pd_tensor* q, const fp8pd_tensor* k_pages,
+                                       const fp8pd_tensor* v_pages, const fp8pd_tensor* k_scale,
+                                       const fp8pd_tensor* v_scale,
+                                       const fp8pd_tensor* block_table,
+                                       const fp8pd_tensor* seq_lens, int32_t window,
+                                       const fp8pd_tensor* sinks, float sm_scale,
+                                       fp8pd_tensor* out, fp8pd_stream_t stream);
+
 /* What a call with these arguments would launch, without launching it. */
 typedef struct fp8pd_plan_info {
   int32_t num_splits;        /* thread blocks per (sequence, KV head, head group) */
