@@ -48,7 +48,7 @@ WORKLOAD_TEXT = {
     "long_b1": "long context: B=1 Hq=64 Hkv=8 D=128 page=64 L=131072 +append",
     "long_b8": "long context: B=8 Hq=64 Hkv=8 D=128 page=64 L=131072 +append",
 }
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic_per_launch.txt")
 
 
 def _peaks() -> dict:
@@ -70,15 +70,17 @@ def _kernel_source_hash() -> str:
 
 
 def _traffic(config: str):
-    """DRAM bytes per split-kernel launch from the committed ncu summary, if
-    it was taken on the current kernel source and this workload."""
+    """DRAM bytes (read + write) per split-kernel launch from the committed ncu
+    summary, if it was taken on the current kernel source and this workload.
+    Lines of that file: ``<workload> <kernel source hash> <bytes>``."""
     try:
         with open(PROFILE_TRAFFIC) as f:
-            d = json.load(f)
-        e = d.get(config)
-        if e and e.get("kernel_hash") == _kernel_source_hash():
-            return float(e["dram_bytes_per_launch"])
-    except Exception:
+            for line in f:
+                parts = line.split()
+                if len(parts) == 3 and not line.startswith("#") and parts[0] == config \
+                        and parts[1] == _kernel_source_hash():
+                    return float(parts[2])
+    except OSError:
         pass
     return None
 
@@ -245,6 +247,10 @@ def run_ours(args) -> dict | None:
            for _ in range(args.steps)]
     torch.cuda.synchronize(dev)
     for i in range(args.steps):
+        # a ~1 ms spin first, so the host has queued the whole step before the
+        # GPU reaches it: the library's per-kernel events then hold device
+        # time only, with no host launch gaps inside them
+        torch.cuda._sleep(2_000_000)
         ev2[i][0].record(stream)
         step.run()
         ev2[i][1].record(stream)
@@ -300,7 +306,7 @@ def run_ours(args) -> dict | None:
         "timing": "device time of CUDA-graph replays of the step (per-step events); "
                   "eager time and per-kernel events from an eager pass of the same steps",
         "eager_ms_per_step": round(eager_ms / args.steps, 6),
-        "roofline": {"bound": "hbm", "kernel": "decode_mma_kernel (split-KV attention, one launch)",
+        "roofline": {"bound": "hbm", "kernel": "decode_tma_kernel (split-KV attention with in-kernel merge, one launch)",
                      "achieved": round(achieved, 2) if achieved else None,
                      "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
                      "unit": "GB/s",
