@@ -152,6 +152,23 @@ def _dist_env():
     return world, rank, local
 
 
+def max_over_ranks(values, device) -> list:
+    """Element-wise maximum of per-rank timings over the process group (every
+    rank gets the same result); the identity without a process group."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_gbs(world: int, bytes_per_rank_step: int, ms_per_step: float) -> float:
+    """Aggregate throughput of N weak-scaled replicas: every rank processes
+    the same bytes per step; the step takes the slowest rank's time."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
 class Step:
     """One decode step of the workload through the library's public API."""
 
@@ -266,18 +283,14 @@ def run_ours(args) -> dict | None:
     # ---- end to end through the public API with host buffers -----------------
     e2e = run_e2e(F, case, dev, flush, args)
 
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e["ms"]], dev)
     if world > 1:
-        t = torch.tensor([total_ms, e2e["ms"]], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
         torch.distributed.destroy_process_group()
-    else:
-        e2e_ms = e2e["ms"]
     if rank != 0:
         return None
 
     ms_per_step = total_ms / args.steps
-    gbs = world * nbytes / (ms_per_step * 1e-3) / 1e9
+    gbs = whole_job_gbs(world, nbytes, ms_per_step)
     peaks = _peaks()
     att_ms = kt["attention_ms"] / max(1, kt["attention_launches"])
     app_ms = kt["append_ms"] / kt["append_launches"] if kt["append_launches"] else None
@@ -315,7 +328,7 @@ def run_ours(args) -> dict | None:
                      "us_per_launch": round(att_ms * 1e3, 3),
                      "append_us_per_launch": round(app_ms * 1e3, 3) if app_ms else None},
         "gpu_launches": launches,
-        "e2e": {"value": round(world * nbytes / (e2e_ms / e2e["steps"] * 1e-3) / 1e9, 2),
+        "e2e": {"value": round(whole_job_gbs(world, nbytes, e2e_ms / e2e["steps"]), 2),
                 "unit": "GB/s", "ms_per_step": round(e2e_ms / e2e["steps"], 6),
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
         "clocks": clocks.summary(),
@@ -496,6 +509,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    world = _dist_env()[0]
+    if world > 1 and args.gpus != world:
+        ap.error(f"--gpus {args.gpus} does not match WORLD_SIZE={world}")
     line = run_reference(args) if args.impl == "reference" else run_ours(args)
     if line is not None:
         print(json.dumps(line), flush=True)
