@@ -49,6 +49,9 @@ WORKLOAD_TEXT = {
     "long_b8": "long context: B=8 Hq=64 Hkv=8 D=128 page=64 L=131072 +append",
 }
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic_per_launch.txt")
+KERNEL_NAME = {1: "decode_tma_kernel (split kernel, merge in the same launch)",
+               2: "decode_flat_kernel (balanced kernel, merge in the same launch)",
+               3: "decode_tma_kernel (proportional splits, merge in the same launch)"}
 
 
 def _peaks() -> dict:
@@ -197,6 +200,7 @@ def run_ours(args) -> dict | None:
     import fp8_paged_decode_split_b200 as F
     F.fp8pd_set_option(F.OPT_K_DECODE, 1 if args.k_decode == "cvt" else 0)
     F.fp8pd_set_option(F.OPT_NUM_SPLITS, args.splits)
+    F.fp8pd_set_option(F.OPT_SCHEDULE, args.schedule)
     world, rank, local = _dist_env()
     if world > 1:
         import torch.distributed as dist
@@ -319,7 +323,7 @@ def run_ours(args) -> dict | None:
         "timing": "device time of CUDA-graph replays of the step (per-step events); "
                   "eager time and per-kernel events from an eager pass of the same steps",
         "eager_ms_per_step": round(eager_ms / args.steps, 6),
-        "roofline": {"bound": "hbm", "kernel": "decode_tma_kernel (split-KV attention with in-kernel merge, one launch)",
+        "roofline": {"bound": "hbm", "kernel": KERNEL_NAME[plan_info["schedule"]],
                      "achieved": round(achieved, 2) if achieved else None,
                      "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
                      "unit": "GB/s",
@@ -332,7 +336,8 @@ def run_ours(args) -> dict | None:
                 "unit": "GB/s", "ms_per_step": round(e2e_ms / e2e["steps"], 6),
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
         "clocks": clocks.summary(),
-        "plan": {k: plan_info[k] for k in ("num_splits", "head_groups", "grid_blocks", "combine")},
+        "plan": {k: plan_info[k] for k in ("schedule", "num_splits", "head_groups", "grid_blocks",
+                                           "combine")},
     }
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case, budget_s=args.cpu_seconds)
@@ -506,6 +511,9 @@ def main():
     ap.add_argument("--k-decode", default="bits", choices=["bits", "cvt"],
                     help="E4M3 -> f16 decode of K: bit assembly or hardware cvt")
     ap.add_argument("--splits", type=int, default=0, help="force a split count (0 = planner)")
+    ap.add_argument("--schedule", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="0 = planner, 1 = uniform splits, 2 = balanced kernel, "
+                         "3 = proportional splits")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -28,14 +28,14 @@ __all__ = [
     "fp8pd_check_errors", "fp8pd_set_option", "fp8pd_get_option", "fp8pd_last_run_info",
     "fp8pd_timing_enable", "fp8pd_timing_collect", "Fp8pdError", "lib", "LIB_PATH",
     "FLAG_PAGE_OOB", "FLAG_SEQLEN_OOB", "FLAG_POS_OOB", "FLAG_INTERNAL", "OPT_NUM_SPLITS",
-    "OPT_VARIANT", "OPT_K_DECODE", "OPT_V_DECODE",
+    "OPT_SCHEDULE", "OPT_K_DECODE", "OPT_V_DECODE",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libfp8pd.so")
 
 DTYPE_U8, DTYPE_I32, DTYPE_F32, DTYPE_BF16 = 1, 2, 3, 4
 FLAG_PAGE_OOB, FLAG_SEQLEN_OOB, FLAG_POS_OOB, FLAG_INTERNAL = 1, 2, 4, 8
-OPT_NUM_SPLITS, OPT_VARIANT, OPT_K_DECODE, OPT_V_DECODE = 1, 2, 3, 4
+OPT_NUM_SPLITS, OPT_SCHEDULE, OPT_K_DECODE, OPT_V_DECODE = 1, 2, 3, 4
 _DTYPES = {torch.uint8: DTYPE_U8, torch.int32: DTYPE_I32, torch.float32: DTYPE_F32,
            torch.bfloat16: DTYPE_BF16}
 
@@ -52,11 +52,12 @@ class Scales(ctypes.Structure):
 class PlanInfo(ctypes.Structure):
     _fields_ = [("num_splits", ctypes.c_int32), ("head_groups", ctypes.c_int32),
                 ("grid_blocks", ctypes.c_int32), ("combine", ctypes.c_int32),
-                ("workspace_bytes", ctypes.c_uint64)]
+                ("workspace_bytes", ctypes.c_uint64), ("schedule", ctypes.c_int32),
+                ("warps", ctypes.c_int32)]
 
 
 class RunInfo(ctypes.Structure):
-    _fields_ = [("variant", ctypes.c_int32), ("num_splits", ctypes.c_int32),
+    _fields_ = [("schedule", ctypes.c_int32), ("num_splits", ctypes.c_int32),
                 ("head_groups", ctypes.c_int32), ("grid_blocks", ctypes.c_int32),
                 ("combine", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("calls", ctypes.c_int64), ("appends", ctypes.c_int64),

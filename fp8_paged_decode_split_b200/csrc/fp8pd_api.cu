@@ -26,7 +26,7 @@ constexpr int kMaxDevices = 64;
 thread_local int32_t t_last_cuda_error = 0;
 thread_local fp8pd_run_info t_run_info = {};
 std::atomic<int64_t> g_calls{0}, g_appends{0}, g_launches{0};
-std::atomic<int64_t> g_opt_num_splits{0}, g_opt_variant{0}, g_opt_k_decode{1}, g_opt_v_decode{1};
+std::atomic<int64_t> g_opt_num_splits{0}, g_opt_schedule{0}, g_opt_k_decode{1}, g_opt_v_decode{1};
 
 struct Workspace {
   void* ptr = nullptr;
@@ -121,6 +121,11 @@ struct Plan {
   size_t grp_ml_bytes = 0;    // merged groups of splits
   size_t grp_o_bytes = 0;
   size_t workspace = 0;
+  int schedule = 1;            // 1 = uniform splits, 2 = balanced kernel, 3 = proportional splits
+  int nbx = 0;                 // proportional: blocks per KV head x head group
+  int warps = 0;               // balanced: warps of the grid
+  int hpu = 1;                 // balanced: heads per partial slot
+  int c1_count = 0;            // balanced: level-1 tickets (the unit tickets follow)
 };
 
 int current_device(int* dev) {
@@ -138,7 +143,123 @@ int current_device(int* dev) {
 // per split (the kernel's per-warp tile list) nor more than kMaxSplits splits.
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
-int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, Plan* plan) {
+int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) sms = v;
+  }
+  cudaGetLastError();
+  return sms;
+}
+
+// Balanced schedule: one full wave of blocks; every warp takes an equal share
+// of the tiles. Chosen (schedule option 0) for head dims 64 and 128 with no
+// forced split count, no window shorter than 2,048 keys, and at least 8 tiles
+// per warp when every sequence has its table's full length; the option can
+// force it wherever it applies (at least 8 groups of one warp per KV head x
+// head group). Returns false when it does not apply.
+bool plan_balanced(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window,
+                   bool allow, Plan* plan) {
+  const int64_t sched = g_opt_schedule.load();
+  if (!allow || sched == 1 || sched == 3 || g_opt_num_splits.load() > 0) return false;
+  if (!(D == 64 || D == 128) || B > fp8pd::kFlatMaxBatch) return false;
+  const int G = Hq / Hkv;
+  const int hg = (G + fp8pd::kHeadsPerGroup - 1) / fp8pd::kHeadsPerGroup;
+  const int64_t HX = static_cast<int64_t>(Hkv) * hg;
+  const int64_t keys = static_cast<int64_t>(max_pages) * ps;
+  const int64_t seq_tiles = window > 0 ? std::min<int64_t>(keys, window) / fp8pd::kTileTokens + 2
+                                       : (keys + fp8pd::kTileTokens - 1) / fp8pd::kTileTokens;
+  const int64_t t_max = B * HX * seq_tiles;  // tiles when every sequence is full
+  if (t_max >= (int64_t(1) << 31) - 1) return false;
+  const int blocks = device_sms() * fp8pd::flat_blocks_per_sm(D, B);
+  const int64_t nwt = static_cast<int64_t>(blocks) * fp8pd::kFlatWarps;
+  const int64_t groups = nwt / HX;  // groups of HX warps, one warp per unit of a column
+  if (groups < 8) return false;
+  if (sched != 2) return false;  // only on request: proportional splits run faster
+  const int64_t U = B * HX;
+  plan->schedule = 2;
+  plan->head_groups = hg;
+  plan->num_splits = 0;
+  plan->chunk_pages = 0;
+  plan->num_groups = 0;
+  plan->grid_blocks = blocks;
+  plan->combine = 1;
+  plan->warps = static_cast<int>(groups * HX);
+  plan->hpu = std::min(G, fp8pd::kHeadsPerGroup);
+  // slots (b + g) HX + x of segment partials; (b + W) HX + x of level-1
+  // tickets and group partials, W <= groups / 8
+  const int64_t slots1 = (B + groups) * HX, slots2 = (B + groups / fp8pd::kFlatFan + 2) * HX;
+  plan->c1_count = static_cast<int>(slots2);
+  const size_t hpu = static_cast<size_t>(plan->hpu);
+  plan->counters_bytes = align256(static_cast<size_t>(slots2 + U) * sizeof(int));
+  plan->ml_bytes = align256(static_cast<size_t>(slots1) * hpu * 2 * sizeof(float));
+  plan->o_bytes = align256(static_cast<size_t>(slots1) * hpu * D * sizeof(float));
+  plan->grp_ml_bytes = align256(static_cast<size_t>(slots2) * hpu * 2 * sizeof(float));
+  plan->grp_o_bytes = align256(static_cast<size_t>(slots2) * hpu * D * sizeof(float));
+  plan->workspace = plan->counters_bytes + plan->ml_bytes + plan->o_bytes + plan->grp_ml_bytes +
+                    plan->grp_o_bytes;
+  return true;
+}
+
+// Proportional splits: the split kernel on a grid of nbx blocks per KV head x
+// head group, shared among the sequences in the kernel in proportion to their
+// tiles (at least one block per sequence with keys, and no split above 8,192
+// keys). nbx is one full wave of blocks, or two when the sequences would
+// take more than half a wave with one block each (then rounding would leave
+// many blocks a whole sequence, so a second wave of halves balances better).
+// Needs at most 1,024 sequences; the planner's own choice also needs at least
+// 4 tiles per block slot when every sequence has its table's full length.
+bool plan_proportional(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window,
+                       Plan* plan) {
+  if (g_opt_num_splits.load() > 0 || B > fp8pd::kPropMaxBatch) return false;
+  const int G = Hq / Hkv;
+  const int hg = (G + fp8pd::kHeadsPerGroup - 1) / fp8pd::kHeadsPerGroup;
+  const int64_t HX = static_cast<int64_t>(Hkv) * hg;
+  const int64_t keys = static_cast<int64_t>(max_pages) * ps;
+  const int64_t seq_tiles = window > 0 ? std::min<int64_t>(keys, window) / fp8pd::kTileTokens + 2
+                                       : (keys + fp8pd::kTileTokens - 1) / fp8pd::kTileTokens;
+  const int64_t m_max = (seq_tiles + fp8pd::kMaxSplitTiles - 1) / fp8pd::kMaxSplitTiles;
+  if (m_max > fp8pd::kMaxSplits) return false;
+  const int64_t slots = static_cast<int64_t>(device_sms()) * fp8pd::decode_blocks_per_sm(D);
+  if (g_opt_schedule.load() == 0 && B * HX * seq_tiles < 4 * slots) return false;  // little work
+  const int64_t waves = (static_cast<int64_t>(B) * HX * 2 > slots) ? 2 : 1;
+  int64_t nbx = (waves * slots + HX - 1) / HX;
+  nbx = std::max<int64_t>(nbx, B * m_max);  // room for every sequence's minimum splits
+  nbx = std::min<int64_t>(nbx, std::min<int64_t>(65535, static_cast<int64_t>(B) * fp8pd::kMaxSplits));
+  if (nbx < B * m_max) return false;
+  plan->schedule = 3;
+  plan->head_groups = hg;
+  plan->nbx = static_cast<int>(nbx);
+  plan->num_splits = 0;
+  plan->chunk_pages = 0;
+  plan->num_groups = 0;
+  plan->grid_blocks = static_cast<int>(std::min<int64_t>(INT32_MAX, HX * nbx));
+  plan->combine = 1;
+  const int64_t groups = nbx / fp8pd::kMergeFan + B + 1;  // >= sum over sequences of ceil(S_b / 8)
+  const size_t rows = static_cast<size_t>(nbx * HX) * fp8pd::kHeadsPerGroup;
+  const size_t grows = static_cast<size_t>(groups * HX) * fp8pd::kHeadsPerGroup;
+  plan->counters_bytes = align256(static_cast<size_t>((B + groups) * HX) * sizeof(int));
+  plan->ml_bytes = align256(rows * 2 * sizeof(float));
+  plan->o_bytes = align256(rows * D * sizeof(float));
+  plan->grp_ml_bytes = align256(grows * 2 * sizeof(float));
+  plan->grp_o_bytes = align256(grows * D * sizeof(float));
+  plan->workspace = plan->counters_bytes + plan->ml_bytes + plan->o_bytes + plan->grp_ml_bytes +
+                    plan->grp_o_bytes;
+  return true;
+}
+
+int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, Plan* plan,
+              bool allow_balanced = true) {
+  if (plan_balanced(B, Hq, Hkv, D, ps, max_pages, window, allow_balanced, plan)) return FP8PD_OK;
+  // Proportional splits balance sequences of uneven length within one launch;
+  // with a short window every sequence has about the same few tiles, and the
+  // uniform splits below cost less.
+  const int64_t sched = g_opt_schedule.load();
+  if ((sched == 3 || (sched == 0 && (window == 0 || window >= 2048))) &&
+      plan_proportional(B, Hq, Hkv, D, ps, max_pages, window, plan))
+    return FP8PD_OK;
+  plan->schedule = 1;
   const int G = Hq / Hkv;
   plan->head_groups = (G + fp8pd::kHeadsPerGroup - 1) / fp8pd::kHeadsPerGroup;
   const int64_t units = static_cast<int64_t>(B) * Hkv * plan->head_groups;
@@ -159,12 +280,7 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
     // Just under two waves of blocks: equal-sized splits fill whole waves
     // for uniform lengths (a partial extra wave would cost a whole split),
     // and the second wave lets the scheduler even out ragged lengths.
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) {
-      int v = 0;
-      if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) sms = v;
-    }
-    cudaGetLastError();
+    const int sms = device_sms();
     const int64_t slots = static_cast<int64_t>(sms) * fp8pd::decode_blocks_per_sm(D);
     S = std::min<int64_t>(s_max, (2 * slots) / units);
     S = std::max<int64_t>(S, 1);
@@ -375,11 +491,13 @@ int validate_decode(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp
 // reads as tickets, and that later call's merges would misfire.
 //
 // The capacity T of the partial area fixes the counter area at
-// align256(T / 64 + 256) bytes. A split call (S >= 2 splits, D >= 64) has at
-// most units * S tickets and at least units * S * 66 floats of partials, so
-// every call whose plan fits in T bytes (fp8pd_plan's workspace_bytes) also
-// fits in the counter area: fp8pd_reserve_workspace(T) covers it.
-size_t counter_area(size_t T) { return align256(T / 64 + 256); }
+// align256(T / 32 + 256) bytes. Every call has at most one ticket per 33
+// floats of partials: a split call (S >= 2 splits, D >= 64) has at most
+// units * S tickets and units * S * 66 floats; a balanced call at most
+// 2 (units + warps) tickets and (units + warps) * 66 floats. So every call
+// whose plan fits in T bytes (fp8pd_plan's workspace_bytes) also fits in the
+// counter area: fp8pd_reserve_workspace(T) covers it.
+size_t counter_area(size_t T) { return align256(T / 32 + 256); }
 
 // Returns the counter and partial areas for a call needing `counters` and
 // `partials` bytes, growing the workspace (zero-filled) unless the stream is
@@ -440,6 +558,52 @@ EventPair* timing_slot(int kind) {
 
 extern "C" {
 
+namespace {
+
+// Kernel parameters that come from the plan, and the workspace layout:
+// counters in the counter area; (m, l) partials, numerators, then the group
+// (m, l) and numerators in the partial area.
+void apply_plan(const Plan& plan, DecodeParams* p) {
+  p->num_splits = plan.num_splits;
+  p->chunk_pages = plan.chunk_pages;
+  p->num_groups = plan.num_groups;
+  p->head_groups = plan.head_groups;
+  p->hpu = plan.hpu;
+  p->c1_count = plan.c1_count;
+  p->prop = plan.schedule == 3 ? 1 : 0;
+  p->nbx = plan.nbx;
+}
+
+void lay_out(const Plan& plan, void* ctr, void* part, DecodeParams* p) {
+  p->counters = static_cast<int*>(ctr);
+  uint8_t* base = static_cast<uint8_t*>(part);
+  p->part_ml = reinterpret_cast<float*>(base);
+  base += plan.ml_bytes;
+  p->part_o = reinterpret_cast<float*>(base);
+  base += plan.o_bytes;
+  p->grp_ml = reinterpret_cast<float*>(base);
+  base += plan.grp_ml_bytes;
+  p->grp_o = reinterpret_cast<float*>(base);
+}
+
+cudaError_t launch_planned(const Plan& plan, const DecodeParams& p, const CUtensorMap& tmk,
+                           const CUtensorMap& tmv, cudaStream_t s) {
+  const bool kc = g_opt_k_decode.load() == 1, vc = g_opt_v_decode.load() == 1;
+  if (plan.schedule == 2) return fp8pd::launch_decode_flat(p, tmk, tmv, kc, vc, plan.grid_blocks, s);
+  return fp8pd::launch_decode(p, tmk, tmv, kc, vc, s);
+}
+
+void record_run(const Plan& plan, int D) {
+  t_run_info.schedule = plan.schedule;
+  t_run_info.num_splits = plan.num_splits;
+  t_run_info.head_groups = plan.head_groups;
+  t_run_info.grid_blocks = plan.grid_blocks;
+  t_run_info.combine = plan.combine;
+  t_run_info.head_dim = D;
+}
+
+}  // namespace
+
 int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_pages,
                                const fp8pd_tensor* v_pages, const fp8pd_tensor* k_scale,
                                const fp8pd_tensor* v_scale, const fp8pd_tensor* block_table,
@@ -452,47 +616,28 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
                           sinks, sm_scale, out, &p, &a);
   if (r) return r;
   if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
-  const int64_t variant = g_opt_variant.load();
-  if (variant == 2) return FP8PD_ERR_UNSUPPORTED;  // CUDA-core variant not built in this library
   Plan plan;
   r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
   if (r) return r;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  p.num_splits = plan.num_splits;
-  p.chunk_pages = plan.chunk_pages;
-  p.num_groups = plan.num_groups;
-  p.head_groups = plan.head_groups;
+  apply_plan(plan, &p);
   if (plan.combine) {
     void *ctr = nullptr, *part = nullptr;
     r = get_workspace(plan.counters_bytes, plan.workspace - plan.counters_bytes, s, &ctr, &part);
     if (r) return r;
-    p.counters = static_cast<int*>(ctr);
-    uint8_t* base = static_cast<uint8_t*>(part);
-    p.part_ml = reinterpret_cast<float*>(base);
-    base += plan.ml_bytes;
-    p.part_o = reinterpret_cast<float*>(base);
-    base += plan.o_bytes;
-    p.grp_ml = reinterpret_cast<float*>(base);
-    base += plan.grp_ml_bytes;
-    p.grp_o = reinterpret_cast<float*>(base);
+    lay_out(plan, ctr, part, &p);
   }
   CUtensorMap tmk, tmv;
   if ((r = make_pool_map(k_pages, &tmk))) return r;
   if ((r = make_pool_map(v_pages, &tmv))) return r;
   EventPair* ev = timing_slot(0);
   if (ev) cudaEventRecord(ev->a, s);
-  cudaError_t e = fp8pd::launch_decode(p, tmk, tmv, g_opt_k_decode.load() == 1,
-                                       g_opt_v_decode.load() == 1, s);
+  cudaError_t e = launch_planned(plan, p, tmk, tmv, s);
   if (e != cudaSuccess) return fail_cuda(e);
   ++g_launches;
   if (ev) cudaEventRecord(ev->b, s);
   ++g_calls;
-  t_run_info.variant = 1;
-  t_run_info.num_splits = plan.num_splits;
-  t_run_info.head_groups = plan.head_groups;
-  t_run_info.grid_blocks = plan.grid_blocks;
-  t_run_info.combine = plan.combine;
-  t_run_info.head_dim = a.D;
+  record_run(plan, a.D);
   return FP8PD_OK;
 }
 
@@ -519,6 +664,8 @@ int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_t
   info->grid_blocks = plan.grid_blocks;
   info->combine = plan.combine;
   info->workspace_bytes = plan.workspace;
+  info->schedule = plan.schedule;
+  info->warps = plan.warps;
   return FP8PD_OK;
 }
 
@@ -614,9 +761,9 @@ int fp8pd_set_option(int32_t option, int64_t value) {
       if (value < 0 || value > 65535) return FP8PD_ERR_ARG;
       g_opt_num_splits = value;
       return FP8PD_OK;
-    case FP8PD_OPT_VARIANT:
-      if (value < 0 || value > 2) return FP8PD_ERR_ARG;
-      g_opt_variant = value;
+    case FP8PD_OPT_SCHEDULE:
+      if (value < 0 || value > 3) return FP8PD_ERR_ARG;
+      g_opt_schedule = value;
       return FP8PD_OK;
     case FP8PD_OPT_K_DECODE:
       if (value < 0 || value > 1) return FP8PD_ERR_ARG;
@@ -634,7 +781,7 @@ int fp8pd_set_option(int32_t option, int64_t value) {
 int64_t fp8pd_get_option(int32_t option) {
   switch (option) {
     case FP8PD_OPT_NUM_SPLITS: return g_opt_num_splits.load();
-    case FP8PD_OPT_VARIANT: return g_opt_variant.load();
+    case FP8PD_OPT_SCHEDULE: return g_opt_schedule.load();
     case FP8PD_OPT_K_DECODE: return g_opt_k_decode.load();
     case FP8PD_OPT_V_DECODE: return g_opt_v_decode.load();
     default: return -1;
@@ -750,16 +897,17 @@ extern "C" int fp8_paged_decode_attention_noalloc(
                           sinks, sm_scale, out, &p, &a);
   if (r) return r;
   if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
-  if (g_opt_variant.load() == 2) return FP8PD_ERR_UNSUPPORTED;
   Plan plan;
   r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
   if (r) return r;
+  if (plan.schedule == 2 && plan.workspace > kNoAllocScratchBytes) {
+    // the balanced layout does not fit: the split kernel's may
+    r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan, false);
+    if (r) return r;
+  }
   if (plan.workspace > kNoAllocScratchBytes) return FP8PD_ERR_TOO_LARGE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  p.num_splits = plan.num_splits;
-  p.chunk_pages = plan.chunk_pages;
-  p.num_groups = plan.num_groups;
-  p.head_groups = plan.head_groups;
+  apply_plan(plan, &p);
   if (plan.combine) {
     void* ws = nullptr;
     r = noalloc_scratch(&ws);
@@ -769,29 +917,15 @@ extern "C" int fp8_paged_decode_attention_noalloc(
     // keeps whatever the previous call left, so clear them on the stream.
     cudaError_t e = cudaMemsetAsync(base, 0, plan.counters_bytes, s);
     if (e != cudaSuccess) return fail_cuda(e);
-    p.counters = reinterpret_cast<int*>(base);
-    base += plan.counters_bytes;
-    p.part_ml = reinterpret_cast<float*>(base);
-    base += plan.ml_bytes;
-    p.part_o = reinterpret_cast<float*>(base);
-    base += plan.o_bytes;
-    p.grp_ml = reinterpret_cast<float*>(base);
-    base += plan.grp_ml_bytes;
-    p.grp_o = reinterpret_cast<float*>(base);
+    lay_out(plan, base, base + plan.counters_bytes, &p);
   }
   CUtensorMap tmk, tmv;
   if ((r = make_pool_map(k_pages, &tmk))) return r;
   if ((r = make_pool_map(v_pages, &tmv))) return r;
-  const cudaError_t e = fp8pd::launch_decode(p, tmk, tmv, g_opt_k_decode.load() == 1,
-                                             g_opt_v_decode.load() == 1, s);
+  const cudaError_t e = launch_planned(plan, p, tmk, tmv, s);
   if (e != cudaSuccess) return fail_cuda(e);
   ++g_launches;
   ++g_calls;
-  t_run_info.variant = 1;
-  t_run_info.num_splits = plan.num_splits;
-  t_run_info.head_groups = plan.head_groups;
-  t_run_info.grid_blocks = plan.grid_blocks;
-  t_run_info.combine = plan.combine;
-  t_run_info.head_dim = a.D;
+  record_run(plan, a.D);
   return FP8PD_OK;
 }

@@ -38,6 +38,16 @@ struct DecodeParams {
   int num_groups;             // ceil(num_splits / 8): groups of the two-level split merge
   int q_vec;                  // 1: q rows are contiguous and 8-byte aligned (vector loads)
   float sm_scale_log2;        // sm_scale * log2(e)
+  // Proportional splits (split kernel with prop = 1): grid (HX, nbx); each
+  // sequence b gets S_b of the nbx blocks of every KV head x head group, at
+  // least ceil(tiles / kMaxSplitTiles), the rest in proportion to its tiles.
+  int prop;
+  int nbx;
+  // Balanced schedule only (decode_flat_kernel): partial slots hold hpu =
+  // min(8, G) heads; the level-1 tickets are counters[0, c1_count), the
+  // per-unit final tickets counters[c1_count, c1_count + units).
+  int hpu;
+  int c1_count;
 };
 
 struct AppendParams {
@@ -63,6 +73,19 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmk, const C
                           bool k_cvt, bool v_cvt, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 
+// Balanced schedule: every warp of one full wave of blocks takes the same
+// number of 16-token tiles of the flat list of (sequence, KV head x head
+// group) units; the grid is `blocks` blocks of 128 threads.
+cudaError_t launch_decode_flat(const DecodeParams& p, const CUtensorMap& tmk,
+                               const CUtensorMap& tmv, bool k_cvt, bool v_cvt, int blocks,
+                               cudaStream_t s);
+// Blocks of the balanced kernel one SM holds for head dim D (64 or 128)
+// and a batch of B sequences.
+int flat_blocks_per_sm(int D, int B);
+constexpr int kFlatWarps = 4;        // warps per block of the balanced kernel
+constexpr int kFlatMaxBatch = 1024;  // sequences the balanced kernel keeps in shared memory
+constexpr int kFlatFan = 8;          // warps per level-1 merge group
+
 // Thread blocks of the split kernel one SM holds for head dim D.
 int decode_blocks_per_sm(int D);
 // Dynamic shared memory of the split kernel for head dim D.
@@ -75,6 +98,9 @@ constexpr int kHeadsPerGroup = 8;   // query heads one thread block serves (MMA 
 constexpr int kTileTokens = 16;     // tokens per MMA row tile
 constexpr int kMaxWarpTiles = 128;  // 16-token tiles one warp takes in a split (list in smem)
 constexpr int kMaxSplitTokens = kMaxWarpTiles * 4 * kTileTokens;  // 8,192 keys per split
+constexpr int kMaxSplitTiles = kMaxSplitTokens / kTileTokens;      // 512 tiles per split
+constexpr int kPropMaxBatch = 1024;  // sequences the proportional planner handles in the kernel
+constexpr int kMergeFan = 8;         // splits per group of the two-level split merge
 constexpr int kMaxSplits = 256;     // splits per (sequence, KV head, head group)
 constexpr int kMaxPages = (1 << 27) - 1;  // pool pages (tile lists pack page << 4)
 

@@ -233,7 +233,6 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
   return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
-constexpr int kMergeFan = 8;  // splits merged per group in the two-level merge
 
 // Pipeline depth (ring stages per warp) and blocks per SM the register budget
 // targets; compile-time settings, overridable for tuning builds.
@@ -341,6 +340,331 @@ __device__ void merge_partials(const float* ml, const float* o, int64_t row0, in
   }
 }
 
+// Byte offset inside a tile of 32-byte block kc for one lane's ldmatrix
+// row: blocks 4.. of a 128-byte line group repeat the offsets of blocks 0..3
+// one 2048-byte column block further (D >= 128).
+template <int D>
+__device__ __forceinline__ uint32_t blk_off(const uint32_t (&off)[4], int kc) {
+  if constexpr (D == 64) return off[kc];
+  else return off[kc & 3] + (kc >> 2) * 2048;
+}
+
+// Per-lane ldmatrix row offsets inside a tile. K (no transpose): matrix
+// i = lane / 8 is rows (lane % 8) + 8 * (i % 2) at byte column 16 * (i / 2)
+// of each 32-byte block; V (transposed): rows (lane % 8) + 8 * (i / 2) at
+// byte column 16 * (i % 2). The swizzle makes the offset of 32-byte block kc
+// depend on kc % 4 (D >= 128) or kc (D = 64), so four offsets per operand.
+template <int D>
+__device__ __forceinline__ void ldsm_offsets(int lane, uint32_t (&koff)[4], uint32_t (&voff)[4]) {
+  const int i = lane >> 3;
+  const int rk = (lane & 7) + 8 * (i & 1), hk = i >> 1;
+  const int rv = (lane & 7) + 8 * (i >> 1), hv = i & 1;
+#pragma unroll
+  for (int kc = 0; kc < 4; ++kc) {
+    koff[kc] = tile_off<D>(rk, 32 * kc + 16 * hk);
+    voff[kc] = tile_off<D>(rv, 32 * kc + 16 * hv);
+  }
+}
+
+// One warp's online-softmax state for up to 8 query heads: O^T[d][head] as
+// PV accumulator fragments (sum of P * v_scale / vref), the running maxima
+// (log2 units) and this lane's share of the running sums of heads 2q and
+// 2q+1, and the running V reference scale vref (the largest |v_scale| seen).
+template <int D>
+struct Acc {
+  float O[D / 32][2][4];
+  float m0, m1, l0, l1, vref, inv_vref;
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int jb = 0; jb < D / 32; ++jb)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) O[jb][h][c] = 0.f;
+    m0 = m1 = -CUDART_INF_F;
+    l0 = l1 = 0.f;
+    vref = inv_vref = 0.f;
+  }
+};
+
+// Attends one 16-token tile already in shared memory (K at sk, V at sv, the
+// swizzled layout of tile_off) for one warp: S = K q'^T on the tensor cores,
+// masking of tokens outside [t0, t1) (or of the whole tile when its page is
+// out of range), the online-softmax update, and O += V^T P with P as an f16
+// hi + lo pair. kfac = score factor of the tile's page (log2 units), vs =
+// its V scale; tok0 = first token of the tile; `full`: every token of the
+// tile is attended (warp-uniform). qfr(kb) gives the q' B-fragment of k16
+// block kb.
+template <int D, bool KCVT, bool VCVT, class QFrag>
+__device__ __forceinline__ void attend_tile(Acc<D>& a, const QFrag& qfr, uint32_t sk, uint32_t sv,
+                                            const uint32_t (&koff)[4], const uint32_t (&voff)[4],
+                                            float kfac, float vs, int tok0, int t0, int t1,
+                                            bool page_ok, bool full, int grp, int qd) {
+  // -- S[token][head] = K q'^T (two independent accumulator chains) --------
+  float Sa[4] = {0.f, 0.f, 0.f, 0.f}, Sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int kc = 0; kc < D / 32; ++kc) {
+    // rows g / g+8, bytes 32kc + 4q.. (regs 0 / 1) and 32kc + 16 + 4q.. (2 / 3)
+    const uint4 kw = ldsm_x4(sk + blk_off<D>(koff, kc));
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int kb = 2 * kc + half;
+      const uint32_t wa = half ? kw.z : kw.x, wb = half ? kw.w : kw.y;
+      uint32_t b0, b1;
+      {
+        const uint2 f = qfr(kb);
+        b0 = f.x;
+        b1 = f.y;
+      }
+      uint32_t a0, a1, a2, a3;
+      if constexpr (KCVT) {
+        a0 = e4m3x2_lo16_to_f16x2(wa);
+        a1 = e4m3x2_lo16_to_f16x2(wb);
+        a2 = e4m3x2_hi16_to_f16x2(wa);
+        a3 = e4m3x2_hi16_to_f16x2(wb);
+      } else {
+        a0 = e4m3x2_b02_to_f16x2(wa);
+        a1 = e4m3x2_b02_to_f16x2(wb);
+        a2 = e4m3x2_b13_to_f16x2(wa);
+        a3 = e4m3x2_b13_to_f16x2(wb);
+      }
+      if (half)
+        mma16816(Sb, a0, a1, a2, a3, b0, b1);
+      else
+        mma16816(Sa, a0, a1, a2, a3, b0, b1);
+    }
+  }
+
+  // -- masked scores (log2 units), online softmax ------------------------
+  // A masked row may hold stale or NaN-decoded bytes: select, never multiply.
+  const int ta = tok0 + grp, tb = ta + 8;
+  const bool va = full || (page_ok && ta >= t0 && ta < t1);
+  const bool vb = full || (page_ok && tb >= t0 && tb < t1);
+  const float s00 = va ? (Sa[0] + Sb[0]) * kfac : -CUDART_INF_F;  // token grp,   head 2qd
+  const float s01 = va ? (Sa[1] + Sb[1]) * kfac : -CUDART_INF_F;  // token grp,   head 2qd+1
+  const float s10 = vb ? (Sa[2] + Sb[2]) * kfac : -CUDART_INF_F;  // token grp+8, head 2qd
+  const float s11 = vb ? (Sa[3] + Sb[3]) * kfac : -CUDART_INF_F;  // token grp+8, head 2qd+1
+  float tm0 = fmaxf(s00, s10), tm1 = fmaxf(s01, s11);
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, o));
+    tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, o));
+  }
+  const float mn0 = fmaxf(a.m0, tm0), mn1 = fmaxf(a.m1, tm1);
+  const float vabs = fabsf(vs);
+  const bool grow_v = vabs > a.vref;  // warp-uniform: one scale per tile
+  if (grow_v || __any_sync(0xffffffffu, (mn0 > a.m0) || (mn1 > a.m1))) {
+    const float c0 = (mn0 > a.m0) ? fast_exp2(a.m0 - mn0) : 1.f;  // exp2(-inf) = 0 for a first max
+    const float c1 = (mn1 > a.m1) ? fast_exp2(a.m1 - mn1) : 1.f;
+    const float fv = grow_v ? a.vref / vabs : 1.f;
+    a.l0 *= c0;
+    a.l1 *= c1;
+    const float o0 = c0 * fv, o1 = c1 * fv;
+#pragma unroll
+    for (int jb = 0; jb < D / 32; ++jb)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        a.O[jb][h][0] *= o0;
+        a.O[jb][h][1] *= o1;
+        a.O[jb][h][2] *= o0;
+        a.O[jb][h][3] *= o1;
+      }
+    a.m0 = mn0;
+    a.m1 = mn1;
+    if (grow_v) {
+      a.vref = vabs;
+      a.inv_vref = 1.f / vabs;
+    }
+  }
+  const float mb0 = (a.m0 == -CUDART_INF_F) ? 0.f : a.m0;
+  const float mb1 = (a.m1 == -CUDART_INF_F) ? 0.f : a.m1;
+  const float p00 = fast_exp2(s00 - mb0), p01 = fast_exp2(s01 - mb1);
+  const float p10 = fast_exp2(s10 - mb0), p11 = fast_exp2(s11 - mb1);
+  a.l0 += p00 + p10;
+  a.l1 += p01 + p11;
+
+  // -- P * v_scale / a.vref as f16 hi + lo; the B fragments of the PV MMA are
+  // the transposes of the score fragment's 8x8 blocks (movmatrix).
+  const float vsr = vs * a.inv_vref;
+  const float w00 = p00 * vsr, w01 = p01 * vsr, w10 = p10 * vsr, w11 = p11 * vsr;
+  const uint32_t ha = pack_f16x2(w00, w01), hb = pack_f16x2(w10, w11);
+  const float2 fa = unpack_f16x2(ha), fb = unpack_f16x2(hb);
+  const uint32_t la = pack_f16x2(w00 - fa.x, w01 - fa.y), lb = pack_f16x2(w10 - fb.x, w11 - fb.y);
+  const uint32_t bh0 = movmatrix_trans(ha), bh1 = movmatrix_trans(hb);  // tokens 2qd.., 2qd+8..
+  const uint32_t bl0 = movmatrix_trans(la), bl1 = movmatrix_trans(lb);
+
+  // -- O^T[d][head] += V^T P ---------------------------------------------
+  // ldmatrix.trans of the 32-byte block jb gives lane (g, q) the bytes
+  // (d, d+1), d = 32jb + 2g, of tokens 2q and 2q+1 (reg 0), the same for
+  // d + 16 (reg 1), and for tokens 2q+8, 2q+9 (regs 2, 3). M tile (jb, 0)
+  // rows g / g+8 are d / d+1; M tile (jb, 1) adds 16.
+  uint32_t vmask_lo = ~0u, vmask_hi = ~0u;
+  if (VCVT && !full) {
+    // with the hardware cvt a masked row must be zeroed (a NaN byte times
+    // P = 0 would still be NaN); bytes 0-1 / 2-3 are tokens 2q / 2q+1
+    const int r = tok0 + 2 * qd;
+    auto in = [&](int t) { return page_ok && t >= t0 && t < t1; };
+    vmask_lo = (in(r) ? 0x0000FFFFu : 0u) | (in(r + 1) ? 0xFFFF0000u : 0u);
+    vmask_hi = (in(r + 8) ? 0x0000FFFFu : 0u) | (in(r + 9) ? 0xFFFF0000u : 0u);
+  }
+#pragma unroll
+  for (int jb = 0; jb < D / 32; ++jb) {
+    const uint4 vw = ldsm_x4_trans(sv + blk_off<D>(voff, jb));
+    uint32_t a0, a1, a2, a3, e0, e1, e2, e3;
+    if constexpr (VCVT) {
+      // [t.d, t'.d, t.d+1, t'.d+1]: each 16-bit half is one column's token pair
+      const uint32_t z0 = prmt(vw.x & vmask_lo, 0, 0x3120), z1 = prmt(vw.y & vmask_lo, 0, 0x3120);
+      const uint32_t z2 = prmt(vw.z & vmask_hi, 0, 0x3120), z3 = prmt(vw.w & vmask_hi, 0, 0x3120);
+      a0 = e4m3x2_lo16_to_f16x2(z0);
+      a1 = e4m3x2_hi16_to_f16x2(z0);
+      a2 = e4m3x2_lo16_to_f16x2(z2);
+      a3 = e4m3x2_hi16_to_f16x2(z2);
+      e0 = e4m3x2_lo16_to_f16x2(z1);
+      e1 = e4m3x2_hi16_to_f16x2(z1);
+      e2 = e4m3x2_lo16_to_f16x2(z3);
+      e3 = e4m3x2_hi16_to_f16x2(z3);
+    } else {
+      // [t.d, t.d+1, t'.d, t'.d+1]: bytes (0,2) and (1,3) are token pairs
+      a0 = e4m3x2_b02_to_f16x2(vw.x);
+      a1 = e4m3x2_b13_to_f16x2(vw.x);
+      a2 = e4m3x2_b02_to_f16x2(vw.z);
+      a3 = e4m3x2_b13_to_f16x2(vw.z);
+      e0 = e4m3x2_b02_to_f16x2(vw.y);
+      e1 = e4m3x2_b13_to_f16x2(vw.y);
+      e2 = e4m3x2_b02_to_f16x2(vw.w);
+      e3 = e4m3x2_b13_to_f16x2(vw.w);
+    }
+    mma16816(a.O[jb][0], a0, a1, a2, a3, bh0, bh1);
+    mma16816(a.O[jb][0], a0, a1, a2, a3, bl0, bl1);
+    mma16816(a.O[jb][1], e0, e1, e2, e3, bh0, bh1);
+    mma16816(a.O[jb][1], e0, e1, e2, e3, bl0, bl1);
+  }
+}
+
+// Proportional splits. From the lengths, every sequence's tiles nt_b and its
+// splits S_b = min(nt_b, kMaxSplits, m_b + floor(nt_b * R / total)), m_b =
+// ceil(nt_b / kMaxSplitTiles), R = nbx - sum m_b (so sum S_b <= nbx), with
+// their prefix sums and those of the merge groups ceil(S_b / 8), in
+// `scratch` (the ring buffer, unused until the first copy). Block blockIdx.y
+// = k takes split k - sp_b of the sequence b whose splits hold k; its tiles
+// are [split * nt_b / S_b, (split + 1) * nt_b / S_b) of the attended range.
+// Every block also writes the zero outputs of sequences k, k + nbx, ...
+// that have no keys. Called by the whole block; ends with a barrier, after
+// which the scratch is free. Returns false for a block beyond all splits.
+template <int NW>
+__device__ bool prop_assign(const DecodeParams& p, int* scratch, int* red, int head0, int nheads,
+                            int& b, int& split, int& S, int& j0, int& j1, int& sp_b, int& gp_b) {
+  constexpr int NT = NW * 32;
+  constexpr unsigned FULL = 0xffffffffu;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int B = p.B;
+  int* s_nt = scratch;       // [B] tiles of each sequence
+  int* s_sp = s_nt + B;      // [B + 1] splits of the sequences before b
+  int* s_gp = s_sp + B + 1;  // [B + 1] merge groups of the sequences before b
+  int tsum = 0, msum = 0;
+  for (int bb = tid; bb < B; bb += NT) {
+    int L = __ldg(p.lens + (int64_t)bb * p.lens_s);
+    if (L < 0 || L > p.max_pages * p.ps) {
+      if (blockIdx.x == 0 && blockIdx.y == 0) raise_flag(FP8PD_FLAG_SEQLEN_OOB);
+      L = 0;
+    }
+    const int lo = p.window > 0 ? max(0, L - p.window) : 0;
+    const int nt = L > lo ? (L - 1) / kTileTokens - lo / kTileTokens + 1 : 0;
+    s_nt[bb] = nt;
+    tsum += nt;
+    msum += (nt + kMaxSplitTiles - 1) / kMaxSplitTiles;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    tsum += __shfl_xor_sync(FULL, tsum, o);
+    msum += __shfl_xor_sync(FULL, msum, o);
+  }
+  if (lane == 0) {
+    red[warp] = tsum;
+    red[NW + warp] = msum;
+  }
+  __syncthreads();
+  int total = 0, mtot = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    total += red[w];
+    mtot += red[NW + w];
+  }
+  const int R = max(0, p.nbx - mtot);
+  auto splits_of = [&](int nt) -> int {
+    if (nt == 0) return 0;
+    const int m = (nt + kMaxSplitTiles - 1) / kMaxSplitTiles;
+    const int s = m + static_cast<int>((int64_t)nt * R / total);
+    return min(min(s, nt), kMaxSplits);
+  };
+  // exclusive prefix sums, a contiguous run of sequences per thread
+  const int per = (B + NT - 1) / NT;
+  const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
+  int ssum = 0, gsum = 0;
+  for (int bb = b0; bb < b1; ++bb) {
+    const int s = splits_of(s_nt[bb]);
+    ssum += s;
+    gsum += (s + kMergeFan - 1) / kMergeFan;
+  }
+  int si = ssum, gi = gsum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int vs = __shfl_up_sync(FULL, si, o), vg = __shfl_up_sync(FULL, gi, o);
+    if (lane >= o) {
+      si += vs;
+      gi += vg;
+    }
+  }
+  __syncthreads();  // everyone has read the block sums
+  if (lane == 31) {
+    red[warp] = si;
+    red[NW + warp] = gi;
+  }
+  __syncthreads();
+  int soff = si - ssum, goff = gi - gsum;
+  for (int w = 0; w < warp; ++w) {
+    soff += red[w];
+    goff += red[NW + w];
+  }
+  for (int bb = b0; bb < b1; ++bb) {
+    s_sp[bb] = soff;
+    s_gp[bb] = goff;
+    const int s = splits_of(s_nt[bb]);
+    soff += s;
+    goff += (s + kMergeFan - 1) / kMergeFan;
+  }
+  if (tid == NT - 1) {
+    s_sp[B] = soff;
+    s_gp[B] = goff;
+  }
+  __syncthreads();
+  const int k = blockIdx.y;
+  for (int bb = k; bb < B; bb += p.nbx) {
+    if (s_nt[bb] != 0) continue;
+    for (int e = tid; e < nheads * p.D; e += NT)
+      p.out[(int64_t)bb * p.o_sb + (int64_t)(head0 + e / p.D) * p.o_sh + (e % p.D)] = 0.f;
+  }
+  const bool has = k < s_sp[B];
+  if (has) {
+    int lo = 0, hi = B;  // the last sequence b with s_sp[b] <= k
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_sp[mid] <= k) lo = mid;
+      else hi = mid;
+    }
+    b = lo;
+    sp_b = s_sp[b];
+    gp_b = s_gp[b];
+    split = k - sp_b;
+    S = s_sp[b + 1] - sp_b;
+    const int nt = s_nt[b];
+    j0 = static_cast<int>((int64_t)split * nt / S);
+    j1 = static_cast<int>((int64_t)(split + 1) * nt / S);
+  }
+  __syncthreads();  // the scratch is free again
+  return has;
+}
+
 // One thread block: (split, KV head x head group, sequence). KCVT / VCVT
 // select the E4M3 -> f16 decode of K / V: false = bit assembly (value * 2^-8),
 // true = hardware cvt.rn.f16x2.e4m3x2 (the value itself). The q fragments
@@ -366,13 +690,29 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, grp = lane >> 2, qd = lane & 3;
-  // grid (KV head x head group, sequence, split): all first splits dispatch
-  // before any second split, so the longest blocks start first
-  const int split = blockIdx.z, b = blockIdx.y;
   const int kvh = blockIdx.x / p.head_groups;
   const int hg = blockIdx.x - kvh * p.head_groups;
   const int head0 = kvh * p.G + hg * 8;
   const int nheads = min(8, p.G - hg * 8);
+
+  // Which split of which sequence this block takes. Uniform splits: grid
+  // (KV head x head group, sequence, split), every sequence cut into S equal
+  // page ranges; all first splits dispatch before any second split, so the
+  // longest blocks start first. Proportional splits: grid (KV head x head
+  // group, nbx); sequence b gets S_b of the nbx blocks, S_b proportional to
+  // its tiles, and its tiles are cut into S_b near-equal ranges.
+  int b, split, S;
+  int prop_j0 = 0, prop_j1 = 0;  // proportional: tiles [j0, j1) of the attended range
+  int sp_b = 0, gp_b = 0;        // proportional: splits and merge groups of sequences < b
+  if (p.prop) {
+    if (!prop_assign<C::NW>(p, reinterpret_cast<int*>(pipe), reinterpret_cast<int*>(misc), head0,
+                            nheads, b, split, S, prop_j0, prop_j1, sp_b, gp_b))
+      return;  // a block beyond the splits of all sequences
+  } else {
+    b = blockIdx.y;
+    split = blockIdx.z;
+    S = p.num_splits;
+  }
 
   // q of this lane's query head (grp): entries 16kb + 4q + {0..3} of every
   // k16 block kb, loaded before anything else so that their latency overlaps
@@ -437,7 +777,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   // before the block exits; a page id outside the pool is never copied.
   const bool spec = p.window == 0;
   if (spec) {
-    const int tf = split * p.chunk_pages * (p.ps / kTileTokens);
+    const int tf = p.prop ? prop_j0 : split * p.chunk_pages * (p.ps / kTileTokens);
     int e = -1;
     if (lane < C::NS - 1) {
       const int tok = (tf + warp + C::NW * lane) * kTileTokens;
@@ -461,12 +801,18 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     L = 0;
   }
   const int lo = p.window > 0 ? max(0, L - p.window) : 0;
-  const int first_page = lo / p.ps;
-  const int n_pages = (L > lo) ? (L - 1) / p.ps - first_page + 1 : 0;
-  const int pg0 = first_page + split * p.chunk_pages;
-  const int pg1 = min(first_page + n_pages, pg0 + p.chunk_pages);
-  const int t0 = max(lo, pg0 * p.ps);
-  const int t1 = min(L, pg1 * p.ps);
+  int t0, t1;
+  if (p.prop) {
+    t0 = max(lo, (lo / kTileTokens + prop_j0) * kTileTokens);
+    t1 = min(L, (lo / kTileTokens + prop_j1) * kTileTokens);
+  } else {
+    const int first_page = lo / p.ps;
+    const int n_pages = (L > lo) ? (L - 1) / p.ps - first_page + 1 : 0;
+    const int pg0 = first_page + split * p.chunk_pages;
+    const int pg1 = min(first_page + n_pages, pg0 + p.chunk_pages);
+    t0 = max(lo, pg0 * p.ps);
+    t1 = min(L, pg1 * p.ps);
+  }
   const int tile_first = t0 / kTileTokens;
   const int n_tiles = (t1 > t0) ? (t1 + kTileTokens - 1) / kTileTokens - tile_first : 0;
   int my_tiles = (n_tiles > warp) ? (n_tiles - warp + C::NW - 1) / C::NW : 0;
@@ -593,41 +939,14 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   __syncwarp();
 
   // ---- per-warp pipeline over 16-token tiles --------------------------------
-  // Per-lane ldmatrix row offsets inside a tile. K (no transpose): matrix
-  // i = lane / 8 is rows (lane % 8) + 8 * (i % 2) at byte column 16 * (i / 2)
-  // of each 32-byte block; V (transposed): rows (lane % 8) + 8 * (i / 2) at
-  // byte column 16 * (i % 2). The swizzle makes the offset of 32-byte block kc
-  // depend on kc % 4 (D >= 128) or kc (D = 64), so four offsets per operand.
   uint32_t koff[4], voff[4];
-  {
-    const int i = lane >> 3;
-    const int rk = (lane & 7) + 8 * (i & 1), hk = i >> 1;
-    const int rv = (lane & 7) + 8 * (i >> 1), hv = i & 1;
-#pragma unroll
-    for (int kc = 0; kc < 4; ++kc) {
-      koff[kc] = tile_off<D>(rk, 32 * kc + 16 * hk);
-      voff[kc] = tile_off<D>(rv, 32 * kc + 16 * hv);
-    }
-  }
-  auto blk_off = [&](const uint32_t (&off)[4], int kc) -> uint32_t {
-    // 32-byte block kc: blocks 4.. of a 128-byte line group repeat the
-    // offsets of blocks 0..3 one 2048-byte column block further (D >= 128)
-    if constexpr (D == 64) return off[kc];
-    else return off[kc & 3] + (kc >> 2) * 2048;
+  ldsm_offsets<D>(lane, koff, voff);
+  auto qfr = [&](int kb) -> uint2 {
+    if constexpr (C::Q_IN_SMEM) return qfrag_s[kb * 32 + lane];
+    else return make_uint2(qf[kb][0], qf[kb][1]);
   };
-
-  float O[D / 32][2][4];
-#pragma unroll
-  for (int jb = 0; jb < D / 32; ++jb)
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) O[jb][h][c] = 0.f;
-  float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F;  // running max, heads 2qd / 2qd+1 (log2 units)
-  float l0 = 0.f, l1 = 0.f;                      // this lane's share of the running sums
-  // Running V reference scale: the largest |v_scale| seen so far. O holds
-  // sum P * v_scale / vref, so every f16 P operand stays <= 1 in magnitude.
-  float vref = 0.f, inv_vref = 0.f;
+  Acc<D> acc;
+  acc.reset();
   bool ok_all = true;
 
   int stage = 0;
@@ -656,155 +975,15 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       phase ^= 1;
     }
 
-    // -- S[token][head] = K q'^T (two independent accumulator chains) --------
-    float Sa[4] = {0.f, 0.f, 0.f, 0.f}, Sb[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int kc = 0; kc < D / 32; ++kc) {
-      // rows g / g+8, bytes 32kc + 4q.. (regs 0 / 1) and 32kc + 16 + 4q.. (2 / 3)
-      const uint4 kw = ldsm_x4(sk + blk_off(koff, kc));
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int kb = 2 * kc + half;
-        const uint32_t wa = half ? kw.z : kw.x, wb = half ? kw.w : kw.y;
-        uint32_t b0, b1;
-        if constexpr (C::Q_IN_SMEM) {
-          const uint2 f = qfrag_s[kb * 32 + lane];
-          b0 = f.x;
-          b1 = f.y;
-        } else {
-          b0 = qf[kb][0];
-          b1 = qf[kb][1];
-        }
-        uint32_t a0, a1, a2, a3;
-        if constexpr (KCVT) {
-          a0 = e4m3x2_lo16_to_f16x2(wa);
-          a1 = e4m3x2_lo16_to_f16x2(wb);
-          a2 = e4m3x2_hi16_to_f16x2(wa);
-          a3 = e4m3x2_hi16_to_f16x2(wb);
-        } else {
-          a0 = e4m3x2_b02_to_f16x2(wa);
-          a1 = e4m3x2_b02_to_f16x2(wb);
-          a2 = e4m3x2_b13_to_f16x2(wa);
-          a3 = e4m3x2_b13_to_f16x2(wb);
-        }
-        if (half)
-          mma16816(Sb, a0, a1, a2, a3, b0, b1);
-        else
-          mma16816(Sa, a0, a1, a2, a3, b0, b1);
-      }
-    }
-
-    // -- masked scores (log2 units), online softmax ------------------------
-    // A masked row may hold stale or NaN-decoded bytes: select, never multiply.
-    const int ta = tok0 + grp, tb = ta + 8;
-    const bool va = full || (page_ok && ta >= t0 && ta < t1);
-    const bool vb = full || (page_ok && tb >= t0 && tb < t1);
-    const float s00 = va ? (Sa[0] + Sb[0]) * kfac : -CUDART_INF_F;  // token grp,   head 2qd
-    const float s01 = va ? (Sa[1] + Sb[1]) * kfac : -CUDART_INF_F;  // token grp,   head 2qd+1
-    const float s10 = vb ? (Sa[2] + Sb[2]) * kfac : -CUDART_INF_F;  // token grp+8, head 2qd
-    const float s11 = vb ? (Sa[3] + Sb[3]) * kfac : -CUDART_INF_F;  // token grp+8, head 2qd+1
-    float tm0 = fmaxf(s00, s10), tm1 = fmaxf(s01, s11);
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, o));
-      tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, o));
-    }
-    const float mn0 = fmaxf(m0, tm0), mn1 = fmaxf(m1, tm1);
-    const float vabs = fabsf(vs);
-    const bool grow_v = vabs > vref;  // warp-uniform: one scale per tile
-    if (grow_v || __any_sync(0xffffffffu, (mn0 > m0) || (mn1 > m1))) {
-      const float c0 = (mn0 > m0) ? fast_exp2(m0 - mn0) : 1.f;  // exp2(-inf) = 0 for a first max
-      const float c1 = (mn1 > m1) ? fast_exp2(m1 - mn1) : 1.f;
-      const float fv = grow_v ? vref / vabs : 1.f;
-      l0 *= c0;
-      l1 *= c1;
-      const float o0 = c0 * fv, o1 = c1 * fv;
-#pragma unroll
-      for (int jb = 0; jb < D / 32; ++jb)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          O[jb][h][0] *= o0;
-          O[jb][h][1] *= o1;
-          O[jb][h][2] *= o0;
-          O[jb][h][3] *= o1;
-        }
-      m0 = mn0;
-      m1 = mn1;
-      if (grow_v) {
-        vref = vabs;
-        inv_vref = 1.f / vabs;
-      }
-    }
-    const float mb0 = (m0 == -CUDART_INF_F) ? 0.f : m0;
-    const float mb1 = (m1 == -CUDART_INF_F) ? 0.f : m1;
-    const float p00 = fast_exp2(s00 - mb0), p01 = fast_exp2(s01 - mb1);
-    const float p10 = fast_exp2(s10 - mb0), p11 = fast_exp2(s11 - mb1);
-    l0 += p00 + p10;
-    l1 += p01 + p11;
-
-    // -- P * v_scale / vref as f16 hi + lo; the B fragments of the PV MMA are
-    // the transposes of the score fragment's 8x8 blocks (movmatrix).
-    const float vsr = vs * inv_vref;
-    const float w00 = p00 * vsr, w01 = p01 * vsr, w10 = p10 * vsr, w11 = p11 * vsr;
-    const uint32_t ha = pack_f16x2(w00, w01), hb = pack_f16x2(w10, w11);
-    const float2 fa = unpack_f16x2(ha), fb = unpack_f16x2(hb);
-    const uint32_t la = pack_f16x2(w00 - fa.x, w01 - fa.y), lb = pack_f16x2(w10 - fb.x, w11 - fb.y);
-    const uint32_t bh0 = movmatrix_trans(ha), bh1 = movmatrix_trans(hb);  // tokens 2qd.., 2qd+8..
-    const uint32_t bl0 = movmatrix_trans(la), bl1 = movmatrix_trans(lb);
-
-    // -- O^T[d][head] += V^T P ---------------------------------------------
-    // ldmatrix.trans of the 32-byte block jb gives lane (g, q) the bytes
-    // (d, d+1), d = 32jb + 2g, of tokens 2q and 2q+1 (reg 0), the same for
-    // d + 16 (reg 1), and for tokens 2q+8, 2q+9 (regs 2, 3). M tile (jb, 0)
-    // rows g / g+8 are d / d+1; M tile (jb, 1) adds 16.
-    uint32_t vmask_lo = ~0u, vmask_hi = ~0u;
-    if (VCVT && !full) {
-      // with the hardware cvt a masked row must be zeroed (a NaN byte times
-      // P = 0 would still be NaN); bytes 0-1 / 2-3 are tokens 2q / 2q+1
-      const int r = tok0 + 2 * qd;
-      auto in = [&](int t) { return page_ok && t >= t0 && t < t1; };
-      vmask_lo = (in(r) ? 0x0000FFFFu : 0u) | (in(r + 1) ? 0xFFFF0000u : 0u);
-      vmask_hi = (in(r + 8) ? 0x0000FFFFu : 0u) | (in(r + 9) ? 0xFFFF0000u : 0u);
-    }
-#pragma unroll
-    for (int jb = 0; jb < D / 32; ++jb) {
-      const uint4 vw = ldsm_x4_trans(sv + blk_off(voff, jb));
-      uint32_t a0, a1, a2, a3, e0, e1, e2, e3;
-      if constexpr (VCVT) {
-        // [t.d, t'.d, t.d+1, t'.d+1]: each 16-bit half is one column's token pair
-        const uint32_t z0 = prmt(vw.x & vmask_lo, 0, 0x3120), z1 = prmt(vw.y & vmask_lo, 0, 0x3120);
-        const uint32_t z2 = prmt(vw.z & vmask_hi, 0, 0x3120), z3 = prmt(vw.w & vmask_hi, 0, 0x3120);
-        a0 = e4m3x2_lo16_to_f16x2(z0);
-        a1 = e4m3x2_hi16_to_f16x2(z0);
-        a2 = e4m3x2_lo16_to_f16x2(z2);
-        a3 = e4m3x2_hi16_to_f16x2(z2);
-        e0 = e4m3x2_lo16_to_f16x2(z1);
-        e1 = e4m3x2_hi16_to_f16x2(z1);
-        e2 = e4m3x2_lo16_to_f16x2(z3);
-        e3 = e4m3x2_hi16_to_f16x2(z3);
-      } else {
-        // [t.d, t.d+1, t'.d, t'.d+1]: bytes (0,2) and (1,3) are token pairs
-        a0 = e4m3x2_b02_to_f16x2(vw.x);
-        a1 = e4m3x2_b13_to_f16x2(vw.x);
-        a2 = e4m3x2_b02_to_f16x2(vw.z);
-        a3 = e4m3x2_b13_to_f16x2(vw.z);
-        e0 = e4m3x2_b02_to_f16x2(vw.y);
-        e1 = e4m3x2_b13_to_f16x2(vw.y);
-        e2 = e4m3x2_b02_to_f16x2(vw.w);
-        e3 = e4m3x2_b13_to_f16x2(vw.w);
-      }
-      mma16816(O[jb][0], a0, a1, a2, a3, bh0, bh1);
-      mma16816(O[jb][0], a0, a1, a2, a3, bl0, bl1);
-      mma16816(O[jb][1], e0, e1, e2, e3, bh0, bh1);
-      mma16816(O[jb][1], e0, e1, e2, e3, bl0, bl1);
-    }
+    attend_tile<D, KCVT, VCVT>(acc, qfr, sk, sv, koff, voff, kfac, vs, tok0, t0, t1, page_ok, full,
+                               grp, qd);
   }
   if (!ok_all) {
     // A copy never completed: leave this warp's result out (its flag is set)
     // and wait, again bounded, for whatever this warp still has in flight.
     for (int s = 0; s < C::NS; ++s) mbar_wait(wbar + 8 * s, phase ^ (s < stage ? 1u : 0u));
-    m0 = m1 = -CUDART_INF_F;
-    l0 = l1 = 0.f;
+    acc.m0 = acc.m1 = -CUDART_INF_F;
+    acc.l0 = acc.l1 = 0.f;
   }
 
   // speculative copies past this warp's last tile (first use of their stage)
@@ -814,35 +993,50 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   // ---- merge the warps ------------------------------------------------------
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    acc.l0 += __shfl_xor_sync(0xffffffffu, acc.l0, o);
+    acc.l1 += __shfl_xor_sync(0xffffffffu, acc.l1, o);
   }
   __syncthreads();  // every warp is done with its ring
   float* Os = reinterpret_cast<float*>(pipe);  // [NW][8][D], already times fold
   float* ml = misc;                            // [NW][8][2]
   // f16 offset of the decoded V (bit assembly only), times the V reference scale
-  const float fold = ok_all ? (VCVT ? 1.f : 256.f) * vref : 0.f;
+  const float fold = ok_all ? (VCVT ? 1.f : 256.f) * acc.vref : 0.f;
 #pragma unroll
   for (int jb = 0; jb < D / 32; ++jb) {
     const int d = 32 * jb + 2 * grp;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       *reinterpret_cast<float2*>(Os + (warp * 8 + 2 * qd) * D + d + 16 * h) =
-          make_float2(O[jb][h][0] * fold, O[jb][h][2] * fold);
+          make_float2(acc.O[jb][h][0] * fold, acc.O[jb][h][2] * fold);
       *reinterpret_cast<float2*>(Os + (warp * 8 + 2 * qd + 1) * D + d + 16 * h) =
-          make_float2(O[jb][h][1] * fold, O[jb][h][3] * fold);
+          make_float2(acc.O[jb][h][1] * fold, acc.O[jb][h][3] * fold);
     }
   }
   if (grp == 0) {
-    ml[(warp * 8 + 2 * qd) * 2 + 0] = m0;
-    ml[(warp * 8 + 2 * qd) * 2 + 1] = l0;
-    ml[(warp * 8 + 2 * qd + 1) * 2 + 0] = m1;
-    ml[(warp * 8 + 2 * qd + 1) * 2 + 1] = l1;
+    ml[(warp * 8 + 2 * qd) * 2 + 0] = acc.m0;
+    ml[(warp * 8 + 2 * qd) * 2 + 1] = acc.l0;
+    ml[(warp * 8 + 2 * qd + 1) * 2 + 0] = acc.m1;
+    ml[(warp * 8 + 2 * qd + 1) * 2 + 1] = acc.l1;
   }
   __syncthreads();
 
   constexpr float kLog2e = 1.4426950408889634f;
-  const int S = p.num_splits;
+  // Partial rows of this (sequence, KV head x head group): head n's rows are
+  // prow0 + n * S + s; its merge-group rows grow0 + n * NG + g; its tickets
+  // ucnt[0 .. NG] (NG = ceil(S / 8)). Proportional splits pack the units of
+  // sequence b after those of the sequences before it.
+  const int NG = (S + kMergeFan - 1) / kMergeFan;
+  const int HX = gridDim.x;
+  int64_t prow0, grow0, cnt0;
+  if (p.prop) {
+    prow0 = ((int64_t)sp_b * HX + (int64_t)blockIdx.x * S) * kHeadsPerGroup;
+    grow0 = ((int64_t)gp_b * HX + (int64_t)blockIdx.x * NG) * kHeadsPerGroup;
+    cnt0 = (int64_t)(b + gp_b) * HX + (int64_t)blockIdx.x * (1 + NG);
+  } else {
+    prow0 = ((int64_t)b * p.Hq + head0) * S;
+    grow0 = ((int64_t)b * p.Hq + head0) * NG;
+    cnt0 = ((int64_t)b * HX + blockIdx.x) * (1 + NG);
+  }
   for (int it = tid; it < 8 * (D / 4); it += 128) {
     const int n = it / (D / 4);
     const int d = (it - n * (D / 4)) * 4;
@@ -880,7 +1074,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       }
       *reinterpret_cast<float4*>(p.out + (int64_t)b * p.o_sb + (int64_t)head * p.o_sh + d) = r;
     } else {
-      const int64_t row = ((int64_t)b * p.Hq + head) * S + split;
+      const int64_t row = prow0 + (int64_t)n * S + split;
       *reinterpret_cast<float4*>(p.part_o + row * D + d) = acc;
       if (d == 0) *reinterpret_cast<float2*>(p.part_ml + row * 2) = make_float2(M, l);
     }
@@ -897,9 +1091,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   __threadfence();
   __syncthreads();
   int* flag = reinterpret_cast<int*>(misc + C::NW * 8 * 2);
-  const int NG = p.num_groups;
-  const int64_t unit = (int64_t)b * gridDim.x + blockIdx.x;
-  int* ucnt = p.counters + unit * (1 + NG);
+  int* ucnt = p.counters + cnt0;
   const int g = split / kMergeFan;
   const int gsize = min(kMergeFan, S - g * kMergeFan);
   if (tid == 0) *flag = (atomicAdd(ucnt + 1 + g, 1) == gsize - 1);
@@ -907,15 +1099,14 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   if (!*flag) return;
   __threadfence();
   float* wts = reinterpret_cast<float*>(pipe);  // [8][32] merge weights
-  const int64_t row_b = (int64_t)b * p.Hq + head0;
   if (NG == 1) {
-    merge_partials<D, C::NW>(p.part_ml, p.part_o, row_b * S, S, S, nheads, true, p, b, head0,
+    merge_partials<D, C::NW>(p.part_ml, p.part_o, prow0, S, S, nheads, true, p, b, head0,
                              nullptr, nullptr, 0, 0, wts);
     if (tid == 0) ucnt[1] = 0;
     return;
   }
-  merge_partials<D, C::NW>(p.part_ml, p.part_o, row_b * S + g * kMergeFan, S, gsize, nheads, false,
-                           p, b, head0, p.grp_ml, p.grp_o, row_b * NG + g, NG, wts);
+  merge_partials<D, C::NW>(p.part_ml, p.part_o, prow0 + g * kMergeFan, S, gsize, nheads, false,
+                           p, b, head0, p.grp_ml, p.grp_o, grow0 + g, NG, wts);
   if (tid == 0) ucnt[1 + g] = 0;
   __threadfence();
   __syncthreads();
@@ -923,9 +1114,558 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   __syncthreads();
   if (!*flag) return;
   __threadfence();
-  merge_partials<D, C::NW>(p.grp_ml, p.grp_o, row_b * NG, NG, NG, nheads, true, p, b, head0,
+  merge_partials<D, C::NW>(p.grp_ml, p.grp_o, grow0, NG, NG, nheads, true, p, b, head0,
                            nullptr, nullptr, 0, 0, wts);
   if (tid == 0) ucnt[0] = 0;
+}
+
+// ---------------------------------------------------------------------------
+// Balanced schedule.
+//
+// The split kernel gives every block an equal share of one sequence's pages,
+// so with uneven lengths some blocks run several times longer than others
+// and the last wave leaves most SMs idle. Here the work is the flat list of
+// the 16-token tile columns of all sequences (column (b, j) = tile j of
+// sequence b's attended range, for every KV head x head group unit x < HX).
+// The grid is one full wave of blocks; its warps form NG groups of HX
+// consecutive warps, and warp x of group g takes columns
+// [floor(g T / NG), floor((g+1) T / NG)) of unit x (T = all columns): every
+// warp streams the same number of tiles (+-1), and the HX warps of a group,
+// which sit in the same or neighbouring blocks, read the same pages at the
+// same time, so a page's KV heads leave DRAM together. Each block derives
+// the partition from the lengths itself (prefix sums in shared memory), so
+// the call stays one launch.
+//
+// A warp's columns cross sequence boundaries; each (sequence, group) piece
+// is a segment. A sequence that lies inside one group is written straight
+// to `out`. Otherwise every segment writes a partial (m, l, O) to slot
+// (b + g) HX + x (unique: along the partition b and g never both decrease),
+// the segments of groups [8W, 8W+8) take tickets of counter (b + W) HX + x
+// and the last merges them; with several such groups the group mergers take
+// the unit's ticket and the last one merges the group partials (slot
+// (b + W) HX + x), adding the sink once. No warp ever waits for another.
+// ---------------------------------------------------------------------------
+#ifndef FP8PD_FLAT_MIN_BLOCKS_D128
+#define FP8PD_FLAT_MIN_BLOCKS_D128 3
+#endif
+#ifndef FP8PD_FLAT_NS_D128
+#define FP8PD_FLAT_NS_D128 3
+#endif
+#ifndef FP8PD_FLAT_NS_D64
+#define FP8PD_FLAT_NS_D64 6
+#endif
+
+template <int D>
+struct FlatCfg {
+  static_assert(D == 64 || D == 128, "the balanced kernel keeps q in registers (D <= 128)");
+  static constexpr int NW = kFlatWarps;
+  static constexpr int NS = (D == 64) ? FP8PD_FLAT_NS_D64 : FP8PD_FLAT_NS_D128;
+  static constexpr int TILE = kTileTokens * D;
+  static constexpr int STAGE = 2 * TILE;
+  static constexpr int WARP_BYTES = NS * STAGE;
+  static constexpr int PIPE_BYTES = NW * WARP_BYTES;
+  static constexpr int BAR_BYTES = NW * NS * 8;
+  static constexpr int MISC_BYTES = 64;  // block-scan partial sums
+  static constexpr int MIN_BLOCKS = (D == 64) ? 4 : FP8PD_FLAT_MIN_BLOCKS_D128;
+  static_assert(PIPE_BYTES % 1024 == 0, "tiles must stay 1024-byte aligned for the swizzle");
+  // dynamic shared memory for B sequences: lengths [B] and prefix [B + 1]
+  static constexpr int smem(int B) { return 1024 + PIPE_BYTES + BAR_BYTES + MISC_BYTES + 8 * (B + 1); }
+};
+
+// The group (of ng) whose column range holds column t: the largest g with
+// floor(g T / ng) <= t.
+__device__ __forceinline__ int flat_group_of(int64_t t, int64_t T, int ng) {
+  return static_cast<int>(((t + 1) * ng - 1) / T);
+}
+
+// Tiles of a sequence with L attended keys: 16-token tiles (absolute token
+// positions) that overlap [lo, L).
+__device__ __forceinline__ int flat_tiles(int L, int window) {
+  const int lo = window > 0 ? max(0, L - window) : 0;
+  return L > lo ? (L - 1) / kTileTokens - lo / kTileTokens + 1 : 0;
+}
+
+// One warp merges K partial slots slot0 + k * stride, k < K (hpu heads each;
+// (m, l) in log2 units, O already multiplied out) for the unit's nheads
+// heads. `final`: the sink of each head enters the denominator once and the
+// result goes to out[b, head0 + n]; otherwise (M, L, O) goes to slot
+// dst_slot of (dst_ml, dst_o). All heads move together: each partial is one
+// round of up to 16 independent loads per lane (lane l holds entries
+// PER*l .. PER*l + PER-1 of every head).
+template <int D>
+__device__ __noinline__ void flat_merge(const float* ml, const float* o, int64_t slot0, int64_t stride, int K,
+                           int nheads, bool final, const DecodeParams& p, int b, int head0,
+                           float* dst_ml, float* dst_o, int64_t dst_slot) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  constexpr int PER = D / 32;  // output entries per lane and head
+  constexpr int H = kHeadsPerGroup;
+  const int lane = threadIdx.x & 31;
+  const int64_t hpu = p.hpu;
+  float M[H];
+#pragma unroll
+  for (int h = 0; h < H; ++h) M[h] = -CUDART_INF_F;
+  for (int k = lane; k < K; k += 32) {
+    const float* row = ml + (slot0 + k * stride) * hpu * 2;
+#pragma unroll
+    for (int h = 0; h < H; ++h)
+      if (h < nheads) M[h] = fmaxf(M[h], ldcg2(row + 2 * h).x);
+  }
+#pragma unroll
+  for (int h = 0; h < H; ++h) {
+    M[h] = warp_max(M[h]);
+    if (final && p.sinks && h < nheads)
+      M[h] = fmaxf(M[h], p.sinks[(int64_t)(head0 + h) * p.sinks_s] * kLog2e);  // M2: sink included
+  }
+  float acc[H][PER], L[H];
+#pragma unroll
+  for (int h = 0; h < H; ++h) {
+    L[h] = 0.f;
+#pragma unroll
+    for (int c = 0; c < PER; ++c) acc[h][c] = 0.f;
+  }
+#pragma unroll 1
+  for (int k = 0; k < K; ++k) {
+    const int64_t s = slot0 + k * stride;
+    float2 mk[H];
+    float v[H][PER];
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+      if (h < nheads) {
+        mk[h] = ldcg2(ml + (s * hpu + h) * 2);
+        const float* src = o + (s * hpu + h) * D + lane * PER;
+        if constexpr (PER == 4) {
+          const float4 x = ldcg4(src);
+          v[h][0] = x.x; v[h][1] = x.y; v[h][2] = x.z; v[h][3] = x.w;
+        } else {
+          const float2 x = ldcg2(src);
+          v[h][0] = x.x; v[h][1] = x.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+      if (h < nheads) {
+        const float wk = (M[h] == -CUDART_INF_F || mk[h].x == -CUDART_INF_F) ? 0.f
+                                                                             : fast_exp2(mk[h].x - M[h]);
+        L[h] += wk * mk[h].y;
+#pragma unroll
+        for (int c = 0; c < PER; ++c) acc[h][c] += wk * v[h][c];
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < H; ++h) {
+    if (h >= nheads) continue;
+    if (final) {
+      const float sl = p.sinks ? p.sinks[(int64_t)(head0 + h) * p.sinks_s] * kLog2e : -CUDART_INF_F;
+      const float den = L[h] + ((p.sinks && M[h] != -CUDART_INF_F) ? fast_exp2(sl - M[h]) : 0.f);
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      float* dst = p.out + (int64_t)b * p.o_sb + (int64_t)(head0 + h) * p.o_sh + lane * PER;
+      if constexpr (PER == 4)
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[h][0] * inv, acc[h][1] * inv,
+                                                      acc[h][2] * inv, acc[h][3] * inv);
+      else
+        *reinterpret_cast<float2*>(dst) = make_float2(acc[h][0] * inv, acc[h][1] * inv);
+    } else {
+      const int64_t row = dst_slot * hpu + h;
+      if (lane == 0) *reinterpret_cast<float2*>(dst_ml + row * 2) = make_float2(M[h], L[h]);
+      float* dst = dst_o + row * D + lane * PER;
+      if constexpr (PER == 4)
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+      else
+        *reinterpret_cast<float2*>(dst) = make_float2(acc[h][0], acc[h][1]);
+    }
+  }
+}
+
+// The balanced kernel (see above). Grid: one wave of blocks of 4 warps;
+// dynamic shared memory FlatCfg<D>::smem(B). KCVT / VCVT as for the split
+// kernel.
+template <int D, bool KCVT, bool VCVT>
+__global__ void __launch_bounds__(128, FlatCfg<D>::MIN_BLOCKS)
+    decode_flat_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
+                       const __grid_constant__ CUtensorMap tmv) {
+  using C = FlatCfg<D>;
+  constexpr int KB = D / 16;
+  constexpr unsigned FULL = 0xffffffffu;
+  constexpr float kLog2e = 1.4426950408889634f;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + C::PIPE_BYTES);
+  int* s_misc = reinterpret_cast<int*>(smem + C::PIPE_BYTES + C::BAR_BYTES);
+  int* s_len = s_misc + C::MISC_BYTES / 4;  // [B] attended keys (0 when out of range)
+  int* s_pre = s_len + p.B;                 // [B + 1] tile columns of sequences < b
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31, grp = lane >> 2, qd = lane & 3;
+  const int B = p.B, HX = p.Hkv * p.head_groups;
+
+  const uint32_t wbar = smem_u32(s_bar + warp * C::NS);
+  const uint32_t wpipe = smem_u32(smem + warp * C::WARP_BYTES);
+  if (lane == 0) {
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+#pragma unroll
+    for (int s = 0; s < C::NS; ++s) mbar_init(wbar + 8 * s, 1);
+    fence_barrier_init();
+    fence_proxy_async();
+  }
+
+  // ---- lengths and the prefix of tile columns over sequences ---------------
+  for (int b = tid; b < B; b += 128) {
+    int L = __ldg(p.lens + (int64_t)b * p.lens_s);
+    if (L < 0 || L > p.max_pages * p.ps) {
+      if (blockIdx.x == 0) raise_flag(FP8PD_FLAG_SEQLEN_OOB);
+      L = 0;
+    }
+    s_len[b] = L;
+  }
+  __syncthreads();
+  {
+    const int per = (B + 127) >> 7;
+    const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
+    int sum = 0;
+    for (int b = b0; b < b1; ++b) sum += flat_tiles(s_len[b], p.window);
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(FULL, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_misc[warp] = incl;
+    __syncthreads();
+    int off = incl - sum;
+    for (int ww = 0; ww < warp; ++ww) off += s_misc[ww];
+    for (int b = b0; b < b1; ++b) {
+      s_pre[b] = off;
+      off += flat_tiles(s_len[b], p.window);
+    }
+    if (tid == 127) s_pre[B] = off;
+  }
+  __syncthreads();  // no block-wide barrier after this point
+
+  const int T = s_pre[B];
+  const int NWT = gridDim.x * C::NW;
+  const int ng = min(NWT / HX, T);  // warp groups with work
+  const int w = blockIdx.x * C::NW + warp;
+  const int g = w / HX, x = w - g * HX;
+
+  // units without tiles: their outputs are 0
+  for (int u = w; u < B * HX; u += NWT) {
+    const int b = u / HX;
+    if (s_pre[b + 1] != s_pre[b]) continue;
+    const int xx = u - b * HX, kvh = xx / p.head_groups, hgi = xx - kvh * p.head_groups;
+    const int head0 = kvh * p.G + hgi * 8, nh = min(8, p.G - hgi * 8);
+    for (int e = lane; e < nh * D; e += 32)
+      p.out[(int64_t)b * p.o_sb + (int64_t)(head0 + e / D) * p.o_sh + (e % D)] = 0.f;
+  }
+  if (g >= ng) return;
+
+  const int kvh = x / p.head_groups, hgi = x - kvh * p.head_groups;
+  const int head0 = kvh * p.G + hgi * 8, nheads = min(8, p.G - hgi * 8);
+  const int c0 = static_cast<int>((int64_t)g * T / ng);
+  const int n = static_cast<int>((int64_t)(g + 1) * T / ng) - c0;
+
+  // ---- this warp's tiles, 32 at a time, one per lane ------------------------
+  // Three chunks are in flight so that no global load is waited for in the
+  // streaming loop: the current chunk (entry = page << 4 | 16-token tile
+  // inside the page, or -1 for a page id outside the pool; sequence; k and v
+  // scale), the next one (the same, its scales still arriving), and the one
+  // after (its block-table entries still arriving). `locate` finds the
+  // sequence and token of tile base + lane and starts its table read;
+  // `resolve` turns that into the entry and starts the scale reads.
+  auto locate = [&](int base, int& page, int& bb, int& tok) {
+    page = -1;
+    bb = 0;
+    tok = -1;
+    const int i = base + lane;
+    if (i >= n) return;
+    const int t = c0 + i;
+    int lo = 0, hi = B;  // the last sequence b with s_pre[b] <= t
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_pre[mid] <= t) lo = mid;
+      else hi = mid;
+    }
+    const int L = s_len[lo];
+    const int lo_tok = p.window > 0 ? max(0, L - p.window) : 0;
+    bb = lo;
+    tok = (lo_tok / kTileTokens + t - s_pre[lo]) * kTileTokens;
+    page = __ldg(p.table + (int64_t)lo * p.tab_sb + (int64_t)(tok / p.ps) * p.tab_sp);
+  };
+  auto resolve = [&](int page, int tok, int& e, float& ks, float& vs) {
+    e = -1;
+    ks = vs = 0.f;
+    if (tok < 0) return;
+    if ((unsigned)page < (unsigned)p.num_pages) {
+      e = (page << 4) | ((tok % p.ps) / kTileTokens);
+      ks = __ldg(p.ks + (int64_t)page * p.ks_sp + (int64_t)kvh * p.ks_sh);
+      vs = __ldg(p.vs + (int64_t)page * p.vs_sp + (int64_t)kvh * p.vs_sh);
+    } else if (hgi == 0) {
+      raise_flag(FP8PD_FLAG_PAGE_OOB);
+    }
+  };
+  int ce, cu, ne, nu, pp, pu, ptok;
+  float cks, cvs, nks, nvs;
+  {
+    int page, tok;
+    locate(0, page, cu, tok);
+    locate(32, pp, nu, ptok);
+    resolve(page, tok, ce, cks, cvs);
+    resolve(pp, ptok, ne, nks, nvs);
+    locate(64, pp, pu, ptok);
+  }
+  int base = 0;
+
+  // Lane 0 copies tile i into ring stage `stage` (all lanes call).
+  int issued = 0;
+  auto issue = [&](int i, int stage) {
+    const int k = i - base;
+    const int e = __shfl_sync(FULL, k < 32 ? ce : ne, k & 31);
+    ++issued;
+    if (lane != 0) return;
+    const uint32_t bar = wbar + 8 * stage;
+    if (e < 0) {
+      mbar_arrive(bar);
+      return;
+    }
+    const int page = e >> 4, slot0 = (e & 15) * kTileTokens;
+    const uint32_t sk = wpipe + stage * C::STAGE;
+    fence_proxy_async();
+    mbar_arrive_expect_tx(bar, 2 * C::TILE);
+    tma_load_5d(sk, &tmk, bar, 0, slot0, 0, kvh, page);
+    tma_load_5d(sk + C::TILE, &tmv, bar, 0, slot0, 0, kvh, page);
+  };
+#pragma unroll 1
+  for (int s = 0; s < C::NS - 1; ++s)
+    if (s < n) issue(s, s);
+
+  uint32_t koff[4], voff[4];
+  ldsm_offsets<D>(lane, koff, voff);
+  Acc<D> acc;
+  uint32_t qf[KB][2] = {};
+  auto qfr = [&](int kb) -> uint2 { return make_uint2(qf[kb][0], qf[kb][1]); };
+
+  // q of query head head0 + grp of sequence bb, bf16 pairs (entries
+  // 16kb + 4q .. 16kb + 4q + 3 of lane quad q); the next segment's q is read
+  // while the current one streams.
+  const bool q_ok = grp < nheads;
+  auto load_q = [&](int bb, uint2 (&dst)[KB]) {
+    const uint16_t* qrow = p.q + (int64_t)bb * p.q_sb + (int64_t)(head0 + (q_ok ? grp : 0)) * p.q_sh;
+#pragma unroll
+    for (int kb = 0; kb < KB; ++kb) {
+      const int d = 16 * kb + 4 * qd;
+      uint2 v = make_uint2(0u, 0u);
+      if (q_ok) {
+        if (p.q_vec) {
+          v = __ldg(reinterpret_cast<const uint2*>(qrow + d));
+        } else {
+          const uint32_t e0 = __ldg(qrow + (int64_t)(d + 0) * p.q_sd);
+          const uint32_t e1 = __ldg(qrow + (int64_t)(d + 1) * p.q_sd);
+          const uint32_t e2 = __ldg(qrow + (int64_t)(d + 2) * p.q_sd);
+          const uint32_t e3 = __ldg(qrow + (int64_t)(d + 3) * p.q_sd);
+          v = make_uint2(e0 | (e1 << 16), e2 | (e3 << 16));
+        }
+      }
+      dst[kb] = v;
+    }
+  };
+  uint2 qn[KB];
+  int qn_b = -1;
+
+  int stage = 0, consumed = 0;
+  uint32_t phase = 0;
+  bool ok_all = true;
+  int i = 0;
+#pragma unroll 1
+  while (i < n) {
+    // ---- segment: the sequence of tile i, up to its last tile in this warp --
+    const int b = __shfl_sync(FULL, cu, i - base);
+    const int u = b * HX + x;
+    const int L = s_len[b];
+    const int lo_tok = p.window > 0 ? max(0, L - p.window) : 0;
+    const int nb = s_pre[b + 1] - s_pre[b];
+    const int j0 = c0 + i - s_pre[b];
+    const int i_end = min(n, i + nb - j0);
+
+    // q of query head head0 + grp as f16 B-fragments, times 2^(15 - e) so
+    // that max|q'| lies in [2^14, 2^15) (the split kernel's q handling)
+    float score_base;
+    {
+      uint2 qraw[KB];
+      if (qn_b == b) {
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb) qraw[kb] = qn[kb];
+      } else {
+        load_q(b, qraw);
+      }
+      if (i_end < n) {  // the next sequence with tiles starts this warp's next segment
+        int nx = b + 1;
+        while (nx < B - 1 && s_pre[nx + 1] == s_pre[nx]) ++nx;
+        load_q(nx, qn);
+        qn_b = nx;
+      }
+      float qmax = 0.f;
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb) {
+        const uint2 v = qraw[kb];
+        qmax = fmaxf(qmax, fmaxf(fmaxf(fabsf(__uint_as_float(v.x << 16)),
+                                       fabsf(__uint_as_float(v.x & 0xFFFF0000u))),
+                                 fmaxf(fabsf(__uint_as_float(v.y << 16)),
+                                       fabsf(__uint_as_float(v.y & 0xFFFF0000u)))));
+      }
+      qmax = warp_max(qmax);
+      int qe = 0;
+      if (qmax > 0.f && isfinite(qmax)) frexpf(qmax, &qe);
+      qe = max(qe, -111);
+      const float qmul = ldexpf(1.f, 15 - qe);
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb) {
+        const uint2 v = qraw[kb];
+        const float x0 = __uint_as_float(v.x << 16), x1 = __uint_as_float(v.x & 0xFFFF0000u);
+        const float x2 = __uint_as_float(v.y << 16), x3 = __uint_as_float(v.y & 0xFFFF0000u);
+        if constexpr (KCVT) {
+          qf[kb][0] = pack_f16x2(x0 * qmul, x1 * qmul);
+          qf[kb][1] = pack_f16x2(x2 * qmul, x3 * qmul);
+        } else {
+          qf[kb][0] = pack_f16x2(x0 * qmul, x2 * qmul);
+          qf[kb][1] = pack_f16x2(x1 * qmul, x3 * qmul);
+        }
+      }
+      score_base = p.sm_scale_log2 * (KCVT ? 1.f : 256.f) / qmul;
+    }
+    acc.reset();
+
+    int tok0 = (lo_tok / kTileTokens + j0) * kTileTokens;
+#pragma unroll 1
+    for (; i < i_end; ++i, tok0 += kTileTokens) {
+      if (ok_all && !mbar_wait(wbar + 8 * stage, phase)) {
+        if (lane == 0) raise_flag(FP8PD_FLAG_TIMEOUT);
+        ok_all = false;
+      }
+      if (ok_all) {
+        __syncwarp();
+        ++consumed;
+        const int nj = i + C::NS - 1;
+        if (nj < n) issue(nj, stage == 0 ? C::NS - 1 : stage - 1);
+        const int k = i - base;
+        const int e = __shfl_sync(FULL, ce, k);
+        const float ks = __shfl_sync(FULL, cks, k), vs = __shfl_sync(FULL, cvs, k);
+        const bool page_ok = e >= 0;
+        const bool full = page_ok && tok0 >= lo_tok && tok0 + kTileTokens <= L;
+        const uint32_t sk = wpipe + stage * C::STAGE;
+        if (++stage == C::NS) {
+          stage = 0;
+          phase ^= 1;
+        }
+        attend_tile<D, KCVT, VCVT>(acc, qfr, sk, sk + C::TILE, koff, voff, score_base * ks, vs,
+                                   tok0, lo_tok, L, page_ok, full, grp, qd);
+      }
+      if (i + 1 - base == 32) {  // the chunks move up by one
+        base += 32;
+        ce = ne;
+        cu = nu;
+        cks = nks;
+        cvs = nvs;
+        nu = pu;
+        resolve(pp, ptok, ne, nks, nvs);
+        locate(base + 64, pp, pu, ptok);
+      }
+    }
+
+    // ---- segment result --------------------------------------------------
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      acc.l0 += __shfl_xor_sync(FULL, acc.l0, o);
+      acc.l1 += __shfl_xor_sync(FULL, acc.l1, o);
+    }
+    if (!ok_all) {
+      acc.m0 = acc.m1 = -CUDART_INF_F;
+      acc.l0 = acc.l1 = 0.f;
+    }
+    const float fold = ok_all ? (VCVT ? 1.f : 256.f) * acc.vref : 0.f;
+    const int gu0 = flat_group_of(s_pre[b], T, ng), gu1 = flat_group_of(s_pre[b] + nb - 1, T, ng);
+    const int h0 = 2 * qd, h1 = 2 * qd + 1;  // this lane's heads
+    float f0 = fold, f1 = fold;
+    float* dst0;
+    float* dst1;
+    if (gu0 == gu1) {
+      // the whole unit is in this warp: numerator / denominator straight to out
+      auto scale_of = [&](int h, float m, float l) -> float {
+        if (h >= nheads) return 0.f;
+        const float sl = p.sinks ? p.sinks[(int64_t)(head0 + h) * p.sinks_s] * kLog2e : -CUDART_INF_F;
+        const float M2 = fmaxf(m, sl);
+        if (M2 == -CUDART_INF_F) return 0.f;
+        const float a = (m == -CUDART_INF_F) ? 0.f : fast_exp2(m - M2);
+        const float den = l * a + (p.sinks ? fast_exp2(sl - M2) : 0.f);
+        return den > 0.f ? a / den : 0.f;
+      };
+      f0 *= scale_of(h0, acc.m0, acc.l0);
+      f1 *= scale_of(h1, acc.m1, acc.l1);
+      dst0 = p.out + (int64_t)b * p.o_sb + (int64_t)(head0 + h0) * p.o_sh;
+      dst1 = p.out + (int64_t)b * p.o_sb + (int64_t)(head0 + h1) * p.o_sh;
+    } else {
+      const int64_t slot = (int64_t)(b + g) * HX + x;
+      dst0 = p.part_o + (slot * p.hpu + h0) * D;
+      dst1 = p.part_o + (slot * p.hpu + h1) * D;
+      if (grp == 0) {
+        if (h0 < nheads) *reinterpret_cast<float2*>(p.part_ml + (slot * p.hpu + h0) * 2) = make_float2(acc.m0, acc.l0);
+        if (h1 < nheads) *reinterpret_cast<float2*>(p.part_ml + (slot * p.hpu + h1) * 2) = make_float2(acc.m1, acc.l1);
+      }
+    }
+#pragma unroll
+    for (int jb = 0; jb < D / 32; ++jb) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int d = 32 * jb + 2 * grp + 16 * hh;
+        if (h0 < nheads)
+          *reinterpret_cast<float2*>(dst0 + d) = make_float2(acc.O[jb][hh][0] * f0, acc.O[jb][hh][2] * f0);
+        if (h1 < nheads)
+          *reinterpret_cast<float2*>(dst1 + d) = make_float2(acc.O[jb][hh][1] * f1, acc.O[jb][hh][3] * f1);
+      }
+    }
+    if (gu0 != gu1) {
+      // level 1: the segments of groups [8W, 8W + 8) of this unit
+      __threadfence();
+      __syncwarp();
+      const int W1 = g / kFlatFan;
+      const int ga = max(gu0, W1 * kFlatFan), gb = min(gu1, W1 * kFlatFan + kFlatFan - 1);
+      const int64_t c1 = (int64_t)(b + W1) * HX + x;
+      int last = 0;
+      if (lane == 0) last = atomicAdd(p.counters + c1, 1) == gb - ga;
+      last = __shfl_sync(FULL, last, 0);
+      if (last) {
+        __threadfence();
+        const bool one_group = (gu0 / kFlatFan) == (gu1 / kFlatFan);
+        flat_merge<D>(p.part_ml, p.part_o, (int64_t)(b + ga) * HX + x, HX, gb - ga + 1, nheads,
+                      one_group, p, b, head0, p.grp_ml, p.grp_o, c1);
+        if (lane == 0) p.counters[c1] = 0;
+        if (!one_group) {
+          // level 2: the unit's groups
+          __threadfence();
+          __syncwarp();
+          const int W0 = gu0 / kFlatFan, nw = gu1 / kFlatFan - W0 + 1;
+          int* ucnt = p.counters + p.c1_count + u;
+          if (lane == 0) last = atomicAdd(ucnt, 1) == nw - 1;
+          last = __shfl_sync(FULL, last, 0);
+          if (last) {
+            __threadfence();
+            flat_merge<D>(p.grp_ml, p.grp_o, (int64_t)(b + W0) * HX + x, HX, nw, nheads, true, p,
+                          b, head0, nullptr, nullptr, 0);
+            if (lane == 0) *ucnt = 0;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  }
+
+  // A copy that never completed: wait, bounded, for this warp's copies still
+  // in flight before the block's shared memory goes away.
+  if (!ok_all) {
+    for (int c = consumed; c < issued; ++c)
+      mbar_wait(wbar + 8 * (c % C::NS), static_cast<uint32_t>((c / C::NS) & 1));
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -1002,7 +1742,8 @@ static cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap& tmk
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  const dim3 grid(p.Hkv * p.head_groups, p.B, p.num_splits);
+  const dim3 grid = p.prop ? dim3(p.Hkv * p.head_groups, p.nbx, 1)
+                           : dim3(p.Hkv * p.head_groups, p.B, p.num_splits);
   decode_tma_kernel<D, KCVT, VCVT><<<grid, 128, smem, s>>>(p, tmk, tmv);
   return cudaGetLastError();
 }
@@ -1025,6 +1766,80 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmk, const C
     case 256: return launch_decode_kv<256>(p, tmk, tmv, k_cvt, v_cvt, s);
     case 512: return launch_decode_kv<512>(p, tmk, tmv, k_cvt, v_cvt, s);
     default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int D, bool KCVT, bool VCVT>
+static cudaError_t launch_flat_d(const DecodeParams& p, const CUtensorMap& tmk,
+                                 const CUtensorMap& tmv, int blocks, cudaStream_t s) {
+  // the largest dynamic shared memory this kernel is launched with (the
+  // longest batch), set once per device like the split kernel's
+  static std::atomic<uint64_t> configured{0};
+  const int smem = FlatCfg<D>::smem(kFlatMaxBatch);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
+  if (!bit || !(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(decode_flat_kernel<D, KCVT, VCVT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  decode_flat_kernel<D, KCVT, VCVT><<<blocks, 128, FlatCfg<D>::smem(p.B), s>>>(p, tmk, tmv);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_flat_kv(const DecodeParams& p, const CUtensorMap& tmk,
+                                  const CUtensorMap& tmv, bool k_cvt, bool v_cvt, int blocks,
+                                  cudaStream_t s) {
+  if (k_cvt)
+    return v_cvt ? launch_flat_d<D, true, true>(p, tmk, tmv, blocks, s)
+                 : launch_flat_d<D, true, false>(p, tmk, tmv, blocks, s);
+  return v_cvt ? launch_flat_d<D, false, true>(p, tmk, tmv, blocks, s)
+               : launch_flat_d<D, false, false>(p, tmk, tmv, blocks, s);
+}
+
+cudaError_t launch_decode_flat(const DecodeParams& p, const CUtensorMap& tmk,
+                               const CUtensorMap& tmv, bool k_cvt, bool v_cvt, int blocks,
+                               cudaStream_t s) {
+  if (p.B > kFlatMaxBatch) return cudaErrorInvalidValue;
+  switch (p.D) {
+    case 64: return launch_flat_kv<64>(p, tmk, tmv, k_cvt, v_cvt, blocks, s);
+    case 128: return launch_flat_kv<128>(p, tmk, tmv, k_cvt, v_cvt, blocks, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Blocks per SM for batches of up to 128 * k sequences (shared memory grows
+// with the batch), cached per bucket k.
+template <int D>
+static int flat_blocks_per_sm_d(int B) {
+  static std::atomic<int> cached[kFlatMaxBatch / 128 + 1];  // 0 = not known yet
+  const int k = (B + 127) / 128;
+  int c = cached[k].load();
+  if (c > 0) return c;
+  int n = 0;
+  if (cudaFuncSetAttribute(decode_flat_kernel<D, true, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           FlatCfg<D>::smem(kFlatMaxBatch)) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_flat_kernel<D, true, true>, 128,
+                                                    FlatCfg<D>::smem(128 * k)) != cudaSuccess) {
+    cudaGetLastError();
+    return FlatCfg<D>::MIN_BLOCKS;  // no device: do not cache the guess
+  }
+  c = n > 0 ? n : 1;
+  cached[k].store(c);
+  return c;
+}
+
+int flat_blocks_per_sm(int D, int B) {
+  if (B < 0 || B > kFlatMaxBatch) return 1;
+  switch (D) {
+    case 64: return flat_blocks_per_sm_d<64>(B);
+    case 128: return flat_blocks_per_sm_d<128>(B);
+    default: return 1;
   }
 }
 

@@ -151,9 +151,15 @@ enum {
  *   sm_scale     finite, > 0.
  *   out          float32 [B, Hq, D]; stride[2] must be 1, rows 16-byte aligned.
  *   stream       CUDA stream.
- * Launches one kernel. When the planner splits the keys of a sequence over
- * several thread blocks, the last block of each (sequence, KV head) merges
- * the splits. The split partials and the blocks' ticket counters live
+ * Launches one kernel, with one of two schedules. The split kernel gives
+ * each (sequence, KV head, head group) one or more blocks, each an equal
+ * share of its pages; the last block of each to finish merges the splits.
+ * The balanced kernel (head dims 64 and 128, up to 1,024 sequences) gives
+ * every warp of one full wave of blocks the same number of 16-token tiles of
+ * all sequences together, whatever their lengths; the last warp of each
+ * group of pieces of a (sequence, KV head, head group) merges them. The
+ * planner takes the balanced kernel for long or uneven batches without a
+ * short window. The partial results and the ticket counters live
  * in a library-owned per-device workspace: it grows on demand outside stream
  * capture; under capture a call that would need to grow it fails with
  * FP8PD_ERR_CAPTURE_WORKSPACE (call fp8pd_reserve_workspace, or run the call
@@ -222,11 +228,14 @@ int fp8_paged_decode_attention_noalloc(const fp8pd_tensor* q, const fp8pd_tensor
 
 /* What a call with these arguments would launch, without launching it. */
 typedef struct fp8pd_plan_info {
-  int32_t num_splits;        /* thread blocks per (sequence, KV head, head group) */
+  int32_t num_splits;        /* split kernel: blocks per (sequence, KV head, head group);
+                                balanced kernel: 0 */
   int32_t head_groups;       /* ceil(G / 8) query-head groups per KV head */
-  int32_t grid_blocks;       /* split-kernel thread blocks */
-  int32_t combine;           /* 1 if the keys are split (the last block merges the splits) */
-  uint64_t workspace_bytes;  /* split workspace the call needs (0 if not split) */
+  int32_t grid_blocks;       /* thread blocks of the launch */
+  int32_t combine;           /* 1 if partial results are merged (workspace used) */
+  uint64_t workspace_bytes;  /* split workspace the call needs (0 if none) */
+  int32_t schedule;          /* 1 = split kernel, 2 = balanced kernel */
+  int32_t warps;             /* balanced kernel: warps sharing the tiles (else 0) */
 } fp8pd_plan_info;
 
 /* Plans a decode-attention call (same argument rules; nothing launched). */
@@ -246,8 +255,9 @@ enum {
   FP8PD_OPT_NUM_SPLITS = 1,  /* 0 = planner chooses (default); n > 0 asks for n splits (raised
                                 so that no split covers more than 8,192 keys, capped at 256
                                 splits and at the number of pages) */
-  FP8PD_OPT_VARIANT = 2,     /* 0 = auto; 1 = tensor-core (mma) split kernel;
-                                2 = CUDA-core (f32 FMA) split kernel */
+  FP8PD_OPT_SCHEDULE = 2,    /* 0 = planner chooses (default); 1 = split kernel; 2 = balanced
+                                kernel where it applies (D <= 128, B <= 1024, no forced split
+                                count), else the split kernel */
   FP8PD_OPT_K_DECODE = 3,    /* E4M3 -> f16 decode of K: 0 = bit assembly,
                                 1 = hardware cvt.rn.f16x2.e4m3x2 (default) */
   FP8PD_OPT_V_DECODE = 4     /* the same for V (default 1) */
@@ -257,7 +267,7 @@ int64_t fp8pd_get_option(int32_t option);
 
 /* What the last attention call on this host thread launched. */
 typedef struct fp8pd_run_info {
-  int32_t variant;           /* 1 = tensor-core, 2 = CUDA-core */
+  int32_t schedule;          /* 1 = split kernel, 2 = balanced kernel */
   int32_t num_splits;
   int32_t head_groups;
   int32_t grid_blocks;

@@ -126,6 +126,11 @@ def test_options_roundtrip(F):
     F.fp8pd_set_option(F.OPT_NUM_SPLITS, 7)
     assert F.fp8pd_get_option(F.OPT_NUM_SPLITS) == 7
     F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
+    F.fp8pd_set_option(F.OPT_SCHEDULE, 2)
+    assert F.fp8pd_get_option(F.OPT_SCHEDULE) == 2
+    F.fp8pd_set_option(F.OPT_SCHEDULE, 0)
+    with pytest.raises(F.Fp8pdError):
+        F.fp8pd_set_option(F.OPT_SCHEDULE, 4)
     with pytest.raises(F.Fp8pdError):
         F.fp8pd_set_option(99, 1)
     with pytest.raises(F.Fp8pdError):
@@ -140,7 +145,14 @@ def _plan(F, B, Hq, Hkv, D, ps, max_pages, window=0):
     return F.fp8pd_plan(q, k, t, window)
 
 
-def test_planner_fills_the_device_with_enough_work_per_split(F):
+@pytest.fixture
+def split_schedule(F):
+    F.fp8pd_set_option(F.OPT_SCHEDULE, 1)
+    yield
+    F.fp8pd_set_option(F.OPT_SCHEDULE, 0)
+
+
+def test_planner_fills_the_device_with_enough_work_per_split(F, split_schedule):
     # long context, one sequence: many splits, each >= 256 keys
     p = _plan(F, 1, 64, 8, 128, 64, 2049)
     assert p["num_splits"] > 16 and p["combine"] == 1
@@ -175,3 +187,55 @@ def test_planner_fills_the_device_with_enough_work_per_split(F):
         assert 240 <= _plan(F, 4, 32, 8, 128, 16, 5000)["num_splits"] <= 256  # capped
     finally:
         F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
+
+
+def test_planner_default_schedule(F):
+    """The planner's own choice: proportional splits for full attention and
+    long windows with enough work, uniform splits otherwise; the balanced
+    kernel only on request. Without a GPU it assumes 148 SMs."""
+    assert _plan(F, 32, 32, 8, 128, 16, 257)["schedule"] == 3           # Llama-like
+    assert _plan(F, 64, 64, 8, 64, 16, 513)["schedule"] == 3            # gpt-oss-like, full
+    assert _plan(F, 64, 64, 8, 64, 16, 513, window=4096)["schedule"] == 3
+    assert _plan(F, 64, 64, 8, 64, 16, 513, window=128)["schedule"] == 1
+    assert _plan(F, 1, 8, 2, 64, 16, 16)["schedule"] == 1               # too little work
+    assert _plan(F, 16, 16, 2, 512, 32, 513)["schedule"] == 3           # any head dim
+
+
+def test_planner_balanced_kernel_on_request(F):
+    """Schedule 2: every warp of one wave of blocks (4 per SM without a GPU:
+    2,368 warps) takes an equal share of the tiles."""
+    F.fp8pd_set_option(F.OPT_SCHEDULE, 2)
+    try:
+        p = _plan(F, 32, 32, 8, 128, 16, 257)
+        assert p["schedule"] == 2 and p["num_splits"] == 0 and p["combine"] == 1
+        assert p["warps"] == 4 * p["grid_blocks"] and p["grid_blocks"] % 148 == 0
+        U, nwt, hpu, D = 32 * 8, p["warps"], 4, 128
+        assert p["workspace_bytes"] >= (U + nwt) * hpu * (D + 2) * 4
+        assert _plan(F, 1, 8, 2, 64, 16, 16)["schedule"] == 2
+        assert _plan(F, 16, 16, 2, 512, 32, 513)["schedule"] == 1      # head dims above 128
+        assert _plan(F, 1025, 8, 8, 128, 16, 4)["schedule"] == 1       # more than 1,024 sequences
+        F.fp8pd_set_option(F.OPT_NUM_SPLITS, 3)
+        assert _plan(F, 32, 32, 8, 128, 16, 257)["schedule"] == 1      # a forced split count wins
+    finally:
+        F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
+        F.fp8pd_set_option(F.OPT_SCHEDULE, 0)
+
+
+def test_planner_proportional_splits(F):
+    """Schedule 3: one wave of split-kernel blocks per KV head x head group
+    (148 SMs x the split kernel's blocks per SM without a GPU), shared among
+    the sequences in the kernel."""
+    F.fp8pd_set_option(F.OPT_SCHEDULE, 3)
+    try:
+        p = _plan(F, 32, 32, 8, 128, 16, 257)
+        assert p["schedule"] == 3 and p["combine"] == 1 and p["num_splits"] == 0
+        assert p["grid_blocks"] % 8 == 0 and p["grid_blocks"] >= 8 * 32
+        # every sequence needs room for splits of at most 8,192 keys
+        p = _plan(F, 4, 8, 8, 128, 64, 2049)                       # 131,136 keys: 17 splits each
+        assert p["schedule"] == 3 and p["grid_blocks"] >= 8 * 4 * 17
+        assert _plan(F, 1025, 8, 8, 128, 16, 4)["schedule"] == 1    # more than 1,024 sequences
+        F.fp8pd_set_option(F.OPT_NUM_SPLITS, 2)
+        assert _plan(F, 32, 32, 8, 128, 16, 257)["schedule"] == 1   # a forced split count wins
+    finally:
+        F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
+        F.fp8pd_set_option(F.OPT_SCHEDULE, 0)

@@ -25,6 +25,16 @@ def F(cuda_device):
     return F
 
 
+@pytest.fixture(autouse=True, params=[1, 2, 3], ids=["split", "balanced", "proportional"])
+def schedule(F, request):
+    """Every test runs with each schedule: uniform splits, the balanced kernel
+    wherever it applies (head dims 64 and 128, no forced split count), and
+    proportional splits (no forced split count)."""
+    F.fp8pd_set_option(F.OPT_SCHEDULE, request.param)
+    yield request.param
+    F.fp8pd_set_option(F.OPT_SCHEDULE, 0)
+
+
 @pytest.fixture(params=[(1, 1), (0, 0)], ids=["cvt", "bits"])
 def kdecode(F, request):
     """Run a test with each E4M3 -> f16 decode of K and V (hardware cvt, bit
@@ -166,6 +176,24 @@ def test_windows(F, cuda_device, window):
     spec = W.Spec("win", B=3, ps=16, layers=(W.LayerSpec(8, 2, 64, window, 0.125),),
                   seq_len=(30, 600), scale_mode="page", sinks=True, seed=window % 97)
     _check_layer(F, W.make_case(spec, cuda_device), where=f"window={window}")
+
+
+def test_the_requested_kernel_runs(F, cuda_device, schedule):
+    case = W.make_case("llama", cuda_device, B=6, seq_len=(40, 700))
+    _check_layer(F, case, where="llama")
+    assert F.fp8pd_last_run_info()["schedule"] == schedule
+
+
+def test_ragged_batch_with_empty_and_long_sequences(F, cuda_device, kdecode):
+    """40 sequences from 0 to 3,000 keys, every seventh empty and one of a
+    single key: the balanced kernel's pieces cross many sequence boundaries."""
+    spec = W.Spec("ragged", B=40, ps=16, layers=(W.LayerSpec(32, 8, 128, 0, None),),
+                  seq_len=(0, 3000), scale_mode="page", sinks=True, seed=77)
+    case = W.make_case(spec, cuda_device)
+    lens = case.attend_lens.clone()
+    lens[::7] = 0
+    lens[3] = min(1, int(lens[3]))
+    _check_layer(F, case, lens=lens, where="ragged")
 
 
 # --------------------------------------------------------------- edge cases

@@ -45,19 +45,25 @@ def _both(F, layer, lens):
     return np_(ref), [np_(o) for o in outs]
 
 
-@pytest.mark.parametrize("name,overrides,splits", [
-    ("llama", dict(B=6, seq_len=(40, 700)), 0),        # ragged lengths, per-page scales
-    ("long_b1", dict(seq_len=20000), 0),               # many splits, two-level merge
-    ("long_b1", dict(seq_len=20000), 5),                # a single merge group
-    ("gptoss_full", dict(B=3, seq_len=1000), 0),        # sinks
+@pytest.mark.parametrize("name,overrides,splits,schedule", [
+    ("llama", dict(B=6, seq_len=(40, 700)), 0, 1),        # ragged lengths, per-page scales
+    ("long_b1", dict(seq_len=20000), 0, 1),               # many splits, two-level merge
+    ("long_b1", dict(seq_len=20000), 5, 1),               # a single merge group
+    ("gptoss_full", dict(B=3, seq_len=1000), 0, 1),       # sinks
+    ("llama", dict(B=6, seq_len=(40, 700)), 0, 2),        # the balanced kernel
+    ("long_b1", dict(seq_len=20000), 0, 2),               # balanced, two-level merge
+    ("llama", dict(B=6, seq_len=(40, 700)), 0, 3),        # proportional splits
 ])
-def test_noalloc_matches_the_allocating_entry_point(F, cuda_device, name, overrides, splits):
+def test_noalloc_matches_the_allocating_entry_point(F, cuda_device, name, overrides, splits,
+                                                    schedule):
     F.fp8pd_set_option(F.OPT_NUM_SPLITS, splits)
+    F.fp8pd_set_option(F.OPT_SCHEDULE, schedule)
     try:
         case = W.make_case(name, cuda_device, **overrides)
         ref, outs = _both(F, case.layers[0], case.attend_lens)
     finally:
         F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
+        F.fp8pd_set_option(F.OPT_SCHEDULE, 0)
     want = oracle_attention(case.layers[0], case.attend_lens)
     report = {}
     for label, arr in [("allocating", ref), ("noalloc 1", outs[0]), ("noalloc 2", outs[1])]:
@@ -73,8 +79,8 @@ def test_noalloc_matches_the_allocating_entry_point(F, cuda_device, name, overri
 
 
 def test_noalloc_refuses_a_call_whose_scratch_exceeds_its_array(F, cuda_device):
-    """8 MiB holds the split partials of every workload here; a call whose plan
-    needs more is refused with FP8PD_ERR_TOO_LARGE and launches nothing."""
+    """A call whose plan needs more than the 8 MiB array is refused with
+    FP8PD_ERR_TOO_LARGE and launches nothing."""
     F.fp8pd_set_option(F.OPT_NUM_SPLITS, 256)
     try:
         case = W.make_case("gptoss_full", cuda_device, B=64, seq_len=1000)
