@@ -4,7 +4,7 @@ One step = the decode hot path for one layer of a synthetic serving batch:
 ``fp8_kv_append`` of one new token per sequence, then
 ``fp8_paged_decode_attention`` over the updated paged E4M3 cache (split
 kernel + combine). Inputs are resident in HBM when the timed region starts;
-L2 is flushed (a 256 MiB write) between timed steps, outside each step's
+L2 is flushed between timed steps, outside each step's
 events. ``value`` = algorithmic bytes (attended K/V once per KV head + q +
 the block-table entries read) / device time, summed over ranks.
 
@@ -86,6 +86,31 @@ def _traffic(config: str):
     except OSError:
         pass
     return None
+
+
+class L2Flush:
+    """Empties the 126 MB L2 between timed steps: a 256 MiB write, then a read
+    of another 256 MiB buffer. The write alone would leave the L2 full of
+    dirty lines whose write-back to HBM then lands inside the next timed
+    step; after the read every line in the L2 is clean, so the step pays only
+    for its own traffic. FLUSH_MODE = "write" keeps the plain write."""
+    MODE = os.environ.get("FP8PD_BENCH_FLUSH", "write+read")
+
+    def __init__(self, device: torch.device):
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        self.r = torch.ones(64 << 20, dtype=torch.float32, device=device)
+        self.sink = torch.empty((), dtype=torch.float32, device=device)
+
+    def fill_(self, v: int = 1) -> None:
+        if "write" in self.MODE:
+            self.w.fill_(v & 0xFF)
+        if "read" in self.MODE:
+            torch.sum(self.r, dim=0, out=self.sink)
+
+    def describe(self) -> str:
+        return {"write": "256 MiB write", "read": "256 MiB read",
+                "write+read": "256 MiB write, then a 256 MiB read of another buffer (no dirty "
+                              "lines left)"}[self.MODE] + ", outside the step events"
 
 
 class ClockSampler:
@@ -212,7 +237,7 @@ def run_ours(args) -> dict | None:
     for layer in case.layers:
         layer.out = torch.empty(layer.q.shape, dtype=torch.float32, device=dev)
     step = Step(F, case)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
     nbytes = _step_bytes(case)
 
@@ -318,7 +343,7 @@ def run_ours(args) -> dict | None:
         "config": {"workload": WORKLOAD_TEXT.get(args.config, args.config),
                    "name": args.config,
                    "bytes_per_step": nbytes, "k_decode": args.k_decode,
-                   "l2": "flushed between timed steps (256 MiB write, outside the step events)",
+                   "l2": "flushed between timed steps: " + flush.describe(),
                    "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
         "timing": "device time of CUDA-graph replays of the step (per-step events); "
                   "eager time and per-kernel events from an eager pass of the same steps",

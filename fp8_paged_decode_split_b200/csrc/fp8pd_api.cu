@@ -223,7 +223,11 @@ bool plan_proportional(int B, int Hq, int Hkv, int D, int ps, int max_pages, int
   if (m_max > fp8pd::kMaxSplits) return false;
   const int64_t slots = static_cast<int64_t>(device_sms()) * fp8pd::decode_blocks_per_sm(D);
   if (g_opt_schedule.load() == 0 && B * HX * seq_tiles < 4 * slots) return false;  // little work
+#ifdef FP8PD_PROP_WAVES
+  const int64_t waves = FP8PD_PROP_WAVES;  // tuning builds
+#else
   const int64_t waves = (static_cast<int64_t>(B) * HX * 2 > slots) ? 2 : 1;
+#endif
   int64_t nbx = (waves * slots + HX - 1) / HX;
   nbx = std::max<int64_t>(nbx, B * m_max);  // room for every sequence's minimum splits
   nbx = std::min<int64_t>(nbx, std::min<int64_t>(65535, static_cast<int64_t>(B) * fp8pd::kMaxSplits));

@@ -194,6 +194,16 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar)
       : "memory");
 }
+// 4-byte asynchronous copy global -> shared (no register round trip); the
+// issuing thread waits for all of its copies with cp_async_wait_all.
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+}
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -541,10 +551,12 @@ __device__ __forceinline__ void attend_tile(Acc<D>& a, const QFrag& qfr, uint32_
   }
 }
 
-// Proportional splits. From the lengths, every sequence's tiles nt_b and its
-// splits S_b = min(nt_b, kMaxSplits, m_b + floor(nt_b * R / total)), m_b =
-// ceil(nt_b / kMaxSplitTiles), R = nbx - sum m_b (so sum S_b <= nbx), with
-// their prefix sums and those of the merge groups ceil(S_b / 8), in
+// Proportional splits. From the lengths, every sequence's tiles nt_b; the
+// smallest split size C (tiles) with sum_b ceil(nt_b / C) <= nbx, found by
+// bisection between ceil(total / nbx) and min(max nt_b, kMaxSplitTiles) (the
+// planner makes nbx at least sum_b ceil(nt_b / kMaxSplitTiles), so that
+// bound holds), which minimises the largest split; S_b = ceil(nt_b / C). The
+// splits and the merge groups ceil(S_b / 8) go into prefix sums in
 // `scratch` (the ring buffer, unused until the first copy). Block blockIdx.y
 // = k takes split k - sp_b of the sequence b whose splits hold k; its tiles
 // are [split * nt_b / S_b, (split + 1) * nt_b / S_b) of the attended range.
@@ -561,7 +573,7 @@ __device__ bool prop_assign(const DecodeParams& p, int* scratch, int* red, int h
   int* s_nt = scratch;       // [B] tiles of each sequence
   int* s_sp = s_nt + B;      // [B + 1] splits of the sequences before b
   int* s_gp = s_sp + B + 1;  // [B + 1] merge groups of the sequences before b
-  int tsum = 0, msum = 0;
+  int tsum = 0, tmax = 0, tcnt = 0;
   for (int bb = tid; bb < B; bb += NT) {
     int L = __ldg(p.lens + (int64_t)bb * p.lens_s);
     if (L < 0 || L > p.max_pages * p.ps) {
@@ -572,31 +584,52 @@ __device__ bool prop_assign(const DecodeParams& p, int* scratch, int* red, int h
     const int nt = L > lo ? (L - 1) / kTileTokens - lo / kTileTokens + 1 : 0;
     s_nt[bb] = nt;
     tsum += nt;
-    msum += (nt + kMaxSplitTiles - 1) / kMaxSplitTiles;
+    tmax = max(tmax, nt);
+    tcnt += nt > 0;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     tsum += __shfl_xor_sync(FULL, tsum, o);
-    msum += __shfl_xor_sync(FULL, msum, o);
+    tmax = max(tmax, __shfl_xor_sync(FULL, tmax, o));
+    tcnt += __shfl_xor_sync(FULL, tcnt, o);
   }
   if (lane == 0) {
     red[warp] = tsum;
-    red[NW + warp] = msum;
+    red[NW + warp] = tmax;
+    red[2 * NW + 1 + warp] = tcnt;
   }
   __syncthreads();
-  int total = 0, mtot = 0;
+  if (warp == 0) {
+    int total = 0, nmax = 0, nne = 0;
 #pragma unroll
-  for (int w = 0; w < NW; ++w) {
-    total += red[w];
-    mtot += red[NW + w];
+    for (int w = 0; w < NW; ++w) {
+      total += red[w];
+      nmax = max(nmax, red[NW + w]);
+      nne += red[2 * NW + 1 + w];
+    }
+    // bisection for the split size C: count(C) = sum_b ceil(nt_b / C). Every
+    // upper bound used satisfies count <= nbx: nmax (count = sequences with
+    // keys), kMaxSplitTiles (the planner's guarantee) and, with more blocks
+    // than such sequences, ceil(total / (nbx - nne)) (count <= total / C + nne).
+    int lo = max(1, max((total + p.nbx - 1) / max(p.nbx, 1), (nmax + kMaxSplits - 1) / kMaxSplits));
+    int hi = min(nmax, kMaxSplitTiles);
+    if (p.nbx > nne) hi = min(hi, (total + (p.nbx - nne) - 1) / (p.nbx - nne));
+    hi = max(lo, hi);
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      int cnt = 0;
+      for (int bb = lane; bb < B; bb += 32) cnt += (s_nt[bb] + mid - 1) / mid;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(FULL, cnt, o);
+      if (cnt <= p.nbx) hi = mid;
+      else lo = mid + 1;
+    }
+    __syncwarp();
+    if (lane == 0) red[2 * NW] = lo;
   }
-  const int R = max(0, p.nbx - mtot);
-  auto splits_of = [&](int nt) -> int {
-    if (nt == 0) return 0;
-    const int m = (nt + kMaxSplitTiles - 1) / kMaxSplitTiles;
-    const int s = m + static_cast<int>((int64_t)nt * R / total);
-    return min(min(s, nt), kMaxSplits);
-  };
+  __syncthreads();
+  const int C = red[2 * NW];
+  auto splits_of = [&](int nt) -> int { return (nt + C - 1) / C; };
   // exclusive prefix sums, a contiguous run of sequences per thread
   const int per = (B + NT - 1) / NT;
   const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
@@ -775,7 +808,9 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   // sequence length, so the first tiles of each warp are copied before the
   // length is known. Copies past the end of a short sequence are drained
   // before the block exits; a page id outside the pool is never copied.
-  const bool spec = p.window == 0;
+  // (Proportional splits know their range by now: they build the tile list
+  // first and copy from it, which saves a second block-table round trip.)
+  const bool spec = p.window == 0 && !p.prop;
   if (spec) {
     const int tf = p.prop ? prop_j0 : split * p.chunk_pages * (p.ps / kTileTokens);
     int e = -1;
@@ -851,18 +886,21 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       if (s < my_tiles) issue(went[s], s);
   }
 
+  // The scales go straight to shared memory (asynchronous copies); each lane
+  // waits for its own copies after the first tile has arrived, so their
+  // latency overlaps that of the first tile copies.
   const float* ksbase = p.ks + (int64_t)kvh * p.ks_sh;
   const float* vsbase = p.vs + (int64_t)kvh * p.vs_sh;
 #pragma unroll 2
   for (int j = lane; j < my_tiles; j += 32) {
     const int e = went[j];
-    float ks = 0.f, vs = 0.f;
     if (e >= 0) {
-      ks = __ldg(ksbase + (int64_t)(e >> 4) * p.ks_sp);
-      vs = __ldg(vsbase + (int64_t)(e >> 4) * p.vs_sp);
+      cp_async4(wks + j, ksbase + (int64_t)(e >> 4) * p.ks_sp);
+      cp_async4(wvs + j, vsbase + (int64_t)(e >> 4) * p.vs_sp);
+    } else {
+      wks[j] = 0.f;
+      wvs[j] = 0.f;
     }
-    wks[j] = ks;
-    wvs[j] = vs;
   }
   // Lane (g, q) holds query head g of the group; the k16 block kb covers
   // head-dim entries 16kb + 4q + {0..3} of lane quad q. Hardware-cvt K pairs
@@ -959,6 +997,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
       ok_all = false;
       break;
     }
+    if (j == 0) cp_async_wait_all();  // this lane's scale copies
     __syncwarp();
     {
       const int nj = j + C::NS - 1;
@@ -981,6 +1020,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   if (!ok_all) {
     // A copy never completed: leave this warp's result out (its flag is set)
     // and wait, again bounded, for whatever this warp still has in flight.
+    cp_async_wait_all();
     for (int s = 0; s < C::NS; ++s) mbar_wait(wbar + 8 * s, phase ^ (s < stage ? 1u : 0u));
     acc.m0 = acc.m1 = -CUDART_INF_F;
     acc.l0 = acc.l1 = 0.f;
