@@ -50,7 +50,7 @@ WORKLOAD_TEXT = {
 }
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic_per_launch.txt")
 KERNEL_NAME = {1: "decode_tma_kernel (split kernel, merge in the same launch)",
-               2: "decode_flat_kernel (balanced kernel, merge in the same launch)",
+               2: "decode_seg_kernel (balanced block ranges across sequences, merge in the same launch)",
                3: "decode_tma_kernel (proportional splits, merge in the same launch)"}
 
 
@@ -537,7 +537,7 @@ def main():
                     help="E4M3 -> f16 decode of K: bit assembly or hardware cvt")
     ap.add_argument("--splits", type=int, default=0, help="force a split count (0 = planner)")
     ap.add_argument("--schedule", type=int, default=0, choices=[0, 1, 2, 3],
-                    help="0 = planner, 1 = uniform splits, 2 = balanced kernel, "
+                    help="0 = planner, 1 = uniform splits, 2 = segment kernel, "
                          "3 = proportional splits")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -121,11 +121,10 @@ struct Plan {
   size_t grp_ml_bytes = 0;    // merged groups of splits
   size_t grp_o_bytes = 0;
   size_t workspace = 0;
-  int schedule = 1;            // 1 = uniform splits, 2 = balanced kernel, 3 = proportional splits
-  int nbx = 0;                 // proportional: blocks per KV head x head group
-  int warps = 0;               // balanced: warps of the grid
-  int hpu = 1;                 // balanced: heads per partial slot
-  int c1_count = 0;            // balanced: level-1 tickets (the unit tickets follow)
+  int schedule = 1;            // 1 = uniform splits, 2 = segment kernel, 3 = proportional splits
+  int nbx = 0;                 // proportional / segment: blocks per KV head x head group
+  int nslot = 0;               // segment: partial slots per (KV head x head group, head)
+  size_t seg_bytes = 0;        // segment: warp rows of the segment ends that do not stop the stream
 };
 
 int current_device(int* dev) {
@@ -153,52 +152,54 @@ int device_sms() {
   return sms;
 }
 
-// Balanced schedule: one full wave of blocks; every warp takes an equal share
-// of the tiles. Chosen (schedule option 0) for head dims 64 and 128 with no
-// forced split count, no window shorter than 2,048 keys, and at least 8 tiles
-// per warp when every sequence has its table's full length; the option can
-// force it wherever it applies (at least 8 groups of one warp per KV head x
-// head group). Returns false when it does not apply.
-bool plan_balanced(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window,
-                   bool allow, Plan* plan) {
+// Segment schedule: one block per SM, floor(SMs / HX) of them per KV head x
+// head group, each with an equal share of the flat list of all sequences'
+// tiles (crossing sequence boundaries). A block's share must fit its tile
+// list, so the grid grows past one wave only when every sequence at its
+// table's full length would not fit; at most kSegMergeFan * 32 blocks per
+// unit (the merge of one sequence's pieces reads at most 32 groups). Only on
+// request (schedule option 2): it balances every SM's work exactly, but its
+// segment ends and end-of-block merges cost more than the proportional
+// splits lose to uneven blocks on every workload measured so far.
+bool plan_seg(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, Plan* plan) {
   const int64_t sched = g_opt_schedule.load();
-  if (!allow || sched == 1 || sched == 3 || g_opt_num_splits.load() > 0) return false;
-  if (!(D == 64 || D == 128) || B > fp8pd::kFlatMaxBatch) return false;
+  if (sched != 2 || g_opt_num_splits.load() > 0) return false;
+  if (B > fp8pd::kSegMaxBatch) return false;
   const int G = Hq / Hkv;
   const int hg = (G + fp8pd::kHeadsPerGroup - 1) / fp8pd::kHeadsPerGroup;
   const int64_t HX = static_cast<int64_t>(Hkv) * hg;
   const int64_t keys = static_cast<int64_t>(max_pages) * ps;
   const int64_t seq_tiles = window > 0 ? std::min<int64_t>(keys, window) / fp8pd::kTileTokens + 2
                                        : (keys + fp8pd::kTileTokens - 1) / fp8pd::kTileTokens;
-  const int64_t t_max = B * HX * seq_tiles;  // tiles when every sequence is full
+  const int64_t t_max = B * seq_tiles;  // tiles of one unit when every sequence is full
   if (t_max >= (int64_t(1) << 31) - 1) return false;
-  const int blocks = device_sms() * fp8pd::flat_blocks_per_sm(D, B);
-  const int64_t nwt = static_cast<int64_t>(blocks) * fp8pd::kFlatWarps;
-  const int64_t groups = nwt / HX;  // groups of HX warps, one warp per unit of a column
-  if (groups < 8) return false;
-  if (sched != 2) return false;  // only on request: proportional splits run faster
-  const int64_t U = B * HX;
+  const int64_t slots = static_cast<int64_t>(device_sms()) * fp8pd::seg_blocks_per_sm(D, B);
+  const int64_t cap = fp8pd::seg_list_tiles(D);
+  const int64_t nbx_max = static_cast<int64_t>(fp8pd::kSegMergeFan) * 32;
+  int64_t nbx = std::max<int64_t>(1, std::min<int64_t>(slots / HX, nbx_max));
+  nbx = std::max<int64_t>(nbx, (t_max + cap - 1) / cap);
+  if (nbx > nbx_max) return false;
+  const int64_t nslot = nbx + B;
   plan->schedule = 2;
   plan->head_groups = hg;
+  plan->nbx = static_cast<int>(nbx);
+  plan->nslot = static_cast<int>(nslot);
   plan->num_splits = 0;
   plan->chunk_pages = 0;
   plan->num_groups = 0;
-  plan->grid_blocks = blocks;
+  plan->grid_blocks = static_cast<int>(HX * nbx);
   plan->combine = 1;
-  plan->warps = static_cast<int>(groups * HX);
-  plan->hpu = std::min(G, fp8pd::kHeadsPerGroup);
-  // slots (b + g) HX + x of segment partials; (b + W) HX + x of level-1
-  // tickets and group partials, W <= groups / 8
-  const int64_t slots1 = (B + groups) * HX, slots2 = (B + groups / fp8pd::kFlatFan + 2) * HX;
-  plan->c1_count = static_cast<int>(slots2);
-  const size_t hpu = static_cast<size_t>(plan->hpu);
-  plan->counters_bytes = align256(static_cast<size_t>(slots2 + U) * sizeof(int));
-  plan->ml_bytes = align256(static_cast<size_t>(slots1) * hpu * 2 * sizeof(float));
-  plan->o_bytes = align256(static_cast<size_t>(slots1) * hpu * D * sizeof(float));
-  plan->grp_ml_bytes = align256(static_cast<size_t>(slots2) * hpu * 2 * sizeof(float));
-  plan->grp_o_bytes = align256(static_cast<size_t>(slots2) * hpu * D * sizeof(float));
+  const size_t rows = static_cast<size_t>(HX * fp8pd::kHeadsPerGroup * nslot);
+  plan->counters_bytes = align256(static_cast<size_t>(HX * nslot + HX * B) * sizeof(int));
+  plan->ml_bytes = align256(rows * 2 * sizeof(float));
+  plan->o_bytes = align256(rows * D * sizeof(float));
+  plan->grp_ml_bytes = plan->ml_bytes;
+  plan->grp_o_bytes = plan->o_bytes;
+  plan->seg_bytes = D > 256 ? 0  // head dim 512 stops the stream at every segment end
+                            : align256(static_cast<size_t>(HX * nbx) * fp8pd::kSegAsync *
+                                       fp8pd::seg_warps(D) * (8 * D + 16) * sizeof(float));
   plan->workspace = plan->counters_bytes + plan->ml_bytes + plan->o_bytes + plan->grp_ml_bytes +
-                    plan->grp_o_bytes;
+                    plan->grp_o_bytes + plan->seg_bytes;
   return true;
 }
 
@@ -254,8 +255,8 @@ bool plan_proportional(int B, int Hq, int Hkv, int D, int ps, int max_pages, int
 }
 
 int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, Plan* plan,
-              bool allow_balanced = true) {
-  if (plan_balanced(B, Hq, Hkv, D, ps, max_pages, window, allow_balanced, plan)) return FP8PD_OK;
+              bool allow_seg = true) {
+  if (allow_seg && plan_seg(B, Hq, Hkv, D, ps, max_pages, window, plan)) return FP8PD_OK;
   // Proportional splits balance sequences of uneven length within one launch;
   // with a short window every sequence has about the same few tiles, and the
   // uniform splits below cost less.
@@ -497,8 +498,8 @@ int validate_decode(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp
 // The capacity T of the partial area fixes the counter area at
 // align256(T / 32 + 256) bytes. Every call has at most one ticket per 33
 // floats of partials: a split call (S >= 2 splits, D >= 64) has at most
-// units * S tickets and units * S * 66 floats; a balanced call at most
-// 2 (units + warps) tickets and (units + warps) * 66 floats. So every call
+// units * S tickets and units * S * 66 floats; a segment call at most
+// 2 * HX * nslot tickets and 2 * HX * 8 * nslot * 66 floats. So every call
 // whose plan fits in T bytes (fp8pd_plan's workspace_bytes) also fits in the
 // counter area: fp8pd_reserve_workspace(T) covers it.
 size_t counter_area(size_t T) { return align256(T / 32 + 256); }
@@ -572,10 +573,9 @@ void apply_plan(const Plan& plan, DecodeParams* p) {
   p->chunk_pages = plan.chunk_pages;
   p->num_groups = plan.num_groups;
   p->head_groups = plan.head_groups;
-  p->hpu = plan.hpu;
-  p->c1_count = plan.c1_count;
   p->prop = plan.schedule == 3 ? 1 : 0;
   p->nbx = plan.nbx;
+  p->nslot = plan.nslot;
 }
 
 void lay_out(const Plan& plan, void* ctr, void* part, DecodeParams* p) {
@@ -588,12 +588,14 @@ void lay_out(const Plan& plan, void* ctr, void* part, DecodeParams* p) {
   p->grp_ml = reinterpret_cast<float*>(base);
   base += plan.grp_ml_bytes;
   p->grp_o = reinterpret_cast<float*>(base);
+  base += plan.grp_o_bytes;
+  p->seg_scratch = plan.seg_bytes ? reinterpret_cast<float*>(base) : nullptr;
 }
 
 cudaError_t launch_planned(const Plan& plan, const DecodeParams& p, const CUtensorMap& tmk,
                            const CUtensorMap& tmv, cudaStream_t s) {
   const bool kc = g_opt_k_decode.load() == 1, vc = g_opt_v_decode.load() == 1;
-  if (plan.schedule == 2) return fp8pd::launch_decode_flat(p, tmk, tmv, kc, vc, plan.grid_blocks, s);
+  if (plan.schedule == 2) return fp8pd::launch_decode_seg(p, tmk, tmv, kc, vc, plan.nbx, s);
   return fp8pd::launch_decode(p, tmk, tmv, kc, vc, s);
 }
 
@@ -669,7 +671,7 @@ int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_t
   info->combine = plan.combine;
   info->workspace_bytes = plan.workspace;
   info->schedule = plan.schedule;
-  info->warps = plan.warps;
+  info->warps = plan.grid_blocks * (plan.schedule == 2 ? fp8pd::seg_warps(static_cast<int>(D)) : 4);
   return FP8PD_OK;
 }
 
@@ -905,7 +907,7 @@ extern "C" int fp8_paged_decode_attention_noalloc(
   r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
   if (r) return r;
   if (plan.schedule == 2 && plan.workspace > kNoAllocScratchBytes) {
-    // the balanced layout does not fit: the split kernel's may
+    // the segment layout does not fit: the split kernel's may
     r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan, false);
     if (r) return r;
   }

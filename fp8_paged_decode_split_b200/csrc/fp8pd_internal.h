@@ -43,11 +43,13 @@ struct DecodeParams {
   // least ceil(tiles / kMaxSplitTiles), the rest in proportion to its tiles.
   int prop;
   int nbx;
-  // Balanced schedule only (decode_flat_kernel): partial slots hold hpu =
-  // min(8, G) heads; the level-1 tickets are counters[0, c1_count), the
-  // per-unit final tickets counters[c1_count, c1_count + units).
-  int hpu;
-  int c1_count;
+  // Segment schedule (decode_seg_kernel): partial and group-partial rows
+  // (hx * 8 + head) * nslot + slot, slot < nslot = nbx + B; group tickets
+  // counters[hx * nslot + slot], sequence tickets counters[HX * nslot + hx * B + b].
+  int nslot;
+  // Rows [HX * nbx * kSegAsync * warps][8 * D + 16]: each warp's state at a
+  // segment end that did not stop the stream.
+  float* seg_scratch;
 };
 
 struct AppendParams {
@@ -73,18 +75,22 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmk, const C
                           bool k_cvt, bool v_cvt, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 
-// Balanced schedule: every warp of one full wave of blocks takes the same
-// number of 16-token tiles of the flat list of (sequence, KV head x head
-// group) units; the grid is `blocks` blocks of 128 threads.
-cudaError_t launch_decode_flat(const DecodeParams& p, const CUtensorMap& tmk,
-                               const CUtensorMap& tmv, bool k_cvt, bool v_cvt, int blocks,
-                               cudaStream_t s);
-// Blocks of the balanced kernel one SM holds for head dim D (64 or 128)
-// and a batch of B sequences.
-int flat_blocks_per_sm(int D, int B);
-constexpr int kFlatWarps = 4;        // warps per block of the balanced kernel
-constexpr int kFlatMaxBatch = 1024;  // sequences the balanced kernel keeps in shared memory
-constexpr int kFlatFan = 8;          // warps per level-1 merge group
+// Segment schedule: the tiles of all sequences of one KV head x head group
+// as one list, cut into nbx equal block ranges; grid (HX, nbx) of blocks of
+// 128 threads.
+cudaError_t launch_decode_seg(const DecodeParams& p, const CUtensorMap& tmk,
+                              const CUtensorMap& tmv, bool k_cvt, bool v_cvt, int nbx,
+                              cudaStream_t s);
+// Blocks of the segment kernel one SM holds for head dim D and a batch of B.
+int seg_blocks_per_sm(int D, int B);
+constexpr int kSegMaxBatch = 1024;    // sequences the segment kernel keeps in shared memory
+// Warps per block of the segment kernel (one block per SM; the rings of all
+// warps fill about 192 KiB of shared memory).
+constexpr int seg_warps(int D) { return D <= 128 ? 16 : D == 256 ? 8 : 4; }
+constexpr int kSegAsync = 4;      // segment ends per block that do not stop the stream
+constexpr int kSegMergeFan = 32;  // pieces of a sequence one merge reads
+// Tile entries of one block's range the segment kernel keeps.
+constexpr int seg_list_tiles(int D) { return D <= 128 ? 4096 : D == 256 ? 2048 : 1024; }
 
 // Thread blocks of the split kernel one SM holds for head dim D.
 int decode_blocks_per_sm(int D);

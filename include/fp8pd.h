@@ -151,15 +151,19 @@ enum {
  *   sm_scale     finite, > 0.
  *   out          float32 [B, Hq, D]; stride[2] must be 1, rows 16-byte aligned.
  *   stream       CUDA stream.
- * Launches one kernel, with one of two schedules. The split kernel gives
- * each (sequence, KV head, head group) one or more blocks, each an equal
- * share of its pages; the last block of each to finish merges the splits.
- * The balanced kernel (head dims 64 and 128, up to 1,024 sequences) gives
- * every warp of one full wave of blocks the same number of 16-token tiles of
- * all sequences together, whatever their lengths; the last warp of each
- * group of pieces of a (sequence, KV head, head group) merges them. The
- * planner takes the balanced kernel for long or uneven batches without a
- * short window. The partial results and the ticket counters live
+ * Launches one kernel, with one of three schedules. Uniform splits (1): the
+ * split kernel gives each (sequence, KV head, head group) the same number of
+ * blocks, each an equal share of its table's pages. Proportional splits (3):
+ * the split kernel on one wave of blocks per KV head x head group, shared
+ * among the sequences in proportion to their tiles (the kernel reads the
+ * lengths). In both, the last block of each (sequence, KV head, head group)
+ * to finish merges its splits. Segment kernel (2, on request): one block per
+ * SM; the 16-token tiles of all sequences form one list per KV head x head
+ * group, cut into equal block ranges that cross sequence boundaries, and the
+ * block's warps share its range through a queue. The planner takes
+ * proportional splits for full attention and windows of at least 2,048 keys
+ * when there is enough work, uniform splits otherwise.
+ * The partial results and the ticket counters live
  * in a library-owned per-device workspace: it grows on demand outside stream
  * capture; under capture a call that would need to grow it fails with
  * FP8PD_ERR_CAPTURE_WORKSPACE (call fp8pd_reserve_workspace, or run the call
@@ -228,14 +232,14 @@ int fp8_paged_decode_attention_noalloc(const fp8pd_tensor* q, const fp8pd_tensor
 
 /* What a call with these arguments would launch, without launching it. */
 typedef struct fp8pd_plan_info {
-  int32_t num_splits;        /* split kernel: blocks per (sequence, KV head, head group);
-                                balanced kernel: 0 */
+  int32_t num_splits;        /* uniform splits: blocks per (sequence, KV head, head group);
+                                proportional splits and the segment kernel: 0 */
   int32_t head_groups;       /* ceil(G / 8) query-head groups per KV head */
   int32_t grid_blocks;       /* thread blocks of the launch */
   int32_t combine;           /* 1 if partial results are merged (workspace used) */
   uint64_t workspace_bytes;  /* split workspace the call needs (0 if none) */
-  int32_t schedule;          /* 1 = split kernel, 2 = balanced kernel */
-  int32_t warps;             /* balanced kernel: warps sharing the tiles (else 0) */
+  int32_t schedule;          /* 1 = uniform splits, 2 = segment kernel, 3 = proportional splits */
+  int32_t warps;             /* warps of the launch */
 } fp8pd_plan_info;
 
 /* Plans a decode-attention call (same argument rules; nothing launched). */
@@ -255,9 +259,10 @@ enum {
   FP8PD_OPT_NUM_SPLITS = 1,  /* 0 = planner chooses (default); n > 0 asks for n splits (raised
                                 so that no split covers more than 8,192 keys, capped at 256
                                 splits and at the number of pages) */
-  FP8PD_OPT_SCHEDULE = 2,    /* 0 = planner chooses (default); 1 = split kernel; 2 = balanced
-                                kernel where it applies (D <= 128, B <= 1024, no forced split
-                                count), else the split kernel */
+  FP8PD_OPT_SCHEDULE = 2,    /* 0 = planner chooses (default); 1 = uniform splits; 2 = segment
+                                kernel where it applies (B <= 1024, no forced split count),
+                                else uniform splits; 3 = proportional splits where they apply
+                                (B <= 1024, no forced split count), else uniform splits */
   FP8PD_OPT_K_DECODE = 3,    /* E4M3 -> f16 decode of K: 0 = bit assembly,
                                 1 = hardware cvt.rn.f16x2.e4m3x2 (default) */
   FP8PD_OPT_V_DECODE = 4     /* the same for V (default 1) */
@@ -267,7 +272,7 @@ int64_t fp8pd_get_option(int32_t option);
 
 /* What the last attention call on this host thread launched. */
 typedef struct fp8pd_run_info {
-  int32_t schedule;          /* 1 = split kernel, 2 = balanced kernel */
+  int32_t schedule;          /* 1 = uniform splits, 2 = segment kernel, 3 = proportional splits */
   int32_t num_splits;
   int32_t head_groups;
   int32_t grid_blocks;

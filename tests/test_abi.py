@@ -191,7 +191,7 @@ def test_planner_fills_the_device_with_enough_work_per_split(F, split_schedule):
 
 def test_planner_default_schedule(F):
     """The planner's own choice: proportional splits for full attention and
-    long windows with enough work, uniform splits otherwise; the balanced
+    long windows with enough work, uniform splits otherwise; the segment
     kernel only on request. Without a GPU it assumes 148 SMs."""
     assert _plan(F, 32, 32, 8, 128, 16, 257)["schedule"] == 3           # Llama-like
     assert _plan(F, 64, 64, 8, 64, 16, 513)["schedule"] == 3            # gpt-oss-like, full
@@ -199,20 +199,29 @@ def test_planner_default_schedule(F):
     assert _plan(F, 64, 64, 8, 64, 16, 513, window=128)["schedule"] == 1
     assert _plan(F, 1, 8, 2, 64, 16, 16)["schedule"] == 1               # too little work
     assert _plan(F, 16, 16, 2, 512, 32, 513)["schedule"] == 3           # any head dim
+    assert _plan(F, 1025, 8, 8, 128, 16, 400)["schedule"] == 1          # more than 1,024 sequences
 
 
-def test_planner_balanced_kernel_on_request(F):
-    """Schedule 2: every warp of one wave of blocks (4 per SM without a GPU:
-    2,368 warps) takes an equal share of the tiles."""
+def test_planner_segment_kernel_on_request(F):
+    """Schedule 2: one block per SM, floor(148 / HX) of them per KV head x
+    head group without a GPU, each an equal share of all tiles; more blocks
+    only when the largest share would overflow a block's tile list (4,096
+    tiles at head dim 128)."""
     F.fp8pd_set_option(F.OPT_SCHEDULE, 2)
     try:
         p = _plan(F, 32, 32, 8, 128, 16, 257)
         assert p["schedule"] == 2 and p["num_splits"] == 0 and p["combine"] == 1
-        assert p["warps"] == 4 * p["grid_blocks"] and p["grid_blocks"] % 148 == 0
-        U, nwt, hpu, D = 32 * 8, p["warps"], 4, 128
-        assert p["workspace_bytes"] >= (U + nwt) * hpu * (D + 2) * 4
-        assert _plan(F, 1, 8, 2, 64, 16, 16)["schedule"] == 2
-        assert _plan(F, 16, 16, 2, 512, 32, 513)["schedule"] == 1      # head dims above 128
+        assert p["grid_blocks"] == 8 * 18
+        nbx, B, D, HX = 18, 32, 128, 8
+        assert p["workspace_bytes"] >= 2 * HX * 8 * (nbx + B) * (D + 2) * 4
+        assert _plan(F, 1, 8, 2, 64, 16, 16)["grid_blocks"] == 2 * 74
+        assert _plan(F, 16, 16, 2, 512, 32, 513)["schedule"] == 2      # every head dim
+        # 8 sequences of 131,136 keys: 65,568 tiles per KV head, 18 blocks of 3,643
+        p = _plan(F, 8, 64, 8, 128, 64, 2049)
+        assert p["schedule"] == 2 and p["grid_blocks"] == 8 * 18
+        # 16 such sequences need 33 blocks of at most 4,096 tiles per KV head
+        p = _plan(F, 16, 64, 8, 128, 64, 2049)
+        assert p["schedule"] == 2 and p["grid_blocks"] == 8 * 33
         assert _plan(F, 1025, 8, 8, 128, 16, 4)["schedule"] == 1       # more than 1,024 sequences
         F.fp8pd_set_option(F.OPT_NUM_SPLITS, 3)
         assert _plan(F, 32, 32, 8, 128, 16, 257)["schedule"] == 1      # a forced split count wins
