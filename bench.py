@@ -1,9 +1,12 @@
 """Benchmark: FP8 paged decode attention, achieved HBM GB/s and us/step.
 
 One step = the decode hot path for one layer of a synthetic serving batch:
-``fp8_kv_append`` of one new token per sequence, then
-``fp8_paged_decode_attention`` over the updated paged E4M3 cache (split
-kernel + combine). Inputs are resident in HBM when the timed region starts;
+the append of one new token per sequence, then decode attention over the
+updated paged E4M3 cache -- by default one ``fp8_paged_decode_append_attention``
+launch (split kernel, append and combine fused); ``--unfused`` runs
+``fp8_kv_append`` and ``fp8_paged_decode_attention`` as two launches.
+Configs without an append run the attention call alone. Inputs are resident
+in HBM when the timed region starts;
 L2 is flushed between timed steps, outside each step's
 events. ``value`` = algorithmic bytes (attended K/V once per KV head + q +
 the block-table entries read) / device time, summed over ranks.
@@ -198,15 +201,25 @@ def whole_job_gbs(world: int, bytes_per_rank_step: int, ms_per_step: float) -> f
 
 
 class Step:
-    """One decode step of the workload through the library's public API."""
+    """One decode step of the workload through the library's public API: with
+    an append, the fused call (append and attention in one launch) unless
+    `fused` is off, then fp8_kv_append followed by the attention call."""
 
-    def __init__(self, F, case: W.Case):
+    def __init__(self, F, case: W.Case, fused: bool = True):
         self.F = F
         self.case = case
+        self.fused = fused and case.spec.append
 
     def run(self, stream=None):
         F, c = self.F, self.case
         for layer in c.layers:
+            if self.fused:
+                F.fp8_paged_decode_append_attention(
+                    layer.q, layer.k_new, layer.v_new, layer.k_pages, layer.v_pages,
+                    layer.k_scale, layer.v_scale, layer.block_table, c.positions,
+                    window=layer.window, sinks=layer.sinks, sm_scale=layer.sm_scale,
+                    out=layer.out, stream=stream)
+                continue
             if c.spec.append:
                 F.fp8_kv_append(layer.k_new, layer.v_new, layer.k_pages, layer.v_pages,
                                 layer.k_scale, layer.v_scale, layer.block_table, c.positions,
@@ -236,7 +249,7 @@ def run_ours(args) -> dict | None:
     case = W.make_case(args.config, dev)
     for layer in case.layers:
         layer.out = torch.empty(layer.q.shape, dtype=torch.float32, device=dev)
-    step = Step(F, case)
+    step = Step(F, case, not args.unfused)
     flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
     nbytes = _step_bytes(case)
@@ -348,7 +361,9 @@ def run_ours(args) -> dict | None:
         "timing": "device time of CUDA-graph replays of the step (per-step events); "
                   "eager time and per-kernel events from an eager pass of the same steps",
         "eager_ms_per_step": round(eager_ms / args.steps, 6),
-        "roofline": {"bound": "hbm", "kernel": KERNEL_NAME[plan_info["schedule"]],
+        "roofline": {"bound": "hbm",
+                     "kernel": KERNEL_NAME[plan_info["schedule"]] +
+                     (", append fused" if step.fused else ""),
                      "achieved": round(achieved, 2) if achieved else None,
                      "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
                      "unit": "GB/s",
@@ -383,12 +398,14 @@ def run_e2e(F, case: W.Case, dev, flush, args) -> dict:
             host_in.append(t.detach().cpu().pin_memory())
             dev_in.append(t)
         host_out.append(torch.empty(layer.q.shape, dtype=torch.float32).pin_memory())
-    for t in [case.attend_lens] + ([case.positions] if case.spec.append else []):
+    step = Step(F, case, not args.unfused)
+    lens = [case.positions] if step.fused else \
+        [case.attend_lens] + ([case.positions] if case.spec.append else [])
+    for t in lens:
         host_in.append(t.cpu().pin_memory())
         dev_in.append(t)
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in host_out)
-    step = Step(F, case)
     steps = max(3, min(args.steps, 20))
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
@@ -532,6 +549,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(W.SPECS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--unfused", action="store_true",
+                    help="run fp8_kv_append and the attention call as two launches")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--k-decode", default="bits", choices=["bits", "cvt"],
                     help="E4M3 -> f16 decode of K: bit assembly or hardware cvt")

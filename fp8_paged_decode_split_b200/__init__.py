@@ -13,6 +13,8 @@ Entry points (same names as the C ABI):
   caller softmax scale.
 * :func:`fp8_kv_append` -- quantize one new bf16 K/V token per sequence to
   E4M3 and store it in its page.
+* :func:`fp8_paged_decode_append_attention` -- both in one launch: the
+  append, then the attention over the updated cache.
 """
 
 from __future__ import annotations
@@ -24,6 +26,7 @@ import torch
 
 __all__ = [
     "fp8_paged_decode_attention", "fp8_paged_decode_attention_noalloc", "fp8_kv_append",
+    "fp8_paged_decode_append_attention",
     "fp8pd_plan", "fp8pd_reserve_workspace",
     "fp8pd_check_errors", "fp8pd_set_option", "fp8pd_get_option", "fp8pd_last_run_info",
     "fp8pd_timing_enable", "fp8pd_timing_collect", "Fp8pdError", "lib", "LIB_PATH",
@@ -76,6 +79,7 @@ def _load() -> ctypes.CDLL:
     lib.fp8_paged_decode_attention.argtypes = [T, T, T, T, T, T, T, i32, T, f32, T, vp]
     lib.fp8_paged_decode_attention_noalloc.argtypes = [T, T, T, T, T, T, T, i32, T, f32, T, vp]
     lib.fp8_kv_append.argtypes = [T, T, T, T, P(Scales), T, T, vp]
+    lib.fp8_paged_decode_append_attention.argtypes = [T, T, T, T, T, T, T, T, T, i32, T, f32, T, vp]
     lib.fp8pd_plan.argtypes = [T, T, T, i32, P(PlanInfo)]
     lib.fp8pd_reserve_workspace.argtypes = [ctypes.c_uint64]
     lib.fp8pd_check_errors.argtypes = [vp, P(ctypes.c_uint32)]
@@ -90,7 +94,7 @@ def _load() -> ctypes.CDLL:
     lib.fp8pd_last_cuda_error.restype = i32
     lib.fp8pd_version.restype = i32
     for name in ("fp8_paged_decode_attention", "fp8_paged_decode_attention_noalloc",
-                 "fp8_kv_append", "fp8pd_plan",
+                 "fp8_kv_append", "fp8_paged_decode_append_attention", "fp8pd_plan",
                  "fp8pd_reserve_workspace", "fp8pd_check_errors", "fp8pd_set_option",
                  "fp8pd_last_run_info", "fp8pd_timing_enable", "fp8pd_timing_collect"):
         getattr(lib, name).restype = i32
@@ -211,6 +215,30 @@ def fp8_kv_append(k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table,
     st = lib.fp8_kv_append(*[_ref(d) for d in ds], ctypes.byref(sc), _ref(dt), _ref(dp),
                            _stream(stream, k_new))
     _check(st, "fp8_kv_append")
+
+
+def fp8_paged_decode_append_attention(q, k_new, v_new, k_pages, v_pages, k_scale, v_scale,
+                                      block_table, positions, window: int = 0, sinks=None,
+                                      sm_scale: float | None = None, out=None,
+                                      stream=None) -> torch.Tensor:
+    """:func:`fp8_kv_append` of k_new / v_new at ``positions`` followed by
+    :func:`fp8_paged_decode_attention` over ``positions + 1`` keys, in one
+    launch (see include/fp8pd.h). The pools are written. Returns out
+    [B, Hq, D] float32."""
+    if sm_scale is None:
+        sm_scale = q.shape[-1] ** -0.5
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    _same_device(q, k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table, positions,
+                 sinks, out)
+    ds = [describe(t) for t in (q, k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table,
+                                positions)]
+    ds_sinks, ds_out = describe(sinks), describe(out)
+    st = lib.fp8_paged_decode_append_attention(*[_ref(d) for d in ds], int(window),
+                                               _ref(ds_sinks), float(sm_scale), _ref(ds_out),
+                                               _stream(stream, q))
+    _check(st, "fp8_paged_decode_append_attention")
+    return out
 
 
 def fp8pd_plan(q, k_pages, block_table, window: int = 0) -> dict:

@@ -610,20 +610,15 @@ void record_run(const Plan& plan, int D) {
 
 }  // namespace
 
-int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_pages,
-                               const fp8pd_tensor* v_pages, const fp8pd_tensor* k_scale,
-                               const fp8pd_tensor* v_scale, const fp8pd_tensor* block_table,
-                               const fp8pd_tensor* seq_lens, int32_t window,
-                               const fp8pd_tensor* sinks, float sm_scale, fp8pd_tensor* out,
-                               fp8pd_stream_t stream) {
-  DecodeParams p;
-  DecodeArgs a;
-  int r = validate_decode(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens, window,
-                          sinks, sm_scale, out, &p, &a);
-  if (r) return r;
-  if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
+namespace {
+
+// Plans, sizes the workspace, encodes the tensor maps and launches one
+// validated decode-attention call. `allow_seg`: the segment kernel may run
+// (it has no fused append).
+int run_decode(DecodeParams& p, const DecodeArgs& a, const fp8pd_tensor* k_pages,
+               const fp8pd_tensor* v_pages, int32_t window, bool allow_seg, fp8pd_stream_t stream) {
   Plan plan;
-  r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
+  int r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan, allow_seg);
   if (r) return r;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   apply_plan(plan, &p);
@@ -645,6 +640,58 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
   ++g_calls;
   record_run(plan, a.D);
   return FP8PD_OK;
+}
+
+}  // namespace
+
+int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_pages,
+                               const fp8pd_tensor* v_pages, const fp8pd_tensor* k_scale,
+                               const fp8pd_tensor* v_scale, const fp8pd_tensor* block_table,
+                               const fp8pd_tensor* seq_lens, int32_t window,
+                               const fp8pd_tensor* sinks, float sm_scale, fp8pd_tensor* out,
+                               fp8pd_stream_t stream) {
+  DecodeParams p;
+  DecodeArgs a;
+  int r = validate_decode(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens, window,
+                          sinks, sm_scale, out, &p, &a);
+  if (r) return r;
+  if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
+  return run_decode(p, a, k_pages, v_pages, window, true, stream);
+}
+
+int fp8_paged_decode_append_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_new,
+                                      const fp8pd_tensor* v_new, fp8pd_tensor* k_pages,
+                                      fp8pd_tensor* v_pages, const fp8pd_tensor* k_scale,
+                                      const fp8pd_tensor* v_scale, const fp8pd_tensor* block_table,
+                                      const fp8pd_tensor* positions, int32_t window,
+                                      const fp8pd_tensor* sinks, float sm_scale, fp8pd_tensor* out,
+                                      fp8pd_stream_t stream) {
+  DecodeParams p;
+  DecodeArgs a;
+  int r = validate_decode(q, k_pages, v_pages, k_scale, v_scale, block_table, positions, window,
+                          sinks, sm_scale, out, &p, &a);
+  if (r) return r;
+  if ((r = check(k_new, FP8PD_DTYPE_BF16, 3))) return r;
+  if ((r = check(v_new, FP8PD_DTYPE_BF16, 3))) return r;
+  for (int i = 0; i < 3; ++i)
+    if (v_new->shape[i] != k_new->shape[i]) return FP8PD_ERR_SHAPE;
+  if (k_new->shape[0] != a.B || k_new->shape[1] != a.Hkv || k_new->shape[2] != a.D)
+    return FP8PD_ERR_SHAPE;
+  if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
+  p.append = 1;
+  p.kn = static_cast<const uint16_t*>(k_new->data);
+  p.vn = static_cast<const uint16_t*>(v_new->data);
+  p.kn_sb = k_new->stride[0];
+  p.kn_sh = k_new->stride[1];
+  p.kn_sd = k_new->stride[2];
+  p.vn_sb = v_new->stride[0];
+  p.vn_sh = v_new->stride[1];
+  p.vn_sd = v_new->stride[2];
+  p.kw = static_cast<uint8_t*>(k_pages->data);
+  p.vw = static_cast<uint8_t*>(v_pages->data);
+  r = run_decode(p, a, k_pages, v_pages, window, false, stream);
+  if (r == FP8PD_OK) ++g_appends;
+  return r;
 }
 
 int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_tensor* block_table,

@@ -50,6 +50,16 @@ struct DecodeParams {
   // Rows [HX * nbx * kSegAsync * warps][8 * D + 16]: each warp's state at a
   // segment end that did not stop the stream.
   float* seg_scratch;
+  // Fused append (split kernel only): `lens` holds positions; sequence b
+  // attends over positions[b] + 1 keys, the last of them the new token
+  // (kn, vn: bf16 [B, Hkv, D]), which the block holding it quantizes, stores
+  // through kw / vw (the pools, writable) and attends.
+  int append;
+  const uint16_t* kn;
+  const uint16_t* vn;
+  int64_t kn_sb, kn_sh, kn_sd, vn_sb, vn_sh, vn_sd;
+  uint8_t* kw;
+  uint8_t* vw;
 };
 
 struct AppendParams {

@@ -551,6 +551,93 @@ __device__ __forceinline__ void attend_tile(Acc<D>& a, const QFrag& qfr, uint32_
   }
 }
 
+// Keys sequence b attends over: its length, or with a fused append its
+// position + 1. An out-of-range value sets `flag` (when `report`) and gives 0.
+__device__ __forceinline__ int attended_keys(const DecodeParams& p, int b, bool report) {
+  const int v = __ldg(p.lens + (int64_t)b * p.lens_s);
+  const int lim = p.max_pages * p.ps;
+  if (p.append) {
+    if (v >= 0 && v < lim) return v + 1;
+    if (report) raise_flag(FP8PD_FLAG_POS_OOB);
+    return 0;
+  }
+  if (v >= 0 && v <= lim) return v;
+  if (report) raise_flag(FP8PD_FLAG_SEQLEN_OOB);
+  return 0;
+}
+
+// E4M3 codes of two f32 values: round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint16_t e4m3x2_rn_sat(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;  // low byte = lo, high byte = hi
+}
+
+// Fused append, one warp: quantizes the new token of (sequence b, KV head
+// kvh) with its page's scales (IEEE f32 division, then E4M3 round to nearest
+// even with saturation, as fp8_kv_append), writes its codes into row r of the
+// K and V tiles in shared memory (the TMA's swizzled layout, see tile_off)
+// and, when `store`, into the pools at (page, slot). Lane l owns head-dim
+// bytes [l D/32, (l+1) D/32).
+template <int D>
+__device__ __noinline__ void append_new_token(const DecodeParams& p, int b, int kvh, bool store,
+                                              int page, int slot, int r, uint32_t sk, uint32_t sv,
+                                              float ks, float vs) {
+  constexpr int PER = D / 32;  // 2, 4, 8 or 16 bytes per lane
+  const int lane = threadIdx.x & 31;
+  const int d0 = lane * PER;
+  const uint16_t* kn = p.kn + (int64_t)b * p.kn_sb + (int64_t)kvh * p.kn_sh;
+  const uint16_t* vn = p.vn + (int64_t)b * p.vn_sb + (int64_t)kvh * p.vn_sh;
+  uint32_t kw[(PER + 3) / 4], vw[(PER + 3) / 4];
+#pragma unroll
+  for (int i = 0; i < (PER + 3) / 4; ++i) kw[i] = vw[i] = 0u;
+#pragma unroll
+  for (int i = 0; i < PER; i += 2) {
+    const int d = d0 + i;
+    const uint32_t kc = e4m3x2_rn_sat(__fdiv_rn(bf16_bits_to_float(kn[(int64_t)d * p.kn_sd]), ks),
+                                      __fdiv_rn(bf16_bits_to_float(kn[(int64_t)(d + 1) * p.kn_sd]), ks));
+    const uint32_t vc = e4m3x2_rn_sat(__fdiv_rn(bf16_bits_to_float(vn[(int64_t)d * p.vn_sd]), vs),
+                                      __fdiv_rn(bf16_bits_to_float(vn[(int64_t)(d + 1) * p.vn_sd]), vs));
+    kw[i / 4] |= kc << (8 * (i % 4));
+    vw[i / 4] |= vc << (8 * (i % 4));
+  }
+  // PER divides 16, so the lane's bytes sit inside one 16-byte chunk of the row
+  const uint32_t off = tile_off<D>(r, d0 & ~15) + (d0 & 15);
+  uint8_t* gk = p.kw + (int64_t)page * p.k_sp + (int64_t)slot * p.k_st + (int64_t)kvh * p.k_sh + d0;
+  uint8_t* gv = p.vw + (int64_t)page * p.v_sp + (int64_t)slot * p.v_st + (int64_t)kvh * p.v_sh + d0;
+  if constexpr (PER == 2) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(sk + off), "h"((uint16_t)kw[0]) : "memory");
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(sv + off), "h"((uint16_t)vw[0]) : "memory");
+    if (store) {
+      *reinterpret_cast<uint16_t*>(gk) = (uint16_t)kw[0];
+      *reinterpret_cast<uint16_t*>(gv) = (uint16_t)vw[0];
+    }
+  } else if constexpr (PER == 4) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(sk + off), "r"(kw[0]) : "memory");
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(sv + off), "r"(vw[0]) : "memory");
+    if (store) {
+      *reinterpret_cast<uint32_t*>(gk) = kw[0];
+      *reinterpret_cast<uint32_t*>(gv) = vw[0];
+    }
+  } else if constexpr (PER == 8) {
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(sk + off), "r"(kw[0]), "r"(kw[1]) : "memory");
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(sv + off), "r"(vw[0]), "r"(vw[1]) : "memory");
+    if (store) {
+      *reinterpret_cast<uint2*>(gk) = make_uint2(kw[0], kw[1]);
+      *reinterpret_cast<uint2*>(gv) = make_uint2(vw[0], vw[1]);
+    }
+  } else {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sk + off), "r"(kw[0]), "r"(kw[1]),
+                 "r"(kw[2]), "r"(kw[3]) : "memory");
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sv + off), "r"(vw[0]), "r"(vw[1]),
+                 "r"(vw[2]), "r"(vw[3]) : "memory");
+    if (store) {
+      *reinterpret_cast<uint4*>(gk) = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+      *reinterpret_cast<uint4*>(gv) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
+    }
+  }
+}
+
 // Proportional splits. From the lengths, every sequence's tiles nt_b; the
 // smallest split size C (tiles) with sum_b ceil(nt_b / C) <= nbx, found by
 // bisection between ceil(total / nbx) and min(max nt_b, kMaxSplitTiles) (the
@@ -575,11 +662,7 @@ __device__ bool prop_assign(const DecodeParams& p, int* scratch, int* red, int h
   int* s_gp = s_sp + B + 1;  // [B + 1] merge groups of the sequences before b
   int tsum = 0, tmax = 0, tcnt = 0;
   for (int bb = tid; bb < B; bb += NT) {
-    int L = __ldg(p.lens + (int64_t)bb * p.lens_s);
-    if (L < 0 || L > p.max_pages * p.ps) {
-      if (blockIdx.x == 0 && blockIdx.y == 0) raise_flag(FP8PD_FLAG_SEQLEN_OOB);
-      L = 0;
-    }
+    const int L = attended_keys(p, bb, blockIdx.x == 0 && blockIdx.y == 0);
     const int lo = p.window > 0 ? max(0, L - p.window) : 0;
     const int nt = L > lo ? (L - 1) / kTileTokens - lo / kTileTokens + 1 : 0;
     s_nt[bb] = nt;
@@ -830,11 +913,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   // Split s of a sequence covers pages [first + s * chunk, first + (s+1) * chunk)
   // of its attended range: equal-sized work per block whatever the length,
   // and the blocks past the end of a short sequence have nothing to do.
-  int L = __ldg(p.lens + (int64_t)b * p.lens_s);
-  if (L < 0 || L > p.max_pages * p.ps) {
-    if (tid == 0 && split == 0 && blockIdx.x == 0) raise_flag(FP8PD_FLAG_SEQLEN_OOB);
-    L = 0;
-  }
+  const int L = attended_keys(p, b, tid == 0 && split == 0 && blockIdx.x == 0);
   const int lo = p.window > 0 ? max(0, L - p.window) : 0;
   int t0, t1;
   if (p.prop) {
@@ -1012,6 +1091,13 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     if (++stage == C::NS) {
       stage = 0;
       phase ^= 1;
+    }
+    if (p.append && page_ok && L - 1 >= tok0 && L - 1 < tok0 + kTileTokens) {
+      // the new token: quantized here, stored by head group 0, attended by all
+      const int r = L - 1 - tok0;
+      append_new_token<D>(p, b, kvh, hg == 0, went[j] >> 4, (went[j] & 15) * kTileTokens + r, r,
+                          sk, sv, wks[j], vs);
+      __syncwarp();
     }
 
     attend_tile<D, KCVT, VCVT>(acc, qfr, sk, sv, koff, voff, kfac, vs, tok0, t0, t1, page_ok, full,
@@ -1926,11 +2012,6 @@ __global__ void __launch_bounds__(SegCfg<D>::NT, 1)
 // division (__fdiv_rn), then cvt.rn.satfinite.e4m3x2.f32, which rounds to
 // nearest even and saturates to +-448 (NaN stays NaN).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint16_t e4m3x2_from_f32(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;  // low byte = lo, high byte = hi
-}
 
 __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
   const int npair = (p.D + 1) / 2;
@@ -1962,8 +2043,8 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
   const float k1 = two ? __fdiv_rn(bf16_bits_to_float(kn[p.kn_sd]), ks) : 0.f;
   const float v0 = __fdiv_rn(bf16_bits_to_float(vn[0]), vs);
   const float v1 = two ? __fdiv_rn(bf16_bits_to_float(vn[p.vn_sd]), vs) : 0.f;
-  const uint16_t kc = e4m3x2_from_f32(k0, k1);
-  const uint16_t vc = e4m3x2_from_f32(v0, v1);
+  const uint16_t kc = e4m3x2_rn_sat(k0, k1);
+  const uint16_t vc = e4m3x2_rn_sat(v0, v1);
   uint8_t* kd = p.k + (int64_t)page * p.k_sp + (int64_t)slot * p.k_st + (int64_t)h * p.k_sh + d;
   uint8_t* vd = p.v + (int64_t)page * p.v_sp + (int64_t)slot * p.v_st + (int64_t)h * p.v_sh + d;
   kd[0] = static_cast<uint8_t>(kc & 0xFF);

@@ -18,6 +18,12 @@
  *                               scope", the one-launch T=1 append; the
  *                               "Lecture 8 -- Inference Path" page, "In-kernel
  *                               KV cache update").
+ *   fp8_paged_decode_append_attention
+ *                               both in one launch: the append, then the
+ *                               attention over the cache that now holds the
+ *                               new token (the same Lecture 8 section: the
+ *                               cache is updated inside the attention kernel,
+ *                               before the query reads it).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -203,6 +209,39 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
                   const fp8pd_tensor* block_table, const fp8pd_tensor* positions,
                   fp8pd_stream_t stream);
 
+
+/*
+ * fp8_paged_decode_append_attention -- fp8_kv_append followed by
+ * fp8_paged_decode_attention, in one kernel launch.
+ *
+ * For each sequence b, with pos = positions[b]: the new token (k_new[b],
+ * v_new[b], bf16 [B, Hkv, D]) is quantized exactly as fp8_kv_append does
+ * (E4M3 code = round-to-nearest-even(float32 x / scale), saturated to +-448,
+ * with the scale of the page that holds position pos), written at position
+ * pos of the pools, and the query then attends over the pos + 1 keys
+ * 0 .. pos, the new one included -- the result of fp8_kv_append(..., positions)
+ * followed by fp8_paged_decode_attention(..., seq_lens = positions + 1),
+ * codes bit-identical and attention within float32 rounding. The block of
+ * the launch that holds position pos quantizes the token, stores it (once
+ * per KV head) and uses the codes it computed, so no block depends on
+ * another's write. The Lecture 8 page ("In-kernel KV cache update") states
+ * the order: the cache is updated, then read.
+ *
+ * Arguments: as fp8_paged_decode_attention, plus k_new / v_new (bf16
+ * [B, Hkv, D], any strides) and positions (int32 [B]) in place of seq_lens;
+ * the pools are written. A position outside [0, max_pages * page_size) sets
+ * FP8PD_FLAG_POS_OOB and that sequence's output is 0, nothing is written; a
+ * block-table entry outside the pool sets FP8PD_FLAG_PAGE_OOB. Runs the split
+ * kernel (uniform or proportional splits; a request for the segment kernel
+ * falls back to uniform splits). Workspace rules as fp8_paged_decode_attention.
+ */
+int fp8_paged_decode_append_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_new,
+                                      const fp8pd_tensor* v_new, fp8pd_tensor* k_pages,
+                                      fp8pd_tensor* v_pages, const fp8pd_tensor* k_scale,
+                                      const fp8pd_tensor* v_scale, const fp8pd_tensor* block_table,
+                                      const fp8pd_tensor* positions, int32_t window,
+                                      const fp8pd_tensor* sinks, float sm_scale, fp8pd_tensor* out,
+                                      fp8pd_stream_t stream);
 /*
  * fp8_paged_decode_attention_noalloc -- the same operation, allocating nothing.
  *

@@ -29,7 +29,8 @@ def _declared_functions():
 
 def test_header_declares_the_boundary():
     names = _declared_functions()
-    for required in ("fp8_paged_decode_attention", "fp8_kv_append", "fp8pd_check_errors",
+    for required in ("fp8_paged_decode_attention", "fp8_kv_append",
+                     "fp8_paged_decode_append_attention", "fp8pd_check_errors",
                      "fp8pd_reserve_workspace", "fp8pd_plan", "fp8pd_status_string"):
         assert required in names
 
@@ -102,6 +103,35 @@ def test_null_descriptors(F):
                                           None, None)
     assert st == -1
     st = F.lib.fp8_kv_append(None, None, None, None, None, None, None, None)
+    assert st == -1
+
+
+def test_fused_append_attention_validation(F):
+    """The fused call checks everything the attention call checks, then the
+    new token's dtype and shape, before any launch."""
+    a = _args()
+    kn = torch.zeros(2, 2, 128, dtype=torch.bfloat16)
+
+    def fused(**over):
+        b = dict(a, kn=kn, vn=kn)
+        b.update(over)
+        try:
+            F.fp8_paged_decode_append_attention(
+                b["q"], b["kn"], b["vn"], b["k"], b["v"], b["ks"], b["vs"], b["table"], b["lens"],
+                window=b["window"], sinks=b["sinks"], sm_scale=b["sm_scale"], out=b["out"],
+                stream=0)
+        except F.Fp8pdError as e:
+            return e.status
+        return 0
+
+    assert fused(kn=kn.float()) == -2
+    assert fused(vn=kn.float()) == -2
+    assert fused(kn=torch.zeros(2, 3, 128, dtype=torch.bfloat16)) == -3
+    assert fused(vn=torch.zeros(2, 2, 64, dtype=torch.bfloat16)) == -3
+    assert fused(window=-1) == -6
+    assert fused(k=torch.zeros(6, 16, 2, 136, dtype=torch.uint8)[..., :128]) == -4
+    st = F.lib.fp8_paged_decode_append_attention(None, None, None, None, None, None, None, None,
+                                                 None, 0, None, 1.0, None, None)
     assert st == -1
 
 
