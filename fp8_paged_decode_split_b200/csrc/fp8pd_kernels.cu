@@ -580,7 +580,7 @@ __device__ __forceinline__ uint16_t e4m3x2_rn_sat(float lo, float hi) {
 // and, when `store`, into the pools at (page, slot). Lane l owns head-dim
 // bytes [l D/32, (l+1) D/32).
 template <int D>
-__device__ __noinline__ void append_new_token(const DecodeParams& p, int b, int kvh, bool store,
+__device__ __forceinline__ void append_new_token(const DecodeParams& p, int b, int kvh, bool store,
                                               int page, int slot, int r, uint32_t sk, uint32_t sv,
                                               float ks, float vs) {
   constexpr int PER = D / 32;  // 2, 4, 8 or 16 bytes per lane
@@ -698,14 +698,45 @@ __device__ bool prop_assign(const DecodeParams& p, int* scratch, int* red, int h
     int hi = min(nmax, kMaxSplitTiles);
     if (p.nbx > nne) hi = min(hi, (total + (p.nbx - nne) - 1) / (p.nbx - nne));
     hi = max(lo, hi);
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      int cnt = 0;
-      for (int bb = lane; bb < B; bb += 32) cnt += (s_nt[bb] + mid - 1) / mid;
+    if (B <= 64) {
+      // Few sequences: each lane counts one candidate over all sequences (no
+      // cross-lane reduction per step), candidates lo + step * lane with lane
+      // 31 at hi (feasible); the smallest feasible one narrows the bracket
+      // about 31-fold per round. ceil(nt
+      // / c) comes from a float product: for nt < 2^22 (a sequence has at
+      // most 2^17 tiles here) it is within 0.5 of nt / c, so its floor is at
+      // most two below the ceiling and two exact corrections give it.
+      while (lo < hi) {
+        const int step = (hi - lo + 30) / 31;
+        const int c = min(hi, lo + step * lane);
+        const float rc = 1.f / static_cast<float>(c);
+        int cnt = 0;
+        for (int bb = 0; bb < B; ++bb) {
+          const int nt = s_nt[bb];
+          int q = static_cast<int>(static_cast<float>(nt) * rc);
+          q += (q * c < nt);
+          q += (q * c < nt);
+          cnt += q;
+        }
+        const unsigned ok = __ballot_sync(FULL, cnt <= p.nbx);  // never 0: lane 31 is at hi
+        const int first = __ffs(ok) - 1;
+        const int c_first = min(hi, lo + step * first);
+        if (first == 0) hi = lo;
+        else {
+          lo = min(hi, lo + step * (first - 1)) + 1;
+          hi = c_first;
+        }
+      }
+    } else {
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        int cnt = 0;
+        for (int bb = lane; bb < B; bb += 32) cnt += (s_nt[bb] + mid - 1) / mid;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(FULL, cnt, o);
-      if (cnt <= p.nbx) hi = mid;
-      else lo = mid + 1;
+        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(FULL, cnt, o);
+        if (cnt <= p.nbx) hi = mid;
+        else lo = mid + 1;
+      }
     }
     __syncwarp();
     if (lane == 0) red[2 * NW] = lo;
@@ -1213,14 +1244,18 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   // merges the group (or, with a single group, produces the output). With
   // several groups, each group merger then takes a ticket of the (sequence,
   // KV head, head group) and the last one merges the group partials, adding
-  // the sink once. Mergers reset their counters; no block ever waits.
-  __threadfence();
+  // the sink once. Mergers reset their counters; no block ever waits. One
+  // thread fences after the barrier: the barrier orders the block's partial
+  // writes before its fence, and the fence orders them before the ticket.
   __syncthreads();
   int* flag = reinterpret_cast<int*>(misc + C::NW * 8 * 2);
   int* ucnt = p.counters + cnt0;
   const int g = split / kMergeFan;
   const int gsize = min(kMergeFan, S - g * kMergeFan);
-  if (tid == 0) *flag = (atomicAdd(ucnt + 1 + g, 1) == gsize - 1);
+  if (tid == 0) {
+    __threadfence();
+    *flag = (atomicAdd(ucnt + 1 + g, 1) == gsize - 1);
+  }
   __syncthreads();
   if (!*flag) return;
   __threadfence();
@@ -1234,9 +1269,11 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   merge_partials<D, C::NW>(p.part_ml, p.part_o, prow0 + g * kMergeFan, S, gsize, nheads, false,
                            p, b, head0, p.grp_ml, p.grp_o, grow0 + g, NG, wts);
   if (tid == 0) ucnt[1 + g] = 0;
-  __threadfence();
   __syncthreads();
-  if (tid == 0) *flag = (atomicAdd(ucnt, 1) == NG - 1);
+  if (tid == 0) {
+    __threadfence();
+    *flag = (atomicAdd(ucnt, 1) == NG - 1);
+  }
   __syncthreads();
   if (!*flag) return;
   __threadfence();
