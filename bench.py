@@ -552,7 +552,7 @@ def main():
     ap.add_argument("--unfused", action="store_true",
                     help="run fp8_kv_append and the attention call as two launches")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--k-decode", default="bits", choices=["bits", "cvt"],
+    ap.add_argument("--k-decode", default="cvt", choices=["bits", "cvt"],
                     help="E4M3 -> f16 decode of K: bit assembly or hardware cvt")
     ap.add_argument("--splits", type=int, default=0, help="force a split count (0 = planner)")
     ap.add_argument("--schedule", type=int, default=0, choices=[0, 1, 2, 3],

@@ -247,10 +247,13 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
 // Pipeline depth (ring stages per warp) and blocks per SM the register budget
 // targets; compile-time settings, overridable for tuning builds.
 #ifndef FP8PD_NS_D64
-#define FP8PD_NS_D64 6
+#define FP8PD_NS_D64 3
 #endif
 #ifndef FP8PD_NS_D128
 #define FP8PD_NS_D128 3
+#endif
+#ifndef FP8PD_MIN_BLOCKS_D64
+#define FP8PD_MIN_BLOCKS_D64 6
 #endif
 #ifndef FP8PD_MIN_BLOCKS_D128
 #define FP8PD_MIN_BLOCKS_D128 4
@@ -288,7 +291,7 @@ struct Cfg {
   static constexpr int MISC_FLOATS = NW * 8 * 2 + 4;
   static constexpr int SMEM = 1024 /* alignment slack */ + PIPE_BYTES + QFRAG_BYTES + LIST_BYTES +
                               BAR_BYTES + MISC_FLOATS * 4;
-  static constexpr int MIN_BLOCKS = (D == 512) ? 1 : (D == 256) ? 2 : FP8PD_MIN_BLOCKS_D128;
+  static constexpr int MIN_BLOCKS = (D == 512) ? 1 : (D == 256) ? 2 : (D == 128) ? FP8PD_MIN_BLOCKS_D128 : FP8PD_MIN_BLOCKS_D64;
   static_assert(PIPE_BYTES % 1024 == 0, "tiles must stay 1024-byte aligned for the swizzle");
   static_assert(NW * 8 * D * 4 <= PIPE_BYTES, "merge scratch must fit in the ring");
   static_assert(8 * 32 * 4 <= PIPE_BYTES, "merge weights must fit in the ring");
