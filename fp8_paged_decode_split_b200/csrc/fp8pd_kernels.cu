@@ -252,6 +252,12 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
 #ifndef FP8PD_NS_D128
 #define FP8PD_NS_D128 3
 #endif
+#ifndef FP8PD_NS_D256
+#define FP8PD_NS_D256 2
+#endif
+#ifndef FP8PD_NS_D512
+#define FP8PD_NS_D512 2
+#endif
 #ifndef FP8PD_MIN_BLOCKS_D64
 #define FP8PD_MIN_BLOCKS_D64 6
 #endif
@@ -279,7 +285,7 @@ __device__ __forceinline__ uint32_t tile_off(int r, int b) {
 template <int D>
 struct Cfg {
   static constexpr int NW = 4;                                        // warps per block
-  static constexpr int NS = (D == 64) ? FP8PD_NS_D64 : (D == 128) ? FP8PD_NS_D128 : 2;  // ring stages per warp
+  static constexpr int NS = (D == 64) ? FP8PD_NS_D64 : (D == 128) ? FP8PD_NS_D128 : (D == 256) ? FP8PD_NS_D256 : FP8PD_NS_D512;  // ring stages per warp
   static constexpr int TILE = kTileTokens * D;                        // bytes of a K or V tile
   static constexpr int STAGE = 2 * TILE;
   static constexpr int WARP_BYTES = NS * STAGE;
