@@ -230,6 +230,11 @@ bool plan_proportional(int B, int Hq, int Hkv, int D, int ps, int max_pages, int
   const int64_t waves = (static_cast<int64_t>(B) * HX * 2 > slots) ? 2 : 1;
 #endif
   int64_t nbx = (waves * slots + HX - 1) / HX;
+  // By default only in one wave: with a second wave every later block pays
+  // the split search again and the blocks without a split still take slots,
+  // and uniform splits measured faster there (equal-length batches of 64
+  // sequences, and 8 sequences of 131k keys).
+  if (g_opt_schedule.load() == 0 && (waves > 1 || B * m_max > nbx)) return false;
   nbx = std::max<int64_t>(nbx, B * m_max);  // room for every sequence's minimum splits
   nbx = std::min<int64_t>(nbx, std::min<int64_t>(65535, static_cast<int64_t>(B) * fp8pd::kMaxSplits));
   if (nbx < B * m_max) return false;

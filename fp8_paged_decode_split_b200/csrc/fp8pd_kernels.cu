@@ -247,10 +247,13 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
 // Pipeline depth (ring stages per warp) and blocks per SM the register budget
 // targets; compile-time settings, overridable for tuning builds.
 #ifndef FP8PD_NS_D64
-#define FP8PD_NS_D64 3
+#define FP8PD_NS_D64 4
 #endif
 #ifndef FP8PD_NS_D128
 #define FP8PD_NS_D128 3
+#endif
+#ifndef FP8PD_PAIR_D64
+#define FP8PD_PAIR_D64 1
 #endif
 #ifndef FP8PD_NS_D256
 #define FP8PD_NS_D256 2
@@ -259,7 +262,7 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
 #define FP8PD_NS_D512 2
 #endif
 #ifndef FP8PD_MIN_BLOCKS_D64
-#define FP8PD_MIN_BLOCKS_D64 6
+#define FP8PD_MIN_BLOCKS_D64 5
 #endif
 #ifndef FP8PD_MIN_BLOCKS_D128
 #define FP8PD_MIN_BLOCKS_D128 4
@@ -286,6 +289,7 @@ template <int D>
 struct Cfg {
   static constexpr int NW = 4;                                        // warps per block
   static constexpr int NS = (D == 64) ? FP8PD_NS_D64 : (D == 128) ? FP8PD_NS_D128 : (D == 256) ? FP8PD_NS_D256 : FP8PD_NS_D512;  // ring stages per warp
+  static constexpr bool PAIR = (D == 64) && FP8PD_PAIR_D64;           // two tiles per softmax step
   static constexpr int TILE = kTileTokens * D;                        // bytes of a K or V tile
   static constexpr int STAGE = 2 * TILE;
   static constexpr int WARP_BYTES = NS * STAGE;
@@ -406,20 +410,19 @@ struct Acc {
   }
 };
 
-// Attends one 16-token tile already in shared memory (K at sk, V at sv, the
-// swizzled layout of tile_off) for one warp: S = K q'^T on the tensor cores,
-// masking of tokens outside [t0, t1) (or of the whole tile when its page is
-// out of range), the online-softmax update, and O += V^T P with P as an f16
-// hi + lo pair. kfac = score factor of the tile's page (log2 units), vs =
-// its V scale; tok0 = first token of the tile; `full`: every token of the
-// tile is attended (warp-uniform). qfr(kb) gives the q' B-fragment of k16
-// block kb.
-template <int D, bool KCVT, bool VCVT, class QFrag>
-__device__ __forceinline__ void attend_tile(Acc<D>& a, const QFrag& qfr, uint32_t sk, uint32_t sv,
-                                            const uint32_t (&koff)[4], const uint32_t (&voff)[4],
-                                            float kfac, float vs, int tok0, int t0, int t1,
-                                            bool page_ok, bool full, int grp, int qd) {
-  // -- S[token][head] = K q'^T (two independent accumulator chains) --------
+// S = K q'^T of one 16-token tile in shared memory (K at sk, the swizzled
+// layout of tile_off) on the tensor cores, then the masked scores in log2
+// units of this lane: tokens grp / grp + 8 of the tile, heads 2qd / 2qd+1,
+// returned as (x, y, z, w) = (grp, 2qd), (grp, 2qd+1), (grp+8, 2qd),
+// (grp+8, 2qd+1). Tokens outside [t0, t1), or the whole tile when its page
+// is out of range, are -inf. kfac = score factor of the tile's page; `full`:
+// every token is attended (warp-uniform). qfr(kb) gives the q' B-fragment
+// of k16 block kb.
+template <int D, bool KCVT, class QFrag>
+__device__ __forceinline__ float4 tile_scores(const QFrag& qfr, uint32_t sk,
+                                              const uint32_t (&koff)[4], float kfac, int tok0,
+                                              int t0, int t1, bool page_ok, bool full, int grp) {
+  // two independent accumulator chains
   float Sa[4] = {0.f, 0.f, 0.f, 0.f}, Sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int kc = 0; kc < D / 32; ++kc) {
@@ -453,25 +456,29 @@ __device__ __forceinline__ void attend_tile(Acc<D>& a, const QFrag& qfr, uint32_
         mma16816(Sa, a0, a1, a2, a3, b0, b1);
     }
   }
-
-  // -- masked scores (log2 units), online softmax ------------------------
   // A masked row may hold stale or NaN-decoded bytes: select, never multiply.
   const int ta = tok0 + grp, tb = ta + 8;
   const bool va = full || (page_ok && ta >= t0 && ta < t1);
   const bool vb = full || (page_ok && tb >= t0 && tb < t1);
-  const float s00 = va ? (Sa[0] + Sb[0]) * kfac : -CUDART_INF_F;  // token grp,   head 2qd
-  const float s01 = va ? (Sa[1] + Sb[1]) * kfac : -CUDART_INF_F;  // token grp,   head 2qd+1
-  const float s10 = vb ? (Sa[2] + Sb[2]) * kfac : -CUDART_INF_F;  // token grp+8, head 2qd
-  const float s11 = vb ? (Sa[3] + Sb[3]) * kfac : -CUDART_INF_F;  // token grp+8, head 2qd+1
-  float tm0 = fmaxf(s00, s10), tm1 = fmaxf(s01, s11);
+  return make_float4(va ? (Sa[0] + Sb[0]) * kfac : -CUDART_INF_F,
+                     va ? (Sa[1] + Sb[1]) * kfac : -CUDART_INF_F,
+                     vb ? (Sa[2] + Sb[2]) * kfac : -CUDART_INF_F,
+                     vb ? (Sa[3] + Sb[3]) * kfac : -CUDART_INF_F);
+}
+
+// Online-softmax update for new scores whose per-head maxima over this
+// lane's tokens are (tm0, tm1) and whose largest |V scale| is vabs: the
+// running maxima and the V reference scale grow, and l and O are rescaled,
+// only when one of them changes (warp-uniform test).
+template <int D>
+__device__ __forceinline__ void softmax_rescale(Acc<D>& a, float tm0, float tm1, float vabs) {
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, o));
     tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, o));
   }
   const float mn0 = fmaxf(a.m0, tm0), mn1 = fmaxf(a.m1, tm1);
-  const float vabs = fabsf(vs);
-  const bool grow_v = vabs > a.vref;  // warp-uniform: one scale per tile
+  const bool grow_v = vabs > a.vref;  // warp-uniform
   if (grow_v || __any_sync(0xffffffffu, (mn0 > a.m0) || (mn1 > a.m1))) {
     const float c0 = (mn0 > a.m0) ? fast_exp2(a.m0 - mn0) : 1.f;  // exp2(-inf) = 0 for a first max
     const float c1 = (mn1 > a.m1) ? fast_exp2(a.m1 - mn1) : 1.f;
@@ -495,28 +502,41 @@ __device__ __forceinline__ void attend_tile(Acc<D>& a, const QFrag& qfr, uint32_
       a.inv_vref = 1.f / vabs;
     }
   }
+}
+
+// P of one tile: exp2 of the scores against the running maxima, added to
+// the running sums; then P * v_scale / vref as an f16 hi + lo pair, whose PV
+// B fragments are the transposes of the score fragment's 8x8 blocks
+// (movmatrix): bh / bl[0] for tokens 2qd.., bh / bl[1] for 2qd+8...
+template <int D>
+__device__ __forceinline__ void tile_probs(Acc<D>& a, float4 sc, float vs, uint32_t (&bh)[2],
+                                           uint32_t (&bl)[2]) {
   const float mb0 = (a.m0 == -CUDART_INF_F) ? 0.f : a.m0;
   const float mb1 = (a.m1 == -CUDART_INF_F) ? 0.f : a.m1;
-  const float p00 = fast_exp2(s00 - mb0), p01 = fast_exp2(s01 - mb1);
-  const float p10 = fast_exp2(s10 - mb0), p11 = fast_exp2(s11 - mb1);
+  const float p00 = fast_exp2(sc.x - mb0), p01 = fast_exp2(sc.y - mb1);
+  const float p10 = fast_exp2(sc.z - mb0), p11 = fast_exp2(sc.w - mb1);
   a.l0 += p00 + p10;
   a.l1 += p01 + p11;
-
-  // -- P * v_scale / a.vref as f16 hi + lo; the B fragments of the PV MMA are
-  // the transposes of the score fragment's 8x8 blocks (movmatrix).
   const float vsr = vs * a.inv_vref;
   const float w00 = p00 * vsr, w01 = p01 * vsr, w10 = p10 * vsr, w11 = p11 * vsr;
   const uint32_t ha = pack_f16x2(w00, w01), hb = pack_f16x2(w10, w11);
   const float2 fa = unpack_f16x2(ha), fb = unpack_f16x2(hb);
   const uint32_t la = pack_f16x2(w00 - fa.x, w01 - fa.y), lb = pack_f16x2(w10 - fb.x, w11 - fb.y);
-  const uint32_t bh0 = movmatrix_trans(ha), bh1 = movmatrix_trans(hb);  // tokens 2qd.., 2qd+8..
-  const uint32_t bl0 = movmatrix_trans(la), bl1 = movmatrix_trans(lb);
+  bh[0] = movmatrix_trans(ha);
+  bh[1] = movmatrix_trans(hb);
+  bl[0] = movmatrix_trans(la);
+  bl[1] = movmatrix_trans(lb);
+}
 
-  // -- O^T[d][head] += V^T P ---------------------------------------------
-  // ldmatrix.trans of the 32-byte block jb gives lane (g, q) the bytes
-  // (d, d+1), d = 32jb + 2g, of tokens 2q and 2q+1 (reg 0), the same for
-  // d + 16 (reg 1), and for tokens 2q+8, 2q+9 (regs 2, 3). M tile (jb, 0)
-  // rows g / g+8 are d / d+1; M tile (jb, 1) adds 16.
+// O^T[d][head] += V^T P of one tile (V at sv). ldmatrix.trans of the
+// 32-byte block jb gives lane (g, q) the bytes (d, d+1), d = 32jb + 2g, of
+// tokens 2q and 2q+1 (reg 0), the same for d + 16 (reg 1), and for tokens
+// 2q+8, 2q+9 (regs 2, 3). M tile (jb, 0) rows g / g+8 are d / d+1; M tile
+// (jb, 1) adds 16.
+template <int D, bool VCVT>
+__device__ __forceinline__ void tile_pv(Acc<D>& a, uint32_t sv, const uint32_t (&voff)[4],
+                                        const uint32_t (&bh)[2], const uint32_t (&bl)[2], int tok0,
+                                        int t0, int t1, bool page_ok, bool full, int qd) {
   uint32_t vmask_lo = ~0u, vmask_hi = ~0u;
   if (VCVT && !full) {
     // with the hardware cvt a masked row must be zeroed (a NaN byte times
@@ -553,11 +573,52 @@ __device__ __forceinline__ void attend_tile(Acc<D>& a, const QFrag& qfr, uint32_
       e2 = e4m3x2_b02_to_f16x2(vw.w);
       e3 = e4m3x2_b13_to_f16x2(vw.w);
     }
-    mma16816(a.O[jb][0], a0, a1, a2, a3, bh0, bh1);
-    mma16816(a.O[jb][0], a0, a1, a2, a3, bl0, bl1);
-    mma16816(a.O[jb][1], e0, e1, e2, e3, bh0, bh1);
-    mma16816(a.O[jb][1], e0, e1, e2, e3, bl0, bl1);
+    mma16816(a.O[jb][0], a0, a1, a2, a3, bh[0], bh[1]);
+    mma16816(a.O[jb][0], a0, a1, a2, a3, bl[0], bl[1]);
+    mma16816(a.O[jb][1], e0, e1, e2, e3, bh[0], bh[1]);
+    mma16816(a.O[jb][1], e0, e1, e2, e3, bl[0], bl[1]);
   }
+}
+
+// Attends one 16-token tile already in shared memory (K at sk, V at sv) for
+// one warp: S = K q'^T, masking, the online-softmax update, and O += V^T P
+// with P as an f16 hi + lo pair. kfac = score factor of the tile's page
+// (log2 units), vs = its V scale; tok0 = first token of the tile.
+template <int D, bool KCVT, bool VCVT, class QFrag>
+__device__ __forceinline__ void attend_tile(Acc<D>& a, const QFrag& qfr, uint32_t sk, uint32_t sv,
+                                            const uint32_t (&koff)[4], const uint32_t (&voff)[4],
+                                            float kfac, float vs, int tok0, int t0, int t1,
+                                            bool page_ok, bool full, int grp, int qd) {
+  const float4 sc = tile_scores<D, KCVT>(qfr, sk, koff, kfac, tok0, t0, t1, page_ok, full, grp);
+  softmax_rescale<D>(a, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), fabsf(vs));
+  uint32_t bh[2], bl[2];
+  tile_probs<D>(a, sc, vs, bh, bl);
+  tile_pv<D, VCVT>(a, sv, voff, bh, bl, tok0, t0, t1, page_ok, full, qd);
+}
+
+// Two tiles (u = 0, 1) at once: both score blocks, one softmax update (one
+// set of maximum shuffles and one rescale test for 32 keys), then both PV
+// blocks; `between` runs after the first tile's PV (its stage is free then).
+template <int D, bool KCVT, bool VCVT, class QFrag, class Between>
+__device__ __forceinline__ void attend_pair(Acc<D>& a, const QFrag& qfr, const uint32_t (&sk)[2],
+                                            const uint32_t (&koff)[4], const uint32_t (&voff)[4],
+                                            const float (&kfac)[2], const float (&vs)[2],
+                                            const int (&tok0)[2], int t0, int t1,
+                                            const bool (&page_ok)[2], const bool (&full)[2],
+                                            int grp, int qd, const Between& between) {
+  constexpr int TILE = kTileTokens * D;
+  const float4 s0 = tile_scores<D, KCVT>(qfr, sk[0], koff, kfac[0], tok0[0], t0, t1, page_ok[0],
+                                         full[0], grp);
+  const float4 s1 = tile_scores<D, KCVT>(qfr, sk[1], koff, kfac[1], tok0[1], t0, t1, page_ok[1],
+                                         full[1], grp);
+  softmax_rescale<D>(a, fmaxf(fmaxf(s0.x, s0.z), fmaxf(s1.x, s1.z)),
+                     fmaxf(fmaxf(s0.y, s0.w), fmaxf(s1.y, s1.w)), fmaxf(fabsf(vs[0]), fabsf(vs[1])));
+  uint32_t bh0[2], bl0[2], bh1[2], bl1[2];
+  tile_probs<D>(a, s0, vs[0], bh0, bl0);
+  tile_probs<D>(a, s1, vs[1], bh1, bl1);
+  tile_pv<D, VCVT>(a, sk[0] + TILE, voff, bh0, bl0, tok0[0], t0, t1, page_ok[0], full[0], qd);
+  between();
+  tile_pv<D, VCVT>(a, sk[1] + TILE, voff, bh1, bl1, tok0[1], t0, t1, page_ok[1], full[1], qd);
 }
 
 // Keys sequence b attends over: its length, or with a fused append its
@@ -1109,8 +1170,64 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   int stage = 0;
   uint32_t phase = 0;
   int tok0 = (tile_first + warp) * kTileTokens;
+  if constexpr (C::PAIR) {
+    // Two tiles per step while two are left (one softmax update per 32 keys;
+    // the copy into the first tile's stage is issued once its PV is done).
 #pragma unroll 1
-  for (int j = 0; j < my_tiles; ++j, tok0 += C::NW * kTileTokens) {
+    for (int j = 0; j + 1 < my_tiles; j += 2, tok0 += 2 * C::NW * kTileTokens) {
+      const int st1 = (stage + 1 == C::NS) ? 0 : stage + 1;
+      const uint32_t ph1 = (stage + 1 == C::NS) ? (phase ^ 1u) : phase;
+      if (!mbar_wait(wbar + 8 * stage, phase) || !mbar_wait(wbar + 8 * st1, ph1)) {
+        if (lane == 0) raise_flag(FP8PD_FLAG_TIMEOUT);
+        ok_all = false;
+        break;
+      }
+      if (j == 0) cp_async_wait_all();  // this lane's scale copies
+      __syncwarp();
+      {
+        const int nj = j + C::NS - 1;
+        if (nj < my_tiles) issue(went[nj], stage == 0 ? C::NS - 1 : stage - 1);
+      }
+      const int st0 = stage;
+      uint32_t sk[2];
+      float kfac[2], vsc[2];
+      int tk[2];
+      bool pok[2], full[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int jj = j + u;
+        tk[u] = tok0 + u * C::NW * kTileTokens;
+        pok[u] = went[jj] >= 0;
+        full[u] = pok[u] && tk[u] >= t0 && tk[u] + kTileTokens <= t1;
+        sk[u] = wpipe + (u ? st1 : st0) * C::STAGE;
+        kfac[u] = score_base * wks[jj];
+        vsc[u] = wvs[jj];
+        if (p.append && pok[u] && L - 1 >= tk[u] && L - 1 < tk[u] + kTileTokens) {
+          // the new token: quantized here, stored by head group 0, attended by all
+          const int r = L - 1 - tk[u];
+          append_new_token<D>(p, b, kvh, hg == 0, went[jj] >> 4,
+                              (went[jj] & 15) * kTileTokens + r, r, sk[u], sk[u] + C::TILE,
+                              wks[jj], vsc[u]);
+          __syncwarp();
+        }
+      }
+      stage = st1;
+      if (++stage == C::NS) {
+        stage = 0;
+        phase = ph1 ^ 1u;
+      } else {
+        phase = ph1;
+      }
+      attend_pair<D, KCVT, VCVT>(acc, qfr, sk, koff, voff, kfac, vsc, tk, t0, t1, pok, full, grp,
+                                 qd, [&]() {
+                                   const int nj = j + C::NS;
+                                   if (nj < my_tiles) issue(went[nj], st0);
+                                 });
+    }
+  }
+#pragma unroll 1
+  for (int j = C::PAIR ? (my_tiles & ~1) : 0; ok_all && j < my_tiles;
+       ++j, tok0 += C::NW * kTileTokens) {
     if (!mbar_wait(wbar + 8 * stage, phase)) {
       if (lane == 0) raise_flag(FP8PD_FLAG_TIMEOUT);
       ok_all = false;

@@ -168,7 +168,8 @@ enum {
  * group, cut into equal block ranges that cross sequence boundaries, and the
  * block's warps share its range through a queue. The planner takes
  * proportional splits for full attention and windows of at least 2,048 keys
- * when there is enough work, uniform splits otherwise.
+ * when there is enough work and their grid fits one wave of the device,
+ * uniform splits otherwise.
  * The partial results and the ticket counters live
  * in a library-owned per-device workspace: it grows on demand outside stream
  * capture; under capture a call that would need to grow it fails with

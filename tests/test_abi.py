@@ -221,14 +221,17 @@ def test_planner_fills_the_device_with_enough_work_per_split(F, split_schedule):
 
 def test_planner_default_schedule(F):
     """The planner's own choice: proportional splits for full attention and
-    long windows with enough work, uniform splits otherwise; the segment
-    kernel only on request. Without a GPU it assumes 148 SMs."""
+    long windows with enough work when their grid is one wave, uniform splits
+    otherwise; the segment kernel only on request. Without a GPU it assumes
+    148 SMs and the launch-bound blocks per SM."""
     assert _plan(F, 32, 32, 8, 128, 16, 257)["schedule"] == 3           # Llama-like
-    assert _plan(F, 64, 64, 8, 64, 16, 513)["schedule"] == 3            # gpt-oss-like, full
-    assert _plan(F, 64, 64, 8, 64, 16, 513, window=4096)["schedule"] == 3
+    assert _plan(F, 1, 64, 8, 128, 64, 2049)["schedule"] == 3           # one 131k-key sequence
+    assert _plan(F, 16, 16, 2, 512, 32, 513)["schedule"] == 3           # any head dim
+    assert _plan(F, 64, 64, 8, 64, 16, 513)["schedule"] == 1            # gpt-oss-like: two waves
+    assert _plan(F, 64, 64, 8, 64, 16, 513, window=4096)["schedule"] == 1
+    assert _plan(F, 8, 64, 8, 128, 64, 2049)["schedule"] == 1           # 8 x 131k keys: > 1 wave
     assert _plan(F, 64, 64, 8, 64, 16, 513, window=128)["schedule"] == 1
     assert _plan(F, 1, 8, 2, 64, 16, 16)["schedule"] == 1               # too little work
-    assert _plan(F, 16, 16, 2, 512, 32, 513)["schedule"] == 3           # any head dim
     assert _plan(F, 1025, 8, 8, 128, 16, 400)["schedule"] == 1          # more than 1,024 sequences
 
 
