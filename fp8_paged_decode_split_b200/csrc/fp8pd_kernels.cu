@@ -1087,26 +1087,44 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   // bytes (0,1) and (2,3): k = 2q -> +0, 2q+1 -> +1, 2q+8 -> +2, 2q+9 -> +3;
   // bit-assembly K pairs (0,2) and (1,3): k = 2q -> +0, 2q+1 -> +2, 2q+8 -> +1,
   // 2q+9 -> +3.
+  auto max4 = [](uint2 v) -> float {
+    return fmaxf(fmaxf(fabsf(__uint_as_float(v.x << 16)), fabsf(__uint_as_float(v.x & 0xFFFF0000u))),
+                 fmaxf(fabsf(__uint_as_float(v.y << 16)), fabsf(__uint_as_float(v.y & 0xFFFF0000u))));
+  };
   float qmax = 0.f;
   if constexpr (C::Q_IN_SMEM) {
-    if (q_head_ok) {
-#pragma unroll 8
-      for (int e = 0; e < D / 4; ++e) {
-        const int d = 16 * (e >> 2) + 4 * qd + (e & 3);
-        qmax = fmaxf(qmax, fabsf(bf16_bits_to_float(__ldg(qrow + (int64_t)d * p.q_sd))));
+    // this warp's k16 blocks (kb = warp mod NW): one 8-byte load of raw bf16
+    // pairs per lane and block, all in flight together, parked in the
+    // fragment slots they become; the block then agrees on max|q|
+#pragma unroll
+    for (int i = 0; i < KB / C::NW; ++i) {
+      const int kb = warp + C::NW * i;
+      const int d = 16 * kb + 4 * qd;
+      uint2 v = make_uint2(0u, 0u);
+      if (q_head_ok) {
+        if (p.q_vec) {
+          v = __ldg(reinterpret_cast<const uint2*>(qrow + d));
+        } else {
+          const uint32_t e0 = __ldg(qrow + (int64_t)(d + 0) * p.q_sd);
+          const uint32_t e1 = __ldg(qrow + (int64_t)(d + 1) * p.q_sd);
+          const uint32_t e2 = __ldg(qrow + (int64_t)(d + 2) * p.q_sd);
+          const uint32_t e3 = __ldg(qrow + (int64_t)(d + 3) * p.q_sd);
+          v = make_uint2(e0 | (e1 << 16), e2 | (e3 << 16));
+        }
       }
+      qfrag_s[kb * 32 + lane] = v;
+      qmax = fmaxf(qmax, max4(v));
     }
+    qmax = warp_max(qmax);
+    if (lane == 0) misc[warp] = qmax;  // free until the warps merge
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < C::NW; ++w) qmax = fmaxf(qmax, misc[w]);
   } else {
 #pragma unroll
-    for (int kb = 0; kb < KB; ++kb) {
-      const uint2 v = qraw[kb];
-      qmax = fmaxf(qmax, fmaxf(fmaxf(fabsf(__uint_as_float(v.x << 16)),
-                                     fabsf(__uint_as_float(v.x & 0xFFFF0000u))),
-                               fmaxf(fabsf(__uint_as_float(v.y << 16)),
-                                     fabsf(__uint_as_float(v.y & 0xFFFF0000u)))));
-    }
+    for (int kb = 0; kb < KB; ++kb) qmax = fmaxf(qmax, max4(qraw[kb]));
+    qmax = warp_max(qmax);
   }
-  qmax = warp_max(qmax);
   // q' = q * 2^(15 - e) puts max|q'| in [2^14, 2^15): exact in f16 for every
   // element above max|q| * 2^-28 (bf16 has 8 significant bits).
   int qe = 0;
@@ -1122,15 +1140,12 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   for (int kb = 0; kb < KB; ++kb) {
     float x0, x1, x2, x3;
     if constexpr (C::Q_IN_SMEM) {
-      if ((kb & 3) != warp) continue;  // the four warps share the work
-      const int d = 16 * kb + 4 * qd;
-      auto qv = [&](int dd) -> float {
-        return q_head_ok ? bf16_bits_to_float(__ldg(qrow + (int64_t)dd * p.q_sd)) : 0.f;
-      };
-      x0 = qv(d);
-      x1 = qv(d + 1);
-      x2 = qv(d + 2);
-      x3 = qv(d + 3);
+      if ((kb % C::NW) != warp) continue;  // this warp's blocks, converted in place
+      const uint2 v = qfrag_s[kb * 32 + lane];
+      x0 = __uint_as_float(v.x << 16);
+      x1 = __uint_as_float(v.x & 0xFFFF0000u);
+      x2 = __uint_as_float(v.y << 16);
+      x3 = __uint_as_float(v.y & 0xFFFF0000u);
     } else {
       const uint2 v = qraw[kb];
       x0 = __uint_as_float(v.x << 16);
