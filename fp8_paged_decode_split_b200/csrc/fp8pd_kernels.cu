@@ -1542,6 +1542,7 @@ __global__ void __launch_bounds__(SegCfg<D>::NT, 1)
   int* s_ndef = s_misc + 35;                               // merges won by this block's tickets
   int* s_def = s_misc + 36;                                // [2] their sequences
   int* s_seg = s_misc + 40;                                // [kSegAsync] sequences of async ends
+  float* s_qmax = reinterpret_cast<float*>(s_misc + 48);   // [NW] q maxima (head dim 512)
   int* s_len = s_misc + 64;                                // [B] attended keys
   int* s_pre = s_len + p.B;                                // [B + 1] tile prefix sums
 
@@ -1753,44 +1754,55 @@ __global__ void __launch_bounds__(SegCfg<D>::NT, 1)
   // All warps call it together when Q_IN_SMEM (they share the fragments).
   auto load_q = [&](int b) {
     const uint16_t* qrow = p.q + (int64_t)b * p.q_sb + (int64_t)(head0 + (q_head_ok ? grp : 0)) * p.q_sh;
-    auto qv = [&](int d) -> float {
-      return q_head_ok ? bf16_bits_to_float(__ldg(qrow + (int64_t)d * p.q_sd)) : 0.f;
+    auto raw = [&](int kb) -> uint2 {  // bf16 entries 16kb + 4qd .. +3 of this lane's head
+      const int d = 16 * kb + 4 * qd;
+      uint2 v = make_uint2(0u, 0u);
+      if (q_head_ok) {
+        if (p.q_vec) {
+          v = __ldg(reinterpret_cast<const uint2*>(qrow + d));
+        } else {
+          const uint32_t x0 = __ldg(qrow + (int64_t)(d + 0) * p.q_sd);
+          const uint32_t x1 = __ldg(qrow + (int64_t)(d + 1) * p.q_sd);
+          const uint32_t x2 = __ldg(qrow + (int64_t)(d + 2) * p.q_sd);
+          const uint32_t x3 = __ldg(qrow + (int64_t)(d + 3) * p.q_sd);
+          v = make_uint2(x0 | (x1 << 16), x2 | (x3 << 16));
+        }
+      }
+      return v;
+    };
+    auto max4 = [](uint2 v) -> float {
+      return fmaxf(fmaxf(fabsf(__uint_as_float(v.x << 16)), fabsf(__uint_as_float(v.x & 0xFFFF0000u))),
+                   fmaxf(fabsf(__uint_as_float(v.y << 16)), fabsf(__uint_as_float(v.y & 0xFFFF0000u))));
     };
     float qmax = 0.f;
     if constexpr (C::Q_IN_SMEM) {
-#pragma unroll 8
-      for (int e = 0; e < D / 4; ++e) qmax = fmaxf(qmax, fabsf(qv(16 * (e >> 2) + 4 * qd + (e & 3))));
+      // this warp's k16 blocks (kb = warp mod NW), parked raw in the fragment
+      // slots they become; the block agrees on max|q| (all warps call this)
+#pragma unroll
+      for (int i = 0; i < KB / NW; ++i) {
+        const int kb = warp + NW * i;
+        const uint2 v = raw(kb);
+        qfrag_s[kb * 32 + lane] = v;
+        qmax = fmaxf(qmax, max4(v));
+      }
+      qmax = warp_max(qmax);
+      if (lane == 0) s_qmax[warp] = qmax;
+      __syncthreads();
+#pragma unroll
+      for (int w = 0; w < NW; ++w) qmax = fmaxf(qmax, s_qmax[w]);
+      __syncthreads();  // s_qmax is read before the next call writes it
     } else {
       uint2 qraw[KB];
 #pragma unroll
-      for (int kb = 0; kb < KB; ++kb) {
-        const int d = 16 * kb + 4 * qd;
-        uint2 v = make_uint2(0u, 0u);
-        if (q_head_ok) {
-          if (p.q_vec) {
-            v = __ldg(reinterpret_cast<const uint2*>(qrow + d));
-          } else {
-            const uint32_t x0 = __ldg(qrow + (int64_t)(d + 0) * p.q_sd);
-            const uint32_t x1 = __ldg(qrow + (int64_t)(d + 1) * p.q_sd);
-            const uint32_t x2 = __ldg(qrow + (int64_t)(d + 2) * p.q_sd);
-            const uint32_t x3 = __ldg(qrow + (int64_t)(d + 3) * p.q_sd);
-            v = make_uint2(x0 | (x1 << 16), x2 | (x3 << 16));
-          }
-        }
-        qraw[kb] = v;
-      }
+      for (int kb = 0; kb < KB; ++kb) qraw[kb] = raw(kb);
 #pragma unroll
       for (int kb = 0; kb < KB; ++kb) {
-        const uint2 v = qraw[kb];
-        qmax = fmaxf(qmax, fmaxf(fmaxf(fabsf(__uint_as_float(v.x << 16)),
-                                       fabsf(__uint_as_float(v.x & 0xFFFF0000u))),
-                                 fmaxf(fabsf(__uint_as_float(v.y << 16)),
-                                       fabsf(__uint_as_float(v.y & 0xFFFF0000u)))));
-        qf[kb][0] = v.x;  // raw bf16 pairs until the scale is known
-        qf[kb][1] = v.y;
+        qmax = fmaxf(qmax, max4(qraw[kb]));
+        qf[kb][0] = qraw[kb].x;  // raw bf16 pairs until the scale is known
+        qf[kb][1] = qraw[kb].y;
       }
+      qmax = warp_max(qmax);
     }
-    qmax = warp_max(qmax);
     int qe = 0;
     if (qmax > 0.f && isfinite(qmax)) frexpf(qmax, &qe);
     qe = max(qe, -111);
@@ -1798,20 +1810,15 @@ __global__ void __launch_bounds__(SegCfg<D>::NT, 1)
     score_base = p.sm_scale_log2 * (KCVT ? 1.f : 256.f) / qmul;
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb) {
-      float x0, x1, x2, x3;
+      uint2 v;
       if constexpr (C::Q_IN_SMEM) {
-        if ((kb % NW) != warp) continue;  // the warps share the work
-        const int d = 16 * kb + 4 * qd;
-        x0 = qv(d);
-        x1 = qv(d + 1);
-        x2 = qv(d + 2);
-        x3 = qv(d + 3);
+        if ((kb % NW) != warp) continue;  // this warp's blocks, converted in place
+        v = qfrag_s[kb * 32 + lane];
       } else {
-        x0 = __uint_as_float(qf[kb][0] << 16);
-        x1 = __uint_as_float(qf[kb][0] & 0xFFFF0000u);
-        x2 = __uint_as_float(qf[kb][1] << 16);
-        x3 = __uint_as_float(qf[kb][1] & 0xFFFF0000u);
+        v = make_uint2(qf[kb][0], qf[kb][1]);
       }
+      const float x0 = __uint_as_float(v.x << 16), x1 = __uint_as_float(v.x & 0xFFFF0000u);
+      const float x2 = __uint_as_float(v.y << 16), x3 = __uint_as_float(v.y & 0xFFFF0000u);
       uint32_t r0, r1;
       if constexpr (KCVT) {
         r0 = pack_f16x2(x0 * qmul, x1 * qmul);
