@@ -1,9 +1,10 @@
 """GPU: every workload at full size, in the launch configuration the benchmark
 times, against the oracle on sampled outputs.
 
-The benchmark's step is used as is: the split planner's default choice, the
-bit-assembly decode of K and the hardware decode of V, the append (where the
-workload has one) followed by attention. The oracle cannot afford every
+The benchmark's step is used as is (bench.Step): the planner's default
+schedule, the hardware decode of K and V, and, where the workload has an
+append, the fused append + attention launch (and, as a second case, the
+append and attention calls on their own). The oracle cannot afford every
 output at these sizes, so a few sequences are sampled (first, last and one
 drawn from a seeded generator), and for each the pages it uses are gathered
 into a small pool that the oracle reads in full: all query heads of the
@@ -27,10 +28,10 @@ pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 def F(cuda_device):
     import fp8_paged_decode_split_b200 as F
     F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
-    F.fp8pd_set_option(F.OPT_K_DECODE, 0)     # the benchmark's default decode of K
+    F.fp8pd_set_option(F.OPT_SCHEDULE, 0)
+    F.fp8pd_set_option(F.OPT_K_DECODE, 1)     # the benchmark's default decodes
     F.fp8pd_set_option(F.OPT_V_DECODE, 1)
-    yield F
-    F.fp8pd_set_option(F.OPT_K_DECODE, 1)
+    return F
 
 
 def _sampled_sequences(B: int, seed: int) -> list:
@@ -49,9 +50,12 @@ def _sub_pool(layer, b: int, n_pages: int):
     return kp, vp, ks, vs
 
 
-@pytest.mark.parametrize("name", ["llama", "gptoss_w128", "gptoss_full", "mixed", "long_b1",
-                                  "long_b8"])
-def test_full_size_step_matches_oracle_on_sampled_sequences(F, cuda_device, name):
+@pytest.mark.parametrize("name,fused", [("llama", True), ("llama", False), ("gptoss_w128", True),
+                                        ("gptoss_full", True), ("mixed", True),
+                                        ("long_b1", True), ("long_b1", False),
+                                        ("long_b8", True)])
+def test_full_size_step_matches_oracle_on_sampled_sequences(F, cuda_device, name, fused):
+    import bench
     case = W.make_case(name, cuda_device)
     spec = case.spec
     seqs = _sampled_sequences(spec.B, 1000 + spec.seed)
@@ -65,17 +69,14 @@ def test_full_size_step_matches_oracle_on_sampled_sequences(F, cuda_device, name
             before[li] = {b: tuple(np_(t).copy() for t in _sub_pool(layer, b, n_pages[b])[:2])
                           for b in seqs}
 
-    outs = []
-    for layer in case.layers:                 # the benchmark's step, layer by layer
-        if spec.append:
-            F.fp8_kv_append(layer.k_new, layer.v_new, layer.k_pages, layer.v_pages,
-                            layer.k_scale, layer.v_scale, layer.block_table, case.positions)
-        outs.append(F.fp8_paged_decode_attention(
-            layer.q, layer.k_pages, layer.v_pages, layer.k_scale, layer.v_scale,
-            layer.block_table, case.attend_lens, window=layer.window, sinks=layer.sinks,
-            sm_scale=layer.sm_scale))
+    for layer in case.layers:
+        layer.out = torch.empty(layer.q.shape, dtype=torch.float32, device=cuda_device)
+    step = bench.Step(F, case, fused)          # the benchmark's step, every layer
+    step.run()
     torch.cuda.synchronize()
     assert F.fp8pd_check_errors() == 0
+    assert step.fused == (fused and spec.append)
+    outs = [layer.out for layer in case.layers]
 
     worst = 0.0
     for li, layer in enumerate(case.layers):
@@ -98,4 +99,4 @@ def test_full_size_step_matches_oracle_on_sampled_sequences(F, cuda_device, name
             assert np.all(np.isfinite(got[b]))
             assert err.max() <= ATOL_REL, f"{name} layer {li} seq {b}: max rel err {err.max():.3g}"
             worst = max(worst, float(err.max()))
-    print(f"{name}: sequences {seqs}, worst error {worst:.3g}")
+    print(f"{name} fused={step.fused}: sequences {seqs}, worst error {worst:.3g}")
