@@ -341,25 +341,47 @@ __device__ void merge_partials(const float* ml, const float* o, int64_t row0, in
     }
   }
   __syncthreads();
-  for (int it = tid; it < nheads * (D / 4); it += NW * 32) {
-    const int n = it / (D / 4);
-    const int d = (it - n * (D / 4)) * 4;
-    const float* po = o + (row0 + n * head_rows) * D + d;
-    const float* wn = wts + n * 32;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  // two output entries per thread and pass, so that both entries' loads of
+  // a group of partials are in flight together
+  const int items = nheads * (D / 4);
+  for (int it0 = tid; it0 < items; it0 += 2 * NW * 32) {
+    int n[2], d[2];
+    const float* po[2];
+    const float* wn[2];
+    bool ok[2];
+    float4 acc[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int it = it0 + u * NW * 32;
+      ok[u] = it < items;
+      const int itc = ok[u] ? it : it0;
+      n[u] = itc / (D / 4);
+      d[u] = (itc - n[u] * (D / 4)) * 4;
+      po[u] = o + (row0 + n[u] * head_rows) * D + d[u];
+      wn[u] = wts + n[u] * 32;
+      acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 #pragma unroll 8
     for (int s = 0; s < K; ++s) {
-      const float ws = wn[s];
-      const float4 v = ldcg4(po + (int64_t)s * D);
-      acc.x += ws * v.x;
-      acc.y += ws * v.y;
-      acc.z += ws * v.z;
-      acc.w += ws * v.w;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float ws = wn[u][s];
+        const float4 v = ldcg4(po[u] + (int64_t)s * D);
+        acc[u].x += ws * v.x;
+        acc[u].y += ws * v.y;
+        acc[u].z += ws * v.z;
+        acc[u].w += ws * v.w;
+      }
     }
-    if (final)
-      *reinterpret_cast<float4*>(p.out + (int64_t)b * p.o_sb + (int64_t)(head0 + n) * p.o_sh + d) = acc;
-    else
-      *reinterpret_cast<float4*>(dst_o + (dst_row0 + n * dst_head_rows) * D + d) = acc;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (!ok[u]) continue;
+      if (final)
+        *reinterpret_cast<float4*>(p.out + (int64_t)b * p.o_sb + (int64_t)(head0 + n[u]) * p.o_sh +
+                                   d[u]) = acc[u];
+      else
+        *reinterpret_cast<float4*>(dst_o + (dst_row0 + n[u] * dst_head_rows) * D + d[u]) = acc[u];
+    }
   }
 }
 
