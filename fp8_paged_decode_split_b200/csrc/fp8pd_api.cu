@@ -295,11 +295,13 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
     S = std::min<int64_t>(s_max, (2 * slots) / units);
     S = std::max<int64_t>(S, 1);
     // A second wave that the splits cannot fill costs a whole split time with
-    // part of the device idle: when one wave of at least half the slots is
-    // possible, take it (a sliding layer of 128 units: 2 splits per unit in
-    // one wave instead of 3 in 1.3 waves).
+    // part of the device idle: when one wave of at least two splits per unit
+    // fills at least half the slots, take it (a sliding layer of 128 units:
+    // 2 splits per unit in one wave instead of 3 in 1.3 waves). With a single
+    // split per unit the blocks are too coarse to even out over the SMs
+    // (gpt-oss full: 1 split per unit measured slower than 2).
     const int64_t one = std::min<int64_t>(s_max, slots / units);
-    if (units * S > slots && one >= std::max<int64_t>(1, s_min) && 2 * units * one >= slots) S = one;
+    if (units * S > slots && one >= std::max<int64_t>(2, s_min) && 2 * units * one >= slots) S = one;
   }
   S = std::max<int64_t>(S, s_min);
   const int64_t chunk = (pages + S - 1) / S;
