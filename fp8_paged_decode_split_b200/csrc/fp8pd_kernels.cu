@@ -3,10 +3,13 @@
 // Method (the "FP8 paged attention for MoE serving" solution page, sections
 // "Why it happens" and "Expected result"): flash-decode over a paged E4M3
 // KV cache with a grid over (sequence, KV head, split), E4M3 decoded in
-// registers by bit assembly, scales read at their natural shape, the query
-// heads of one KV head packed so each K/V byte is read once, online softmax
-// with a sliding window and sink logits, and a log-sum-exp combine of the
-// splits.
+// registers (exactly, by the hardware cvt or by bit assembly), scales read
+// at their natural shape, the query heads of one KV head packed so each K/V
+// byte is read once, online softmax with a sliding window and sink logits,
+// and a log-sum-exp combine of the splits. With a fused append (the
+// "Lecture 8 -- Inference Path" page, "In-kernel KV cache update") the block
+// holding a sequence's new position quantizes the new token, stores it and
+// attends it.
 //
 // Design on B200:
 // * One thread block = one (sequence b, KV head h, group of <= 8 query
@@ -15,7 +18,7 @@
 //   TMA (one cp.async.bulk.tensor per K or V tile, issued by one lane, no
 //   multicast) into a private multi-stage ring completed on mbarriers (no
 //   block-wide barrier in the main loop) and keeps its own online-softmax
-//   state. The warps are
+//   state (at head dim 64, two tiles per softmax step). The warps are
 //   merged once at the end; when the keys are split over several blocks the
 //   last block of a (sequence, KV head, head group) to finish merges the
 //   splits (a ticket counter, never a wait), so one launch does the call.
