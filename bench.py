@@ -28,6 +28,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -128,7 +129,7 @@ class ClockSampler:
         except Exception:
             self.index = str(device.index or 0)
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"fp8pd_clocks_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
