@@ -17,4 +17,6 @@ from .fp8pd_oracle import (  # noqa: F401
     kv_append,
     paged_decode_attention,
     quantize,
+    quantize_per_token,
+    token_scale,
 )

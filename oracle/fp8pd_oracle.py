@@ -34,7 +34,11 @@ Readings of the pages (each is listed with its reason in the design notes):
 * token t of sequence b lives in physical page block_table[b, t // ps] at
   slot t % ps (P2 "Paged KV cache").
 * a K/V scale is indexed by the physical page id and the KV head; a
-  per-KV-head scale is the same array broadcast over pages.
+  per-KV-head scale is the same array broadcast over pages. The
+  per-token-per-head form (P1 "Supported scope", ``quantize_kv_fp8``) keeps
+  one scale per stored (page, slot, KV head), shaped like the cache without
+  its last axis, and is max|x| / 448 of that token and head in float32 (an
+  all-zero row takes scale 1); the append writes it with the codes.
 * empty attention (no keys, no sink) returns 0.
 """
 
@@ -139,17 +143,44 @@ def quantize(x, scale) -> np.ndarray:
     return e4m3_encode(quot.astype(np.float64))
 
 
+def token_scale(x) -> np.ndarray:
+    """Per-token-per-head scale of ``x`` [..., D]: max_d |x| / 448 in float32.
+
+    P1 "Supported scope" names ``quantize_kv_fp8`` as per-token-per-head E4M3
+    with an fp32 scale; the scale that maps each row's largest magnitude onto
+    the largest finite E4M3 value (448) is the plainest reading. The maximum
+    skips NaN entries; a row whose maximum is 0 takes scale 1 (its codes are
+    then signed zeros). The division is IEEE float32.
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.fmax.reduce(np.abs(x32), axis=-1)          # fmax: NaN entries are skipped
+    amax = np.where(np.isnan(amax), np.float32(0.0), amax).astype(np.float32)
+    with np.errstate(over="ignore"):
+        s = np.divide(amax, np.float32(E4M3_MAX), dtype=np.float32)
+    return np.where(amax == 0, np.float32(1.0), s).astype(np.float32)
+
+
+def quantize_per_token(x) -> tuple[np.ndarray, np.ndarray]:
+    """(codes, scales) of ``x`` [..., D] with one scale per row (token, head):
+    scales = :func:`token_scale`, codes = :func:`quantize` of x / scale."""
+    s = token_scale(x)
+    return quantize(x, s[..., None]), s
+
+
 # ---------------------------------------------------------------------------
 # Paged gather, attention and append
 # ---------------------------------------------------------------------------
 
-def _scale_of(scale: np.ndarray, page: np.ndarray, head: int) -> np.ndarray:
-    """Scale for (physical page, KV head): ``scale`` is [Hkv] (per KV head)
-    or [num_pages, Hkv] (per physical page and KV head)."""
+def _scale_of(scale: np.ndarray, page: np.ndarray, slot: np.ndarray, head: int) -> np.ndarray:
+    """Scale of the token stored at (physical page, slot) for KV head ``head``:
+    ``scale`` is [Hkv] (per KV head), [num_pages, Hkv] (per physical page and
+    KV head) or [num_pages, ps, Hkv] (per stored token and KV head)."""
     scale = np.asarray(scale)
     if scale.ndim == 1:
         return np.full(np.shape(page), np.float64(scale[head]))
-    return scale[page, head].astype(np.float64)
+    if scale.ndim == 2:
+        return scale[page, head].astype(np.float64)
+    return scale[page, slot, head].astype(np.float64)
 
 
 def gather_tokens(pages: np.ndarray, block_table_row: np.ndarray, positions: np.ndarray,
@@ -179,8 +210,8 @@ def paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_table, s
     """Single-query attention over a paged E4M3 KV cache, float64.
 
     q [B, Hq, D] (bf16 values given as floats), k_pages / v_pages
-    [num_pages, ps, Hkv, D] uint8 codes, k_scale / v_scale [Hkv] or
-    [num_pages, Hkv] float32, block_table [B, max_pages] int32,
+    [num_pages, ps, Hkv, D] uint8 codes, k_scale / v_scale [Hkv],
+    [num_pages, Hkv] or [num_pages, ps, Hkv] float32, block_table [B, max_pages] int32,
     seq_lens [B] = number of keys 0..L-1 visible to the query,
     sinks [Hq] float32 or None. Returns out [B, Hq, D] float64.
 
@@ -188,7 +219,7 @@ def paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_table, s
       s_t  = sm_scale * sum_d q[b,hq,d] * K(t,d)
       M    = max(max_t s_t, sink)
       out  = sum_t exp(s_t - M) V(t) / (sum_t exp(s_t - M) + exp(sink - M))
-    where K(t,d) = decode(code) * k_scale(page(t), h). This is plain softmax
+    where K(t,d) = decode(code) * k_scale(page(t), slot(t), h). This is plain softmax
     attention over the dequantized values (P1 "Smallest correct example"),
     with the window, sinks and scale of P1 "Expected result".
 
@@ -216,8 +247,9 @@ def paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_table, s
                 continue
             kc, phys = gather_tokens(k_pages, block_table[b], positions, h)
             vc, _ = gather_tokens(v_pages, block_table[b], positions, h)
-            K = e4m3_decode(kc) * _scale_of(k_scale, phys, h)[:, None]
-            V = e4m3_decode(vc) * _scale_of(v_scale, phys, h)[:, None]
+            slots = positions % k_pages.shape[1]
+            K = e4m3_decode(kc) * _scale_of(k_scale, phys, slots, h)[:, None]
+            V = e4m3_decode(vc) * _scale_of(v_scale, phys, slots, h)[:, None]
             for hq in heads:
                 s = sm * (K @ q[b, hq])
                 sink = None if sinks is None else float(sinks[hq])
@@ -237,10 +269,13 @@ def kv_append(k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table, pos
 
     k_new / v_new [B, Hkv, D] (bf16 values as floats), pages
     [num_pages, ps, Hkv, D] uint8 (numpy arrays, written in place), scales
-    [Hkv] or [num_pages, Hkv] float32 (read only), positions [B].
+    [Hkv], [num_pages, Hkv] or [num_pages, ps, Hkv] float32, positions [B].
     Token position p of sequence b goes to page block_table[b, p // ps], slot
-    p % ps, as code = E4M3(float32(x) / scale(page, h)) (P1 "Supported scope",
-    the one-launch T=1 append; P2 "In-kernel KV cache update").
+    p % ps, as code = E4M3(float32(x) / scale) (P1 "Supported scope", the
+    one-launch T=1 append; P2 "In-kernel KV cache update"). A per-head or
+    per-page scale is read only. A per-token scale is the new token's own
+    (:func:`token_scale` of its D values, per KV head) and is written to
+    ``scale[page, slot, h]`` with the codes.
     """
     B, Hkv, _ = np.shape(k_new)
     ps = k_pages.shape[1]
@@ -249,7 +284,9 @@ def kv_append(k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table, pos
         page = int(block_table[b][p // ps])
         slot = p % ps
         for h in range(Hkv):
-            ks = _scale_of(k_scale, np.array(page), h)
-            vs = _scale_of(v_scale, np.array(page), h)
-            k_pages[page, slot, h, :] = quantize(np.asarray(k_new[b][h], np.float32), np.float32(ks))
-            v_pages[page, slot, h, :] = quantize(np.asarray(v_new[b][h], np.float32), np.float32(vs))
+            for x, pages, scale in ((k_new[b][h], k_pages, k_scale), (v_new[b][h], v_pages, v_scale)):
+                x32 = np.asarray(x, np.float32)
+                if np.ndim(scale) == 3:
+                    scale[page, slot, h] = token_scale(x32)
+                s = np.float32(_scale_of(scale, np.array(page), np.array(slot), h))
+                pages[page, slot, h, :] = quantize(x32, s)

@@ -187,12 +187,21 @@ def _dense_case(rng, B=2, Hq=8, Hkv=2, D=16, ps=16, L=(37, 50), scale_mode="page
     if scale_mode == "page":
         ks = rng.uniform(0.001, 0.02, size=(total, Hkv)).astype(np.float32)
         vs = rng.uniform(0.001, 0.02, size=(total, Hkv)).astype(np.float32)
+    elif scale_mode == "token":
+        ks = rng.uniform(0.001, 0.02, size=(total, ps, Hkv)).astype(np.float32)
+        vs = rng.uniform(0.001, 0.02, size=(total, ps, Hkv)).astype(np.float32)
     else:
         ks = rng.uniform(0.001, 0.02, size=Hkv).astype(np.float32)
         vs = rng.uniform(0.001, 0.02, size=Hkv).astype(np.float32)
     q = torch.randn(B, Hq, D, generator=torch.Generator().manual_seed(int(rng.integers(1 << 30))))
     q = q.to(torch.bfloat16).double().numpy()
     return dict(q=q, k=k, v=v, ks=ks, vs=vs, table=table, lens=lens)
+
+
+def _scale_rows(sc, phys, slots, h):
+    if sc.ndim == 3:
+        return sc[phys, slots, h]
+    return sc[phys, h] if sc.ndim == 2 else np.full(len(phys), sc[h])
 
 
 def _sdpa_reference(c, window, sinks, sm_scale):
@@ -213,8 +222,8 @@ def _sdpa_reference(c, window, sinks, sm_scale):
         V = np.zeros((Hq, L + 1, D))
         for hq in range(Hq):
             h = hq // G
-            kscale = ks[phys, h] if ks.ndim == 2 else np.full(L, ks[h])
-            vscale = vs[phys, h] if vs.ndim == 2 else np.full(L, vs[h])
+            kscale = _scale_rows(ks, phys, t % ps, h)
+            vscale = _scale_rows(vs, phys, t % ps, h)
             K[hq, :L] = torch.from_numpy(k[phys, t % ps, h]).view(torch.float8_e4m3fn).double().numpy() \
                 * kscale[:, None]
             V[hq, :L] = torch.from_numpy(v[phys, t % ps, h]).view(torch.float8_e4m3fn).double().numpy() \
@@ -236,7 +245,8 @@ def _run(c, **kw):
 
 
 @pytest.mark.parametrize("window,with_sinks,scale_mode",
-                         [(0, False, "page"), (0, True, "head"), (20, False, "head"), (7, True, "page")])
+                         [(0, False, "page"), (0, True, "head"), (20, False, "head"), (7, True, "page"),
+                          (0, False, "token"), (9, True, "token")])
 def test_attention_matches_library_sdpa(window, with_sinks, scale_mode):
     rng = np.random.default_rng(100 + window)
     c = _dense_case(rng, scale_mode=scale_mode)
@@ -422,3 +432,142 @@ def test_append_writes_only_the_new_slot():
                 assert np.all((got[~small] & 0x7F) == 0x7E)   # beyond it E4M3 saturates
     assert np.array_equal(kp[~touched], k0[~touched])
     assert np.array_equal(vp[~touched], v0[~touched])
+
+
+# ---------------------------------------------------------------- per-token scales
+
+def test_token_scale_matches_library_amax_over_448():
+    g = torch.Generator().manual_seed(21)
+    x = (torch.randn(64, 4, 96, generator=g) * torch.rand(64, 4, 1, generator=g) * 50).to(torch.bfloat16).float()
+    want = (x.abs().amax(-1) / torch.tensor(448.0)).numpy()        # float32 IEEE division
+    got = O.token_scale(x.numpy())
+    assert got.dtype == np.float32 and np.array_equal(got, want)
+
+
+def test_token_scale_special_rows():
+    rows = np.array([[0.0, -0.0, 0.0, 0.0],            # all zero -> 1
+                     [np.nan, 2.0, -3.0, 1.0],          # NaN skipped -> 3 / 448
+                     [-896.0, 1.0, 0.5, 0.0]], np.float32)
+    s = O.token_scale(rows)
+    assert s[0] == 1.0
+    assert s[1] == np.float32(3.0) / np.float32(448.0)
+    assert s[2] == 2.0
+    codes, _ = O.quantize_per_token(rows[[0, 2]])
+    assert list(codes[0]) == [0x00, 0x80, 0x00, 0x00]
+    assert codes[1][0] == 0xFE                          # -448: the row's maximum
+
+
+def test_quantize_per_token_maximum_maps_to_448_and_error_bound():
+    """Every row's largest magnitude lands on code 0x7E / 0xFE (448), and the
+    dequantized value is within half an E4M3 step: 2^-4 relative in the
+    normal range, 2^-10 * scale below it (P1 "Supported scope")."""
+    rng = np.random.default_rng(22)
+    x = (rng.standard_normal((200, 3, 64)) * rng.uniform(1e-3, 1e3, (200, 3, 1))).astype(np.float32)
+    codes, s = O.quantize_per_token(x)
+    idx = np.abs(x).argmax(-1)
+    top = np.take_along_axis(codes, idx[..., None], -1)[..., 0]
+    assert np.all((top & 0x7F) == 0x7E)
+    deq = O.e4m3_decode(codes) * s[..., None].astype(np.float64)
+    err = np.abs(deq - x.astype(np.float64))
+    normal = np.abs(x) / s[..., None] >= 2.0 ** -6
+    assert np.all(err[normal] <= 2.0 ** -4 * np.abs(x[normal]) * (1 + 1e-6))
+    sub = np.broadcast_to(s[..., None], x.shape)[~normal].astype(np.float64)
+    assert np.all(err[~normal] <= 2.0 ** -10 * sub * (1 + 1e-6))
+
+
+def test_per_token_scale_constant_over_slots_equals_per_page():
+    rng = np.random.default_rng(23)
+    c = _dense_case(rng, scale_mode="page")
+    ps = c["k"].shape[1]
+    c3 = dict(c, ks=np.repeat(c["ks"][:, None, :], ps, 1), vs=np.repeat(c["vs"][:, None, :], ps, 1))
+    for w in (0, 11):
+        assert np.array_equal(_run(c, window=w, sm_scale=0.2), _run(c3, window=w, sm_scale=0.2))
+
+
+def _logical_scale_case(B=3, Hq=4, Hkv=2, D=8, ps=16, lens=(5, 40, 33), seed=24):
+    """Every K and V code is 0x38 (1.0); scales are set per logical position
+    t of each sequence through a permuted block table."""
+    rng = np.random.default_rng(seed)
+    lens = np.array(lens)
+    npg = (lens + ps - 1) // ps
+    total = int(npg.sum()) + 2
+    perm = rng.permutation(total)
+    table = np.full((B, npg.max()), -1, np.int32)
+    off = 0
+    for b in range(B):
+        table[b, :npg[b]] = perm[off:off + npg[b]]
+        off += npg[b]
+    k = np.full((total, ps, Hkv, D), 0x38, np.uint8)
+    v = np.full((total, ps, Hkv, D), 0x38, np.uint8)
+    return table, k, v, lens, total
+
+
+def test_per_token_v_scale_closed_form():
+    """Scores all 0 (q = 0): out = mean over the attended keys of the V scale
+    of each key, which is set to 1 + t + 1000 h at logical position t; the
+    mean of an arithmetic series is 1 + 1000 h + (lo + L - 1) / 2."""
+    B, Hq, Hkv, D, ps = 3, 4, 2, 8, 16
+    table, k, v, lens, total = _logical_scale_case(B, Hq, Hkv, D, ps)
+    ks = np.ones((total, ps, Hkv), np.float32)
+    vs = np.zeros((total, ps, Hkv), np.float32)
+    for b in range(B):
+        for t in range(lens[b]):
+            vs[table[b, t // ps], t % ps, :] = 1 + t + 1000 * np.arange(Hkv)
+    q = np.zeros((B, Hq, D))
+    for window in (0, 4, 100):
+        out = O.paged_decode_attention(q, k, v, ks, vs, table, lens, window=window, sm_scale=0.5)
+        for b in range(B):
+            lo, L = max(0, lens[b] - window) if window else 0, lens[b]
+            for hq in range(Hq):
+                h = hq // (Hq // Hkv)
+                assert np.allclose(out[b, hq], 1 + 1000 * h + (lo + L - 1) / 2, rtol=1e-13)
+
+
+def test_per_token_k_scale_closed_form():
+    """q = 1 everywhere, K scale a * t and V scale t at logical position t:
+    the weights are r^t with r = exp(sm * D * a), so out is the r-weighted
+    mean of t over the attended keys."""
+    B, Hq, Hkv, D, ps = 3, 4, 2, 8, 16
+    table, k, v, lens, total = _logical_scale_case(B, Hq, Hkv, D, ps, seed=25)
+    a, sm = 0.01, 0.5
+    ks = np.zeros((total, ps, Hkv), np.float32)
+    vs = np.zeros((total, ps, Hkv), np.float32)
+    for b in range(B):
+        for t in range(lens[b]):
+            ks[table[b, t // ps], t % ps, :] = np.float32(a * t)
+            vs[table[b, t // ps], t % ps, :] = t
+    q = np.ones((B, Hq, D))
+    out = O.paged_decode_attention(q, k, v, ks, vs, table, lens, sm_scale=sm)
+    for b in range(B):
+        t = np.arange(lens[b])
+        w = np.exp(sm * D * np.float32(a * t).astype(np.float64) * 1.0)
+        want = (w * t).sum() / w.sum()
+        assert np.allclose(out[b], want, rtol=1e-12)
+
+
+def test_append_per_token_writes_its_scale_and_codes():
+    rng = np.random.default_rng(26)
+    num_pages, ps, Hkv, D, B = 10, 16, 2, 64, 3
+    kp = rng.integers(0, 256, (num_pages, ps, Hkv, D)).astype(np.uint8)
+    vp = kp.copy()
+    ks = rng.uniform(0.01, 0.02, (num_pages, ps, Hkv)).astype(np.float32)
+    vs = ks.copy()
+    k0, v0, ks0, vs0 = kp.copy(), vp.copy(), ks.copy(), vs.copy()
+    table = rng.permutation(num_pages)[:B * 3].reshape(B, 3).astype(np.int32)
+    pos = np.array([0, 20, 47])
+    g = torch.Generator().manual_seed(26)
+    kn = (torch.randn(B, Hkv, D, generator=g) * 7).to(torch.bfloat16).float()
+    vn = (torch.randn(B, Hkv, D, generator=g) * 0.01).to(torch.bfloat16).float()
+    O.kv_append(kn.numpy(), vn.numpy(), kp, vp, ks, vs, table, pos)
+    touched = np.zeros((num_pages, ps), bool)
+    for b in range(B):
+        p, s = table[b, pos[b] // ps], pos[b] % ps
+        touched[p, s] = True
+        for pages, scales, x in ((kp, ks, kn[b]), (vp, vs, vn[b])):
+            lib_s = (x.abs().amax(-1) / torch.tensor(448.0)).numpy()
+            assert np.array_equal(scales[p, s], lib_s)
+            quot = x / torch.from_numpy(lib_s)[:, None]
+            lib = quot.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            assert np.array_equal(pages[p, s], lib)
+    assert np.array_equal(kp[~touched], k0[~touched]) and np.array_equal(vp[~touched], v0[~touched])
+    assert np.array_equal(ks[~touched], ks0[~touched]) and np.array_equal(vs[~touched], vs0[~touched])
