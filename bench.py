@@ -247,7 +247,7 @@ def run_ours(args) -> dict | None:
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
-    case = W.make_case(args.config, dev)
+    case = W.make_case(args.config, dev, **_scale_override(args))
     for layer in case.layers:
         layer.out = torch.empty(layer.q.shape, dtype=torch.float32, device=dev)
     step = Step(F, case, not args.unfused)
@@ -339,7 +339,7 @@ def run_ours(args) -> dict | None:
     app_ms = kt["append_ms"] / kt["append_launches"] if kt["append_launches"] else None
     layer_bytes = nbytes / max(1, len(case.layers))
     achieved = layer_bytes / (att_ms * 1e-3) / 1e9 if att_ms > 0 else None
-    traffic = _traffic(args.config)
+    traffic = _traffic(args.config) if args.scales == "workload" else None
     line = {
         "metric": METRIC,
         "value": round(gbs, 2),
@@ -354,9 +354,10 @@ def run_ours(args) -> dict | None:
         "vs_baseline": None,
         "dtype": "e4m3 cache; f16 tensor-core MMA, f32 accumulate",
         "data": "synthetic (seeded), no dataset",
-        "config": {"workload": WORKLOAD_TEXT.get(args.config, args.config),
+        "config": {"workload": _workload_text(args),
                    "name": args.config,
                    "bytes_per_step": nbytes, "k_decode": args.k_decode,
+                   "scales": _scales_text(case),
                    "l2": "flushed between timed steps: " + flush.describe(),
                    "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
         "timing": "device time of CUDA-graph replays of the step (per-step events); "
@@ -472,11 +473,11 @@ def _case_to_numpy(case: W.Case, seqs) -> tuple[dict, np.ndarray, np.ndarray | N
             off += npg[i]
         idx = torch.as_tensor(ids, device=layer.k_pages.device)
         f = lambda t: t.detach().float().cpu().numpy().astype(np.float64)  # noqa: E731
-        per_page = layer.k_scale.dim() == 2
+        # per-page and per-token scales follow their pages; per-head ones do not
+        pick = lambda sc: (sc[idx] if sc.dim() >= 2 else sc).cpu().numpy()  # noqa: E731
         d = {"q": f(layer.q[list(seqs)]),
              "k_pages": layer.k_pages[idx].cpu().numpy(), "v_pages": layer.v_pages[idx].cpu().numpy(),
-             "k_scale": (layer.k_scale[idx] if per_page else layer.k_scale).cpu().numpy(),
-             "v_scale": (layer.v_scale[idx] if per_page else layer.v_scale).cpu().numpy(),
+             "k_scale": pick(layer.k_scale), "v_scale": pick(layer.v_scale),
              "block_table": new_tbl, "window": layer.window, "sm_scale": layer.sm_scale,
              "sinks": layer.sinks.cpu().numpy() if layer.sinks is not None else None,
              "k_new": f(layer.k_new[list(seqs)]) if layer.k_new is not None else None,
@@ -487,6 +488,8 @@ def _case_to_numpy(case: W.Case, seqs) -> tuple[dict, np.ndarray, np.ndarray | N
             lo = max(0, Lb - layer.window) if layer.window > 0 else 0
             n = Lb - lo
             nbytes += 2 * n * layer.spec.Hkv * layer.spec.D
+            nbytes += sum(4 * n * layer.spec.Hkv for sc in (layer.k_scale, layer.v_scale)
+                          if sc.dim() == 3)
             if n > 0:
                 nbytes += 4 * ((Lb - 1) // ps - lo // ps + 1)
         nbytes += 2 * d["q"].size
@@ -517,6 +520,22 @@ def cpu_baseline(case: W.Case, budget_s: float = 10.0) -> dict:
             "seconds": round(t_total, 2)}
 
 
+def _scale_override(args) -> dict:
+    """``--scales token``: the workload with one scale per stored token and KV
+    head instead of its own scale form."""
+    return {"scale_mode": "token"} if args.scales == "token" else {}
+
+
+def _workload_text(args) -> str:
+    text = WORKLOAD_TEXT.get(args.config, args.config)
+    return text + " (scales replaced: per (token, KV head))" if args.scales == "token" else text
+
+
+def _scales_text(case) -> str:
+    return {"head": "per KV head", "page": "per (page, KV head)",
+            "token": "per (token, KV head)"}[case.spec.scale_mode]
+
+
 def run_reference(args) -> dict | None:
     """The float64 CPU oracle on this host: each step is one bounded sample of
     the workload (rank 0 only)."""
@@ -524,7 +543,7 @@ def run_reference(args) -> dict | None:
     if rank != 0:
         return None
     from threadpoolctl import threadpool_limits
-    case = W.make_case(args.config, "cpu")
+    case = W.make_case(args.config, "cpu", **_scale_override(args))
     B = case.spec.B
     # bounded sample per step: as many whole sequences as fit in ~1.5 s
     seqs = list(range(B))
@@ -550,7 +569,8 @@ def run_reference(args) -> dict | None:
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded), no dataset",
-        "config": {"workload": WORKLOAD_TEXT.get(args.config, args.config), "name": args.config},
+        "config": {"workload": _workload_text(args), "name": args.config,
+                   "scales": _scales_text(case)},
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -572,6 +592,8 @@ def main():
     ap.add_argument("--k-decode", default="cvt", choices=["bits", "cvt"],
                     help="E4M3 -> f16 decode of K: bit assembly or hardware cvt")
     ap.add_argument("--splits", type=int, default=0, help="force a split count (0 = planner)")
+    ap.add_argument("--scales", default="workload", choices=["workload", "token"],
+                    help="token: per-token-per-head K/V scales instead of the workload's form")
     ap.add_argument("--schedule", type=int, default=0, choices=[0, 1, 2, 3],
                     help="0 = planner, 1 = uniform splits, 2 = segment kernel, "
                          "3 = proportional splits")

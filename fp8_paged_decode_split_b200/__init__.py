@@ -161,7 +161,8 @@ def fp8_paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_tabl
 
     q [B, Hq, D] bf16; k_pages / v_pages [num_pages, ps, Hkv, D] uint8 views
     (any page stride that is a multiple of 16 bytes); k_scale / v_scale
-    float32 [Hkv] or [num_pages, Hkv]; block_table int32 [B, max_pages];
+    float32 [Hkv], [num_pages, Hkv] or [num_pages, ps, Hkv] (per stored
+    token and KV head); block_table int32 [B, max_pages];
     seq_lens int32 [B] (keys visible to the query); sinks float32 [Hq] or
     None; sm_scale defaults to D ** -0.5. Returns out [B, Hq, D] float32.
     """
@@ -205,7 +206,9 @@ def fp8_paged_decode_attention_noalloc(q, k_pages, v_pages, k_scale, v_scale, bl
 def fp8_kv_append(k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table, positions,
                   stream=None) -> None:
     """Quantize k_new / v_new [B, Hkv, D] bf16 to E4M3 and write them at
-    positions[b] of each sequence's pages (see include/fp8pd.h)."""
+    positions[b] of each sequence's pages (see include/fp8pd.h). Scales of
+    shape [num_pages, ps, Hkv] are per token: the new token's own
+    max|x| / 448 is written with its codes."""
     _same_device(k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table, positions)
     sc = Scales()
     sc.k_scale = describe(k_scale)

@@ -70,10 +70,16 @@ int check(const fp8pd_tensor* t, int32_t dtype, int32_t ndim) {
 
 bool fits_i32(int64_t v) { return v >= 0 && v <= INT32_MAX; }
 
-// Scale descriptor -> (page stride, head stride) in elements.
-int scale_strides(const fp8pd_tensor* s, int64_t num_pages, int64_t hkv, int64_t* sp, int64_t* sh) {
+// Scale descriptor -> (page, slot, head) strides in elements; *tok = 1 for
+// the per-token form [num_pages, ps, Hkv] (one scale per stored token and KV
+// head), 0 for [Hkv] (slot and page strides 0) and [num_pages, Hkv] (slot
+// stride 0).
+int scale_strides(const fp8pd_tensor* s, int64_t num_pages, int64_t ps, int64_t hkv, int64_t* sp,
+                  int64_t* st, int64_t* sh, int* tok) {
   if (!s || !s->data) return FP8PD_ERR_NULL;
   if (s->dtype != FP8PD_DTYPE_F32) return FP8PD_ERR_DTYPE;
+  *st = 0;
+  *tok = 0;
   if (s->ndim == 1) {
     if (s->shape[0] != hkv) return FP8PD_ERR_SHAPE;
     *sp = 0;
@@ -84,6 +90,14 @@ int scale_strides(const fp8pd_tensor* s, int64_t num_pages, int64_t hkv, int64_t
     if (s->shape[0] != num_pages || s->shape[1] != hkv) return FP8PD_ERR_SHAPE;
     *sp = s->stride[0];
     *sh = s->stride[1];
+    return FP8PD_OK;
+  }
+  if (s->ndim == 3) {
+    if (s->shape[0] != num_pages || s->shape[1] != ps || s->shape[2] != hkv) return FP8PD_ERR_SHAPE;
+    *sp = s->stride[0];
+    *st = s->stride[1];
+    *sh = s->stride[2];
+    *tok = 1;
     return FP8PD_OK;
   }
   return FP8PD_ERR_SHAPE;
@@ -434,9 +448,10 @@ int validate_decode(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp
     return FP8PD_ERR_ALIGN;
   if (window < 0) return FP8PD_ERR_ARG;
   if (!(std::isfinite(sm_scale) && sm_scale > 0.f)) return FP8PD_ERR_ARG;
-  int64_t ks_sp, ks_sh, vs_sp, vs_sh;
-  if ((r = scale_strides(k_scale, P, Hkv, &ks_sp, &ks_sh))) return r;
-  if ((r = scale_strides(v_scale, P, Hkv, &vs_sp, &vs_sh))) return r;
+  int64_t ks_sp, ks_st, ks_sh, vs_sp, vs_st, vs_sh;
+  int k_tok, v_tok;
+  if ((r = scale_strides(k_scale, P, ps, Hkv, &ks_sp, &ks_st, &ks_sh, &k_tok))) return r;
+  if ((r = scale_strides(v_scale, P, ps, Hkv, &vs_sp, &vs_st, &vs_sh, &v_tok))) return r;
   if (sinks) {
     if ((r = check(sinks, FP8PD_DTYPE_F32, 1))) return r;
     if (sinks->shape[0] != Hq) return FP8PD_ERR_SHAPE;
@@ -465,6 +480,10 @@ int validate_decode(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp
   p->ks_sh = ks_sh;
   p->vs_sp = vs_sp;
   p->vs_sh = vs_sh;
+  p->ks_st = ks_st;
+  p->vs_st = vs_st;
+  p->k_tok = k_tok;
+  p->v_tok = v_tok;
   p->table = static_cast<const int32_t*>(block_table->data);
   p->tab_sb = block_table->stride[0];
   p->tab_sp = block_table->stride[1];
@@ -627,11 +646,13 @@ namespace {
 
 // Plans, sizes the workspace, encodes the tensor maps and launches one
 // validated decode-attention call. `allow_seg`: the segment kernel may run
-// (it has no fused append).
+// (it has no fused append). It reads no per-token scales either: with those
+// the split kernel runs.
 int run_decode(DecodeParams& p, const DecodeArgs& a, const fp8pd_tensor* k_pages,
                const fp8pd_tensor* v_pages, int32_t window, bool allow_seg, fp8pd_stream_t stream) {
   Plan plan;
-  int r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan, allow_seg);
+  int r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan,
+                    allow_seg && !(p.k_tok || p.v_tok));
   if (r) return r;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   apply_plan(plan, &p);
@@ -702,6 +723,8 @@ int fp8_paged_decode_append_attention(const fp8pd_tensor* q, const fp8pd_tensor*
   p.vn_sd = v_new->stride[2];
   p.kw = static_cast<uint8_t*>(k_pages->data);
   p.vw = static_cast<uint8_t*>(v_pages->data);
+  p.ksw = static_cast<float*>(k_scale->data);
+  p.vsw = static_cast<float*>(v_scale->data);
   r = run_decode(p, a, k_pages, v_pages, window, false, stream);
   if (r == FP8PD_OK) ++g_appends;
   return r;
@@ -755,9 +778,10 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
   if (k_pages->shape[2] != Hkv || k_pages->shape[3] != D) return FP8PD_ERR_SHAPE;
   if (block_table->shape[0] != B || positions->shape[0] != B) return FP8PD_ERR_SHAPE;
   if (ps < 1) return FP8PD_ERR_UNSUPPORTED;
-  int64_t ks_sp, ks_sh, vs_sp, vs_sh;
-  if ((r = scale_strides(&scales->k_scale, P, Hkv, &ks_sp, &ks_sh))) return r;
-  if ((r = scale_strides(&scales->v_scale, P, Hkv, &vs_sp, &vs_sh))) return r;
+  int64_t ks_sp, ks_st, ks_sh, vs_sp, vs_st, vs_sh;
+  int k_tok, v_tok;
+  if ((r = scale_strides(&scales->k_scale, P, ps, Hkv, &ks_sp, &ks_st, &ks_sh, &k_tok))) return r;
+  if ((r = scale_strides(&scales->v_scale, P, ps, Hkv, &vs_sp, &vs_st, &vs_sh, &v_tok))) return r;
   const int64_t max_pages = block_table->shape[1];
   if (!fits_i32(B) || !fits_i32(P) || !fits_i32(Hkv) || !fits_i32(D) || !fits_i32(max_pages) ||
       max_pages * ps > INT32_MAX || B * Hkv * ((D + 1) / 2) > (int64_t(1) << 40))
@@ -787,6 +811,12 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
   p.ks_sh = ks_sh;
   p.vs_sp = vs_sp;
   p.vs_sh = vs_sh;
+  p.ks_st = ks_st;
+  p.vs_st = vs_st;
+  p.k_tok = k_tok;
+  p.v_tok = v_tok;
+  p.ksw = static_cast<float*>(scales->k_scale.data);
+  p.vsw = static_cast<float*>(scales->v_scale.data);
   p.table = static_cast<const int32_t*>(block_table->data);
   p.tab_sb = block_table->stride[0];
   p.tab_sp = block_table->stride[1];
@@ -964,7 +994,7 @@ extern "C" int fp8_paged_decode_attention_noalloc(
   if (r) return r;
   if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
   Plan plan;
-  r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
+  r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan, !(p.k_tok || p.v_tok));
   if (r) return r;
   if (plan.schedule == 2 && plan.workspace > kNoAllocScratchBytes) {
     // the segment layout does not fit: the split kernel's may

@@ -17,9 +17,11 @@ struct DecodeParams {
   const uint8_t* v;
   int64_t k_sp, k_st, k_sh;
   int64_t v_sp, v_st, v_sh;
-  const float* ks;            // scale(page, h) = ks[page * ks_sp + h * ks_sh]
+  const float* ks;            // scale(page, slot, h) = ks[page * ks_sp + slot * ks_st + h * ks_sh]
   const float* vs;
   int64_t ks_sp, ks_sh, vs_sp, vs_sh;
+  int64_t ks_st, vs_st;       // 0 unless the scales are per token
+  int k_tok, v_tok;           // 1: per-token-per-head scales [num_pages, ps, Hkv]
   const int32_t* table;       // [B, max_pages]
   int64_t tab_sb, tab_sp;
   const int32_t* lens;        // [B]
@@ -60,6 +62,8 @@ struct DecodeParams {
   int64_t kn_sb, kn_sh, kn_sd, vn_sb, vn_sh, vn_sd;
   uint8_t* kw;
   uint8_t* vw;
+  float* ksw;                 // the scales, writable: a per-token scale of the new token is stored
+  float* vsw;
 };
 
 struct AppendParams {
@@ -72,6 +76,10 @@ struct AppendParams {
   const float* ks;
   const float* vs;
   int64_t ks_sp, ks_sh, vs_sp, vs_sh;
+  int64_t ks_st, vs_st;       // slot strides (per-token scales), else 0
+  int k_tok, v_tok;           // 1: the scale is the new token's own max|x| / 448, written here
+  float* ksw;
+  float* vsw;
   const int32_t* table;
   int64_t tab_sb, tab_sp;
   const int32_t* pos;

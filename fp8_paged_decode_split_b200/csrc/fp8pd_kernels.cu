@@ -440,13 +440,15 @@ struct Acc {
 // units of this lane: tokens grp / grp + 8 of the tile, heads 2qd / 2qd+1,
 // returned as (x, y, z, w) = (grp, 2qd), (grp, 2qd+1), (grp+8, 2qd),
 // (grp+8, 2qd+1). Tokens outside [t0, t1), or the whole tile when its page
-// is out of range, are -inf. kfac = score factor of the tile's page; `full`:
+// is out of range, are -inf. kfa / kfb = score factors of tokens grp /
+// grp + 8 (equal unless the scales are per token); `full`:
 // every token is attended (warp-uniform). qfr(kb) gives the q' B-fragment
 // of k16 block kb.
 template <int D, bool KCVT, class QFrag>
 __device__ __forceinline__ float4 tile_scores(const QFrag& qfr, uint32_t sk,
-                                              const uint32_t (&koff)[4], float kfac, int tok0,
-                                              int t0, int t1, bool page_ok, bool full, int grp) {
+                                              const uint32_t (&koff)[4], float kfa, float kfb,
+                                              int tok0, int t0, int t1, bool page_ok, bool full,
+                                              int grp) {
   // two independent accumulator chains
   float Sa[4] = {0.f, 0.f, 0.f, 0.f}, Sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -485,10 +487,10 @@ __device__ __forceinline__ float4 tile_scores(const QFrag& qfr, uint32_t sk,
   const int ta = tok0 + grp, tb = ta + 8;
   const bool va = full || (page_ok && ta >= t0 && ta < t1);
   const bool vb = full || (page_ok && tb >= t0 && tb < t1);
-  return make_float4(va ? (Sa[0] + Sb[0]) * kfac : -CUDART_INF_F,
-                     va ? (Sa[1] + Sb[1]) * kfac : -CUDART_INF_F,
-                     vb ? (Sa[2] + Sb[2]) * kfac : -CUDART_INF_F,
-                     vb ? (Sa[3] + Sb[3]) * kfac : -CUDART_INF_F);
+  return make_float4(va ? (Sa[0] + Sb[0]) * kfa : -CUDART_INF_F,
+                     va ? (Sa[1] + Sb[1]) * kfa : -CUDART_INF_F,
+                     vb ? (Sa[2] + Sb[2]) * kfb : -CUDART_INF_F,
+                     vb ? (Sa[3] + Sb[3]) * kfb : -CUDART_INF_F);
 }
 
 // Online-softmax update for new scores whose per-head maxima over this
@@ -533,17 +535,18 @@ __device__ __forceinline__ void softmax_rescale(Acc<D>& a, float tm0, float tm1,
 // the running sums; then P * v_scale / vref as an f16 hi + lo pair, whose PV
 // B fragments are the transposes of the score fragment's 8x8 blocks
 // (movmatrix): bh / bl[0] for tokens 2qd.., bh / bl[1] for 2qd+8...
+// vsa / vsb: V scales of tokens grp / grp + 8.
 template <int D>
-__device__ __forceinline__ void tile_probs(Acc<D>& a, float4 sc, float vs, uint32_t (&bh)[2],
-                                           uint32_t (&bl)[2]) {
+__device__ __forceinline__ void tile_probs(Acc<D>& a, float4 sc, float vsa, float vsb,
+                                           uint32_t (&bh)[2], uint32_t (&bl)[2]) {
   const float mb0 = (a.m0 == -CUDART_INF_F) ? 0.f : a.m0;
   const float mb1 = (a.m1 == -CUDART_INF_F) ? 0.f : a.m1;
   const float p00 = fast_exp2(sc.x - mb0), p01 = fast_exp2(sc.y - mb1);
   const float p10 = fast_exp2(sc.z - mb0), p11 = fast_exp2(sc.w - mb1);
   a.l0 += p00 + p10;
   a.l1 += p01 + p11;
-  const float vsr = vs * a.inv_vref;
-  const float w00 = p00 * vsr, w01 = p01 * vsr, w10 = p10 * vsr, w11 = p11 * vsr;
+  const float vra = vsa * a.inv_vref, vrb = vsb * a.inv_vref;
+  const float w00 = p00 * vra, w01 = p01 * vra, w10 = p10 * vrb, w11 = p11 * vrb;
   const uint32_t ha = pack_f16x2(w00, w01), hb = pack_f16x2(w10, w11);
   const float2 fa = unpack_f16x2(ha), fb = unpack_f16x2(hb);
   const uint32_t la = pack_f16x2(w00 - fa.x, w01 - fa.y), lb = pack_f16x2(w10 - fb.x, w11 - fb.y);
@@ -607,17 +610,21 @@ __device__ __forceinline__ void tile_pv(Acc<D>& a, uint32_t sv, const uint32_t (
 
 // Attends one 16-token tile already in shared memory (K at sk, V at sv) for
 // one warp: S = K q'^T, masking, the online-softmax update, and O += V^T P
-// with P as an f16 hi + lo pair. kfac = score factor of the tile's page
-// (log2 units), vs = its V scale; tok0 = first token of the tile.
+// with P as an f16 hi + lo pair. kfa / kfb = score factors (log2 units) and
+// vsa / vsb = V scales of this lane's tokens grp / grp + 8, vabs = the
+// largest |V scale| of the tile's attended tokens; tok0 = first token of the
+// tile.
 template <int D, bool KCVT, bool VCVT, class QFrag>
 __device__ __forceinline__ void attend_tile(Acc<D>& a, const QFrag& qfr, uint32_t sk, uint32_t sv,
                                             const uint32_t (&koff)[4], const uint32_t (&voff)[4],
-                                            float kfac, float vs, int tok0, int t0, int t1,
-                                            bool page_ok, bool full, int grp, int qd) {
-  const float4 sc = tile_scores<D, KCVT>(qfr, sk, koff, kfac, tok0, t0, t1, page_ok, full, grp);
-  softmax_rescale<D>(a, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), fabsf(vs));
+                                            float kfa, float kfb, float vsa, float vsb, float vabs,
+                                            int tok0, int t0, int t1, bool page_ok, bool full,
+                                            int grp, int qd) {
+  const float4 sc =
+      tile_scores<D, KCVT>(qfr, sk, koff, kfa, kfb, tok0, t0, t1, page_ok, full, grp);
+  softmax_rescale<D>(a, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), vabs);
   uint32_t bh[2], bl[2];
-  tile_probs<D>(a, sc, vs, bh, bl);
+  tile_probs<D>(a, sc, vsa, vsb, bh, bl);
   tile_pv<D, VCVT>(a, sv, voff, bh, bl, tok0, t0, t1, page_ok, full, qd);
 }
 
@@ -632,15 +639,15 @@ __device__ __forceinline__ void attend_pair(Acc<D>& a, const QFrag& qfr, const u
                                             const bool (&page_ok)[2], const bool (&full)[2],
                                             int grp, int qd, const Between& between) {
   constexpr int TILE = kTileTokens * D;
-  const float4 s0 = tile_scores<D, KCVT>(qfr, sk[0], koff, kfac[0], tok0[0], t0, t1, page_ok[0],
-                                         full[0], grp);
-  const float4 s1 = tile_scores<D, KCVT>(qfr, sk[1], koff, kfac[1], tok0[1], t0, t1, page_ok[1],
-                                         full[1], grp);
+  const float4 s0 = tile_scores<D, KCVT>(qfr, sk[0], koff, kfac[0], kfac[0], tok0[0], t0, t1,
+                                         page_ok[0], full[0], grp);
+  const float4 s1 = tile_scores<D, KCVT>(qfr, sk[1], koff, kfac[1], kfac[1], tok0[1], t0, t1,
+                                         page_ok[1], full[1], grp);
   softmax_rescale<D>(a, fmaxf(fmaxf(s0.x, s0.z), fmaxf(s1.x, s1.z)),
                      fmaxf(fmaxf(s0.y, s0.w), fmaxf(s1.y, s1.w)), fmaxf(fabsf(vs[0]), fabsf(vs[1])));
   uint32_t bh0[2], bl0[2], bh1[2], bl1[2];
-  tile_probs<D>(a, s0, vs[0], bh0, bl0);
-  tile_probs<D>(a, s1, vs[1], bh1, bl1);
+  tile_probs<D>(a, s0, vs[0], vs[0], bh0, bl0);
+  tile_probs<D>(a, s1, vs[1], vs[1], bh1, bl1);
   tile_pv<D, VCVT>(a, sk[0] + TILE, voff, bh0, bl0, tok0[0], t0, t1, page_ok[0], full[0], qd);
   between();
   tile_pv<D, VCVT>(a, sk[1] + TILE, voff, bh1, bl1, tok0[1], t0, t1, page_ok[1], full[1], qd);
@@ -668,31 +675,60 @@ __device__ __forceinline__ uint16_t e4m3x2_rn_sat(float lo, float hi) {
   return r;  // low byte = lo, high byte = hi
 }
 
+// Per-token-per-head scale of one head's D values spread over a warp (PER
+// per lane): max |x| / 448 in IEEE f32, NaN entries skipped (fmaxf), 1 for an
+// all-zero row.
+template <int PER>
+__device__ __forceinline__ float warp_token_scale(const float (&x)[PER]) {
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) m = fmaxf(m, fabsf(x[i]));
+  m = warp_max(m);
+  return m == 0.f ? 1.f : __fdiv_rn(m, 448.f);
+}
+
 // Fused append, one warp: quantizes the new token of (sequence b, KV head
-// kvh) with its page's scales (IEEE f32 division, then E4M3 round to nearest
-// even with saturation, as fp8_kv_append), writes its codes into row r of the
-// K and V tiles in shared memory (the TMA's swizzled layout, see tile_off)
-// and, when `store`, into the pools at (page, slot). Lane l owns head-dim
-// bytes [l D/32, (l+1) D/32).
-template <int D>
+// kvh) (IEEE f32 division, then E4M3 round to nearest even with saturation,
+// as fp8_kv_append), writes its codes into row r of the K and V tiles in
+// shared memory (the TMA's swizzled layout, see tile_off) and, when `store`,
+// into the pools at (page, slot). Lane l owns head-dim bytes
+// [l D/32, (l+1) D/32). ks / vs: the page's scales; with per-token scales
+// (TOK and p.k_tok / p.v_tok) they are replaced by the new token's own,
+// which `store` also writes to the scale array.
+template <int D, bool TOK>
 __device__ __forceinline__ void append_new_token(const DecodeParams& p, int b, int kvh, bool store,
                                               int page, int slot, int r, uint32_t sk, uint32_t sv,
-                                              float ks, float vs) {
+                                              float& ks, float& vs) {
   constexpr int PER = D / 32;  // 2, 4, 8 or 16 bytes per lane
   const int lane = threadIdx.x & 31;
   const int d0 = lane * PER;
   const uint16_t* kn = p.kn + (int64_t)b * p.kn_sb + (int64_t)kvh * p.kn_sh;
   const uint16_t* vn = p.vn + (int64_t)b * p.vn_sb + (int64_t)kvh * p.vn_sh;
+  float xk[PER], xv[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    xk[i] = bf16_bits_to_float(kn[(int64_t)(d0 + i) * p.kn_sd]);
+    xv[i] = bf16_bits_to_float(vn[(int64_t)(d0 + i) * p.vn_sd]);
+  }
+  if constexpr (TOK) {
+    if (p.k_tok) {
+      ks = warp_token_scale<PER>(xk);
+      if (store && lane == 0)
+        p.ksw[(int64_t)page * p.ks_sp + (int64_t)slot * p.ks_st + (int64_t)kvh * p.ks_sh] = ks;
+    }
+    if (p.v_tok) {
+      vs = warp_token_scale<PER>(xv);
+      if (store && lane == 0)
+        p.vsw[(int64_t)page * p.vs_sp + (int64_t)slot * p.vs_st + (int64_t)kvh * p.vs_sh] = vs;
+    }
+  }
   uint32_t kw[(PER + 3) / 4], vw[(PER + 3) / 4];
 #pragma unroll
   for (int i = 0; i < (PER + 3) / 4; ++i) kw[i] = vw[i] = 0u;
 #pragma unroll
   for (int i = 0; i < PER; i += 2) {
-    const int d = d0 + i;
-    const uint32_t kc = e4m3x2_rn_sat(__fdiv_rn(bf16_bits_to_float(kn[(int64_t)d * p.kn_sd]), ks),
-                                      __fdiv_rn(bf16_bits_to_float(kn[(int64_t)(d + 1) * p.kn_sd]), ks));
-    const uint32_t vc = e4m3x2_rn_sat(__fdiv_rn(bf16_bits_to_float(vn[(int64_t)d * p.vn_sd]), vs),
-                                      __fdiv_rn(bf16_bits_to_float(vn[(int64_t)(d + 1) * p.vn_sd]), vs));
+    const uint32_t kc = e4m3x2_rn_sat(__fdiv_rn(xk[i], ks), __fdiv_rn(xk[i + 1], ks));
+    const uint32_t vc = e4m3x2_rn_sat(__fdiv_rn(xv[i], vs), __fdiv_rn(xv[i + 1], vs));
     kw[i / 4] |= kc << (8 * (i % 4));
     vw[i / 4] |= vc << (8 * (i % 4));
   }
@@ -912,8 +948,9 @@ __device__ bool prop_assign(const DecodeParams& p, int* scratch, int* red, int h
 // true = hardware cvt.rn.f16x2.e4m3x2 (the value itself). The q fragments
 // follow the K byte pairing. tmk / tmv: 5-D tensor maps over the K / V pool
 // views, dims (head-dim bytes within a 128-byte block, slot, 128-byte block,
-// KV head, page), box (min(D,128), 16, max(1, D/128), 1, 1).
-template <int D, bool KCVT, bool VCVT>
+// KV head, page), box (min(D,128), 16, max(1, D/128), 1, 1). TOK: the scales
+// are read per token (one per stored token and KV head) instead of per page.
+template <int D, bool KCVT, bool VCVT, bool TOK>
 __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     decode_tma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
@@ -1096,15 +1133,17 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   // latency overlaps that of the first tile copies.
   const float* ksbase = p.ks + (int64_t)kvh * p.ks_sh;
   const float* vsbase = p.vs + (int64_t)kvh * p.vs_sh;
+  if constexpr (!TOK) {
 #pragma unroll 2
-  for (int j = lane; j < my_tiles; j += 32) {
-    const int e = went[j];
-    if (e >= 0) {
-      cp_async4(wks + j, ksbase + (int64_t)(e >> 4) * p.ks_sp);
-      cp_async4(wvs + j, vsbase + (int64_t)(e >> 4) * p.vs_sp);
-    } else {
-      wks[j] = 0.f;
-      wvs[j] = 0.f;
+    for (int j = lane; j < my_tiles; j += 32) {
+      const int e = went[j];
+      if (e >= 0) {
+        cp_async4(wks + j, ksbase + (int64_t)(e >> 4) * p.ks_sp);
+        cp_async4(wvs + j, vsbase + (int64_t)(e >> 4) * p.vs_sp);
+      } else {
+        wks[j] = 0.f;
+        wvs[j] = 0.f;
+      }
     }
   }
   // Lane (g, q) holds query head g of the group; the k16 block kb covers
@@ -1207,10 +1246,27 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   acc.reset();
   bool ok_all = true;
 
+  // Per-token scales (TOK): lane l < 16 holds the K scale of token l of a
+  // tile and lane 16 + l its V scale, 0 for a token outside [t0, t1); the
+  // next tile's are loaded while this one is attended.
+  auto tok_scale = [&](int j) -> float {
+    const int e = went[j];
+    const int r = lane & 15;
+    const int t = (tile_first + warp + C::NW * j) * kTileTokens + r;
+    if (e < 0 || t < t0 || t >= t1) return 0.f;
+    const int64_t slot = (e & 15) * kTileTokens + r;
+    return lane < 16 ? __ldg(ksbase + (int64_t)(e >> 4) * p.ks_sp + slot * p.ks_st)
+                     : __ldg(vsbase + (int64_t)(e >> 4) * p.vs_sp + slot * p.vs_st);
+  };
+  float tsc_next = 0.f;
+  if constexpr (TOK) {
+    if (my_tiles > 0) tsc_next = tok_scale(0);
+  }
+
   int stage = 0;
   uint32_t phase = 0;
   int tok0 = (tile_first + warp) * kTileTokens;
-  if constexpr (C::PAIR) {
+  if constexpr (C::PAIR && !TOK) {
     // Two tiles per step while two are left (one softmax update per 32 keys;
     // the copy into the first tile's stage is issued once its PV is done).
 #pragma unroll 1
@@ -1245,9 +1301,10 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
         if (p.append && pok[u] && L - 1 >= tk[u] && L - 1 < tk[u] + kTileTokens) {
           // the new token: quantized here, stored by head group 0, attended by all
           const int r = L - 1 - tk[u];
-          append_new_token<D>(p, b, kvh, hg == 0, went[jj] >> 4,
-                              (went[jj] & 15) * kTileTokens + r, r, sk[u], sk[u] + C::TILE,
-                              wks[jj], vsc[u]);
+          float ks = wks[jj];
+          append_new_token<D, false>(p, b, kvh, hg == 0, went[jj] >> 4,
+                                     (went[jj] & 15) * kTileTokens + r, r, sk[u],
+                                     sk[u] + C::TILE, ks, vsc[u]);
           __syncwarp();
         }
       }
@@ -1266,7 +1323,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     }
   }
 #pragma unroll 1
-  for (int j = C::PAIR ? (my_tiles & ~1) : 0; ok_all && j < my_tiles;
+  for (int j = (C::PAIR && !TOK) ? (my_tiles & ~1) : 0; ok_all && j < my_tiles;
        ++j, tok0 += C::NW * kTileTokens) {
     if (!mbar_wait(wbar + 8 * stage, phase)) {
       if (lane == 0) raise_flag(FP8PD_FLAG_TIMEOUT);
@@ -1283,22 +1340,43 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     const bool full = page_ok && tok0 >= t0 && tok0 + kTileTokens <= t1;  // warp-uniform
     const uint32_t sk = wpipe + stage * C::STAGE;
     const uint32_t sv = sk + C::TILE;
-    const float kfac = score_base * wks[j];
-    const float vs = wvs[j];
     if (++stage == C::NS) {
       stage = 0;
       phase ^= 1;
     }
-    if (p.append && page_ok && L - 1 >= tok0 && L - 1 < tok0 + kTileTokens) {
-      // the new token: quantized here, stored by head group 0, attended by all
-      const int r = L - 1 - tok0;
-      append_new_token<D>(p, b, kvh, hg == 0, went[j] >> 4, (went[j] & 15) * kTileTokens + r, r,
-                          sk, sv, wks[j], vs);
-      __syncwarp();
+    // the new token: quantized here, stored by head group 0, attended by all
+    const bool has_new = p.append && page_ok && L - 1 >= tok0 && L - 1 < tok0 + kTileTokens;
+    if constexpr (TOK) {
+      float tsc = tsc_next;
+      if (j + 1 < my_tiles) tsc_next = tok_scale(j + 1);
+      if (has_new) {
+        const int r = L - 1 - tok0;
+        float ks = __shfl_sync(0xffffffffu, tsc, r), vs = __shfl_sync(0xffffffffu, tsc, 16 + r);
+        append_new_token<D, true>(p, b, kvh, hg == 0, went[j] >> 4,
+                                  (went[j] & 15) * kTileTokens + r, r, sk, sv, ks, vs);
+        if (lane == r) tsc = ks;
+        if (lane == 16 + r) tsc = vs;
+        __syncwarp();
+      }
+      const float kfa = score_base * __shfl_sync(0xffffffffu, tsc, grp);
+      const float kfb = score_base * __shfl_sync(0xffffffffu, tsc, grp + 8);
+      const float vsa = __shfl_sync(0xffffffffu, tsc, 16 + grp);
+      const float vsb = __shfl_sync(0xffffffffu, tsc, 24 + grp);
+      const float vabs = warp_max(lane >= 16 ? fabsf(tsc) : 0.f);
+      attend_tile<D, KCVT, VCVT>(acc, qfr, sk, sv, koff, voff, kfa, kfb, vsa, vsb, vabs, tok0, t0,
+                                 t1, page_ok, full, grp, qd);
+    } else {
+      const float kfac = score_base * wks[j];
+      float ks = wks[j], vs = wvs[j];
+      if (has_new) {
+        const int r = L - 1 - tok0;
+        append_new_token<D, false>(p, b, kvh, hg == 0, went[j] >> 4,
+                                   (went[j] & 15) * kTileTokens + r, r, sk, sv, ks, vs);
+        __syncwarp();
+      }
+      attend_tile<D, KCVT, VCVT>(acc, qfr, sk, sv, koff, voff, kfac, kfac, vs, vs, fabsf(vs), tok0,
+                                 t0, t1, page_ok, full, grp, qd);
     }
-
-    attend_tile<D, KCVT, VCVT>(acc, qfr, sk, sv, koff, voff, kfac, vs, tok0, t0, t1, page_ok, full,
-                               grp, qd);
   }
   if (!ok_all) {
     // A copy never completed: leave this warp's result out (its flag is set)
@@ -2073,8 +2151,8 @@ __global__ void __launch_bounds__(SegCfg<D>::NT, 1)
     const uint32_t sk = wpipe + cur * C::STAGE;
     const float kfac = score_base * wscl[2 * cur];
     const float vs = wscl[2 * cur + 1];
-    attend_tile<D, KCVT, VCVT>(acc, qfr, sk, sk + C::TILE, koff, voff, kfac, vs, tok0, lo, L,
-                               page_ok, full, grp, qd);
+    attend_tile<D, KCVT, VCVT>(acc, qfr, sk, sk + C::TILE, koff, voff, kfac, kfac, vs, vs,
+                               fabsf(vs), tok0, lo, L, page_ok, full, grp, qd);
   }
   // the block's remaining segment ends (every warp takes part in each)
 #pragma unroll 1
@@ -2223,6 +2301,14 @@ __global__ void __launch_bounds__(SegCfg<D>::NT, 1)
 // nearest even and saturates to +-448 (NaN stays NaN).
 // ---------------------------------------------------------------------------
 
+// Per-token-per-head scale of one bf16 row of n values (stride sd): max |x| /
+// 448 in IEEE f32, NaN entries skipped (fmaxf), 1 for an all-zero row.
+__device__ float row_token_scale(const uint16_t* x, int64_t sd, int n) {
+  float m = 0.f;
+  for (int i = 0; i < n; ++i) m = fmaxf(m, fabsf(bf16_bits_to_float(x[(int64_t)i * sd])));
+  return m == 0.f ? 1.f : __fdiv_rn(m, 448.f);
+}
+
 __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
   const int npair = (p.D + 1) / 2;
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -2245,10 +2331,20 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
   }
   const int slot = pos - lp * p.ps;
   const bool two = d + 1 < p.D;
-  const float ks = p.ks[(int64_t)page * p.ks_sp + (int64_t)h * p.ks_sh];
-  const float vs = p.vs[(int64_t)page * p.vs_sp + (int64_t)h * p.vs_sh];
-  const uint16_t* kn = p.kn + (int64_t)b * p.kn_sb + (int64_t)h * p.kn_sh + (int64_t)d * p.kn_sd;
-  const uint16_t* vn = p.vn + (int64_t)b * p.vn_sb + (int64_t)h * p.vn_sh + (int64_t)d * p.vn_sd;
+  const uint16_t* knr = p.kn + (int64_t)b * p.kn_sb + (int64_t)h * p.kn_sh;
+  const uint16_t* vnr = p.vn + (int64_t)b * p.vn_sb + (int64_t)h * p.vn_sh;
+  const int64_t kso = (int64_t)page * p.ks_sp + (int64_t)slot * p.ks_st + (int64_t)h * p.ks_sh;
+  const int64_t vso = (int64_t)page * p.vs_sp + (int64_t)slot * p.vs_st + (int64_t)h * p.vs_sh;
+  // A per-token scale is the new token's own: every thread of the row
+  // derives it from the row's D values, the row's first thread stores it.
+  const float ks = p.k_tok ? row_token_scale(knr, p.kn_sd, p.D) : p.ks[kso];
+  const float vs = p.v_tok ? row_token_scale(vnr, p.vn_sd, p.D) : p.vs[vso];
+  if (d == 0) {
+    if (p.k_tok) p.ksw[kso] = ks;
+    if (p.v_tok) p.vsw[vso] = vs;
+  }
+  const uint16_t* kn = knr + (int64_t)d * p.kn_sd;
+  const uint16_t* vn = vnr + (int64_t)d * p.vn_sd;
   const float k0 = __fdiv_rn(bf16_bits_to_float(kn[0]), ks);
   const float k1 = two ? __fdiv_rn(bf16_bits_to_float(kn[p.kn_sd]), ks) : 0.f;
   const float v0 = __fdiv_rn(bf16_bits_to_float(vn[0]), vs);
@@ -2268,7 +2364,7 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
 // ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
-template <int D, bool KCVT, bool VCVT>
+template <int D, bool KCVT, bool VCVT, bool TOK>
 static cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap& tmk,
                                    const CUtensorMap& tmv, cudaStream_t s) {
   // The shared-memory opt-in is a per-device function attribute: set it once
@@ -2280,34 +2376,42 @@ static cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap& tmk
   if (e != cudaSuccess) return e;
   const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
   if (!bit || !(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(decode_tma_kernel<D, KCVT, VCVT>,
+    e = cudaFuncSetAttribute(decode_tma_kernel<D, KCVT, VCVT, TOK>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
   const dim3 grid = p.prop ? dim3(p.Hkv * p.head_groups, p.nbx, 1)
                            : dim3(p.Hkv * p.head_groups, p.B, p.num_splits);
-  decode_tma_kernel<D, KCVT, VCVT><<<grid, 128, smem, s>>>(p, tmk, tmv);
+  decode_tma_kernel<D, KCVT, VCVT, TOK><<<grid, 128, smem, s>>>(p, tmk, tmv);
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool TOK>
 static cudaError_t launch_decode_kv(const DecodeParams& p, const CUtensorMap& tmk,
                                    const CUtensorMap& tmv, bool k_cvt, bool v_cvt, cudaStream_t s) {
   if (k_cvt)
-    return v_cvt ? launch_decode_d<D, true, true>(p, tmk, tmv, s)
-                 : launch_decode_d<D, true, false>(p, tmk, tmv, s);
-  return v_cvt ? launch_decode_d<D, false, true>(p, tmk, tmv, s)
-               : launch_decode_d<D, false, false>(p, tmk, tmv, s);
+    return v_cvt ? launch_decode_d<D, true, true, TOK>(p, tmk, tmv, s)
+                 : launch_decode_d<D, true, false, TOK>(p, tmk, tmv, s);
+  return v_cvt ? launch_decode_d<D, false, true, TOK>(p, tmk, tmv, s)
+               : launch_decode_d<D, false, false, TOK>(p, tmk, tmv, s);
+}
+
+template <int D>
+static cudaError_t launch_decode_dt(const DecodeParams& p, const CUtensorMap& tmk,
+                                    const CUtensorMap& tmv, bool k_cvt, bool v_cvt,
+                                    cudaStream_t s) {
+  if (p.k_tok || p.v_tok) return launch_decode_kv<D, true>(p, tmk, tmv, k_cvt, v_cvt, s);
+  return launch_decode_kv<D, false>(p, tmk, tmv, k_cvt, v_cvt, s);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                           bool k_cvt, bool v_cvt, cudaStream_t s) {
   switch (p.D) {
-    case 64: return launch_decode_kv<64>(p, tmk, tmv, k_cvt, v_cvt, s);
-    case 128: return launch_decode_kv<128>(p, tmk, tmv, k_cvt, v_cvt, s);
-    case 256: return launch_decode_kv<256>(p, tmk, tmv, k_cvt, v_cvt, s);
-    case 512: return launch_decode_kv<512>(p, tmk, tmv, k_cvt, v_cvt, s);
+    case 64: return launch_decode_dt<64>(p, tmk, tmv, k_cvt, v_cvt, s);
+    case 128: return launch_decode_dt<128>(p, tmk, tmv, k_cvt, v_cvt, s);
+    case 256: return launch_decode_dt<256>(p, tmk, tmv, k_cvt, v_cvt, s);
+    case 512: return launch_decode_dt<512>(p, tmk, tmv, k_cvt, v_cvt, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -2397,9 +2501,9 @@ static int blocks_per_sm_d() {
   int c = cached.load();
   if (c >= 0) return c;
   int n = 0;
-  if (cudaFuncSetAttribute(decode_tma_kernel<D, true, true>,
+  if (cudaFuncSetAttribute(decode_tma_kernel<D, true, true, false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tma_kernel<D, true, true>, 128,
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tma_kernel<D, true, true, false>, 128,
                                                     Cfg<D>::SMEM) != cudaSuccess) {
     cudaGetLastError();
     return Cfg<D>::MIN_BLOCKS;  // no device: do not cache the guess

@@ -81,9 +81,12 @@ typedef struct fp8pd_tensor {
   int64_t stride[4];
 } fp8pd_tensor;
 
-/* K and V scales for fp8_kv_append (read only). Each is float32 of shape
- * [Hkv] (one scale per KV head) or [num_pages, Hkv] (one per physical page
- * and KV head, indexed by the page id found in the block table). */
+/* K and V scales for fp8_kv_append. Each is float32 of shape [Hkv] (one
+ * scale per KV head), [num_pages, Hkv] (one per physical page and KV head,
+ * indexed by the page id found in the block table) -- both read only -- or
+ * [num_pages, ps, Hkv] (one per stored token and KV head, the cache-write
+ * quantizer's per-token-per-head form named in the solution page's
+ * "Supported scope"), which the append writes. */
 typedef struct fp8pd_scales {
   fp8pd_tensor k_scale;
   fp8pd_tensor v_scale;
@@ -125,7 +128,7 @@ enum {
  *
  * Defines (for each sequence b and query head hq, h = hq / (Hq / Hkv)):
  *   keys t in [lo, L), L = seq_lens[b], lo = window > 0 ? max(0, L - window) : 0
- *   K(t, d) = e4m3(k_pages[page(t), t % ps, h, d]) * k_scale(page(t), h)
+ *   K(t, d) = e4m3(k_pages[page(t), t % ps, h, d]) * k_scale(page(t), t % ps, h)
  *   V(t, d) likewise, page(t) = block_table[b, t / ps]
  *   s_t = sm_scale * sum_d q[b, hq, d] * K(t, d)
  *   M = max(max_t s_t, sink[hq]);  den = sum_t exp(s_t - M) + exp(sink[hq] - M)
@@ -147,8 +150,12 @@ enum {
  *                strides; the 16-byte rule follows DeepGEMM PR #459's paged
  *                accessor). D in {64, 128, 256, 512}; ps a multiple of 16, <= 256;
  *                num_pages < 2^27.
- *   k_scale,     float32 [Hkv] or [num_pages, Hkv], any strides (0 = broadcast).
- *   v_scale
+ *   k_scale,     float32 [Hkv] (per KV head), [num_pages, Hkv] (per page and KV
+ *   v_scale      head) or [num_pages, ps, Hkv] (per stored token and KV head),
+ *                any strides (0 = broadcast); k_scale(page, slot, h) ignores
+ *                the missing axes. K and V may use different forms. With a
+ *                per-token form the segment schedule is not used (a request
+ *                for it runs the split kernel's own plan).
  *   block_table  int32 [B, max_pages]: physical page of each logical page.
  *                Entries past the attended range are never read.
  *   seq_lens     int32 [B]: number of keys visible to the query (positions 0..L-1).
@@ -187,11 +194,14 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
  * fp8_kv_append -- quantize one new token per sequence and store it.
  *
  * For each b and KV head h, with p = positions[b], page = block_table[b, p / ps]:
- *   k_pages[page, p % ps, h, d] = E4M3_RNE_SAT( float(k_new[b, h, d]) / k_scale(page, h) )
+ *   k_pages[page, p % ps, h, d] = E4M3_RNE_SAT( float(k_new[b, h, d]) / ks )
  * and the same for V. The division is IEEE float32 round-to-nearest; the
  * rounding to E4M3 is round-to-nearest-even, saturating to +-448 (a NaN
- * input gives the NaN code). Scales are read only. Nothing else in the
- * pools is written. The new token is then visible to an attention call with
+ * input gives the NaN code). A per-head or per-page scale is read only:
+ * ks = k_scale(page, h). A per-token scale ([num_pages, ps, Hkv]) is the new
+ * token's own, ks = max_d |k_new[b, h, d]| / 448 in IEEE float32 (NaN entries
+ * skipped, 1 for an all-zero row), and is written to k_scale[page, p % ps, h].
+ * Nothing else in the pools or scales is written. The new token is then visible to an attention call with
  * seq_lens[b] = p + 1 (the "Lecture 8" page's kv-cache update before the
  * decode attention).
  *
@@ -218,7 +228,8 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
  * For each sequence b, with pos = positions[b]: the new token (k_new[b],
  * v_new[b], bf16 [B, Hkv, D]) is quantized exactly as fp8_kv_append does
  * (E4M3 code = round-to-nearest-even(float32 x / scale), saturated to +-448,
- * with the scale of the page that holds position pos), written at position
+ * with the scale of the page that holds position pos, or with a per-token
+ * form the token's own max|x| / 448, which is written too), written at position
  * pos of the pools, and the query then attends over the pos + 1 keys
  * 0 .. pos, the new one included -- the result of fp8_kv_append(..., positions)
  * followed by fp8_paged_decode_attention(..., seq_lens = positions + 1),

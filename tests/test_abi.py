@@ -86,6 +86,11 @@ def _call(F, a):
     (dict(sm_scale=float("nan")), -6),
     (dict(ks=torch.ones(3)), -3),
     (dict(vs=torch.ones(5, 2)), -3),
+    (dict(ks=torch.ones(6, 8, 2)), -3),                                      # per-token: ps
+    (dict(vs=torch.ones(5, 16, 2)), -3),                                     # per-token: pages
+    (dict(ks=torch.ones(6, 16, 3)), -3),                                     # per-token: Hkv
+    (dict(vs=torch.ones(6, 16, 2, 1)), -3),                                  # 4-D scale
+    (dict(ks=torch.ones(6, 16, 2, dtype=torch.float64)), -2),
     (dict(sinks=torch.zeros(7)), -3),
     (dict(table=torch.zeros(3, 3, dtype=torch.int32)), -3),
     (dict(lens=torch.zeros(2, dtype=torch.int64)), -2),
@@ -149,6 +154,9 @@ def test_append_validation(F):
     assert e.value.status == -3
     with pytest.raises(F.Fp8pdError) as e:
         F.fp8_kv_append(kn, kn, kp, kp, ks, ks, tbl, torch.zeros(3, dtype=torch.int32), stream=0)
+    assert e.value.status == -3
+    with pytest.raises(F.Fp8pdError) as e:                  # per-token scale with the wrong ps
+        F.fp8_kv_append(kn, kn, kp, kp, torch.ones(4, 8, 2), ks, tbl, pos, stream=0)
     assert e.value.status == -3
 
 

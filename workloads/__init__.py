@@ -44,7 +44,7 @@ class Spec:
     ps: int
     layers: tuple                       # tuple[LayerSpec, ...]; >1 = layers sharing one pool
     seq_len: int | tuple = 256          # int, or (lo, hi) inclusive uniform range per sequence
-    scale_mode: str = "head"            # "head": [Hkv]; "page": [num_pages, Hkv]
+    scale_mode: str = "head"            # "head": [Hkv]; "page": [num_pages, Hkv]; "token": [num_pages, ps, Hkv]
     dist: str = "normal"                # "normal": N(0,1); "normal2_outliers": N(0,2), 1% x20
     sinks: bool = False
     append: bool = False                # one new token per sequence at position seq_len
@@ -84,7 +84,7 @@ class LayerCase:
     q: torch.Tensor                     # [B, Hq, D] bf16
     k_pages: torch.Tensor               # [num_pages, ps, Hkv, D] uint8 view of the K pool
     v_pages: torch.Tensor
-    k_scale: torch.Tensor               # [Hkv] or [num_pages, Hkv] float32
+    k_scale: torch.Tensor               # [Hkv], [num_pages, Hkv] or [num_pages, ps, Hkv] float32
     v_scale: torch.Tensor
     block_table: torch.Tensor           # [B, max_pages] int32 (-1 = unused entry)
     sinks: torch.Tensor | None          # [Hq] float32
@@ -225,11 +225,16 @@ def make_case(name_or_spec, device="cpu", chunk_pages: int = 1024, **overrides) 
             # pass 1: scales from the values (including the token to append)
             if spec.scale_mode == "head":
                 amax = torch.zeros(L.Hkv, device=device)
+            elif spec.scale_mode == "token":
+                amax = torch.zeros(total_pages, spec.ps, L.Hkv, device=device)
             else:
                 amax = torch.zeros(total_pages, L.Hkv, device=device)
             for p0 in range(0, total_pages, chunk_pages):
                 p1 = min(total_pages, p0 + chunk_pages)
                 x = page_values_bf16_new(page_values(p0, p1, which), p0, p1)
+                if spec.scale_mode == "token":
+                    amax[p0:p1] = x.abs().amax(dim=3)             # [pages, ps, Hkv]
+                    continue
                 a = x.abs().amax(dim=(1, 3))                      # [pages, Hkv]
                 if spec.scale_mode == "head":
                     amax = torch.maximum(amax, a.amax(dim=0))
@@ -243,8 +248,12 @@ def make_case(name_or_spec, device="cpu", chunk_pages: int = 1024, **overrides) 
             for p0 in range(0, total_pages, chunk_pages):
                 p1 = min(total_pages, p0 + chunk_pages)
                 x = page_values_bf16_new(page_values(p0, p1, which), p0, p1)
-                sc = scale.view(1, 1, L.Hkv, 1) if spec.scale_mode == "head" else \
-                    scale[p0:p1].view(-1, 1, L.Hkv, 1)
+                if spec.scale_mode == "head":
+                    sc = scale.view(1, 1, L.Hkv, 1)
+                elif spec.scale_mode == "token":
+                    sc = scale[p0:p1].view(-1, spec.ps, L.Hkv, 1)
+                else:
+                    sc = scale[p0:p1].view(-1, 1, L.Hkv, 1)
                 codes = (x / sc).to(torch.float8_e4m3fn).view(torch.uint8)
                 if spec.append:
                     for b in range(spec.B):
@@ -268,7 +277,9 @@ def make_case(name_or_spec, device="cpu", chunk_pages: int = 1024, **overrides) 
 def algorithmic_bytes(case: Case, layer: int = 0) -> int:
     """Bytes a decode step must read for one layer: the attended K and V bytes
     (window-limited, once per KV head), q, and the block-table entries of the
-    attended pages. Scales, the output and split partials are not counted."""
+    attended pages; with per-token scales also the attended tokens' K and V
+    scales (4 bytes each per KV head). Per-head and per-page scales, the
+    output and split partials are not counted."""
     L = case.layers[layer]
     lens = case.attend_lens.cpu().numpy().astype(np.int64)
     ps = case.spec.ps
@@ -281,7 +292,9 @@ def algorithmic_bytes(case: Case, layer: int = 0) -> int:
         if n > 0:
             tbl += 4 * ((Lb - 1) // ps - lo // ps + 1)
     q = L.q.numel() * 2
-    return int(kv + q + tbl)
+    # per-token scales: 4 bytes per attended token and KV head, for K and for V
+    tok_scales = sum(kv // L.spec.D * 2 for sc in (L.k_scale, L.v_scale) if sc.dim() == 3)
+    return int(kv + q + tbl + tok_scales)
 
 
 def describe(spec: Spec) -> str:
