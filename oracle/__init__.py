@@ -13,7 +13,9 @@ from .fp8pd_oracle import (  # noqa: F401
     e4m3_code_value,
     e4m3_decode,
     e4m3_encode,
+    expand_groups,
     gather_tokens,
+    group_scale,
     kv_append,
     paged_decode_attention,
     quantize,

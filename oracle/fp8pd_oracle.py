@@ -38,7 +38,9 @@ Readings of the pages (each is listed with its reason in the design notes):
   per-token-per-head form (P1 "Supported scope", ``quantize_kv_fp8``) keeps
   one scale per stored (page, slot, KV head), shaped like the cache without
   its last axis, and is max|x| / 448 of that token and head in float32 (an
-  all-zero row takes scale 1); the append writes it with the codes.
+  all-zero row takes scale 1); the append writes it with the codes. Sub-row
+  groups (P1 "Supported scope", ``k_groups``) add a last axis of ``groups``
+  scales, group g covering entries [g D/groups, (g+1) D/groups).
 * empty attention (no keys, no sink) returns 0.
 """
 
@@ -167,6 +169,26 @@ def quantize_per_token(x) -> tuple[np.ndarray, np.ndarray]:
     return quantize(x, s[..., None]), s
 
 
+def group_scale(x, groups: int) -> np.ndarray:
+    """Sub-row scales of ``x`` [..., D]: the D values of a row cut into
+    ``groups`` equal runs of D / groups consecutive entries, each with its own
+    :func:`token_scale`. Returns [..., groups] (P1 "Supported scope":
+    ``k_groups`` sub-row key scales, ``quantize_kv_fp8`` with sub-row groups).
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    D = x32.shape[-1]
+    if groups < 1 or D % groups:
+        raise ValueError("groups must divide the head dim")
+    return token_scale(x32.reshape(*x32.shape[:-1], groups, D // groups))
+
+
+def expand_groups(scales: np.ndarray, D: int) -> np.ndarray:
+    """[..., groups] sub-row scales -> [..., D]: entry d takes the scale of its
+    group d // (D / groups)."""
+    scales = np.asarray(scales)
+    return np.repeat(scales, D // scales.shape[-1], axis=-1)
+
+
 # ---------------------------------------------------------------------------
 # Paged gather, attention and append
 # ---------------------------------------------------------------------------
@@ -174,13 +196,27 @@ def quantize_per_token(x) -> tuple[np.ndarray, np.ndarray]:
 def _scale_of(scale: np.ndarray, page: np.ndarray, slot: np.ndarray, head: int) -> np.ndarray:
     """Scale of the token stored at (physical page, slot) for KV head ``head``:
     ``scale`` is [Hkv] (per KV head), [num_pages, Hkv] (per physical page and
-    KV head) or [num_pages, ps, Hkv] (per stored token and KV head)."""
+    KV head) or [num_pages, ps, Hkv] (per stored token and KV head). With
+    [num_pages, ps, Hkv, groups] (sub-row groups) the result has a trailing
+    axis of the token's group scales."""
     scale = np.asarray(scale)
     if scale.ndim == 1:
         return np.full(np.shape(page), np.float64(scale[head]))
     if scale.ndim == 2:
         return scale[page, head].astype(np.float64)
-    return scale[page, slot, head].astype(np.float64)
+    if scale.ndim == 3:
+        return scale[page, slot, head].astype(np.float64)
+    return scale[page, slot, head, :].astype(np.float64)
+
+
+def _dequantize(codes: np.ndarray, scale: np.ndarray, page, slot, head: int) -> np.ndarray:
+    """Values of the codes [n, D] of KV head ``head`` stored at (page, slot):
+    decode(code) times the scale of each entry (a group scale, when the scale
+    array has sub-row groups, covers its run of D / groups entries)."""
+    s = _scale_of(scale, page, slot, head)
+    D = codes.shape[-1]
+    s = expand_groups(s, D) if np.ndim(scale) == 4 else s[..., None]
+    return e4m3_decode(codes) * s
 
 
 def gather_tokens(pages: np.ndarray, block_table_row: np.ndarray, positions: np.ndarray,
@@ -211,15 +247,16 @@ def paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_table, s
 
     q [B, Hq, D] (bf16 values given as floats), k_pages / v_pages
     [num_pages, ps, Hkv, D] uint8 codes, k_scale / v_scale [Hkv],
-    [num_pages, Hkv] or [num_pages, ps, Hkv] float32, block_table [B, max_pages] int32,
-    seq_lens [B] = number of keys 0..L-1 visible to the query,
+    [num_pages, Hkv] or [num_pages, ps, Hkv] float32, or
+    [num_pages, ps, Hkv, groups] (sub-row groups of D / groups entries),
+    block_table [B, max_pages] int32, seq_lens [B] = number of keys 0..L-1 visible to the query,
     sinks [Hq] float32 or None. Returns out [B, Hq, D] float64.
 
     For each (b, hq), with h = hq // G and keys t in [lo, L):
       s_t  = sm_scale * sum_d q[b,hq,d] * K(t,d)
       M    = max(max_t s_t, sink)
       out  = sum_t exp(s_t - M) V(t) / (sum_t exp(s_t - M) + exp(sink - M))
-    where K(t,d) = decode(code) * k_scale(page(t), slot(t), h). This is plain softmax
+    where K(t,d) = decode(code) * k_scale(page(t), slot(t), h[, d // (D / groups)]). This is plain softmax
     attention over the dequantized values (P1 "Smallest correct example"),
     with the window, sinks and scale of P1 "Expected result".
 
@@ -248,8 +285,8 @@ def paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_table, s
             kc, phys = gather_tokens(k_pages, block_table[b], positions, h)
             vc, _ = gather_tokens(v_pages, block_table[b], positions, h)
             slots = positions % k_pages.shape[1]
-            K = e4m3_decode(kc) * _scale_of(k_scale, phys, slots, h)[:, None]
-            V = e4m3_decode(vc) * _scale_of(v_scale, phys, slots, h)[:, None]
+            K = _dequantize(kc, k_scale, phys, slots, h)
+            V = _dequantize(vc, v_scale, phys, slots, h)
             for hq in heads:
                 s = sm * (K @ q[b, hq])
                 sink = None if sinks is None else float(sinks[hq])
@@ -269,13 +306,16 @@ def kv_append(k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table, pos
 
     k_new / v_new [B, Hkv, D] (bf16 values as floats), pages
     [num_pages, ps, Hkv, D] uint8 (numpy arrays, written in place), scales
-    [Hkv], [num_pages, Hkv] or [num_pages, ps, Hkv] float32, positions [B].
+    [Hkv], [num_pages, Hkv], [num_pages, ps, Hkv] or
+    [num_pages, ps, Hkv, groups] float32, positions [B].
     Token position p of sequence b goes to page block_table[b, p // ps], slot
     p % ps, as code = E4M3(float32(x) / scale) (P1 "Supported scope", the
     one-launch T=1 append; P2 "In-kernel KV cache update"). A per-head or
     per-page scale is read only. A per-token scale is the new token's own
     (:func:`token_scale` of its D values, per KV head) and is written to
-    ``scale[page, slot, h]`` with the codes.
+    ``scale[page, slot, h]`` with the codes; with sub-row groups each group's
+    scale (:func:`group_scale`) is written to ``scale[page, slot, h, g]`` and
+    quantizes its run of entries.
     """
     B, Hkv, _ = np.shape(k_new)
     ps = k_pages.shape[1]
@@ -286,6 +326,11 @@ def kv_append(k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table, pos
         for h in range(Hkv):
             for x, pages, scale in ((k_new[b][h], k_pages, k_scale), (v_new[b][h], v_pages, v_scale)):
                 x32 = np.asarray(x, np.float32)
+                if np.ndim(scale) == 4:
+                    scale[page, slot, h, :] = group_scale(x32, np.shape(scale)[3])
+                    s = expand_groups(np.asarray(scale[page, slot, h, :], np.float32), x32.shape[-1])
+                    pages[page, slot, h, :] = quantize(x32, s)
+                    continue
                 if np.ndim(scale) == 3:
                     scale[page, slot, h] = token_scale(x32)
                 s = np.float32(_scale_of(scale, np.array(page), np.array(slot), h))

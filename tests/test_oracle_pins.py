@@ -571,3 +571,109 @@ def test_append_per_token_writes_its_scale_and_codes():
             assert np.array_equal(pages[p, s], lib)
     assert np.array_equal(kp[~touched], k0[~touched]) and np.array_equal(vp[~touched], v0[~touched])
     assert np.array_equal(ks[~touched], ks0[~touched]) and np.array_equal(vs[~touched], vs0[~touched])
+
+
+# ---------------------------------------------------------------- sub-row key groups
+
+def test_group_scale_matches_library():
+    g = torch.Generator().manual_seed(31)
+    x = (torch.randn(40, 2, 128, generator=g) * 9).to(torch.bfloat16).float()
+    for G in (1, 2, 4, 8):
+        want = (x.view(40, 2, G, 128 // G).abs().amax(-1) / torch.tensor(448.0)).numpy()
+        got = O.group_scale(x.numpy(), G)
+        assert got.shape == (40, 2, G) and np.array_equal(got, want)
+    assert np.array_equal(O.group_scale(x.numpy(), 1)[..., 0], O.token_scale(x.numpy()))
+
+
+def test_one_group_equals_per_token():
+    rng = np.random.default_rng(32)
+    c = _dense_case(rng, scale_mode="token")
+    c4 = dict(c, ks=c["ks"][..., None])
+    for w in (0, 13):
+        assert np.array_equal(_run(c, window=w, sm_scale=0.3), _run(c4, window=w, sm_scale=0.3))
+
+
+def test_grouped_key_scales_match_library_sdpa():
+    """K scales per (token, KV head, group of D/4 entries), dequantized here
+    by index arithmetic of the test's own, against torch SDPA."""
+    rng = np.random.default_rng(33)
+    c = _dense_case(rng, scale_mode="token")
+    total, ps, Hkv = c["ks"].shape
+    G, D = 4, c["k"].shape[-1]
+    ks4 = rng.uniform(0.001, 0.05, size=(total, ps, Hkv, G)).astype(np.float32)
+    sinks = rng.standard_normal(8).astype(np.float32)
+    got = _run(dict(c, ks=ks4), window=9, sinks=sinks, sm_scale=0.4)
+    # fold each group's scale into the codes' values: a per-token K scale of 1
+    # and K values decoded by the library, times the group scale per entry
+    kval = torch.from_numpy(c["k"]).view(torch.float8_e4m3fn).double().numpy()
+    kval = kval * np.stack([ks4[..., d * G // D] for d in range(D)], axis=-1)
+    q, B = c["q"], c["q"].shape[0]
+    out = np.zeros_like(got)
+    for b in range(B):
+        L = int(c["lens"][b])
+        t = np.arange(L)
+        phys, slot = c["table"][b][t // ps], t % ps
+        for hq in range(q.shape[1]):
+            h = hq // (q.shape[1] // Hkv)
+            K = torch.from_numpy(kval[phys, slot, h])[None]
+            V = torch.from_numpy(torch.from_numpy(c["v"][phys, slot, h]).view(torch.float8_e4m3fn)
+                                 .double().numpy() * c["vs"][phys, slot, h][:, None])[None]
+            K = torch.cat([K, torch.zeros(1, 1, D, dtype=K.dtype)], 1)
+            V = torch.cat([V, torch.zeros(1, 1, D, dtype=V.dtype)], 1)
+            mask = np.zeros((1, 1, L + 1))
+            mask[..., :max(0, L - 9)] = -np.inf
+            mask[..., L] = sinks[hq]
+            o = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q[b, hq])[None, None], K, V, attn_mask=torch.from_numpy(mask),
+                scale=float(np.float32(0.4)))
+            out[b, hq] = o[0, 0].numpy()
+    assert np.allclose(got, out, rtol=1e-12, atol=1e-12)
+
+
+def test_grouped_key_scale_closed_form():
+    """q is 1 on the entries of group 2 and 0 elsewhere, every code is 0x38
+    (1.0); group 2's K scale is a * t at logical position t, the other groups'
+    scales are huge. The scores are sm * (D/4) * a * t, so out is the r^t
+    weighted mean of the V scale t, whatever the other groups hold."""
+    B, Hq, Hkv, D, ps = 3, 4, 2, 16, 16
+    table, k, v, lens, total = _logical_scale_case(B, Hq, Hkv, D, ps, seed=34)
+    a, sm, G = 0.01, 0.5, 4
+    ks = np.full((total, ps, Hkv, G), 1e6, np.float32)
+    vs = np.zeros((total, ps, Hkv), np.float32)
+    for b in range(B):
+        for t in range(lens[b]):
+            ks[table[b, t // ps], t % ps, :, 2] = np.float32(a * t)
+            vs[table[b, t // ps], t % ps, :] = t
+    q = np.zeros((B, Hq, D))
+    q[:, :, 2 * D // G:3 * D // G] = 1.0
+    out = O.paged_decode_attention(q, k, v, ks, vs, table, lens, sm_scale=sm)
+    for b in range(B):
+        t = np.arange(lens[b])
+        w = np.exp(sm * (D // G) * np.float32(a * t).astype(np.float64))
+        assert np.allclose(out[b], (w * t).sum() / w.sum(), rtol=1e-12)
+
+
+def test_append_grouped_key_scales():
+    rng = np.random.default_rng(35)
+    num_pages, ps, Hkv, D, B, G = 8, 16, 2, 64, 3, 4
+    kp = rng.integers(0, 256, (num_pages, ps, Hkv, D)).astype(np.uint8)
+    vp = kp.copy()
+    ks = rng.uniform(0.01, 0.02, (num_pages, ps, Hkv, G)).astype(np.float32)
+    vs = rng.uniform(0.01, 0.02, (num_pages, ps, Hkv)).astype(np.float32)
+    k0, ks0 = kp.copy(), ks.copy()
+    table = rng.permutation(num_pages)[:B * 2].reshape(B, 2).astype(np.int32)
+    pos = np.array([3, 16, 31])
+    g = torch.Generator().manual_seed(35)
+    kn = (torch.randn(B, Hkv, D, generator=g) * torch.tensor([1e-3, 1.0, 30.0, 0.1]).repeat_interleave(D // G)
+          ).to(torch.bfloat16).float()
+    vn = torch.randn(B, Hkv, D, generator=g).to(torch.bfloat16).float()
+    O.kv_append(kn.numpy(), vn.numpy(), kp, vp, ks, vs, table, pos)
+    touched = np.zeros((num_pages, ps), bool)
+    for b in range(B):
+        p, s = table[b, pos[b] // ps], pos[b] % ps
+        touched[p, s] = True
+        lib_s = (kn[b].view(Hkv, G, D // G).abs().amax(-1) / torch.tensor(448.0))
+        assert np.array_equal(ks[p, s], lib_s.numpy())
+        quot = kn[b] / lib_s.repeat_interleave(D // G, dim=-1)
+        assert np.array_equal(kp[p, s], quot.to(torch.float8_e4m3fn).view(torch.uint8).numpy())
+    assert np.array_equal(kp[~touched], k0[~touched]) and np.array_equal(ks[~touched], ks0[~touched])
