@@ -488,8 +488,8 @@ def _case_to_numpy(case: W.Case, seqs) -> tuple[dict, np.ndarray, np.ndarray | N
             lo = max(0, Lb - layer.window) if layer.window > 0 else 0
             n = Lb - lo
             nbytes += 2 * n * layer.spec.Hkv * layer.spec.D
-            nbytes += sum(4 * n * layer.spec.Hkv for sc in (layer.k_scale, layer.v_scale)
-                          if sc.dim() == 3)
+            nbytes += sum(4 * n * layer.spec.Hkv * (sc.shape[3] if sc.dim() == 4 else 1)
+                          for sc in (layer.k_scale, layer.v_scale) if sc.dim() >= 3)
             if n > 0:
                 nbytes += 4 * ((Lb - 1) // ps - lo // ps + 1)
         nbytes += 2 * d["q"].size
@@ -523,17 +523,25 @@ def cpu_baseline(case: W.Case, budget_s: float = 10.0) -> dict:
 def _scale_override(args) -> dict:
     """``--scales token``: the workload with one scale per stored token and KV
     head instead of its own scale form."""
-    return {"scale_mode": "token"} if args.scales == "token" else {}
+    if args.scales != "token":
+        return {}
+    return {"scale_mode": "token", "k_groups": args.k_groups}
 
 
 def _workload_text(args) -> str:
     text = WORKLOAD_TEXT.get(args.config, args.config)
-    return text + " (scales replaced: per (token, KV head))" if args.scales == "token" else text
+    if args.scales != "token":
+        return text
+    groups = f", K in {args.k_groups} sub-row groups" if args.k_groups > 1 else ""
+    return text + f" (scales replaced: per (token, KV head){groups})"
 
 
 def _scales_text(case) -> str:
-    return {"head": "per KV head", "page": "per (page, KV head)",
+    text = {"head": "per KV head", "page": "per (page, KV head)",
             "token": "per (token, KV head)"}[case.spec.scale_mode]
+    if case.spec.scale_mode == "token" and case.spec.k_groups > 1:
+        text += f"; K per (token, KV head, group of D/{case.spec.k_groups})"
+    return text
 
 
 def run_reference(args) -> dict | None:
@@ -594,6 +602,8 @@ def main():
     ap.add_argument("--splits", type=int, default=0, help="force a split count (0 = planner)")
     ap.add_argument("--scales", default="workload", choices=["workload", "token"],
                     help="token: per-token-per-head K/V scales instead of the workload's form")
+    ap.add_argument("--k-groups", type=int, default=1,
+                    help="with --scales token: K scales per sub-row group of D / k_groups entries")
     ap.add_argument("--schedule", type=int, default=0, choices=[0, 1, 2, 3],
                     help="0 = planner, 1 = uniform splits, 2 = segment kernel, "
                          "3 = proportional splits")

@@ -162,7 +162,8 @@ def fp8_paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_tabl
     q [B, Hq, D] bf16; k_pages / v_pages [num_pages, ps, Hkv, D] uint8 views
     (any page stride that is a multiple of 16 bytes); k_scale / v_scale
     float32 [Hkv], [num_pages, Hkv] or [num_pages, ps, Hkv] (per stored
-    token and KV head); block_table int32 [B, max_pages];
+    token and KV head; K also [num_pages, ps, Hkv, G], one scale per run of
+    D / G head-dim entries); block_table int32 [B, max_pages];
     seq_lens int32 [B] (keys visible to the query); sinks float32 [Hq] or
     None; sm_scale defaults to D ** -0.5. Returns out [B, Hq, D] float32.
     """

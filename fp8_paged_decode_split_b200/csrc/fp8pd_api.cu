@@ -70,16 +70,21 @@ int check(const fp8pd_tensor* t, int32_t dtype, int32_t ndim) {
 
 bool fits_i32(int64_t v) { return v >= 0 && v <= INT32_MAX; }
 
-// Scale descriptor -> (page, slot, head) strides in elements; *tok = 1 for
-// the per-token form [num_pages, ps, Hkv] (one scale per stored token and KV
-// head), 0 for [Hkv] (slot and page strides 0) and [num_pages, Hkv] (slot
-// stride 0).
-int scale_strides(const fp8pd_tensor* s, int64_t num_pages, int64_t ps, int64_t hkv, int64_t* sp,
-                  int64_t* st, int64_t* sh, int* tok) {
+// Scale descriptor -> (page, slot, head, group) strides in elements; *tok =
+// 1 for the per-token form [num_pages, ps, Hkv] (one scale per stored token
+// and KV head), 0 for [Hkv] (slot and page strides 0) and [num_pages, Hkv]
+// (slot stride 0). [num_pages, ps, Hkv, groups] adds sub-row groups (*groups
+// = the last extent, a power of two up to 16 dividing d; 1 otherwise);
+// `max_groups` caps it (1: no sub-row groups).
+int scale_strides(const fp8pd_tensor* s, int64_t num_pages, int64_t ps, int64_t hkv, int64_t d,
+                  int max_groups, int64_t* sp, int64_t* st, int64_t* sh, int64_t* sg, int* tok,
+                  int* groups) {
   if (!s || !s->data) return FP8PD_ERR_NULL;
   if (s->dtype != FP8PD_DTYPE_F32) return FP8PD_ERR_DTYPE;
   *st = 0;
+  *sg = 0;
   *tok = 0;
+  *groups = 1;
   if (s->ndim == 1) {
     if (s->shape[0] != hkv) return FP8PD_ERR_SHAPE;
     *sp = 0;
@@ -92,12 +97,19 @@ int scale_strides(const fp8pd_tensor* s, int64_t num_pages, int64_t ps, int64_t 
     *sh = s->stride[1];
     return FP8PD_OK;
   }
-  if (s->ndim == 3) {
+  if (s->ndim == 3 || s->ndim == 4) {
     if (s->shape[0] != num_pages || s->shape[1] != ps || s->shape[2] != hkv) return FP8PD_ERR_SHAPE;
     *sp = s->stride[0];
     *st = s->stride[1];
     *sh = s->stride[2];
     *tok = 1;
+    if (s->ndim == 4) {
+      const int64_t g = s->shape[3];
+      if (g < 1 || g > 16 || (g & (g - 1)) || d % g) return FP8PD_ERR_UNSUPPORTED;
+      if (g > max_groups) return FP8PD_ERR_UNSUPPORTED;
+      *sg = s->stride[3];
+      *groups = static_cast<int>(g);
+    }
     return FP8PD_OK;
   }
   return FP8PD_ERR_SHAPE;
@@ -448,10 +460,16 @@ int validate_decode(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp
     return FP8PD_ERR_ALIGN;
   if (window < 0) return FP8PD_ERR_ARG;
   if (!(std::isfinite(sm_scale) && sm_scale > 0.f)) return FP8PD_ERR_ARG;
-  int64_t ks_sp, ks_st, ks_sh, vs_sp, vs_st, vs_sh;
-  int k_tok, v_tok;
-  if ((r = scale_strides(k_scale, P, ps, Hkv, &ks_sp, &ks_st, &ks_sh, &k_tok))) return r;
-  if ((r = scale_strides(v_scale, P, ps, Hkv, &vs_sp, &vs_st, &vs_sh, &v_tok))) return r;
+  // Sub-row K groups: each covers whole 16-entry blocks of the QK contraction
+  // (D / groups >= 16); V takes one scale per token at most.
+  int64_t ks_sp, ks_st, ks_sh, ks_sg, vs_sp, vs_st, vs_sh, vs_sg;
+  int k_tok, v_tok, k_groups, v_groups;
+  if ((r = scale_strides(k_scale, P, ps, Hkv, D, static_cast<int>(D / 16), &ks_sp, &ks_st, &ks_sh,
+                         &ks_sg, &k_tok, &k_groups)))
+    return r;
+  if ((r = scale_strides(v_scale, P, ps, Hkv, D, 1, &vs_sp, &vs_st, &vs_sh, &vs_sg, &v_tok,
+                         &v_groups)))
+    return r;
   if (sinks) {
     if ((r = check(sinks, FP8PD_DTYPE_F32, 1))) return r;
     if (sinks->shape[0] != Hq) return FP8PD_ERR_SHAPE;
@@ -484,6 +502,8 @@ int validate_decode(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp
   p->vs_st = vs_st;
   p->k_tok = k_tok;
   p->v_tok = v_tok;
+  p->ks_sg = ks_sg;
+  p->k_groups = k_groups;
   p->table = static_cast<const int32_t*>(block_table->data);
   p->tab_sb = block_table->stride[0];
   p->tab_sp = block_table->stride[1];
@@ -778,10 +798,14 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
   if (k_pages->shape[2] != Hkv || k_pages->shape[3] != D) return FP8PD_ERR_SHAPE;
   if (block_table->shape[0] != B || positions->shape[0] != B) return FP8PD_ERR_SHAPE;
   if (ps < 1) return FP8PD_ERR_UNSUPPORTED;
-  int64_t ks_sp, ks_st, ks_sh, vs_sp, vs_st, vs_sh;
-  int k_tok, v_tok;
-  if ((r = scale_strides(&scales->k_scale, P, ps, Hkv, &ks_sp, &ks_st, &ks_sh, &k_tok))) return r;
-  if ((r = scale_strides(&scales->v_scale, P, ps, Hkv, &vs_sp, &vs_st, &vs_sh, &v_tok))) return r;
+  int64_t ks_sp, ks_st, ks_sh, ks_sg, vs_sp, vs_st, vs_sh, vs_sg;
+  int k_tok, v_tok, k_groups, v_groups;
+  if ((r = scale_strides(&scales->k_scale, P, ps, Hkv, D, 16, &ks_sp, &ks_st, &ks_sh, &ks_sg,
+                         &k_tok, &k_groups)))
+    return r;
+  if ((r = scale_strides(&scales->v_scale, P, ps, Hkv, D, 1, &vs_sp, &vs_st, &vs_sh, &vs_sg,
+                         &v_tok, &v_groups)))
+    return r;
   const int64_t max_pages = block_table->shape[1];
   if (!fits_i32(B) || !fits_i32(P) || !fits_i32(Hkv) || !fits_i32(D) || !fits_i32(max_pages) ||
       max_pages * ps > INT32_MAX || B * Hkv * ((D + 1) / 2) > (int64_t(1) << 40))
@@ -815,6 +839,8 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
   p.vs_st = vs_st;
   p.k_tok = k_tok;
   p.v_tok = v_tok;
+  p.ks_sg = ks_sg;
+  p.k_groups = k_groups;
   p.ksw = static_cast<float*>(scales->k_scale.data);
   p.vsw = static_cast<float*>(scales->v_scale.data);
   p.table = static_cast<const int32_t*>(block_table->data);

@@ -22,6 +22,8 @@ struct DecodeParams {
   int64_t ks_sp, ks_sh, vs_sp, vs_sh;
   int64_t ks_st, vs_st;       // 0 unless the scales are per token
   int k_tok, v_tok;           // 1: per-token-per-head scales [num_pages, ps, Hkv]
+  int64_t ks_sg;              // K sub-row groups [num_pages, ps, Hkv, k_groups]: group stride
+  int k_groups;               // 1, or 2..16 (D / k_groups >= 16): K entry d uses group d / (D / k_groups)
   const int32_t* table;       // [B, max_pages]
   int64_t tab_sb, tab_sp;
   const int32_t* lens;        // [B]
@@ -78,6 +80,8 @@ struct AppendParams {
   int64_t ks_sp, ks_sh, vs_sp, vs_sh;
   int64_t ks_st, vs_st;       // slot strides (per-token scales), else 0
   int k_tok, v_tok;           // 1: the scale is the new token's own max|x| / 448, written here
+  int64_t ks_sg;              // K sub-row groups: group stride; k_groups groups of D / k_groups
+  int k_groups;
   float* ksw;
   float* vsw;
   const int32_t* table;

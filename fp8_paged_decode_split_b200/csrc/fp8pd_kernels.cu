@@ -493,6 +493,58 @@ __device__ __forceinline__ float4 tile_scores(const QFrag& qfr, uint32_t sk,
                      vb ? (Sa[3] + Sb[3]) * kfb : -CUDART_INF_F);
 }
 
+// tile_scores with sub-row K group scales: the MMAs of each run of D / G
+// head-dim entries (2^bpg_log2 k16 blocks) accumulate on their own, then
+// are scaled by the group's K scale of this lane's token rows grp / grp + 8
+// (ga[g] / gb[g], shared memory) and summed. kf = the score factor without
+// the K scale. Masking as tile_scores.
+template <int D, bool KCVT, class QFrag>
+__device__ __forceinline__ float4 tile_scores_groups(const QFrag& qfr, uint32_t sk,
+                                                     const uint32_t (&koff)[4], const float* ga,
+                                                     const float* gb, int bpg_log2, float kf,
+                                                     int tok0, int t0, int t1, bool page_ok,
+                                                     bool full, int grp) {
+  float S[4] = {0.f, 0.f, 0.f, 0.f}, Sg[4] = {0.f, 0.f, 0.f, 0.f};
+  const int bpg_mask = (1 << bpg_log2) - 1;
+#pragma unroll
+  for (int kc = 0; kc < D / 32; ++kc) {
+    const uint4 kw = ldsm_x4(sk + blk_off<D>(koff, kc));
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int kb = 2 * kc + half;
+      const uint32_t wa = half ? kw.z : kw.x, wb = half ? kw.w : kw.y;
+      const uint2 f = qfr(kb);
+      uint32_t a0, a1, a2, a3;
+      if constexpr (KCVT) {
+        a0 = e4m3x2_lo16_to_f16x2(wa);
+        a1 = e4m3x2_lo16_to_f16x2(wb);
+        a2 = e4m3x2_hi16_to_f16x2(wa);
+        a3 = e4m3x2_hi16_to_f16x2(wb);
+      } else {
+        a0 = e4m3x2_b02_to_f16x2(wa);
+        a1 = e4m3x2_b02_to_f16x2(wb);
+        a2 = e4m3x2_b13_to_f16x2(wa);
+        a3 = e4m3x2_b13_to_f16x2(wb);
+      }
+      mma16816(Sg, a0, a1, a2, a3, f.x, f.y);
+      if ((kb & bpg_mask) == bpg_mask) {  // the group's last k16 block
+        const int g = kb >> bpg_log2;
+        const float sa = ga[g], sb = gb[g];
+        S[0] = fmaf(Sg[0], sa, S[0]);
+        S[1] = fmaf(Sg[1], sa, S[1]);
+        S[2] = fmaf(Sg[2], sb, S[2]);
+        S[3] = fmaf(Sg[3], sb, S[3]);
+        Sg[0] = Sg[1] = Sg[2] = Sg[3] = 0.f;
+      }
+    }
+  }
+  const int ta = tok0 + grp, tb = ta + 8;
+  const bool va = full || (page_ok && ta >= t0 && ta < t1);
+  const bool vb = full || (page_ok && tb >= t0 && tb < t1);
+  return make_float4(va ? S[0] * kf : -CUDART_INF_F, va ? S[1] * kf : -CUDART_INF_F,
+                     vb ? S[2] * kf : -CUDART_INF_F, vb ? S[3] * kf : -CUDART_INF_F);
+}
+
 // Online-softmax update for new scores whose per-head maxima over this
 // lane's tokens are (tm0, tm1) and whose largest |V scale| is vabs: the
 // running maxima and the V reference scale grow, and l and O are rescaled,
@@ -694,7 +746,8 @@ __device__ __forceinline__ float warp_token_scale(const float (&x)[PER]) {
 // into the pools at (page, slot). Lane l owns head-dim bytes
 // [l D/32, (l+1) D/32). ks / vs: the page's scales; with per-token scales
 // (TOK and p.k_tok / p.v_tok) they are replaced by the new token's own,
-// which `store` also writes to the scale array.
+// which `store` also writes to the scale array (with sub-row K groups, ks is
+// the scale of this lane's group: its 32 / k_groups lanes hold one group).
 template <int D, bool TOK>
 __device__ __forceinline__ void append_new_token(const DecodeParams& p, int b, int kvh, bool store,
                                               int page, int slot, int r, uint32_t sk, uint32_t sv,
@@ -711,7 +764,19 @@ __device__ __forceinline__ void append_new_token(const DecodeParams& p, int b, i
     xv[i] = bf16_bits_to_float(vn[(int64_t)(d0 + i) * p.vn_sd]);
   }
   if constexpr (TOK) {
-    if (p.k_tok) {
+    if (p.k_tok && p.k_groups > 1) {
+      // sub-row groups: the 32 / k_groups lanes of a group agree on its
+      // maximum; ks becomes this lane's group scale
+      const int lpg = 32 / p.k_groups;
+      float m = 0.f;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) m = fmaxf(m, fabsf(xk[i]));
+      for (int o = 1; o < lpg; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      ks = m == 0.f ? 1.f : __fdiv_rn(m, 448.f);
+      if (store && (lane & (lpg - 1)) == 0)
+        p.ksw[(int64_t)page * p.ks_sp + (int64_t)slot * p.ks_st + (int64_t)kvh * p.ks_sh +
+              (int64_t)(lane / lpg) * p.ks_sg] = ks;
+    } else if (p.k_tok) {
       ks = warp_token_scale<PER>(xk);
       if (store && lane == 0)
         p.ksw[(int64_t)page * p.ks_sp + (int64_t)slot * p.ks_st + (int64_t)kvh * p.ks_sh] = ks;
@@ -1253,14 +1318,42 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     const int e = went[j];
     const int r = lane & 15;
     const int t = (tile_first + warp + C::NW * j) * kTileTokens + r;
-    if (e < 0 || t < t0 || t >= t1) return 0.f;
+    if (e < 0 || t < t0 || t >= t1 || (lane < 16 && p.k_groups > 1)) return 0.f;
     const int64_t slot = (e & 15) * kTileTokens + r;
     return lane < 16 ? __ldg(ksbase + (int64_t)(e >> 4) * p.ks_sp + slot * p.ks_st)
                      : __ldg(vsbase + (int64_t)(e >> 4) * p.vs_sp + slot * p.vs_st);
   };
   float tsc_next = 0.f;
+  // Sub-row K groups (TOK, k_groups = G > 1, G <= D / 16): the tile's
+  // 16 x G K scales, entry i = 16-token row r = i / G, group g = i % G; lane l
+  // loads entries l + 32 m (m < G / 2 <= GKN) of the next tile into gk_next and, when the tile
+  // comes up, stores them in shared memory (rows 0-7 in this warp's wks,
+  // rows 8-15 in its wvs, G floats per row; both are free with TOK).
+  const int kg = TOK ? p.k_groups : 1;
+  const int kg_log2 = 31 - __clz(kg);
+  const int kb_log2 = 31 - __clz(max(1, KB / kg));  // k16 blocks per group (log2)
+  constexpr int GKN = (D / 32 < 8) ? D / 32 : 8;
+  float gk_next[GKN];
+  auto group_scales = [&](int j, float (&o)[GKN]) {
+    const int e = went[j];
+#pragma unroll
+    for (int m = 0; m < GKN; ++m) {
+      const int i = lane + 32 * m;
+      float v = 0.f;
+      if (e >= 0 && i < 16 * kg) {
+        const int r = i >> kg_log2, g = i & (kg - 1);
+        v = __ldg(ksbase + (int64_t)(e >> 4) * p.ks_sp +
+                  (int64_t)((e & 15) * kTileTokens + r) * p.ks_st + (int64_t)g * p.ks_sg);
+      }
+      o[m] = v;
+    }
+  };
+  auto group_row = [&](int r) -> float* { return (r < 8 ? wks : wvs) + (r & 7) * kg; };
   if constexpr (TOK) {
-    if (my_tiles > 0) tsc_next = tok_scale(0);
+    if (my_tiles > 0) {
+      tsc_next = tok_scale(0);
+      if (kg > 1) group_scales(0, gk_next);
+    }
   }
 
   int stage = 0;
@@ -1349,22 +1442,50 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     if constexpr (TOK) {
       float tsc = tsc_next;
       if (j + 1 < my_tiles) tsc_next = tok_scale(j + 1);
+      if (kg > 1) {
+        float gk[GKN];
+#pragma unroll
+        for (int m = 0; m < GKN; ++m) gk[m] = gk_next[m];
+        if (j + 1 < my_tiles) group_scales(j + 1, gk_next);
+        __syncwarp();  // the previous tile's reads of the rows are done
+#pragma unroll
+        for (int m = 0; m < GKN; ++m) {
+          const int i = lane + 32 * m;
+          if (i < 16 * kg) group_row(i >> kg_log2)[i & (kg - 1)] = gk[m];
+        }
+        __syncwarp();
+      }
       if (has_new) {
         const int r = L - 1 - tok0;
         float ks = __shfl_sync(0xffffffffu, tsc, r), vs = __shfl_sync(0xffffffffu, tsc, 16 + r);
         append_new_token<D, true>(p, b, kvh, hg == 0, went[j] >> 4,
                                   (went[j] & 15) * kTileTokens + r, r, sk, sv, ks, vs);
-        if (lane == r) tsc = ks;
+        if (kg > 1) {
+          const int lpg = 32 / kg;  // lanes of one K group in the append
+          if ((lane & (lpg - 1)) == 0) group_row(r)[lane / lpg] = ks;
+        } else if (lane == r) {
+          tsc = ks;
+        }
         if (lane == 16 + r) tsc = vs;
         __syncwarp();
       }
-      const float kfa = score_base * __shfl_sync(0xffffffffu, tsc, grp);
-      const float kfb = score_base * __shfl_sync(0xffffffffu, tsc, grp + 8);
       const float vsa = __shfl_sync(0xffffffffu, tsc, 16 + grp);
       const float vsb = __shfl_sync(0xffffffffu, tsc, 24 + grp);
       const float vabs = warp_max(lane >= 16 ? fabsf(tsc) : 0.f);
-      attend_tile<D, KCVT, VCVT>(acc, qfr, sk, sv, koff, voff, kfa, kfb, vsa, vsb, vabs, tok0, t0,
-                                 t1, page_ok, full, grp, qd);
+      if (kg > 1) {
+        const float4 sc = tile_scores_groups<D, KCVT>(
+            qfr, sk, koff, group_row(grp), group_row(grp + 8), kb_log2, score_base, tok0, t0, t1,
+            page_ok, full, grp);
+        softmax_rescale<D>(acc, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), vabs);
+        uint32_t bh[2], bl[2];
+        tile_probs<D>(acc, sc, vsa, vsb, bh, bl);
+        tile_pv<D, VCVT>(acc, sv, voff, bh, bl, tok0, t0, t1, page_ok, full, qd);
+      } else {
+        const float kfa = score_base * __shfl_sync(0xffffffffu, tsc, grp);
+        const float kfb = score_base * __shfl_sync(0xffffffffu, tsc, grp + 8);
+        attend_tile<D, KCVT, VCVT>(acc, qfr, sk, sv, koff, voff, kfa, kfb, vsa, vsb, vabs, tok0,
+                                   t0, t1, page_ok, full, grp, qd);
+      }
     } else {
       const float kfac = score_base * wks[j];
       float ks = wks[j], vs = wvs[j];
@@ -2337,16 +2458,26 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
   const int64_t vso = (int64_t)page * p.vs_sp + (int64_t)slot * p.vs_st + (int64_t)h * p.vs_sh;
   // A per-token scale is the new token's own: every thread of the row
   // derives it from the row's D values, the row's first thread stores it.
-  const float ks = p.k_tok ? row_token_scale(knr, p.kn_sd, p.D) : p.ks[kso];
-  const float vs = p.v_tok ? row_token_scale(vnr, p.vn_sd, p.D) : p.vs[vso];
-  if (d == 0) {
-    if (p.k_tok) p.ksw[kso] = ks;
-    if (p.v_tok) p.vsw[vso] = vs;
+  float ks = 0.f, ks1 = 0.f;  // K scales of entries d and d + 1
+  if (p.k_tok && p.k_groups > 1) {
+    // sub-row groups of gs entries: each entry's group scale; the thread
+    // holding a group's first entry stores it
+    const int gs = p.D / p.k_groups;
+    const int g0 = d / gs, g1 = two ? (d + 1) / gs : g0;
+    ks = row_token_scale(knr + (int64_t)g0 * gs * p.kn_sd, p.kn_sd, gs);
+    ks1 = g1 == g0 ? ks : row_token_scale(knr + (int64_t)g1 * gs * p.kn_sd, p.kn_sd, gs);
+    if (d == g0 * gs) p.ksw[kso + (int64_t)g0 * p.ks_sg] = ks;
+    if (g1 != g0 && d + 1 == g1 * gs) p.ksw[kso + (int64_t)g1 * p.ks_sg] = ks1;
+  } else {
+    ks = ks1 = p.k_tok ? row_token_scale(knr, p.kn_sd, p.D) : p.ks[kso];
+    if (d == 0 && p.k_tok) p.ksw[kso] = ks;
   }
+  const float vs = p.v_tok ? row_token_scale(vnr, p.vn_sd, p.D) : p.vs[vso];
+  if (d == 0 && p.v_tok) p.vsw[vso] = vs;
   const uint16_t* kn = knr + (int64_t)d * p.kn_sd;
   const uint16_t* vn = vnr + (int64_t)d * p.vn_sd;
   const float k0 = __fdiv_rn(bf16_bits_to_float(kn[0]), ks);
-  const float k1 = two ? __fdiv_rn(bf16_bits_to_float(kn[p.kn_sd]), ks) : 0.f;
+  const float k1 = two ? __fdiv_rn(bf16_bits_to_float(kn[p.kn_sd]), ks1) : 0.f;
   const float v0 = __fdiv_rn(bf16_bits_to_float(vn[0]), vs);
   const float v1 = two ? __fdiv_rn(bf16_bits_to_float(vn[p.vn_sd]), vs) : 0.f;
   const uint16_t kc = e4m3x2_rn_sat(k0, k1);

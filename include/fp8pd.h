@@ -153,9 +153,13 @@ enum {
  *   k_scale,     float32 [Hkv] (per KV head), [num_pages, Hkv] (per page and KV
  *   v_scale      head) or [num_pages, ps, Hkv] (per stored token and KV head),
  *                any strides (0 = broadcast); k_scale(page, slot, h) ignores
- *                the missing axes. K and V may use different forms. With a
- *                per-token form the segment schedule is not used (a request
- *                for it runs the split kernel's own plan).
+ *                the missing axes. K and V may use different forms. K may
+ *                also be [num_pages, ps, Hkv, G] (the solution page's k_groups
+ *                sub-row key scales): head-dim entry d of a key uses scale
+ *                [page, slot, h, d / (D / G)]; G in {1, 2, 4, 8, 16} with
+ *                D / G >= 16, else FP8PD_ERR_UNSUPPORTED. V takes G = 1 only.
+ *                With a per-token form the segment schedule is not used (a
+ *                request for it runs the split kernel's own plan).
  *   block_table  int32 [B, max_pages]: physical page of each logical page.
  *                Entries past the attended range are never read.
  *   seq_lens     int32 [B]: number of keys visible to the query (positions 0..L-1).
@@ -201,6 +205,8 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
  * ks = k_scale(page, h). A per-token scale ([num_pages, ps, Hkv]) is the new
  * token's own, ks = max_d |k_new[b, h, d]| / 448 in IEEE float32 (NaN entries
  * skipped, 1 for an all-zero row), and is written to k_scale[page, p % ps, h].
+ * With sub-row groups ([num_pages, ps, Hkv, G], G a power of two up to 16
+ * dividing D) each run of D / G entries takes and writes its own scale.
  * Nothing else in the pools or scales is written. The new token is then visible to an attention call with
  * seq_lens[b] = p + 1 (the "Lecture 8" page's kv-cache update before the
  * decode attention).

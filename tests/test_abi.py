@@ -89,8 +89,12 @@ def _call(F, a):
     (dict(ks=torch.ones(6, 8, 2)), -3),                                      # per-token: ps
     (dict(vs=torch.ones(5, 16, 2)), -3),                                     # per-token: pages
     (dict(ks=torch.ones(6, 16, 3)), -3),                                     # per-token: Hkv
-    (dict(vs=torch.ones(6, 16, 2, 1)), -3),                                  # 4-D scale
+    (dict(vs=torch.ones(())), -3),                                           # 0-D scale
     (dict(ks=torch.ones(6, 16, 2, dtype=torch.float64)), -2),
+    (dict(ks=torch.ones(6, 16, 2, 16)), -5),                                 # D / groups < 16
+    (dict(ks=torch.ones(6, 16, 2, 3)), -5),                                  # groups not a power of 2
+    (dict(vs=torch.ones(6, 16, 2, 2)), -5),                                  # V sub-row groups
+    (dict(ks=torch.ones(6, 16, 3, 2)), -3),
     (dict(sinks=torch.zeros(7)), -3),
     (dict(table=torch.zeros(3, 3, dtype=torch.int32)), -3),
     (dict(lens=torch.zeros(2, dtype=torch.int64)), -2),
@@ -158,6 +162,9 @@ def test_append_validation(F):
     with pytest.raises(F.Fp8pdError) as e:                  # per-token scale with the wrong ps
         F.fp8_kv_append(kn, kn, kp, kp, torch.ones(4, 8, 2), ks, tbl, pos, stream=0)
     assert e.value.status == -3
+    with pytest.raises(F.Fp8pdError) as e:                  # 32 groups: more than 16
+        F.fp8_kv_append(kn, kn, kp, kp, torch.ones(4, 16, 2, 32), ks, tbl, pos, stream=0)
+    assert e.value.status == -5
 
 
 def test_options_roundtrip(F):

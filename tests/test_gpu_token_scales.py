@@ -220,3 +220,96 @@ def test_fused_same_bytes_as_append_then_attention(F, cuda_device):
     assert torch.equal(la.k_scale, lb.k_scale) and torch.equal(la.v_scale, lb.v_scale)
     assert torch.equal(la.k_pages, lb.k_pages) and torch.equal(la.v_pages, lb.v_pages)
     assert torch.equal(got, want)
+
+
+# ---------------------------------------------------------------- sub-row K groups
+
+@pytest.mark.parametrize("name,G", [("gptoss_full", 2), ("gptoss_w128", 4), ("llama", 2),
+                                    ("llama", 8), ("mixed", 16)])
+def test_key_groups_attention(F, cuda_device, name, G):
+    """K scales [num_pages, ps, Hkv, G]: each group of D / G head-dim entries
+    has its own scale per token (D / G >= 16)."""
+    case = W.make_case(name, cuda_device, B=3, seq_len=(20, 1500), scale_mode="token",
+                       k_groups=G)
+    for li in range(len(case.layers)):
+        _attention(F, case, li=li, where=f"{name} k_groups={G} layer {li}")
+
+
+def test_key_groups_decode_variants(F, cuda_device):
+    F.fp8pd_set_option(F.OPT_K_DECODE, 0)
+    F.fp8pd_set_option(F.OPT_V_DECODE, 0)
+    try:
+        case = W.make_case("llama", cuda_device, B=3, seq_len=(30, 600), scale_mode="token",
+                           k_groups=4)
+        _attention(F, case, where="k_groups=4 bit assembly")
+    finally:
+        F.fp8pd_set_option(F.OPT_K_DECODE, 1)
+        F.fp8pd_set_option(F.OPT_V_DECODE, 1)
+
+
+def test_one_key_group_equals_per_token(F, cuda_device):
+    case = W.make_case("llama", cuda_device, B=4, seq_len=(30, 700), scale_mode="token")
+    layer = case.layers[0]
+    a = gpu_attention(F, layer, case.cache_lens)
+    b = F.fp8_paged_decode_attention(layer.q, layer.k_pages, layer.v_pages,
+                                     layer.k_scale.unsqueeze(-1), layer.v_scale.unsqueeze(-1),
+                                     layer.block_table, case.cache_lens, sm_scale=layer.sm_scale)
+    torch.cuda.synchronize()
+    assert F.fp8pd_check_errors() == 0
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("D,G", [(64, 4), (128, 8), (80, 16), (96, 2)])
+def test_append_key_groups(F, cuda_device, D, G):
+    """fp8_kv_append with sub-row K groups: codes and group scales bit-exact
+    against the oracle. D = 80, G = 16 puts group starts at odd entries."""
+    g = torch.Generator(device=cuda_device).manual_seed(60 + D)
+    P, ps, Hkv, B = 10, 16, 2, 4
+    kp = torch.randint(0, 256, (P, ps, Hkv, D), dtype=torch.uint8, device=cuda_device, generator=g)
+    vp = kp.clone()
+    ks = torch.rand(P, ps, Hkv, G, device=cuda_device, generator=g) + 0.5
+    vs = torch.rand(P, ps, Hkv, device=cuda_device, generator=g) + 0.5
+    mag = torch.logspace(-3, 2, G, device=cuda_device).repeat_interleave(D // G)
+    kn = (torch.randn(B, Hkv, D, device=cuda_device, generator=g) * mag).to(torch.bfloat16)
+    vn = torch.randn(B, Hkv, D, device=cuda_device, generator=g).to(torch.bfloat16)
+    kn[1, 0, :D // G] = 0.0                      # one all-zero group
+    table = torch.tensor(np.random.default_rng(D).permutation(P)[:B * 2].reshape(B, 2),
+                         dtype=torch.int32, device=cuda_device)
+    pos = torch.tensor([0, 7, 16, 31], dtype=torch.int32, device=cuda_device)
+    want = [np_(t).copy() for t in (kp, vp, ks, vs)]
+    F.fp8_kv_append(kn, vn, kp, vp, ks, vs, table, pos)
+    torch.cuda.synchronize()
+    assert F.fp8pd_check_errors() == 0
+    O.kv_append(np_(kn), np_(vn), *want, np_(table), np_(pos))
+    for got, w, name in zip((kp, vp, ks, vs), want, ("K pool", "V pool", "K scale", "V scale")):
+        assert np.array_equal(np_(got), w), name
+
+
+@pytest.mark.parametrize("name,G", [("llama", 4), ("gptoss_w128", 4), ("mixed", 16)])
+def test_fused_key_groups(F, cuda_device, name, G):
+    case = W.make_case(name, cuda_device, B=3, seq_len=(40, 1200), append=True,
+                       scale_mode="token", k_groups=G)
+    for li in range(len(case.layers)):
+        _fused(F, case, li=li, where=f"fused {name} k_groups={G} layer {li}")
+
+
+def test_fused_key_groups_same_bytes_as_two_calls(F, cuda_device):
+    kw = dict(B=5, seq_len=(40, 900), scale_mode="token", k_groups=8)
+    a = W.make_case("llama", cuda_device, **kw)
+    b = W.make_case("llama", cuda_device, **kw)
+    la, lb = a.layers[0], b.layers[0]
+    # page-edge positions, none past the slot each sequence's table reserves
+    pos = torch.minimum(torch.tensor([0, 15, 16, 400, 17], dtype=torch.int32, device=cuda_device),
+                        a.positions)
+    got = F.fp8_paged_decode_append_attention(
+        la.q, la.k_new, la.v_new, la.k_pages, la.v_pages, la.k_scale, la.v_scale,
+        la.block_table, pos, sm_scale=la.sm_scale)
+    F.fp8_kv_append(lb.k_new, lb.v_new, lb.k_pages, lb.v_pages, lb.k_scale, lb.v_scale,
+                    lb.block_table, pos)
+    want = F.fp8_paged_decode_attention(lb.q, lb.k_pages, lb.v_pages, lb.k_scale, lb.v_scale,
+                                        lb.block_table, pos + 1, sm_scale=lb.sm_scale)
+    torch.cuda.synchronize()
+    assert F.fp8pd_check_errors() == 0
+    assert torch.equal(la.k_scale, lb.k_scale) and torch.equal(la.v_scale, lb.v_scale)
+    assert torch.equal(la.k_pages, lb.k_pages) and torch.equal(la.v_pages, lb.v_pages)
+    assert torch.equal(got, want)

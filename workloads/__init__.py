@@ -45,6 +45,7 @@ class Spec:
     layers: tuple                       # tuple[LayerSpec, ...]; >1 = layers sharing one pool
     seq_len: int | tuple = 256          # int, or (lo, hi) inclusive uniform range per sequence
     scale_mode: str = "head"            # "head": [Hkv]; "page": [num_pages, Hkv]; "token": [num_pages, ps, Hkv]
+    k_groups: int = 1                   # "token" only: K scales [num_pages, ps, Hkv, k_groups] when > 1
     dist: str = "normal"                # "normal": N(0,1); "normal2_outliers": N(0,2), 1% x20
     sinks: bool = False
     append: bool = False                # one new token per sequence at position seq_len
@@ -223,8 +224,11 @@ def make_case(name_or_spec, device="cpu", chunk_pages: int = 1024, **overrides) 
         views, scales, news = [], [], []
         for which, pool in ((0, k_pool), (1, v_pool)):
             # pass 1: scales from the values (including the token to append)
+            G = spec.k_groups if (spec.scale_mode == "token" and which == 0) else 1
             if spec.scale_mode == "head":
                 amax = torch.zeros(L.Hkv, device=device)
+            elif spec.scale_mode == "token" and G > 1:
+                amax = torch.zeros(total_pages, spec.ps, L.Hkv, G, device=device)
             elif spec.scale_mode == "token":
                 amax = torch.zeros(total_pages, spec.ps, L.Hkv, device=device)
             else:
@@ -232,6 +236,9 @@ def make_case(name_or_spec, device="cpu", chunk_pages: int = 1024, **overrides) 
             for p0 in range(0, total_pages, chunk_pages):
                 p1 = min(total_pages, p0 + chunk_pages)
                 x = page_values_bf16_new(page_values(p0, p1, which), p0, p1)
+                if spec.scale_mode == "token" and G > 1:          # [pages, ps, Hkv, G]
+                    amax[p0:p1] = x.view(p1 - p0, spec.ps, L.Hkv, G, L.D // G).abs().amax(dim=4)
+                    continue
                 if spec.scale_mode == "token":
                     amax[p0:p1] = x.abs().amax(dim=3)             # [pages, ps, Hkv]
                     continue
@@ -250,6 +257,8 @@ def make_case(name_or_spec, device="cpu", chunk_pages: int = 1024, **overrides) 
                 x = page_values_bf16_new(page_values(p0, p1, which), p0, p1)
                 if spec.scale_mode == "head":
                     sc = scale.view(1, 1, L.Hkv, 1)
+                elif spec.scale_mode == "token" and G > 1:
+                    sc = scale[p0:p1].repeat_interleave(L.D // G, dim=3)
                 elif spec.scale_mode == "token":
                     sc = scale[p0:p1].view(-1, spec.ps, L.Hkv, 1)
                 else:
@@ -278,7 +287,7 @@ def algorithmic_bytes(case: Case, layer: int = 0) -> int:
     """Bytes a decode step must read for one layer: the attended K and V bytes
     (window-limited, once per KV head), q, and the block-table entries of the
     attended pages; with per-token scales also the attended tokens' K and V
-    scales (4 bytes each per KV head). Per-head and per-page scales, the
+    scales (4 bytes each per KV head and sub-row group). Per-head and per-page scales, the
     output and split partials are not counted."""
     L = case.layers[layer]
     lens = case.attend_lens.cpu().numpy().astype(np.int64)
@@ -292,8 +301,9 @@ def algorithmic_bytes(case: Case, layer: int = 0) -> int:
         if n > 0:
             tbl += 4 * ((Lb - 1) // ps - lo // ps + 1)
     q = L.q.numel() * 2
-    # per-token scales: 4 bytes per attended token and KV head, for K and for V
-    tok_scales = sum(kv // L.spec.D * 2 for sc in (L.k_scale, L.v_scale) if sc.dim() == 3)
+    # per-token scales: 4 bytes per attended token, KV head and group, for K and for V
+    tok_scales = sum(kv // L.spec.D * 2 * (sc.shape[3] if sc.dim() == 4 else 1)
+                     for sc in (L.k_scale, L.v_scale) if sc.dim() >= 3)
     return int(kv + q + tbl + tok_scales)
 
 
