@@ -27,7 +27,7 @@ import torch
 __all__ = [
     "fp8_paged_decode_attention", "fp8_paged_decode_attention_noalloc", "fp8_kv_append",
     "fp8_paged_decode_append_attention",
-    "fp8pd_plan", "fp8pd_reserve_workspace",
+    "fp8pd_plan", "fp8pd_reserve_workspace", "fp8pd_e4m3_encode",
     "fp8pd_check_errors", "fp8pd_set_option", "fp8pd_get_option", "fp8pd_last_run_info",
     "fp8pd_timing_enable", "fp8pd_timing_collect", "Fp8pdError", "lib", "LIB_PATH",
     "FLAG_PAGE_OOB", "FLAG_SEQLEN_OOB", "FLAG_POS_OOB", "FLAG_INTERNAL", "OPT_NUM_SPLITS",
@@ -82,6 +82,7 @@ def _load() -> ctypes.CDLL:
     lib.fp8_paged_decode_append_attention.argtypes = [T, T, T, T, T, T, T, T, T, i32, T, f32, T, vp]
     lib.fp8pd_plan.argtypes = [T, T, T, i32, P(PlanInfo)]
     lib.fp8pd_reserve_workspace.argtypes = [ctypes.c_uint64]
+    lib.fp8pd_e4m3_encode.argtypes = [T, T, vp]
     lib.fp8pd_check_errors.argtypes = [vp, P(ctypes.c_uint32)]
     lib.fp8pd_set_option.argtypes = [i32, ctypes.c_int64]
     lib.fp8pd_get_option.argtypes = [i32]
@@ -242,6 +243,18 @@ def fp8_paged_decode_append_attention(q, k_new, v_new, k_pages, v_pages, k_scale
                                                _ref(ds_sinks), float(sm_scale), _ref(ds_out),
                                                _stream(stream, q))
     _check(st, "fp8_paged_decode_append_attention")
+    return out
+
+
+def fp8pd_e4m3_encode(x, out=None, stream=None) -> torch.Tensor:
+    """E4M3 codes (uint8) of a 1-D float32 tensor with the append's rounding:
+    nearest even, saturating to +-448, NaN to the NaN code (see
+    include/fp8pd.h)."""
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _same_device(x, out)
+    dx, do = describe(x), describe(out)
+    _check(lib.fp8pd_e4m3_encode(_ref(dx), _ref(do), _stream(stream, x)), "fp8pd_e4m3_encode")
     return out
 
 

@@ -864,6 +864,22 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
   return FP8PD_OK;
 }
 
+int fp8pd_e4m3_encode(const fp8pd_tensor* x, fp8pd_tensor* codes, fp8pd_stream_t stream) {
+  int r;
+  if ((r = check(x, FP8PD_DTYPE_F32, 1))) return r;
+  if ((r = check(codes, FP8PD_DTYPE_U8, 1))) return r;
+  if (codes->shape[0] != x->shape[0]) return FP8PD_ERR_SHAPE;
+  if (x->stride[0] < 0 || codes->stride[0] < 0) return FP8PD_ERR_SHAPE;
+  const int64_t n = x->shape[0];
+  if (n == 0) return FP8PD_OK;
+  const cudaError_t e = fp8pd::launch_encode(
+      static_cast<const float*>(x->data), x->stride[0], static_cast<uint8_t*>(codes->data),
+      codes->stride[0], n, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e);
+  ++g_launches;
+  return FP8PD_OK;
+}
+
 int fp8pd_reserve_workspace(uint64_t bytes) {
   void *ctr = nullptr, *part = nullptr;
   return get_workspace(0, static_cast<size_t>(bytes), nullptr, &ctr, &part);

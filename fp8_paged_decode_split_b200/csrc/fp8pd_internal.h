@@ -96,6 +96,9 @@ struct AppendParams {
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                           bool k_cvt, bool v_cvt, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+// E4M3 codes (the append's rounding) of n float32 values; strides in elements.
+cudaError_t launch_encode(const float* x, int64_t xs, uint8_t* c, int64_t cs, int64_t n,
+                          cudaStream_t s);
 
 // Segment schedule: the tiles of all sequences of one KV head x head group
 // as one list, cut into nbx equal block ranges; grid (HX, nbx) of blocks of

@@ -2664,6 +2664,27 @@ int decode_smem_bytes(int D) {
   }
 }
 
+// E4M3 codes of n float32 values with the append's rounding
+// (cvt.rn.satfinite: nearest, ties to even, +-448 for larger magnitudes and
+// infinities, NaN to the NaN code with its sign); strides in elements.
+__global__ void __launch_bounds__(256)
+    encode_kernel(const float* x, int64_t xs, uint8_t* c, int64_t cs, int64_t n) {
+  const int64_t step = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += step)
+    c[i * cs] = static_cast<uint8_t>(e4m3x2_rn_sat(x[i * xs], 0.f) & 0xFFu);
+}
+
+cudaError_t launch_encode(const float* x, int64_t xs, uint8_t* c, int64_t cs, int64_t n,
+                          cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t want = (n + threads - 1) / threads;
+  const int64_t cap = 148 * 32;  // a grid-stride loop past 32 blocks per SM
+  encode_kernel<<<static_cast<unsigned>(want < cap ? want : cap), threads, 0, s>>>(x, xs, c, cs,
+                                                                                   n);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
   const int64_t total = (int64_t)p.B * p.Hkv * ((p.D + 1) / 2);
   if (total == 0) return cudaSuccess;

@@ -303,6 +303,19 @@ typedef struct fp8pd_plan_info {
 int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages,
                const fp8pd_tensor* block_table, int32_t window, fp8pd_plan_info* info);
 
+/*
+ * fp8pd_e4m3_encode -- E4M3 codes of float32 values, with the rounding the
+ * append applies to its quotients: round to nearest, ties to an even
+ * mantissa, magnitudes above 448 and infinities saturated to +-448, NaN to
+ * the NaN code with its sign, -0 to 0x80 (the E4M3 RNE with saturation named
+ * by the solution page's "Supported scope" for the cache's quantizer).
+ *   x      float32 [n] in device memory, any stride >= 0.
+ *   codes  uint8 [n] in device memory, any stride >= 0 (written).
+ * One kernel launch; n = 0 launches nothing (the data pointers must still be
+ * non-NULL, as for every descriptor).
+ */
+int fp8pd_e4m3_encode(const fp8pd_tensor* x, fp8pd_tensor* codes, fp8pd_stream_t stream);
+
 /* Grows the current device's split workspace to at least `bytes` (never
  * shrinks). Must not be called while a stream of the device is capturing. */
 int fp8pd_reserve_workspace(uint64_t bytes);

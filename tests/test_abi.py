@@ -167,6 +167,20 @@ def test_append_validation(F):
     assert e.value.status == -5
 
 
+def test_encode_validation(F):
+    x = torch.zeros(8)
+    c = torch.zeros(8, dtype=torch.uint8)
+    for bad, status in ((dict(x=x.double()), -2), (dict(c=c.to(torch.int32)), -2),
+                        (dict(c=torch.zeros(7, dtype=torch.uint8)), -3),
+                        (dict(x=torch.zeros(2, 4)), -3)):
+        a = dict(x=x, c=c)
+        a.update(bad)
+        with pytest.raises(F.Fp8pdError) as e:
+            F.fp8pd_e4m3_encode(a["x"], out=a["c"], stream=0)
+        assert e.value.status == status
+    assert F.lib.fp8pd_e4m3_encode(None, None, None) == -1
+
+
 def test_options_roundtrip(F):
     F.fp8pd_set_option(F.OPT_NUM_SPLITS, 7)
     assert F.fp8pd_get_option(F.OPT_NUM_SPLITS) == 7
