@@ -25,6 +25,13 @@
  *                               cache is updated inside the attention kernel,
  *                               before the query reads it).
  *
+ * K and V scales come per KV head, per (page, KV head) or per (stored token,
+ * KV head), K also in sub-row groups (the solution page's "Supported scope":
+ * quantize_kv_fp8's per-token-per-head scales and k_groups). Helpers: an
+ * allocation-free attention entry point, planning, workspace, options, the
+ * device error word, timing, and fp8pd_e4m3_encode (the append's rounding on
+ * a float32 array).
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  * - Every buffer is caller-owned device memory described by fp8pd_tensor
@@ -86,7 +93,8 @@ typedef struct fp8pd_tensor {
  * indexed by the page id found in the block table) -- both read only -- or
  * [num_pages, ps, Hkv] (one per stored token and KV head, the cache-write
  * quantizer's per-token-per-head form named in the solution page's
- * "Supported scope"), which the append writes. */
+ * "Supported scope"), which the append writes; K also
+ * [num_pages, ps, Hkv, G] (sub-row groups, written per group). */
 typedef struct fp8pd_scales {
   fp8pd_tensor k_scale;
   fp8pd_tensor v_scale;
