@@ -313,3 +313,30 @@ def test_fused_key_groups_same_bytes_as_two_calls(F, cuda_device):
     assert torch.equal(la.k_scale, lb.k_scale) and torch.equal(la.v_scale, lb.v_scale)
     assert torch.equal(la.k_pages, lb.k_pages) and torch.equal(la.v_pages, lb.v_pages)
     assert torch.equal(got, want)
+
+
+def test_page1_worked_example_per_token(F, cuda_device):
+    """The solution page's worked example as it is written there: 16-token
+    blocks quantized per token and KV head into a permuted block table
+    (2, 0, 1), GQA 2:1, 40 live tokens, one decode query, D ** -0.5."""
+    BT, HKV, HQ, D, T = 16, 2, 4, 64, 40
+    table = np.array([[2, 0, 1]], np.int32)
+    g = torch.Generator().manual_seed(1)
+    kt = torch.randn(3 * BT, HKV, D, generator=g).numpy().astype(np.float32)
+    vt = torch.randn(3 * BT, HKV, D, generator=g).numpy().astype(np.float32)
+    kp = np.zeros((3, BT, HKV, D), np.uint8)
+    vp = np.zeros_like(kp)
+    ks = np.zeros((3, BT, HKV), np.float32)
+    vs = np.zeros_like(ks)
+    for i in range(3):
+        r = table[0, i]
+        kp[r], ks[r] = O.quantize_per_token(kt[i * BT:(i + 1) * BT])
+        vp[r], vs[r] = O.quantize_per_token(vt[i * BT:(i + 1) * BT])
+    q = torch.randn(1, HQ, D, generator=g).to(torch.bfloat16)
+    dev = lambda a: torch.from_numpy(a).to(cuda_device)  # noqa: E731
+    out = F.fp8_paged_decode_attention(q.to(cuda_device), dev(kp), dev(vp), dev(ks), dev(vs),
+                                       dev(table), dev(np.array([T], np.int32)))
+    torch.cuda.synchronize()
+    assert F.fp8pd_check_errors() == 0
+    want = O.paged_decode_attention(q.double().numpy(), kp, vp, ks, vs, table, np.array([T]))
+    assert_attention_close(np_(out), want, "worked example, per-token scales")

@@ -403,6 +403,51 @@ def test_page1_worked_example_shape():
     assert float(spec["tolerance"][0]) == 1e-2
 
 
+def test_page1_worked_example_per_token_scales():
+    """The worked example as the page writes it: each 16-token block goes
+    through the per-token-per-head quantizer (one scale per token and KV
+    head) into its permuted page; the paged oracle then reproduces plain
+    softmax attention over the dequantized values."""
+    spec = {}
+    with open(os.path.join(GOLDEN, "page1_worked_example.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                k, *v = line.split()
+                spec[k] = v
+    BT, HKV, HQ, D, T = (int(spec[k][0]) for k in
+                         ("block_tokens", "n_kv_heads", "n_q_heads", "head_dim", "live_tokens"))
+    table = np.array([[int(x) for x in spec["block_table"]]], np.int32)
+    n_blk = (T + BT - 1) // BT
+    g = torch.Generator().manual_seed(1)
+    kt = torch.randn(n_blk * BT, HKV, D, generator=g).numpy().astype(np.float32)
+    vt = torch.randn(n_blk * BT, HKV, D, generator=g).numpy().astype(np.float32)
+    kp = np.zeros((n_blk, BT, HKV, D), np.uint8)
+    vp = np.zeros_like(kp)
+    ks = np.zeros((n_blk, BT, HKV), np.float32)
+    vs = np.zeros_like(ks)
+    kd, vd = [], []
+    for i in range(n_blk):
+        r = table[0, i]
+        kp[r], ks[r] = O.quantize_per_token(kt[i * BT:(i + 1) * BT])
+        vp[r], vs[r] = O.quantize_per_token(vt[i * BT:(i + 1) * BT])
+        # dequantized through the library float8 type, not the oracle's table
+        f8 = lambda c: torch.from_numpy(c).view(torch.float8_e4m3fn).double().numpy()  # noqa: E731
+        kd.append(f8(kp[r]) * ks[r][..., None])
+        vd.append(f8(vp[r]) * vs[r][..., None])
+    kd = np.concatenate(kd)[:T].transpose(1, 0, 2)
+    vd = np.concatenate(vd)[:T].transpose(1, 0, 2)
+    q = torch.randn(1, HQ, D, generator=g).to(torch.bfloat16).double().numpy()
+    out = O.paged_decode_attention(q, kp, vp, ks, vs, table, np.array([T]), window=0)
+    qq = q[0].reshape(HKV, HQ // HKV, D)
+    w = torch.softmax(torch.einsum("hgd,htd->hgt", torch.from_numpy(qq), torch.from_numpy(kd)) * D ** -0.5,
+                      dim=-1)
+    want = torch.einsum("hgt,htd->hgd", w, torch.from_numpy(vd)).reshape(1, HQ, D).numpy()
+    assert np.allclose(out, want, rtol=1e-12, atol=1e-12)
+    # per-token scales keep every value within half an E4M3 step of its row
+    ks_rows = np.concatenate([ks[table[0, i]] for i in range(n_blk)])[:T][..., None]
+    assert np.all(np.abs(kd.transpose(1, 0, 2) - kt[:T]) <= np.abs(kt[:T]) / 16 + 2.0 ** -10 * ks_rows)
+
+
 # ---------------------------------------------------------------- append
 
 def test_append_writes_only_the_new_slot():
