@@ -4,7 +4,8 @@
 // "Why it happens" and "Expected result"): flash-decode over a paged E4M3
 // KV cache with a grid over (sequence, KV head, split), E4M3 decoded in
 // registers (exactly, by the hardware cvt or by bit assembly), scales read
-// at their natural shape, the query heads of one KV head packed so each K/V
+// at their natural shape (per KV head, per page, per stored token, K also in
+// sub-row groups: "Supported scope"), the query heads of one KV head packed so each K/V
 // byte is read once, online softmax with a sliding window and sink logits,
 // and a log-sum-exp combine of the splits. With a fused append (the
 // "Lecture 8 -- Inference Path" page, "In-kernel KV cache update") the block
