@@ -523,14 +523,14 @@ def cpu_baseline(case: W.Case, budget_s: float = 10.0) -> dict:
 def _scale_override(args) -> dict:
     """``--scales token``: the workload with one scale per stored token and KV
     head instead of its own scale form."""
-    if args.scales != "token":
+    if getattr(args, "scales", "workload") != "token":
         return {}
-    return {"scale_mode": "token", "k_groups": args.k_groups}
+    return {"scale_mode": "token", "k_groups": getattr(args, "k_groups", 1)}
 
 
 def _workload_text(args) -> str:
     text = WORKLOAD_TEXT.get(args.config, args.config)
-    if args.scales != "token":
+    if getattr(args, "scales", "workload") != "token":
         return text
     groups = f", K in {args.k_groups} sub-row groups" if args.k_groups > 1 else ""
     return text + f" (scales replaced: per (token, KV head){groups})"
