@@ -46,3 +46,26 @@ def assert_attention_close(got, want, where: str = "", mask=None) -> float:
     worst = float(err.max()) if err.size else 0.0
     assert worst <= ATOL_REL, f"{where}: max scaled error {worst:.3e} > {ATOL_REL}"
     return worst
+
+
+def footer_pool(num_pages: int, ps: int, hkv: int, d: int, device="cpu"):
+    """One pool whose pages hold the E4M3 codes of ps tokens x hkv heads x d,
+    then one float32 scale per (token, head) as a page footer: the packed
+    pages of the solution page's pack_kv_block rows and of DeepGEMM's
+    64 x (64 + 4) = 4352-byte index pages. Returns (pool bytes, codes view
+    [num_pages, ps, hkv, d], scales view [num_pages, ps, hkv]); the views
+    alias the pool."""
+    page = ps * hkv * d + 4 * ps * hkv
+    pool = torch.zeros(num_pages * page, dtype=torch.uint8, device=device)
+    return (pool, *footer_views(pool, num_pages, ps, hkv, d))
+
+
+def footer_views(pool: torch.Tensor, num_pages: int, ps: int, hkv: int, d: int):
+    """(codes, scales) views of a footer pool made by :func:`footer_pool`."""
+    code_bytes = ps * hkv * d
+    page = code_bytes + 4 * ps * hkv
+    assert page % 16 == 0 and code_bytes % 4 == 0 and pool.numel() == num_pages * page
+    codes = torch.as_strided(pool, (num_pages, ps, hkv, d), (page, hkv * d, d, 1))
+    scales = torch.as_strided(pool.view(torch.float32), (num_pages, ps, hkv), (page // 4, hkv, 1),
+                              code_bytes // 4)
+    return codes, scales

@@ -9,7 +9,8 @@ import torch
 
 import oracle as O
 import workloads as W
-from tests._common import assert_attention_close, gpu_attention, np_, oracle_attention
+from tests._common import (assert_attention_close, footer_pool, footer_views, gpu_attention, np_,
+                           oracle_attention)
 
 pytestmark = pytest.mark.gpu
 
@@ -340,3 +341,78 @@ def test_page1_worked_example_per_token(F, cuda_device):
     assert F.fp8pd_check_errors() == 0
     want = O.paged_decode_attention(q.double().numpy(), kp, vp, ks, vs, table, np.array([T]))
     assert_attention_close(np_(out), want, "worked example, per-token scales")
+
+
+# ---------------------------------------------------------------- scales in a page footer
+
+def _footer_case(B, Hq, Hkv, D, ps, lens, seed, append):
+    """K and V pools whose pages carry their tokens' per-token scales as a
+    footer (built on the host with the oracle's per-token quantizer), a
+    permuted block table, q and the new token."""
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(lens)
+    npg = (lens + (1 if append else 0) + ps - 1) // ps
+    P = int(npg.sum()) + 2
+    perm = rng.permutation(P)
+    table = np.full((B, int(npg.max())), -1, np.int32)
+    off = 0
+    for b in range(B):
+        table[b, :npg[b]] = perm[off:off + npg[b]]
+        off += npg[b]
+    g = torch.Generator().manual_seed(seed)
+    pools = []
+    for _ in range(2):
+        pool, codes, scales = footer_pool(P, ps, Hkv, D)
+        x = torch.randn(P, ps, Hkv, D, generator=g) * (0.1 + 4 * torch.rand(P, ps, Hkv, 1, generator=g))
+        c, s = O.quantize_per_token(x.numpy())
+        codes.copy_(torch.from_numpy(c))
+        scales.copy_(torch.from_numpy(s))
+        pools.append(pool)
+    q = torch.randn(B, Hq, D, generator=g).to(torch.bfloat16)
+    kn = torch.randn(B, Hkv, D, generator=g).to(torch.bfloat16)
+    vn = torch.randn(B, Hkv, D, generator=g).to(torch.bfloat16)
+    return dict(pools=pools, P=P, table=table, lens=lens, q=q, kn=kn, vn=vn)
+
+
+@pytest.mark.parametrize("shape", [(3, 16, 1, 64, 64), (3, 8, 2, 64, 16), (2, 16, 2, 128, 32)],
+                         ids=["4352-byte-pages", "p1-rows-16x2x64", "ps32-D128"])
+def test_scales_in_page_footer(F, cuda_device, shape):
+    """Per-token scales stored after the codes of each page (DeepGEMM's
+    64 x (64 + 4) = 4352-byte pages; the solution page's packed 16-token
+    rows): the scale tensors are float32 views into the pool itself."""
+    B, Hq, Hkv, D, ps = shape
+    c = _footer_case(B, Hq, Hkv, D, ps, [5, 700, 1500][:B], 70 + D + ps, append=False)
+    dev_pools = [p.to(cuda_device) for p in c["pools"]]
+    (kc, ks), (vc, vs) = (footer_views(p, c["P"], ps, Hkv, D) for p in dev_pools)
+    out = F.fp8_paged_decode_attention(c["q"].to(cuda_device), kc, vc, ks, vs,
+                                       torch.from_numpy(c["table"]).to(cuda_device),
+                                       torch.from_numpy(c["lens"].astype(np.int32)).to(cuda_device))
+    torch.cuda.synchronize()
+    assert F.fp8pd_check_errors() == 0
+    (hkc, hks), (hvc, hvs) = (footer_views(p, c["P"], ps, Hkv, D) for p in c["pools"])
+    want = O.paged_decode_attention(c["q"].double().numpy(), hkc.numpy(), hvc.numpy(), hks.numpy(),
+                                    hvs.numpy(), c["table"], c["lens"])
+    assert_attention_close(np_(out), want, f"footer {shape}")
+
+
+def test_fused_append_into_page_footer(F, cuda_device):
+    """The fused call writes the new token's codes and its own scale into the
+    page and the page's footer: the whole pool, bytes and all, as the
+    oracle's append leaves it."""
+    B, Hq, Hkv, D, ps = 3, 16, 1, 64, 64
+    c = _footer_case(B, Hq, Hkv, D, ps, [63, 64, 900], 90, append=True)
+    dev_pools = [p.to(cuda_device) for p in c["pools"]]
+    (kc, ks), (vc, vs) = (footer_views(p, c["P"], ps, Hkv, D) for p in dev_pools)
+    pos = c["lens"].astype(np.int32)
+    out = F.fp8_paged_decode_append_attention(
+        c["q"].to(cuda_device), c["kn"].to(cuda_device), c["vn"].to(cuda_device), kc, vc, ks, vs,
+        torch.from_numpy(c["table"]).to(cuda_device), torch.from_numpy(pos).to(cuda_device))
+    torch.cuda.synchronize()
+    assert F.fp8pd_check_errors() == 0
+    (hkc, hks), (hvc, hvs) = (footer_views(p, c["P"], ps, Hkv, D) for p in c["pools"])
+    views = [t.numpy() for t in (hkc, hvc, hks, hvs)]      # numpy views: the append writes the pools
+    O.kv_append(np_(c["kn"]), np_(c["vn"]), *views, c["table"], pos)
+    for got, want in zip(dev_pools, c["pools"]):
+        assert torch.equal(got.cpu(), want)
+    want = O.paged_decode_attention(c["q"].double().numpy(), *views, c["table"], pos + 1)
+    assert_attention_close(np_(out), want, "fused footer")
