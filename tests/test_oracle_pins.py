@@ -722,3 +722,133 @@ def test_append_grouped_key_scales():
         quot = kn[b] / lib_s.repeat_interleave(D // G, dim=-1)
         assert np.array_equal(kp[p, s], quot.to(torch.float8_e4m3fn).view(torch.uint8).numpy())
     assert np.array_equal(kp[~touched], k0[~touched]) and np.array_equal(ks[~touched], ks0[~touched])
+
+
+# ------------------------------------------------------ window boundary pins
+# The window is defined in words on the pages: the solution page's "Expected
+# result" keeps "the last W keys", and the gpt-oss workload keeps the keys at
+# positions greater than cur_pos - W, cur_pos = L - 1 being the query's own
+# position. The pins below derive the attended set from those words with a
+# per-position predicate (never from the oracle's lower bound) and read the
+# set the oracle actually used off its output.
+
+def _marker_case(L: int, ps: int = 16, Hq: int = 2, Hkv: int = 1, seed: int = 31):
+    """One sequence of L keys whose value at logical position t is the unit
+    vector e_t (code 0x38 = 1.0 at dim t, scale 1) and whose keys are
+    random: with q = 0 every attended key gets the same weight, so the
+    output is 1/n on exactly the attended positions and 0 elsewhere."""
+    rng = np.random.default_rng(seed)
+    D = L
+    npg = (L + ps - 1) // ps
+    perm = rng.permutation(npg + 2)
+    table = perm[:npg].astype(np.int32)[None]
+    k = rng.integers(0, 0x70, size=(npg + 2, ps, Hkv, D)).astype(np.uint8)
+    v = np.zeros((npg + 2, ps, Hkv, D), np.uint8)
+    for t in range(L):
+        v[table[0, t // ps], t % ps, :, t] = 0x38
+    ones = np.ones(Hkv, np.float32)
+    return dict(q=np.zeros((1, Hq, D)), k=k, v=v, ks=ones, vs=ones, table=table,
+                lens=np.array([L]))
+
+
+def _last_w_keys(L: int, W: int) -> list:
+    """Positions t in [0, L) with t > cur_pos - W, cur_pos = L - 1; every key
+    when W = 0 (no window)."""
+    cur = L - 1
+    return [t for t in range(L) if W == 0 or t > cur - W]
+
+
+@pytest.mark.parametrize("L", [1, 2, 17, 40])
+def test_window_keeps_exactly_the_last_w_keys(L):
+    c = _marker_case(L)
+    for W in sorted({0, 1, 2, 3, L - 1, L, L + 1, 2 * L + 5}):
+        got = _run(c, window=W)[0]
+        want_set = _last_w_keys(L, W)
+        assert len(want_set) == (min(L, W) if W > 0 else L)
+        support = [t for t in range(L) if got[0, t] != 0.0]
+        assert support == want_set, (L, W, support)
+        assert np.allclose(got[:, want_set], 1.0 / len(want_set), rtol=0, atol=1e-15)
+
+
+def test_window_one_is_the_current_key_alone():
+    """W = 1: only the query's own position is attended, so the output is
+    that key's value exactly; with a sink s (no value) the weight of the one
+    key is e^score / (e^score + e^s)."""
+    rng = np.random.default_rng(41)
+    c = _dense_case(rng, B=2, scale_mode="page", L=(37, 50))
+    ps = c["k"].shape[1]
+    G = 4
+    got = _run(c, window=1, sm_scale=0.3)
+    sinks = np.linspace(-1.5, 2.0, 8).astype(np.float32)
+    got_s = _run(c, window=1, sinks=sinks, sm_scale=0.3)
+    for b in range(2):
+        t = int(c["lens"][b]) - 1
+        p = int(c["table"][b][t // ps])
+        for hq in range(8):
+            h = hq // G
+            kv = O.e4m3_decode(c["k"][p, t % ps, h]) * float(c["ks"][p, h])
+            vv = O.e4m3_decode(c["v"][p, t % ps, h]) * float(c["vs"][p, h])
+            assert np.array_equal(got[b, hq], vv)
+            s = float(np.float32(0.3)) * float(kv @ c["q"][b, hq])
+            w = math.exp(s) / (math.exp(s) + math.exp(float(sinks[hq])))
+            assert np.allclose(got_s[b, hq], w * vv, rtol=1e-13, atol=1e-16)
+
+
+def test_window_two_is_the_two_key_softmax():
+    """W = 2: the keys at positions L-2 and L-1, a two-term softmax written
+    out by hand."""
+    rng = np.random.default_rng(42)
+    c = _dense_case(rng, B=2, scale_mode="token", L=(33, 16))
+    ps = c["k"].shape[1]
+    G = 4
+    sm = float(np.float32(0.25))
+    got = _run(c, window=2, sm_scale=0.25)
+    for b in range(2):
+        L = int(c["lens"][b])
+        for hq in range(8):
+            h = hq // G
+            s, vals = [], []
+            for t in (L - 2, L - 1):
+                p = int(c["table"][b][t // ps])
+                kv = O.e4m3_decode(c["k"][p, t % ps, h]) * float(c["ks"][p, t % ps, h])
+                vals.append(O.e4m3_decode(c["v"][p, t % ps, h]) * float(c["vs"][p, t % ps, h]))
+                s.append(sm * float(kv @ c["q"][b, hq]))
+            e0, e1 = math.exp(s[0] - max(s)), math.exp(s[1] - max(s))
+            want = (e0 * vals[0] + e1 * vals[1]) / (e0 + e1)
+            assert np.allclose(got[b, hq], want, rtol=1e-13, atol=1e-16)
+
+
+def test_window_of_all_but_one_drops_key_zero():
+    """W = L - 1 equals full attention over the sequence with its first key
+    removed: the same keys re-stored, one position earlier, in a fresh pool
+    (key 0 is left out by slicing the data, not by a window)."""
+    rng = np.random.default_rng(43)
+    ps, Hkv, D, L = 16, 2, 16, 45
+    K = rng.integers(0, 0x70, size=(L, Hkv, D)).astype(np.uint8) | \
+        (rng.integers(0, 2, size=(L, Hkv, D)).astype(np.uint8) << 7)
+    V = rng.integers(0, 0x70, size=(L, Hkv, D)).astype(np.uint8)
+    ks = np.array([0.01, 0.02], np.float32)
+    vs = np.array([0.03, 0.005], np.float32)
+    q = torch.randn(1, 8, D, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    q = q.double().numpy()
+
+    def paged(keys, vals):
+        n = keys.shape[0]
+        npg = (n + ps - 1) // ps
+        perm = rng.permutation(npg)
+        kp = np.zeros((npg, ps, Hkv, D), np.uint8)
+        vp = np.zeros((npg, ps, Hkv, D), np.uint8)
+        for t in range(n):
+            kp[perm[t // ps], t % ps] = keys[t]
+            vp[perm[t // ps], t % ps] = vals[t]
+        return dict(q=q, k=kp, v=vp, ks=ks, vs=vs, table=perm.astype(np.int32)[None],
+                    lens=np.array([n]))
+
+    full = paged(K, V)
+    trimmed = paged(K[1:], V[1:])
+    sinks = np.linspace(-1, 1, 8).astype(np.float32)
+    for sk in (None, sinks):
+        a = _run(full, window=L - 1, sinks=sk, sm_scale=0.2)
+        b = _run(trimmed, window=0, sinks=sk, sm_scale=0.2)
+        assert np.allclose(a, b, rtol=1e-13, atol=1e-16)
+        assert not np.allclose(a, _run(full, window=0, sinks=sk, sm_scale=0.2), rtol=1e-6, atol=0)
