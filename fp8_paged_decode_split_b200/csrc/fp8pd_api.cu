@@ -147,10 +147,8 @@ struct Plan {
   size_t grp_ml_bytes = 0;    // merged groups of splits
   size_t grp_o_bytes = 0;
   size_t workspace = 0;
-  int schedule = 1;            // 1 = uniform splits, 2 = segment kernel, 3 = proportional splits
-  int nbx = 0;                 // proportional / segment: blocks per KV head x head group
-  int nslot = 0;               // segment: partial slots per (KV head x head group, head)
-  size_t seg_bytes = 0;        // segment: warp rows of the segment ends that do not stop the stream
+  int schedule = 1;            // 1 = uniform splits, 3 = proportional splits
+  int nbx = 0;                 // proportional: blocks per KV head x head group
 };
 
 int current_device(int* dev) {
@@ -176,57 +174,6 @@ int device_sms() {
   }
   cudaGetLastError();
   return sms;
-}
-
-// Segment schedule: one block per SM, floor(SMs / HX) of them per KV head x
-// head group, each with an equal share of the flat list of all sequences'
-// tiles (crossing sequence boundaries). A block's share must fit its tile
-// list, so the grid grows past one wave only when every sequence at its
-// table's full length would not fit; at most kSegMergeFan * 32 blocks per
-// unit (the merge of one sequence's pieces reads at most 32 groups). Only on
-// request (schedule option 2): it balances every SM's work exactly, but its
-// segment ends and end-of-block merges cost more than the proportional
-// splits lose to uneven blocks on every workload measured so far.
-bool plan_seg(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, Plan* plan) {
-  const int64_t sched = g_opt_schedule.load();
-  if (sched != 2 || g_opt_num_splits.load() > 0) return false;
-  if (B > fp8pd::kSegMaxBatch) return false;
-  const int G = Hq / Hkv;
-  const int hg = (G + fp8pd::kHeadsPerGroup - 1) / fp8pd::kHeadsPerGroup;
-  const int64_t HX = static_cast<int64_t>(Hkv) * hg;
-  const int64_t keys = static_cast<int64_t>(max_pages) * ps;
-  const int64_t seq_tiles = window > 0 ? std::min<int64_t>(keys, window) / fp8pd::kTileTokens + 2
-                                       : (keys + fp8pd::kTileTokens - 1) / fp8pd::kTileTokens;
-  const int64_t t_max = B * seq_tiles;  // tiles of one unit when every sequence is full
-  if (t_max >= (int64_t(1) << 31) - 1) return false;
-  const int64_t slots = static_cast<int64_t>(device_sms()) * fp8pd::seg_blocks_per_sm(D, B);
-  const int64_t cap = fp8pd::seg_list_tiles(D);
-  const int64_t nbx_max = static_cast<int64_t>(fp8pd::kSegMergeFan) * 32;
-  int64_t nbx = std::max<int64_t>(1, std::min<int64_t>(slots / HX, nbx_max));
-  nbx = std::max<int64_t>(nbx, (t_max + cap - 1) / cap);
-  if (nbx > nbx_max) return false;
-  const int64_t nslot = nbx + B;
-  plan->schedule = 2;
-  plan->head_groups = hg;
-  plan->nbx = static_cast<int>(nbx);
-  plan->nslot = static_cast<int>(nslot);
-  plan->num_splits = 0;
-  plan->chunk_pages = 0;
-  plan->num_groups = 0;
-  plan->grid_blocks = static_cast<int>(HX * nbx);
-  plan->combine = 1;
-  const size_t rows = static_cast<size_t>(HX * fp8pd::kHeadsPerGroup * nslot);
-  plan->counters_bytes = align256(static_cast<size_t>(HX * nslot + HX * B) * sizeof(int));
-  plan->ml_bytes = align256(rows * 2 * sizeof(float));
-  plan->o_bytes = align256(rows * D * sizeof(float));
-  plan->grp_ml_bytes = plan->ml_bytes;
-  plan->grp_o_bytes = plan->o_bytes;
-  plan->seg_bytes = D > 256 ? 0  // head dim 512 stops the stream at every segment end
-                            : align256(static_cast<size_t>(HX * nbx) * fp8pd::kSegAsync *
-                                       fp8pd::seg_warps(D) * (8 * D + 16) * sizeof(float));
-  plan->workspace = plan->counters_bytes + plan->ml_bytes + plan->o_bytes + plan->grp_ml_bytes +
-                    plan->grp_o_bytes + plan->seg_bytes;
-  return true;
 }
 
 // Proportional splits: the split kernel on a grid of nbx blocks per KV head x
@@ -285,9 +232,7 @@ bool plan_proportional(int B, int Hq, int Hkv, int D, int ps, int max_pages, int
   return true;
 }
 
-int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, Plan* plan,
-              bool allow_seg = true) {
-  if (allow_seg && plan_seg(B, Hq, Hkv, D, ps, max_pages, window, plan)) return FP8PD_OK;
+int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, Plan* plan) {
   // Proportional splits balance sequences of uneven length within one launch;
   // with a short window every sequence has about the same few tiles, and the
   // uniform splits below cost less.
@@ -550,8 +495,9 @@ int validate_decode(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp
 // The capacity T of the partial area fixes the counter area at
 // align256(T / 32 + 256) bytes. Every call has at most one ticket per 33
 // floats of partials: a split call (S >= 2 splits, D >= 64) has at most
-// units * S tickets and units * S * 66 floats; a segment call at most
-// 2 * HX * nslot tickets and 2 * HX * 8 * nslot * 66 floats. So every call
+// units * S tickets and units * S * 66 floats; a proportional call
+// (nbx >= B blocks per KV head x head group) at most (2B + nbx / 8 + 1) * HX
+// <= 3 * nbx * HX tickets and nbx * HX * 8 * 66 floats. So every call
 // whose plan fits in T bytes (fp8pd_plan's workspace_bytes) also fits in the
 // counter area: fp8pd_reserve_workspace(T) covers it.
 size_t counter_area(size_t T) { return align256(T / 32 + 256); }
@@ -627,7 +573,6 @@ void apply_plan(const Plan& plan, DecodeParams* p) {
   p->head_groups = plan.head_groups;
   p->prop = plan.schedule == 3 ? 1 : 0;
   p->nbx = plan.nbx;
-  p->nslot = plan.nslot;
 }
 
 void lay_out(const Plan& plan, void* ctr, void* part, DecodeParams* p) {
@@ -640,14 +585,12 @@ void lay_out(const Plan& plan, void* ctr, void* part, DecodeParams* p) {
   p->grp_ml = reinterpret_cast<float*>(base);
   base += plan.grp_ml_bytes;
   p->grp_o = reinterpret_cast<float*>(base);
-  base += plan.grp_o_bytes;
-  p->seg_scratch = plan.seg_bytes ? reinterpret_cast<float*>(base) : nullptr;
 }
 
 cudaError_t launch_planned(const Plan& plan, const DecodeParams& p, const CUtensorMap& tmk,
                            const CUtensorMap& tmv, cudaStream_t s) {
   const bool kc = g_opt_k_decode.load() == 1, vc = g_opt_v_decode.load() == 1;
-  if (plan.schedule == 2) return fp8pd::launch_decode_seg(p, tmk, tmv, kc, vc, plan.nbx, s);
+  (void)plan;
   return fp8pd::launch_decode(p, tmk, tmv, kc, vc, s);
 }
 
@@ -665,14 +608,11 @@ void record_run(const Plan& plan, int D) {
 namespace {
 
 // Plans, sizes the workspace, encodes the tensor maps and launches one
-// validated decode-attention call. `allow_seg`: the segment kernel may run
-// (it has no fused append). It reads no per-token scales either: with those
-// the split kernel runs.
+// validated decode-attention call.
 int run_decode(DecodeParams& p, const DecodeArgs& a, const fp8pd_tensor* k_pages,
-               const fp8pd_tensor* v_pages, int32_t window, bool allow_seg, fp8pd_stream_t stream) {
+               const fp8pd_tensor* v_pages, int32_t window, fp8pd_stream_t stream) {
   Plan plan;
-  int r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan,
-                    allow_seg && !(p.k_tok || p.v_tok));
+  int r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
   if (r) return r;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   apply_plan(plan, &p);
@@ -710,7 +650,7 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
                           sinks, sm_scale, out, &p, &a);
   if (r) return r;
   if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
-  return run_decode(p, a, k_pages, v_pages, window, true, stream);
+  return run_decode(p, a, k_pages, v_pages, window, stream);
 }
 
 int fp8_paged_decode_append_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_new,
@@ -745,7 +685,7 @@ int fp8_paged_decode_append_attention(const fp8pd_tensor* q, const fp8pd_tensor*
   p.vw = static_cast<uint8_t*>(v_pages->data);
   p.ksw = static_cast<float*>(k_scale->data);
   p.vsw = static_cast<float*>(v_scale->data);
-  r = run_decode(p, a, k_pages, v_pages, window, false, stream);
+  r = run_decode(p, a, k_pages, v_pages, window, stream);
   if (r == FP8PD_OK) ++g_appends;
   return r;
 }
@@ -774,7 +714,7 @@ int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_t
   info->combine = plan.combine;
   info->workspace_bytes = plan.workspace;
   info->schedule = plan.schedule;
-  info->warps = plan.grid_blocks * (plan.schedule == 2 ? fp8pd::seg_warps(static_cast<int>(D)) : 4);
+  info->warps = plan.grid_blocks * 4;
   return FP8PD_OK;
 }
 
@@ -900,7 +840,7 @@ int fp8pd_set_option(int32_t option, int64_t value) {
       g_opt_num_splits = value;
       return FP8PD_OK;
     case FP8PD_OPT_SCHEDULE:
-      if (value < 0 || value > 3) return FP8PD_ERR_ARG;
+      if (value != 0 && value != 1 && value != 3) return FP8PD_ERR_ARG;
       g_opt_schedule = value;
       return FP8PD_OK;
     case FP8PD_OPT_K_DECODE:
@@ -1036,13 +976,8 @@ extern "C" int fp8_paged_decode_attention_noalloc(
   if (r) return r;
   if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
   Plan plan;
-  r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan, !(p.k_tok || p.v_tok));
+  r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
   if (r) return r;
-  if (plan.schedule == 2 && plan.workspace > kNoAllocScratchBytes) {
-    // the segment layout does not fit: the split kernel's may
-    r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan, false);
-    if (r) return r;
-  }
   if (plan.workspace > kNoAllocScratchBytes) return FP8PD_ERR_TOO_LARGE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   apply_plan(plan, &p);

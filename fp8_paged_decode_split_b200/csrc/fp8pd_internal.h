@@ -47,13 +47,6 @@ struct DecodeParams {
   // least ceil(tiles / kMaxSplitTiles), the rest in proportion to its tiles.
   int prop;
   int nbx;
-  // Segment schedule (decode_seg_kernel): partial and group-partial rows
-  // (hx * 8 + head) * nslot + slot, slot < nslot = nbx + B; group tickets
-  // counters[hx * nslot + slot], sequence tickets counters[HX * nslot + hx * B + b].
-  int nslot;
-  // Rows [HX * nbx * kSegAsync * warps][8 * D + 16]: each warp's state at a
-  // segment end that did not stop the stream.
-  float* seg_scratch;
   // Fused append (split kernel only): `lens` holds positions; sequence b
   // attends over positions[b] + 1 keys, the last of them the new token
   // (kn, vn: bf16 [B, Hkv, D]), which the block holding it quantizes, stores
@@ -99,23 +92,6 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 // E4M3 codes (the append's rounding) of n float32 values; strides in elements.
 cudaError_t launch_encode(const float* x, int64_t xs, uint8_t* c, int64_t cs, int64_t n,
                           cudaStream_t s);
-
-// Segment schedule: the tiles of all sequences of one KV head x head group
-// as one list, cut into nbx equal block ranges; grid (HX, nbx) of blocks of
-// 128 threads.
-cudaError_t launch_decode_seg(const DecodeParams& p, const CUtensorMap& tmk,
-                              const CUtensorMap& tmv, bool k_cvt, bool v_cvt, int nbx,
-                              cudaStream_t s);
-// Blocks of the segment kernel one SM holds for head dim D and a batch of B.
-int seg_blocks_per_sm(int D, int B);
-constexpr int kSegMaxBatch = 1024;    // sequences the segment kernel keeps in shared memory
-// Warps per block of the segment kernel (one block per SM; the rings of all
-// warps fill about 192 KiB of shared memory).
-constexpr int seg_warps(int D) { return D <= 128 ? 16 : D == 256 ? 8 : 4; }
-constexpr int kSegAsync = 4;      // segment ends per block that do not stop the stream
-constexpr int kSegMergeFan = 32;  // pieces of a sequence one merge reads
-// Tile entries of one block's range the segment kernel keeps.
-constexpr int seg_list_tiles(int D) { return D <= 128 ? 4096 : D == 256 ? 2048 : 1024; }
 
 // Thread blocks of the split kernel one SM holds for head dim D.
 int decode_blocks_per_sm(int D);

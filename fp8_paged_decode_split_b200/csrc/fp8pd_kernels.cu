@@ -1649,774 +1649,6 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
 }
 
 // ---------------------------------------------------------------------------
-// Balanced block ranges (the segment schedule).
-//
-// The split kernel gives each block a piece of ONE sequence, so with uneven
-// lengths the pieces differ in size and the largest piece decides when the
-// launch ends. Here the work of one KV head x head group is the flat list of
-// the 16-token tiles of all sequences, one after the other (sequence b owns
-// entries [pre_b, pre_{b+1}) of the list); block k of the nbx blocks of that
-// unit takes entries [floor(k T / nbx), floor((k+1) T / nbx)), so every
-// block has the same number of tiles, +-1, whatever the lengths. Each block
-// derives the list from the lengths itself (a prefix sum in shared memory),
-// so one launch does the call.
-//
-// One block per SM, its warps sharing the block's range through a queue in
-// shared memory: a warp takes the next tile whenever it frees a ring stage,
-// so warps that the SM's schedulers favour simply take more tiles and the
-// block ends within about one tile time of its last warp. (Blocks of equal
-// work sharing an SM finish up to a third apart: the schedulers favour the
-// block dispatched first.) The grid is (KV head x head group, nbx) with the
-// heads fastest, so the blocks reading the same tile range of every KV head
-// run side by side and each page leaves DRAM while its rows are open.
-//
-// A block's range crosses sequence boundaries: the part of one sequence
-// inside it is a segment. Every warp processes its tiles in increasing order
-// and, before its first tile past a segment, takes part in closing the
-// segment: each warp writes its online-softmax state into the ring stage it
-// consumed last (a stage of 2 x 16 x D bytes holds exactly 8 heads x D f32),
-// the block merges the states, and either writes the output (the block holds
-// the whole sequence) or a partial (m, l, O) to slot k + b, which is unique
-// because along the partition neither k nor b ever decreases. The pieces of
-// a sequence form groups of kSegMergeFan; the block drawing a group's last
-// ticket merges the group, and with several groups the last group merger
-// merges the groups, adding the sink once. No block ever waits for another.
-// ---------------------------------------------------------------------------
-#ifndef FP8PD_SEG_NS_D64
-#define FP8PD_SEG_NS_D64 6
-#endif
-#ifndef FP8PD_SEG_NS_D128
-#define FP8PD_SEG_NS_D128 3
-#endif
-
-template <int D>
-struct SegCfg {
-  static constexpr int NW = seg_warps(D);
-  static constexpr int NT = NW * 32;
-  static constexpr int NS = (D == 64) ? FP8PD_SEG_NS_D64 : (D == 128) ? FP8PD_SEG_NS_D128 : 3;
-  static constexpr int TILE = kTileTokens * D;
-  static constexpr int STAGE = 2 * TILE;  // = 8 heads x D f32: one warp's state at a segment end
-  static constexpr int WARP_BYTES = NS * STAGE;
-  static constexpr int PIPE_BYTES = NW * WARP_BYTES;
-  static constexpr bool Q_IN_SMEM = (D > 256);
-  static constexpr int QFRAG_BYTES = Q_IN_SMEM ? (D / 16) * 32 * 8 : 0;
-  static constexpr int LB = seg_list_tiles(D);  // tile entries of a block's range
-  static constexpr int LIST_BYTES = LB * 4;
-  static constexpr int SCL_BYTES = NW * NS * 8;  // (k, v) scale of each ring stage
-  static constexpr int BAR_BYTES = NW * NS * 8;
-  static constexpr int ML_BYTES = NW * 8 * 2 * 4;
-  static constexpr int WTS_BYTES = 8 * 32 * 4;
-  static constexpr int MISC_BYTES = 64 * 4;
-  static constexpr int FIXED = 1024 /* alignment slack */ + PIPE_BYTES + QFRAG_BYTES + LIST_BYTES +
-                               SCL_BYTES + BAR_BYTES + ML_BYTES + WTS_BYTES + MISC_BYTES;
-  // lengths [B] and tile prefix sums [B + 1]
-  static constexpr int smem(int B) { return FIXED + 4 * (2 * B + 1); }
-  static_assert(STAGE == 8 * D * 4, "a ring stage must hold one warp's 8 x D state");
-  static_assert(PIPE_BYTES % 1024 == 0, "tiles must stay 1024-byte aligned for the swizzle");
-  static_assert(NW <= 16, "shared-memory bookkeeping holds at most 16 warps");
-};
-
-// 16-token tiles (absolute token positions) that overlap the attended keys
-// [lo, L) of a sequence with L keys.
-__device__ __forceinline__ int seg_tiles(int L, int window) {
-  const int lo = window > 0 ? max(0, L - window) : 0;
-  return L > lo ? (L - 1) / kTileTokens - lo / kTileTokens + 1 : 0;
-}
-
-// The block (of n) whose range holds flat tile f of a list of T tiles: the
-// largest k with floor(k T / n) <= f.
-__device__ __forceinline__ int seg_block_of(int f, int T, int n) {
-  return static_cast<int>(((int64_t)(f + 1) * n - 1) / T);
-}
-
-// Arrival on an mbarrier once every cp.async this thread issued before it has
-// landed (the arrival is one of the barrier's expected arrivals).
-__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_n(uint32_t bar, uint32_t n) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(n) : "memory");
-}
-
-// Grid (HX = KV heads x head groups, nbx), one block per SM; SegCfg<D>::NT
-// threads; dynamic shared memory SegCfg<D>::smem(B). KCVT / VCVT as for the
-// split kernel.
-template <int D, bool KCVT, bool VCVT>
-__global__ void __launch_bounds__(SegCfg<D>::NT, 1)
-    decode_seg_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
-                      const __grid_constant__ CUtensorMap tmv) {
-  using C = SegCfg<D>;
-  constexpr int KB = D / 16;
-  constexpr int NW = C::NW, NT = C::NT, NS = C::NS;
-  constexpr unsigned FULL = 0xffffffffu;
-  constexpr float kLog2e = 1.4426950408889634f;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  uint8_t* pipe = smem;
-  uint2* qfrag_s = reinterpret_cast<uint2*>(smem + C::PIPE_BYTES);
-  int32_t* s_ent = reinterpret_cast<int32_t*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES);
-  float* s_scl = reinterpret_cast<float*>(s_ent + C::LB);
-  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_scl + NW * NS * 2);
-  float* s_ml = reinterpret_cast<float*>(s_bar + NW * NS);  // [NW][8][2]
-  float* s_wts = s_ml + NW * 16;                           // [8][32] merge weights
-  int* s_misc = reinterpret_cast<int*>(s_wts + 256);       // [64]
-  int* s_wsum = s_misc;                                    // [16] scan: sums of the warps
-  int* s_fst = s_misc + 16;                                // [16] each warp's free stage
-  int* s_flag = s_misc + 32;                               // [2] ticket results
-  int* s_next = s_misc + 34;                               // the block's tile queue
-  int* s_ndef = s_misc + 35;                               // merges won by this block's tickets
-  int* s_def = s_misc + 36;                                // [2] their sequences
-  int* s_seg = s_misc + 40;                                // [kSegAsync] sequences of async ends
-  float* s_qmax = reinterpret_cast<float*>(s_misc + 48);   // [NW] q maxima (head dim 512)
-  int* s_len = s_misc + 64;                                // [B] attended keys
-  int* s_pre = s_len + p.B;                                // [B + 1] tile prefix sums
-
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31, grp = lane >> 2, qd = lane & 3;
-  const int B = p.B;
-  const int HX = gridDim.x, hx = blockIdx.x;
-  const int nbx = gridDim.y, kblk = blockIdx.y;
-  const int kvh = hx / p.head_groups;
-  const int hg = hx - kvh * p.head_groups;
-  const int head0 = kvh * p.G + hg * 8;
-  const int nheads = min(8, p.G - hg * 8);
-
-  const uint32_t wbar = smem_u32(s_bar + warp * NS);
-  const uint32_t wpipe = smem_u32(pipe + warp * C::WARP_BYTES);
-  float* wscl = s_scl + warp * NS * 2;
-  if (lane == 0) {
-    if (warp == 0) {
-      prefetch_tensormap(&tmk);
-      prefetch_tensormap(&tmv);
-      *s_next = 0;
-      *s_ndef = 0;
-    }
-    // two arrivals per phase: the copy issuer's expect_tx and the landing of
-    // its scale copies
-#pragma unroll
-    for (int s = 0; s < NS; ++s) mbar_init(wbar + 8 * s, 2);
-    fence_barrier_init();
-    fence_proxy_async();
-  }
-
-  // ---- lengths and tile prefix sums (a contiguous run of sequences per thread)
-  {
-    constexpr int PER_MAX = (kSegMaxBatch + NT - 1) / NT;
-    const int per = (B + NT - 1) / NT;
-    const int b0 = min(B, tid * per);
-    int Lr[PER_MAX];
-#pragma unroll
-    for (int u = 0; u < PER_MAX; ++u)
-      Lr[u] = (u < per && b0 + u < B) ? __ldg(p.lens + (int64_t)(b0 + u) * p.lens_s) : 0;
-    // while the lengths load: bring this block's slice of the block table
-    // into L2, so that every block's later table reads hit L2
-    {
-      const int64_t lines = ((int64_t)p.max_pages * 4 + 127) / 128;
-      const int64_t nl = (int64_t)B * lines, blocks = (int64_t)HX * nbx;
-      const int64_t lin = (int64_t)kblk * HX + hx;
-      for (int64_t i = lin * NT + tid; i < nl; i += blocks * NT) {
-        const int64_t b = i / lines, l = i - b * lines;
-        const int32_t* a = p.table + b * p.tab_sb + l * 32 * p.tab_sp;
-        if (l * 32 < p.max_pages) asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
-      }
-    }
-    int cnt[PER_MAX];
-    int sum = 0;
-#pragma unroll
-    for (int u = 0; u < PER_MAX; ++u) {
-      int L = Lr[u];
-      if (L < 0 || L > p.max_pages * p.ps) {
-        if (hx == 0 && kblk == 0) raise_flag(FP8PD_FLAG_SEQLEN_OOB);
-        L = 0;
-      }
-      cnt[u] = 0;
-      if (u < per && b0 + u < B) {
-        s_len[b0 + u] = L;
-        cnt[u] = seg_tiles(L, p.window);
-      }
-      sum += cnt[u];
-    }
-    int incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(FULL, incl, o);
-      if (lane >= o) incl += v;
-    }
-    if (lane == 31) s_wsum[warp] = incl;
-    __syncthreads();
-    int off = incl - sum;
-    for (int w = 0; w < warp; ++w) off += s_wsum[w];
-#pragma unroll
-    for (int u = 0; u < PER_MAX; ++u) {
-      if (u < per && b0 + u < B) s_pre[b0 + u] = off;
-      off += cnt[u];
-    }
-    if (tid == NT - 1) s_pre[B] = off;
-    __syncthreads();
-  }
-  const int T = s_pre[B];
-  // With fewer tiles than blocks, blocks nbe.. stay idle and every block
-  // below nbe has at least one tile (so every block a sequence spans holds a
-  // piece of it).
-  const int nbe = min(nbx, T);
-  const int f0 = kblk < nbe ? static_cast<int>((int64_t)kblk * T / nbe) : T;
-  const int f1 = kblk < nbe ? static_cast<int>((int64_t)(kblk + 1) * T / nbe) : T;
-  const int nblk = f1 - f0;
-
-  // sequences without keys: their outputs are 0 (spread over the blocks)
-  for (int b = kblk; b < B; b += nbx) {
-    if (s_pre[b + 1] != s_pre[b]) continue;
-    for (int e = tid; e < nheads * D; e += NT)
-      p.out[(int64_t)b * p.o_sb + (int64_t)(head0 + e / D) * p.o_sh + (e % D)] = 0.f;
-  }
-  if (nblk <= 0) return;
-  if (nblk > C::LB) {  // the planner never does this; refuse rather than overflow
-    if (tid == 0) raise_flag(FP8PD_FLAG_INTERNAL);
-    return;
-  }
-
-  // The sequences of this block: b_first .. b_last (those with tiles).
-  auto seq_of = [&](int f, int lo_b, int hi_b) -> int {  // last b in [lo_b, hi_b] with pre_b <= f
-    while (hi_b > lo_b) {
-      const int mid = (lo_b + hi_b + 1) >> 1;
-      if (s_pre[mid] <= f) lo_b = mid;
-      else hi_b = mid - 1;
-    }
-    return lo_b;
-  };
-  const int b_first = seq_of(f0, 0, B - 1);
-  const int b_last = seq_of(f1 - 1, b_first, B - 1);
-  // q of these sequences is read again at every segment start: bring it into
-  // L2 now (its 128-byte lines; D * 2 bytes per head)
-  {
-    constexpr int QL = (D * 2 + 127) / 128;
-    const int nq = (b_last - b_first + 1) * nheads * QL;
-    for (int i = tid; i < nq; i += NT) {
-      const int bq = b_first + i / (nheads * QL);
-      const int r = i % (nheads * QL);
-      const uint16_t* a = p.q + (int64_t)bq * p.q_sb + (int64_t)(head0 + r / QL) * p.q_sh +
-                          (int64_t)(r % QL) * 64 * p.q_sd;
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
-    }
-  }
-
-  // ---- the block's tile list ---------------------------------------------
-  // Entry i (flat tile f0 + i) = (page << 4) | (16-token tile inside the
-  // page), or -1 for a block-table entry outside the pool.
-  auto entry_of = [&](int f) -> int {
-    const int b = seq_of(f, b_first, b_last);
-    const int L = s_len[b];
-    const int lo = p.window > 0 ? max(0, L - p.window) : 0;
-    const int tok = (lo / kTileTokens + (f - s_pre[b])) * kTileTokens;
-    const int lp = tok / p.ps;
-    const int page = __ldg(p.table + (int64_t)b * p.tab_sb + (int64_t)lp * p.tab_sp);
-    if ((unsigned)page < (unsigned)p.num_pages) return (page << 4) | ((tok - lp * p.ps) / kTileTokens);
-    if (hg == 0) raise_flag(FP8PD_FLAG_PAGE_OOB);
-    return -1;
-  };
-
-  const float* ksbase = p.ks + (int64_t)kvh * p.ks_sh;
-  const float* vsbase = p.vs + (int64_t)kvh * p.vs_sh;
-  // Lane 0 copies tile i of the block into ring stage `stage`: one TMA for K,
-  // one for V and the page's two scales (cp.async), all completing on the
-  // stage's barrier. A tile whose page is out of range is not copied; its
-  // barrier phase still completes. Called by the whole warp.
-  int issued = 0;
-  auto issue = [&](int i, int stage) {
-    ++issued;
-    if (lane != 0) return;
-    const int e = s_ent[i];
-    const uint32_t bar = wbar + 8 * stage;
-    if (e < 0) {
-      wscl[2 * stage] = 0.f;  // a masked tile must not carry a stale scale
-      wscl[2 * stage + 1] = 0.f;
-      mbar_arrive_n(bar, 2);
-      return;
-    }
-    const int page = e >> 4, slot0 = (e & 15) * kTileTokens;
-    const uint32_t sk = wpipe + stage * C::STAGE;
-    fence_proxy_async();  // this warp's earlier accesses to the stage come first
-    mbar_arrive_expect_tx(bar, 2 * C::TILE);
-    tma_load_5d(sk, &tmk, bar, 0, slot0, 0, kvh, page);
-    tma_load_5d(sk + C::TILE, &tmv, bar, 0, slot0, 0, kvh, page);
-    cp_async4(wscl + 2 * stage, ksbase + (int64_t)page * p.ks_sp);
-    cp_async4(wscl + 2 * stage + 1, vsbase + (int64_t)page * p.vs_sp);
-    cp_async_mbar_arrive(bar);
-  };
-  // The next tile of the block's queue for this warp (nblk when none is left).
-  auto take = [&]() -> int {
-    int i = 0;
-    if (lane == 0) i = atomicAdd(s_next, 1);
-    return min(__shfl_sync(FULL, i, 0), nblk);
-  };
-
-  // The first entries (one per thread), the first copies of every warp
-  // (tiles warp, warp + NW, ... of the first round), then the rest.
-  if (tid < nblk) s_ent[tid] = entry_of(f0 + tid);
-  __syncthreads();
-  // tiles in this warp's ring, oldest first (nblk: none)
-  int tq[NS - 1];
-#pragma unroll
-  for (int s = 0; s < NS - 1; ++s) {
-    const int i = warp + NW * s;
-    tq[s] = (i < nblk && i < NT) ? i : nblk;
-    if (tq[s] < nblk) issue(tq[s], s);
-  }
-  if (tid == 0) *s_next = min(nblk, min(NT, NW * (NS - 1)));
-#pragma unroll 4
-  for (int i = tid + NT; i < nblk; i += NT) s_ent[i] = entry_of(f0 + i);
-  __syncthreads();  // the whole list and the queue's start are visible
-
-  // ---- per-segment q fragments ---------------------------------------------
-  // Lane (g, q) holds query head g of the group; k16 block kb covers head-dim
-  // entries 16kb + 4q + {0..3}, paired as the K decode needs (see the split
-  // kernel). q' = q * 2^(15 - e) puts max|q'| in [2^14, 2^15); the power of
-  // two and sm_scale * log2(e) (times 2^8 for the bit-assembly K decode) go
-  // into the per-tile score factor.
-  const bool q_head_ok = grp < nheads;
-  uint32_t qf[C::Q_IN_SMEM ? 1 : KB][2];
-  float score_base = 0.f;
-  // All warps call it together when Q_IN_SMEM (they share the fragments).
-  auto load_q = [&](int b) {
-    const uint16_t* qrow = p.q + (int64_t)b * p.q_sb + (int64_t)(head0 + (q_head_ok ? grp : 0)) * p.q_sh;
-    auto raw = [&](int kb) -> uint2 {  // bf16 entries 16kb + 4qd .. +3 of this lane's head
-      const int d = 16 * kb + 4 * qd;
-      uint2 v = make_uint2(0u, 0u);
-      if (q_head_ok) {
-        if (p.q_vec) {
-          v = __ldg(reinterpret_cast<const uint2*>(qrow + d));
-        } else {
-          const uint32_t x0 = __ldg(qrow + (int64_t)(d + 0) * p.q_sd);
-          const uint32_t x1 = __ldg(qrow + (int64_t)(d + 1) * p.q_sd);
-          const uint32_t x2 = __ldg(qrow + (int64_t)(d + 2) * p.q_sd);
-          const uint32_t x3 = __ldg(qrow + (int64_t)(d + 3) * p.q_sd);
-          v = make_uint2(x0 | (x1 << 16), x2 | (x3 << 16));
-        }
-      }
-      return v;
-    };
-    auto max4 = [](uint2 v) -> float {
-      return fmaxf(fmaxf(fabsf(__uint_as_float(v.x << 16)), fabsf(__uint_as_float(v.x & 0xFFFF0000u))),
-                   fmaxf(fabsf(__uint_as_float(v.y << 16)), fabsf(__uint_as_float(v.y & 0xFFFF0000u))));
-    };
-    float qmax = 0.f;
-    if constexpr (C::Q_IN_SMEM) {
-      // this warp's k16 blocks (kb = warp mod NW), parked raw in the fragment
-      // slots they become; the block agrees on max|q| (all warps call this)
-#pragma unroll
-      for (int i = 0; i < KB / NW; ++i) {
-        const int kb = warp + NW * i;
-        const uint2 v = raw(kb);
-        qfrag_s[kb * 32 + lane] = v;
-        qmax = fmaxf(qmax, max4(v));
-      }
-      qmax = warp_max(qmax);
-      if (lane == 0) s_qmax[warp] = qmax;
-      __syncthreads();
-#pragma unroll
-      for (int w = 0; w < NW; ++w) qmax = fmaxf(qmax, s_qmax[w]);
-      __syncthreads();  // s_qmax is read before the next call writes it
-    } else {
-      uint2 qraw[KB];
-#pragma unroll
-      for (int kb = 0; kb < KB; ++kb) qraw[kb] = raw(kb);
-#pragma unroll
-      for (int kb = 0; kb < KB; ++kb) {
-        qmax = fmaxf(qmax, max4(qraw[kb]));
-        qf[kb][0] = qraw[kb].x;  // raw bf16 pairs until the scale is known
-        qf[kb][1] = qraw[kb].y;
-      }
-      qmax = warp_max(qmax);
-    }
-    int qe = 0;
-    if (qmax > 0.f && isfinite(qmax)) frexpf(qmax, &qe);
-    qe = max(qe, -111);
-    const float qmul = ldexpf(1.f, 15 - qe);
-    score_base = p.sm_scale_log2 * (KCVT ? 1.f : 256.f) / qmul;
-#pragma unroll
-    for (int kb = 0; kb < KB; ++kb) {
-      uint2 v;
-      if constexpr (C::Q_IN_SMEM) {
-        if ((kb % NW) != warp) continue;  // this warp's blocks, converted in place
-        v = qfrag_s[kb * 32 + lane];
-      } else {
-        v = make_uint2(qf[kb][0], qf[kb][1]);
-      }
-      const float x0 = __uint_as_float(v.x << 16), x1 = __uint_as_float(v.x & 0xFFFF0000u);
-      const float x2 = __uint_as_float(v.y << 16), x3 = __uint_as_float(v.y & 0xFFFF0000u);
-      uint32_t r0, r1;
-      if constexpr (KCVT) {
-        r0 = pack_f16x2(x0 * qmul, x1 * qmul);
-        r1 = pack_f16x2(x2 * qmul, x3 * qmul);
-      } else {
-        r0 = pack_f16x2(x0 * qmul, x2 * qmul);
-        r1 = pack_f16x2(x1 * qmul, x3 * qmul);
-      }
-      if constexpr (C::Q_IN_SMEM) {
-        qfrag_s[kb * 32 + lane] = make_uint2(r0, r1);
-      } else {
-        qf[kb][0] = r0;
-        qf[kb][1] = r1;
-      }
-    }
-  };
-  auto qfr = [&](int kb) -> uint2 {
-    if constexpr (C::Q_IN_SMEM) return qfrag_s[kb * 32 + lane];
-    else return make_uint2(qf[kb][0], qf[kb][1]);
-  };
-
-  uint32_t koff[4], voff[4];
-  ldsm_offsets<D>(lane, koff, voff);
-  Acc<D> acc;
-  acc.reset();
-  bool ok_all = true;
-  int stage = 0, consumed = 0;
-  uint32_t phase = 0;
-
-  // ---- end of a segment: merge the warps, write the output or a partial ---
-  // Called by every warp for every segment of the block, in order. The ring
-  // stage this warp consumed last is free until its next copy is issued.
-  auto close_segment = [&](int b) {
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      acc.l0 += __shfl_xor_sync(FULL, acc.l0, o);
-      acc.l1 += __shfl_xor_sync(FULL, acc.l1, o);
-    }
-    if (!ok_all) {
-      acc.m0 = acc.m1 = -CUDART_INF_F;
-      acc.l0 = acc.l1 = 0.f;
-    }
-    const int fstage = stage == 0 ? NS - 1 : stage - 1;
-    float* Os = reinterpret_cast<float*>(pipe + warp * C::WARP_BYTES + fstage * C::STAGE);  // [8][D]
-    // V decode offset (bit assembly) times the running V reference scale
-    const float fold = ok_all ? (VCVT ? 1.f : 256.f) * acc.vref : 0.f;
-#pragma unroll
-    for (int jb = 0; jb < D / 32; ++jb) {
-      const int d = 32 * jb + 2 * grp;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        *reinterpret_cast<float2*>(Os + (2 * qd) * D + d + 16 * h) =
-            make_float2(acc.O[jb][h][0] * fold, acc.O[jb][h][2] * fold);
-        *reinterpret_cast<float2*>(Os + (2 * qd + 1) * D + d + 16 * h) =
-            make_float2(acc.O[jb][h][1] * fold, acc.O[jb][h][3] * fold);
-      }
-    }
-    if (grp == 0) {
-      s_ml[(warp * 8 + 2 * qd) * 2 + 0] = acc.m0;
-      s_ml[(warp * 8 + 2 * qd) * 2 + 1] = acc.l0;
-      s_ml[(warp * 8 + 2 * qd + 1) * 2 + 0] = acc.m1;
-      s_ml[(warp * 8 + 2 * qd + 1) * 2 + 1] = acc.l1;
-    }
-    if (lane == 0) s_fst[warp] = fstage;
-    fence_proxy_async();  // the dump precedes later copies into the stage
-    __syncthreads();
-
-    const int pb0 = s_pre[b], pb1 = s_pre[b + 1];
-    const bool whole = pb0 >= f0 && pb1 <= f1;
-    const int kf = seg_block_of(pb0, T, nbe), kl = seg_block_of(pb1 - 1, T, nbe);
-    const int P = kl - kf + 1;  // pieces of this sequence
-    const int NSLOT = p.nslot;
-    const int64_t rbase = (int64_t)hx * 8 * NSLOT;  // + n * NSLOT + slot
-    for (int it = tid; it < 8 * (D / 4); it += NT) {
-      const int n = it / (D / 4);
-      const int d = (it - n * (D / 4)) * 4;
-      if (n >= nheads) continue;
-      float M = -CUDART_INF_F;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, s_ml[(w * 8 + n) * 2]);
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-      float l = 0.f;
-      if (M != -CUDART_INF_F) {
-#pragma unroll 4
-        for (int w = 0; w < NW; ++w) {
-          const float mw = s_ml[(w * 8 + n) * 2];
-          if (mw == -CUDART_INF_F) continue;  // an empty warp's stage holds no state
-          const float f = fast_exp2(mw - M);
-          const float* Ow = reinterpret_cast<const float*>(pipe + w * C::WARP_BYTES + s_fst[w] * C::STAGE);
-          const float4 x = *reinterpret_cast<const float4*>(Ow + n * D + d);
-          o.x += f * x.x;
-          o.y += f * x.y;
-          o.z += f * x.z;
-          o.w += f * x.w;
-          l += f * s_ml[(w * 8 + n) * 2 + 1];
-        }
-      }
-      if (whole) {
-        const int head = head0 + n;
-        const float sl = p.sinks ? p.sinks[(int64_t)head * p.sinks_s] * kLog2e : -CUDART_INF_F;
-        const float M2 = fmaxf(M, sl);
-        float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (M2 != -CUDART_INF_F) {
-          const float a = (M == -CUDART_INF_F) ? 0.f : fast_exp2(M - M2);
-          const float den = l * a + (p.sinks ? fast_exp2(sl - M2) : 0.f);
-          if (den > 0.f) {
-            const float f = a / den;
-            r = make_float4(o.x * f, o.y * f, o.z * f, o.w * f);
-          }
-        }
-        *reinterpret_cast<float4*>(p.out + (int64_t)b * p.o_sb + (int64_t)head * p.o_sh + d) = r;
-      } else {
-        const int64_t row = rbase + (int64_t)n * NSLOT + (kblk + b);
-        *reinterpret_cast<float4*>(p.part_o + row * D + d) = o;
-        if (d == 0) *reinterpret_cast<float2*>(p.part_ml + row * 2) = make_float2(M, l);
-      }
-    }
-    __syncthreads();  // every warp's dump has been read; the block's rows are written
-    if (!whole && tid == 0) {
-      // This piece's ticket in its group of kSegMergeFan pieces. The last piece
-      // merges the group, but only at the block's end, so that the merge
-      // stalls no stream.
-      const int gi = (kblk - kf) / kSegMergeFan;
-      const int gsize = min(kSegMergeFan, P - gi * kSegMergeFan);
-      __threadfence();  // the rows the barrier ordered before this thread go first
-      if (atomicAdd(p.counters + (int64_t)hx * NSLOT + kf + b + gi, 1) == gsize - 1)
-        s_def[(*s_ndef)++] = b;
-    }
-    acc.reset();
-  };
-
-  // ---- end of a segment without stopping the stream ---------------------
-  // The first kSegAsync segment ends of a block that are not its last: each
-  // warp writes its state to its own row of the block's scratch in global
-  // memory and streams on; the block merges those rows after its last tile.
-  // Every warp does it for the same segments (all warps count segment ends
-  // alike). `xs`: index of the segment in the block.
-  const int64_t blin = (int64_t)kblk * HX + hx;
-  constexpr int kSegRow = 8 * D + 16;
-  auto dump_async = [&](int xs, int b) {
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      acc.l0 += __shfl_xor_sync(FULL, acc.l0, o);
-      acc.l1 += __shfl_xor_sync(FULL, acc.l1, o);
-    }
-    if (!ok_all) {
-      acc.m0 = acc.m1 = -CUDART_INF_F;
-      acc.l0 = acc.l1 = 0.f;
-    }
-    float* Os = p.seg_scratch + ((blin * kSegAsync + xs) * NW + warp) * kSegRow;
-    const float fold = ok_all ? (VCVT ? 1.f : 256.f) * acc.vref : 0.f;
-    const bool h0 = 2 * qd < nheads, h1 = 2 * qd + 1 < nheads;
-#pragma unroll
-    for (int jb = 0; jb < D / 32; ++jb) {
-      const int d = 32 * jb + 2 * grp;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (h0)
-          *reinterpret_cast<float2*>(Os + (2 * qd) * D + d + 16 * h) =
-              make_float2(acc.O[jb][h][0] * fold, acc.O[jb][h][2] * fold);
-        if (h1)
-          *reinterpret_cast<float2*>(Os + (2 * qd + 1) * D + d + 16 * h) =
-              make_float2(acc.O[jb][h][1] * fold, acc.O[jb][h][3] * fold);
-      }
-    }
-    if (grp == 0)
-      *reinterpret_cast<float4*>(Os + 8 * D + 4 * qd) = make_float4(acc.m0, acc.l0, acc.m1, acc.l1);
-    if (tid == 0) s_seg[xs] = b;
-    acc.reset();
-  };
-
-  // ---- stream the tiles, segment by segment --------------------------------
-  auto next_seq = [&](int b) -> int {  // the next sequence with tiles
-    ++b;
-    while (b < b_last && s_pre[b + 1] == s_pre[b]) ++b;
-    return b;
-  };
-  int cb = b_first;
-  load_q(cb);
-  if constexpr (C::Q_IN_SMEM) __syncthreads();
-  int L = s_len[cb];
-  int lo = p.window > 0 ? max(0, L - p.window) : 0;
-  int seg_end = s_pre[cb + 1];
-  int xs = 0;
-#pragma unroll 1
-  while (tq[0] < nblk) {
-    const int i = tq[0];
-    const int f = f0 + i;
-    while (f >= seg_end) {
-      if (!C::Q_IN_SMEM && xs < kSegAsync) dump_async(xs, cb);
-      else close_segment(cb);
-      ++xs;
-      cb = next_seq(cb);
-      load_q(cb);
-      if constexpr (C::Q_IN_SMEM) __syncthreads();
-      L = s_len[cb];
-      lo = p.window > 0 ? max(0, L - p.window) : 0;
-      seg_end = s_pre[cb + 1];
-    }
-    if (ok_all && !mbar_wait(wbar + 8 * stage, phase)) {
-      if (lane == 0) raise_flag(FP8PD_FLAG_TIMEOUT);
-      ok_all = false;
-    }
-    const int cur = stage;
-    if (++stage == NS) {
-      stage = 0;
-      phase ^= 1;
-    }
-    // the ring moves up; a new tile goes into the stage freed last time
-#pragma unroll
-    for (int s = 0; s < NS - 2; ++s) tq[s] = tq[s + 1];
-    tq[NS - 2] = nblk;
-    if (!ok_all) continue;
-    ++consumed;
-    __syncwarp();
-    {
-      const int nt = take();
-      if (nt < nblk) {
-        issue(nt, cur == 0 ? NS - 1 : cur - 1);
-        tq[NS - 2] = nt;
-      }
-    }
-    const int e = s_ent[i];
-    const bool page_ok = e >= 0;
-    const int tok0 = (lo / kTileTokens + (f - s_pre[cb])) * kTileTokens;
-    const bool full = page_ok && tok0 >= lo && tok0 + kTileTokens <= L;  // warp-uniform
-    const uint32_t sk = wpipe + cur * C::STAGE;
-    const float kfac = score_base * wscl[2 * cur];
-    const float vs = wscl[2 * cur + 1];
-    attend_tile<D, KCVT, VCVT>(acc, qfr, sk, sk + C::TILE, koff, voff, kfac, kfac, vs, vs,
-                               fabsf(vs), tok0, lo, L, page_ok, full, grp, qd);
-  }
-  // the block's remaining segment ends (every warp takes part in each)
-#pragma unroll 1
-  while (true) {
-    if (!C::Q_IN_SMEM && xs < kSegAsync && cb < b_last) dump_async(xs, cb);
-    else close_segment(cb);
-    ++xs;
-    if (cb >= b_last) break;
-    cb = next_seq(cb);
-    if constexpr (C::Q_IN_SMEM) {
-      load_q(cb);
-      __syncthreads();
-    }
-  }
-
-  // ---- merge the warps' rows of the segments that ended without stopping ---
-  const int nas = C::Q_IN_SMEM ? 0 : min(xs - 1, kSegAsync);
-  if (nas > 0) {
-    __syncthreads();  // every warp's rows are written (and visible to the block)
-    for (int it = tid; it < nas * 8 * (D / 4); it += NT) {
-      const int x = it / (8 * (D / 4));
-      const int r = it - x * (8 * (D / 4));
-      const int n = r / (D / 4);
-      const int d = (r - n * (D / 4)) * 4;
-      if (n >= nheads) continue;
-      const int b = s_seg[x];
-      const float* rows = p.seg_scratch + (blin * kSegAsync + x) * NW * kSegRow;
-      // every row's (m, l) and numerators in one round of loads
-      float2 ml[NW];
-      float4 v[NW];
-#pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        ml[w] = ldcg2(rows + w * kSegRow + 8 * D + 2 * n);
-        v[w] = ldcg4(rows + w * kSegRow + n * D + d);
-      }
-      float M = -CUDART_INF_F;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, ml[w].x);
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-      float l = 0.f;
-      if (M != -CUDART_INF_F) {
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          // an empty warp's row holds m = -inf and numerators of 0
-          const float f = ml[w].x == -CUDART_INF_F ? 0.f : fast_exp2(ml[w].x - M);
-          o.x += f * v[w].x;
-          o.y += f * v[w].y;
-          o.z += f * v[w].z;
-          o.w += f * v[w].w;
-          l += f * ml[w].y;
-        }
-      }
-      const int pb0 = s_pre[b], pb1 = s_pre[b + 1];
-      if (pb0 >= f0 && pb1 <= f1) {  // the whole sequence: the output
-        const int head = head0 + n;
-        const float sl = p.sinks ? p.sinks[(int64_t)head * p.sinks_s] * kLog2e : -CUDART_INF_F;
-        const float M2 = fmaxf(M, sl);
-        float4 rr = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (M2 != -CUDART_INF_F) {
-          const float a = (M == -CUDART_INF_F) ? 0.f : fast_exp2(M - M2);
-          const float den = l * a + (p.sinks ? fast_exp2(sl - M2) : 0.f);
-          if (den > 0.f) {
-            const float f = a / den;
-            rr = make_float4(o.x * f, o.y * f, o.z * f, o.w * f);
-          }
-        }
-        *reinterpret_cast<float4*>(p.out + (int64_t)b * p.o_sb + (int64_t)head * p.o_sh + d) = rr;
-      } else {
-        const int64_t row = (int64_t)hx * 8 * p.nslot + (int64_t)n * p.nslot + (kblk + b);
-        *reinterpret_cast<float4*>(p.part_o + row * D + d) = o;
-        if (d == 0) *reinterpret_cast<float2*>(p.part_ml + row * 2) = make_float2(M, l);
-      }
-    }
-    __syncthreads();  // the block's rows are written
-    if (tid == 0) {
-      // only the block's first segment can be a piece here
-      const int b = s_seg[0];
-      const int pb0 = s_pre[b], pb1 = s_pre[b + 1];
-      if (!(pb0 >= f0 && pb1 <= f1)) {
-        const int kf = seg_block_of(pb0, T, nbe), kl = seg_block_of(pb1 - 1, T, nbe);
-        const int P = kl - kf + 1;
-        const int gi = (kblk - kf) / kSegMergeFan;
-        const int gsize = min(kSegMergeFan, P - gi * kSegMergeFan);
-        __threadfence();
-        if (atomicAdd(p.counters + (int64_t)hx * p.nslot + kf + b + gi, 1) == gsize - 1)
-          s_def[(*s_ndef)++] = b;
-      }
-    }
-  }
-
-  // ---- the merges this block's tickets won (at most its first and last
-  // segments are pieces) ----------------------------------------------------
-  __syncthreads();
-  const int ndef = *s_ndef;
-  const int NSLOT = p.nslot;
-  const int64_t rbase = (int64_t)hx * 8 * NSLOT;
-#pragma unroll 1
-  for (int di = 0; di < ndef; ++di) {
-    const int b = s_def[di];
-    const int kf = seg_block_of(s_pre[b], T, nbe), kl = seg_block_of(s_pre[b + 1] - 1, T, nbe);
-    const int P = kl - kf + 1;
-    const int gi = (kblk - kf) / kSegMergeFan;
-    const int gsize = min(kSegMergeFan, P - gi * kSegMergeFan);
-    const int NG = (P + kSegMergeFan - 1) / kSegMergeFan;
-    const int gslot = kf + b + gi;  // group slot: unique like the piece slots
-    int* gcnt = p.counters + (int64_t)hx * NSLOT + gslot;
-    __threadfence();
-    const int64_t first = rbase + kf + b + gi * kSegMergeFan;  // slot of the group's first piece
-    if (NG == 1) {
-      merge_partials<D, NW>(p.part_ml, p.part_o, first, NSLOT, gsize, nheads, true, p, b, head0,
-                            nullptr, nullptr, 0, 0, s_wts);
-      if (tid == 0) *gcnt = 0;
-    } else {
-      merge_partials<D, NW>(p.part_ml, p.part_o, first, NSLOT, gsize, nheads, false, p, b, head0,
-                            p.grp_ml, p.grp_o, rbase + gslot, NSLOT, s_wts);
-      __syncthreads();
-      int* ucnt = p.counters + (int64_t)HX * NSLOT + (int64_t)hx * B + b;
-      if (tid == 0) {
-        *gcnt = 0;
-        __threadfence();
-        s_flag[1] = (atomicAdd(ucnt, 1) == NG - 1);
-      }
-      __syncthreads();
-      if (s_flag[1]) {
-        __threadfence();
-        merge_partials<D, NW>(p.grp_ml, p.grp_o, rbase + kf + b, NSLOT, NG, nheads, true, p, b,
-                              head0, nullptr, nullptr, 0, 0, s_wts);
-        if (tid == 0) *ucnt = 0;
-      }
-    }
-    __syncthreads();  // s_flag and s_wts are free again
-  }
-
-  // A copy that never completed: wait, bounded, for this warp's copies still
-  // in flight before the block's shared memory goes away.
-  if (!ok_all) {
-    for (int c = consumed; c < issued; ++c)
-      mbar_wait(wbar + 8 * (c % NS), static_cast<uint32_t>((c / NS) & 1));
-  }
-}
-
-// ---------------------------------------------------------------------------
 // Quantize-append: one thread per (sequence, KV head, pair of head-dim
 // entries), for K and V. code = E4M3_RNE_SAT(float32(x) / scale): IEEE float32
 // division (__fdiv_rn), then cvt.rn.satfinite.e4m3x2.f32, which rounds to
@@ -2545,85 +1777,6 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmk, const C
     case 256: return launch_decode_dt<256>(p, tmk, tmv, k_cvt, v_cvt, s);
     case 512: return launch_decode_dt<512>(p, tmk, tmv, k_cvt, v_cvt, s);
     default: return cudaErrorInvalidValue;
-  }
-}
-
-template <int D, bool KCVT, bool VCVT>
-static cudaError_t launch_seg_d(const DecodeParams& p, const CUtensorMap& tmk,
-                                const CUtensorMap& tmv, int nbx, cudaStream_t s) {
-  // the largest dynamic shared memory this kernel is launched with (the
-  // longest batch), set once per device like the split kernel's
-  static std::atomic<uint64_t> configured{0};
-  const int smem_max = SegCfg<D>::smem(kSegMaxBatch);
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
-  if (!bit || !(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(decode_seg_kernel<D, KCVT, VCVT>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
-    if (e != cudaSuccess) return e;
-    configured.fetch_or(bit);
-  }
-  const dim3 grid(p.Hkv * p.head_groups, nbx, 1);
-  decode_seg_kernel<D, KCVT, VCVT><<<grid, SegCfg<D>::NT, SegCfg<D>::smem(p.B), s>>>(p, tmk, tmv);
-  return cudaGetLastError();
-}
-
-template <int D>
-static cudaError_t launch_seg_kv(const DecodeParams& p, const CUtensorMap& tmk,
-                                 const CUtensorMap& tmv, bool k_cvt, bool v_cvt, int nbx,
-                                 cudaStream_t s) {
-  if (k_cvt)
-    return v_cvt ? launch_seg_d<D, true, true>(p, tmk, tmv, nbx, s)
-                 : launch_seg_d<D, true, false>(p, tmk, tmv, nbx, s);
-  return v_cvt ? launch_seg_d<D, false, true>(p, tmk, tmv, nbx, s)
-               : launch_seg_d<D, false, false>(p, tmk, tmv, nbx, s);
-}
-
-cudaError_t launch_decode_seg(const DecodeParams& p, const CUtensorMap& tmk,
-                              const CUtensorMap& tmv, bool k_cvt, bool v_cvt, int nbx,
-                              cudaStream_t s) {
-  if (p.B > kSegMaxBatch) return cudaErrorInvalidValue;
-  switch (p.D) {
-    case 64: return launch_seg_kv<64>(p, tmk, tmv, k_cvt, v_cvt, nbx, s);
-    case 128: return launch_seg_kv<128>(p, tmk, tmv, k_cvt, v_cvt, nbx, s);
-    case 256: return launch_seg_kv<256>(p, tmk, tmv, k_cvt, v_cvt, nbx, s);
-    case 512: return launch_seg_kv<512>(p, tmk, tmv, k_cvt, v_cvt, nbx, s);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-// Blocks per SM for batches of up to 128 * k sequences (shared memory grows
-// with the batch), cached per bucket k.
-template <int D>
-static int seg_blocks_per_sm_d(int B) {
-  static std::atomic<int> cached[kSegMaxBatch / 128 + 1];  // 0 = not known yet
-  const int k = (B + 127) / 128;
-  int c = cached[k].load();
-  if (c > 0) return c;
-  int n = 0;
-  if (cudaFuncSetAttribute(decode_seg_kernel<D, true, true>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           SegCfg<D>::smem(kSegMaxBatch)) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_seg_kernel<D, true, true>,
-                                                    SegCfg<D>::NT, SegCfg<D>::smem(128 * k)) != cudaSuccess) {
-    cudaGetLastError();
-    return 1;  // no device: do not cache the guess
-  }
-  c = n > 0 ? n : 1;
-  cached[k].store(c);
-  return c;
-}
-
-int seg_blocks_per_sm(int D, int B) {
-  if (B < 0 || B > kSegMaxBatch) return 1;
-  switch (D) {
-    case 64: return seg_blocks_per_sm_d<64>(B);
-    case 128: return seg_blocks_per_sm_d<128>(B);
-    case 256: return seg_blocks_per_sm_d<256>(B);
-    case 512: return seg_blocks_per_sm_d<512>(B);
-    default: return 1;
   }
 }
 

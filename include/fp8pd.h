@@ -166,8 +166,6 @@ enum {
  *                sub-row key scales): head-dim entry d of a key uses scale
  *                [page, slot, h, d / (D / G)]; G in {1, 2, 4, 8, 16} with
  *                D / G >= 16, else FP8PD_ERR_UNSUPPORTED. V takes G = 1 only.
- *                With a per-token form the segment schedule is not used (a
- *                request for it runs the split kernel's own plan).
  *   block_table  int32 [B, max_pages]: physical page of each logical page.
  *                Entries past the attended range are never read.
  *   seq_lens     int32 [B]: number of keys visible to the query (positions 0..L-1).
@@ -176,19 +174,15 @@ enum {
  *   sm_scale     finite, > 0.
  *   out          float32 [B, Hq, D]; stride[2] must be 1, rows 16-byte aligned.
  *   stream       CUDA stream.
- * Launches one kernel, with one of three schedules. Uniform splits (1): the
+ * Launches one kernel, with one of two schedules. Uniform splits (1): the
  * split kernel gives each (sequence, KV head, head group) the same number of
  * blocks, each an equal share of its table's pages. Proportional splits (3):
  * the split kernel on one wave of blocks per KV head x head group, shared
  * among the sequences in proportion to their tiles (the kernel reads the
  * lengths). In both, the last block of each (sequence, KV head, head group)
- * to finish merges its splits. Segment kernel (2, on request): one block per
- * SM; the 16-token tiles of all sequences form one list per KV head x head
- * group, cut into equal block ranges that cross sequence boundaries, and the
- * block's warps share its range through a queue. The planner takes
- * proportional splits for full attention and windows of at least 2,048 keys
- * when there is enough work and their grid fits one wave of the device,
- * uniform splits otherwise.
+ * to finish merges its splits. The planner takes proportional splits for
+ * full attention and windows of at least 2,048 keys when there is enough
+ * work and their grid fits one wave of the device, uniform splits otherwise.
  * The partial results and the ticket counters live
  * in a library-owned per-device workspace: it grows on demand outside stream
  * capture; under capture a call that would need to grow it fails with
@@ -258,8 +252,7 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
  * the pools are written. A position outside [0, max_pages * page_size) sets
  * FP8PD_FLAG_POS_OOB and that sequence's output is 0, nothing is written; a
  * block-table entry outside the pool sets FP8PD_FLAG_PAGE_OOB. Runs the split
- * kernel (uniform or proportional splits; a request for the segment kernel
- * falls back to uniform splits). Workspace rules as fp8_paged_decode_attention.
+ * kernel (uniform or proportional splits). Workspace rules as fp8_paged_decode_attention.
  */
 int fp8_paged_decode_append_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_new,
                                       const fp8pd_tensor* v_new, fp8pd_tensor* k_pages,
@@ -298,12 +291,12 @@ int fp8_paged_decode_attention_noalloc(const fp8pd_tensor* q, const fp8pd_tensor
 /* What a call with these arguments would launch, without launching it. */
 typedef struct fp8pd_plan_info {
   int32_t num_splits;        /* uniform splits: blocks per (sequence, KV head, head group);
-                                proportional splits and the segment kernel: 0 */
+                                proportional splits: 0 */
   int32_t head_groups;       /* ceil(G / 8) query-head groups per KV head */
   int32_t grid_blocks;       /* thread blocks of the launch */
   int32_t combine;           /* 1 if partial results are merged (workspace used) */
   uint64_t workspace_bytes;  /* split workspace the call needs (0 if none) */
-  int32_t schedule;          /* 1 = uniform splits, 2 = segment kernel, 3 = proportional splits */
+  int32_t schedule;          /* 1 = uniform splits, 3 = proportional splits */
   int32_t warps;             /* warps of the launch */
 } fp8pd_plan_info;
 
@@ -337,10 +330,10 @@ enum {
   FP8PD_OPT_NUM_SPLITS = 1,  /* 0 = planner chooses (default); n > 0 asks for n splits (raised
                                 so that no split covers more than 8,192 keys, capped at 256
                                 splits and at the number of pages) */
-  FP8PD_OPT_SCHEDULE = 2,    /* 0 = planner chooses (default); 1 = uniform splits; 2 = segment
-                                kernel where it applies (B <= 1024, no forced split count),
-                                else uniform splits; 3 = proportional splits where they apply
-                                (B <= 1024, no forced split count), else uniform splits */
+  FP8PD_OPT_SCHEDULE = 2,    /* 0 = planner chooses (default); 1 = uniform splits;
+                                3 = proportional splits where they apply (B <= 1024, no
+                                forced split count), else uniform splits; any other value
+                                is refused with FP8PD_ERR_ARG */
   FP8PD_OPT_K_DECODE = 3,    /* E4M3 -> f16 decode of K: 0 = bit assembly,
                                 1 = hardware cvt.rn.f16x2.e4m3x2 (default) */
   FP8PD_OPT_V_DECODE = 4     /* the same for V (default 1) */
@@ -350,7 +343,7 @@ int64_t fp8pd_get_option(int32_t option);
 
 /* What the last attention call on this host thread launched. */
 typedef struct fp8pd_run_info {
-  int32_t schedule;          /* 1 = uniform splits, 2 = segment kernel, 3 = proportional splits */
+  int32_t schedule;          /* 1 = uniform splits, 3 = proportional splits */
   int32_t num_splits;
   int32_t head_groups;
   int32_t grid_blocks;

@@ -185,11 +185,13 @@ def test_options_roundtrip(F):
     F.fp8pd_set_option(F.OPT_NUM_SPLITS, 7)
     assert F.fp8pd_get_option(F.OPT_NUM_SPLITS) == 7
     F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
-    F.fp8pd_set_option(F.OPT_SCHEDULE, 2)
-    assert F.fp8pd_get_option(F.OPT_SCHEDULE) == 2
+    F.fp8pd_set_option(F.OPT_SCHEDULE, 3)
+    assert F.fp8pd_get_option(F.OPT_SCHEDULE) == 3
     F.fp8pd_set_option(F.OPT_SCHEDULE, 0)
-    with pytest.raises(F.Fp8pdError):
-        F.fp8pd_set_option(F.OPT_SCHEDULE, 4)
+    for bad in (2, 5, -1):
+        with pytest.raises(F.Fp8pdError):
+            F.fp8pd_set_option(F.OPT_SCHEDULE, bad)
+    assert F.fp8pd_get_option(F.OPT_SCHEDULE) == 0
     with pytest.raises(F.Fp8pdError):
         F.fp8pd_set_option(99, 1)
     with pytest.raises(F.Fp8pdError):
@@ -251,7 +253,7 @@ def test_planner_fills_the_device_with_enough_work_per_split(F, split_schedule):
 def test_planner_default_schedule(F):
     """The planner's own choice: proportional splits for full attention and
     long windows with enough work when their grid is one wave, uniform splits
-    otherwise; the segment kernel only on request. Without a GPU it assumes
+    otherwise. Without a GPU it assumes
     148 SMs and the launch-bound blocks per SM."""
     assert _plan(F, 32, 32, 8, 128, 16, 257)["schedule"] == 3           # Llama-like
     assert _plan(F, 1, 64, 8, 128, 64, 2049)["schedule"] == 3           # one 131k-key sequence
@@ -262,34 +264,6 @@ def test_planner_default_schedule(F):
     assert _plan(F, 64, 64, 8, 64, 16, 513, window=128)["schedule"] == 1
     assert _plan(F, 1, 8, 2, 64, 16, 16)["schedule"] == 1               # too little work
     assert _plan(F, 1025, 8, 8, 128, 16, 400)["schedule"] == 1          # more than 1,024 sequences
-
-
-def test_planner_segment_kernel_on_request(F):
-    """Schedule 2: one block per SM, floor(148 / HX) of them per KV head x
-    head group without a GPU, each an equal share of all tiles; more blocks
-    only when the largest share would overflow a block's tile list (4,096
-    tiles at head dim 128)."""
-    F.fp8pd_set_option(F.OPT_SCHEDULE, 2)
-    try:
-        p = _plan(F, 32, 32, 8, 128, 16, 257)
-        assert p["schedule"] == 2 and p["num_splits"] == 0 and p["combine"] == 1
-        assert p["grid_blocks"] == 8 * 18
-        nbx, B, D, HX = 18, 32, 128, 8
-        assert p["workspace_bytes"] >= 2 * HX * 8 * (nbx + B) * (D + 2) * 4
-        assert _plan(F, 1, 8, 2, 64, 16, 16)["grid_blocks"] == 2 * 74
-        assert _plan(F, 16, 16, 2, 512, 32, 513)["schedule"] == 2      # every head dim
-        # 8 sequences of 131,136 keys: 65,568 tiles per KV head, 18 blocks of 3,643
-        p = _plan(F, 8, 64, 8, 128, 64, 2049)
-        assert p["schedule"] == 2 and p["grid_blocks"] == 8 * 18
-        # 16 such sequences need 33 blocks of at most 4,096 tiles per KV head
-        p = _plan(F, 16, 64, 8, 128, 64, 2049)
-        assert p["schedule"] == 2 and p["grid_blocks"] == 8 * 33
-        assert _plan(F, 1025, 8, 8, 128, 16, 4)["schedule"] == 1       # more than 1,024 sequences
-        F.fp8pd_set_option(F.OPT_NUM_SPLITS, 3)
-        assert _plan(F, 32, 32, 8, 128, 16, 257)["schedule"] == 1      # a forced split count wins
-    finally:
-        F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
-        F.fp8pd_set_option(F.OPT_SCHEDULE, 0)
 
 
 def test_planner_proportional_splits(F):

@@ -25,11 +25,10 @@ def F(cuda_device):
     return F
 
 
-@pytest.fixture(autouse=True, params=[1, 2, 3], ids=["split", "segment", "proportional"])
+@pytest.fixture(autouse=True, params=[1, 3], ids=["split", "proportional"])
 def schedule(F, request):
-    """Every test runs with each schedule: uniform splits, the segment kernel
-    (balanced block ranges across sequences; no forced split count) and
-    proportional splits (no forced split count)."""
+    """Every test runs with each schedule: uniform splits and proportional
+    splits (no forced split count)."""
     F.fp8pd_set_option(F.OPT_SCHEDULE, request.param)
     yield request.param
     F.fp8pd_set_option(F.OPT_SCHEDULE, 0)
@@ -186,7 +185,8 @@ def test_the_requested_kernel_runs(F, cuda_device, schedule):
 
 def test_ragged_batch_with_empty_and_long_sequences(F, cuda_device, kdecode):
     """40 sequences from 0 to 3,000 keys, every seventh empty and one of a
-    single key: the segment kernel's block ranges cross many sequence boundaries."""
+    single key: proportional splits give the long ones many blocks and the
+    empty ones none."""
     spec = W.Spec("ragged", B=40, ps=16, layers=(W.LayerSpec(32, 8, 128, 0, None),),
                   seq_len=(0, 3000), scale_mode="page", sinks=True, seed=77)
     case = W.make_case(spec, cuda_device)

@@ -50,9 +50,8 @@ def _both(F, layer, lens):
     ("long_b1", dict(seq_len=20000), 0, 1),               # many splits, two-level merge
     ("long_b1", dict(seq_len=20000), 5, 1),               # a single merge group
     ("gptoss_full", dict(B=3, seq_len=1000), 0, 1),       # sinks
-    ("llama", dict(B=6, seq_len=(40, 700)), 0, 2),        # the segment kernel
-    ("long_b1", dict(seq_len=20000), 0, 2),               # segment kernel, two-level merge
     ("llama", dict(B=6, seq_len=(40, 700)), 0, 3),        # proportional splits
+    ("long_b1", dict(seq_len=60000), 0, 3),               # proportional, two-level merge
 ])
 def test_noalloc_matches_the_allocating_entry_point(F, cuda_device, name, overrides, splits,
                                                     schedule):
