@@ -3,28 +3,37 @@
 One step = the decode hot path for one layer of a synthetic serving batch:
 the append of one new token per sequence, then decode attention over the
 updated paged E4M3 cache -- by default one ``fp8_paged_decode_append_attention``
-launch (split kernel, append and combine fused); ``--unfused`` runs
-``fp8_kv_append`` and ``fp8_paged_decode_attention`` as two launches.
-Configs without an append run the attention call alone. Inputs are resident
-in HBM when the timed region starts;
-L2 is flushed between timed steps, outside each step's
-events. ``value`` = algorithmic bytes (attended K/V once per KV head + q +
-the block-table entries read) / device time, summed over ranks.
+launch (append and split combine fused); ``--unfused`` runs ``fp8_kv_append``
+and ``fp8_paged_decode_attention`` as two launches. Configs without an append
+run the attention call alone. Inputs are resident in HBM when the timed
+region starts; L2 is flushed between timed steps, outside each step's events.
+``value`` = algorithmic bytes (attended K/V once per KV head + q + the
+block-table entries read) / device time, summed over ranks.
+
+The headline workload is the largest single-GPU one (long context, 8
+sequences of 131,072 keys). At N = 1 the same JSON line also carries a
+``configs`` object with the other serving workloads (Llama-like, gpt-oss-like
+full and windowed, the mixed pool with one roofline per layer, long context
+B = 1), each timed the same way.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
 
-With N > 1 (torchrun, one process per GPU) every rank runs its own copy of
-the workload on its GPU (independent sequences: no data-path collective);
-time is the max over ranks, throughput the sum (weak scaling).
-``--impl reference`` times the float64 CPU oracle on the same workload (rank
-0 only).
+With N > 1 every rank runs its own copy of the workload on its GPU
+(independent sequences: no data-path collective); time is the max over ranks,
+throughput the sum (weak scaling). Started without a launcher, ``--gpus N``
+re-runs itself under ``torch.distributed.run`` with N ranks (and refuses when
+fewer than N GPUs are visible). ``--impl reference`` times the float64 CPU
+oracle on the same workload on every host core (rank 0 only).
 """
 
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import json
 import os
+import platform
+import socket
 import statistics
 import subprocess
 import sys
@@ -41,7 +50,9 @@ if ROOT not in sys.path:
 import workloads as W  # noqa: E402
 
 METRIC = "FP8 paged decode attention: achieved HBM GB/s and µs/step on 1 B200"
-DEFAULT_CONFIG = "llama"
+DEFAULT_CONFIG = "long_b8"
+#: the other workloads timed beside the headline (N = 1 only)
+SWEEP = ("llama", "gptoss_full", "gptoss_w128", "mixed", "long_b1")
 WORKLOAD_TEXT = {
     "llama": "Llama-3-8B-like layer: B=32 Hq=32 Hkv=8 D=128 page=16 seq_len~U[512,4096] "
              "per-(page,head) scales, +1 appended token/seq",
@@ -49,13 +60,16 @@ WORKLOAD_TEXT = {
     "gptoss_full": "gpt-oss-like: B=64 Hq=64 Hkv=8 D=64 page=16 L=8192 sinks, full attention",
     "gptoss_w128": "gpt-oss-like: B=64 Hq=64 Hkv=8 D=64 page=16 L=8192 sinks, window=128",
     "mixed": "mixed pool: B=16 page=32 L~U[2048,16384]; sliding D=256 W=1024 + full D=512",
-    "long_b1": "long context: B=1 Hq=64 Hkv=8 D=128 page=64 L=131072 +append",
-    "long_b8": "long context: B=8 Hq=64 Hkv=8 D=128 page=64 L=131072 +append",
+    "long_b1": "long context: B=1 Hq=64 Hkv=8 D=128 page=64 L=131072 per-KV-head scales, "
+               "+1 appended token",
+    "long_b8": "long context: B=8 Hq=64 Hkv=8 D=128 page=64 L=131072 per-KV-head scales, "
+               "+1 appended token/seq",
 }
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic_per_launch.txt")
 KERNEL_NAME = {1: "decode_tma_kernel (split kernel, merge in the same launch)",
-               2: "decode_seg_kernel (balanced block ranges across sequences, merge in the same launch)",
                3: "decode_tma_kernel (proportional splits, merge in the same launch)"}
+L2_TEXT = ("flushed between timed steps: 256 MiB write, then a 256 MiB read of another buffer "
+           "(no dirty lines left), outside the step events")
 
 
 def _peaks() -> dict:
@@ -76,15 +90,16 @@ def _kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def _traffic(config: str):
-    """DRAM bytes (read + write) per split-kernel launch from the committed ncu
-    summary, if it was taken on the current kernel source and this workload.
-    Lines of that file: ``<workload> <kernel source hash> <bytes>``."""
+def _traffic(config: str, layer: int = 0):
+    """DRAM bytes (read + write) per attention-kernel launch from the committed
+    ncu summary, if it was taken on the current kernel source. Lines of that
+    file: ``<workload>[:<layer>] <kernel source hash> <bytes> [how]``."""
+    key = config if layer == 0 else f"{config}:{layer}"
     try:
         with open(PROFILE_TRAFFIC) as f:
             for line in f:
                 parts = line.split()
-                if len(parts) == 3 and not line.startswith("#") and parts[0] == config \
+                if len(parts) >= 3 and not line.startswith("#") and parts[0] == key \
                         and parts[1] == _kernel_source_hash():
                     return float(parts[2])
     except OSError:
@@ -97,8 +112,7 @@ class L2Flush:
     of another 256 MiB buffer. The write alone would leave the L2 full of
     dirty lines whose write-back to HBM then lands inside the next timed
     step; after the read every line in the L2 is clean, so the step pays only
-    for its own traffic. FLUSH_MODE = "write" keeps the plain write."""
-    MODE = os.environ.get("FP8PD_BENCH_FLUSH", "write+read")
+    for its own traffic."""
 
     def __init__(self, device: torch.device):
         self.w = torch.empty(256 << 20, dtype=torch.uint8, device=device)
@@ -106,15 +120,8 @@ class L2Flush:
         self.sink = torch.empty((), dtype=torch.float32, device=device)
 
     def fill_(self, v: int = 1) -> None:
-        if "write" in self.MODE:
-            self.w.fill_(v & 0xFF)
-        if "read" in self.MODE:
-            torch.sum(self.r, dim=0, out=self.sink)
-
-    def describe(self) -> str:
-        return {"write": "256 MiB write", "read": "256 MiB read",
-                "write+read": "256 MiB write, then a 256 MiB read of another buffer (no dirty "
-                              "lines left)"}[self.MODE] + ", outside the step events"
+        self.w.fill_(v & 0xFF)
+        torch.sum(self.r, dim=0, out=self.sink)
 
 
 class ClockSampler:
@@ -204,16 +211,19 @@ def whole_job_gbs(world: int, bytes_per_rank_step: int, ms_per_step: float) -> f
 class Step:
     """One decode step of the workload through the library's public API: with
     an append, the fused call (append and attention in one launch) unless
-    `fused` is off, then fp8_kv_append followed by the attention call."""
+    `fused` is off, then fp8_kv_append followed by the attention call.
+    ``layers`` restricts the step to some layers (per-layer timing)."""
 
-    def __init__(self, F, case: W.Case, fused: bool = True):
+    def __init__(self, F, case: W.Case, fused: bool = True, layers=None):
         self.F = F
         self.case = case
         self.fused = fused and case.spec.append
+        self.layers = list(range(len(case.layers))) if layers is None else list(layers)
 
     def run(self, stream=None):
         F, c = self.F, self.case
-        for layer in c.layers:
+        for li in self.layers:
+            layer = c.layers[li]
             if self.fused:
                 F.fp8_paged_decode_append_attention(
                     layer.q, layer.k_new, layer.v_new, layer.k_pages, layer.v_pages,
@@ -235,27 +245,46 @@ def _step_bytes(case: W.Case) -> int:
     return sum(W.algorithmic_bytes(case, i) for i in range(len(case.layers)))
 
 
-def run_ours(args) -> dict | None:
-    import fp8_paged_decode_split_b200 as F
-    F.fp8pd_set_option(F.OPT_K_DECODE, 1 if args.k_decode == "cvt" else 0)
-    F.fp8pd_set_option(F.OPT_NUM_SPLITS, args.splits)
-    F.fp8pd_set_option(F.OPT_SCHEDULE, args.schedule)
-    world, rank, local = _dist_env()
-    if world > 1:
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
-    dev = torch.device("cuda", local if world > 1 else 0)
-    torch.cuda.set_device(dev)
-    case = W.make_case(args.config, dev, **_scale_override(args))
-    for layer in case.layers:
-        layer.out = torch.empty(layer.q.shape, dtype=torch.float32, device=dev)
-    step = Step(F, case, not args.unfused)
-    flush = L2Flush(dev)
-    stream = torch.cuda.current_stream(dev)
-    nbytes = _step_bytes(case)
+def _config_dict(args, name: str, case_or_none=None, nbytes=None) -> dict:
+    """The ``config`` object of a line: the same keys and values for both arms."""
+    spec = W.spec_with(name, **_scale_override(args))
+    if nbytes is None:
+        # algorithmic bytes depend only on lengths and shapes: a CPU copy of
+        # the workload's lengths is enough (no pools are built)
+        nbytes = _spec_bytes(spec)
+    world = _dist_env()[0]
+    return {"workload": _workload_text(args, name), "name": name, "bytes_per_step": int(nbytes),
+            "scales": _scales_text(spec),
+            "l2": L2_TEXT, "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"}
 
-    for _ in range(args.warmup):
+
+def _spec_bytes(spec: W.Spec) -> int:
+    """Algorithmic bytes of one step of ``spec`` from its lengths and shapes
+    (the same count as workloads.algorithmic_bytes, without building pools)."""
+    rng = np.random.default_rng(spec.seed)
+    lens = W._lengths(spec, rng) + (1 if spec.append else 0)
+    total = 0
+    for L in spec.layers:
+        for Lb in lens:
+            lo = max(0, Lb - L.window) if L.window > 0 else 0
+            n = max(0, Lb - lo)
+            total += 2 * n * L.Hkv * L.D
+            if n > 0:
+                total += 4 * ((Lb - 1) // spec.ps - lo // spec.ps + 1)
+            if spec.scale_mode == "token":
+                total += 4 * n * L.Hkv * (spec.k_groups + 1)
+        total += 2 * spec.B * L.Hq * L.D
+    return int(total)
+
+
+def time_case(F, case: W.Case, dev, args, flush: L2Flush, steps: int, warmup: int,
+              clocks: bool = False) -> dict:
+    """Device time of the workload's step as CUDA-graph replays (per-step
+    events, L2 flushed between), then each layer's attention kernel alone from
+    an eager pass (the library's events around its launch)."""
+    stream = torch.cuda.current_stream(dev)
+    step = Step(F, case, not args.unfused)
+    for _ in range(warmup):
         step.run()
         flush.fill_(1)
     torch.cuda.synchronize(dev)
@@ -263,8 +292,8 @@ def run_ours(args) -> dict | None:
         raise RuntimeError("device error word set during warm-up")
     info0 = F.fp8pd_last_run_info()
     step.run()
-    plan_info = F.fp8pd_last_run_info()
-    launches_per_step = int(plan_info["kernel_launches"] - info0["kernel_launches"])
+    info1 = F.fp8pd_last_run_info()
+    launches_per_step = int(info1["kernel_launches"] - info0["kernel_launches"])
     torch.cuda.synchronize(dev)
 
     # ---- the step as a CUDA graph (how a serving loop replays decode steps) --
@@ -276,57 +305,149 @@ def run_ours(args) -> dict | None:
     stream.wait_stream(side)
     with torch.cuda.graph(graph):
         step.run()
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         graph.replay()
         flush.fill_(1)
     torch.cuda.synchronize(dev)
 
-    # ---- device-timed region: inputs resident, per-step events, L2 flushed between
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+          for _ in range(steps)]
+    world = _dist_env()[0]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(dev) as clocks:
-        for i in range(args.steps):
+    sampler = ClockSampler(dev) if clocks else None
+    if sampler:
+        sampler.__enter__()
+    try:
+        for i in range(steps):
             ev[i][0].record(stream)
             graph.replay()
             ev[i][1].record(stream)
             flush.fill_(i & 0xFF)
         torch.cuda.synchronize(dev)
+    finally:
+        if sampler:
+            sampler.__exit__()
     if world > 1:
         torch.distributed.barrier()
     total_ms = sum(a.elapsed_time(b) for a, b in ev)
-    launches = launches_per_step * args.steps
-
-    # ---- per-kernel durations: the same steps eagerly, the library's events
-    # around each of its kernels on the launching stream, L2 flushed between
-    F.fp8pd_timing_enable(True)
-    F.fp8pd_timing_collect()
-    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        # a ~1 ms spin first, so the host has queued the whole step before the
-        # GPU reaches it: the library's per-kernel events then hold device
-        # time only, with no host launch gaps inside them
-        torch.cuda._sleep(2_000_000)
-        ev2[i][0].record(stream)
-        step.run()
-        ev2[i][1].record(stream)
-        flush.fill_(i & 0xFF)
-    torch.cuda.synchronize(dev)
-    eager_ms = sum(a.elapsed_time(b) for a, b in ev2)
-    kt = F.fp8pd_timing_collect()
-    F.fp8pd_timing_enable(False)
-    if F.fp8pd_check_errors() != 0:
-        raise RuntimeError("device error word set during the timed region")
     del graph
 
-    # ---- end to end through the public API with host buffers -----------------
-    e2e = run_e2e(F, case, dev, flush, args)
+    # ---- per-layer kernel durations: eager, one layer at a time, the
+    # library's events around each launch on the launching stream
+    per_layer = []
+    eager_ms = 0.0
+    for li in range(len(case.layers)):
+        lstep = Step(F, case, not args.unfused, layers=[li])
+        F.fp8pd_timing_enable(True)
+        F.fp8pd_timing_collect()
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        torch.cuda.synchronize(dev)
+        for i in range(steps):
+            # a ~1 ms spin first, so the host has queued the whole step before
+            # the GPU reaches it: the per-kernel events then hold device time
+            # only, with no host launch gaps inside them
+            torch.cuda._sleep(2_000_000)
+            ev2[i][0].record(stream)
+            lstep.run()
+            ev2[i][1].record(stream)
+            flush.fill_(i & 0xFF)
+        torch.cuda.synchronize(dev)
+        eager_ms += sum(a.elapsed_time(b) for a, b in ev2)
+        kt = F.fp8pd_timing_collect()
+        F.fp8pd_timing_enable(False)
+        run = F.fp8pd_last_run_info()
+        att_ms = kt["attention_ms"] / max(1, kt["attention_launches"])
+        app_ms = kt["append_ms"] / kt["append_launches"] if kt["append_launches"] else None
+        per_layer.append({"bytes": W.algorithmic_bytes(case, li), "kernel_ms": att_ms,
+                          "append_ms": app_ms,
+                          "plan": {k: run[k] for k in ("schedule", "num_splits", "head_groups",
+                                                       "grid_blocks", "combine")}})
+    if F.fp8pd_check_errors() != 0:
+        raise RuntimeError("device error word set during the timed region")
+    return {"ms_per_step": total_ms / steps, "eager_ms_per_step": eager_ms / steps,
+            "launches_per_step": launches_per_step, "layers": per_layer,
+            "clocks": sampler.summary() if sampler else None, "fused": step.fused}
 
-    total_ms, e2e_ms = max_over_ranks([total_ms, e2e["ms"]], dev)
+
+def _roofline(entry: dict, peaks: dict, fused: bool, traffic=None) -> dict:
+    ms = entry["kernel_ms"]
+    achieved = entry["bytes"] / (ms * 1e-3) / 1e9 if ms > 0 else None
+    kernel = KERNEL_NAME.get(entry["plan"]["schedule"], "decode kernel") + \
+        (", append fused" if fused else "")
+    return {"bound": "hbm", "kernel": kernel,
+            "achieved": round(achieved, 2) if achieved else None,
+            "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4) if achieved else None,
+            "traffic": traffic, "bytes_per_launch": int(entry["bytes"]),
+            "us_per_launch": round(ms * 1e3, 3),
+            "append_us_per_launch": round(entry["append_ms"] * 1e3, 3) if entry["append_ms"] else None,
+            "plan": entry["plan"]}
+
+
+def _build_case(name: str, dev, args) -> W.Case:
+    case = W.make_case(name, dev, **_scale_override(args))
+    for layer in case.layers:
+        layer.out = torch.empty(layer.q.shape, dtype=torch.float32, device=dev)
+    return case
+
+
+def _set_options(F, args) -> None:
+    F.fp8pd_set_option(F.OPT_K_DECODE, 1 if args.k_decode == "cvt" else 0)
+    F.fp8pd_set_option(F.OPT_NUM_SPLITS, args.splits)
+    F.fp8pd_set_option(F.OPT_SCHEDULE, args.schedule)
+
+
+def run_ours(args) -> dict | None:
+    import fp8_paged_decode_split_b200 as F
+    _set_options(F, args)
+    world, rank, local = _dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    peaks = _peaks()
+    flush = L2Flush(dev)
+
+    case = _build_case(args.config, dev, args)
+    nbytes = _step_bytes(case)
+    t = time_case(F, case, dev, args, flush, args.steps, args.warmup, clocks=True)
+    e2e = run_e2e(F, case, dev, flush, args)
+    total_ms, e2e_ms = max_over_ranks([t["ms_per_step"] * args.steps, e2e["ms"]], dev)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(case, budget_s=args.cpu_seconds)
+    del case
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads (one GPU only: the scaling runs time the headline)
+    sweep = {}
+    if world == 1 and not args.no_sweep:
+        for name in SWEEP:
+            if name == args.config:
+                continue
+            c = _build_case(name, dev, args)
+            ts = time_case(F, c, dev, args, flush, max(5, min(args.steps, 20)),
+                           max(3, args.warmup))
+            nb = _step_bytes(c)
+            ent = {"workload": _workload_text(args, name),
+                   "us_per_step": round(ts["ms_per_step"] * 1e3, 3),
+                   "value": round(nb / (ts["ms_per_step"] * 1e-3) / 1e9, 2), "unit": "GB/s",
+                   "bytes_per_step": nb,
+                   "roofline": [_roofline(e, peaks, ts["fused"],
+                                          _traffic(name, i) if args.scales == "workload" else None)
+                                for i, e in enumerate(ts["layers"])]}
+            if len(ent["roofline"]) == 1:
+                ent["roofline"] = ent["roofline"][0]
+            sweep[name] = ent
+            del c
+            torch.cuda.empty_cache()
+
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank != 0:
@@ -334,12 +455,7 @@ def run_ours(args) -> dict | None:
 
     ms_per_step = total_ms / args.steps
     gbs = whole_job_gbs(world, nbytes, ms_per_step)
-    peaks = _peaks()
-    att_ms = kt["attention_ms"] / max(1, kt["attention_launches"])
-    app_ms = kt["append_ms"] / kt["append_launches"] if kt["append_launches"] else None
-    layer_bytes = nbytes / max(1, len(case.layers))
-    achieved = layer_bytes / (att_ms * 1e-3) / 1e9 if att_ms > 0 else None
-    traffic = _traffic(args.config) if args.scales == "workload" else None
+    head = t["layers"][0]
     line = {
         "metric": METRIC,
         "value": round(gbs, 2),
@@ -354,35 +470,22 @@ def run_ours(args) -> dict | None:
         "vs_baseline": None,
         "dtype": "e4m3 cache; f16 tensor-core MMA, f32 accumulate",
         "data": "synthetic (seeded), no dataset",
-        "config": {"workload": _workload_text(args),
-                   "name": args.config,
-                   "bytes_per_step": nbytes, "k_decode": args.k_decode,
-                   "scales": _scales_text(case),
-                   "l2": "flushed between timed steps: " + flush.describe(),
-                   "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
+        "config": _config_dict(args, args.config, nbytes=nbytes),
         "timing": "device time of CUDA-graph replays of the step (per-step events); "
-                  "eager time and per-kernel events from an eager pass of the same steps",
-        "eager_ms_per_step": round(eager_ms / args.steps, 6),
-        "roofline": {"bound": "hbm",
-                     "kernel": KERNEL_NAME[plan_info["schedule"]] +
-                     (", append fused" if step.fused else ""),
-                     "achieved": round(achieved, 2) if achieved else None,
-                     "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
-                     "unit": "GB/s",
-                     "frac": round(achieved / peaks["hbm_gbs"], 4) if achieved else None,
-                     "traffic": traffic,
-                     "us_per_launch": round(att_ms * 1e3, 3),
-                     "append_us_per_launch": round(app_ms * 1e3, 3) if app_ms else None},
-        "gpu_launches": launches,
+                  "per-kernel events from an eager pass of the same steps",
+        "eager_ms_per_step": round(t["eager_ms_per_step"], 6),
+        "roofline": _roofline(head, peaks, t["fused"],
+                              _traffic(args.config) if args.scales == "workload" else None),
+        "gpu_launches": t["launches_per_step"] * args.steps,
         "e2e": {"value": round(whole_job_gbs(world, nbytes, e2e_ms / e2e["steps"]), 2),
                 "unit": "GB/s", "ms_per_step": round(e2e_ms / e2e["steps"], 6),
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
-        "clocks": clocks.summary(),
-        "plan": {k: plan_info[k] for k in ("schedule", "num_splits", "head_groups", "grid_blocks",
-                                           "combine")},
+        "clocks": t["clocks"],
     }
-    if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(case, budget_s=args.cpu_seconds)
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if sweep:
+        line["configs"] = sweep
     return line
 
 
@@ -444,24 +547,84 @@ def run_e2e(F, case: W.Case, dev, flush, args) -> dict:
     return {"ms": ms, "steps": steps, "h2d": int(h2d), "d2h": int(d2h)}
 
 
-def _oracle_step(case_np: dict, lens, positions, append: bool):
+# ---------------------------------------------------------------------------
+# The oracle on the host's cores
+# ---------------------------------------------------------------------------
+
+def host_threads() -> int:
+    """Host cores this process may run on."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def _oracle_tasks(case_np: dict, lens) -> list:
+    """The oracle's work as (layer, sequence, KV head, algorithmic bytes)
+    tasks: the attended K and V bytes of that KV head, its block-table
+    entries and the q rows of its query heads."""
+    tasks = []
+    for li, L in enumerate(case_np["layers"]):
+        B, Hq, D = L["q"].shape
+        ps, Hkv = L["k_pages"].shape[1], L["k_pages"].shape[2]
+        G = Hq // Hkv
+        for b in range(B):
+            Lb = int(lens[b])
+            lo = max(0, Lb - L["window"]) if L["window"] > 0 else 0
+            n = max(0, Lb - lo)
+            tok = sum(4 * n * (sc.shape[3] if sc.ndim == 4 else 1)
+                      for sc in (L["k_scale"], L["v_scale"]) if sc.ndim >= 3)
+            tbl = 4 * ((Lb - 1) // ps - lo // ps + 1) if n > 0 else 0
+            for h in range(Hkv):  # the table row is read once per sequence
+                tasks.append((li, b, h, 2 * n * D + tok + (tbl if h == 0 else 0) + 2 * G * D))
+    return tasks
+
+
+def _oracle_step(case_np: dict, lens, positions, append: bool, tasks, pool=None):
+    """One step of the oracle over ``tasks``: the appends of their sequences
+    (one token each, in order), then the attention of every task's
+    (sequence, KV head) as its own job on ``pool`` (numpy releases the GIL
+    inside its array kernels, so the jobs run on several cores at once)."""
     import oracle as O
-    for L in case_np["layers"]:
-        if append:
-            O.kv_append(L["k_new"], L["v_new"], L["k_pages"], L["v_pages"], L["k_scale"],
-                        L["v_scale"], L["block_table"], positions)
-        O.paged_decode_attention(L["q"], L["k_pages"], L["v_pages"], L["k_scale"], L["v_scale"],
-                                 L["block_table"], lens, window=L["window"], sinks=L["sinks"],
-                                 sm_scale=L["sm_scale"])
+    seqs = sorted({b for _, b, _, _ in tasks})
+    if append:
+        for L in case_np["layers"]:
+            idx = np.array(seqs)
+            O.kv_append(L["k_new"][idx], L["v_new"][idx], L["k_pages"], L["v_pages"],
+                        L["k_scale"], L["v_scale"], L["block_table"][idx], positions[idx])
+    jobs = []
+    for li, b, h, _ in tasks:
+        L = case_np["layers"][li]
+        G = L["q"].shape[1] // L["k_pages"].shape[2]
+        args = (L["q"], L["k_pages"], L["v_pages"], L["k_scale"], L["v_scale"],
+                L["block_table"], lens)
+        kw = dict(window=L["window"], sinks=L["sinks"], sm_scale=L["sm_scale"],
+                  batch_heads=[(b, h * G + g) for g in range(G)])
+        if pool is None:
+            O.paged_decode_attention(*args, **kw)
+        else:
+            jobs.append(pool.submit(O.paged_decode_attention, *args, **kw))
+    for j in jobs:
+        j.result()
 
 
-def _case_to_numpy(case: W.Case, seqs) -> tuple[dict, np.ndarray, np.ndarray | None, int]:
+def _case_to_numpy(case: W.Case, seqs) -> tuple[dict, np.ndarray, np.ndarray | None]:
     """Host copy of the sequences ``seqs`` of a case (their pages only)."""
     out = {"layers": []}
     ps = case.spec.ps
     lens = case.attend_lens.cpu().numpy()[seqs]
     pos = case.positions.cpu().numpy()[seqs] if case.positions is not None else None
-    nbytes = 0
     for li, layer in enumerate(case.layers):
         tbl = layer.block_table.cpu().numpy()[seqs]
         npg = (lens + ps - 1) // ps
@@ -475,48 +638,64 @@ def _case_to_numpy(case: W.Case, seqs) -> tuple[dict, np.ndarray, np.ndarray | N
         f = lambda t: t.detach().float().cpu().numpy().astype(np.float64)  # noqa: E731
         # per-page and per-token scales follow their pages; per-head ones do not
         pick = lambda sc: (sc[idx] if sc.dim() >= 2 else sc).cpu().numpy()  # noqa: E731
-        d = {"q": f(layer.q[list(seqs)]),
-             "k_pages": layer.k_pages[idx].cpu().numpy(), "v_pages": layer.v_pages[idx].cpu().numpy(),
-             "k_scale": pick(layer.k_scale), "v_scale": pick(layer.v_scale),
-             "block_table": new_tbl, "window": layer.window, "sm_scale": layer.sm_scale,
-             "sinks": layer.sinks.cpu().numpy() if layer.sinks is not None else None,
-             "k_new": f(layer.k_new[list(seqs)]) if layer.k_new is not None else None,
-             "v_new": f(layer.v_new[list(seqs)]) if layer.v_new is not None else None}
-        out["layers"].append(d)
-        for b in range(len(seqs)):
-            Lb = int(lens[b])
-            lo = max(0, Lb - layer.window) if layer.window > 0 else 0
-            n = Lb - lo
-            nbytes += 2 * n * layer.spec.Hkv * layer.spec.D
-            nbytes += sum(4 * n * layer.spec.Hkv * (sc.shape[3] if sc.dim() == 4 else 1)
-                          for sc in (layer.k_scale, layer.v_scale) if sc.dim() >= 3)
-            if n > 0:
-                nbytes += 4 * ((Lb - 1) // ps - lo // ps + 1)
-        nbytes += 2 * d["q"].size
-    return out, lens, pos, nbytes
+        out["layers"].append({
+            "q": f(layer.q[list(seqs)]),
+            "k_pages": layer.k_pages[idx].cpu().numpy(), "v_pages": layer.v_pages[idx].cpu().numpy(),
+            "k_scale": pick(layer.k_scale), "v_scale": pick(layer.v_scale),
+            "block_table": new_tbl, "window": layer.window, "sm_scale": layer.sm_scale,
+            "sinks": layer.sinks.cpu().numpy() if layer.sinks is not None else None,
+            "k_new": f(layer.k_new[list(seqs)]) if layer.k_new is not None else None,
+            "v_new": f(layer.v_new[list(seqs)]) if layer.v_new is not None else None})
+    return out, lens, pos
+
+
+def _oracle_sample(case: W.Case, step_seconds: float, threads: int, pool):
+    """A bounded sample of the workload for the oracle: the first sequences
+    of the batch (their pages copied to the host), and as many of their
+    (layer, sequence, KV head) tasks, in order, as the host's cores finish in
+    about ``step_seconds`` (sized from one timed task; at least one task)."""
+    B = case.spec.B
+    per_seq = _step_bytes(case) / max(1, B)
+    # enough sequences for the largest sample the time budget could take
+    nseq = max(1, min(B, int(2e9 / max(1.0, per_seq)) + 1))
+    seqs = list(range(nseq))
+    case_np, lens, pos = _case_to_numpy(case, seqs)
+    tasks = _oracle_tasks(case_np, lens)
+    probe = tasks[:1]
+    t0 = time.perf_counter()
+    _oracle_step(case_np, lens, pos, case.spec.append, probe, None)
+    one = max(1e-4, time.perf_counter() - t0)
+    n = max(1, min(len(tasks), int(step_seconds * threads / one)))
+    chosen = tasks[:n]
+    # keep the host copy of the sequences the sample uses only
+    used = sorted({b for _, b, _, _ in chosen})
+    if len(used) < len(seqs):
+        case_np, lens, pos = _case_to_numpy(case, used)
+        remap = {b: i for i, b in enumerate(used)}
+        chosen = [(li, remap[b], h, nb) for li, b, h, nb in chosen]
+    nbytes = sum(nb for *_, nb in chosen)
+    text = (f"{len(chosen)} of {len(tasks) * B // nseq} (layer, sequence, KV head) tasks over "
+            f"{len(used)}/{B} sequences ({nbytes / 1e6:.1f} MB algorithmic per step), float64 "
+            f"numpy, {threads} threads on {cpu_model()}")
+    return case_np, lens, pos, chosen, nbytes, text
 
 
 def cpu_baseline(case: W.Case, budget_s: float = 10.0) -> dict:
-    """The oracle as it stands, timed on this host on a bounded sample of the
-    workload: whole steps over the first sequences of the batch, repeated
-    until about ``budget_s`` seconds, single BLAS thread."""
+    """The oracle as it stands, timed on every core of this host on a bounded
+    sample of the workload, repeated until about ``budget_s`` seconds, one
+    BLAS thread per job."""
     from threadpoolctl import threadpool_limits
-    B = case.spec.B
-    total = _step_bytes(case)
-    nseq = max(1, min(B, int(B * 160e6 / max(1, total))))   # ~1 s of oracle work per step
-    seqs = list(range(nseq))
-    case_np, lens, pos, nbytes = _case_to_numpy(case, seqs)
-    reps, t_total = 0, 0.0
-    with threadpool_limits(1):
+    threads = host_threads()
+    with threadpool_limits(1), concurrent.futures.ThreadPoolExecutor(threads) as pool:
+        case_np, lens, pos, tasks, nbytes, text = _oracle_sample(case, 1.5, threads, pool)
+        reps, t_total = 0, 0.0
         while t_total < budget_s and reps < 1000:
             t0 = time.perf_counter()
-            _oracle_step(case_np, lens, pos, case.spec.append)
+            _oracle_step(case_np, lens, pos, case.spec.append, tasks, pool)
             t_total += time.perf_counter() - t0
             reps += 1
-    return {"value": round(nbytes * reps / t_total / 1e9, 4), "unit": "GB/s", "cores": 1,
-            "kind": "oracle",
-            "sample": f"{reps} full step(s) over {nseq}/{B} sequences "
-                      f"({nbytes / 1e6:.1f} MB/step algorithmic), float64 numpy, 1 thread",
+    return {"value": round(nbytes * reps / t_total / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle", "sample": f"{reps} step(s) of {text}",
             "seconds": round(t_total, 2)}
 
 
@@ -528,65 +707,113 @@ def _scale_override(args) -> dict:
     return {"scale_mode": "token", "k_groups": getattr(args, "k_groups", 1)}
 
 
-def _workload_text(args) -> str:
-    text = WORKLOAD_TEXT.get(args.config, args.config)
+def _workload_text(args, name: str | None = None) -> str:
+    name = name or args.config
+    text = WORKLOAD_TEXT.get(name, name)
     if getattr(args, "scales", "workload") != "token":
         return text
     groups = f", K in {args.k_groups} sub-row groups" if args.k_groups > 1 else ""
     return text + f" (scales replaced: per (token, KV head){groups})"
 
 
-def _scales_text(case) -> str:
+def _scales_text(spec) -> str:
     text = {"head": "per KV head", "page": "per (page, KV head)",
-            "token": "per (token, KV head)"}[case.spec.scale_mode]
-    if case.spec.scale_mode == "token" and case.spec.k_groups > 1:
-        text += f"; K per (token, KV head, group of D/{case.spec.k_groups})"
+            "token": "per (token, KV head)"}[spec.scale_mode]
+    if spec.scale_mode == "token" and spec.k_groups > 1:
+        text += f"; K per (token, KV head, group of D/{spec.k_groups})"
     return text
 
 
 def run_reference(args) -> dict | None:
-    """The float64 CPU oracle on this host: each step is one bounded sample of
-    the workload (rank 0 only)."""
+    """The float64 CPU oracle on this host's cores: each step is one bounded
+    sample of the workload (rank 0 only)."""
     world, rank, _ = _dist_env()
     if rank != 0:
         return None
     from threadpoolctl import threadpool_limits
     case = W.make_case(args.config, "cpu", **_scale_override(args))
-    B = case.spec.B
-    # bounded sample per step: as many whole sequences as fit in ~1.5 s
-    seqs = list(range(B))
-    case_np, lens, pos, nbytes = _case_to_numpy(case, seqs)
-    with threadpool_limits(1):
-        t0 = time.perf_counter()
-        _oracle_step(case_np, lens, pos, case.spec.append)
-        one = time.perf_counter() - t0
-        if one > 1.5 and B > 1:
-            keep = max(1, int(B * 1.5 / one))
-            seqs = list(range(keep))
-            case_np, lens, pos, nbytes = _case_to_numpy(case, seqs)
+    threads = host_threads()
+    with threadpool_limits(1), concurrent.futures.ThreadPoolExecutor(threads) as pool:
+        case_np, lens, pos, tasks, nbytes, text = _oracle_sample(case, 1.5, threads, pool)
         for _ in range(args.warmup):
-            _oracle_step(case_np, lens, pos, case.spec.append)
+            _oracle_step(case_np, lens, pos, case.spec.append, tasks, pool)
         t0 = time.perf_counter()
         for _ in range(args.steps):
-            _oracle_step(case_np, lens, pos, case.spec.append)
+            _oracle_step(case_np, lens, pos, case.spec.append, tasks, pool)
         total = time.perf_counter() - t0
     gbs = nbytes * args.steps / total / 1e9
-    sample = f"{len(seqs)}/{B} sequences per step ({nbytes / 1e6:.1f} MB algorithmic), float64 numpy"
     return {
         "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded), no dataset",
-        "config": {"workload": _workload_text(args), "name": args.config,
-                   "scales": _scales_text(case)},
-        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+        "config": _config_dict(args, args.config),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": text},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
 
 
-def main():
+# ---------------------------------------------------------------------------
+# Launching N ranks
+# ---------------------------------------------------------------------------
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_ranks(argv: list, gpus: int, dry_run: bool, timeout_s: float = 1800.0) -> int:
+    """Re-runs this script under ``torch.distributed.run`` with ``gpus`` ranks
+    on this node (rendezvous on 127.0.0.1) and returns its exit code. Refuses,
+    before starting anything, when fewer than ``gpus`` GPUs are visible
+    (a dry run needs none)."""
+    if not dry_run:
+        visible = torch.cuda.device_count() if torch.cuda.is_available() else 0
+        if visible < gpus:
+            print(f"bench.py: --gpus {gpus} needs {gpus} visible GPUs, found {visible}",
+                  file=sys.stderr)
+            return 2
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={gpus}", "--master-addr=127.0.0.1",
+           f"--master-port={_free_port()}", os.path.abspath(__file__), *argv]
+    env = dict(os.environ)
+    env.pop("WORLD_SIZE", None)
+    try:
+        return subprocess.run(cmd, env=env, timeout=timeout_s).returncode
+    except subprocess.TimeoutExpired:
+        print("bench.py: ranks did not finish in time", file=sys.stderr)
+        return 3
+
+
+def run_dry(args) -> dict | None:
+    """Host logic of an N-rank run without a GPU: gloo ranks, a host-timed
+    stand-in step, the max-over-ranks reduction and the weak-scaled total."""
+    import datetime
+    import torch.distributed as dist
+    world, rank, _ = _dist_env()
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    nbytes = _spec_bytes(W.spec_with(args.config))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        np.dot(np.ones(1 << 16), np.ones(1 << 16))
+    ms = (time.perf_counter() - t0) * 1e3 / max(1, args.steps) + 1e-3 * (1 + rank)
+    (ms_max,) = max_over_ranks([ms], torch.device("cpu"))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    return {"dry_run": True, "metric": METRIC, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max,
+            "value": round(whole_job_gbs(world, nbytes, ms_max), 2), "unit": "GB/s",
+            "scaling": "weak", "config": _config_dict(args, args.config, nbytes=nbytes)}
+
+
+def build_parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -594,6 +821,10 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(W.SPECS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="time the headline workload only (no configs object)")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="host logic of the N-rank run only (gloo, no GPU)")
     ap.add_argument("--unfused", action="store_true",
                     help="run fp8_kv_append and the attention call as two launches")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -604,19 +835,34 @@ def main():
                     help="token: per-token-per-head K/V scales instead of the workload's form")
     ap.add_argument("--k-groups", type=int, default=1,
                     help="with --scales token: K scales per sub-row group of D / k_groups entries")
-    ap.add_argument("--schedule", type=int, default=0, choices=[0, 1, 2, 3],
-                    help="0 = planner, 1 = uniform splits, 2 = segment kernel, "
-                         "3 = proportional splits")
-    args = ap.parse_args()
+    ap.add_argument("--schedule", type=int, default=0, choices=[0, 1, 3],
+                    help="0 = planner, 1 = uniform splits, 3 = proportional splits")
+    return ap
+
+
+def main(argv=None) -> int:
+    argv = sys.argv[1:] if argv is None else list(argv)
+    ap = build_parser()
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
     world = _dist_env()[0]
-    if world > 1 and args.gpus != world:
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return launch_ranks(argv, args.gpus, args.dry_run)
+    if args.gpus != world:
         ap.error(f"--gpus {args.gpus} does not match WORLD_SIZE={world}")
-    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if args.dry_run:
+        line = run_dry(args)
+    elif args.impl == "reference":
+        line = run_reference(args)
+    else:
+        line = run_ours(args)
     if line is not None:
         print(json.dumps(line), flush=True)
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

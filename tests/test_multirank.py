@@ -87,3 +87,73 @@ def test_max_over_ranks_without_a_process_group_is_the_identity():
     import bench
     assert not dist.is_initialized()
     assert bench.max_over_ranks([1.5, 2.5], torch.device("cpu")) == [1.5, 2.5]
+
+
+def test_bench_starts_n_ranks_itself_in_a_dry_run():
+    """``bench.py --gpus 2`` without a launcher re-runs itself under
+    torch.distributed.run with two ranks; the dry run (gloo, no GPU) reports
+    n_gpus 2 from rank 0 only, with the weak-scaled total."""
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dry-run",
+                        "--steps", "3", "--warmup", "3", "--config", "tiny"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = lines[0]
+    assert line["n_gpus"] == 2 and line["dry_run"] is True
+    assert line["config"]["parallelism"] == "2 independent replicas"
+    import bench
+    assert line["value"] == pytest.approx(
+        bench.whole_job_gbs(2, line["config"]["bytes_per_step"], line["ms_per_step"]), abs=0.01)
+
+
+def test_bench_refuses_more_gpus_than_it_sees():
+    import subprocess
+    if torch.cuda.is_available() and torch.cuda.device_count() >= 64:
+        pytest.skip("this host has 64 GPUs")
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "64",
+                        "--steps", "3", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert r.returncode == 2
+    assert "needs 64 visible GPUs" in r.stderr
+    assert not [x for x in r.stdout.splitlines() if x.startswith("{")]
+
+
+@pytest.mark.parametrize("name,overrides", [
+    ("tiny", {}), ("llama", dict(B=5)), ("gptoss_w128", dict(B=3, seq_len=700)),
+    ("gptoss_full", dict(B=2, seq_len=300)), ("mixed", dict(B=3, seq_len=(100, 1500))),
+    ("long_b1", dict(seq_len=3000)), ("llama", dict(B=3, scale_mode="token", k_groups=4)),
+])
+def test_bench_bytes_from_the_spec_equal_the_workload_count(name, overrides):
+    """The reference arm's config states the bytes per step without building
+    the pools; they equal the count over the built workload."""
+    import bench
+    import workloads as W
+    spec = W.spec_with(name, **overrides)
+    case = W.make_case(spec, "cpu")
+    assert bench._spec_bytes(spec) == bench._step_bytes(case)
+
+
+def test_bench_oracle_tasks_cover_the_step_bytes():
+    import bench
+    import workloads as W
+    case = W.make_case("llama", "cpu", B=4)
+    case_np, lens, _ = bench._case_to_numpy(case, list(range(4)))
+    tasks = bench._oracle_tasks(case_np, lens)
+    assert len(tasks) == 4 * 8
+    assert sum(t[3] for t in tasks) == bench._step_bytes(case)
+
+
+def test_both_arms_state_the_same_config():
+    import bench
+
+    class Args:
+        config, steps, warmup, scales, k_groups = "llama", 1, 3, "workload", 1
+    import workloads as W
+    case = W.make_case("llama", "cpu")
+    ours = bench._config_dict(Args, "llama", nbytes=bench._step_bytes(case))
+    ref = bench._config_dict(Args, "llama")
+    assert ours == ref
