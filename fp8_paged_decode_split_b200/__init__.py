@@ -31,14 +31,16 @@ __all__ = [
     "fp8pd_check_errors", "fp8pd_set_option", "fp8pd_get_option", "fp8pd_last_run_info",
     "fp8pd_timing_enable", "fp8pd_timing_collect", "Fp8pdError", "lib", "LIB_PATH",
     "FLAG_PAGE_OOB", "FLAG_SEQLEN_OOB", "FLAG_POS_OOB", "FLAG_INTERNAL", "OPT_NUM_SPLITS",
-    "OPT_SCHEDULE", "OPT_K_DECODE", "OPT_V_DECODE",
+    "OPT_SCHEDULE", "OPT_K_DECODE", "OPT_V_DECODE", "OPT_WAIT_POLLS",
+    "OPT_TEST_STALL", "FLAG_TIMEOUT",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libfp8pd.so")
 
 DTYPE_U8, DTYPE_I32, DTYPE_F32, DTYPE_BF16 = 1, 2, 3, 4
-FLAG_PAGE_OOB, FLAG_SEQLEN_OOB, FLAG_POS_OOB, FLAG_INTERNAL = 1, 2, 4, 8
+FLAG_PAGE_OOB, FLAG_SEQLEN_OOB, FLAG_POS_OOB, FLAG_INTERNAL, FLAG_TIMEOUT = 1, 2, 4, 8, 16
 OPT_NUM_SPLITS, OPT_SCHEDULE, OPT_K_DECODE, OPT_V_DECODE = 1, 2, 3, 4
+OPT_WAIT_POLLS, OPT_TEST_STALL = 6, 7
 _DTYPES = {torch.uint8: DTYPE_U8, torch.int32: DTYPE_I32, torch.float32: DTYPE_F32,
            torch.bfloat16: DTYPE_BF16}
 

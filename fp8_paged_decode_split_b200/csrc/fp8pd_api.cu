@@ -26,7 +26,8 @@ constexpr int kMaxDevices = 64;
 thread_local int32_t t_last_cuda_error = 0;
 thread_local fp8pd_run_info t_run_info = {};
 std::atomic<int64_t> g_calls{0}, g_appends{0}, g_launches{0};
-std::atomic<int64_t> g_opt_num_splits{0}, g_opt_schedule{0}, g_opt_k_decode{1}, g_opt_v_decode{1};
+std::atomic<int64_t> g_opt_num_splits{0}, g_opt_schedule{0}, g_opt_k_decode{1}, g_opt_v_decode{1},
+    g_opt_wait_polls{1 << 17}, g_opt_test_stall{0};
 
 struct Workspace {
   void* ptr = nullptr;
@@ -573,6 +574,8 @@ void apply_plan(const Plan& plan, DecodeParams* p) {
   p->head_groups = plan.head_groups;
   p->prop = plan.schedule == 3 ? 1 : 0;
   p->nbx = plan.nbx;
+  p->wait_polls = static_cast<int>(g_opt_wait_polls.load());
+  p->test_stall = g_opt_test_stall.load() ? 1 : 0;
 }
 
 void lay_out(const Plan& plan, void* ctr, void* part, DecodeParams* p) {
@@ -714,7 +717,7 @@ int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_t
   info->combine = plan.combine;
   info->workspace_bytes = plan.workspace;
   info->schedule = plan.schedule;
-  info->warps = plan.grid_blocks * 4;
+  info->warps = plan.grid_blocks * fp8pd::decode_warps_per_block(static_cast<int>(D));
   return FP8PD_OK;
 }
 
@@ -851,6 +854,14 @@ int fp8pd_set_option(int32_t option, int64_t value) {
       if (value < 0 || value > 1) return FP8PD_ERR_ARG;
       g_opt_v_decode = value;
       return FP8PD_OK;
+    case FP8PD_OPT_WAIT_POLLS:
+      if (value < 1 || value > (1 << 20)) return FP8PD_ERR_ARG;
+      g_opt_wait_polls = value;
+      return FP8PD_OK;
+    case FP8PD_OPT_TEST_STALL:
+      if (value < 0 || value > 1) return FP8PD_ERR_ARG;
+      g_opt_test_stall = value;
+      return FP8PD_OK;
     default:
       return FP8PD_ERR_ARG;
   }
@@ -862,6 +873,8 @@ int64_t fp8pd_get_option(int32_t option) {
     case FP8PD_OPT_SCHEDULE: return g_opt_schedule.load();
     case FP8PD_OPT_K_DECODE: return g_opt_k_decode.load();
     case FP8PD_OPT_V_DECODE: return g_opt_v_decode.load();
+    case FP8PD_OPT_WAIT_POLLS: return g_opt_wait_polls.load();
+    case FP8PD_OPT_TEST_STALL: return g_opt_test_stall.load();
     default: return -1;
   }
 }

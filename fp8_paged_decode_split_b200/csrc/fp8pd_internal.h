@@ -47,6 +47,11 @@ struct DecodeParams {
   // least ceil(tiles / kMaxSplitTiles), the rest in proportion to its tiles.
   int prop;
   int nbx;
+  // Bounded waits: polls of a tile barrier before a wait gives up (sets
+  // FLAG_TIMEOUT); test_stall: the first block's warp 0 never issues its
+  // first copy (the timeout path's test hook).
+  int wait_polls;
+  int test_stall;
   // Fused append (split kernel only): `lens` holds positions; sequence b
   // attends over positions[b] + 1 keys, the last of them the new token
   // (kn, vn: bf16 [B, Hkv, D]), which the block holding it quantizes, stores
@@ -95,6 +100,8 @@ cudaError_t launch_encode(const float* x, int64_t xs, uint8_t* c, int64_t cs, in
 
 // Thread blocks of the split kernel one SM holds for head dim D.
 int decode_blocks_per_sm(int D);
+// Warps per block of the split kernel for head dim D.
+int decode_warps_per_block(int D);
 // Dynamic shared memory of the split kernel for head dim D.
 int decode_smem_bytes(int D);
 

@@ -167,11 +167,11 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 }
 // Waits for phase `parity` of the barrier. Each poll lets the warp sleep in
 // the barrier for up to 20 us (the suspend-time hint) instead of spinning;
-// after 2^17 polls (about 2.6 s) it gives up and returns false, so a lost copy
-// can never hang the GPU.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// after `polls` polls (by default 2^17, about 2.6 s) it gives up and returns
+// false, so a lost copy can never hang the GPU.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int polls) {
 #pragma unroll 1
-  for (int it = 0; it < (1 << 17); ++it) {
+  for (int it = 0; it < polls; ++it) {
     uint32_t ok;
     asm volatile(
         "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 20000;\n"
@@ -271,6 +271,19 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
 #ifndef FP8PD_MIN_BLOCKS_D128
 #define FP8PD_MIN_BLOCKS_D128 4
 #endif
+#ifndef FP8PD_MIN_BLOCKS_D256
+#define FP8PD_MIN_BLOCKS_D256 2
+#endif
+// Warps per block (each streams its own tiles through its own ring).
+#ifndef FP8PD_NW_D64
+#define FP8PD_NW_D64 4
+#endif
+#ifndef FP8PD_NW_D128
+#define FP8PD_NW_D128 4
+#endif
+#ifndef FP8PD_NW_D256
+#define FP8PD_NW_D256 4
+#endif
 
 // ---------------------------------------------------------------------------
 // Shared-memory tile layout. The TMA writes one 16-token tile of one KV head
@@ -291,7 +304,8 @@ __device__ __forceinline__ uint32_t tile_off(int r, int b) {
 
 template <int D>
 struct Cfg {
-  static constexpr int NW = 4;                                        // warps per block
+  static constexpr int NW = (D == 64) ? FP8PD_NW_D64 : (D == 128) ? FP8PD_NW_D128 : (D == 256) ? FP8PD_NW_D256 : 4;  // warps per block
+  static constexpr int NT = NW * 32;                                  // threads per block
   static constexpr int NS = (D == 64) ? FP8PD_NS_D64 : (D == 128) ? FP8PD_NS_D128 : (D == 256) ? FP8PD_NS_D256 : FP8PD_NS_D512;  // ring stages per warp
   static constexpr bool PAIR = (D == 64) && FP8PD_PAIR_D64;           // two tiles per softmax step
   static constexpr int TILE = kTileTokens * D;                        // bytes of a K or V tile
@@ -305,7 +319,7 @@ struct Cfg {
   static constexpr int MISC_FLOATS = NW * 8 * 2 + 4;
   static constexpr int SMEM = 1024 /* alignment slack */ + PIPE_BYTES + QFRAG_BYTES + LIST_BYTES +
                               BAR_BYTES + MISC_FLOATS * 4;
-  static constexpr int MIN_BLOCKS = (D == 512) ? 1 : (D == 256) ? 2 : (D == 128) ? FP8PD_MIN_BLOCKS_D128 : FP8PD_MIN_BLOCKS_D64;
+  static constexpr int MIN_BLOCKS = (D == 512) ? 1 : (D == 256) ? FP8PD_MIN_BLOCKS_D256 : (D == 128) ? FP8PD_MIN_BLOCKS_D128 : FP8PD_MIN_BLOCKS_D64;
   static_assert(PIPE_BYTES % 1024 == 0, "tiles must stay 1024-byte aligned for the swizzle");
   static_assert(NW * 8 * D * 4 <= PIPE_BYTES, "merge scratch must fit in the ring");
   static_assert(8 * 32 * 4 <= PIPE_BYTES, "merge weights must fit in the ring");
@@ -1017,7 +1031,7 @@ __device__ bool prop_assign(const DecodeParams& p, int* scratch, int* red, int h
 // KV head, page), box (min(D,128), 16, max(1, D/128), 1, 1). TOK: the scales
 // are read per token (one per stored token and KV head) instead of per page.
 template <int D, bool KCVT, bool VCVT, bool TOK>
-__global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
+__global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
     decode_tma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
   using C = Cfg<D>;
@@ -1102,6 +1116,10 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
   // one TMA for K, one for V, both completing on the stage's barrier. A tile
   // whose page is out of range is not copied; its barrier phase still
   // completes.
+  // Test hook of the bounded waits (p.test_stall): warp 0 of the launch's
+  // first block posts the bytes of its first copy on the stage's barrier but
+  // issues no copy, so that wait, and only that one, runs out.
+  bool stall = p.test_stall && warp == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
   auto issue = [&](int e, int stage) {
     if (lane != 0) return;
     const uint32_t bar = wbar + 8 * stage;
@@ -1113,6 +1131,10 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     const uint32_t sk = wpipe + stage * C::STAGE;
     fence_proxy_async();  // this warp's earlier reads of the stage come first
     mbar_arrive_expect_tx(bar, 2 * C::TILE);
+    if (stall) {
+      stall = false;
+      return;
+    }
     tma_load_5d(sk, &tmk, bar, 0, slot0, 0, kvh, page);
     tma_load_5d(sk + C::TILE, &tmv, bar, 0, slot0, 0, kvh, page);
   };
@@ -1367,7 +1389,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     for (int j = 0; j + 1 < my_tiles; j += 2, tok0 += 2 * C::NW * kTileTokens) {
       const int st1 = (stage + 1 == C::NS) ? 0 : stage + 1;
       const uint32_t ph1 = (stage + 1 == C::NS) ? (phase ^ 1u) : phase;
-      if (!mbar_wait(wbar + 8 * stage, phase) || !mbar_wait(wbar + 8 * st1, ph1)) {
+      if (!mbar_wait(wbar + 8 * stage, phase, p.wait_polls) || !mbar_wait(wbar + 8 * st1, ph1, p.wait_polls)) {
         if (lane == 0) raise_flag(FP8PD_FLAG_TIMEOUT);
         ok_all = false;
         break;
@@ -1419,7 +1441,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
 #pragma unroll 1
   for (int j = (C::PAIR && !TOK) ? (my_tiles & ~1) : 0; ok_all && j < my_tiles;
        ++j, tok0 += C::NW * kTileTokens) {
-    if (!mbar_wait(wbar + 8 * stage, phase)) {
+    if (!mbar_wait(wbar + 8 * stage, phase, p.wait_polls)) {
       if (lane == 0) raise_flag(FP8PD_FLAG_TIMEOUT);
       ok_all = false;
       break;
@@ -1504,14 +1526,14 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     // A copy never completed: leave this warp's result out (its flag is set)
     // and wait, again bounded, for whatever this warp still has in flight.
     cp_async_wait_all();
-    for (int s = 0; s < C::NS; ++s) mbar_wait(wbar + 8 * s, phase ^ (s < stage ? 1u : 0u));
+    for (int s = 0; s < C::NS; ++s) mbar_wait(wbar + 8 * s, phase ^ (s < stage ? 1u : 0u), p.wait_polls);
     acc.m0 = acc.m1 = -CUDART_INF_F;
     acc.l0 = acc.l1 = 0.f;
   }
 
   // speculative copies past this warp's last tile (first use of their stage)
   if (spec)
-    for (int j = my_tiles; j < C::NS - 1; ++j) mbar_wait(wbar + 8 * j, 0);
+    for (int j = my_tiles; j < C::NS - 1; ++j) mbar_wait(wbar + 8 * j, 0, p.wait_polls);
 
   // ---- merge the warps ------------------------------------------------------
 #pragma unroll
@@ -1560,7 +1582,7 @@ __global__ void __launch_bounds__(128, Cfg<D>::MIN_BLOCKS)
     grow0 = ((int64_t)b * p.Hq + head0) * NG;
     cnt0 = ((int64_t)b * HX + blockIdx.x) * (1 + NG);
   }
-  for (int it = tid; it < 8 * (D / 4); it += 128) {
+  for (int it = tid; it < 8 * (D / 4); it += C::NT) {
     const int n = it / (D / 4);
     const int d = (it - n * (D / 4)) * 4;
     if (n >= nheads) continue;
@@ -1747,7 +1769,7 @@ static cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap& tmk
   }
   const dim3 grid = p.prop ? dim3(p.Hkv * p.head_groups, p.nbx, 1)
                            : dim3(p.Hkv * p.head_groups, p.B, p.num_splits);
-  decode_tma_kernel<D, KCVT, VCVT, TOK><<<grid, 128, smem, s>>>(p, tmk, tmv);
+  decode_tma_kernel<D, KCVT, VCVT, TOK><<<grid, Cfg<D>::NT, smem, s>>>(p, tmk, tmv);
   return cudaGetLastError();
 }
 
@@ -1788,7 +1810,7 @@ static int blocks_per_sm_d() {
   int n = 0;
   if (cudaFuncSetAttribute(decode_tma_kernel<D, true, true, false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tma_kernel<D, true, true, false>, 128,
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tma_kernel<D, true, true, false>, Cfg<D>::NT,
                                                     Cfg<D>::SMEM) != cudaSuccess) {
     cudaGetLastError();
     return Cfg<D>::MIN_BLOCKS;  // no device: do not cache the guess
@@ -1805,6 +1827,16 @@ int decode_blocks_per_sm(int D) {
     case 256: return blocks_per_sm_d<256>();
     case 512: return blocks_per_sm_d<512>();
     default: return 1;
+  }
+}
+
+int decode_warps_per_block(int D) {
+  switch (D) {
+    case 64: return Cfg<64>::NW;
+    case 128: return Cfg<128>::NW;
+    case 256: return Cfg<256>::NW;
+    case 512: return Cfg<512>::NW;
+    default: return 4;
   }
 }
 

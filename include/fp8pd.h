@@ -336,7 +336,15 @@ enum {
                                 is refused with FP8PD_ERR_ARG */
   FP8PD_OPT_K_DECODE = 3,    /* E4M3 -> f16 decode of K: 0 = bit assembly,
                                 1 = hardware cvt.rn.f16x2.e4m3x2 (default) */
-  FP8PD_OPT_V_DECODE = 4     /* the same for V (default 1) */
+  FP8PD_OPT_V_DECODE = 4,    /* the same for V (default 1) */
+  FP8PD_OPT_WAIT_POLLS = 6,  /* polls of a tile copy's barrier before the wait gives up and sets
+                                FP8PD_FLAG_TIMEOUT; each poll sleeps at most 20 us. Default
+                                131,072 (about 2.6 s); 1 .. 1,048,576 */
+  FP8PD_OPT_TEST_STALL = 7   /* test hook of the timeout path, 0 (default) or 1: warp 0 of the
+                                first block of each attention launch never issues its first tile
+                                copy, so that one wait runs out; the keys of that warp are left
+                                out and FP8PD_FLAG_TIMEOUT is set. No copy is in flight on the
+                                stalled stage, so the launch ends normally. */
 };
 int fp8pd_set_option(int32_t option, int64_t value);
 int64_t fp8pd_get_option(int32_t option);

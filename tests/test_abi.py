@@ -192,6 +192,15 @@ def test_options_roundtrip(F):
         with pytest.raises(F.Fp8pdError):
             F.fp8pd_set_option(F.OPT_SCHEDULE, bad)
     assert F.fp8pd_get_option(F.OPT_SCHEDULE) == 0
+    assert F.fp8pd_get_option(F.OPT_WAIT_POLLS) == 1 << 17
+    F.fp8pd_set_option(F.OPT_WAIT_POLLS, 64)
+    assert F.fp8pd_get_option(F.OPT_WAIT_POLLS) == 64
+    F.fp8pd_set_option(F.OPT_WAIT_POLLS, 1 << 17)
+    for opt, bad in ((F.OPT_WAIT_POLLS, 0), (F.OPT_WAIT_POLLS, (1 << 20) + 1),
+                     (F.OPT_TEST_STALL, 2), (F.OPT_TEST_STALL, -1)):
+        with pytest.raises(F.Fp8pdError):
+            F.fp8pd_set_option(opt, bad)
+    assert F.fp8pd_get_option(F.OPT_TEST_STALL) == 0
     with pytest.raises(F.Fp8pdError):
         F.fp8pd_set_option(99, 1)
     with pytest.raises(F.Fp8pdError):
