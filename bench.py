@@ -395,7 +395,7 @@ def _build_case(name: str, dev, args) -> W.Case:
 
 
 def _set_options(F, args) -> None:
-    F.fp8pd_set_option(F.OPT_K_DECODE, 1 if args.k_decode == "cvt" else 0)
+    F.fp8pd_set_option(F.OPT_K_DECODE, {"bits": 0, "cvt": 1, "mma8": 2}[args.k_decode])
     F.fp8pd_set_option(F.OPT_NUM_SPLITS, args.splits)
     F.fp8pd_set_option(F.OPT_SCHEDULE, args.schedule)
 
@@ -828,8 +828,9 @@ def build_parser() -> argparse.ArgumentParser:
     ap.add_argument("--unfused", action="store_true",
                     help="run fp8_kv_append and the attention call as two launches")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--k-decode", default="cvt", choices=["bits", "cvt"],
-                    help="E4M3 -> f16 decode of K: bit assembly or hardware cvt")
+    ap.add_argument("--k-decode", default="cvt", choices=["bits", "cvt", "mma8"],
+                    help="QK contraction: K decoded to f16 by bit assembly or the hardware cvt, "
+                         "or K's E4M3 bytes in E4M3 MMAs (mma8)")
     ap.add_argument("--splits", type=int, default=0, help="force a split count (0 = planner)")
     ap.add_argument("--scales", default="workload", choices=["workload", "token"],
                     help="token: per-token-per-head K/V scales instead of the workload's form")

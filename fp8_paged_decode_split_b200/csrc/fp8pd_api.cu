@@ -16,6 +16,11 @@
 #include "../../include/fp8pd.h"
 #include "fp8pd_internal.h"
 
+// L2 promotion of the pool tensor maps' tile loads (a build setting).
+#ifndef FP8PD_L2_PROMOTION
+#define FP8PD_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+#endif
+
 using fp8pd::AppendParams;
 using fp8pd::DecodeParams;
 
@@ -365,7 +370,7 @@ int make_pool_map(const fp8pd_tensor* pool, CUtensorMap* out) {
   const CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, pool->data, dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE,
                          D == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                         FP8PD_L2_PROMOTION, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail_cuda(cudaErrorInvalidValue);
   {
     std::lock_guard<std::mutex> lock(g_map_mutex);
@@ -592,9 +597,9 @@ void lay_out(const Plan& plan, void* ctr, void* part, DecodeParams* p) {
 
 cudaError_t launch_planned(const Plan& plan, const DecodeParams& p, const CUtensorMap& tmk,
                            const CUtensorMap& tmv, cudaStream_t s) {
-  const bool kc = g_opt_k_decode.load() == 1, vc = g_opt_v_decode.load() == 1;
   (void)plan;
-  return fp8pd::launch_decode(p, tmk, tmv, kc, vc, s);
+  return fp8pd::launch_decode(p, tmk, tmv, static_cast<int>(g_opt_k_decode.load()),
+                              g_opt_v_decode.load() == 1, s);
 }
 
 void record_run(const Plan& plan, int D) {
@@ -847,7 +852,7 @@ int fp8pd_set_option(int32_t option, int64_t value) {
       g_opt_schedule = value;
       return FP8PD_OK;
     case FP8PD_OPT_K_DECODE:
-      if (value < 0 || value > 1) return FP8PD_ERR_ARG;
+      if (value < 0 || value > 2) return FP8PD_ERR_ARG;
       g_opt_k_decode = value;
       return FP8PD_OK;
     case FP8PD_OPT_V_DECODE:

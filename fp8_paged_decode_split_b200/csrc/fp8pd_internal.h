@@ -91,8 +91,10 @@ struct AppendParams {
 
 // Launchers (defined with the kernels). Return a cudaError_t of the launch.
 // tmk / tmv: tensor maps over the K / V pool views (see make_pool_map).
+// k_mode: 0 / 1 = K decoded to f16 (bit assembly / hardware cvt) for f16
+// MMAs, 2 = E4M3 MMAs on K's bytes; v_cvt: V decoded by the hardware cvt.
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                          bool k_cvt, bool v_cvt, cudaStream_t s);
+                          int k_mode, bool v_cvt, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 // E4M3 codes (the append's rounding) of n float32 values; strides in elements.
 cudaError_t launch_encode(const float* x, int64_t xs, uint8_t* c, int64_t cs, int64_t n,

@@ -109,6 +109,19 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D[16x8] += A[16x32] * B[32x8], E4M3 inputs, f32 accumulate. A fragment:
+// a0 / a2 = row g, k = 4t .. 4t+3 / 16+4t .. 16+4t+3; a1 / a3 the same for
+// row g+8; B fragment: b0 / b1 = column g, k = 4t .. / 16+4t .. (g = lane /
+// 4, t = lane % 4, byte i of a register = element k + i).
+__device__ __forceinline__ void mma16832_e4m3(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -189,14 +202,27 @@ __device__ __forceinline__ void fence_barrier_init() {
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
-// 5-D tiled TMA load (no multicast) into this block's shared memory.
+// 5-D tiled TMA load (no multicast) into this block's shared memory. With
+// FP8PD_EVICT_FIRST (a build setting) the load carries an L2 evict-first
+// policy: K/V bytes are read once per step.
 __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0,
                                             int c1, int c2, int c3, int c4) {
+#ifdef FP8PD_EVICT_FIRST
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar),
+      "l"(pol)
+      : "memory");
+#else
   asm volatile(
       "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
       "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];\n" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar)
       : "memory");
+#endif
 }
 // 4-byte asynchronous copy global -> shared (no register round trip); the
 // issuing thread waits for all of its copies with cp_async_wait_all.
@@ -260,10 +286,10 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
 #define FP8PD_PAIR_D64 1
 #endif
 #ifndef FP8PD_NS_D256
-#define FP8PD_NS_D256 2
+#define FP8PD_NS_D256 3
 #endif
 #ifndef FP8PD_NS_D512
-#define FP8PD_NS_D512 2
+#define FP8PD_NS_D512 3
 #endif
 #ifndef FP8PD_MIN_BLOCKS_D64
 #define FP8PD_MIN_BLOCKS_D64 5
@@ -458,14 +484,28 @@ struct Acc {
 // is out of range, are -inf. kfa / kfb = score factors of tokens grp /
 // grp + 8 (equal unless the scales are per token); `full`:
 // every token is attended (warp-uniform). qfr(kb) gives the q' B-fragment
-// of k16 block kb.
-template <int D, bool KCVT, class QFrag>
+// of k16 block kb. KM selects the contraction: 0 / 1 = E4M3 decoded to f16 by
+// bit assembly / the hardware cvt, then f16 MMAs (m16n8k16); 2 = the E4M3
+// bytes themselves in E4M3 MMAs (m16n8k32), q' as two E4M3 terms (qfr(kb) =
+// (hi, lo) of the k16 block's four entries per lane), no conversion of K.
+template <int D, int KM, class QFrag>
 __device__ __forceinline__ float4 tile_scores(const QFrag& qfr, uint32_t sk,
                                               const uint32_t (&koff)[4], float kfa, float kfb,
                                               int tok0, int t0, int t1, bool page_ok, bool full,
                                               int grp) {
   // two independent accumulator chains
   float Sa[4] = {0.f, 0.f, 0.f, 0.f}, Sb[4] = {0.f, 0.f, 0.f, 0.f};
+  if constexpr (KM == 2) {
+    // the ldmatrix of a 32-byte block is the MMA's A fragment as is: rows g /
+    // g+8, bytes 4t.. (x / y) and 16+4t.. (z / w)
+#pragma unroll
+    for (int kc = 0; kc < D / 32; ++kc) {
+      const uint4 kw = ldsm_x4(sk + blk_off<D>(koff, kc));
+      const uint2 f0 = qfr(2 * kc), f1 = qfr(2 * kc + 1);
+      mma16832_e4m3(Sa, kw.x, kw.y, kw.z, kw.w, f0.x, f1.x);
+      mma16832_e4m3(Sb, kw.x, kw.y, kw.z, kw.w, f0.y, f1.y);
+    }
+  } else {
 #pragma unroll
   for (int kc = 0; kc < D / 32; ++kc) {
     // rows g / g+8, bytes 32kc + 4q.. (regs 0 / 1) and 32kc + 16 + 4q.. (2 / 3)
@@ -481,7 +521,7 @@ __device__ __forceinline__ float4 tile_scores(const QFrag& qfr, uint32_t sk,
         b1 = f.y;
       }
       uint32_t a0, a1, a2, a3;
-      if constexpr (KCVT) {
+      if constexpr (KM == 1) {
         a0 = e4m3x2_lo16_to_f16x2(wa);
         a1 = e4m3x2_lo16_to_f16x2(wb);
         a2 = e4m3x2_hi16_to_f16x2(wa);
@@ -498,6 +538,7 @@ __device__ __forceinline__ float4 tile_scores(const QFrag& qfr, uint32_t sk,
         mma16816(Sa, a0, a1, a2, a3, b0, b1);
     }
   }
+  }
   // A masked row may hold stale or NaN-decoded bytes: select, never multiply.
   const int ta = tok0 + grp, tb = ta + 8;
   const bool va = full || (page_ok && ta >= t0 && ta < t1);
@@ -513,7 +554,7 @@ __device__ __forceinline__ float4 tile_scores(const QFrag& qfr, uint32_t sk,
 // are scaled by the group's K scale of this lane's token rows grp / grp + 8
 // (ga[g] / gb[g], shared memory) and summed. kf = the score factor without
 // the K scale. Masking as tile_scores.
-template <int D, bool KCVT, class QFrag>
+template <int D, int KM, class QFrag>
 __device__ __forceinline__ float4 tile_scores_groups(const QFrag& qfr, uint32_t sk,
                                                      const uint32_t (&koff)[4], const float* ga,
                                                      const float* gb, int bpg_log2, float kf,
@@ -530,7 +571,8 @@ __device__ __forceinline__ float4 tile_scores_groups(const QFrag& qfr, uint32_t 
       const uint32_t wa = half ? kw.z : kw.x, wb = half ? kw.w : kw.y;
       const uint2 f = qfr(kb);
       uint32_t a0, a1, a2, a3;
-      if constexpr (KCVT) {
+      static_assert(KM != 2, "sub-row K groups use a 16-bit decode of K");
+      if constexpr (KM == 1) {
         a0 = e4m3x2_lo16_to_f16x2(wa);
         a1 = e4m3x2_lo16_to_f16x2(wb);
         a2 = e4m3x2_hi16_to_f16x2(wa);
@@ -681,14 +723,14 @@ __device__ __forceinline__ void tile_pv(Acc<D>& a, uint32_t sv, const uint32_t (
 // vsa / vsb = V scales of this lane's tokens grp / grp + 8, vabs = the
 // largest |V scale| of the tile's attended tokens; tok0 = first token of the
 // tile.
-template <int D, bool KCVT, bool VCVT, class QFrag>
+template <int D, int KM, bool VCVT, class QFrag>
 __device__ __forceinline__ void attend_tile(Acc<D>& a, const QFrag& qfr, uint32_t sk, uint32_t sv,
                                             const uint32_t (&koff)[4], const uint32_t (&voff)[4],
                                             float kfa, float kfb, float vsa, float vsb, float vabs,
                                             int tok0, int t0, int t1, bool page_ok, bool full,
                                             int grp, int qd) {
   const float4 sc =
-      tile_scores<D, KCVT>(qfr, sk, koff, kfa, kfb, tok0, t0, t1, page_ok, full, grp);
+      tile_scores<D, KM>(qfr, sk, koff, kfa, kfb, tok0, t0, t1, page_ok, full, grp);
   softmax_rescale<D>(a, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), vabs);
   uint32_t bh[2], bl[2];
   tile_probs<D>(a, sc, vsa, vsb, bh, bl);
@@ -698,7 +740,7 @@ __device__ __forceinline__ void attend_tile(Acc<D>& a, const QFrag& qfr, uint32_
 // Two tiles (u = 0, 1) at once: both score blocks, one softmax update (one
 // set of maximum shuffles and one rescale test for 32 keys), then both PV
 // blocks; `between` runs after the first tile's PV (its stage is free then).
-template <int D, bool KCVT, bool VCVT, class QFrag, class Between>
+template <int D, int KM, bool VCVT, class QFrag, class Between>
 __device__ __forceinline__ void attend_pair(Acc<D>& a, const QFrag& qfr, const uint32_t (&sk)[2],
                                             const uint32_t (&koff)[4], const uint32_t (&voff)[4],
                                             const float (&kfac)[2], const float (&vs)[2],
@@ -706,9 +748,9 @@ __device__ __forceinline__ void attend_pair(Acc<D>& a, const QFrag& qfr, const u
                                             const bool (&page_ok)[2], const bool (&full)[2],
                                             int grp, int qd, const Between& between) {
   constexpr int TILE = kTileTokens * D;
-  const float4 s0 = tile_scores<D, KCVT>(qfr, sk[0], koff, kfac[0], kfac[0], tok0[0], t0, t1,
+  const float4 s0 = tile_scores<D, KM>(qfr, sk[0], koff, kfac[0], kfac[0], tok0[0], t0, t1,
                                          page_ok[0], full[0], grp);
-  const float4 s1 = tile_scores<D, KCVT>(qfr, sk[1], koff, kfac[1], kfac[1], tok0[1], t0, t1,
+  const float4 s1 = tile_scores<D, KM>(qfr, sk[1], koff, kfac[1], kfac[1], tok0[1], t0, t1,
                                          page_ok[1], full[1], grp);
   softmax_rescale<D>(a, fmaxf(fmaxf(s0.x, s0.z), fmaxf(s1.x, s1.z)),
                      fmaxf(fmaxf(s0.y, s0.w), fmaxf(s1.y, s1.w)), fmaxf(fabsf(vs[0]), fabsf(vs[1])));
@@ -740,6 +782,20 @@ __device__ __forceinline__ uint16_t e4m3x2_rn_sat(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;  // low byte = lo, high byte = hi
+}
+
+// Two E4M3 terms of four values x (|x| < 256): hi = E4M3(x) (round to
+// nearest even), lo = E4M3(x - hi), one value per byte. A bf16 value whose
+// magnitude is at least 2^-2 splits exactly (its 8 significant bits are hi's
+// 4 and at most 4 more, above E4M3's smallest subnormal 2^-9); smaller ones
+// keep an error below 2^-10.
+__device__ __forceinline__ void e4m3_split4(float x0, float x1, float x2, float x3, uint32_t& hi,
+                                            uint32_t& lo) {
+  hi = (uint32_t)e4m3x2_rn_sat(x0, x1) | ((uint32_t)e4m3x2_rn_sat(x2, x3) << 16);
+  const float2 h01 = unpack_f16x2(e4m3x2_lo16_to_f16x2(hi));  // exact
+  const float2 h23 = unpack_f16x2(e4m3x2_hi16_to_f16x2(hi));
+  lo = (uint32_t)e4m3x2_rn_sat(x0 - h01.x, x1 - h01.y) |
+       ((uint32_t)e4m3x2_rn_sat(x2 - h23.x, x3 - h23.y) << 16);
 }
 
 // Per-token-per-head scale of one head's D values spread over a warp (PER
@@ -1023,14 +1079,16 @@ __device__ bool prop_assign(const DecodeParams& p, int* scratch, int* red, int h
   return has;
 }
 
-// One thread block: (split, KV head x head group, sequence). KCVT / VCVT
-// select the E4M3 -> f16 decode of K / V: false = bit assembly (value * 2^-8),
-// true = hardware cvt.rn.f16x2.e4m3x2 (the value itself). The q fragments
-// follow the K byte pairing. tmk / tmv: 5-D tensor maps over the K / V pool
+// One thread block: (split, KV head x head group, sequence). KM selects the
+// QK contraction: 0 = K decoded to f16 by bit assembly (value * 2^-8), 1 = by
+// the hardware cvt.rn.f16x2.e4m3x2 (the value itself), both into f16 MMAs;
+// 2 = K's E4M3 bytes straight into E4M3 MMAs with q as two E4M3 terms. VCVT
+// selects the E4M3 -> f16 decode of V (false = bit assembly, true = cvt). The
+// q fragments follow the K byte pairing. tmk / tmv: 5-D tensor maps over the K / V pool
 // views, dims (head-dim bytes within a 128-byte block, slot, 128-byte block,
 // KV head, page), box (min(D,128), 16, max(1, D/128), 1, 1). TOK: the scales
 // are read per token (one per stored token and KV head) instead of per page.
-template <int D, bool KCVT, bool VCVT, bool TOK>
+template <int D, int KM, bool VCVT, bool TOK>
 __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
     decode_tma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
@@ -1278,15 +1336,17 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
     qmax = warp_max(qmax);
   }
   // q' = q * 2^(15 - e) puts max|q'| in [2^14, 2^15): exact in f16 for every
-  // element above max|q| * 2^-28 (bf16 has 8 significant bits).
+  // element above max|q| * 2^-28 (bf16 has 8 significant bits). For the E4M3
+  // contraction q' = q * 2^(8 - e) puts it in [2^7, 2^8), below E4M3's 448,
+  // and every element above max|q| * 2^-10 splits exactly into two terms.
   int qe = 0;
   if (qmax > 0.f && isfinite(qmax)) frexpf(qmax, &qe);
   qe = max(qe, -111);
-  const float qmul = ldexpf(1.f, 15 - qe);
+  const float qmul = ldexpf(1.f, (KM == 2 ? 8 : 15) - qe);
   // kfac = sm_scale * log2(e) / qmul * k_scale(page), times 2^8 when K is
   // decoded by bit assembly (which yields value * 2^-8); the hardware cvt
-  // yields the value itself.
-  const float score_base = p.sm_scale_log2 * (KCVT ? 1.f : 256.f) / qmul;
+  // and the E4M3 MMA take the value itself.
+  const float score_base = p.sm_scale_log2 * (KM == 0 ? 256.f : 1.f) / qmul;
   uint32_t qf[C::Q_IN_SMEM ? 1 : KB][2];
 #pragma unroll
   for (int kb = 0; kb < KB; ++kb) {
@@ -1306,7 +1366,9 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
       x3 = __uint_as_float(v.y & 0xFFFF0000u);
     }
     uint32_t r0, r1;
-    if constexpr (KCVT) {
+    if constexpr (KM == 2) {
+      e4m3_split4(x0 * qmul, x1 * qmul, x2 * qmul, x3 * qmul, r0, r1);  // (hi, lo)
+    } else if constexpr (KM == 1) {
       r0 = pack_f16x2(x0 * qmul, x1 * qmul);
       r1 = pack_f16x2(x2 * qmul, x3 * qmul);
     } else {
@@ -1431,7 +1493,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
       } else {
         phase = ph1;
       }
-      attend_pair<D, KCVT, VCVT>(acc, qfr, sk, koff, voff, kfac, vsc, tk, t0, t1, pok, full, grp,
+      attend_pair<D, KM, VCVT>(acc, qfr, sk, koff, voff, kfac, vsc, tk, t0, t1, pok, full, grp,
                                  qd, [&]() {
                                    const int nj = j + C::NS;
                                    if (nj < my_tiles) issue(went[nj], st0);
@@ -1496,7 +1558,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
       const float vsb = __shfl_sync(0xffffffffu, tsc, 24 + grp);
       const float vabs = warp_max(lane >= 16 ? fabsf(tsc) : 0.f);
       if (kg > 1) {
-        const float4 sc = tile_scores_groups<D, KCVT>(
+        const float4 sc = tile_scores_groups<D, (KM == 0 ? 0 : 1)>(
             qfr, sk, koff, group_row(grp), group_row(grp + 8), kb_log2, score_base, tok0, t0, t1,
             page_ok, full, grp);
         softmax_rescale<D>(acc, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), vabs);
@@ -1506,7 +1568,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
       } else {
         const float kfa = score_base * __shfl_sync(0xffffffffu, tsc, grp);
         const float kfb = score_base * __shfl_sync(0xffffffffu, tsc, grp + 8);
-        attend_tile<D, KCVT, VCVT>(acc, qfr, sk, sv, koff, voff, kfa, kfb, vsa, vsb, vabs, tok0,
+        attend_tile<D, KM, VCVT>(acc, qfr, sk, sv, koff, voff, kfa, kfb, vsa, vsb, vabs, tok0,
                                    t0, t1, page_ok, full, grp, qd);
       }
     } else {
@@ -1518,7 +1580,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
                                    (went[j] & 15) * kTileTokens + r, r, sk, sv, ks, vs);
         __syncwarp();
       }
-      attend_tile<D, KCVT, VCVT>(acc, qfr, sk, sv, koff, voff, kfac, kfac, vs, vs, fabsf(vs), tok0,
+      attend_tile<D, KM, VCVT>(acc, qfr, sk, sv, koff, voff, kfac, kfac, vs, vs, fabsf(vs), tok0,
                                  t0, t1, page_ok, full, grp, qd);
     }
   }
@@ -1750,7 +1812,7 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
 // ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
-template <int D, bool KCVT, bool VCVT, bool TOK>
+template <int D, int KM, bool VCVT, bool TOK>
 static cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap& tmk,
                                    const CUtensorMap& tmv, cudaStream_t s) {
   // The shared-memory opt-in is a per-device function attribute: set it once
@@ -1762,42 +1824,48 @@ static cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap& tmk
   if (e != cudaSuccess) return e;
   const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
   if (!bit || !(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(decode_tma_kernel<D, KCVT, VCVT, TOK>,
+    e = cudaFuncSetAttribute(decode_tma_kernel<D, KM, VCVT, TOK>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
   const dim3 grid = p.prop ? dim3(p.Hkv * p.head_groups, p.nbx, 1)
                            : dim3(p.Hkv * p.head_groups, p.B, p.num_splits);
-  decode_tma_kernel<D, KCVT, VCVT, TOK><<<grid, Cfg<D>::NT, smem, s>>>(p, tmk, tmv);
+  decode_tma_kernel<D, KM, VCVT, TOK><<<grid, Cfg<D>::NT, smem, s>>>(p, tmk, tmv);
   return cudaGetLastError();
 }
 
+// K mode 2 (E4M3 MMAs) is built with the cvt decode of V and without
+// per-token scales; other combinations take mode 1 for K.
 template <int D, bool TOK>
 static cudaError_t launch_decode_kv(const DecodeParams& p, const CUtensorMap& tmk,
-                                   const CUtensorMap& tmv, bool k_cvt, bool v_cvt, cudaStream_t s) {
-  if (k_cvt)
-    return v_cvt ? launch_decode_d<D, true, true, TOK>(p, tmk, tmv, s)
-                 : launch_decode_d<D, true, false, TOK>(p, tmk, tmv, s);
-  return v_cvt ? launch_decode_d<D, false, true, TOK>(p, tmk, tmv, s)
-               : launch_decode_d<D, false, false, TOK>(p, tmk, tmv, s);
+                                    const CUtensorMap& tmv, int k_mode, bool v_cvt,
+                                    cudaStream_t s) {
+  if constexpr (!TOK) {
+    if (k_mode == 2 && v_cvt) return launch_decode_d<D, 2, true, false>(p, tmk, tmv, s);
+  }
+  if (k_mode >= 1)
+    return v_cvt ? launch_decode_d<D, 1, true, TOK>(p, tmk, tmv, s)
+                 : launch_decode_d<D, 1, false, TOK>(p, tmk, tmv, s);
+  return v_cvt ? launch_decode_d<D, 0, true, TOK>(p, tmk, tmv, s)
+               : launch_decode_d<D, 0, false, TOK>(p, tmk, tmv, s);
 }
 
 template <int D>
 static cudaError_t launch_decode_dt(const DecodeParams& p, const CUtensorMap& tmk,
-                                    const CUtensorMap& tmv, bool k_cvt, bool v_cvt,
+                                    const CUtensorMap& tmv, int k_mode, bool v_cvt,
                                     cudaStream_t s) {
-  if (p.k_tok || p.v_tok) return launch_decode_kv<D, true>(p, tmk, tmv, k_cvt, v_cvt, s);
-  return launch_decode_kv<D, false>(p, tmk, tmv, k_cvt, v_cvt, s);
+  if (p.k_tok || p.v_tok) return launch_decode_kv<D, true>(p, tmk, tmv, k_mode, v_cvt, s);
+  return launch_decode_kv<D, false>(p, tmk, tmv, k_mode, v_cvt, s);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                          bool k_cvt, bool v_cvt, cudaStream_t s) {
+                          int k_mode, bool v_cvt, cudaStream_t s) {
   switch (p.D) {
-    case 64: return launch_decode_dt<64>(p, tmk, tmv, k_cvt, v_cvt, s);
-    case 128: return launch_decode_dt<128>(p, tmk, tmv, k_cvt, v_cvt, s);
-    case 256: return launch_decode_dt<256>(p, tmk, tmv, k_cvt, v_cvt, s);
-    case 512: return launch_decode_dt<512>(p, tmk, tmv, k_cvt, v_cvt, s);
+    case 64: return launch_decode_dt<64>(p, tmk, tmv, k_mode, v_cvt, s);
+    case 128: return launch_decode_dt<128>(p, tmk, tmv, k_mode, v_cvt, s);
+    case 256: return launch_decode_dt<256>(p, tmk, tmv, k_mode, v_cvt, s);
+    case 512: return launch_decode_dt<512>(p, tmk, tmv, k_mode, v_cvt, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1808,9 +1876,9 @@ static int blocks_per_sm_d() {
   int c = cached.load();
   if (c >= 0) return c;
   int n = 0;
-  if (cudaFuncSetAttribute(decode_tma_kernel<D, true, true, false>,
+  if (cudaFuncSetAttribute(decode_tma_kernel<D, 1, true, false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tma_kernel<D, true, true, false>, Cfg<D>::NT,
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tma_kernel<D, 1, true, false>, Cfg<D>::NT,
                                                     Cfg<D>::SMEM) != cudaSuccess) {
     cudaGetLastError();
     return Cfg<D>::MIN_BLOCKS;  // no device: do not cache the guess

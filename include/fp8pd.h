@@ -334,8 +334,11 @@ enum {
                                 3 = proportional splits where they apply (B <= 1024, no
                                 forced split count), else uniform splits; any other value
                                 is refused with FP8PD_ERR_ARG */
-  FP8PD_OPT_K_DECODE = 3,    /* E4M3 -> f16 decode of K: 0 = bit assembly,
-                                1 = hardware cvt.rn.f16x2.e4m3x2 (default) */
+  FP8PD_OPT_K_DECODE = 3,    /* the QK contraction: 0 = K decoded to f16 by bit assembly,
+                                1 = by the hardware cvt.rn.f16x2.e4m3x2 (both into f16 MMAs),
+                                2 = K's E4M3 bytes into E4M3 MMAs, q as two exact E4M3 terms
+                                (no decode of K); mode 2 applies with the cvt decode of V and
+                                page or head scales, mode 1 runs otherwise. Default 1. */
   FP8PD_OPT_V_DECODE = 4,    /* the same for V (default 1) */
   FP8PD_OPT_WAIT_POLLS = 6,  /* polls of a tile copy's barrier before the wait gives up and sets
                                 FP8PD_FLAG_TIMEOUT; each poll sleeps at most 20 us. Default

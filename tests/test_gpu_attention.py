@@ -34,10 +34,10 @@ def schedule(F, request):
     F.fp8pd_set_option(F.OPT_SCHEDULE, 0)
 
 
-@pytest.fixture(params=[(1, 1), (0, 0)], ids=["cvt", "bits"])
+@pytest.fixture(params=[(1, 1), (0, 0), (2, 1)], ids=["cvt", "bits", "mma8"])
 def kdecode(F, request):
     """Run a test with each E4M3 -> f16 decode of K and V (hardware cvt, bit
-    assembly)."""
+    assembly), and with K's E4M3 bytes in E4M3 MMAs (V by the cvt)."""
     F.fp8pd_set_option(F.OPT_K_DECODE, request.param[0])
     F.fp8pd_set_option(F.OPT_V_DECODE, request.param[1])
     yield request.param

@@ -29,7 +29,7 @@ def schedule(F, request):
     F.fp8pd_set_option(F.OPT_SCHEDULE, 0)
 
 
-@pytest.fixture(params=[(1, 1), (0, 0), (0, 1)], ids=["cvt", "bits", "kbits-vcvt"])
+@pytest.fixture(params=[(1, 1), (0, 0), (0, 1), (2, 1)], ids=["cvt", "bits", "kbits-vcvt", "mma8"])
 def kdecode(F, request):
     F.fp8pd_set_option(F.OPT_K_DECODE, request.param[0])
     F.fp8pd_set_option(F.OPT_V_DECODE, request.param[1])
