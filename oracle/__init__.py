@@ -13,6 +13,8 @@ from .fp8pd_oracle import (  # noqa: F401
     e4m3_code_value,
     e4m3_decode,
     e4m3_encode,
+    e4m3_round,
+    fp8_compute_query,
     expand_groups,
     gather_tokens,
     group_scale,

@@ -42,6 +42,13 @@ Readings of the pages (each is listed with its reason in the design notes):
   groups (P1 "Supported scope", ``k_groups``) add a last axis of ``groups``
   scales, group g covering entries [g D/groups, (g+1) D/groups).
 * empty attention (no keys, no sink) returns 0.
+* the opt-in "fp8 compute" path (P1 "Two compute paths", ``compute="fp8"``,
+  and "Limitations": it adds one E4M3 rounding on q and on p) rounds each
+  query row to E4M3 after a power-of-two scale that puts its largest
+  magnitude in [2^7, 2^8), and each softmax weight p_t = exp(s_t - M_s)
+  taken against the largest score M_s (at most 1) to E4M3 as p_t * 2^8, in
+  the weighted sum of values only; the denominator sums the unrounded
+  weights and the sink's exp(sink - M_s).
 """
 
 from __future__ import annotations
@@ -240,9 +247,28 @@ def attended_range(seq_len: int, window: int) -> tuple[int, int]:
     return lo, L
 
 
+def e4m3_round(x) -> np.ndarray:
+    """x rounded to the nearest E4M3 value (ties to an even mantissa,
+    saturating to +-448), as float64."""
+    return e4m3_decode(e4m3_encode(x))
+
+
+def fp8_compute_query(q_row) -> np.ndarray:
+    """One E4M3 rounding of a query row (the fp8 compute path): scaled by
+    2^k so that its largest magnitude lies in [2^7, 2^8), rounded, scaled
+    back. A zero row stays zero."""
+    q_row = np.asarray(q_row, dtype=np.float64)
+    amax = float(np.max(np.abs(q_row))) if q_row.size else 0.0
+    if amax == 0.0 or not math.isfinite(amax):
+        return q_row.copy()
+    _, e = math.frexp(amax)                 # amax in [2^(e-1), 2^e)
+    k = 8 - e
+    return e4m3_round(q_row * 2.0 ** k) * 2.0 ** -k
+
+
 def paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens,
                            window: int = 0, sinks=None, sm_scale: float | None = None,
-                           batch_heads=None) -> np.ndarray:
+                           batch_heads=None, compute: str = "f32") -> np.ndarray:
     """Single-query attention over a paged E4M3 KV cache, float64.
 
     q [B, Hq, D] (bf16 values given as floats), k_pages / v_pages
@@ -262,7 +288,15 @@ def paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_table, s
 
     ``batch_heads``: optional list of (b, hq) pairs; only those outputs are
     computed (the others stay 0), for sampled checks at full size.
+
+    ``compute="fp8"`` is P1's fp8 compute path: q is replaced by
+    :func:`fp8_compute_query` of its row, the weights are taken against the
+    largest score, w_t = exp(s_t - max_t s_t), and in the numerator each is
+    replaced by E4M3(w_t * 2^8) / 2^8; the denominator is
+    sum_t w_t + exp(sink - max_t s_t).
     """
+    if compute not in ("f32", "fp8"):
+        raise ValueError(compute)
     q = np.asarray(q, dtype=np.float64)
     B, Hq, D = q.shape
     Hkv = k_pages.shape[2]
@@ -288,16 +322,20 @@ def paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_table, s
             K = _dequantize(kc, k_scale, phys, slots, h)
             V = _dequantize(vc, v_scale, phys, slots, h)
             for hq in heads:
-                s = sm * (K @ q[b, hq])
+                qrow = fp8_compute_query(q[b, hq]) if compute == "fp8" else q[b, hq]
+                s = sm * (K @ qrow)
                 sink = None if sinks is None else float(sinks[hq])
                 m_keys = s.max() if s.size else -math.inf
                 M = m_keys if sink is None else max(m_keys, sink)
+                if compute == "fp8" and s.size:
+                    M = m_keys  # the rounded weights are taken against the largest score
                 if M == -math.inf:
                     continue                       # no keys and no finite sink: 0
                 w = np.exp(s - M)
                 den = w.sum() + (0.0 if sink is None else math.exp(sink - M))
+                wv = e4m3_round(w * 2.0 ** 8) * 2.0 ** -8 if compute == "fp8" else w
                 if den > 0.0:
-                    out[b, hq] = (w @ V) / den
+                    out[b, hq] = (wv @ V) / den
     return out
 
 

@@ -852,3 +852,95 @@ def test_window_of_all_but_one_drops_key_zero():
         b = _run(trimmed, window=0, sinks=sk, sm_scale=0.2)
         assert np.allclose(a, b, rtol=1e-13, atol=1e-16)
         assert not np.allclose(a, _run(full, window=0, sinks=sk, sm_scale=0.2), rtol=1e-6, atol=0)
+
+
+# ------------------------------------------------- fp8 compute path (opt-in)
+# The solution page's "Two compute paths" table and "Limitations": the fp8
+# path adds one E4M3 rounding on q and one on p, and is held to 1.5e-1.
+
+def _torch_e4m3(x) -> np.ndarray:
+    return torch.tensor(np.asarray(x, dtype=np.float64)).float().to(torch.float8_e4m3fn) \
+        .double().numpy()
+
+
+def test_fp8_query_rounding_matches_library_float8():
+    rng = np.random.default_rng(51)
+    for trial in range(200):
+        row = rng.standard_normal(64) * 10.0 ** rng.uniform(-6, 6)
+        row = torch.tensor(row).to(torch.bfloat16).double().numpy()
+        amax = np.abs(row).max()
+        k = 7 - math.floor(math.log2(amax))           # 2^7 <= amax * 2^k < 2^8
+        assert 128 <= amax * 2.0 ** k < 256
+        want = _torch_e4m3(row * 2.0 ** k) * 2.0 ** -k
+        assert np.array_equal(O.fp8_compute_query(row), want)
+    assert np.array_equal(O.fp8_compute_query(np.zeros(8)), np.zeros(8))
+
+
+def test_fp8_compute_equals_f32_where_nothing_rounds():
+    """q = 0 (every weight is exactly 1), a single key (one weight of 1, the
+    value alone) and W = 1 give the f32 result exactly."""
+    rng = np.random.default_rng(52)
+    c = _dense_case(rng, scale_mode="page")
+    c0 = dict(c, q=np.zeros_like(c["q"]))
+    sinks = np.linspace(-1, 1, 8).astype(np.float32)     # above and below the scores
+    for kw in (dict(window=0), dict(window=9, sinks=sinks)):
+        assert np.allclose(_run(c0, compute="fp8", **kw), _run(c0, **kw), rtol=1e-14, atol=1e-16)
+    c1 = dict(c, lens=np.array([1, 1]))
+    assert np.array_equal(_run(c1, compute="fp8"), _run(c1))
+    assert np.array_equal(_run(c, window=1, compute="fp8"), _run(c, window=1))
+
+
+def test_fp8_compute_brute_force_tiny_inputs():
+    """Pure-Python softmax with the two roundings done by the library float8
+    type: q per row after the power-of-two scale, each weight as w * 2^8."""
+    rng = np.random.default_rng(53)
+    for trial in range(20):
+        D = int(rng.integers(1, 9))
+        L = int(rng.integers(2, 9))
+        c = _dense_case(rng, B=1, Hq=2, Hkv=1, D=D, ps=16, L=(L,), scale_mode="page")
+        sinks = rng.standard_normal(2).astype(np.float32) if trial % 2 else None
+        sm = float(np.float32(rng.uniform(0.05, 0.5)))
+        got = _run(c, sinks=sinks, sm_scale=sm, compute="fp8")
+        for hq in range(2):
+            row = c["q"][0, hq]
+            amax = float(np.abs(row).max())
+            k = 7 - math.floor(math.log2(amax))
+            qr = [float(x) for x in _torch_e4m3(row * 2.0 ** k) * 2.0 ** -k]
+            s = []
+            vals = []
+            for t in range(L):
+                p = int(c["table"][0][t // 16])
+                kv = [e4m3(int(c["k"][p, t % 16, 0, d])) * float(c["ks"][p, 0]) for d in range(D)]
+                vals.append([e4m3(int(c["v"][p, t % 16, 0, d])) * float(c["vs"][p, 0]) for d in range(D)])
+                s.append(sm * sum(qr[d] * kv[d] for d in range(D)))
+            M = max(s)                              # weights against the largest score
+            w = [math.exp(x - M) for x in s]
+            den = sum(w) + (0.0 if sinks is None else math.exp(float(sinks[hq]) - M))
+            wr = [float(_torch_e4m3([x * 256.0])[0]) / 256.0 for x in w]
+            want = [sum(wr[t] * vals[t][d] for t in range(L)) / den for d in range(D)]
+            assert np.allclose(got[0, hq], want, rtol=1e-12, atol=1e-14)
+
+
+def test_fp8_compute_stays_within_the_pages_tolerance_of_f32():
+    """Serving-like data (K and V drawn N(0,1), quantized with amax / 448
+    scales per KV head, q N(0,1) in bf16, sm_scale = D^-0.5): the fp8 path
+    is within the page's 1.5e-1 of the f32 path, and differs from it."""
+    rng = np.random.default_rng(54)
+    for D, L, window, with_sinks in ((64, 300, 0, True), (128, 173, 40, False), (128, 1000, 0, False)):
+        B, Hq, Hkv, ps = 2, 8, 2, 16
+        npg = (L + ps - 1) // ps
+        x = rng.standard_normal((2, B * npg, ps, Hkv, D))
+        amax = np.abs(x).max(axis=(1, 2, 4))                       # [2, Hkv]
+        sc = (amax / 448.0).astype(np.float32)
+        k = O.quantize(x[0], sc[0][None, None, :, None])
+        v = O.quantize(x[1], sc[1][None, None, :, None])
+        table = rng.permutation(B * npg).astype(np.int32).reshape(B, npg)
+        q = torch.randn(B, Hq, D, generator=torch.Generator().manual_seed(7)).to(torch.bfloat16)
+        c = dict(q=q.double().numpy(), k=k, v=v, ks=sc[0], vs=sc[1], table=table,
+                 lens=np.array([L, L - 7]))
+        sinks = rng.standard_normal(Hq).astype(np.float32) if with_sinks else None
+        f32 = _run(c, window=window, sinks=sinks, sm_scale=D ** -0.5)
+        f8 = _run(c, window=window, sinks=sinks, sm_scale=D ** -0.5, compute="fp8")
+        err = np.abs(f8 - f32) / np.maximum(1.0, np.abs(f32))
+        assert err.max() <= 1.5e-1, err.max()
+        assert err.max() > 0.0                      # the roundings do change the result
