@@ -398,6 +398,7 @@ def _set_options(F, args) -> None:
     F.fp8pd_set_option(F.OPT_K_DECODE, {"bits": 0, "cvt": 1, "mma8": 2}[args.k_decode])
     F.fp8pd_set_option(F.OPT_NUM_SPLITS, args.splits)
     F.fp8pd_set_option(F.OPT_SCHEDULE, args.schedule)
+    F.fp8pd_set_option(F.OPT_COMPUTE, 1 if args.compute == "fp8" else 0)
 
 
 def run_ours(args) -> dict | None:
@@ -468,7 +469,9 @@ def run_ours(args) -> dict | None:
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "e4m3 cache; f16 tensor-core MMA, f32 accumulate",
+        "dtype": ("e4m3 cache; f16 tensor-core MMA, f32 accumulate" if args.compute == "f32" else
+                  "e4m3 cache; fp8 compute: q and P rounded to e4m3, e4m3 tensor-core MMA, "
+                  "f32 accumulate"),
         "data": "synthetic (seeded), no dataset",
         "config": _config_dict(args, args.config, nbytes=nbytes),
         "timing": "device time of CUDA-graph replays of the step (per-step events); "
@@ -836,6 +839,9 @@ def build_parser() -> argparse.ArgumentParser:
                     help="token: per-token-per-head K/V scales instead of the workload's form")
     ap.add_argument("--k-groups", type=int, default=1,
                     help="with --scales token: K scales per sub-row group of D / k_groups entries")
+    ap.add_argument("--compute", default="f32", choices=["f32", "fp8"],
+                    help="numerical path: f32 (default, 1e-3) or the opt-in fp8 compute path "
+                         "(q and P rounded once to E4M3; 1.5e-1)")
     ap.add_argument("--schedule", type=int, default=0, choices=[0, 1, 3],
                     help="0 = planner, 1 = uniform splits, 3 = proportional splits")
     return ap

@@ -30,9 +30,10 @@ __all__ = [
     "fp8pd_plan", "fp8pd_reserve_workspace", "fp8pd_e4m3_encode",
     "fp8pd_check_errors", "fp8pd_set_option", "fp8pd_get_option", "fp8pd_last_run_info",
     "fp8pd_timing_enable", "fp8pd_timing_collect", "Fp8pdError", "lib", "LIB_PATH",
+    "fp8_paged_decode_attention_partial", "fp8pd_combine_partials",
     "FLAG_PAGE_OOB", "FLAG_SEQLEN_OOB", "FLAG_POS_OOB", "FLAG_INTERNAL", "OPT_NUM_SPLITS",
     "OPT_SCHEDULE", "OPT_K_DECODE", "OPT_V_DECODE", "OPT_WAIT_POLLS",
-    "OPT_TEST_STALL", "FLAG_TIMEOUT",
+    "OPT_TEST_STALL", "OPT_COMPUTE", "FLAG_TIMEOUT",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libfp8pd.so")
@@ -40,7 +41,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "lib
 DTYPE_U8, DTYPE_I32, DTYPE_F32, DTYPE_BF16 = 1, 2, 3, 4
 FLAG_PAGE_OOB, FLAG_SEQLEN_OOB, FLAG_POS_OOB, FLAG_INTERNAL, FLAG_TIMEOUT = 1, 2, 4, 8, 16
 OPT_NUM_SPLITS, OPT_SCHEDULE, OPT_K_DECODE, OPT_V_DECODE = 1, 2, 3, 4
-OPT_WAIT_POLLS, OPT_TEST_STALL = 6, 7
+OPT_WAIT_POLLS, OPT_TEST_STALL, OPT_COMPUTE = 6, 7, 8
 _DTYPES = {torch.uint8: DTYPE_U8, torch.int32: DTYPE_I32, torch.float32: DTYPE_F32,
            torch.bfloat16: DTYPE_BF16}
 
@@ -66,7 +67,7 @@ class RunInfo(ctypes.Structure):
                 ("head_groups", ctypes.c_int32), ("grid_blocks", ctypes.c_int32),
                 ("combine", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("calls", ctypes.c_int64), ("appends", ctypes.c_int64),
-                ("kernel_launches", ctypes.c_int64)]
+                ("kernel_launches", ctypes.c_int64), ("compute", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -81,6 +82,8 @@ def _load() -> ctypes.CDLL:
     lib.fp8_paged_decode_attention.argtypes = [T, T, T, T, T, T, T, i32, T, f32, T, vp]
     lib.fp8_paged_decode_attention_noalloc.argtypes = [T, T, T, T, T, T, T, i32, T, f32, T, vp]
     lib.fp8_kv_append.argtypes = [T, T, T, T, P(Scales), T, T, vp]
+    lib.fp8_paged_decode_attention_partial.argtypes = [T, T, T, T, T, T, T, T, i32, f32, T, T, vp]
+    lib.fp8pd_combine_partials.argtypes = [T, T, T, T, vp]
     lib.fp8_paged_decode_append_attention.argtypes = [T, T, T, T, T, T, T, T, T, i32, T, f32, T, vp]
     lib.fp8pd_plan.argtypes = [T, T, T, i32, P(PlanInfo)]
     lib.fp8pd_reserve_workspace.argtypes = [ctypes.c_uint64]
@@ -204,6 +207,45 @@ def fp8_paged_decode_attention_noalloc(q, k_pages, v_pages, k_scale, v_scale, bl
                                                 _ref(ds_sinks), float(sm_scale), _ref(ds_out),
                                                 _stream(stream, q))
     _check(st, "fp8_paged_decode_attention_noalloc")
+    return out
+
+
+def fp8_paged_decode_attention_partial(q, k_pages, v_pages, k_scale, v_scale, block_table,
+                                       seq_lens, key_ranges=None, window: int = 0,
+                                       sm_scale: float | None = None, part_o=None, part_ml=None,
+                                       stream=None):
+    """Unnormalized decode attention over the keys [key_ranges[b, 0],
+    key_ranges[b, 1]) of each sequence's window (all of it when key_ranges is
+    None), for context-parallel split-KV. Returns (part_o [B, Hq, D],
+    part_ml [B, Hq, 2]): the numerator, and the maximum score in log2 units
+    with its sum of exponentials; no sink (fp8pd_combine_partials adds it)."""
+    if sm_scale is None:
+        sm_scale = q.shape[-1] ** -0.5
+    if part_o is None:
+        part_o = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    if part_ml is None:
+        part_ml = torch.empty(q.shape[0], q.shape[1], 2, dtype=torch.float32, device=q.device)
+    _same_device(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens, key_ranges,
+                 part_o, part_ml)
+    ds = [describe(t) for t in (q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens,
+                                key_ranges)]
+    d_o, d_ml = describe(part_o), describe(part_ml)
+    st = lib.fp8_paged_decode_attention_partial(*[_ref(d) for d in ds], int(window),
+                                                float(sm_scale), _ref(d_o), _ref(d_ml),
+                                                _stream(stream, q))
+    _check(st, "fp8_paged_decode_attention_partial")
+    return part_o, part_ml
+
+
+def fp8pd_combine_partials(part_o, part_ml, sinks=None, out=None, stream=None) -> torch.Tensor:
+    """Merges R partial results (part_o [R, B, Hq, D], part_ml [R, B, Hq, 2])
+    into the attention output [B, Hq, D], adding the sink once."""
+    if out is None:
+        out = torch.empty(part_o.shape[1:], dtype=torch.float32, device=part_o.device)
+    _same_device(part_o, part_ml, sinks, out)
+    d = [describe(t) for t in (part_o, part_ml, sinks, out)]
+    st = lib.fp8pd_combine_partials(*[_ref(x) for x in d], _stream(stream, part_o))
+    _check(st, "fp8pd_combine_partials")
     return out
 
 

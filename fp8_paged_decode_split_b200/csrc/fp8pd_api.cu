@@ -32,7 +32,7 @@ thread_local int32_t t_last_cuda_error = 0;
 thread_local fp8pd_run_info t_run_info = {};
 std::atomic<int64_t> g_calls{0}, g_appends{0}, g_launches{0};
 std::atomic<int64_t> g_opt_num_splits{0}, g_opt_schedule{0}, g_opt_k_decode{1}, g_opt_v_decode{1},
-    g_opt_wait_polls{1 << 17}, g_opt_test_stall{0};
+    g_opt_wait_polls{1 << 17}, g_opt_test_stall{0}, g_opt_compute{0};
 
 struct Workspace {
   void* ptr = nullptr;
@@ -598,8 +598,8 @@ void lay_out(const Plan& plan, void* ctr, void* part, DecodeParams* p) {
 cudaError_t launch_planned(const Plan& plan, const DecodeParams& p, const CUtensorMap& tmk,
                            const CUtensorMap& tmv, cudaStream_t s) {
   (void)plan;
-  return fp8pd::launch_decode(p, tmk, tmv, static_cast<int>(g_opt_k_decode.load()),
-                              g_opt_v_decode.load() == 1, s);
+  const int k_mode = g_opt_compute.load() == 1 ? 3 : static_cast<int>(g_opt_k_decode.load());
+  return fp8pd::launch_decode(p, tmk, tmv, k_mode, g_opt_v_decode.load() == 1, s);
 }
 
 void record_run(const Plan& plan, int D) {
@@ -609,6 +609,7 @@ void record_run(const Plan& plan, int D) {
   t_run_info.grid_blocks = plan.grid_blocks;
   t_run_info.combine = plan.combine;
   t_run_info.head_dim = D;
+  t_run_info.compute = static_cast<int32_t>(g_opt_compute.load());
 }
 
 }  // namespace
@@ -619,6 +620,8 @@ namespace {
 // validated decode-attention call.
 int run_decode(DecodeParams& p, const DecodeArgs& a, const fp8pd_tensor* k_pages,
                const fp8pd_tensor* v_pages, int32_t window, fp8pd_stream_t stream) {
+  // the fp8 compute path takes page and head scales only: refused, never downgraded
+  if (g_opt_compute.load() == 1 && (p.k_tok || p.v_tok)) return FP8PD_ERR_UNSUPPORTED;
   Plan plan;
   int r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
   if (r) return r;
@@ -659,6 +662,85 @@ int fp8_paged_decode_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_page
   if (r) return r;
   if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
   return run_decode(p, a, k_pages, v_pages, window, stream);
+}
+
+namespace {
+bool contiguous(const fp8pd_tensor* t) {
+  int64_t st = 1;
+  for (int i = t->ndim - 1; i >= 0; --i) {
+    if (t->shape[i] > 1 && t->stride[i] != st) return false;
+    st *= t->shape[i];
+  }
+  return true;
+}
+}  // namespace
+
+int fp8_paged_decode_attention_partial(const fp8pd_tensor* q, const fp8pd_tensor* k_pages,
+                                       const fp8pd_tensor* v_pages, const fp8pd_tensor* k_scale,
+                                       const fp8pd_tensor* v_scale,
+                                       const fp8pd_tensor* block_table,
+                                       const fp8pd_tensor* seq_lens,
+                                       const fp8pd_tensor* key_ranges, int32_t window,
+                                       float sm_scale, fp8pd_tensor* part_o,
+                                       fp8pd_tensor* part_ml, fp8pd_stream_t stream) {
+  DecodeParams p;
+  DecodeArgs a;
+  int r = validate_decode(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens, window,
+                          nullptr, sm_scale, part_o, &p, &a);
+  if (r) return r;
+  if (!contiguous(part_o)) return FP8PD_ERR_ALIGN;
+  if ((r = check(part_ml, FP8PD_DTYPE_F32, 3))) return r;
+  if (part_ml->shape[0] != a.B || part_ml->shape[1] != a.Hq || part_ml->shape[2] != 2)
+    return FP8PD_ERR_SHAPE;
+  if (!contiguous(part_ml) || reinterpret_cast<uintptr_t>(part_ml->data) % 8) return FP8PD_ERR_ALIGN;
+  if (key_ranges) {
+    if ((r = check(key_ranges, FP8PD_DTYPE_I32, 2))) return r;
+    if (key_ranges->shape[0] != a.B || key_ranges->shape[1] != 2) return FP8PD_ERR_SHAPE;
+    p.kr = static_cast<const int32_t*>(key_ranges->data);
+    p.kr_sb = key_ranges->stride[0];
+    p.kr_s1 = key_ranges->stride[1];
+  }
+  p.pout_o = static_cast<float*>(part_o->data);
+  p.pout_ml = static_cast<float*>(part_ml->data);
+  if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
+  return run_decode(p, a, k_pages, v_pages, window, stream);
+}
+
+int fp8pd_combine_partials(const fp8pd_tensor* part_o, const fp8pd_tensor* part_ml,
+                           const fp8pd_tensor* sinks, fp8pd_tensor* out, fp8pd_stream_t stream) {
+  int r;
+  if ((r = check(part_o, FP8PD_DTYPE_F32, 4))) return r;
+  if ((r = check(part_ml, FP8PD_DTYPE_F32, 4))) return r;
+  if ((r = check(out, FP8PD_DTYPE_F32, 3))) return r;
+  const int64_t R = part_o->shape[0], B = part_o->shape[1], Hq = part_o->shape[2],
+                D = part_o->shape[3];
+  if (part_ml->shape[0] != R || part_ml->shape[1] != B || part_ml->shape[2] != Hq ||
+      part_ml->shape[3] != 2)
+    return FP8PD_ERR_SHAPE;
+  if (out->shape[0] != B || out->shape[1] != Hq || out->shape[2] != D) return FP8PD_ERR_SHAPE;
+  if (R < 1 || R > 1024) return FP8PD_ERR_TOO_LARGE;
+  if (D % 4) return FP8PD_ERR_UNSUPPORTED;
+  if (!contiguous(part_o) || !contiguous(part_ml) ||
+      reinterpret_cast<uintptr_t>(part_o->data) % 16 || reinterpret_cast<uintptr_t>(part_ml->data) % 8)
+    return FP8PD_ERR_ALIGN;
+  if (out->stride[2] != 1 || reinterpret_cast<uintptr_t>(out->data) % 16 || out->stride[0] % 4 ||
+      out->stride[1] % 4)
+    return FP8PD_ERR_ALIGN;
+  if (sinks) {
+    if ((r = check(sinks, FP8PD_DTYPE_F32, 1))) return r;
+    if (sinks->shape[0] != Hq) return FP8PD_ERR_SHAPE;
+  }
+  if (!fits_i32(B) || !fits_i32(Hq) || !fits_i32(D) || B * Hq > INT32_MAX) return FP8PD_ERR_TOO_LARGE;
+  if (B == 0 || Hq == 0 || D == 0) return FP8PD_OK;
+  const cudaError_t e = fp8pd::launch_combine(
+      static_cast<const float*>(part_o->data), static_cast<const float*>(part_ml->data),
+      static_cast<int>(R), static_cast<int>(B), static_cast<int>(Hq), static_cast<int>(D),
+      sinks ? static_cast<const float*>(sinks->data) : nullptr, sinks ? sinks->stride[0] : 0,
+      static_cast<float*>(out->data), out->stride[0], out->stride[1],
+      reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e);
+  ++g_launches;
+  return FP8PD_OK;
 }
 
 int fp8_paged_decode_append_attention(const fp8pd_tensor* q, const fp8pd_tensor* k_new,
@@ -867,6 +949,10 @@ int fp8pd_set_option(int32_t option, int64_t value) {
       if (value < 0 || value > 1) return FP8PD_ERR_ARG;
       g_opt_test_stall = value;
       return FP8PD_OK;
+    case FP8PD_OPT_COMPUTE:
+      if (value < 0 || value > 1) return FP8PD_ERR_ARG;
+      g_opt_compute = value;
+      return FP8PD_OK;
     default:
       return FP8PD_ERR_ARG;
   }
@@ -880,6 +966,7 @@ int64_t fp8pd_get_option(int32_t option) {
     case FP8PD_OPT_V_DECODE: return g_opt_v_decode.load();
     case FP8PD_OPT_WAIT_POLLS: return g_opt_wait_polls.load();
     case FP8PD_OPT_TEST_STALL: return g_opt_test_stall.load();
+    case FP8PD_OPT_COMPUTE: return g_opt_compute.load();
     default: return -1;
   }
 }
@@ -993,6 +1080,7 @@ extern "C" int fp8_paged_decode_attention_noalloc(
                           sinks, sm_scale, out, &p, &a);
   if (r) return r;
   if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
+  if (g_opt_compute.load() == 1 && (p.k_tok || p.v_tok)) return FP8PD_ERR_UNSUPPORTED;
   Plan plan;
   r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
   if (r) return r;

@@ -52,6 +52,14 @@ struct DecodeParams {
   // first copy (the timeout path's test hook).
   int wait_polls;
   int test_stall;
+  // Context-parallel slices: kr (int32 [B, 2], or nullptr) cuts each
+  // sequence's attended keys to [kr[b][0], kr[b][1]); with pout_o set, each
+  // (sequence, query head) is written unnormalized to pout_o [B * Hq, D] and
+  // (m, l) to pout_ml [B * Hq, 2] (m in log2 units, no sink) instead of out.
+  const int32_t* kr;
+  int64_t kr_sb, kr_s1;
+  float* pout_o;
+  float* pout_ml;
   // Fused append (split kernel only): `lens` holds positions; sequence b
   // attends over positions[b] + 1 keys, the last of them the new token
   // (kn, vn: bf16 [B, Hkv, D]), which the block holding it quantizes, stores
@@ -92,10 +100,17 @@ struct AppendParams {
 // Launchers (defined with the kernels). Return a cudaError_t of the launch.
 // tmk / tmv: tensor maps over the K / V pool views (see make_pool_map).
 // k_mode: 0 / 1 = K decoded to f16 (bit assembly / hardware cvt) for f16
-// MMAs, 2 = E4M3 MMAs on K's bytes; v_cvt: V decoded by the hardware cvt.
+// MMAs, 2 = E4M3 MMAs on K's bytes, 3 = the fp8 compute path (q and P
+// rounded once to E4M3, E4M3 MMAs on K's and V's bytes); v_cvt: V decoded by
+// the hardware cvt.
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                           int k_mode, bool v_cvt, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+// Merge of R partial results (O, m, l) per (sequence, query head) into out,
+// adding the sink once: po [R][BH][D], pml [R][BH][2] contiguous, BH = B * Hq.
+cudaError_t launch_combine(const float* po, const float* pml, int R, int B, int Hq, int D,
+                           const float* sinks, int64_t sinks_s, float* out, int64_t o_sb,
+                           int64_t o_sh, cudaStream_t s);
 // E4M3 codes (the append's rounding) of n float32 values; strides in elements.
 cudaError_t launch_encode(const float* x, int64_t xs, uint8_t* c, int64_t cs, int64_t n,
                           cudaStream_t s);

@@ -152,6 +152,13 @@ __device__ __forceinline__ uint32_t e4m3x2_hi16_to_f16x2(uint32_t w) {
   return r;
 }
 
+// E4M3 codes of two f32 values: round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint16_t e4m3x2_rn_sat(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;  // low byte = lo, high byte = hi
+}
+
 __device__ __forceinline__ float4 ldcg4(const float* p) {
   float4 v;
   asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];\n"
@@ -492,10 +499,20 @@ template <int D, int KM, class QFrag>
 __device__ __forceinline__ float4 tile_scores(const QFrag& qfr, uint32_t sk,
                                               const uint32_t (&koff)[4], float kfa, float kfb,
                                               int tok0, int t0, int t1, bool page_ok, bool full,
-                                              int grp) {
+                                              int grp, float2 hf = make_float2(1.f, 1.f)) {
   // two independent accumulator chains
   float Sa[4] = {0.f, 0.f, 0.f, 0.f}, Sb[4] = {0.f, 0.f, 0.f, 0.f};
-  if constexpr (KM == 2) {
+  if constexpr (KM == 3) {
+    // fp8 compute: q' as one E4M3 term (qfr(kb).x), per-head factors hf of
+    // this lane's heads 2qd / 2qd + 1; the two k32 blocks' chains alternate
+#pragma unroll
+    for (int kc = 0; kc < D / 32; ++kc) {
+      const uint4 kw = ldsm_x4(sk + blk_off<D>(koff, kc));
+      const uint2 f0 = qfr(2 * kc), f1 = qfr(2 * kc + 1);
+      if (kc & 1) mma16832_e4m3(Sb, kw.x, kw.y, kw.z, kw.w, f0.x, f1.x);
+      else mma16832_e4m3(Sa, kw.x, kw.y, kw.z, kw.w, f0.x, f1.x);
+    }
+  } else if constexpr (KM == 2) {
     // the ldmatrix of a 32-byte block is the MMA's A fragment as is: rows g /
     // g+8, bytes 4t.. (x / y) and 16+4t.. (z / w)
 #pragma unroll
@@ -543,6 +560,12 @@ __device__ __forceinline__ float4 tile_scores(const QFrag& qfr, uint32_t sk,
   const int ta = tok0 + grp, tb = ta + 8;
   const bool va = full || (page_ok && ta >= t0 && ta < t1);
   const bool vb = full || (page_ok && tb >= t0 && tb < t1);
+  if constexpr (KM == 3) {
+    return make_float4(va ? (Sa[0] + Sb[0]) * (kfa * hf.x) : -CUDART_INF_F,
+                       va ? (Sa[1] + Sb[1]) * (kfa * hf.y) : -CUDART_INF_F,
+                       vb ? (Sa[2] + Sb[2]) * (kfb * hf.x) : -CUDART_INF_F,
+                       vb ? (Sa[3] + Sb[3]) * (kfb * hf.y) : -CUDART_INF_F);
+  }
   return make_float4(va ? (Sa[0] + Sb[0]) * kfa : -CUDART_INF_F,
                      va ? (Sa[1] + Sb[1]) * kfa : -CUDART_INF_F,
                      vb ? (Sa[2] + Sb[2]) * kfb : -CUDART_INF_F,
@@ -717,6 +740,88 @@ __device__ __forceinline__ void tile_pv(Acc<D>& a, uint32_t sv, const uint32_t (
   }
 }
 
+// ---------------------------------------------------------------------------
+// The fp8 compute path (opt-in; the solution page's compute="fp8"): P is
+// rounded once to E4M3 and multiplies V's E4M3 bytes in E4M3 MMAs
+// (m16n8k32), so neither K nor V is decoded. The MMA's 32 k-entries are 32
+// tokens: this lane's k = 4t .. 4t+3 are tokens 2t, 2t+1, 2t+8, 2t+9 of the
+// first tile and k = 16 + 4t .. those of the second (zero for a single tile).
+// ---------------------------------------------------------------------------
+
+// f16x2 -> E4M3x2 of values already on the E4M3 grid (exact).
+__device__ __forceinline__ uint32_t f16x2_to_e4m3x2(uint32_t h) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(h));
+  return r;
+}
+
+// P of one tile for the fp8 path: exp2 of the scores against the running
+// maxima, added to the running sums (unrounded), then P * v_scale / vref *
+// 2^8 rounded once to E4M3 (from f32), moved to the PV B layout through
+// movmatrix as exact f16 values: returns this lane's bytes [p(2t), p(2t+1),
+// p(2t+8), p(2t+9)] of head g = lane / 4.
+template <int D>
+__device__ __forceinline__ uint32_t tile_probs8(Acc<D>& a, float4 sc, float vsa, float vsb) {
+  const float mb0 = (a.m0 == -CUDART_INF_F) ? 0.f : a.m0;
+  const float mb1 = (a.m1 == -CUDART_INF_F) ? 0.f : a.m1;
+  const float p00 = fast_exp2(sc.x - mb0), p01 = fast_exp2(sc.y - mb1);
+  const float p10 = fast_exp2(sc.z - mb0), p11 = fast_exp2(sc.w - mb1);
+  a.l0 += p00 + p10;
+  a.l1 += p01 + p11;
+  const float vra = vsa * a.inv_vref * 256.f, vrb = vsb * a.inv_vref * 256.f;
+  const uint32_t ea = e4m3x2_rn_sat(p00 * vra, p01 * vra);  // token g, heads 2t, 2t+1
+  const uint32_t eb = e4m3x2_rn_sat(p10 * vrb, p11 * vrb);  // token g + 8
+  const uint32_t ha = movmatrix_trans(e4m3x2_lo16_to_f16x2(ea));  // head g, tokens 2t, 2t+1
+  const uint32_t hb = movmatrix_trans(e4m3x2_lo16_to_f16x2(eb));  // head g, tokens 2t+8, 2t+9
+  return f16x2_to_e4m3x2(ha) | (f16x2_to_e4m3x2(hb) << 16);
+}
+
+// This lane's token bytes of a transposed V block for the fp8 path: from the
+// ldmatrix.trans words (bytes [t.d, t.d+1, t'.d, t'.d+1] of tokens 2t, 2t+1
+// in lo and 2t+8, 2t+9 in hi), the bytes of head-dim entry d (even = false)
+// or d + 1 (true) of tokens 2t, 2t+1, 2t+8, 2t+9.
+__device__ __forceinline__ uint32_t v_tokens4(uint32_t lo, uint32_t hi, bool odd) {
+  return prmt(lo, hi, odd ? 0x7531u : 0x6420u);
+}
+
+// Byte mask of this lane's tokens 2t, 2t+1, 2t+8, 2t+9 of a tile (0 for a
+// masked token: its V bytes may be NaN codes, and NaN * 0 is NaN).
+__device__ __forceinline__ uint32_t tok_mask4(int tok0, int t0, int t1, bool page_ok, bool full,
+                                              int qd) {
+  if (full) return ~0u;
+  const int r = tok0 + 2 * qd;
+  auto in = [&](int t) { return page_ok && t >= t0 && t < t1; };
+  return (in(r) ? 0xFFu : 0u) | (in(r + 1) ? 0xFF00u : 0u) | (in(r + 8) ? 0xFF0000u : 0u) |
+         (in(r + 9) ? 0xFF000000u : 0u);
+}
+
+// O^T[d][head] += V^T P for one or two tiles (V at sv[u], P bytes pb[u]) in
+// E4M3 MMAs; the accumulator rows are those of tile_pv (d / d+1 of 32-byte
+// block jb, and d + 16 / d + 17), so the epilogue is shared.
+template <int D, int NT>
+__device__ __forceinline__ void tile_pv8(Acc<D>& a, const uint32_t (&sv)[2], const uint32_t (&voff)[4],
+                                         const uint32_t (&pb)[2], const uint32_t (&vm)[2]) {
+#pragma unroll
+  for (int jb = 0; jb < D / 32; ++jb) {
+    uint32_t e[2][4];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (u < NT) {
+        const uint4 vw = ldsm_x4_trans(sv[u] + blk_off<D>(voff, jb));
+        e[u][0] = v_tokens4(vw.x, vw.z, false) & vm[u];  // entry d
+        e[u][1] = v_tokens4(vw.x, vw.z, true) & vm[u];   // d + 1
+        e[u][2] = v_tokens4(vw.y, vw.w, false) & vm[u];  // d + 16
+        e[u][3] = v_tokens4(vw.y, vw.w, true) & vm[u];   // d + 17
+      } else {
+        e[u][0] = e[u][1] = e[u][2] = e[u][3] = 0u;
+      }
+    }
+    const uint32_t b1 = NT > 1 ? pb[1] : 0u;
+    mma16832_e4m3(a.O[jb][0], e[0][0], e[0][1], e[1][0], e[1][1], pb[0], b1);
+    mma16832_e4m3(a.O[jb][1], e[0][2], e[0][3], e[1][2], e[1][3], pb[0], b1);
+  }
+}
+
 // Attends one 16-token tile already in shared memory (K at sk, V at sv) for
 // one warp: S = K q'^T, masking, the online-softmax update, and O += V^T P
 // with P as an f16 hi + lo pair. kfa / kfb = score factors (log2 units) and
@@ -728,13 +833,20 @@ __device__ __forceinline__ void attend_tile(Acc<D>& a, const QFrag& qfr, uint32_
                                             const uint32_t (&koff)[4], const uint32_t (&voff)[4],
                                             float kfa, float kfb, float vsa, float vsb, float vabs,
                                             int tok0, int t0, int t1, bool page_ok, bool full,
-                                            int grp, int qd) {
+                                            int grp, int qd, float2 hf = make_float2(1.f, 1.f)) {
   const float4 sc =
-      tile_scores<D, KM>(qfr, sk, koff, kfa, kfb, tok0, t0, t1, page_ok, full, grp);
+      tile_scores<D, KM>(qfr, sk, koff, kfa, kfb, tok0, t0, t1, page_ok, full, grp, hf);
   softmax_rescale<D>(a, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), vabs);
-  uint32_t bh[2], bl[2];
-  tile_probs<D>(a, sc, vsa, vsb, bh, bl);
-  tile_pv<D, VCVT>(a, sv, voff, bh, bl, tok0, t0, t1, page_ok, full, qd);
+  if constexpr (KM == 3) {
+    const uint32_t pb[2] = {tile_probs8<D>(a, sc, vsa, vsb), 0u};
+    const uint32_t svv[2] = {sv, sv};
+    const uint32_t vm[2] = {tok_mask4(tok0, t0, t1, page_ok, full, qd), 0u};
+    tile_pv8<D, 1>(a, svv, voff, pb, vm);
+  } else {
+    uint32_t bh[2], bl[2];
+    tile_probs<D>(a, sc, vsa, vsb, bh, bl);
+    tile_pv<D, VCVT>(a, sv, voff, bh, bl, tok0, t0, t1, page_ok, full, qd);
+  }
 }
 
 // Two tiles (u = 0, 1) at once: both score blocks, one softmax update (one
@@ -746,14 +858,25 @@ __device__ __forceinline__ void attend_pair(Acc<D>& a, const QFrag& qfr, const u
                                             const float (&kfac)[2], const float (&vs)[2],
                                             const int (&tok0)[2], int t0, int t1,
                                             const bool (&page_ok)[2], const bool (&full)[2],
-                                            int grp, int qd, const Between& between) {
+                                            int grp, int qd, const Between& between,
+                                            float2 hf = make_float2(1.f, 1.f)) {
   constexpr int TILE = kTileTokens * D;
   const float4 s0 = tile_scores<D, KM>(qfr, sk[0], koff, kfac[0], kfac[0], tok0[0], t0, t1,
-                                         page_ok[0], full[0], grp);
+                                         page_ok[0], full[0], grp, hf);
   const float4 s1 = tile_scores<D, KM>(qfr, sk[1], koff, kfac[1], kfac[1], tok0[1], t0, t1,
-                                         page_ok[1], full[1], grp);
+                                         page_ok[1], full[1], grp, hf);
   softmax_rescale<D>(a, fmaxf(fmaxf(s0.x, s0.z), fmaxf(s1.x, s1.z)),
                      fmaxf(fmaxf(s0.y, s0.w), fmaxf(s1.y, s1.w)), fmaxf(fabsf(vs[0]), fabsf(vs[1])));
+  if constexpr (KM == 3) {
+    // one k32 MMA per 32-byte block covers both tiles' tokens
+    const uint32_t pb[2] = {tile_probs8<D>(a, s0, vs[0], vs[0]), tile_probs8<D>(a, s1, vs[1], vs[1])};
+    const uint32_t svv[2] = {sk[0] + TILE, sk[1] + TILE};
+    const uint32_t vm[2] = {tok_mask4(tok0[0], t0, t1, page_ok[0], full[0], qd),
+                            tok_mask4(tok0[1], t0, t1, page_ok[1], full[1], qd)};
+    tile_pv8<D, 2>(a, svv, voff, pb, vm);
+    between();
+    return;
+  }
   uint32_t bh0[2], bl0[2], bh1[2], bl1[2];
   tile_probs<D>(a, s0, vs[0], vs[0], bh0, bl0);
   tile_probs<D>(a, s1, vs[1], vs[1], bh1, bl1);
@@ -777,12 +900,29 @@ __device__ __forceinline__ int attended_keys(const DecodeParams& p, int b, bool 
   return 0;
 }
 
-// E4M3 codes of two f32 values: round to nearest even, saturating to +-448.
-__device__ __forceinline__ uint16_t e4m3x2_rn_sat(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;  // low byte = lo, high byte = hi
+// The keys [lo, hi) sequence b attends, of its L: the window's range, cut to
+// the sequence's key range [begin, end) when the call has one (a context-
+// parallel slice).
+__device__ __forceinline__ void key_range(const DecodeParams& p, int b, int L, int& lo, int& hi) {
+  lo = p.window > 0 ? max(0, L - p.window) : 0;
+  hi = L;
+  if (p.kr) {
+    lo = max(lo, __ldg(p.kr + (int64_t)b * p.kr_sb));
+    hi = min(hi, __ldg(p.kr + (int64_t)b * p.kr_sb + p.kr_s1));
+    hi = max(hi, lo);
+  }
 }
+
+// Unnormalized result of one (sequence, query head) in partial-output mode
+// (the context-parallel slices): O = sum_t 2^(s2_t - m) v_t, m = max_t s2_t
+// (log2 units: the scaled score times log2 e), l = sum_t 2^(s2_t - m); no sink.
+__device__ __forceinline__ void store_partial(const DecodeParams& p, int b, int head, int d,
+                                              float4 o, float m, float l) {
+  const int64_t row = (int64_t)b * p.Hq + head;
+  *reinterpret_cast<float4*>(p.pout_o + row * p.D + d) = o;
+  if (d == 0) *reinterpret_cast<float2*>(p.pout_ml + row * 2) = make_float2(m, l);
+}
+
 
 // Two E4M3 terms of four values x (|x| < 256): hi = E4M3(x) (round to
 // nearest even), lo = E4M3(x - hi), one value per byte. A bf16 value whose
@@ -930,8 +1070,9 @@ __device__ bool prop_assign(const DecodeParams& p, int* scratch, int* red, int h
   int tsum = 0, tmax = 0, tcnt = 0;
   for (int bb = tid; bb < B; bb += NT) {
     const int L = attended_keys(p, bb, blockIdx.x == 0 && blockIdx.y == 0);
-    const int lo = p.window > 0 ? max(0, L - p.window) : 0;
-    const int nt = L > lo ? (L - 1) / kTileTokens - lo / kTileTokens + 1 : 0;
+    int lo, hi;
+    key_range(p, bb, L, lo, hi);
+    const int nt = hi > lo ? (hi - 1) / kTileTokens - lo / kTileTokens + 1 : 0;
     s_nt[bb] = nt;
     tsum += nt;
     tmax = max(tmax, nt);
@@ -1055,8 +1196,16 @@ __device__ bool prop_assign(const DecodeParams& p, int* scratch, int* red, int h
   const int k = blockIdx.y;
   for (int bb = k; bb < B; bb += p.nbx) {
     if (s_nt[bb] != 0) continue;
-    for (int e = tid; e < nheads * p.D; e += NT)
-      p.out[(int64_t)bb * p.o_sb + (int64_t)(head0 + e / p.D) * p.o_sh + (e % p.D)] = 0.f;
+    for (int e = tid; e < nheads * p.D; e += NT) {
+      if (p.pout_o) {
+        const int64_t row = (int64_t)bb * p.Hq + head0 + e / p.D;
+        p.pout_o[row * p.D + (e % p.D)] = 0.f;
+        if (e % p.D == 0) *reinterpret_cast<float2*>(p.pout_ml + row * 2) =
+            make_float2(-CUDART_INF_F, 0.f);
+      } else {
+        p.out[(int64_t)bb * p.o_sb + (int64_t)(head0 + e / p.D) * p.o_sh + (e % p.D)] = 0.f;
+      }
+    }
   }
   const bool has = k < s_sp[B];
   if (has) {
@@ -1202,7 +1351,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
   // before the block exits; a page id outside the pool is never copied.
   // (Proportional splits know their range by now: they build the tile list
   // first and copy from it, which saves a second block-table round trip.)
-  const bool spec = p.window == 0 && !p.prop;
+  const bool spec = p.window == 0 && !p.prop && !p.kr;
   if (spec) {
     const int tf = p.prop ? prop_j0 : split * p.chunk_pages * (p.ps / kTileTokens);
     int e = -1;
@@ -1223,18 +1372,19 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
   // of its attended range: equal-sized work per block whatever the length,
   // and the blocks past the end of a short sequence have nothing to do.
   const int L = attended_keys(p, b, tid == 0 && split == 0 && blockIdx.x == 0);
-  const int lo = p.window > 0 ? max(0, L - p.window) : 0;
+  int lo, hi;  // the attended keys of the sequence
+  key_range(p, b, L, lo, hi);
   int t0, t1;
   if (p.prop) {
     t0 = max(lo, (lo / kTileTokens + prop_j0) * kTileTokens);
-    t1 = min(L, (lo / kTileTokens + prop_j1) * kTileTokens);
+    t1 = min(hi, (lo / kTileTokens + prop_j1) * kTileTokens);
   } else {
     const int first_page = lo / p.ps;
-    const int n_pages = (L > lo) ? (L - 1) / p.ps - first_page + 1 : 0;
+    const int n_pages = (hi > lo) ? (hi - 1) / p.ps - first_page + 1 : 0;
     const int pg0 = first_page + split * p.chunk_pages;
     const int pg1 = min(first_page + n_pages, pg0 + p.chunk_pages);
     t0 = max(lo, pg0 * p.ps);
-    t1 = min(L, pg1 * p.ps);
+    t1 = min(hi, pg1 * p.ps);
   }
   const int tile_first = t0 / kTileTokens;
   const int n_tiles = (t1 > t0) ? (t1 + kTileTokens - 1) / kTileTokens - tile_first : 0;
@@ -1325,15 +1475,31 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
       qfrag_s[kb * 32 + lane] = v;
       qmax = fmaxf(qmax, max4(v));
     }
-    qmax = warp_max(qmax);
-    if (lane == 0) misc[warp] = qmax;  // free until the warps merge
-    __syncthreads();
+    if constexpr (KM == 3) {
+      // fp8 compute: one maximum per query head (this lane's head g lives in
+      // lanes 4g .. 4g+3 of every warp)
+      qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, 1));
+      qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, 2));
+      if (qd == 0) misc[warp * 8 + grp] = qmax;  // free until the warps merge
+      __syncthreads();
 #pragma unroll
-    for (int w = 0; w < C::NW; ++w) qmax = fmaxf(qmax, misc[w]);
+      for (int w = 0; w < C::NW; ++w) qmax = fmaxf(qmax, misc[w * 8 + grp]);
+    } else {
+      qmax = warp_max(qmax);
+      if (lane == 0) misc[warp] = qmax;  // free until the warps merge
+      __syncthreads();
+#pragma unroll
+      for (int w = 0; w < C::NW; ++w) qmax = fmaxf(qmax, misc[w]);
+    }
   } else {
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb) qmax = fmaxf(qmax, max4(qraw[kb]));
-    qmax = warp_max(qmax);
+    if constexpr (KM == 3) {
+      qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, 1));
+      qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, 2));
+    } else {
+      qmax = warp_max(qmax);
+    }
   }
   // q' = q * 2^(15 - e) puts max|q'| in [2^14, 2^15): exact in f16 for every
   // element above max|q| * 2^-28 (bf16 has 8 significant bits). For the E4M3
@@ -1342,11 +1508,18 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
   int qe = 0;
   if (qmax > 0.f && isfinite(qmax)) frexpf(qmax, &qe);
   qe = max(qe, -111);
-  const float qmul = ldexpf(1.f, (KM == 2 ? 8 : 15) - qe);
+  const float qmul = ldexpf(1.f, (KM >= 2 ? 8 : 15) - qe);
   // kfac = sm_scale * log2(e) / qmul * k_scale(page), times 2^8 when K is
   // decoded by bit assembly (which yields value * 2^-8); the hardware cvt
-  // and the E4M3 MMA take the value itself.
-  const float score_base = p.sm_scale_log2 * (KM == 0 ? 256.f : 1.f) / qmul;
+  // and the E4M3 MMA take the value itself. The fp8 compute path scales each
+  // query head by its own power of two: its factors hf (of this lane's score
+  // heads 2qd and 2qd + 1) stay out of score_base.
+  const float score_base = p.sm_scale_log2 * (KM == 0 ? 256.f : 1.f) / (KM == 3 ? 1.f : qmul);
+  float2 hf = make_float2(1.f, 1.f);
+  if constexpr (KM == 3) {
+    const float inv = 1.f / qmul;  // a power of two: exact
+    hf = make_float2(__shfl_sync(0xffffffffu, inv, 8 * qd), __shfl_sync(0xffffffffu, inv, 8 * qd + 4));
+  }
   uint32_t qf[C::Q_IN_SMEM ? 1 : KB][2];
 #pragma unroll
   for (int kb = 0; kb < KB; ++kb) {
@@ -1366,7 +1539,12 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
       x3 = __uint_as_float(v.y & 0xFFFF0000u);
     }
     uint32_t r0, r1;
-    if constexpr (KM == 2) {
+    if constexpr (KM == 3) {
+      // one E4M3 rounding of q (the fp8 compute path)
+      r0 = (uint32_t)e4m3x2_rn_sat(x0 * qmul, x1 * qmul) |
+           ((uint32_t)e4m3x2_rn_sat(x2 * qmul, x3 * qmul) << 16);
+      r1 = 0u;
+    } else if constexpr (KM == 2) {
       e4m3_split4(x0 * qmul, x1 * qmul, x2 * qmul, x3 * qmul, r0, r1);  // (hi, lo)
     } else if constexpr (KM == 1) {
       r0 = pack_f16x2(x0 * qmul, x1 * qmul);
@@ -1444,7 +1622,8 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
   int stage = 0;
   uint32_t phase = 0;
   int tok0 = (tile_first + warp) * kTileTokens;
-  if constexpr (C::PAIR && !TOK) {
+  constexpr bool PAIRS = C::PAIR || KM == 3;  // two tiles per softmax step
+  if constexpr (PAIRS && !TOK) {
     // Two tiles per step while two are left (one softmax update per 32 keys;
     // the copy into the first tile's stage is issued once its PV is done).
 #pragma unroll 1
@@ -1497,11 +1676,11 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
                                  qd, [&]() {
                                    const int nj = j + C::NS;
                                    if (nj < my_tiles) issue(went[nj], st0);
-                                 });
+                                 }, hf);
     }
   }
 #pragma unroll 1
-  for (int j = (C::PAIR && !TOK) ? (my_tiles & ~1) : 0; ok_all && j < my_tiles;
+  for (int j = (PAIRS && !TOK) ? (my_tiles & ~1) : 0; ok_all && j < my_tiles;
        ++j, tok0 += C::NW * kTileTokens) {
     if (!mbar_wait(wbar + 8 * stage, phase, p.wait_polls)) {
       if (lane == 0) raise_flag(FP8PD_FLAG_TIMEOUT);
@@ -1581,7 +1760,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
         __syncwarp();
       }
       attend_tile<D, KM, VCVT>(acc, qfr, sk, sv, koff, voff, kfac, kfac, vs, vs, fabsf(vs), tok0,
-                                 t0, t1, page_ok, full, grp, qd);
+                                 t0, t1, page_ok, full, grp, qd, hf);
     }
   }
   if (!ok_all) {
@@ -1607,7 +1786,8 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
   float* Os = reinterpret_cast<float*>(pipe);  // [NW][8][D], already times fold
   float* ml = misc;                            // [NW][8][2]
   // f16 offset of the decoded V (bit assembly only), times the V reference scale
-  const float fold = ok_all ? (VCVT ? 1.f : 256.f) * acc.vref : 0.f;
+  const float fold = !ok_all ? 0.f : KM == 3 ? acc.vref * (1.f / 256.f)
+                                              : (VCVT ? 1.f : 256.f) * acc.vref;
 #pragma unroll
   for (int jb = 0; jb < D / 32; ++jb) {
     const int d = 32 * jb + 2 * grp;
@@ -1667,7 +1847,9 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
       }
     }
     const int head = head0 + n;
-    if (S == 1) {
+    if (S == 1 && p.pout_o) {
+      store_partial(p, b, head, d, acc, M, l);
+    } else if (S == 1) {
       const float sl = p.sinks ? p.sinks[(int64_t)head * p.sinks_s] * kLog2e : -CUDART_INF_F;
       const float M2 = fmaxf(M, sl);
       float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1710,9 +1892,14 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
   if (!*flag) return;
   __threadfence();
   float* wts = reinterpret_cast<float*>(pipe);  // [8][32] merge weights
+  // partial-output mode: the final merges write (O, m, l) rows, no sink
+  const bool fin = p.pout_o == nullptr;
+  float* fml = fin ? nullptr : p.pout_ml;
+  float* fo = fin ? nullptr : p.pout_o;
+  const int64_t frow = (int64_t)b * p.Hq + head0;
   if (NG == 1) {
-    merge_partials<D, C::NW>(p.part_ml, p.part_o, prow0, S, S, nheads, true, p, b, head0,
-                             nullptr, nullptr, 0, 0, wts);
+    merge_partials<D, C::NW>(p.part_ml, p.part_o, prow0, S, S, nheads, fin, p, b, head0,
+                             fml, fo, frow, 1, wts);
     if (tid == 0) ucnt[1] = 0;
     return;
   }
@@ -1727,8 +1914,8 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
   __syncthreads();
   if (!*flag) return;
   __threadfence();
-  merge_partials<D, C::NW>(p.grp_ml, p.grp_o, grow0, NG, NG, nheads, true, p, b, head0,
-                           nullptr, nullptr, 0, 0, wts);
+  merge_partials<D, C::NW>(p.grp_ml, p.grp_o, grow0, NG, NG, nheads, fin, p, b, head0,
+                           fml, fo, frow, 1, wts);
   if (tid == 0) ucnt[0] = 0;
 }
 
@@ -1836,13 +2023,17 @@ static cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap& tmk
 }
 
 // K mode 2 (E4M3 MMAs) is built with the cvt decode of V and without
-// per-token scales; other combinations take mode 1 for K.
+// per-token scales; other combinations take mode 1 for K. Mode 3 is the fp8
+// compute path (V is not decoded), page and head scales only.
 template <int D, bool TOK>
 static cudaError_t launch_decode_kv(const DecodeParams& p, const CUtensorMap& tmk,
                                     const CUtensorMap& tmv, int k_mode, bool v_cvt,
                                     cudaStream_t s) {
   if constexpr (!TOK) {
+    if (k_mode == 3) return launch_decode_d<D, 3, true, false>(p, tmk, tmv, s);
     if (k_mode == 2 && v_cvt) return launch_decode_d<D, 2, true, false>(p, tmk, tmv, s);
+  } else {
+    if (k_mode == 3) return cudaErrorInvalidValue;  // refused by the host first
   }
   if (k_mode >= 1)
     return v_cvt ? launch_decode_d<D, 1, true, TOK>(p, tmk, tmv, s)
@@ -1916,6 +2107,68 @@ int decode_smem_bytes(int D) {
     case 512: return Cfg<512>::SMEM;
     default: return 0;
   }
+}
+
+// Merge of R context-parallel partials of each (sequence, query head): with
+// m_r, l_r, O_r the rank's maximum (log2 units), sum and numerator,
+// M = max(max_r m_r, sink * log2 e), den = sum_r l_r 2^(m_r - M) + 2^(sink
+// log2 e - M), out = sum_r O_r 2^(m_r - M) / den (0 when den is 0). One block
+// of 128 threads per (sequence, query head); R <= kCombineMaxRanks.
+constexpr int kCombineMaxRanks = 1024;
+__global__ void __launch_bounds__(128)
+    combine_kernel(const float* po, const float* pml, int R, int BH, int Hq, int D,
+                   const float* sinks, int64_t sinks_s, float* out, int64_t o_sb, int64_t o_sh) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  __shared__ float w[kCombineMaxRanks];
+  __shared__ float red[2];
+  const int row = blockIdx.x, b = row / Hq, h = row - b * Hq;
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (tid < 32) {
+    float M = -CUDART_INF_F;
+    for (int r = lane; r < R; r += 32) M = fmaxf(M, pml[((int64_t)r * BH + row) * 2]);
+    M = warp_max(M);
+    const float sl = sinks ? sinks[(int64_t)h * sinks_s] * kLog2e : -CUDART_INF_F;
+    const float M2 = fmaxf(M, sl);
+    float den = 0.f;
+    for (int r = lane; r < R; r += 32) {
+      const float2 ml = *reinterpret_cast<const float2*>(pml + ((int64_t)r * BH + row) * 2);
+      const float wr = (M2 == -CUDART_INF_F || ml.x == -CUDART_INF_F) ? 0.f : fast_exp2(ml.x - M2);
+      w[r] = wr;
+      den += wr * ml.y;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (lane == 0) {
+      if (sinks && M2 != -CUDART_INF_F) den += fast_exp2(sl - M2);
+      red[0] = den > 0.f ? 1.f / den : 0.f;
+    }
+  }
+  __syncthreads();
+  const float inv = red[0];
+  for (int d = tid * 4; d < D; d += 128 * 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = 0; r < R; ++r) {
+      const float wr = w[r];
+      if (wr == 0.f) continue;  // an empty or masked rank: its numerator may be anything
+      const float4 v = *reinterpret_cast<const float4*>(po + ((int64_t)r * BH + row) * D + d);
+      acc.x += wr * v.x;
+      acc.y += wr * v.y;
+      acc.z += wr * v.z;
+      acc.w += wr * v.w;
+    }
+    *reinterpret_cast<float4*>(out + (int64_t)b * o_sb + (int64_t)h * o_sh + d) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
+}
+
+cudaError_t launch_combine(const float* po, const float* pml, int R, int B, int Hq, int D,
+                           const float* sinks, int64_t sinks_s, float* out, int64_t o_sb,
+                           int64_t o_sh, cudaStream_t s) {
+  if (R < 1 || R > kCombineMaxRanks || D % 4) return cudaErrorInvalidValue;
+  const int BH = B * Hq;
+  if (BH == 0) return cudaSuccess;
+  combine_kernel<<<BH, 128, 0, s>>>(po, pml, R, BH, Hq, D, sinks, sinks_s, out, o_sb, o_sh);
+  return cudaGetLastError();
 }
 
 // E4M3 codes of n float32 values with the append's rounding

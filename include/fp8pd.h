@@ -262,6 +262,61 @@ int fp8_paged_decode_append_attention(const fp8pd_tensor* q, const fp8pd_tensor*
                                       const fp8pd_tensor* sinks, float sm_scale, fp8pd_tensor* out,
                                       fp8pd_stream_t stream);
 /*
+ * fp8_paged_decode_attention_partial -- decode attention over a slice of each
+ * sequence's keys, left unnormalized, for context-parallel split-KV: each GPU
+ * holds part of a long sequence's pages, attends its slice, and the slices'
+ * results are merged by fp8pd_combine_partials (the log-sum-exp combine of
+ * splits; the solution page's "Why it happens": a grid over (sequence, KV
+ * head, split), splitting a long sequence's keys being what keeps every SM --
+ * here every GPU -- busy).
+ *
+ * For each b and query head hq, with the keys [lo, hi) = the window's range
+ * of the L = seq_lens[b] keys (as fp8_paged_decode_attention) cut to
+ * [key_ranges[b, 0], key_ranges[b, 1]) (the whole range when key_ranges is
+ * NULL), and s2_t = sm_scale * log2(e) * q . K(t):
+ *   part_ml[b, hq, 0] = m = max_t s2_t             (-inf with no keys)
+ *   part_ml[b, hq, 1] = l = sum_t 2^(s2_t - m)     (0 with no keys)
+ *   part_o[b, hq, :]  =     sum_t 2^(s2_t - m) V(t) (0 with no keys)
+ * There is no sink term: fp8pd_combine_partials adds it once. Only the pages
+ * holding attended keys are read, so a rank's block table may mark every
+ * other entry unused (-1).
+ *
+ * Arguments: as fp8_paged_decode_attention without sinks, plus
+ *   key_ranges  int32 [B, 2] (begin, end) or NULL, any strides;
+ *   part_o      float32 [B, Hq, D], contiguous, 16-byte aligned;
+ *   part_ml     float32 [B, Hq, 2], contiguous, 8-byte aligned.
+ * Same planning, workspace and error rules as fp8_paged_decode_attention
+ * (FP8PD_OPT_COMPUTE applies).
+ */
+int fp8_paged_decode_attention_partial(const fp8pd_tensor* q, const fp8pd_tensor* k_pages,
+                                       const fp8pd_tensor* v_pages, const fp8pd_tensor* k_scale,
+                                       const fp8pd_tensor* v_scale,
+                                       const fp8pd_tensor* block_table,
+                                       const fp8pd_tensor* seq_lens,
+                                       const fp8pd_tensor* key_ranges, int32_t window,
+                                       float sm_scale, fp8pd_tensor* part_o,
+                                       fp8pd_tensor* part_ml, fp8pd_stream_t stream);
+
+/*
+ * fp8pd_combine_partials -- merges R partial results per (sequence, query
+ * head), as fp8_paged_decode_attention_partial writes them, into the
+ * attention output, adding the sink once (the log-sum-exp combine of splits;
+ * the solution page's "Expected result" for the sink: one logit per query
+ * head in the denominator, no value):
+ *   M = max(max_r m_r, sink * log2 e)
+ *   den = sum_r l_r 2^(m_r - M) + 2^(sink * log2 e - M)
+ *   out = sum_r O_r 2^(m_r - M) / den              (0 when den is 0)
+ * A rank with no keys (m = -inf) contributes nothing, whatever its O holds.
+ *   part_o   float32 [R, B, Hq, D], contiguous, 16-byte aligned, D % 4 == 0;
+ *   part_ml  float32 [R, B, Hq, 2], contiguous, 8-byte aligned; 1 <= R <= 1024;
+ *   sinks    float32 [Hq] or NULL;
+ *   out      float32 [B, Hq, D]; stride[2] must be 1, rows 16-byte aligned.
+ * One kernel launch; no workspace.
+ */
+int fp8pd_combine_partials(const fp8pd_tensor* part_o, const fp8pd_tensor* part_ml,
+                           const fp8pd_tensor* sinks, fp8pd_tensor* out, fp8pd_stream_t stream);
+
+/*
  * fp8_paged_decode_attention_noalloc -- the same operation, allocating nothing.
  *
  * This entry point has no counterpart in the method's description; it is for
@@ -343,11 +398,19 @@ enum {
   FP8PD_OPT_WAIT_POLLS = 6,  /* polls of a tile copy's barrier before the wait gives up and sets
                                 FP8PD_FLAG_TIMEOUT; each poll sleeps at most 20 us. Default
                                 131,072 (about 2.6 s); 1 .. 1,048,576 */
-  FP8PD_OPT_TEST_STALL = 7   /* test hook of the timeout path, 0 (default) or 1: warp 0 of the
+  FP8PD_OPT_TEST_STALL = 7,  /* test hook of the timeout path, 0 (default) or 1: warp 0 of the
                                 first block of each attention launch never issues its first tile
                                 copy, so that one wait runs out; the keys of that warp are left
                                 out and FP8PD_FLAG_TIMEOUT is set. No copy is in flight on the
                                 stalled stage, so the launch ends normally. */
+  FP8PD_OPT_COMPUTE = 8      /* numerical path of the attention: 0 (default) = f32 compute (K and
+                                V decoded exactly, q exact in f16, P as an f16 hi + lo pair; max
+                                |err| <= 1e-3 * max(1, |ref|)); 1 = fp8 compute (the solution
+                                page's compute="fp8": q rounded once to E4M3 per query head after
+                                a power-of-two scale, each weight exp(s - running max) * v_scale /
+                                max v_scale * 2^8 rounded once to E4M3, K and V bytes into E4M3
+                                MMAs; the page holds it to 1.5e-1). Per-token scales are refused
+                                on the fp8 path with FP8PD_ERR_UNSUPPORTED, never downgraded. */
 };
 int fp8pd_set_option(int32_t option, int64_t value);
 int64_t fp8pd_get_option(int32_t option);
@@ -363,6 +426,7 @@ typedef struct fp8pd_run_info {
   int64_t calls;             /* attention calls made by this process */
   int64_t appends;           /* append calls made by this process */
   int64_t kernel_launches;   /* kernels this library launched in this process */
+  int32_t compute;           /* FP8PD_OPT_COMPUTE of the last attention call (0 f32, 1 fp8) */
 } fp8pd_run_info;
 int fp8pd_last_run_info(fp8pd_run_info* info);
 

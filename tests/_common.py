@@ -20,14 +20,14 @@ def np_(t: torch.Tensor | None):
     return t.detach().cpu().numpy()
 
 
-def oracle_attention(layer, lens, batch_heads=None, pages=None) -> np.ndarray:
+def oracle_attention(layer, lens, batch_heads=None, pages=None, compute="f32") -> np.ndarray:
     """Oracle output for one layer of a workload (inputs copied to the host)."""
     return O.paged_decode_attention(
         np_(layer.q), np_(layer.k_pages if pages is None else pages[0]),
         np_(layer.v_pages if pages is None else pages[1]),
         np_(layer.k_scale), np_(layer.v_scale), np_(layer.block_table), np_(lens),
         window=layer.window, sinks=np_(layer.sinks), sm_scale=layer.sm_scale,
-        batch_heads=batch_heads)
+        batch_heads=batch_heads, compute=compute)
 
 
 def gpu_attention(F, layer, lens, out=None):

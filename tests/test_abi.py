@@ -201,6 +201,18 @@ def test_options_roundtrip(F):
         with pytest.raises(F.Fp8pdError):
             F.fp8pd_set_option(opt, bad)
     assert F.fp8pd_get_option(F.OPT_TEST_STALL) == 0
+    assert F.fp8pd_get_option(F.OPT_COMPUTE) == 0
+    F.fp8pd_set_option(F.OPT_COMPUTE, 1)
+    assert F.fp8pd_get_option(F.OPT_COMPUTE) == 1
+    F.fp8pd_set_option(F.OPT_COMPUTE, 0)
+    for bad in (2, -1):
+        with pytest.raises(F.Fp8pdError):
+            F.fp8pd_set_option(F.OPT_COMPUTE, bad)
+    F.fp8pd_set_option(F.OPT_K_DECODE, 2)
+    assert F.fp8pd_get_option(F.OPT_K_DECODE) == 2
+    F.fp8pd_set_option(F.OPT_K_DECODE, 1)
+    with pytest.raises(F.Fp8pdError):
+        F.fp8pd_set_option(F.OPT_K_DECODE, 3)
     with pytest.raises(F.Fp8pdError):
         F.fp8pd_set_option(99, 1)
     with pytest.raises(F.Fp8pdError):
