@@ -10,6 +10,7 @@ from .fp8pd_oracle import (  # noqa: F401
     E4M3_NAN_CODE,
     E4M3_TABLE,
     attended_range,
+    combine_partials,
     e4m3_code_value,
     e4m3_decode,
     e4m3_encode,
@@ -20,6 +21,7 @@ from .fp8pd_oracle import (  # noqa: F401
     group_scale,
     kv_append,
     paged_decode_attention,
+    paged_decode_partial,
     quantize,
     quantize_per_token,
     token_scale,

@@ -339,6 +339,77 @@ def paged_decode_attention(q, k_pages, v_pages, k_scale, v_scale, block_table, s
     return out
 
 
+LOG2E = 1.0 / math.log(2.0)
+
+
+def paged_decode_partial(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens,
+                         key_ranges=None, window: int = 0, sm_scale: float | None = None):
+    """Unnormalized attention over a slice of each sequence's keys (one GPU's
+    share of a context-parallel split), float64.
+
+    Keys: the window's range [lo, L) of :func:`attended_range` cut to
+    [key_ranges[b, 0], key_ranges[b, 1]) (all of it when key_ranges is None).
+    With s_t the scaled scores of those keys (as in
+    :func:`paged_decode_attention`, no sink) and m = max_t s_t:
+      ml[b, hq] = (m * log2(e), sum_t exp(s_t - m)),  o[b, hq] = sum_t exp(s_t - m) V(t);
+    (-inf, 0) and 0 with no keys. Returns (o [B, Hq, D], ml [B, Hq, 2]).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, D = q.shape
+    Hkv = k_pages.shape[2]
+    G = Hq // Hkv
+    if sm_scale is None:
+        sm_scale = D ** -0.5
+    sm = float(np.float32(sm_scale))
+    o = np.zeros((B, Hq, D))
+    ml = np.zeros((B, Hq, 2))
+    ml[:, :, 0] = -math.inf
+    for b in range(B):
+        lo, L = attended_range(int(seq_lens[b]), int(window))
+        if key_ranges is not None:
+            lo, L = max(lo, int(key_ranges[b][0])), min(L, int(key_ranges[b][1]))
+        if L <= lo:
+            continue
+        positions = np.arange(lo, L, dtype=np.int64)
+        for h in range(Hkv):
+            kc, phys = gather_tokens(k_pages, block_table[b], positions, h)
+            vc, _ = gather_tokens(v_pages, block_table[b], positions, h)
+            slots = positions % k_pages.shape[1]
+            K = _dequantize(kc, k_scale, phys, slots, h)
+            V = _dequantize(vc, v_scale, phys, slots, h)
+            for hq in range(h * G, (h + 1) * G):
+                s = sm * (K @ q[b, hq])
+                m = s.max()
+                w = np.exp(s - m)
+                o[b, hq] = w @ V
+                ml[b, hq] = (m * LOG2E, w.sum())
+    return o, ml
+
+
+def combine_partials(part_o, part_ml, sinks=None) -> np.ndarray:
+    """The log-sum-exp combine of R partials (as :func:`paged_decode_partial`
+    writes them) into the attention output, the sink added once:
+    M = max(max_r m_r, sink log2 e), den = sum_r l_r 2^(m_r - M) + 2^(sink log2 e - M),
+    out = sum_r o_r 2^(m_r - M) / den, 0 when den is 0. part_o [R, B, Hq, D],
+    part_ml [R, B, Hq, 2]."""
+    part_o = np.asarray(part_o, dtype=np.float64)
+    part_ml = np.asarray(part_ml, dtype=np.float64)
+    R, B, Hq, D = part_o.shape
+    out = np.zeros((B, Hq, D))
+    for b in range(B):
+        for hq in range(Hq):
+            m = part_ml[:, b, hq, 0]
+            sl = -math.inf if sinks is None else float(sinks[hq]) * LOG2E
+            M = max(float(m.max()), sl)
+            if M == -math.inf:
+                continue
+            w = np.where(m == -math.inf, 0.0, np.exp2(np.where(m == -math.inf, 0.0, m) - M))
+            den = float((w * part_ml[:, b, hq, 1]).sum()) + (0.0 if sinks is None else 2.0 ** (sl - M))
+            if den > 0.0:
+                out[b, hq] = (w[:, None] * part_o[:, b, hq]).sum(0) / den
+    return out
+
+
 def kv_append(k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table, positions) -> None:
     """Quantize one new token per sequence and store it in its page, in place.
 

@@ -944,3 +944,61 @@ def test_fp8_compute_stays_within_the_pages_tolerance_of_f32():
         err = np.abs(f8 - f32) / np.maximum(1.0, np.abs(f32))
         assert err.max() <= 1.5e-1, err.max()
         assert err.max() > 0.0                      # the roundings do change the result
+
+
+# ------------------------------------------- context-parallel partials + combine
+# Splitting a sequence's keys over GPUs and merging the slices' partial
+# results must give the attention over all keys (the log-sum-exp combine of
+# splits). The pins check the oracle's partial and combine against the full
+# attention (pinned above), not against themselves.
+
+def _partition(rng, L, R, ps, aligned=True):
+    """R contiguous slices covering [0, L): page-aligned cut points, or
+    arbitrary ones; some slices may be empty."""
+    cuts = rng.integers(0, L + 1, size=R - 1)
+    if aligned:
+        cuts = (cuts // ps) * ps
+    cuts = np.sort(np.concatenate([[0], cuts, [L]]))
+    return [(int(cuts[i]), int(cuts[i + 1])) for i in range(R)]
+
+
+@pytest.mark.parametrize("window,with_sinks", [(0, False), (0, True), (50, True), (7, False)])
+def test_combined_partials_over_any_partition_equal_full_attention(window, with_sinks):
+    rng = np.random.default_rng(61 + window)
+    c = _dense_case(rng, B=3, L=(120, 77, 33), scale_mode="page")
+    sinks = rng.standard_normal(8).astype(np.float32) if with_sinks else None
+    want = _run(c, window=window, sinks=sinks, sm_scale=0.3)
+    for R, aligned in ((1, True), (2, True), (3, False), (8, True), (8, False)):
+        ranges = [_partition(rng, int(L), R, 16, aligned) for L in c["lens"]]
+        parts = [O.paged_decode_partial(c["q"], c["k"], c["v"], c["ks"], c["vs"], c["table"],
+                                        c["lens"], np.array([ranges[b][r] for b in range(3)]),
+                                        window=window, sm_scale=0.3) for r in range(R)]
+        got = O.combine_partials(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]),
+                                 sinks)
+        assert np.allclose(got, want, rtol=1e-12, atol=1e-14), (R, aligned)
+
+
+def test_partial_closed_forms():
+    """q = 0: every score is 0, so m = 0, l = the slice's key count and o the
+    plain sum of its values; an empty slice gives (-inf, 0, 0) and adds
+    nothing to a combine."""
+    rng = np.random.default_rng(62)
+    c = _dense_case(rng, B=2, L=(90, 40), scale_mode="head")
+    c0 = dict(c, q=np.zeros_like(c["q"]))
+    kr = np.array([[16, 70], [0, 40]])
+    o, ml = O.paged_decode_partial(c0["q"], c0["k"], c0["v"], c0["ks"], c0["vs"], c0["table"],
+                                   c0["lens"], kr)
+    G, ps = 4, 16
+    for b in range(2):
+        t = np.arange(kr[b][0], kr[b][1])
+        phys = c["table"][b][t // ps]
+        for hq in range(8):
+            V = O.e4m3_decode(c["v"][phys, t % ps, hq // G]) * float(c["vs"][hq // G])
+            assert ml[b, hq, 0] == 0.0 and ml[b, hq, 1] == len(t)
+            assert np.allclose(o[b, hq], V.sum(0), rtol=1e-13, atol=1e-15)
+    o_e, ml_e = O.paged_decode_partial(c["q"], c["k"], c["v"], c["ks"], c["vs"], c["table"],
+                                       c["lens"], np.array([[5, 5], [40, 90]]))
+    assert np.all(ml_e[:, :, 0] == -np.inf) and np.all(ml_e[:, :, 1] == 0) and np.all(o_e == 0)
+    full = O.paged_decode_partial(c["q"], c["k"], c["v"], c["ks"], c["vs"], c["table"], c["lens"])
+    both = O.combine_partials(np.stack([full[0], o_e]), np.stack([full[1], ml_e]))
+    assert np.array_equal(both, O.combine_partials(full[0][None], full[1][None]))
