@@ -15,11 +15,14 @@ from .fp8pd_oracle import (  # noqa: F401
     e4m3_decode,
     e4m3_encode,
     e4m3_round,
+    e8m0_decode,
     fp8_compute_query,
     expand_groups,
     gather_tokens,
     group_scale,
     kv_append,
+    mx_quantize,
+    mx_scale_code,
     paged_decode_attention,
     paged_decode_partial,
     quantize,

@@ -42,6 +42,15 @@ Readings of the pages (each is listed with its reason in the design notes):
   groups (P1 "Supported scope", ``k_groups``) add a last axis of ``groups``
   scales, group g covering entries [g D/groups, (g+1) D/groups).
 * empty attention (no keys, no sink) returns 0.
+* MXFP8 (P3, "Attention MXFP8 TKG", decode attention over an MXFP8 KV
+  cache; the page names the format without spelling it out): the OCP
+  microscaling format, E4M3 elements in blocks of 32 consecutive entries
+  that share one E8M0 scale 2^(c - 127) (c = 255 is NaN). A cache row of D
+  entries per (token, KV head) has D / 32 scale bytes, stored as a uint8
+  array [num_pages, ps, Hkv, D / 32] beside the codes. A block's scale is
+  2^(floor(log2 max|x|) - 8) (8 = E4M3's largest exponent; all-zero block:
+  2^0), clamped to the E8M0 range, and its codes are E4M3 of x / scale,
+  saturating at 448.
 * the opt-in "fp8 compute" path (P1 "Two compute paths", ``compute="fp8"``,
   and "Limitations": it adds one E4M3 rounding on q and on p) rounds each
   query row to E4M3 after a power-of-two scale that puts its largest
@@ -189,6 +198,48 @@ def group_scale(x, groups: int) -> np.ndarray:
     return token_scale(x32.reshape(*x32.shape[:-1], groups, D // groups))
 
 
+MX_BLOCK = 32
+
+
+def e8m0_decode(codes) -> np.ndarray:
+    """E8M0 scale codes to float64: 2^(c - 127), NaN for 255."""
+    c = np.asarray(codes, dtype=np.int64)
+    return np.where(c == 255, np.nan, np.exp2((c - 127).astype(np.float64)))
+
+
+def mx_scale_code(block) -> int:
+    """E8M0 code of one block's shared scale: c = floor(log2 max|x|) - 8 +
+    127, clamped to [0, 254]; NaN entries are skipped and an all-zero block
+    takes c = 127 (scale 1)."""
+    a = np.abs(np.asarray(block, dtype=np.float64))
+    a = a[~np.isnan(a)]
+    amax = float(a.max()) if a.size else 0.0
+    if amax == 0.0:
+        return 127
+    if not math.isfinite(amax):
+        return 254
+    _, e = math.frexp(amax)            # amax in [2^(e-1), 2^e)
+    return int(min(254, max(0, (e - 1) - 8 + 127)))
+
+
+def mx_quantize(x) -> tuple[np.ndarray, np.ndarray]:
+    """MXFP8 quantization of rows x [..., D] (D a multiple of 32): returns
+    (E4M3 codes [..., D], E8M0 scale codes [..., D / 32]). Each element is
+    E4M3(x / 2^(c - 127)) of float32 x, the division by a power of two exact
+    in float64, rounded to nearest even and saturated at 448."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    D = x.shape[-1]
+    if D % MX_BLOCK:
+        raise ValueError("D must be a multiple of 32")
+    blocks = x.reshape(x.shape[:-1] + (D // MX_BLOCK, MX_BLOCK))
+    sc = np.zeros(blocks.shape[:-1], dtype=np.uint8)
+    for idx in np.ndindex(*sc.shape):
+        sc[idx] = mx_scale_code(blocks[idx])
+    scale = np.exp2(sc.astype(np.float64) - 127.0)[..., None]
+    codes = e4m3_encode(blocks / scale).reshape(x.shape)
+    return codes, sc
+
+
 def expand_groups(scales: np.ndarray, D: int) -> np.ndarray:
     """[..., groups] sub-row scales -> [..., D]: entry d takes the scale of its
     group d // (D / groups)."""
@@ -207,6 +258,8 @@ def _scale_of(scale: np.ndarray, page: np.ndarray, slot: np.ndarray, head: int) 
     [num_pages, ps, Hkv, groups] (sub-row groups) the result has a trailing
     axis of the token's group scales."""
     scale = np.asarray(scale)
+    if scale.dtype == np.uint8:  # MXFP8: E8M0 block scales [num_pages, ps, Hkv, D / 32]
+        return e8m0_decode(scale[page, slot, head, :])
     if scale.ndim == 1:
         return np.full(np.shape(page), np.float64(scale[head]))
     if scale.ndim == 2:
@@ -435,6 +488,11 @@ def kv_append(k_new, v_new, k_pages, v_pages, k_scale, v_scale, block_table, pos
         for h in range(Hkv):
             for x, pages, scale in ((k_new[b][h], k_pages, k_scale), (v_new[b][h], v_pages, v_scale)):
                 x32 = np.asarray(x, np.float32)
+                if np.asarray(scale).dtype == np.uint8:   # MXFP8: the token's own block scales
+                    codes, sc = mx_quantize(x32)
+                    scale[page, slot, h, :] = sc
+                    pages[page, slot, h, :] = codes
+                    continue
                 if np.ndim(scale) == 4:
                     scale[page, slot, h, :] = group_scale(x32, np.shape(scale)[3])
                     s = expand_groups(np.asarray(scale[page, slot, h, :], np.float32), x32.shape[-1])

@@ -1002,3 +1002,112 @@ def test_partial_closed_forms():
     full = O.paged_decode_partial(c["q"], c["k"], c["v"], c["ks"], c["vs"], c["table"], c["lens"])
     both = O.combine_partials(np.stack([full[0], o_e]), np.stack([full[1], ml_e]))
     assert np.array_equal(both, O.combine_partials(full[0][None], full[1][None]))
+
+
+# ------------------------------------------------------------------ MXFP8
+# The OCP microscaling reading of the MXFP8 cache: E4M3 elements in blocks of
+# 32 entries sharing one E8M0 scale. Pins: the library's own E8M0 and E4M3
+# types, the scale rule written out from its definition, and attention over
+# values dequantized through the library types.
+
+def test_e8m0_decode_matches_library_type_on_all_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    lib = torch.from_numpy(codes).view(torch.float8_e8m0fnu).double().numpy()
+    assert np.array_equal(O.e8m0_decode(codes), lib, equal_nan=True)
+    assert O.e8m0_decode(127) == 1.0 and O.e8m0_decode(0) == 2.0 ** -127
+    assert np.isnan(O.e8m0_decode(255))
+
+
+def test_mx_quantize_matches_the_library_casts():
+    """Scale: the block's largest magnitude, divided by the scale, lies in
+    [2^8, 2^9) (2^8 = E4M3's largest binade); codes: the library's E4M3 cast of
+    the clamped quotient."""
+    rng = np.random.default_rng(81)
+    for trial in range(40):
+        D = int(rng.choice([32, 64, 128, 256, 512]))
+        x = (rng.standard_normal((3, D)) * 10.0 ** rng.uniform(-8, 8)).astype(np.float32)
+        x[0, :32] *= 0                                       # an all-zero block
+        codes, sc = O.mx_quantize(x)
+        assert sc.shape == (3, D // 32) and sc.dtype == np.uint8
+        assert sc[0, 0] == 127
+        scale = torch.from_numpy(sc).view(torch.float8_e8m0fnu).double().numpy()
+        blocks = x.astype(np.float64).reshape(3, D // 32, 32)
+        amax = np.abs(blocks).max(-1)
+        nz = amax > 0
+        ratio = amax[nz] / scale[nz]
+        assert np.all((ratio >= 256) & (ratio < 512))
+        q = np.clip(blocks / scale[..., None], -448, 448).reshape(3, D)
+        want = torch.from_numpy(q).float().to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(codes, want)
+
+
+@pytest.mark.parametrize("window,with_sinks", [(0, False), (40, True)])
+def test_mx_attention_matches_library_sdpa(window, with_sinks):
+    """K and V in MXFP8 (codes and E8M0 block scales, as mx_quantize writes
+    them): the oracle against torch SDPA over values dequantized with the
+    library's float8 types, one scale per 32-entry block."""
+    rng = np.random.default_rng(82)
+    B, Hq, Hkv, D, ps = 2, 8, 2, 64, 16
+    lens = np.array([70, 33])
+    npg = (lens + ps - 1) // ps
+    total = int(npg.sum()) + 2
+    perm = rng.permutation(total)
+    table = np.full((B, npg.max()), -1, np.int32)
+    off = 0
+    for b in range(B):
+        table[b, :npg[b]] = perm[off:off + npg[b]]
+        off += npg[b]
+    xk = rng.standard_normal((total, ps, Hkv, D)) * np.exp(rng.uniform(-3, 3, (total, ps, Hkv, 1)))
+    xv = rng.standard_normal((total, ps, Hkv, D)) * np.exp(rng.uniform(-3, 3, (total, ps, Hkv, 1)))
+    k, ks = O.mx_quantize(xk)
+    v, vs = O.mx_quantize(xv)
+    q = torch.randn(B, Hq, D, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16).double()
+    sinks = rng.standard_normal(Hq).astype(np.float32) if with_sinks else None
+    sm = 0.15
+    got = O.paged_decode_attention(q.numpy(), k, v, ks, vs, table, lens, window=window,
+                                   sinks=sinks, sm_scale=sm)
+    deq = lambda c, s: (torch.from_numpy(c).view(torch.float8_e4m3fn).double() *  # noqa: E731
+                        torch.from_numpy(s).view(torch.float8_e8m0fnu).double()
+                        .repeat_interleave(32, dim=-1))
+    K, V = deq(k, ks), deq(v, vs)
+    G = Hq // Hkv
+    for b in range(B):
+        L = int(lens[b])
+        lo = max(0, L - window) if window else 0
+        t = np.arange(L)
+        phys = table[b][t // ps]
+        Kb = K[phys, t % ps].permute(1, 0, 2).repeat_interleave(G, 0)   # [Hq, L, D]
+        Vb = V[phys, t % ps].permute(1, 0, 2).repeat_interleave(G, 0)
+        mask = torch.zeros(Hq, 1, L + 1, dtype=torch.float64)
+        mask[:, :, :lo] = -math.inf
+        mask[:, :, L] = -math.inf if sinks is None else torch.from_numpy(sinks).double()[:, None]
+        Kb = torch.cat([Kb, torch.zeros(Hq, 1, D, dtype=torch.float64)], 1)
+        Vb = torch.cat([Vb, torch.zeros(Hq, 1, D, dtype=torch.float64)], 1)
+        o = torch.nn.functional.scaled_dot_product_attention(q[b][:, None, :], Kb, Vb,
+                                                             attn_mask=mask,
+                                                             scale=float(np.float32(sm)))
+        assert np.allclose(got[b], o[:, 0].numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_mx_append_writes_the_tokens_block_scales_and_codes():
+    rng = np.random.default_rng(83)
+    B, Hkv, D, ps, P = 3, 2, 128, 16, 9
+    kp = rng.integers(0, 256, (P, ps, Hkv, D)).astype(np.uint8)
+    vp = kp.copy()
+    ks = rng.integers(0, 255, (P, ps, Hkv, D // 32)).astype(np.uint8)
+    vs = ks.copy()
+    table = rng.permutation(P)[:B * 3].reshape(B, 3).astype(np.int32)
+    pos = np.array([5, 16, 47])
+    kn = torch.randn(B, Hkv, D).to(torch.bfloat16).double().numpy() * 3
+    vn = torch.randn(B, Hkv, D).to(torch.bfloat16).double().numpy() * 1e-3
+    kp0, vp0, ks0, vs0 = kp.copy(), vp.copy(), ks.copy(), vs.copy()
+    O.kv_append(kn, vn, kp, vp, ks, vs, table, pos)
+    touched = np.zeros((P, ps), bool)
+    for b in range(B):
+        page, slot = table[b][pos[b] // ps], pos[b] % ps
+        touched[page, slot] = True
+        for new, pages, sc in ((kn, kp, ks), (vn, vp, vs)):
+            c, s = O.mx_quantize(new[b])
+            assert np.array_equal(pages[page, slot], c) and np.array_equal(sc[page, slot], s)
+    for a, a0 in ((kp, kp0), (vp, vp0), (ks, ks0), (vs, vs0)):
+        assert np.array_equal(a[~touched], a0[~touched])
