@@ -273,6 +273,8 @@ def _spec_bytes(spec: W.Spec) -> int:
                 total += 4 * ((Lb - 1) // spec.ps - lo // spec.ps + 1)
             if spec.scale_mode == "token":
                 total += 4 * n * L.Hkv * (spec.k_groups + 1)
+            elif spec.scale_mode == "mx":
+                total += 2 * n * L.Hkv * (L.D // 32)
         total += 2 * spec.B * L.Hq * L.D
     return int(total)
 
@@ -705,7 +707,10 @@ def cpu_baseline(case: W.Case, budget_s: float = 10.0) -> dict:
 def _scale_override(args) -> dict:
     """``--scales token``: the workload with one scale per stored token and KV
     head instead of its own scale form."""
-    if getattr(args, "scales", "workload") != "token":
+    scales = getattr(args, "scales", "workload")
+    if scales == "mx":
+        return {"scale_mode": "mx"}
+    if scales != "token":
         return {}
     return {"scale_mode": "token", "k_groups": getattr(args, "k_groups", 1)}
 
@@ -713,6 +718,8 @@ def _scale_override(args) -> dict:
 def _workload_text(args, name: str | None = None) -> str:
     name = name or args.config
     text = WORKLOAD_TEXT.get(name, name)
+    if getattr(args, "scales", "workload") == "mx":
+        return text + " (K and V stored as MXFP8: E8M0 scale per 32-entry block)"
     if getattr(args, "scales", "workload") != "token":
         return text
     groups = f", K in {args.k_groups} sub-row groups" if args.k_groups > 1 else ""
@@ -721,7 +728,8 @@ def _workload_text(args, name: str | None = None) -> str:
 
 def _scales_text(spec) -> str:
     text = {"head": "per KV head", "page": "per (page, KV head)",
-            "token": "per (token, KV head)"}[spec.scale_mode]
+            "token": "per (token, KV head)",
+            "mx": "MXFP8: E8M0 per (token, KV head, 32-entry block)"}[spec.scale_mode]
     if spec.scale_mode == "token" and spec.k_groups > 1:
         text += f"; K per (token, KV head, group of D/{spec.k_groups})"
     return text
@@ -835,8 +843,9 @@ def build_parser() -> argparse.ArgumentParser:
                     help="QK contraction: K decoded to f16 by bit assembly or the hardware cvt, "
                          "or K's E4M3 bytes in E4M3 MMAs (mma8)")
     ap.add_argument("--splits", type=int, default=0, help="force a split count (0 = planner)")
-    ap.add_argument("--scales", default="workload", choices=["workload", "token"],
-                    help="token: per-token-per-head K/V scales instead of the workload's form")
+    ap.add_argument("--scales", default="workload", choices=["workload", "token", "mx"],
+                    help="token: per-token-per-head K/V scales instead of the workload's form; "
+                         "mx: the MXFP8 cache (E8M0 scale per 32-entry block)")
     ap.add_argument("--k-groups", type=int, default=1,
                     help="with --scales token: K scales per sub-row group of D / k_groups entries")
     ap.add_argument("--compute", default="f32", choices=["f32", "fp8"],

@@ -84,13 +84,30 @@ bool fits_i32(int64_t v) { return v >= 0 && v <= INT32_MAX; }
 // `max_groups` caps it (1: no sub-row groups).
 int scale_strides(const fp8pd_tensor* s, int64_t num_pages, int64_t ps, int64_t hkv, int64_t d,
                   int max_groups, int64_t* sp, int64_t* st, int64_t* sh, int64_t* sg, int* tok,
-                  int* groups) {
+                  int* groups, int* mx = nullptr) {
   if (!s || !s->data) return FP8PD_ERR_NULL;
-  if (s->dtype != FP8PD_DTYPE_F32) return FP8PD_ERR_DTYPE;
   *st = 0;
   *sg = 0;
   *tok = 0;
   *groups = 1;
+  if (mx) *mx = 0;
+  if (s->dtype == FP8PD_DTYPE_U8) {
+    // MXFP8: E8M0 block scales [num_pages, ps, Hkv, D / 32], one byte per 32 entries
+    if (!mx) return FP8PD_ERR_DTYPE;
+    if (s->ndim != 4) return FP8PD_ERR_SHAPE;
+    if (d % 32) return FP8PD_ERR_UNSUPPORTED;
+    if (s->shape[0] != num_pages || s->shape[1] != ps || s->shape[2] != hkv || s->shape[3] != d / 32)
+      return FP8PD_ERR_SHAPE;
+    *sp = s->stride[0];
+    *st = s->stride[1];
+    *sh = s->stride[2];
+    *sg = s->stride[3];
+    *tok = 1;
+    *groups = static_cast<int>(d / 32);
+    *mx = 1;
+    return FP8PD_OK;
+  }
+  if (s->dtype != FP8PD_DTYPE_F32) return FP8PD_ERR_DTYPE;
   if (s->ndim == 1) {
     if (s->shape[0] != hkv) return FP8PD_ERR_SHAPE;
     *sp = 0;
@@ -414,12 +431,12 @@ int validate_decode(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp
   // Sub-row K groups: each covers whole 16-entry blocks of the QK contraction
   // (D / groups >= 16); V takes one scale per token at most.
   int64_t ks_sp, ks_st, ks_sh, ks_sg, vs_sp, vs_st, vs_sh, vs_sg;
-  int k_tok, v_tok, k_groups, v_groups;
+  int k_tok, v_tok, k_groups, v_groups, k_mx, v_mx;
   if ((r = scale_strides(k_scale, P, ps, Hkv, D, static_cast<int>(D / 16), &ks_sp, &ks_st, &ks_sh,
-                         &ks_sg, &k_tok, &k_groups)))
+                         &ks_sg, &k_tok, &k_groups, &k_mx)))
     return r;
   if ((r = scale_strides(v_scale, P, ps, Hkv, D, 1, &vs_sp, &vs_st, &vs_sh, &vs_sg, &v_tok,
-                         &v_groups)))
+                         &v_groups, &v_mx)))
     return r;
   if (sinks) {
     if ((r = check(sinks, FP8PD_DTYPE_F32, 1))) return r;
@@ -455,6 +472,9 @@ int validate_decode(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp
   p->v_tok = v_tok;
   p->ks_sg = ks_sg;
   p->k_groups = k_groups;
+  p->k_mx = k_mx;
+  p->v_mx = v_mx;
+  p->vs_sg = vs_sg;
   p->table = static_cast<const int32_t*>(block_table->data);
   p->tab_sb = block_table->stride[0];
   p->tab_sp = block_table->stride[1];
@@ -829,12 +849,12 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
   if (block_table->shape[0] != B || positions->shape[0] != B) return FP8PD_ERR_SHAPE;
   if (ps < 1) return FP8PD_ERR_UNSUPPORTED;
   int64_t ks_sp, ks_st, ks_sh, ks_sg, vs_sp, vs_st, vs_sh, vs_sg;
-  int k_tok, v_tok, k_groups, v_groups;
+  int k_tok, v_tok, k_groups, v_groups, k_mx, v_mx;
   if ((r = scale_strides(&scales->k_scale, P, ps, Hkv, D, 16, &ks_sp, &ks_st, &ks_sh, &ks_sg,
-                         &k_tok, &k_groups)))
+                         &k_tok, &k_groups, &k_mx)))
     return r;
   if ((r = scale_strides(&scales->v_scale, P, ps, Hkv, D, 1, &vs_sp, &vs_st, &vs_sh, &vs_sg,
-                         &v_tok, &v_groups)))
+                         &v_tok, &v_groups, &v_mx)))
     return r;
   const int64_t max_pages = block_table->shape[1];
   if (!fits_i32(B) || !fits_i32(P) || !fits_i32(Hkv) || !fits_i32(D) || !fits_i32(max_pages) ||
@@ -871,6 +891,9 @@ int fp8_kv_append(const fp8pd_tensor* k_new, const fp8pd_tensor* v_new, fp8pd_te
   p.v_tok = v_tok;
   p.ks_sg = ks_sg;
   p.k_groups = k_groups;
+  p.k_mx = k_mx;
+  p.v_mx = v_mx;
+  p.vs_sg = vs_sg;
   p.ksw = static_cast<float*>(scales->k_scale.data);
   p.vsw = static_cast<float*>(scales->v_scale.data);
   p.table = static_cast<const int32_t*>(block_table->data);

@@ -24,6 +24,11 @@ struct DecodeParams {
   int k_tok, v_tok;           // 1: per-token-per-head scales [num_pages, ps, Hkv]
   int64_t ks_sg;              // K sub-row groups [num_pages, ps, Hkv, k_groups]: group stride
   int k_groups;               // 1, or 2..16 (D / k_groups >= 16): K entry d uses group d / (D / k_groups)
+  // MXFP8: K / V scales are E8M0 bytes [num_pages, ps, Hkv, D / 32] (ks / vs
+  // then point at uint8, strides in bytes); K takes k_groups = D / 32, V one
+  // code per 32-entry block (vs_sg its stride).
+  int k_mx, v_mx;
+  int64_t vs_sg;
   const int32_t* table;       // [B, max_pages]
   int64_t tab_sb, tab_sp;
   const int32_t* lens;        // [B]
@@ -88,6 +93,8 @@ struct AppendParams {
   int k_tok, v_tok;           // 1: the scale is the new token's own max|x| / 448, written here
   int64_t ks_sg;              // K sub-row groups: group stride; k_groups groups of D / k_groups
   int k_groups;
+  int k_mx, v_mx;             // MXFP8 block scales (E8M0 bytes, one per 32 entries), written here
+  int64_t vs_sg;
   float* ksw;
   float* vsw;
   const int32_t* table;

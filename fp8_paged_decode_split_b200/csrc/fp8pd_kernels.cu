@@ -159,6 +159,24 @@ __device__ __forceinline__ uint16_t e4m3x2_rn_sat(float lo, float hi) {
   return r;  // low byte = lo, high byte = hi
 }
 
+// MXFP8 (OCP microscaling): an E8M0 scale code c is 2^(c - 127), exact in
+// f32 (c = 0 is the subnormal 2^-127; c = 255 is NaN).
+__device__ __forceinline__ float e8m0_to_f32(uint32_t c) {
+  if (c == 0u) return __uint_as_float(0x00400000u);
+  if (c == 255u) return __uint_as_float(0x7fc00000u);
+  return __uint_as_float(c << 23);
+}
+// The E8M0 code of an MX block whose largest magnitude is m (NaN entries
+// already skipped): floor(log2 m) - 8 + 127, so that m / scale lies in
+// [2^8, 2^9), clamped to [0, 254]; an all-zero block takes 127 (scale 1).
+__device__ __forceinline__ uint32_t mx_code(float m) {
+  if (!(m > 0.f)) return 127u;
+  if (isinf(m)) return 254u;
+  int e;
+  frexpf(m, &e);  // m in [2^(e-1), 2^e)
+  return static_cast<uint32_t>(min(254, max(0, e - 1 - 8 + 127)));
+}
+
 __device__ __forceinline__ float4 ldcg4(const float* p) {
   float4 v;
   asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];\n"
@@ -693,10 +711,26 @@ __device__ __forceinline__ void tile_probs(Acc<D>& a, float4 sc, float vsa, floa
 // tokens 2q and 2q+1 (reg 0), the same for d + 16 (reg 1), and for tokens
 // 2q+8, 2q+9 (regs 2, 3). M tile (jb, 0) rows g / g+8 are d / d+1; M tile
 // (jb, 1) adds 16.
+// f16 bits of 2^d for an MX block exponent difference d <= 0 (subnormal from
+// -15 down to -24, 0 below).
+__device__ __forceinline__ uint32_t f16_pow2(int d) {
+  if (d >= -14) return static_cast<uint32_t>(d + 15) << 10;
+  if (d >= -24) return 1u << (d + 24);
+  return 0u;
+}
+
+// With vmx (MXFP8 V): vmw = this lane's words of its token's E8M0 codes
+// (lanes 16 + r: token r of the tile, byte g = block g), E = the tile's
+// largest code: each decoded V pair of tokens (2qd, 2qd+1) and (2qd+8,
+// 2qd+9) in 32-entry block jb is multiplied by 2^(code - E), exactly (the
+// tile's 2^(E - 127) goes through P as its V scale).
 template <int D, bool VCVT>
 __device__ __forceinline__ void tile_pv(Acc<D>& a, uint32_t sv, const uint32_t (&voff)[4],
                                         const uint32_t (&bh)[2], const uint32_t (&bl)[2], int tok0,
-                                        int t0, int t1, bool page_ok, bool full, int qd) {
+                                        int t0, int t1, bool page_ok, bool full, int qd,
+                                        bool vmx = false, const uint32_t* vmw = nullptr,
+                                        int E = 0) {
+  uint32_t wa0 = 0u, wa1 = 0u, wb0 = 0u, wb1 = 0u;
   uint32_t vmask_lo = ~0u, vmask_hi = ~0u;
   if (VCVT && !full) {
     // with the hardware cvt a masked row must be zeroed (a NaN byte times
@@ -732,6 +766,33 @@ __device__ __forceinline__ void tile_pv(Acc<D>& a, uint32_t sv, const uint32_t (
       e1 = e4m3x2_b13_to_f16x2(vw.y);
       e2 = e4m3x2_b02_to_f16x2(vw.w);
       e3 = e4m3x2_b13_to_f16x2(vw.w);
+    }
+    if (vmx) {
+      if ((jb & 3) == 0) {
+        const uint32_t w = vmw[jb >> 2];
+        wa0 = __shfl_sync(0xffffffffu, w, 16 + 2 * qd);
+        wa1 = __shfl_sync(0xffffffffu, w, 17 + 2 * qd);
+        wb0 = __shfl_sync(0xffffffffu, w, 24 + 2 * qd);
+        wb1 = __shfl_sync(0xffffffffu, w, 25 + 2 * qd);
+      }
+      const int sh = 8 * (jb & 3);
+      const uint32_t fa = f16_pow2(static_cast<int>((wa0 >> sh) & 0xFFu) - E) |
+                          (f16_pow2(static_cast<int>((wa1 >> sh) & 0xFFu) - E) << 16);
+      const uint32_t fb = f16_pow2(static_cast<int>((wb0 >> sh) & 0xFFu) - E) |
+                          (f16_pow2(static_cast<int>((wb1 >> sh) & 0xFFu) - E) << 16);
+      auto mul = [](uint32_t x, uint32_t f) -> uint32_t {
+        const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&x),
+                                  *reinterpret_cast<const __half2*>(&f));
+        return *reinterpret_cast<const uint32_t*>(&r);
+      };
+      a0 = mul(a0, fa);
+      a1 = mul(a1, fa);
+      e0 = mul(e0, fa);
+      e1 = mul(e1, fa);
+      a2 = mul(a2, fb);
+      a3 = mul(a3, fb);
+      e2 = mul(e2, fb);
+      e3 = mul(e3, fb);
     }
     mma16816(a.O[jb][0], a0, a1, a2, a3, bh[0], bh[1]);
     mma16816(a.O[jb][0], a0, a1, a2, a3, bl[0], bl[1]);
@@ -962,7 +1023,7 @@ __device__ __forceinline__ float warp_token_scale(const float (&x)[PER]) {
 template <int D, bool TOK>
 __device__ __forceinline__ void append_new_token(const DecodeParams& p, int b, int kvh, bool store,
                                               int page, int slot, int r, uint32_t sk, uint32_t sv,
-                                              float& ks, float& vs) {
+                                              float& ks, float& vs, uint32_t* vcode = nullptr) {
   constexpr int PER = D / 32;  // 2, 4, 8 or 16 bytes per lane
   const int lane = threadIdx.x & 31;
   const int d0 = lane * PER;
@@ -983,16 +1044,36 @@ __device__ __forceinline__ void append_new_token(const DecodeParams& p, int b, i
 #pragma unroll
       for (int i = 0; i < PER; ++i) m = fmaxf(m, fabsf(xk[i]));
       for (int o = 1; o < lpg; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      ks = m == 0.f ? 1.f : __fdiv_rn(m, 448.f);
-      if (store && (lane & (lpg - 1)) == 0)
-        p.ksw[(int64_t)page * p.ks_sp + (int64_t)slot * p.ks_st + (int64_t)kvh * p.ks_sh +
-              (int64_t)(lane / lpg) * p.ks_sg] = ks;
+      const int64_t so = (int64_t)page * p.ks_sp + (int64_t)slot * p.ks_st + (int64_t)kvh * p.ks_sh +
+                         (int64_t)(lane / lpg) * p.ks_sg;
+      if (p.k_mx) {  // MXFP8: the block's E8M0 code (k_groups = D / 32)
+        const uint32_t c = mx_code(m);
+        ks = e8m0_to_f32(c);
+        if (store && (lane & (lpg - 1)) == 0) reinterpret_cast<uint8_t*>(p.ksw)[so] = c;
+      } else {
+        ks = m == 0.f ? 1.f : __fdiv_rn(m, 448.f);
+        if (store && (lane & (lpg - 1)) == 0) p.ksw[so] = ks;
+      }
     } else if (p.k_tok) {
       ks = warp_token_scale<PER>(xk);
       if (store && lane == 0)
         p.ksw[(int64_t)page * p.ks_sp + (int64_t)slot * p.ks_st + (int64_t)kvh * p.ks_sh] = ks;
     }
-    if (p.v_tok) {
+    if (p.v_mx) {
+      // MXFP8 V: the 1024 / D lanes of a 32-entry block agree on its code
+      constexpr int LPB = 1024 / D;
+      float m = 0.f;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) m = fmaxf(m, fabsf(xv[i]));
+#pragma unroll
+      for (int o = 1; o < LPB; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const uint32_t c = mx_code(m);
+      vs = e8m0_to_f32(c);
+      if (vcode) *vcode = c;
+      if (store && (lane & (LPB - 1)) == 0)
+        reinterpret_cast<uint8_t*>(p.vsw)[(int64_t)page * p.vs_sp + (int64_t)slot * p.vs_st +
+                                          (int64_t)kvh * p.vs_sh + (int64_t)(lane / LPB) * p.vs_sg] = c;
+    } else if (p.v_tok) {
       vs = warp_token_scale<PER>(xv);
       if (store && lane == 0)
         p.vsw[(int64_t)page * p.vs_sp + (int64_t)slot * p.vs_st + (int64_t)kvh * p.vs_sh] = vs;
@@ -1237,11 +1318,13 @@ __device__ bool prop_assign(const DecodeParams& p, int* scratch, int* red, int h
 // views, dims (head-dim bytes within a 128-byte block, slot, 128-byte block,
 // KV head, page), box (min(D,128), 16, max(1, D/128), 1, 1). TOK: the scales
 // are read per token (one per stored token and KV head) instead of per page.
-template <int D, int KM, bool VCVT, bool TOK>
+template <int D, int KM, bool VCVT, int SC>
 __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
     decode_tma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
   using C = Cfg<D>;
+  constexpr bool TOK = SC >= 1;  // scales read per stored token
+  constexpr bool VMX = SC == 2;  // V in MXFP8 (E8M0 block scales)
   constexpr int KB = D / 16;  // k16 blocks of the QK contraction
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base for the swizzled tiles
@@ -1582,11 +1665,34 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
     const int r = lane & 15;
     const int t = (tile_first + warp + C::NW * j) * kTileTokens + r;
     if (e < 0 || t < t0 || t >= t1 || (lane < 16 && p.k_groups > 1)) return 0.f;
+    if (VMX && lane >= 16) return 1.f;  // attended; the tile's MX scale comes later
     const int64_t slot = (e & 15) * kTileTokens + r;
     return lane < 16 ? __ldg(ksbase + (int64_t)(e >> 4) * p.ks_sp + slot * p.ks_st)
                      : __ldg(vsbase + (int64_t)(e >> 4) * p.vs_sp + slot * p.vs_st);
   };
   float tsc_next = 0.f;
+  // MXFP8 V (VMX): lane 16 + r holds the D / 32 E8M0 codes of token r of a
+  // tile in VW words (byte g = block g; 0 for a token outside the keys), the
+  // next tile's loaded while this one is attended.
+  constexpr int VW = VMX ? (D / 32 + 3) / 4 : 1;
+  const uint8_t* vs8 = reinterpret_cast<const uint8_t*>(p.vs) + (int64_t)kvh * p.vs_sh;
+  uint32_t vmw[VW], vmw_next[VW];
+#pragma unroll
+  for (int k = 0; k < VW; ++k) vmw[k] = vmw_next[k] = 0u;
+  auto vmx_load = [&](int j, uint32_t (&w)[VW]) {
+#pragma unroll
+    for (int k = 0; k < VW; ++k) w[k] = 0u;
+    if (!VMX || lane < 16) return;
+    const int e = went[j];
+    const int r = lane - 16;
+    const int t = (tile_first + warp + C::NW * j) * kTileTokens + r;
+    if (e < 0 || t < t0 || t >= t1) return;
+    const uint8_t* src = vs8 + (int64_t)(e >> 4) * p.vs_sp +
+                         (int64_t)((e & 15) * kTileTokens + r) * p.vs_st;
+#pragma unroll
+    for (int g = 0; g < D / 32; ++g)
+      w[g >> 2] |= static_cast<uint32_t>(__ldg(src + (int64_t)g * p.vs_sg)) << (8 * (g & 3));
+  };
   // Sub-row K groups (TOK, k_groups = G > 1, G <= D / 16): the tile's
   // 16 x G K scales, entry i = 16-token row r = i / G, group g = i % G; lane l
   // loads entries l + 32 m (m < G / 2 <= GKN) of the next tile into gk_next and, when the tile
@@ -1605,8 +1711,11 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
       float v = 0.f;
       if (e >= 0 && i < 16 * kg) {
         const int r = i >> kg_log2, g = i & (kg - 1);
-        v = __ldg(ksbase + (int64_t)(e >> 4) * p.ks_sp +
-                  (int64_t)((e & 15) * kTileTokens + r) * p.ks_st + (int64_t)g * p.ks_sg);
+        const int64_t off = (int64_t)(e >> 4) * p.ks_sp +
+                            (int64_t)((e & 15) * kTileTokens + r) * p.ks_st + (int64_t)g * p.ks_sg;
+        v = p.k_mx ? e8m0_to_f32(__ldg(reinterpret_cast<const uint8_t*>(p.ks) +
+                                       (int64_t)kvh * p.ks_sh + off))
+                   : __ldg(ksbase + off);
       }
       o[m] = v;
     }
@@ -1616,6 +1725,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
     if (my_tiles > 0) {
       tsc_next = tok_scale(0);
       if (kg > 1) group_scales(0, gk_next);
+      if constexpr (VMX) vmx_load(0, vmw_next);
     }
   }
 
@@ -1706,6 +1816,11 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
     if constexpr (TOK) {
       float tsc = tsc_next;
       if (j + 1 < my_tiles) tsc_next = tok_scale(j + 1);
+      if constexpr (VMX) {
+#pragma unroll
+        for (int k = 0; k < VW; ++k) vmw[k] = vmw_next[k];
+        if (j + 1 < my_tiles) vmx_load(j + 1, vmw_next);
+      }
       if (kg > 1) {
         float gk[GKN];
 #pragma unroll
@@ -1722,8 +1837,9 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
       if (has_new) {
         const int r = L - 1 - tok0;
         float ks = __shfl_sync(0xffffffffu, tsc, r), vs = __shfl_sync(0xffffffffu, tsc, 16 + r);
+        uint32_t vcode = 0u;
         append_new_token<D, true>(p, b, kvh, hg == 0, went[j] >> 4,
-                                  (went[j] & 15) * kTileTokens + r, r, sk, sv, ks, vs);
+                                  (went[j] & 15) * kTileTokens + r, r, sk, sv, ks, vs, &vcode);
         if (kg > 1) {
           const int lpg = 32 / kg;  // lanes of one K group in the append
           if ((lane & (lpg - 1)) == 0) group_row(r)[lane / lpg] = ks;
@@ -1731,25 +1847,49 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
           tsc = ks;
         }
         if (lane == 16 + r) tsc = vs;
+        if constexpr (VMX) {
+          // the new token's block codes into the words of lane 16 + r
+#pragma unroll
+          for (int g = 0; g < D / 32; ++g) {
+            const uint32_t c = __shfl_sync(0xffffffffu, vcode, g * (1024 / D));
+            if (lane == 16 + r) {
+              if ((g & 3) == 0) vmw[g >> 2] = 0u;
+              vmw[g >> 2] |= c << (8 * (g & 3));
+            }
+          }
+        }
         __syncwarp();
+      }
+      int vE = 0;  // MXFP8 V: the tile's largest block code of an attended token
+      if constexpr (VMX) {
+        int mine = -1;
+        if (lane >= 16 && tsc != 0.f) {
+#pragma unroll
+          for (int g = 0; g < D / 32; ++g)
+            mine = max(mine, static_cast<int>((vmw[g >> 2] >> (8 * (g & 3))) & 0xFFu));
+        }
+        vE = __reduce_max_sync(0xffffffffu, mine);
+        const float vtile = vE >= 0 ? e8m0_to_f32(static_cast<uint32_t>(vE)) : 0.f;
+        if (lane >= 16) tsc = tsc != 0.f ? vtile : 0.f;
       }
       const float vsa = __shfl_sync(0xffffffffu, tsc, 16 + grp);
       const float vsb = __shfl_sync(0xffffffffu, tsc, 24 + grp);
       const float vabs = warp_max(lane >= 16 ? fabsf(tsc) : 0.f);
+      float4 sc;
       if (kg > 1) {
-        const float4 sc = tile_scores_groups<D, (KM == 0 ? 0 : 1)>(
+        sc = tile_scores_groups<D, (KM == 0 ? 0 : 1)>(
             qfr, sk, koff, group_row(grp), group_row(grp + 8), kb_log2, score_base, tok0, t0, t1,
             page_ok, full, grp);
-        softmax_rescale<D>(acc, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), vabs);
-        uint32_t bh[2], bl[2];
-        tile_probs<D>(acc, sc, vsa, vsb, bh, bl);
-        tile_pv<D, VCVT>(acc, sv, voff, bh, bl, tok0, t0, t1, page_ok, full, qd);
       } else {
         const float kfa = score_base * __shfl_sync(0xffffffffu, tsc, grp);
         const float kfb = score_base * __shfl_sync(0xffffffffu, tsc, grp + 8);
-        attend_tile<D, KM, VCVT>(acc, qfr, sk, sv, koff, voff, kfa, kfb, vsa, vsb, vabs, tok0,
-                                   t0, t1, page_ok, full, grp, qd);
+        sc = tile_scores<D, (KM == 0 ? 0 : 1)>(qfr, sk, koff, kfa, kfb, tok0, t0, t1, page_ok,
+                                               full, grp);
       }
+      softmax_rescale<D>(acc, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), vabs);
+      uint32_t bh[2], bl[2];
+      tile_probs<D>(acc, sc, vsa, vsb, bh, bl);
+      tile_pv<D, VCVT>(acc, sv, voff, bh, bl, tok0, t0, t1, page_ok, full, qd, VMX, vmw, vE);
     } else {
       const float kfac = score_base * wks[j];
       float ks = wks[j], vs = wvs[j];
@@ -1928,9 +2068,13 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
 
 // Per-token-per-head scale of one bf16 row of n values (stride sd): max |x| /
 // 448 in IEEE f32, NaN entries skipped (fmaxf), 1 for an all-zero row.
-__device__ float row_token_scale(const uint16_t* x, int64_t sd, int n) {
+__device__ float row_amax(const uint16_t* x, int64_t sd, int n) {
   float m = 0.f;
   for (int i = 0; i < n; ++i) m = fmaxf(m, fabsf(bf16_bits_to_float(x[(int64_t)i * sd])));
+  return m;
+}
+__device__ float row_token_scale(const uint16_t* x, int64_t sd, int n) {
+  const float m = row_amax(x, sd, n);
   return m == 0.f ? 1.f : __fdiv_rn(m, 448.f);
 }
 
@@ -1963,7 +2107,14 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
   // A per-token scale is the new token's own: every thread of the row
   // derives it from the row's D values, the row's first thread stores it.
   float ks = 0.f, ks1 = 0.f;  // K scales of entries d and d + 1
-  if (p.k_tok && p.k_groups > 1) {
+  if (p.k_mx) {
+    // MXFP8: the 32-entry block of d and d + 1 (d is even): its E8M0 code,
+    // stored by the thread holding the block's first entry
+    const int blk = d / 32;
+    const uint32_t c = mx_code(row_amax(knr + (int64_t)blk * 32 * p.kn_sd, p.kn_sd, 32));
+    ks = ks1 = e8m0_to_f32(c);
+    if (d == blk * 32) reinterpret_cast<uint8_t*>(p.ksw)[kso + (int64_t)blk * p.ks_sg] = c;
+  } else if (p.k_tok && p.k_groups > 1) {
     // sub-row groups of gs entries: each entry's group scale; the thread
     // holding a group's first entry stores it
     const int gs = p.D / p.k_groups;
@@ -1976,8 +2127,16 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
     ks = ks1 = p.k_tok ? row_token_scale(knr, p.kn_sd, p.D) : p.ks[kso];
     if (d == 0 && p.k_tok) p.ksw[kso] = ks;
   }
-  const float vs = p.v_tok ? row_token_scale(vnr, p.vn_sd, p.D) : p.vs[vso];
-  if (d == 0 && p.v_tok) p.vsw[vso] = vs;
+  float vs;
+  if (p.v_mx) {
+    const int blk = d / 32;
+    const uint32_t c = mx_code(row_amax(vnr + (int64_t)blk * 32 * p.vn_sd, p.vn_sd, 32));
+    vs = e8m0_to_f32(c);
+    if (d == blk * 32) reinterpret_cast<uint8_t*>(p.vsw)[vso + (int64_t)blk * p.vs_sg] = c;
+  } else {
+    vs = p.v_tok ? row_token_scale(vnr, p.vn_sd, p.D) : p.vs[vso];
+    if (d == 0 && p.v_tok) p.vsw[vso] = vs;
+  }
   const uint16_t* kn = knr + (int64_t)d * p.kn_sd;
   const uint16_t* vn = vnr + (int64_t)d * p.vn_sd;
   const float k0 = __fdiv_rn(bf16_bits_to_float(kn[0]), ks);
@@ -1999,7 +2158,7 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
 // ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
-template <int D, int KM, bool VCVT, bool TOK>
+template <int D, int KM, bool VCVT, int SC>
 static cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap& tmk,
                                    const CUtensorMap& tmv, cudaStream_t s) {
   // The shared-memory opt-in is a per-device function attribute: set it once
@@ -2011,43 +2170,51 @@ static cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap& tmk
   if (e != cudaSuccess) return e;
   const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
   if (!bit || !(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(decode_tma_kernel<D, KM, VCVT, TOK>,
+    e = cudaFuncSetAttribute(decode_tma_kernel<D, KM, VCVT, SC>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
   const dim3 grid = p.prop ? dim3(p.Hkv * p.head_groups, p.nbx, 1)
                            : dim3(p.Hkv * p.head_groups, p.B, p.num_splits);
-  decode_tma_kernel<D, KM, VCVT, TOK><<<grid, Cfg<D>::NT, smem, s>>>(p, tmk, tmv);
+  decode_tma_kernel<D, KM, VCVT, SC><<<grid, Cfg<D>::NT, smem, s>>>(p, tmk, tmv);
   return cudaGetLastError();
 }
 
 // K mode 2 (E4M3 MMAs) is built with the cvt decode of V and without
 // per-token scales; other combinations take mode 1 for K. Mode 3 is the fp8
-// compute path (V is not decoded), page and head scales only.
-template <int D, bool TOK>
+// compute path (V is not decoded), page and head scales only. SC: 0 = page
+// or head scales, 1 = per-token scales (K sub-row groups, MXFP8 K), 2 = MXFP8
+// V (built with the cvt decodes only).
+template <int D, int SC>
 static cudaError_t launch_decode_kv(const DecodeParams& p, const CUtensorMap& tmk,
                                     const CUtensorMap& tmv, int k_mode, bool v_cvt,
                                     cudaStream_t s) {
-  if constexpr (!TOK) {
-    if (k_mode == 3) return launch_decode_d<D, 3, true, false>(p, tmk, tmv, s);
-    if (k_mode == 2 && v_cvt) return launch_decode_d<D, 2, true, false>(p, tmk, tmv, s);
-  } else {
+  if constexpr (SC == 2) {
     if (k_mode == 3) return cudaErrorInvalidValue;  // refused by the host first
+    return launch_decode_d<D, 1, true, 2>(p, tmk, tmv, s);
+  } else {
+    if constexpr (SC == 0) {
+      if (k_mode == 3) return launch_decode_d<D, 3, true, 0>(p, tmk, tmv, s);
+      if (k_mode == 2 && v_cvt) return launch_decode_d<D, 2, true, 0>(p, tmk, tmv, s);
+    } else {
+      if (k_mode == 3) return cudaErrorInvalidValue;  // refused by the host first
+    }
+    if (k_mode >= 1)
+      return v_cvt ? launch_decode_d<D, 1, true, SC>(p, tmk, tmv, s)
+                   : launch_decode_d<D, 1, false, SC>(p, tmk, tmv, s);
+    return v_cvt ? launch_decode_d<D, 0, true, SC>(p, tmk, tmv, s)
+                 : launch_decode_d<D, 0, false, SC>(p, tmk, tmv, s);
   }
-  if (k_mode >= 1)
-    return v_cvt ? launch_decode_d<D, 1, true, TOK>(p, tmk, tmv, s)
-                 : launch_decode_d<D, 1, false, TOK>(p, tmk, tmv, s);
-  return v_cvt ? launch_decode_d<D, 0, true, TOK>(p, tmk, tmv, s)
-               : launch_decode_d<D, 0, false, TOK>(p, tmk, tmv, s);
 }
 
 template <int D>
 static cudaError_t launch_decode_dt(const DecodeParams& p, const CUtensorMap& tmk,
                                     const CUtensorMap& tmv, int k_mode, bool v_cvt,
                                     cudaStream_t s) {
-  if (p.k_tok || p.v_tok) return launch_decode_kv<D, true>(p, tmk, tmv, k_mode, v_cvt, s);
-  return launch_decode_kv<D, false>(p, tmk, tmv, k_mode, v_cvt, s);
+  if (p.v_mx) return launch_decode_kv<D, 2>(p, tmk, tmv, k_mode, v_cvt, s);
+  if (p.k_tok || p.v_tok) return launch_decode_kv<D, 1>(p, tmk, tmv, k_mode, v_cvt, s);
+  return launch_decode_kv<D, 0>(p, tmk, tmv, k_mode, v_cvt, s);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
@@ -2067,9 +2234,9 @@ static int blocks_per_sm_d() {
   int c = cached.load();
   if (c >= 0) return c;
   int n = 0;
-  if (cudaFuncSetAttribute(decode_tma_kernel<D, 1, true, false>,
+  if (cudaFuncSetAttribute(decode_tma_kernel<D, 1, true, 0>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tma_kernel<D, 1, true, false>, Cfg<D>::NT,
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tma_kernel<D, 1, true, 0>, Cfg<D>::NT,
                                                     Cfg<D>::SMEM) != cudaSuccess) {
     cudaGetLastError();
     return Cfg<D>::MIN_BLOCKS;  // no device: do not cache the guess

@@ -95,6 +95,9 @@ def _call(F, a):
     (dict(ks=torch.ones(6, 16, 2, 3)), -5),                                  # groups not a power of 2
     (dict(vs=torch.ones(6, 16, 2, 2)), -5),                                  # V sub-row groups
     (dict(ks=torch.ones(6, 16, 3, 2)), -3),
+    (dict(ks=torch.zeros(6, 16, 2, 5, dtype=torch.uint8)), -3),             # MX: D / 32 blocks
+    (dict(vs=torch.zeros(6, 16, 2, dtype=torch.uint8)), -3),                 # MX: 4-D only
+    (dict(vs=torch.zeros(6, 8, 2, 4, dtype=torch.uint8)), -3),               # MX: ps
     (dict(sinks=torch.zeros(7)), -3),
     (dict(table=torch.zeros(3, 3, dtype=torch.int32)), -3),
     (dict(lens=torch.zeros(2, dtype=torch.int64)), -2),
@@ -305,3 +308,43 @@ def test_planner_proportional_splits(F):
     finally:
         F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
         F.fp8pd_set_option(F.OPT_SCHEDULE, 0)
+
+
+def test_partial_and_combine_validation(F):
+    """The context-parallel entry points refuse bad arguments before any
+    launch: the partial call as the attention call plus its own outputs and
+    key ranges; the combine call its shapes, layout and rank count."""
+    a = _args()
+    kw = dict(window=0, sm_scale=0.1, stream=0)
+
+    def partial(**over):
+        b = dict(a, kr=torch.zeros(2, 2, dtype=torch.int32), po=torch.zeros(2, 8, 128),
+                 pml=torch.zeros(2, 8, 2))
+        b.update(over)
+        try:
+            F.fp8_paged_decode_attention_partial(b["q"], b["k"], b["v"], b["ks"], b["vs"], b["table"],
+                                                 b["lens"], b["kr"], part_o=b["po"],
+                                                 part_ml=b["pml"], **kw)
+        except F.Fp8pdError as e:
+            return e.status
+        return 0
+    assert partial(kr=torch.zeros(2, 3, dtype=torch.int32)) == -3
+    assert partial(kr=torch.zeros(2, 2, dtype=torch.int64)) == -2
+    assert partial(pml=torch.zeros(2, 8, 3)) == -3
+    assert partial(po=torch.zeros(2, 16, 128)[:, ::2]) == -4          # not contiguous
+    assert partial(q=torch.zeros(2, 8, 128)) == -2
+
+    def combine(o, ml, sinks=None, out=None):
+        try:
+            F.fp8pd_combine_partials(o, ml, sinks=sinks, out=out, stream=0)
+        except F.Fp8pdError as e:
+            return e.status
+        return 0
+    o, ml = torch.zeros(3, 2, 8, 128), torch.zeros(3, 2, 8, 2)
+    assert combine(o, ml[:2]) == -3
+    assert combine(o, ml, out=torch.zeros(2, 8, 64)) == -3
+    assert combine(o, ml, sinks=torch.zeros(5)) == -3
+    assert combine(o.double(), ml) == -2
+    assert combine(o[:, :, :, :126], ml) == -5                        # D % 4
+    assert combine(torch.zeros(1025, 1, 1, 4), torch.zeros(1025, 1, 1, 2)) == -10
+    assert F.lib.fp8pd_combine_partials(None, None, None, None, None) == -1

@@ -126,6 +126,7 @@ def test_bench_refuses_more_gpus_than_it_sees():
     ("tiny", {}), ("llama", dict(B=5)), ("gptoss_w128", dict(B=3, seq_len=700)),
     ("gptoss_full", dict(B=2, seq_len=300)), ("mixed", dict(B=3, seq_len=(100, 1500))),
     ("long_b1", dict(seq_len=3000)), ("llama", dict(B=3, scale_mode="token", k_groups=4)),
+    ("mixed", dict(B=2, seq_len=(100, 900), scale_mode="mx")),
 ])
 def test_bench_bytes_from_the_spec_equal_the_workload_count(name, overrides):
     """The reference arm's config states the bytes per step without building

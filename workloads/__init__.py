@@ -44,7 +44,8 @@ class Spec:
     ps: int
     layers: tuple                       # tuple[LayerSpec, ...]; >1 = layers sharing one pool
     seq_len: int | tuple = 256          # int, or (lo, hi) inclusive uniform range per sequence
-    scale_mode: str = "head"            # "head": [Hkv]; "page": [num_pages, Hkv]; "token": [num_pages, ps, Hkv]
+    scale_mode: str = "head"            # "head": [Hkv]; "page": [num_pages, Hkv]; "token": [num_pages, ps, Hkv];
+                                        # "mx": MXFP8, uint8 E8M0 [num_pages, ps, Hkv, D / 32] for K and V
     k_groups: int = 1                   # "token" only: K scales [num_pages, ps, Hkv, k_groups] when > 1
     dist: str = "normal"                # "normal": N(0,1); "normal2_outliers": N(0,2), 1% x20
     sinks: bool = False
@@ -225,6 +226,37 @@ def make_case(name_or_spec, device="cpu", chunk_pages: int = 1024, **overrides) 
         for which, pool in ((0, k_pool), (1, v_pool)):
             # pass 1: scales from the values (including the token to append)
             G = spec.k_groups if (spec.scale_mode == "token" and which == 0) else 1
+            if spec.scale_mode == "mx":
+                # MXFP8: per 32-entry block, 2^(floor(log2 amax) - 8) as an E8M0 code
+                # (127 for an all-zero block), codes the clamped E4M3 cast of x / scale
+                view = torch.as_strided(pool, (total_pages, spec.ps, L.Hkv, L.D),
+                                        (page_stride, L.Hkv * L.D, L.D, 1))
+                codes_sc = torch.full((total_pages, spec.ps, L.Hkv, L.D // 32), 127,
+                                      dtype=torch.uint8, device=device)
+                new = torch.zeros(spec.B, L.Hkv, L.D, dtype=torch.bfloat16, device=device)
+                for p0 in range(0, total_pages, chunk_pages):
+                    p1 = min(total_pages, p0 + chunk_pages)
+                    x = page_values_bf16_new(page_values(p0, p1, which), p0, p1)
+                    xb = x.view(p1 - p0, spec.ps, L.Hkv, L.D // 32, 32)
+                    amax = xb.abs().amax(dim=-1)
+                    e = torch.frexp(amax).exponent.to(torch.int32) - 1 - 8 + 127
+                    c = torch.where(amax > 0, e.clamp(0, 254), torch.full_like(e, 127))
+                    sc = torch.pow(2.0, (c - 127).to(torch.float64)).float()
+                    quot = (xb / sc[..., None]).clamp(-E4M3_MAX, E4M3_MAX).reshape(x.shape)
+                    codes = quot.to(torch.float8_e4m3fn).view(torch.uint8)
+                    if spec.append:
+                        for b in range(spec.B):
+                            p = int(append_page[b])
+                            if p0 <= p < p1:
+                                s = int(cache_lens[b] % spec.ps)
+                                new[b] = x[p - p0, s].to(torch.bfloat16)
+                                codes[p - p0, s] = 0
+                    view[p0:p1] = codes
+                    codes_sc[p0:p1] = c.to(torch.uint8)
+                views.append(view)
+                scales.append(codes_sc)
+                news.append(new if spec.append else None)
+                continue
             if spec.scale_mode == "head":
                 amax = torch.zeros(L.Hkv, device=device)
             elif spec.scale_mode == "token" and G > 1:
@@ -302,7 +334,9 @@ def algorithmic_bytes(case: Case, layer: int = 0) -> int:
             tbl += 4 * ((Lb - 1) // ps - lo // ps + 1)
     q = L.q.numel() * 2
     # per-token scales: 4 bytes per attended token, KV head and group, for K and for V
-    tok_scales = sum(kv // L.spec.D * 2 * (sc.shape[3] if sc.dim() == 4 else 1)
+    # (MXFP8: one byte per 32-entry block)
+    tok_scales = sum(kv // L.spec.D // 2 * (sc.shape[3] if sc.dim() == 4 else 1) *
+                     (1 if sc.dtype == torch.uint8 else 4)
                      for sc in (L.k_scale, L.v_scale) if sc.dim() >= 3)
     return int(kv + q + tbl + tok_scales)
 
