@@ -335,6 +335,9 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
 #ifndef FP8PD_NW_D256
 #define FP8PD_NW_D256 4
 #endif
+#ifndef FP8PD_NW_D512
+#define FP8PD_NW_D512 4
+#endif
 
 // ---------------------------------------------------------------------------
 // Shared-memory tile layout. The TMA writes one 16-token tile of one KV head
@@ -355,7 +358,7 @@ __device__ __forceinline__ uint32_t tile_off(int r, int b) {
 
 template <int D>
 struct Cfg {
-  static constexpr int NW = (D == 64) ? FP8PD_NW_D64 : (D == 128) ? FP8PD_NW_D128 : (D == 256) ? FP8PD_NW_D256 : 4;  // warps per block
+  static constexpr int NW = (D == 64) ? FP8PD_NW_D64 : (D == 128) ? FP8PD_NW_D128 : (D == 256) ? FP8PD_NW_D256 : FP8PD_NW_D512;  // warps per block
   static constexpr int NT = NW * 32;                                  // threads per block
   static constexpr int NS = (D == 64) ? FP8PD_NS_D64 : (D == 128) ? FP8PD_NS_D128 : (D == 256) ? FP8PD_NS_D256 : FP8PD_NS_D512;  // ring stages per warp
   static constexpr bool PAIR = (D == 64) && FP8PD_PAIR_D64;           // two tiles per softmax step
@@ -488,6 +491,7 @@ template <int D>
 struct Acc {
   float O[D / 32][2][4];
   float m0, m1, l0, l1, vref, inv_vref;
+  float x0, x1;  // lazy maxima: this lane's largest scores of heads 2qd / 2qd+1 so far
   __device__ __forceinline__ void reset() {
 #pragma unroll
     for (int jb = 0; jb < D / 32; ++jb)
@@ -495,7 +499,7 @@ struct Acc {
       for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int c = 0; c < 4; ++c) O[jb][h][c] = 0.f;
-    m0 = m1 = -CUDART_INF_F;
+    m0 = m1 = x0 = x1 = -CUDART_INF_F;
     l0 = l1 = 0.f;
     vref = inv_vref = 0.f;
   }
@@ -647,8 +651,22 @@ __device__ __forceinline__ float4 tile_scores_groups(const QFrag& qfr, uint32_t 
 // lane's tokens are (tm0, tm1) and whose largest |V scale| is vabs: the
 // running maxima and the V reference scale grow, and l and O are rescaled,
 // only when one of them changes (warp-uniform test).
-template <int D>
+// LAZY: the reference maxima m0 / m1 move only when some score exceeds them
+// by more than kLazyLog2 (or the V scale grows), so most tiles skip the
+// cross-lane maximum; P = 2^(s - m) then stays below 2^kLazyLog2, which the
+// f16 hi + lo operands hold exactly as before. Each lane keeps its own true
+// maxima (x0 / x1); lazy_finish moves l and O onto them once at the end.
+constexpr float kLazyLog2 = 8.f;
+
+template <int D, bool LAZY = false>
 __device__ __forceinline__ void softmax_rescale(Acc<D>& a, float tm0, float tm1, float vabs) {
+  if constexpr (LAZY) {
+    a.x0 = fmaxf(a.x0, tm0);
+    a.x1 = fmaxf(a.x1, tm1);
+    if (!(vabs > a.vref) &&
+        !__any_sync(0xffffffffu, (tm0 > a.m0 + kLazyLog2) || (tm1 > a.m1 + kLazyLog2)))
+      return;
+  }
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, o));
@@ -679,6 +697,34 @@ __device__ __forceinline__ void softmax_rescale(Acc<D>& a, float tm0, float tm1,
       a.inv_vref = 1.f / vabs;
     }
   }
+}
+
+// End of a lazy stream: the exact per-head maxima of this warp's scores
+// (reduced over the 8 lanes of a head pair) replace the reference maxima, l
+// and O scaled to match, so a partial's m is the maximum score as documented.
+template <int D>
+__device__ __forceinline__ void lazy_finish(Acc<D>& a) {
+  float x0 = a.x0, x1 = a.x1;
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, o));
+    x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, o));
+  }
+  const float c0 = (x0 > a.m0) ? fast_exp2(a.m0 - x0) : 1.f;
+  const float c1 = (x1 > a.m1) ? fast_exp2(a.m1 - x1) : 1.f;
+  a.l0 *= c0;
+  a.l1 *= c1;
+#pragma unroll
+  for (int jb = 0; jb < D / 32; ++jb)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      a.O[jb][h][0] *= c0;
+      a.O[jb][h][1] *= c1;
+      a.O[jb][h][2] *= c0;
+      a.O[jb][h][3] *= c1;
+    }
+  a.m0 = fmaxf(a.m0, x0);
+  a.m1 = fmaxf(a.m1, x1);
 }
 
 // P of one tile: exp2 of the scores against the running maxima, added to
@@ -897,7 +943,7 @@ __device__ __forceinline__ void attend_tile(Acc<D>& a, const QFrag& qfr, uint32_
                                             int grp, int qd, float2 hf = make_float2(1.f, 1.f)) {
   const float4 sc =
       tile_scores<D, KM>(qfr, sk, koff, kfa, kfb, tok0, t0, t1, page_ok, full, grp, hf);
-  softmax_rescale<D>(a, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), vabs);
+  softmax_rescale<D, KM != 3>(a, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), vabs);
   if constexpr (KM == 3) {
     const uint32_t pb[2] = {tile_probs8<D>(a, sc, vsa, vsb), 0u};
     const uint32_t svv[2] = {sv, sv};
@@ -926,7 +972,7 @@ __device__ __forceinline__ void attend_pair(Acc<D>& a, const QFrag& qfr, const u
                                          page_ok[0], full[0], grp, hf);
   const float4 s1 = tile_scores<D, KM>(qfr, sk[1], koff, kfac[1], kfac[1], tok0[1], t0, t1,
                                          page_ok[1], full[1], grp, hf);
-  softmax_rescale<D>(a, fmaxf(fmaxf(s0.x, s0.z), fmaxf(s1.x, s1.z)),
+  softmax_rescale<D, KM != 3>(a, fmaxf(fmaxf(s0.x, s0.z), fmaxf(s1.x, s1.z)),
                      fmaxf(fmaxf(s0.y, s0.w), fmaxf(s1.y, s1.w)), fmaxf(fabsf(vs[0]), fabsf(vs[1])));
   if constexpr (KM == 3) {
     // one k32 MMA per 32-byte block covers both tiles' tokens
@@ -1540,8 +1586,9 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
     // pairs per lane and block, all in flight together, parked in the
     // fragment slots they become; the block then agrees on max|q|
 #pragma unroll
-    for (int i = 0; i < KB / C::NW; ++i) {
+    for (int i = 0; i < (KB + C::NW - 1) / C::NW; ++i) {
       const int kb = warp + C::NW * i;
+      if (kb >= KB) break;
       const int d = 16 * kb + 4 * qd;
       uint2 v = make_uint2(0u, 0u);
       if (q_head_ok) {
@@ -1732,7 +1779,9 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
   int stage = 0;
   uint32_t phase = 0;
   int tok0 = (tile_first + warp) * kTileTokens;
-  constexpr bool PAIRS = C::PAIR || KM == 3;  // two tiles per softmax step
+  // two tiles per softmax step: the ring must hold both next to the one being
+  // refilled, so the step needs at least three stages
+  constexpr bool PAIRS = (C::PAIR || KM == 3) && C::NS >= 3;
   if constexpr (PAIRS && !TOK) {
     // Two tiles per step while two are left (one softmax update per 32 keys;
     // the copy into the first tile's stage is issued once its PV is done).
@@ -1886,7 +1935,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
         sc = tile_scores<D, (KM == 0 ? 0 : 1)>(qfr, sk, koff, kfa, kfb, tok0, t0, t1, page_ok,
                                                full, grp);
       }
-      softmax_rescale<D>(acc, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), vabs);
+      softmax_rescale<D, true>(acc, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), vabs);
       uint32_t bh[2], bl[2];
       tile_probs<D>(acc, sc, vsa, vsb, bh, bl);
       tile_pv<D, VCVT>(acc, sv, voff, bh, bl, tok0, t0, t1, page_ok, full, qd, VMX, vmw, vE);
@@ -1903,6 +1952,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
                                  t0, t1, page_ok, full, grp, qd, hf);
     }
   }
+  if constexpr (KM != 3) lazy_finish<D>(acc);
   if (!ok_all) {
     // A copy never completed: leave this warp's result out (its flag is set)
     // and wait, again bounded, for whatever this warp still has in flight.
