@@ -68,6 +68,10 @@ WORKLOAD_TEXT = {
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic_per_launch.txt")
 KERNEL_NAME = {1: "decode_tma_kernel (split kernel, merge in the same launch)",
                3: "decode_tma_kernel (proportional splits, merge in the same launch)"}
+UMMA_NAME = {1: "decode_umma_kernel (tcgen05, TMEM accumulators; split kernel, merge in the same "
+                "launch)",
+             3: "decode_umma_kernel (tcgen05, TMEM accumulators; proportional splits, merge in "
+                "the same launch)"}
 L2_TEXT = ("flushed between timed steps: 256 MiB write, then a 256 MiB read of another buffer "
            "(no dirty lines left), outside the step events")
 
@@ -365,8 +369,8 @@ def time_case(F, case: W.Case, dev, args, flush: L2Flush, steps: int, warmup: in
         app_ms = kt["append_ms"] / kt["append_launches"] if kt["append_launches"] else None
         per_layer.append({"bytes": W.algorithmic_bytes(case, li), "kernel_ms": att_ms,
                           "append_ms": app_ms,
-                          "plan": {k: run[k] for k in ("schedule", "num_splits", "head_groups",
-                                                       "grid_blocks", "combine")}})
+                          "plan": {k: run[k] for k in ("kernel", "schedule", "num_splits",
+                                                       "head_groups", "grid_blocks", "combine")}})
     if F.fp8pd_check_errors() != 0:
         raise RuntimeError("device error word set during the timed region")
     return {"ms_per_step": total_ms / steps, "eager_ms_per_step": eager_ms / steps,
@@ -377,7 +381,8 @@ def time_case(F, case: W.Case, dev, args, flush: L2Flush, steps: int, warmup: in
 def _roofline(entry: dict, peaks: dict, fused: bool, traffic=None) -> dict:
     ms = entry["kernel_ms"]
     achieved = entry["bytes"] / (ms * 1e-3) / 1e9 if ms > 0 else None
-    kernel = KERNEL_NAME.get(entry["plan"]["schedule"], "decode kernel") + \
+    names = UMMA_NAME if entry["plan"].get("kernel") == 2 else KERNEL_NAME
+    kernel = names.get(entry["plan"]["schedule"], "decode kernel") + \
         (", append fused" if fused else "")
     return {"bound": "hbm", "kernel": kernel,
             "achieved": round(achieved, 2) if achieved else None,
@@ -401,6 +406,7 @@ def _set_options(F, args) -> None:
     F.fp8pd_set_option(F.OPT_NUM_SPLITS, args.splits)
     F.fp8pd_set_option(F.OPT_SCHEDULE, args.schedule)
     F.fp8pd_set_option(F.OPT_COMPUTE, 1 if args.compute == "fp8" else 0)
+    F.fp8pd_set_option(F.OPT_KERNEL, args.kernel)
 
 
 def run_ours(args) -> dict | None:
@@ -853,6 +859,9 @@ def build_parser() -> argparse.ArgumentParser:
                          "(q and P rounded once to E4M3; 1.5e-1)")
     ap.add_argument("--schedule", type=int, default=0, choices=[0, 1, 3],
                     help="0 = planner, 1 = uniform splits, 3 = proportional splits")
+    ap.add_argument("--kernel", type=int, default=0, choices=[0, 1, 2],
+                    help="0 = planner's choice, 1 = split kernel (mma.sync), "
+                         "2 = tensor-memory kernel (tcgen05) where it applies")
     return ap
 
 

@@ -33,7 +33,7 @@ __all__ = [
     "fp8_paged_decode_attention_partial", "fp8pd_combine_partials",
     "FLAG_PAGE_OOB", "FLAG_SEQLEN_OOB", "FLAG_POS_OOB", "FLAG_INTERNAL", "OPT_NUM_SPLITS",
     "OPT_SCHEDULE", "OPT_K_DECODE", "OPT_V_DECODE", "OPT_WAIT_POLLS",
-    "OPT_TEST_STALL", "OPT_COMPUTE", "FLAG_TIMEOUT",
+    "OPT_TEST_STALL", "OPT_COMPUTE", "OPT_KERNEL", "FLAG_TIMEOUT",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libfp8pd.so")
@@ -41,7 +41,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "lib
 DTYPE_U8, DTYPE_I32, DTYPE_F32, DTYPE_BF16 = 1, 2, 3, 4
 FLAG_PAGE_OOB, FLAG_SEQLEN_OOB, FLAG_POS_OOB, FLAG_INTERNAL, FLAG_TIMEOUT = 1, 2, 4, 8, 16
 OPT_NUM_SPLITS, OPT_SCHEDULE, OPT_K_DECODE, OPT_V_DECODE = 1, 2, 3, 4
-OPT_WAIT_POLLS, OPT_TEST_STALL, OPT_COMPUTE = 6, 7, 8
+OPT_WAIT_POLLS, OPT_TEST_STALL, OPT_COMPUTE, OPT_KERNEL = 6, 7, 8, 9
 _DTYPES = {torch.uint8: DTYPE_U8, torch.int32: DTYPE_I32, torch.float32: DTYPE_F32,
            torch.bfloat16: DTYPE_BF16}
 
@@ -67,7 +67,8 @@ class RunInfo(ctypes.Structure):
                 ("head_groups", ctypes.c_int32), ("grid_blocks", ctypes.c_int32),
                 ("combine", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("calls", ctypes.c_int64), ("appends", ctypes.c_int64),
-                ("kernel_launches", ctypes.c_int64), ("compute", ctypes.c_int32)]
+                ("kernel_launches", ctypes.c_int64), ("compute", ctypes.c_int32),
+                ("kernel", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:

@@ -32,7 +32,7 @@ thread_local int32_t t_last_cuda_error = 0;
 thread_local fp8pd_run_info t_run_info = {};
 std::atomic<int64_t> g_calls{0}, g_appends{0}, g_launches{0};
 std::atomic<int64_t> g_opt_num_splits{0}, g_opt_schedule{0}, g_opt_k_decode{1}, g_opt_v_decode{1},
-    g_opt_wait_polls{1 << 17}, g_opt_test_stall{0}, g_opt_compute{0};
+    g_opt_wait_polls{1 << 17}, g_opt_test_stall{0}, g_opt_compute{0}, g_opt_kernel{0};
 
 struct Workspace {
   void* ptr = nullptr;
@@ -207,8 +207,26 @@ int device_sms() {
 // many blocks a whole sequence, so a second wave of halves balances better).
 // Needs at most 1,024 sequences; the planner's own choice also needs at least
 // 4 tiles per block slot when every sequence has its table's full length.
+// Whether the tensor-memory kernel runs a call: head dim 64 or 128, page or
+// head scales (no per-token, sub-row or MX scales), f32 compute with the
+// hardware-cvt decodes, no timeout test hook, and FP8PD_OPT_KERNEL not 1.
+constexpr bool kUmmaByDefault = false;
+bool use_umma(int D, bool tok, bool mx, int k_groups) {
+  const int64_t k = g_opt_kernel.load();
+  if (k == 1 || (D != 64 && D != 128) || tok || mx || k_groups > 1) return false;
+  if (g_opt_compute.load() != 0 || g_opt_k_decode.load() != 1 || g_opt_v_decode.load() != 1 ||
+      g_opt_test_stall.load() != 0)
+    return false;
+  return k == 2 || kUmmaByDefault;
+}
+
+// Thread blocks one SM holds for the kernel that will run.
+int blocks_per_sm(int D, bool umma) {
+  return umma ? fp8pd::decode_umma_blocks_per_sm(D) : fp8pd::decode_blocks_per_sm(D);
+}
+
 bool plan_proportional(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window,
-                       Plan* plan) {
+                       Plan* plan, bool umma) {
   if (g_opt_num_splits.load() > 0 || B > fp8pd::kPropMaxBatch) return false;
   const int G = Hq / Hkv;
   const int hg = (G + fp8pd::kHeadsPerGroup - 1) / fp8pd::kHeadsPerGroup;
@@ -218,7 +236,7 @@ bool plan_proportional(int B, int Hq, int Hkv, int D, int ps, int max_pages, int
                                        : (keys + fp8pd::kTileTokens - 1) / fp8pd::kTileTokens;
   const int64_t m_max = (seq_tiles + fp8pd::kMaxSplitTiles - 1) / fp8pd::kMaxSplitTiles;
   if (m_max > fp8pd::kMaxSplits) return false;
-  const int64_t slots = static_cast<int64_t>(device_sms()) * fp8pd::decode_blocks_per_sm(D);
+  const int64_t slots = static_cast<int64_t>(device_sms()) * blocks_per_sm(D, umma);
   if (g_opt_schedule.load() == 0 && B * HX * seq_tiles < 4 * slots) return false;  // little work
 #ifdef FP8PD_PROP_WAVES
   const int64_t waves = FP8PD_PROP_WAVES;  // tuning builds
@@ -255,13 +273,14 @@ bool plan_proportional(int B, int Hq, int Hkv, int D, int ps, int max_pages, int
   return true;
 }
 
-int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, Plan* plan) {
+int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, Plan* plan,
+              bool umma = false) {
   // Proportional splits balance sequences of uneven length within one launch;
   // with a short window every sequence has about the same few tiles, and the
   // uniform splits below cost less.
   const int64_t sched = g_opt_schedule.load();
   if ((sched == 3 || (sched == 0 && (window == 0 || window >= 2048))) &&
-      plan_proportional(B, Hq, Hkv, D, ps, max_pages, window, plan))
+      plan_proportional(B, Hq, Hkv, D, ps, max_pages, window, plan, umma))
     return FP8PD_OK;
   plan->schedule = 1;
   const int G = Hq / Hkv;
@@ -285,7 +304,7 @@ int make_plan(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window, 
     // for uniform lengths (a partial extra wave would cost a whole split),
     // and the second wave lets the scheduler even out ragged lengths.
     const int sms = device_sms();
-    const int64_t slots = static_cast<int64_t>(sms) * fp8pd::decode_blocks_per_sm(D);
+    const int64_t slots = static_cast<int64_t>(sms) * blocks_per_sm(D, umma);
     S = std::min<int64_t>(s_max, (2 * slots) / units);
     S = std::max<int64_t>(S, 1);
     // A second wave that the splits cannot fill costs a whole split time with
@@ -622,7 +641,8 @@ cudaError_t launch_planned(const Plan& plan, const DecodeParams& p, const CUtens
   return fp8pd::launch_decode(p, tmk, tmv, k_mode, g_opt_v_decode.load() == 1, s);
 }
 
-void record_run(const Plan& plan, int D) {
+void record_run(const Plan& plan, int D, bool umma) {
+  t_run_info.kernel = umma ? 2 : 1;
   t_run_info.schedule = plan.schedule;
   t_run_info.num_splits = plan.num_splits;
   t_run_info.head_groups = plan.head_groups;
@@ -643,10 +663,12 @@ int run_decode(DecodeParams& p, const DecodeArgs& a, const fp8pd_tensor* k_pages
   // the fp8 compute path takes page and head scales only: refused, never downgraded
   if (g_opt_compute.load() == 1 && (p.k_tok || p.v_tok)) return FP8PD_ERR_UNSUPPORTED;
   Plan plan;
-  int r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
+  const bool um = use_umma(a.D, p.k_tok || p.v_tok, p.k_mx || p.v_mx, p.k_groups);
+  int r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan, um);
   if (r) return r;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   apply_plan(plan, &p);
+  p.umma = um ? 1 : 0;
   if (plan.combine) {
     void *ctr = nullptr, *part = nullptr;
     r = get_workspace(plan.counters_bytes, plan.workspace - plan.counters_bytes, s, &ctr, &part);
@@ -663,7 +685,7 @@ int run_decode(DecodeParams& p, const DecodeArgs& a, const fp8pd_tensor* k_pages
   ++g_launches;
   if (ev) cudaEventRecord(ev->b, s);
   ++g_calls;
-  record_run(plan, a.D);
+  record_run(plan, a.D, p.umma != 0);
   return FP8PD_OK;
 }
 
@@ -815,8 +837,9 @@ int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_t
   if (window < 0) return FP8PD_ERR_ARG;
   if (!fits_i32(B) || !fits_i32(block_table->shape[1])) return FP8PD_ERR_TOO_LARGE;
   Plan plan;
+  const bool um = use_umma(static_cast<int>(D), false, false, 1);  // page or head scales
   r = make_plan(static_cast<int>(B), static_cast<int>(Hq), static_cast<int>(Hkv), static_cast<int>(D),
-                static_cast<int>(ps), static_cast<int>(block_table->shape[1]), window, &plan);
+                static_cast<int>(ps), static_cast<int>(block_table->shape[1]), window, &plan, um);
   if (r) return r;
   info->num_splits = plan.num_splits;
   info->head_groups = plan.head_groups;
@@ -824,7 +847,7 @@ int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_t
   info->combine = plan.combine;
   info->workspace_bytes = plan.workspace;
   info->schedule = plan.schedule;
-  info->warps = plan.grid_blocks * fp8pd::decode_warps_per_block(static_cast<int>(D));
+  info->warps = plan.grid_blocks * (um ? 5 : fp8pd::decode_warps_per_block(static_cast<int>(D)));
   return FP8PD_OK;
 }
 
@@ -976,6 +999,10 @@ int fp8pd_set_option(int32_t option, int64_t value) {
       if (value < 0 || value > 1) return FP8PD_ERR_ARG;
       g_opt_compute = value;
       return FP8PD_OK;
+    case FP8PD_OPT_KERNEL:
+      if (value < 0 || value > 2) return FP8PD_ERR_ARG;
+      g_opt_kernel = value;
+      return FP8PD_OK;
     default:
       return FP8PD_ERR_ARG;
   }
@@ -990,6 +1017,7 @@ int64_t fp8pd_get_option(int32_t option) {
     case FP8PD_OPT_WAIT_POLLS: return g_opt_wait_polls.load();
     case FP8PD_OPT_TEST_STALL: return g_opt_test_stall.load();
     case FP8PD_OPT_COMPUTE: return g_opt_compute.load();
+    case FP8PD_OPT_KERNEL: return g_opt_kernel.load();
     default: return -1;
   }
 }
@@ -1105,11 +1133,13 @@ extern "C" int fp8_paged_decode_attention_noalloc(
   if (a.B == 0 || a.Hq == 0) return FP8PD_OK;
   if (g_opt_compute.load() == 1 && (p.k_tok || p.v_tok)) return FP8PD_ERR_UNSUPPORTED;
   Plan plan;
-  r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan);
+  const bool um = use_umma(a.D, p.k_tok || p.v_tok, p.k_mx || p.v_mx, p.k_groups);
+  r = make_plan(a.B, a.Hq, a.Hkv, a.D, a.ps, a.max_pages, window, &plan, um);
   if (r) return r;
   if (plan.workspace > kNoAllocScratchBytes) return FP8PD_ERR_TOO_LARGE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   apply_plan(plan, &p);
+  p.umma = um ? 1 : 0;
   if (plan.combine) {
     void* ws = nullptr;
     r = noalloc_scratch(&ws);
@@ -1128,6 +1158,6 @@ extern "C" int fp8_paged_decode_attention_noalloc(
   if (e != cudaSuccess) return fail_cuda(e);
   ++g_launches;
   ++g_calls;
-  record_run(plan, a.D);
+  record_run(plan, a.D, p.umma != 0);
   return FP8PD_OK;
 }

@@ -77,6 +77,9 @@ struct DecodeParams {
   uint8_t* vw;
   float* ksw;                 // the scales, writable: a per-token scale of the new token is stored
   float* vsw;
+  // 1: the tensor-memory kernel (D = 64 / 128, page or head scales, f32
+  // compute) runs this call
+  int umma;
 };
 
 struct AppendParams {
@@ -124,6 +127,8 @@ cudaError_t launch_encode(const float* x, int64_t xs, uint8_t* c, int64_t cs, in
 
 // Thread blocks of the split kernel one SM holds for head dim D.
 int decode_blocks_per_sm(int D);
+// Thread blocks of the tensor-memory kernel one SM holds (D = 64 / 128; else 0).
+int decode_umma_blocks_per_sm(int D);
 // Warps per block of the split kernel for head dim D.
 int decode_warps_per_block(int D);
 // Dynamic shared memory of the split kernel for head dim D.

@@ -2110,6 +2110,702 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
 }
 
 // ---------------------------------------------------------------------------
+// Tensor-memory split kernel (tcgen05). The same splits, plans, masking,
+// fused append and split merge as the kernel above, with the attention of
+// each 128-token chunk on the 5th-generation tensor cores:
+//   S = K q'^T   kind::f8f6f4, M = 128 tokens, N = 16 (8 query heads x the two
+//                E4M3 terms of q'), K's E4M3 bytes straight from the TMA tile;
+//   O^T += V^T P kind::f16, M = D, N = 16 (8 heads x the f16 hi + lo terms of
+//                P), V decoded once to f16 in shared memory.
+// Both accumulators live in tensor memory. Two warpgroups of four warps take
+// alternate chunks (group g the chunks c = g mod 2), each with its own S, P,
+// f16 V buffer, O accumulator and online-softmax state, merged at the end.
+// Warp w of a group owns tokens 32w .. 32w+31 of its chunks (its TMEM lane
+// quarter): it reads S, runs the softmax (one token per thread, the 8 heads in
+// registers), writes P and the decoded V rows, and copies its own two tiles of
+// each chunk (lanes 0-3: K and V of tiles 2w, 2w+1, on its own barrier),
+// refilling them once it has decoded their V rows. Warp 8 issues the MMAs and
+// their commits from one lane. Every wait is bounded.
+// ---------------------------------------------------------------------------
+
+#ifndef FP8PD_UNS_D64
+#define FP8PD_UNS_D64 8
+#endif
+#ifndef FP8PD_UNS_D128
+#define FP8PD_UNS_D128 4
+#endif
+
+template <int D>
+struct UCfg {
+  static_assert(D == 64 || D == 128, "tensor-memory kernel: D = 64 or 128");
+  static constexpr int NS = (D == 64) ? FP8PD_UNS_D64 : FP8PD_UNS_D128;  // K/V ring stages
+  static_assert(NS % 2 == 0 && NS >= 2, "a stage keeps its warpgroup: an even ring");
+  static constexpr int NWG = 2;                      // warpgroups (alternate chunks)
+  static constexpr int NCW = 4 * NWG;                // compute warps
+  static constexpr int NT = (NCW + 1) * 32;          // + the MMA warp
+  static constexpr int CHUNK = 128;                  // tokens per chunk (MMA M of QK)
+  static constexpr int KV = CHUNK * D;               // K (or V) bytes of a chunk
+  static constexpr int STAGE = 2 * KV;
+  static constexpr int RING = NS * STAGE;
+  static constexpr int VF16 = CHUNK * D * 2;         // V of a chunk as f16 (one per group)
+  static constexpr int PBUF = CHUNK * 32;            // P of a chunk: 16 f16 per token (one per group)
+  static constexpr int QT = 16 * D;                  // q' as 16 rows of E4M3 (8 heads x 2 terms)
+  static constexpr int LIST = kMaxSplitTiles * 12;   // per tile: entry, k scale, v scale
+  static constexpr int NBAR = 5 * NS + 5;            // full[NS][4], sbar[2], pready[NS], pvbar[2], patched
+  static constexpr int MISC = 256;                   // floats
+  static constexpr int SMEM = 1024 + RING + NWG * (VF16 + PBUF) + QT + LIST + NBAR * 8 + MISC * 4;
+  static constexpr int MIN_BLOCKS = 1;
+  static constexpr uint32_t TMEM_COLS = 64;          // S[g] at 16 g, O[g] at 32 + 16 g
+  static constexpr uint32_t SWZ = (D == 128) ? 2u : 4u;  // descriptor layout: 128-byte / 64-byte swizzle
+  static_assert(RING % 1024 == 0 && VF16 % 1024 == 0 && PBUF % 1024 == 0 && QT % 1024 == 0,
+                "1024-byte aligned operand buffers");
+  static_assert(NWG * (8 * D + 16) * 4 <= 16384 && 16384 + 8 * 32 * 4 <= RING,
+                "epilogue scratch and merge weights fit in the ring");
+};
+
+// byte offsets (all >> 4), version 1, layout type (swizzle) in bits 61-63.
+__device__ __forceinline__ uint64_t umma_sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                               uint32_t layout) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) |
+         (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(layout) << 61);
+}
+
+__device__ __forceinline__ void umma_f8f6f4(uint32_t tmem_d, uint64_t da, uint64_t db,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n}\n" ::"r"(
+          tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(accumulate), "r"(0u)
+      : "memory");
+}
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n}\n" ::"r"(
+          tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(accumulate), "r"(0u)
+      : "memory");
+}
+// Arrives on the barrier once every MMA this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+// 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
+}
+
+
+template <int D>
+__global__ void __launch_bounds__(UCfg<D>::NT, UCfg<D>::MIN_BLOCKS)
+    decode_umma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
+                       const __grid_constant__ CUtensorMap tmv) {
+  using C = UCfg<D>;
+  constexpr float kLog2e = 1.4426950408889634f;
+  constexpr unsigned FULL = 0xffffffffu;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const uint32_t s_ring = smem_u32(smem);
+  const uint32_t s_vf = s_ring + C::RING;            // [group] f16 V
+  const uint32_t s_p = s_vf + C::NWG * C::VF16;      // [group] P
+  const uint32_t s_q = s_p + C::NWG * C::PBUF;
+  int32_t* l_ent = reinterpret_cast<int32_t*>(smem + C::RING + C::NWG * (C::VF16 + C::PBUF) + C::QT);
+  float* l_ks = reinterpret_cast<float*>(l_ent + kMaxSplitTiles);
+  float* l_vs = l_ks + kMaxSplitTiles;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(l_vs + kMaxSplitTiles);
+  float* misc = reinterpret_cast<float*>(bars + C::NBAR);
+  const uint32_t b_full = smem_u32(bars), b_s = b_full + 32 * C::NS, b_pr = b_s + 16,
+                 b_pv = b_pr + 8 * C::NS, b_patch = b_pv + 16;
+  // misc: [0] TMEM base, [1] abort, [2..4) vote words (per group), [8..72)
+  // per-warp head maxima, [72..80) per-warp |v scale| maxima, [80..144) per-warp
+  // l sums, [144..160) q maximum exchange
+  uint32_t* m_tmem = reinterpret_cast<uint32_t*>(misc);
+  volatile int* m_abort = reinterpret_cast<volatile int*>(misc + 1);
+  volatile uint32_t* m_vote = reinterpret_cast<volatile uint32_t*>(misc + 2);
+  float* m_hmax = misc + 8;
+  float* m_vmax = misc + 72;
+  float* m_lsum = misc + 80;
+  float* m_qmax = misc + 144;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int kvh = blockIdx.x / p.head_groups;
+  const int hg = blockIdx.x - kvh * p.head_groups;
+  const int head0 = kvh * p.G + hg * 8;
+  const int nheads = min(8, p.G - hg * 8);
+
+  int b, split, S;
+  int prop_j0 = 0, prop_j1 = 0, sp_b = 0, gp_b = 0;
+  if (p.prop) {
+    if (!prop_assign<C::NCW + 1>(p, reinterpret_cast<int*>(smem), reinterpret_cast<int*>(misc),
+                                 head0, nheads, b, split, S, prop_j0, prop_j1, sp_b, gp_b))
+      return;
+  } else {
+    b = blockIdx.y;
+    split = blockIdx.z;
+    S = p.num_splits;
+  }
+  const int L = attended_keys(p, b, tid == 0 && split == 0 && blockIdx.x == 0);
+  int lo, hi;
+  key_range(p, b, L, lo, hi);
+  int t0, t1;
+  if (p.prop) {
+    t0 = max(lo, (lo / kTileTokens + prop_j0) * kTileTokens);
+    t1 = min(hi, (lo / kTileTokens + prop_j1) * kTileTokens);
+  } else {
+    const int first_page = lo / p.ps;
+    const int n_pages = (hi > lo) ? (hi - 1) / p.ps - first_page + 1 : 0;
+    const int pg0 = first_page + split * p.chunk_pages;
+    const int pg1 = min(first_page + n_pages, pg0 + p.chunk_pages);
+    t0 = max(lo, pg0 * p.ps);
+    t1 = min(hi, pg1 * p.ps);
+  }
+  const int tile_first = t0 / kTileTokens;
+  int n_tiles = (t1 > t0) ? (t1 + kTileTokens - 1) / kTileTokens - tile_first : 0;
+  if (n_tiles > kMaxSplitTiles) {
+    if (tid == 0) raise_flag(FP8PD_FLAG_INTERNAL);
+    n_tiles = 0;
+  }
+  const int nch = (n_tiles + 7) / 8;
+
+  // ---- tile list (entry = page << 4 | tile in page, -1 = outside the pool), scales
+  const int32_t* trow = p.table + (int64_t)b * p.tab_sb;
+  const float* ksbase = p.ks + (int64_t)kvh * p.ks_sh;
+  const float* vsbase = p.vs + (int64_t)kvh * p.vs_sh;
+  for (int j = tid; j < n_tiles; j += C::NT) {
+    const int tok = (tile_first + j) * kTileTokens;
+    const int lp = tok / p.ps;
+    const int page = __ldg(trow + (int64_t)lp * p.tab_sp);
+    int e = -1;
+    float ks = 0.f, vs = 0.f;
+    if ((unsigned)page < (unsigned)p.num_pages) {
+      e = (page << 4) | ((tok - lp * p.ps) / kTileTokens);
+      ks = __ldg(ksbase + (int64_t)page * p.ks_sp);
+      vs = __ldg(vsbase + (int64_t)page * p.vs_sp);
+    } else if (hg == 0) {
+      raise_flag(FP8PD_FLAG_PAGE_OOB);
+    }
+    l_ent[j] = e;
+    l_ks[j] = ks;
+    l_vs[j] = vs;
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 4 * C::NS; ++i) mbar_init(b_full + 8 * i, 1);
+    for (int s = 0; s < C::NS; ++s) mbar_init(b_pr + 8 * s, 4 * 32);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(b_s + 8 * i, 1);
+      mbar_init(b_pv + 8 * i, 1);
+    }
+    mbar_init(b_patch, 1);
+    *m_abort = 0;
+    m_vote[0] = m_vote[1] = 0u;
+    fence_barrier_init();
+  }
+  if (warp == C::NCW) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                     smem_u32(m_tmem)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  // the new token (fused append): its tile and chunk in this block's range
+  int j_new = -1;
+  if (p.append && L - 1 >= t0 && L - 1 < t1) j_new = (L - 1) / kTileTokens - tile_first;
+  const int c_new = j_new >= 0 ? j_new / 8 : -1;
+
+  // ---- q' = q * 2^(8 - e) (max |q'| in [2^7, 2^8)) as two E4M3 terms, rows
+  // n (hi of head n) and 8 + n (lo), K-major with the tiles' swizzle
+  constexpr int QITEMS = 8 * (D / 16);
+  float qv[16];
+  int q_n = -1, q_c = 0;
+  float qm = 0.f;
+  if (tid < QITEMS) {
+    q_n = tid / (D / 16);
+    q_c = tid - q_n * (D / 16);
+    const bool ok = q_n < nheads;
+    const uint16_t* qrow = p.q + (int64_t)b * p.q_sb + (int64_t)(head0 + (ok ? q_n : 0)) * p.q_sh;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      qv[i] = ok ? bf16_bits_to_float(__ldg(qrow + (int64_t)(16 * q_c + i) * p.q_sd)) : 0.f;
+      qm = fmaxf(qm, fabsf(qv[i]));
+    }
+  }
+  qm = warp_max(qm);
+  if (lane == 0) m_qmax[warp] = qm;
+  __syncthreads();
+  qm = 0.f;
+#pragma unroll
+  for (int w = 0; w <= C::NCW; ++w) qm = fmaxf(qm, m_qmax[w]);
+  int qe = 0;
+  if (qm > 0.f && isfinite(qm)) frexpf(qm, &qe);
+  qe = max(qe, -111);
+  const float qmul = ldexpf(1.f, 8 - qe);
+  const float score_base = p.sm_scale_log2 / qmul;
+  if (tid < QITEMS) {
+    uint32_t h4[4], l4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      e4m3_split4(qv[4 * i] * qmul, qv[4 * i + 1] * qmul, qv[4 * i + 2] * qmul,
+                  qv[4 * i + 3] * qmul, h4[i], l4[i]);
+    const uint32_t ah = s_q + tile_off<D>(q_n, 16 * q_c), al = s_q + tile_off<D>(8 + q_n, 16 * q_c);
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(ah), "r"(h4[0]), "r"(h4[1]),
+                 "r"(h4[2]), "r"(h4[3]) : "memory");
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(al), "r"(l4[0]), "r"(l4[1]),
+                 "r"(l4[2]), "r"(l4[3]) : "memory");
+  }
+  fence_proxy_async();  // q' (and later P, V) reach the tensor core through the async proxy
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *m_tmem;
+  // S of group g at columns 16 g, O of group g at 32 + 16 g
+  constexpr uint32_t IDESC_QK = (1u << 4) | (2u << 17) | (8u << 24);  // f32 += e4m3 x e4m3, M 128, N 16
+  constexpr uint32_t IDESC_PV = (1u << 4) | (1u << 15) | (1u << 16) | (2u << 17) |
+                                (static_cast<uint32_t>(D >> 4) << 24);  // f32 += f16 x f16, MN-major
+  const int polls = p.wait_polls;
+  bool failed = false;
+  // A wait that gives up marks the warp failed (warp-uniform); the warp then
+  // skips its later waits but still walks every chunk and named barrier, so no
+  // other warp blocks on it, and the block's result is zero.
+  auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    if (failed) return false;
+    const bool ok = __all_sync(FULL, mbar_wait(bar, parity, polls) && !*m_abort);
+    if (!ok) {
+      failed = true;
+      if (lane == 0) {
+        raise_flag(FP8PD_FLAG_TIMEOUT);
+        *m_abort = 1;
+      }
+    }
+    return ok;
+  };
+  // warp q of group c % 2 copies tiles 2q, 2q+1 of chunk c (K and V); they land
+  // on full(c % NS, q). The group releases stage c % NS on pready(c % NS).
+  auto full_bar = [&](int c, int q) { return b_full + 8 * ((c % C::NS) * 4 + q); };
+  auto pready_bar = [&](int c) { return b_pr + 8 * (c % C::NS); };
+
+  if (warp == C::NCW) {
+    // ======================= MMA warp (one lane issues) =======================
+    int pv_done = 0;  // chunks whose PV MMAs were issued
+    auto do_pv = [&](int c) {
+      if (!wait(pready_bar(c), (c / C::NS) & 1)) return;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t vb = s_vf + (c & 1) * C::VF16, pb = s_p + (c & 1) * C::PBUF;
+        for (int kk = 0; kk < C::CHUNK / 16; ++kk) {
+          const uint64_t da = umma_sdesc(vb + kk * 2048, 16384, 1024, 2);
+          const uint64_t db = umma_sdesc(pb + kk * 512, 4096, 256, 6);
+          umma_f16(tmem + 32 + 16 * (c & 1), da, db, IDESC_PV, (c > 1 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(b_pv + 8 * (c & 1));
+      }
+      __syncwarp();
+      pv_done = c + 1;
+    };
+    for (int c = 0; c < nch && !failed; ++c) {
+      const int s = c % C::NS;
+      bool ok = true;
+      for (int q = 0; q < 4 && ok; ++q) ok = wait(full_bar(c, q), (c / C::NS) & 1);
+      if (!ok) break;
+      if (c == c_new && !wait(b_patch, 0)) break;
+      if (c >= 2 && !wait(pready_bar(c - 2), ((c - 2) / C::NS) & 1)) break;  // S[c & 1] read
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t ka = s_ring + s * C::STAGE;
+#pragma unroll
+        for (int kc = 0; kc < D / 32; ++kc) {
+          const uint64_t da = umma_sdesc(ka + 32 * kc, 16, 8 * D, C::SWZ);
+          const uint64_t db = umma_sdesc(s_q + 32 * kc, 16, 8 * D, C::SWZ);
+          umma_f8f6f4(tmem + 16 * (c & 1), da, db, IDESC_QK, kc > 0 ? 1u : 0u);
+        }
+        umma_commit(b_s + 8 * (c & 1));
+      }
+      __syncwarp();
+      if (c >= 1) do_pv(c - 1);
+    }
+    if (!failed && nch > 0) do_pv(nch - 1);
+    // drain: every committed MMA has finished before the block moves on
+    for (int c = max(0, pv_done - 2); c < pv_done; ++c)
+      mbar_wait(b_pv + 8 * (c & 1), (c >> 1) & 1, polls);
+  } else {
+    // ======================= compute warpgroups =======================
+    const int g = warp >> 2, wq = warp & 3;
+    const int t = tid & 127;  // token row of the group's chunks, and TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
+    const uint32_t t_s = tmem + lane_base + 16 * g, t_o = tmem + lane_base + 32 + 16 * g;
+    const uint32_t vbuf = s_vf + g * C::VF16, pbuf = s_p + g * C::PBUF;
+    float m[8], l[8], x[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      m[h] = -CUDART_INF_F;
+      l[h] = 0.f;
+      x[h] = -CUDART_INF_F;
+    }
+    float vref = 0.f, inv_vref = 0.f;
+    const int kt = t >> 4, r = t & 15;  // tile of the chunk, row of the tile
+    int issued = -1;  // the last chunk this warp issued copies for
+    auto issue_part = [&](int c) {
+      const int s = c % C::NS;
+      const int k = 2 * wq + ((lane >> 1) & 1);
+      const int j = 8 * c + k;
+      const int e = (lane < 4 && j < n_tiles) ? l_ent[j] : -1;
+      const int tiles = __popc(__ballot_sync(FULL, e >= 0 && (lane & 1) == 0));
+      const uint32_t bar = full_bar(c, wq);
+      if (lane == 0) {
+        fence_proxy_async();  // this warp's reads of the stage come first
+        if (tiles) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(tiles) * 2u * kTileTokens * D);
+        else mbar_arrive(bar);  // nothing to copy: the phase completes empty
+      }
+      __syncwarp();
+      if (e >= 0) {
+        const uint32_t dst = s_ring + s * C::STAGE + ((lane & 1) ? C::KV : 0) + k * kTileTokens * D;
+        tma_load_5d(dst, (lane & 1) ? &tmv : &tmk, bar, 0, (e & 15) * kTileTokens, 0, kvh, e >> 4);
+      }
+      issued = c;
+    };
+    if (lane == 0 && warp == 0) {
+      prefetch_tensormap(&tmk);
+      prefetch_tensormap(&tmv);
+    }
+    for (int c = g; c < min(C::NS, nch); c += 2) issue_part(c);
+    int last = -1;  // this group's last chunk
+    for (int c = g; c < nch; c += 2) {
+      last = c;
+      const int s = c % C::NS;
+      const uint32_t sk = s_ring + s * C::STAGE, sv = sk + C::KV;
+      const int j = 8 * c + kt;
+      const int e = j < n_tiles ? l_ent[j] : -1;
+      const int tok = (tile_first + j) * kTileTokens + r;
+      const bool valid = e >= 0 && tok >= t0 && tok < t1;
+      const float ks = e >= 0 ? l_ks[j] : 0.f, vs = e >= 0 ? l_vs[j] : 0.f;
+      if (c == c_new && wq == (j_new % 8) >> 1) {
+        // the new token: quantized with its page's scales, stored by head
+        // group 0, patched into the chunk before the QK MMA reads it
+        if (wait(full_bar(c, wq), (c / C::NS) & 1)) {
+          const int en = l_ent[j_new];
+          if (en >= 0) {
+            float kss = l_ks[j_new], vss = l_vs[j_new];
+            const int rn = (L - 1) - (tile_first + j_new) * kTileTokens;
+            append_new_token<D, false>(p, b, kvh, hg == 0, en >> 4, (en & 15) * kTileTokens + rn,
+                                       rn, sk + (j_new % 8) * kTileTokens * D,
+                                       sv + (j_new % 8) * kTileTokens * D, kss, vss);
+          }
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_patch);
+        }
+      }
+      wait(b_s + 8 * g, (c >> 1) & 1);
+      tc_fence_after();
+      uint32_t sr[16];
+      tmem_ld16(t_s, sr);
+      tc_fence_before();
+      const float kf = score_base * ks;
+      float sc[8];
+      bool trig = valid && fabsf(vs) > vref;
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        sc[h] = (valid && h < nheads)
+                    ? (__uint_as_float(sr[h]) + __uint_as_float(sr[8 + h])) * kf
+                    : -CUDART_INF_F;
+        x[h] = fmaxf(x[h], sc[h]);
+        trig = trig || (sc[h] > m[h] + kLazyLog2);
+      }
+      // group-wide vote on a rescale (the chunk's P share one reference per head)
+      const unsigned vote = __ballot_sync(FULL, trig);
+      if (lane == 0 && vote) atomicOr(const_cast<uint32_t*>(m_vote + g), 1u << wq);
+      named_sync(1 + g, 128);
+      const uint32_t any = m_vote[g];
+      if (any) {
+        float wm[8];
+#pragma unroll
+        for (int h = 0; h < 8; ++h) wm[h] = warp_max(sc[h]);
+        const float wv = warp_max(valid ? fabsf(vs) : 0.f);
+        if (lane == 0) {
+#pragma unroll
+          for (int h = 0; h < 8; ++h) m_hmax[warp * 8 + h] = wm[h];
+          m_vmax[warp] = wv;
+        }
+        named_sync(1 + g, 128);
+        if (t == 0) m_vote[g] = 0u;  // read by every warp of the group before this barrier
+        float cf[8];
+        float nv = vref;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) nv = fmaxf(nv, m_vmax[4 * g + w]);
+        const float fv = (nv > vref && vref > 0.f) ? vref / nv : 1.f;
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+          float nm = m[h];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) nm = fmaxf(nm, m_hmax[(4 * g + w) * 8 + h]);
+          cf[h] = (nm > m[h]) ? fast_exp2(m[h] - nm) : 1.f;
+          l[h] *= cf[h];
+          m[h] = nm;
+        }
+        if (nv > vref) {
+          vref = nv;
+          inv_vref = 1.f / nv;
+        }
+        if (c >= 2 && wait(b_pv + 8 * g, ((c - 2) >> 1) & 1)) {
+          // O holds this group's chunks < c: its last PV has run; rescale O in place
+          tc_fence_after();
+          uint32_t o[16];
+          tmem_ld16(t_o, o);
+#pragma unroll
+          for (int h = 0; h < 8; ++h) {
+            o[h] = __float_as_uint(__uint_as_float(o[h]) * cf[h] * fv);
+            o[8 + h] = __float_as_uint(__uint_as_float(o[8 + h]) * cf[h] * fv);
+          }
+          tmem_st16(t_o, o);
+          tc_fence_before();
+        }
+        named_sync(1 + g, 128);  // everyone has read the maxima before they are reused
+      }
+      // P = 2^(s - m) * v_scale / vref as f16 hi + lo, columns h (hi) and 8 + h (lo)
+      uint32_t ph[4], pl[4];
+      const float vr = vs * inv_vref;
+#pragma unroll
+      for (int h = 0; h < 8; h += 2) {
+        const float mb0 = (m[h] == -CUDART_INF_F) ? 0.f : m[h];
+        const float mb1 = (m[h + 1] == -CUDART_INF_F) ? 0.f : m[h + 1];
+        const float p0 = fast_exp2(sc[h] - mb0), p1 = fast_exp2(sc[h + 1] - mb1);
+        l[h] += p0;
+        l[h + 1] += p1;
+        const float w0 = p0 * vr, w1 = p1 * vr;
+        const uint32_t hh = pack_f16x2(w0, w1);
+        const float2 fh = unpack_f16x2(hh);
+        ph[h >> 1] = hh;
+        pl[h >> 1] = pack_f16x2(w0 - fh.x, w1 - fh.y);
+      }
+      // the group's P and V buffers are free once the PV of its previous chunk has run
+      if (c >= 2) wait(b_pv + 8 * g, ((c - 2) >> 1) & 1);
+      {
+        // P row t: 32 bytes, 32-byte swizzle (chunk ^= bit 2 of t)
+        const uint32_t pr = pbuf + t * 32, sw = (t >> 2) & 1;
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(pr + (sw << 4)), "r"(ph[0]),
+                     "r"(ph[1]), "r"(ph[2]), "r"(ph[3]) : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(pr + ((sw ^ 1) << 4)),
+                     "r"(pl[0]), "r"(pl[1]), "r"(pl[2]), "r"(pl[3]) : "memory");
+      }
+      {
+        // V row t decoded to f16, MN-major with the 128-byte swizzle: head-dim
+        // entries 64a .. 64a+63 of token t in the 128-byte row t % 8 of k-group
+        // t / 8 of atom a; 16-byte chunk q of that row at q ^ (t % 8)
+        const uint32_t vrow = sv + kt * kTileTokens * D;
+#pragma unroll
+        for (int cb = 0; cb < D / 16; ++cb) {
+          uint4 w = make_uint4(0u, 0u, 0u, 0u);
+          if (valid) {
+            const uint32_t a = vrow + tile_off<D>(r, 16 * cb);
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w) : "r"(a));
+          }
+          const uint32_t f[8] = {e4m3x2_lo16_to_f16x2(w.x), e4m3x2_hi16_to_f16x2(w.x),
+                                 e4m3x2_lo16_to_f16x2(w.y), e4m3x2_hi16_to_f16x2(w.y),
+                                 e4m3x2_lo16_to_f16x2(w.z), e4m3x2_hi16_to_f16x2(w.z),
+                                 e4m3x2_lo16_to_f16x2(w.w), e4m3x2_hi16_to_f16x2(w.w)};
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int d0 = 16 * cb + 8 * u;
+            const int atom = d0 >> 6, q = (d0 & 63) >> 3;
+            const uint32_t dst = vbuf + atom * 16384 + (t >> 3) * 1024 + (t & 7) * 128 +
+                                 ((q ^ (t & 7)) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(f[4 * u]),
+                         "r"(f[4 * u + 1]), "r"(f[4 * u + 2]), "r"(f[4 * u + 3]) : "memory");
+          }
+        }
+      }
+      fence_proxy_async();
+      __syncwarp();  // the warp's V rows of this stage are decoded: refill its tiles
+      if (c + C::NS < nch && !failed) issue_part(c + C::NS);
+      mbar_arrive(pready_bar(c));
+    }
+    // copies of this warp still in flight (only after a failed wait) land first
+    for (int c = issued; c >= 0 && c > issued - C::NS; c -= 2)
+      mbar_wait(full_bar(c, wq), (c / C::NS) & 1, polls);
+    // ---- this group's (m, l, O) moved onto the exact maxima, l over its tokens
+    if (last >= 0) wait(b_pv + 8 * g, (last >> 1) & 1);
+    tc_fence_after();
+    // the epilogue scratch overlays ring stage 0: both groups are past their
+    // last chunk (and its copies and MMAs) before either writes it
+    named_sync(3, C::NCW * 32);
+    float* Os = reinterpret_cast<float*>(smem);  // [group][8][D] (the ring is idle now)
+    float* ml = Os + C::NWG * 8 * D;             // [group][8][2]
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      const float xm = warp_max(x[h]);
+      if (lane == 0) m_hmax[warp * 8 + h] = xm;
+      float ls = l[h];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(FULL, ls, o);
+      if (lane == 0) m_lsum[warp * 8 + h] = ls;
+    }
+    named_sync(1 + g, 128);
+    float fx[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      float xm = -CUDART_INF_F, ls = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        xm = fmaxf(xm, m_hmax[(4 * g + w) * 8 + h]);
+        ls += m_lsum[(4 * g + w) * 8 + h];
+      }
+      // l and O are relative to the reference m; move them onto the maximum
+      fx[h] = (xm > m[h] && m[h] != -CUDART_INF_F) ? fast_exp2(m[h] - xm) : 1.f;
+      if (failed || last < 0) {
+        xm = -CUDART_INF_F;
+        ls = 0.f;
+      }
+      if (t == 0) {
+        ml[(g * 8 + h) * 2] = xm;
+        ml[(g * 8 + h) * 2 + 1] = ls * fx[h];
+      }
+    }
+    // O rows: D = 128, lane = head-dim entry; D = 64 (M = 64), entry 16q + i
+    // sits in lane i < 16 of the warp's quarter
+    const int d = (D == 128) ? t : (lane < 16 ? 16 * wq + lane : -1);
+    uint32_t o[16];
+    const bool have = last >= 0 && !failed;
+    if (have) tmem_ld16(t_o, o);
+    tc_fence_before();
+    if (d >= 0) {
+#pragma unroll
+      for (int h = 0; h < 8; ++h)
+        Os[(g * 8 + h) * D + d] =
+            have ? (__uint_as_float(o[h]) + __uint_as_float(o[8 + h])) * vref * fx[h] : 0.f;
+    }
+  }
+  __syncthreads();
+  if (warp == C::NCW) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+  }
+
+  // ---- the two groups' results merged, then published and the splits merged
+  // (as the kernel above)
+  float* Os = reinterpret_cast<float*>(smem);
+  const float* ml = Os + C::NWG * 8 * D;
+  const int NG = (S + kMergeFan - 1) / kMergeFan;
+  const int HX = gridDim.x;
+  int64_t prow0, grow0, cnt0;
+  if (p.prop) {
+    prow0 = ((int64_t)sp_b * HX + (int64_t)blockIdx.x * S) * kHeadsPerGroup;
+    grow0 = ((int64_t)gp_b * HX + (int64_t)blockIdx.x * NG) * kHeadsPerGroup;
+    cnt0 = (int64_t)(b + gp_b) * HX + (int64_t)blockIdx.x * (1 + NG);
+  } else {
+    prow0 = ((int64_t)b * p.Hq + head0) * S;
+    grow0 = ((int64_t)b * p.Hq + head0) * NG;
+    cnt0 = ((int64_t)b * HX + blockIdx.x) * (1 + NG);
+  }
+  for (int it = tid; it < 8 * (D / 4); it += C::NT) {
+    const int n = it / (D / 4);
+    const int dd = (it - n * (D / 4)) * 4;
+    if (n >= nheads) continue;
+    const float m0 = ml[(0 * 8 + n) * 2], l0 = ml[(0 * 8 + n) * 2 + 1];
+    const float m1 = ml[(1 * 8 + n) * 2], l1 = ml[(1 * 8 + n) * 2 + 1];
+    const float M = fmaxf(m0, m1);
+    const float w0 = (m0 == -CUDART_INF_F) ? 0.f : fast_exp2(m0 - M);
+    const float w1 = (m1 == -CUDART_INF_F) ? 0.f : fast_exp2(m1 - M);
+    const float l = w0 * l0 + w1 * l1;
+    const float4 a0 = *reinterpret_cast<const float4*>(Os + (0 * 8 + n) * D + dd);
+    const float4 a1 = *reinterpret_cast<const float4*>(Os + (1 * 8 + n) * D + dd);
+    const float4 acc = make_float4(w0 * a0.x + w1 * a1.x, w0 * a0.y + w1 * a1.y,
+                                   w0 * a0.z + w1 * a1.z, w0 * a0.w + w1 * a1.w);
+    const int head = head0 + n;
+    if (S == 1 && p.pout_o) {
+      store_partial(p, b, head, dd, acc, M, l);
+    } else if (S == 1) {
+      const float sl = p.sinks ? p.sinks[(int64_t)head * p.sinks_s] * kLog2e : -CUDART_INF_F;
+      const float M2 = fmaxf(M, sl);
+      float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (M2 != -CUDART_INF_F) {
+        const float a = (M == -CUDART_INF_F) ? 0.f : fast_exp2(M - M2);
+        const float den = l * a + (p.sinks ? fast_exp2(sl - M2) : 0.f);
+        if (den > 0.f) {
+          const float f = a / den;
+          res = make_float4(acc.x * f, acc.y * f, acc.z * f, acc.w * f);
+        }
+      }
+      *reinterpret_cast<float4*>(p.out + (int64_t)b * p.o_sb + (int64_t)head * p.o_sh + dd) = res;
+    } else {
+      const int64_t row = prow0 + (int64_t)n * S + split;
+      *reinterpret_cast<float4*>(p.part_o + row * D + dd) = acc;
+      if (dd == 0) *reinterpret_cast<float2*>(p.part_ml + row * 2) = make_float2(M, l);
+    }
+  }
+  if (S == 1) return;
+  __syncthreads();
+  int* flag = reinterpret_cast<int*>(misc + 1);
+  int* ucnt = p.counters + cnt0;
+  const int gi = split / kMergeFan;
+  const int gsize = min(kMergeFan, S - gi * kMergeFan);
+  if (tid == 0) {
+    __threadfence();
+    *flag = (atomicAdd(ucnt + 1 + gi, 1) == gsize - 1);
+  }
+  __syncthreads();
+  if (!*flag) return;
+  __threadfence();
+  float* wts = reinterpret_cast<float*>(smem + 16384);  // [8][32] merge weights
+  const bool fin = p.pout_o == nullptr;
+  float* fml = fin ? nullptr : p.pout_ml;
+  float* fo = fin ? nullptr : p.pout_o;
+  const int64_t frow = (int64_t)b * p.Hq + head0;
+  if (NG == 1) {
+    merge_partials<D, C::NCW + 1>(p.part_ml, p.part_o, prow0, S, S, nheads, fin, p, b, head0, fml,
+                                  fo, frow, 1, wts);
+    if (tid == 0) ucnt[1] = 0;
+    return;
+  }
+  merge_partials<D, C::NCW + 1>(p.part_ml, p.part_o, prow0 + gi * kMergeFan, S, gsize, nheads,
+                                false, p, b, head0, p.grp_ml, p.grp_o, grow0 + gi, NG, wts);
+  if (tid == 0) ucnt[1 + gi] = 0;
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    *flag = (atomicAdd(ucnt, 1) == NG - 1);
+  }
+  __syncthreads();
+  if (!*flag) return;
+  __threadfence();
+  merge_partials<D, C::NCW + 1>(p.grp_ml, p.grp_o, grow0, NG, NG, nheads, fin, p, b, head0, fml,
+                                fo, frow, 1, wts);
+  if (tid == 0) ucnt[0] = 0;
+}
+
+// ---------------------------------------------------------------------------
 // Quantize-append: one thread per (sequence, KV head, pair of head-dim
 // entries), for K and V. code = E4M3_RNE_SAT(float32(x) / scale): IEEE float32
 // division (__fdiv_rn), then cvt.rn.satfinite.e4m3x2.f32, which rounds to
@@ -2259,9 +2955,33 @@ static cudaError_t launch_decode_kv(const DecodeParams& p, const CUtensorMap& tm
 }
 
 template <int D>
+static cudaError_t launch_decode_umma(const DecodeParams& p, const CUtensorMap& tmk,
+                                      const CUtensorMap& tmv, cudaStream_t s) {
+  static std::atomic<uint64_t> configured{0};
+  const int smem = UCfg<D>::SMEM;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
+  if (!bit || !(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(decode_umma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  const dim3 grid = p.prop ? dim3(p.Hkv * p.head_groups, p.nbx, 1)
+                           : dim3(p.Hkv * p.head_groups, p.B, p.num_splits);
+  decode_umma_kernel<D><<<grid, UCfg<D>::NT, smem, s>>>(p, tmk, tmv);
+  return cudaGetLastError();
+}
+
+template <int D>
 static cudaError_t launch_decode_dt(const DecodeParams& p, const CUtensorMap& tmk,
                                     const CUtensorMap& tmv, int k_mode, bool v_cvt,
                                     cudaStream_t s) {
+  if constexpr (D == 64 || D == 128) {
+    if (p.umma) return launch_decode_umma<D>(p, tmk, tmv, s);
+  }
   if (p.v_mx) return launch_decode_kv<D, 2>(p, tmk, tmv, k_mode, v_cvt, s);
   if (p.k_tok || p.v_tok) return launch_decode_kv<D, 1>(p, tmk, tmv, k_mode, v_cvt, s);
   return launch_decode_kv<D, 0>(p, tmk, tmv, k_mode, v_cvt, s);
@@ -2294,6 +3014,32 @@ static int blocks_per_sm_d() {
   c = n > 0 ? n : 1;
   cached.store(c);
   return c;
+}
+
+template <int D>
+static int umma_blocks_per_sm_d() {
+  static std::atomic<int> cached{-1};
+  int c = cached.load();
+  if (c >= 0) return c;
+  int n = 0;
+  if (cudaFuncSetAttribute(decode_umma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           UCfg<D>::SMEM) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_umma_kernel<D>, UCfg<D>::NT,
+                                                    UCfg<D>::SMEM) != cudaSuccess) {
+    cudaGetLastError();
+    return UCfg<D>::MIN_BLOCKS;  // no device: do not cache the guess
+  }
+  c = n > 0 ? n : 1;
+  cached.store(c);
+  return c;
+}
+
+int decode_umma_blocks_per_sm(int D) {
+  switch (D) {
+    case 64: return umma_blocks_per_sm_d<64>();
+    case 128: return umma_blocks_per_sm_d<128>();
+    default: return 0;
+  }
 }
 
 int decode_blocks_per_sm(int D) {

@@ -403,7 +403,7 @@ enum {
                                 copy, so that one wait runs out; the keys of that warp are left
                                 out and FP8PD_FLAG_TIMEOUT is set. No copy is in flight on the
                                 stalled stage, so the launch ends normally. */
-  FP8PD_OPT_COMPUTE = 8      /* numerical path of the attention: 0 (default) = f32 compute (K and
+  FP8PD_OPT_COMPUTE = 8,     /* numerical path of the attention: 0 (default) = f32 compute (K and
                                 V decoded exactly, q exact in f16, P as an f16 hi + lo pair; max
                                 |err| <= 1e-3 * max(1, |ref|)); 1 = fp8 compute (the solution
                                 page's compute="fp8": q rounded once to E4M3 per query head after
@@ -411,6 +411,13 @@ enum {
                                 max v_scale * 2^8 rounded once to E4M3, K and V bytes into E4M3
                                 MMAs; the page holds it to 1.5e-1). Per-token scales are refused
                                 on the fp8 path with FP8PD_ERR_UNSUPPORTED, never downgraded. */
+  FP8PD_OPT_KERNEL = 9       /* the attention kernel: 0 = the planner's choice (default), 1 = the
+                                split kernel (mma.sync tiles of 16 tokens per warp), 2 = the
+                                tensor-memory kernel (tcgen05 MMAs on 128-token chunks,
+                                accumulators in TMEM) where it applies -- head dim 64 or 128,
+                                page or head scales, f32 compute, FP8PD_OPT_K_DECODE and
+                                FP8PD_OPT_V_DECODE at 1, no timeout test hook -- else the split
+                                kernel. Both give the same results within the f32 tolerance. */
 };
 int fp8pd_set_option(int32_t option, int64_t value);
 int64_t fp8pd_get_option(int32_t option);
@@ -427,6 +434,7 @@ typedef struct fp8pd_run_info {
   int64_t appends;           /* append calls made by this process */
   int64_t kernel_launches;   /* kernels this library launched in this process */
   int32_t compute;           /* FP8PD_OPT_COMPUTE of the last attention call (0 f32, 1 fp8) */
+  int32_t kernel;            /* kernel of the last attention call: 1 split, 2 tensor-memory */
 } fp8pd_run_info;
 int fp8pd_last_run_info(fp8pd_run_info* info);
 

@@ -19,3 +19,14 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.fail("this test needs a CUDA device; run it with -m gpu on a GPU host")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(autouse=True, scope="session")
+def _attention_kernel_choice():
+    """FP8PD_TEST_KERNEL=1|2 runs the whole suite with FP8PD_OPT_KERNEL set
+    (1 = split kernel, 2 = tensor-memory kernel where it applies)."""
+    k = os.environ.get("FP8PD_TEST_KERNEL")
+    if k is not None:
+        import fp8_paged_decode_split_b200 as F
+        F.fp8pd_set_option(F.OPT_KERNEL, int(k))
+    yield
