@@ -847,7 +847,8 @@ int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_t
   info->combine = plan.combine;
   info->workspace_bytes = plan.workspace;
   info->schedule = plan.schedule;
-  info->warps = plan.grid_blocks * (um ? 5 : fp8pd::decode_warps_per_block(static_cast<int>(D)));
+  // the tensor-memory kernel: 8 compute warps and the QK and PV issuing warps
+  info->warps = plan.grid_blocks * (um ? 10 : fp8pd::decode_warps_per_block(static_cast<int>(D)));
   return FP8PD_OK;
 }
 

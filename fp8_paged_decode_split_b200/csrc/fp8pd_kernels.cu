@@ -2129,7 +2129,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
 // ---------------------------------------------------------------------------
 
 #ifndef FP8PD_UNS_D64
-#define FP8PD_UNS_D64 8
+#define FP8PD_UNS_D64 10
 #endif
 #ifndef FP8PD_UNS_D128
 #define FP8PD_UNS_D128 4
@@ -2142,7 +2142,7 @@ struct UCfg {
   static_assert(NS % 2 == 0 && NS >= 2, "a stage keeps its warpgroup: an even ring");
   static constexpr int NWG = 2;                      // warpgroups (alternate chunks)
   static constexpr int NCW = 4 * NWG;                // compute warps
-  static constexpr int NT = (NCW + 1) * 32;          // + the MMA warp
+  static constexpr int NT = (NCW + 2) * 32;          // + the QK and PV MMA warps
   static constexpr int CHUNK = 128;                  // tokens per chunk (MMA M of QK)
   static constexpr int KV = CHUNK * D;               // K (or V) bytes of a chunk
   static constexpr int STAGE = 2 * KV;
@@ -2222,6 +2222,29 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
   asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
 }
+// Waits for phase `parity` of the barrier with short polls (no suspend hint:
+// a hand-off between warps is seen within the hardware's own short limit),
+// giving up after polls * 20 us of global time (the same bound as mbar_wait).
+__device__ __forceinline__ bool mbar_wait_poll(uint32_t bar, uint32_t parity, int polls) {
+  uint64_t t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  const uint64_t limit = static_cast<uint64_t>(polls) * 20000u;
+#pragma unroll 1
+  for (;;) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (t - t0 > limit) return false;
+  }
+}
+
 __device__ __forceinline__ void named_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
 }
@@ -2267,7 +2290,7 @@ __global__ void __launch_bounds__(UCfg<D>::NT, UCfg<D>::MIN_BLOCKS)
   int b, split, S;
   int prop_j0 = 0, prop_j1 = 0, sp_b = 0, gp_b = 0;
   if (p.prop) {
-    if (!prop_assign<C::NCW + 1>(p, reinterpret_cast<int*>(smem), reinterpret_cast<int*>(misc),
+    if (!prop_assign<C::NCW + 2>(p, reinterpret_cast<int*>(smem), reinterpret_cast<int*>(misc),
                                  head0, nheads, b, split, S, prop_j0, prop_j1, sp_b, gp_b))
       return;
   } else {
@@ -2365,7 +2388,7 @@ __global__ void __launch_bounds__(UCfg<D>::NT, UCfg<D>::MIN_BLOCKS)
   __syncthreads();
   qm = 0.f;
 #pragma unroll
-  for (int w = 0; w <= C::NCW; ++w) qm = fmaxf(qm, m_qmax[w]);
+  for (int w = 0; w < C::NCW + 2; ++w) qm = fmaxf(qm, m_qmax[w]);
   int qe = 0;
   if (qm > 0.f && isfinite(qm)) frexpf(qm, &qe);
   qe = max(qe, -111);
@@ -2399,7 +2422,7 @@ __global__ void __launch_bounds__(UCfg<D>::NT, UCfg<D>::MIN_BLOCKS)
   // other warp blocks on it, and the block's result is zero.
   auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
     if (failed) return false;
-    const bool ok = __all_sync(FULL, mbar_wait(bar, parity, polls) && !*m_abort);
+    const bool ok = __all_sync(FULL, mbar_wait_poll(bar, parity, polls) && !*m_abort);
     if (!ok) {
       failed = true;
       if (lane == 0) {
@@ -2415,23 +2438,7 @@ __global__ void __launch_bounds__(UCfg<D>::NT, UCfg<D>::MIN_BLOCKS)
   auto pready_bar = [&](int c) { return b_pr + 8 * (c % C::NS); };
 
   if (warp == C::NCW) {
-    // ======================= MMA warp (one lane issues) =======================
-    int pv_done = 0;  // chunks whose PV MMAs were issued
-    auto do_pv = [&](int c) {
-      if (!wait(pready_bar(c), (c / C::NS) & 1)) return;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t vb = s_vf + (c & 1) * C::VF16, pb = s_p + (c & 1) * C::PBUF;
-        for (int kk = 0; kk < C::CHUNK / 16; ++kk) {
-          const uint64_t da = umma_sdesc(vb + kk * 2048, 16384, 1024, 2);
-          const uint64_t db = umma_sdesc(pb + kk * 512, 4096, 256, 6);
-          umma_f16(tmem + 32 + 16 * (c & 1), da, db, IDESC_PV, (c > 1 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(b_pv + 8 * (c & 1));
-      }
-      __syncwarp();
-      pv_done = c + 1;
-    };
+    // ======================= QK warp (one lane issues) =======================
     for (int c = 0; c < nch && !failed; ++c) {
       const int s = c % C::NS;
       bool ok = true;
@@ -2451,9 +2458,25 @@ __global__ void __launch_bounds__(UCfg<D>::NT, UCfg<D>::MIN_BLOCKS)
         umma_commit(b_s + 8 * (c & 1));
       }
       __syncwarp();
-      if (c >= 1) do_pv(c - 1);
     }
-    if (!failed && nch > 0) do_pv(nch - 1);
+  } else if (warp == C::NCW + 1) {
+    // ======================= PV warp (one lane issues) =======================
+    int pv_done = 0;  // chunks whose PV MMAs were issued
+    for (int c = 0; c < nch && !failed; ++c) {
+      if (!wait(pready_bar(c), (c / C::NS) & 1)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t vb = s_vf + (c & 1) * C::VF16, pb = s_p + (c & 1) * C::PBUF;
+        for (int kk = 0; kk < C::CHUNK / 16; ++kk) {
+          const uint64_t da = umma_sdesc(vb + kk * 2048, 16384, 1024, 2);
+          const uint64_t db = umma_sdesc(pb + kk * 512, 4096, 256, 6);
+          umma_f16(tmem + 32 + 16 * (c & 1), da, db, IDESC_PV, (c > 1 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(b_pv + 8 * (c & 1));
+      }
+      __syncwarp();
+      pv_done = c + 1;
+    }
     // drain: every committed MMA has finished before the block moves on
     for (int c = max(0, pv_done - 2); c < pv_done; ++c)
       mbar_wait(b_pv + 8 * (c & 1), (c >> 1) & 1, polls);
@@ -2525,8 +2548,45 @@ __global__ void __launch_bounds__(UCfg<D>::NT, UCfg<D>::MIN_BLOCKS)
           if (lane == 0) mbar_arrive(b_patch);
         }
       }
+      // this warp's tiles of the chunk have landed; the group's P and f16 V
+      // buffers are free once the PV of its previous chunk has run
+      wait(full_bar(c, wq), (c / C::NS) & 1);
+      if (c >= 2) wait(b_pv + 8 * g, ((c - 2) >> 1) & 1);
+      {
+        // V row t decoded to f16, MN-major with the 128-byte swizzle: head-dim
+        // entries 64a .. 64a+63 of token t in the 128-byte row t % 8 of k-group
+        // t / 8 of atom a; 16-byte chunk q of that row at q ^ (t % 8)
+        const uint32_t vrow = sv + kt * kTileTokens * D;
+#pragma unroll
+        for (int cb = 0; cb < D / 16; ++cb) {
+          uint4 w = make_uint4(0u, 0u, 0u, 0u);
+          if (valid) {
+            const uint32_t a = vrow + tile_off<D>(r, 16 * cb);
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w) : "r"(a));
+          }
+          const uint32_t f[8] = {e4m3x2_lo16_to_f16x2(w.x), e4m3x2_hi16_to_f16x2(w.x),
+                                 e4m3x2_lo16_to_f16x2(w.y), e4m3x2_hi16_to_f16x2(w.y),
+                                 e4m3x2_lo16_to_f16x2(w.z), e4m3x2_hi16_to_f16x2(w.z),
+                                 e4m3x2_lo16_to_f16x2(w.w), e4m3x2_hi16_to_f16x2(w.w)};
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int d0 = 16 * cb + 8 * u;
+            const int atom = d0 >> 6, q = (d0 & 63) >> 3;
+            const uint32_t dst = vbuf + atom * 16384 + (t >> 3) * 1024 + (t & 7) * 128 +
+                                 ((q ^ (t & 7)) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(f[4 * u]),
+                         "r"(f[4 * u + 1]), "r"(f[4 * u + 2]), "r"(f[4 * u + 3]) : "memory");
+          }
+        }
+      }
+      // QK of the chunk has run: its K is consumed and this warp's V rows are
+      // decoded, so the warp refills its tiles of the stage right away
       wait(b_s + 8 * g, (c >> 1) & 1);
       tc_fence_after();
+      fence_proxy_async();
+      __syncwarp();
+      if (c + C::NS < nch && !failed) issue_part(c + C::NS);
       uint32_t sr[16];
       tmem_ld16(t_s, sr);
       tc_fence_before();
@@ -2576,7 +2636,7 @@ __global__ void __launch_bounds__(UCfg<D>::NT, UCfg<D>::MIN_BLOCKS)
           vref = nv;
           inv_vref = 1.f / nv;
         }
-        if (c >= 2 && wait(b_pv + 8 * g, ((c - 2) >> 1) & 1)) {
+        if (c >= 2 && !failed) {
           // O holds this group's chunks < c: its last PV has run; rescale O in place
           tc_fence_after();
           uint32_t o[16];
@@ -2607,8 +2667,6 @@ __global__ void __launch_bounds__(UCfg<D>::NT, UCfg<D>::MIN_BLOCKS)
         ph[h >> 1] = hh;
         pl[h >> 1] = pack_f16x2(w0 - fh.x, w1 - fh.y);
       }
-      // the group's P and V buffers are free once the PV of its previous chunk has run
-      if (c >= 2) wait(b_pv + 8 * g, ((c - 2) >> 1) & 1);
       {
         // P row t: 32 bytes, 32-byte swizzle (chunk ^= bit 2 of t)
         const uint32_t pr = pbuf + t * 32, sw = (t >> 2) & 1;
@@ -2617,37 +2675,7 @@ __global__ void __launch_bounds__(UCfg<D>::NT, UCfg<D>::MIN_BLOCKS)
         asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(pr + ((sw ^ 1) << 4)),
                      "r"(pl[0]), "r"(pl[1]), "r"(pl[2]), "r"(pl[3]) : "memory");
       }
-      {
-        // V row t decoded to f16, MN-major with the 128-byte swizzle: head-dim
-        // entries 64a .. 64a+63 of token t in the 128-byte row t % 8 of k-group
-        // t / 8 of atom a; 16-byte chunk q of that row at q ^ (t % 8)
-        const uint32_t vrow = sv + kt * kTileTokens * D;
-#pragma unroll
-        for (int cb = 0; cb < D / 16; ++cb) {
-          uint4 w = make_uint4(0u, 0u, 0u, 0u);
-          if (valid) {
-            const uint32_t a = vrow + tile_off<D>(r, 16 * cb);
-            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w) : "r"(a));
-          }
-          const uint32_t f[8] = {e4m3x2_lo16_to_f16x2(w.x), e4m3x2_hi16_to_f16x2(w.x),
-                                 e4m3x2_lo16_to_f16x2(w.y), e4m3x2_hi16_to_f16x2(w.y),
-                                 e4m3x2_lo16_to_f16x2(w.z), e4m3x2_hi16_to_f16x2(w.z),
-                                 e4m3x2_lo16_to_f16x2(w.w), e4m3x2_hi16_to_f16x2(w.w)};
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int d0 = 16 * cb + 8 * u;
-            const int atom = d0 >> 6, q = (d0 & 63) >> 3;
-            const uint32_t dst = vbuf + atom * 16384 + (t >> 3) * 1024 + (t & 7) * 128 +
-                                 ((q ^ (t & 7)) << 4);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(f[4 * u]),
-                         "r"(f[4 * u + 1]), "r"(f[4 * u + 2]), "r"(f[4 * u + 3]) : "memory");
-          }
-        }
-      }
       fence_proxy_async();
-      __syncwarp();  // the warp's V rows of this stage are decoded: refill its tiles
-      if (c + C::NS < nch && !failed) issue_part(c + C::NS);
       mbar_arrive(pready_bar(c));
     }
     // copies of this warp still in flight (only after a failed wait) land first
@@ -2784,12 +2812,12 @@ __global__ void __launch_bounds__(UCfg<D>::NT, UCfg<D>::MIN_BLOCKS)
   float* fo = fin ? nullptr : p.pout_o;
   const int64_t frow = (int64_t)b * p.Hq + head0;
   if (NG == 1) {
-    merge_partials<D, C::NCW + 1>(p.part_ml, p.part_o, prow0, S, S, nheads, fin, p, b, head0, fml,
+    merge_partials<D, C::NCW + 2>(p.part_ml, p.part_o, prow0, S, S, nheads, fin, p, b, head0, fml,
                                   fo, frow, 1, wts);
     if (tid == 0) ucnt[1] = 0;
     return;
   }
-  merge_partials<D, C::NCW + 1>(p.part_ml, p.part_o, prow0 + gi * kMergeFan, S, gsize, nheads,
+  merge_partials<D, C::NCW + 2>(p.part_ml, p.part_o, prow0 + gi * kMergeFan, S, gsize, nheads,
                                 false, p, b, head0, p.grp_ml, p.grp_o, grow0 + gi, NG, wts);
   if (tid == 0) ucnt[1 + gi] = 0;
   __syncthreads();
@@ -2800,7 +2828,7 @@ __global__ void __launch_bounds__(UCfg<D>::NT, UCfg<D>::MIN_BLOCKS)
   __syncthreads();
   if (!*flag) return;
   __threadfence();
-  merge_partials<D, C::NCW + 1>(p.grp_ml, p.grp_o, grow0, NG, NG, nheads, fin, p, b, head0, fml,
+  merge_partials<D, C::NCW + 2>(p.grp_ml, p.grp_o, grow0, NG, NG, nheads, fin, p, b, head0, fml,
                                 fo, frow, 1, wts);
   if (tid == 0) ucnt[0] = 0;
 }

@@ -216,6 +216,13 @@ def test_options_roundtrip(F):
     F.fp8pd_set_option(F.OPT_K_DECODE, 1)
     with pytest.raises(F.Fp8pdError):
         F.fp8pd_set_option(F.OPT_K_DECODE, 3)
+    assert F.fp8pd_get_option(F.OPT_KERNEL) == 0
+    for k in (1, 2, 0):
+        F.fp8pd_set_option(F.OPT_KERNEL, k)
+        assert F.fp8pd_get_option(F.OPT_KERNEL) == k
+    for bad in (3, -1):
+        with pytest.raises(F.Fp8pdError):
+            F.fp8pd_set_option(F.OPT_KERNEL, bad)
     with pytest.raises(F.Fp8pdError):
         F.fp8pd_set_option(99, 1)
     with pytest.raises(F.Fp8pdError):
@@ -308,6 +315,24 @@ def test_planner_proportional_splits(F):
     finally:
         F.fp8pd_set_option(F.OPT_NUM_SPLITS, 0)
         F.fp8pd_set_option(F.OPT_SCHEDULE, 0)
+
+
+def test_planner_plans_for_the_kernel_that_runs(F):
+    """With the tensor-memory kernel requested (head dim 64 / 128), the plan
+    counts that kernel's blocks per SM (one without a GPU, against four or
+    five for the split kernel), so it plans fewer blocks; head dims it does not
+    take plan as before."""
+    try:
+        F.fp8pd_set_option(F.OPT_KERNEL, 1)
+        split = _plan(F, 8, 64, 8, 128, 64, 2049)
+        d256 = _plan(F, 4, 16, 8, 256, 32, 200)
+        F.fp8pd_set_option(F.OPT_KERNEL, 2)
+        umma = _plan(F, 8, 64, 8, 128, 64, 2049)
+        assert umma["grid_blocks"] < split["grid_blocks"]
+        assert umma["warps"] == umma["grid_blocks"] * 10
+        assert _plan(F, 4, 16, 8, 256, 32, 200) == d256
+    finally:
+        F.fp8pd_set_option(F.OPT_KERNEL, 0)
 
 
 def test_partial_and_combine_validation(F):
