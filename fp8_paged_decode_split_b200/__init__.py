@@ -68,7 +68,7 @@ class RunInfo(ctypes.Structure):
                 ("combine", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("calls", ctypes.c_int64), ("appends", ctypes.c_int64),
                 ("kernel_launches", ctypes.c_int64), ("compute", ctypes.c_int32),
-                ("kernel", ctypes.c_int32)]
+                ("kernel", ctypes.c_int32), ("dim_split", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:

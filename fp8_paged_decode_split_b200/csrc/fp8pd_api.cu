@@ -220,9 +220,18 @@ bool use_umma(int D, bool tok, bool mx, int k_groups) {
   return k == 2 || kUmmaByDefault;
 }
 
+// Whether the split kernel runs a call with two warps per tile stream, each
+// on half of the head dim: D = 512 with page or head scales, f32 compute with
+// the hardware-cvt decodes and no fused append (at D = 512 a block of four
+// whole-width streams fills the SM's shared memory with four warps).
+bool use_dsplit(int D, bool tok, bool mx, int k_groups, bool append, bool umma) {
+  if (D != 512 || umma || tok || mx || k_groups > 1 || append) return false;
+  return g_opt_compute.load() == 0 && g_opt_k_decode.load() == 1 && g_opt_v_decode.load() == 1;
+}
+
 // Thread blocks one SM holds for the kernel that will run.
-int blocks_per_sm(int D, bool umma) {
-  return umma ? fp8pd::decode_umma_blocks_per_sm(D) : fp8pd::decode_blocks_per_sm(D);
+int blocks_per_sm(int D, bool umma, int dsplit = 1) {
+  return umma ? fp8pd::decode_umma_blocks_per_sm(D) : fp8pd::decode_blocks_per_sm(D, dsplit);
 }
 
 bool plan_proportional(int B, int Hq, int Hkv, int D, int ps, int max_pages, int window,
@@ -362,9 +371,10 @@ struct MapKey {
   const void* base;
   int64_t shape[4];
   int64_t stride[4];
+  int dsplit;
   bool operator==(const MapKey& o) const {
     return base == o.base && std::memcmp(shape, o.shape, sizeof(shape)) == 0 &&
-           std::memcmp(stride, o.stride, sizeof(stride)) == 0;
+           std::memcmp(stride, o.stride, sizeof(stride)) == 0 && dsplit == o.dsplit;
   }
 };
 struct MapEntry {
@@ -374,8 +384,11 @@ struct MapEntry {
 std::mutex g_map_mutex;
 std::vector<MapEntry> g_maps;  // small most-recently-used cache
 
-int make_pool_map(const fp8pd_tensor* pool, CUtensorMap* out) {
-  MapKey key{pool->data, {}, {}};
+// The box is one 16-token tile of one KV head: whole rows, or with dsplit = 2
+// the first half of each row (the kernel moves the start to the second half).
+int make_pool_map(const fp8pd_tensor* pool, CUtensorMap* out, int dsplit = 1) {
+  if (dsplit != 2) dsplit = 1;
+  MapKey key{pool->data, {}, {}, dsplit};
   for (int i = 0; i < 4; ++i) {
     key.shape[i] = pool->shape[i];
     key.stride[i] = pool->stride[i];
@@ -399,8 +412,9 @@ int make_pool_map(const fp8pd_tensor* pool, CUtensorMap* out) {
   const cuuint64_t strides[4] = {static_cast<cuuint64_t>(pool->stride[1]), 128,
                                  static_cast<cuuint64_t>(pool->stride[2]),
                                  static_cast<cuuint64_t>(pool->stride[0])};
+  if (nblk % dsplit != 0) return FP8PD_ERR_SHAPE;
   const cuuint32_t box[5] = {static_cast<cuuint32_t>(x), static_cast<cuuint32_t>(fp8pd::kTileTokens),
-                             static_cast<cuuint32_t>(nblk), 1, 1};
+                             static_cast<cuuint32_t>(nblk / dsplit), 1, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUtensorMap map;
   const CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, pool->data, dims, strides, box, estr,
@@ -641,8 +655,9 @@ cudaError_t launch_planned(const Plan& plan, const DecodeParams& p, const CUtens
   return fp8pd::launch_decode(p, tmk, tmv, k_mode, g_opt_v_decode.load() == 1, s);
 }
 
-void record_run(const Plan& plan, int D, bool umma) {
+void record_run(const Plan& plan, int D, bool umma, int dsplit) {
   t_run_info.kernel = umma ? 2 : 1;
+  t_run_info.dim_split = umma ? 1 : dsplit;
   t_run_info.schedule = plan.schedule;
   t_run_info.num_splits = plan.num_splits;
   t_run_info.head_groups = plan.head_groups;
@@ -669,6 +684,8 @@ int run_decode(DecodeParams& p, const DecodeArgs& a, const fp8pd_tensor* k_pages
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   apply_plan(plan, &p);
   p.umma = um ? 1 : 0;
+  p.dsplit = use_dsplit(a.D, p.k_tok || p.v_tok, p.k_mx || p.v_mx, p.k_groups, p.append != 0, um)
+                 ? 2 : 1;
   if (plan.combine) {
     void *ctr = nullptr, *part = nullptr;
     r = get_workspace(plan.counters_bytes, plan.workspace - plan.counters_bytes, s, &ctr, &part);
@@ -676,8 +693,8 @@ int run_decode(DecodeParams& p, const DecodeArgs& a, const fp8pd_tensor* k_pages
     lay_out(plan, ctr, part, &p);
   }
   CUtensorMap tmk, tmv;
-  if ((r = make_pool_map(k_pages, &tmk))) return r;
-  if ((r = make_pool_map(v_pages, &tmv))) return r;
+  if ((r = make_pool_map(k_pages, &tmk, p.dsplit))) return r;
+  if ((r = make_pool_map(v_pages, &tmv, p.dsplit))) return r;
   EventPair* ev = timing_slot(0);
   if (ev) cudaEventRecord(ev->a, s);
   cudaError_t e = launch_planned(plan, p, tmk, tmv, s);
@@ -685,7 +702,7 @@ int run_decode(DecodeParams& p, const DecodeArgs& a, const fp8pd_tensor* k_pages
   ++g_launches;
   if (ev) cudaEventRecord(ev->b, s);
   ++g_calls;
-  record_run(plan, a.D, p.umma != 0);
+  record_run(plan, a.D, p.umma != 0, p.dsplit);
   return FP8PD_OK;
 }
 
@@ -848,7 +865,8 @@ int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_t
   info->workspace_bytes = plan.workspace;
   info->schedule = plan.schedule;
   // the tensor-memory kernel: 8 compute warps and the QK and PV issuing warps
-  info->warps = plan.grid_blocks * (um ? 10 : fp8pd::decode_warps_per_block(static_cast<int>(D)));
+  const int ds = use_dsplit(static_cast<int>(D), false, false, 1, false, um) ? 2 : 1;
+  info->warps = plan.grid_blocks * (um ? 10 : fp8pd::decode_warps_per_block(static_cast<int>(D), ds));
   return FP8PD_OK;
 }
 
@@ -1141,6 +1159,8 @@ extern "C" int fp8_paged_decode_attention_noalloc(
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   apply_plan(plan, &p);
   p.umma = um ? 1 : 0;
+  p.dsplit = use_dsplit(a.D, p.k_tok || p.v_tok, p.k_mx || p.v_mx, p.k_groups, p.append != 0, um)
+                 ? 2 : 1;
   if (plan.combine) {
     void* ws = nullptr;
     r = noalloc_scratch(&ws);
@@ -1153,12 +1173,12 @@ extern "C" int fp8_paged_decode_attention_noalloc(
     lay_out(plan, base, base + plan.counters_bytes, &p);
   }
   CUtensorMap tmk, tmv;
-  if ((r = make_pool_map(k_pages, &tmk))) return r;
-  if ((r = make_pool_map(v_pages, &tmv))) return r;
+  if ((r = make_pool_map(k_pages, &tmk, p.dsplit))) return r;
+  if ((r = make_pool_map(v_pages, &tmv, p.dsplit))) return r;
   const cudaError_t e = launch_planned(plan, p, tmk, tmv, s);
   if (e != cudaSuccess) return fail_cuda(e);
   ++g_launches;
   ++g_calls;
-  record_run(plan, a.D, p.umma != 0);
+  record_run(plan, a.D, p.umma != 0, p.dsplit);
   return FP8PD_OK;
 }

@@ -80,6 +80,10 @@ struct DecodeParams {
   // 1: the tensor-memory kernel (D = 64 / 128, page or head scales, f32
   // compute) runs this call
   int umma;
+  // Warps sharing each tile stream of the split kernel, each on its part of
+  // the head dim: 1, or 2 at D = 512 (page or head scales, f32 compute with
+  // the cvt decodes, no fused append), where the tensor maps copy half rows.
+  int dsplit;
 };
 
 struct AppendParams {
@@ -125,14 +129,15 @@ cudaError_t launch_combine(const float* po, const float* pml, int R, int B, int 
 cudaError_t launch_encode(const float* x, int64_t xs, uint8_t* c, int64_t cs, int64_t n,
                           cudaStream_t s);
 
-// Thread blocks of the split kernel one SM holds for head dim D.
-int decode_blocks_per_sm(int D);
+// Thread blocks of the split kernel one SM holds for head dim D (dsplit: the
+// warps sharing each tile stream, 1 or 2).
+int decode_blocks_per_sm(int D, int dsplit = 1);
 // Thread blocks of the tensor-memory kernel one SM holds (D = 64 / 128; else 0).
 int decode_umma_blocks_per_sm(int D);
 // Warps per block of the split kernel for head dim D.
-int decode_warps_per_block(int D);
+int decode_warps_per_block(int D, int dsplit = 1);
 // Dynamic shared memory of the split kernel for head dim D.
-int decode_smem_bytes(int D);
+int decode_smem_bytes(int D, int dsplit = 1);
 
 // Device error word (one per device): read and cleared by the host API.
 cudaError_t read_and_clear_error_word(uint32_t* value, cudaStream_t s);

@@ -356,27 +356,40 @@ __device__ __forceinline__ uint32_t tile_off(int r, int b) {
   }
 }
 
-template <int D>
+// DS (head-dim split): each tile stream of a block is shared by DS warps,
+// warp h of the stream copying and contracting head-dim entries
+// [h * D / DS, (h + 1) * D / DS) of every tile (its own ring of half-width
+// tiles), the partial scores summed through shared memory once per tile.
+// DS = 2 is built for D = 512 only, where a block of four whole-width
+// streams fills the SM's shared memory with four warps.
+template <int D, int DS = 1>
 struct Cfg {
-  static constexpr int NW = (D == 64) ? FP8PD_NW_D64 : (D == 128) ? FP8PD_NW_D128 : (D == 256) ? FP8PD_NW_D256 : FP8PD_NW_D512;  // warps per block
+  static_assert(DS == 1 || (DS == 2 && D == 512), "head-dim split: D = 512, two warps");
+  static constexpr int DW = D / DS;                                    // head-dim entries per warp
+  static constexpr int NLW = (D == 64) ? FP8PD_NW_D64 : (D == 128) ? FP8PD_NW_D128 : (D == 256) ? FP8PD_NW_D256 : FP8PD_NW_D512;  // tile streams per block
+  static constexpr int NW = NLW * DS;                                  // warps per block
   static constexpr int NT = NW * 32;                                  // threads per block
   static constexpr int NS = (D == 64) ? FP8PD_NS_D64 : (D == 128) ? FP8PD_NS_D128 : (D == 256) ? FP8PD_NS_D256 : FP8PD_NS_D512;  // ring stages per warp
   static constexpr bool PAIR = (D == 64) && FP8PD_PAIR_D64;           // two tiles per softmax step
-  static constexpr int TILE = kTileTokens * D;                        // bytes of a K or V tile
+  static constexpr int TILE = kTileTokens * DW;                       // bytes of a warp's K or V tile
   static constexpr int STAGE = 2 * TILE;
   static constexpr int WARP_BYTES = NS * STAGE;
   static constexpr int PIPE_BYTES = NW * WARP_BYTES;                  // multiple of 1024
   static constexpr bool Q_IN_SMEM = (D > 256);                        // q fragments in smem
   static constexpr int QFRAG_BYTES = Q_IN_SMEM ? (D / 16) * 32 * 8 : 0;
-  static constexpr int LIST_BYTES = NW * kMaxWarpTiles * 12;          // tile entry, k / v scale
+  // per stream, two buffers of the DS warps' score fragments (float4 per lane) and their flags
+  static constexpr int XCH_BYTES = DS > 1 ? NLW * 2 * DS * (32 * 16 + 16) : 0;
+  static constexpr int LIST_BYTES = NLW * kMaxWarpTiles * 12;         // tile entry, k / v scale
   static constexpr int BAR_BYTES = NW * NS * 8;
   static constexpr int MISC_FLOATS = NW * 8 * 2 + 4;
-  static constexpr int SMEM = 1024 /* alignment slack */ + PIPE_BYTES + QFRAG_BYTES + LIST_BYTES +
-                              BAR_BYTES + MISC_FLOATS * 4;
+  static constexpr int SMEM = 1024 /* alignment slack */ + PIPE_BYTES + QFRAG_BYTES + XCH_BYTES +
+                              LIST_BYTES + BAR_BYTES + MISC_FLOATS * 4;
   static constexpr int MIN_BLOCKS = (D == 512) ? 1 : (D == 256) ? FP8PD_MIN_BLOCKS_D256 : (D == 128) ? FP8PD_MIN_BLOCKS_D128 : FP8PD_MIN_BLOCKS_D64;
   static_assert(PIPE_BYTES % 1024 == 0, "tiles must stay 1024-byte aligned for the swizzle");
-  static_assert(NW * 8 * D * 4 <= PIPE_BYTES, "merge scratch must fit in the ring");
+  static_assert(DW % 128 == 0 || DS == 1, "a warp's part of a row is whole 128-byte blocks");
+  static_assert(NLW * 8 * D * 4 <= PIPE_BYTES, "merge scratch must fit in the ring");
   static_assert(8 * 32 * 4 <= PIPE_BYTES, "merge weights must fit in the ring");
+  static_assert(SMEM <= 232448, "shared memory per block");
 };
 
 // Merges K partial rows (max m, sum l, numerator O, all in log2 units) of one
@@ -1364,11 +1377,14 @@ __device__ bool prop_assign(const DecodeParams& p, int* scratch, int* red, int h
 // views, dims (head-dim bytes within a 128-byte block, slot, 128-byte block,
 // KV head, page), box (min(D,128), 16, max(1, D/128), 1, 1). TOK: the scales
 // are read per token (one per stored token and KV head) instead of per page.
-template <int D, int KM, bool VCVT, int SC>
-__global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
+template <int D, int KM, bool VCVT, int SC, int DS = 1>
+__global__ void __launch_bounds__(Cfg<D, DS>::NT, Cfg<D, DS>::MIN_BLOCKS)
     decode_tma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
-  using C = Cfg<D>;
+  using C = Cfg<D, DS>;
+  static_assert(DS == 1 || (KM == 1 && VCVT && SC == 0 && C::Q_IN_SMEM),
+                "head-dim split: page or head scales, cvt decodes, q fragments in smem");
+  constexpr int DW = C::DW;  // head-dim entries this warp copies and contracts
   constexpr bool TOK = SC >= 1;  // scales read per stored token
   constexpr bool VMX = SC == 2;  // V in MXFP8 (E8M0 block scales)
   constexpr int KB = D / 16;  // k16 blocks of the QK contraction
@@ -1377,14 +1393,22 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* pipe = smem;
   uint2* qfrag_s = reinterpret_cast<uint2*>(smem + C::PIPE_BYTES);
-  int32_t* s_ent = reinterpret_cast<int32_t*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES);
-  float* s_ks = reinterpret_cast<float*>(s_ent + C::NW * kMaxWarpTiles);
-  float* s_vs = s_ks + C::NW * kMaxWarpTiles;
-  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_vs + C::NW * kMaxWarpTiles);
+  float4* s_xch = reinterpret_cast<float4*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES);
+  int32_t* s_ent = reinterpret_cast<int32_t*>(smem + C::PIPE_BYTES + C::QFRAG_BYTES + C::XCH_BYTES);
+  float* s_ks = reinterpret_cast<float*>(s_ent + C::NLW * kMaxWarpTiles);
+  float* s_vs = s_ks + C::NLW * kMaxWarpTiles;
+  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_vs + C::NLW * kMaxWarpTiles);
   float* misc = reinterpret_cast<float*>(s_bar + C::NW * C::NS);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, grp = lane >> 2, qd = lane & 3;
+  // tile stream lw of the block; this warp's part of its head dim: `half`
+  const int lw = warp / DS, half = warp - lw * DS;
+  // The DS warps of a stream meet at named barrier 1 + lw (64 threads).
+  auto stream_sync = [&]() {
+    if constexpr (DS > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + lw), "r"(DS * 32) : "memory");
+    else __syncwarp();
+  };
   const int kvh = blockIdx.x / p.head_groups;
   const int hg = blockIdx.x - kvh * p.head_groups;
   const int head0 = kvh * p.G + hg * 8;
@@ -1471,8 +1495,8 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
       stall = false;
       return;
     }
-    tma_load_5d(sk, &tmk, bar, 0, slot0, 0, kvh, page);
-    tma_load_5d(sk + C::TILE, &tmv, bar, 0, slot0, 0, kvh, page);
+    tma_load_5d(sk, &tmk, bar, 0, slot0, half * (DW / 128), kvh, page);
+    tma_load_5d(sk + C::TILE, &tmv, bar, 0, slot0, half * (DW / 128), kvh, page);
   };
   // Without a window a split starts at page split * chunk whatever the
   // sequence length, so the first tiles of each warp are copied before the
@@ -1485,7 +1509,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
     const int tf = p.prop ? prop_j0 : split * p.chunk_pages * (p.ps / kTileTokens);
     int e = -1;
     if (lane < C::NS - 1) {
-      const int tok = (tf + warp + C::NW * lane) * kTileTokens;
+      const int tok = (tf + lw + C::NLW * lane) * kTileTokens;
       const int lp = tok / p.ps;
       if (lp < p.max_pages) {
         const int page = __ldg(trow + (int64_t)lp * p.tab_sp);
@@ -1517,24 +1541,24 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
   }
   const int tile_first = t0 / kTileTokens;
   const int n_tiles = (t1 > t0) ? (t1 + kTileTokens - 1) / kTileTokens - tile_first : 0;
-  int my_tiles = (n_tiles > warp) ? (n_tiles - warp + C::NW - 1) / C::NW : 0;
+  int my_tiles = (n_tiles > lw) ? (n_tiles - lw + C::NLW - 1) / C::NLW : 0;
   if (my_tiles > kMaxWarpTiles) {  // the planner never does this; refuse rather than overflow
     if (lane == 0) raise_flag(FP8PD_FLAG_INTERNAL);
     my_tiles = 0;
   }
 
   // ---- warp-local setup: tile list, first copies, scales, q fragments -------
-  // Tile j of warp w starts at token 16 * (tile_first + w + 4j). Its entry is
+  // Tile j of stream w starts at token 16 * (tile_first + w + 4j). Its entry is
   // (page << 4) | (tile index inside the page), or -1 for a block-table entry
   // outside the pool; the page's k and v scales sit beside it. The page ids
   // come first so the first tile copies are in flight while the scales and
   // the q fragments load.
-  int32_t* went = s_ent + warp * kMaxWarpTiles;
-  float* wks = s_ks + warp * kMaxWarpTiles;
-  float* wvs = s_vs + warp * kMaxWarpTiles;
+  int32_t* went = s_ent + lw * kMaxWarpTiles;
+  float* wks = s_ks + lw * kMaxWarpTiles;
+  float* wvs = s_vs + lw * kMaxWarpTiles;
 #pragma unroll 2
-  for (int j = lane; j < my_tiles; j += 32) {
-    const int tok = (tile_first + warp + C::NW * j) * kTileTokens;
+  for (int j = lane; half == 0 && j < my_tiles; j += 32) {
+    const int tok = (tile_first + lw + C::NLW * j) * kTileTokens;
     const int lp = tok / p.ps;
     const int page = __ldg(trow + (int64_t)lp * p.tab_sp);
     int e = -1;
@@ -1545,7 +1569,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
     }
     went[j] = e;
   }
-  __syncwarp();
+  stream_sync();
 
   if (!spec) {
 #pragma unroll 1
@@ -1560,7 +1584,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
   const float* vsbase = p.vs + (int64_t)kvh * p.vs_sh;
   if constexpr (!TOK) {
 #pragma unroll 2
-    for (int j = lane; j < my_tiles; j += 32) {
+    for (int j = lane; half == 0 && j < my_tiles; j += 32) {
       const int e = went[j];
       if (e >= 0) {
         cp_async4(wks + j, ksbase + (int64_t)(e >> 4) * p.ks_sp);
@@ -1690,17 +1714,21 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
       qf[kb][1] = r1;
     }
   }
+  // With a head-dim split the stream's first warp copied the scales: its
+  // copies complete before the block barrier, which shows them to the other.
+  if constexpr (DS > 1) cp_async_wait_all();
   if constexpr (C::Q_IN_SMEM) __syncthreads();
   __syncwarp();
 
   // ---- per-warp pipeline over 16-token tiles --------------------------------
   uint32_t koff[4], voff[4];
-  ldsm_offsets<D>(lane, koff, voff);
+  ldsm_offsets<DW>(lane, koff, voff);
+  // q' fragment of k16 block kb of this warp's part of the head dim
   auto qfr = [&](int kb) -> uint2 {
-    if constexpr (C::Q_IN_SMEM) return qfrag_s[kb * 32 + lane];
+    if constexpr (C::Q_IN_SMEM) return qfrag_s[(kb + half * (DW / 16)) * 32 + lane];
     else return make_uint2(qf[kb][0], qf[kb][1]);
   };
-  Acc<D> acc;
+  Acc<DW> acc;
   acc.reset();
   bool ok_all = true;
 
@@ -1710,7 +1738,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
   auto tok_scale = [&](int j) -> float {
     const int e = went[j];
     const int r = lane & 15;
-    const int t = (tile_first + warp + C::NW * j) * kTileTokens + r;
+    const int t = (tile_first + lw + C::NLW * j) * kTileTokens + r;
     if (e < 0 || t < t0 || t >= t1 || (lane < 16 && p.k_groups > 1)) return 0.f;
     if (VMX && lane >= 16) return 1.f;  // attended; the tile's MX scale comes later
     const int64_t slot = (e & 15) * kTileTokens + r;
@@ -1732,7 +1760,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
     if (!VMX || lane < 16) return;
     const int e = went[j];
     const int r = lane - 16;
-    const int t = (tile_first + warp + C::NW * j) * kTileTokens + r;
+    const int t = (tile_first + lw + C::NLW * j) * kTileTokens + r;
     if (e < 0 || t < t0 || t >= t1) return;
     const uint8_t* src = vs8 + (int64_t)(e >> 4) * p.vs_sp +
                          (int64_t)((e & 15) * kTileTokens + r) * p.vs_st;
@@ -1778,15 +1806,15 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
 
   int stage = 0;
   uint32_t phase = 0;
-  int tok0 = (tile_first + warp) * kTileTokens;
+  int tok0 = (tile_first + lw) * kTileTokens;
   // two tiles per softmax step: the ring must hold both next to the one being
   // refilled, so the step needs at least three stages
-  constexpr bool PAIRS = (C::PAIR || KM == 3) && C::NS >= 3;
+  constexpr bool PAIRS = (C::PAIR || KM == 3) && C::NS >= 3 && DS == 1;
   if constexpr (PAIRS && !TOK) {
     // Two tiles per step while two are left (one softmax update per 32 keys;
     // the copy into the first tile's stage is issued once its PV is done).
 #pragma unroll 1
-    for (int j = 0; j + 1 < my_tiles; j += 2, tok0 += 2 * C::NW * kTileTokens) {
+    for (int j = 0; j + 1 < my_tiles; j += 2, tok0 += 2 * C::NLW * kTileTokens) {
       const int st1 = (stage + 1 == C::NS) ? 0 : stage + 1;
       const uint32_t ph1 = (stage + 1 == C::NS) ? (phase ^ 1u) : phase;
       if (!mbar_wait(wbar + 8 * stage, phase, p.wait_polls) || !mbar_wait(wbar + 8 * st1, ph1, p.wait_polls)) {
@@ -1808,7 +1836,7 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int jj = j + u;
-        tk[u] = tok0 + u * C::NW * kTileTokens;
+        tk[u] = tok0 + u * C::NLW * kTileTokens;
         pok[u] = went[jj] >= 0;
         full[u] = pok[u] && tk[u] >= t0 && tk[u] + kTileTokens <= t1;
         sk[u] = wpipe + (u ? st1 : st0) * C::STAGE;
@@ -1838,9 +1866,54 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
                                  }, hf);
     }
   }
+  if constexpr (DS > 1) {
+    // Head-dim split: each warp of the stream waits for its own half-width
+    // tile, contracts its part of S, and the two parts (and whether each
+    // copy arrived) meet in shared memory, so both warps run the same
+    // softmax on the same scores and leave the loop together; then each
+    // accumulates its own head-dim part of O. The copy into the previous
+    // stage is issued once both have decided to go on.
+    int* s_xok = reinterpret_cast<int*>(s_xch + C::NLW * 2 * DS * 32);
+#pragma unroll 1
+    for (int j = 0; ok_all && j < my_tiles; ++j, tok0 += C::NLW * kTileTokens) {
+      const bool got = mbar_wait(wbar + 8 * stage, phase, p.wait_polls);
+      if (!got && lane == 0) raise_flag(FP8PD_FLAG_TIMEOUT);
+      const bool page_ok = went[j] >= 0;
+      const bool full = page_ok && tok0 >= t0 && tok0 + kTileTokens <= t1;  // warp-uniform
+      const uint32_t sk = wpipe + stage * C::STAGE;
+      const uint32_t sv = sk + C::TILE;
+      const float kfac = score_base * wks[j];
+      const float vs = wvs[j];
+      // (a tile that never arrived is read all the same; its scores are dropped)
+      float4 sc = tile_scores<DW, 1>(qfr, sk, koff, kfac, kfac, tok0, t0, t1, page_ok, full, grp);
+      const int xb = (lw * 2 + (j & 1)) * DS;  // this tile's buffer of the stream
+      s_xch[(xb + half) * 32 + lane] = sc;
+      if (lane == 0) s_xok[xb + half] = got ? 1 : 0;
+      stream_sync();
+      const float4 o = s_xch[(xb + (half ^ 1)) * 32 + lane];
+      if (!got || s_xok[xb + (half ^ 1)] == 0) {
+        ok_all = false;
+        break;
+      }
+      // a + b == b + a: both warps hold the same sums
+      sc = make_float4(sc.x + o.x, sc.y + o.y, sc.z + o.z, sc.w + o.w);
+      {
+        const int nj = j + C::NS - 1;
+        if (nj < my_tiles) issue(went[nj], stage == 0 ? C::NS - 1 : stage - 1);
+      }
+      if (++stage == C::NS) {
+        stage = 0;
+        phase ^= 1;
+      }
+      softmax_rescale<DW, true>(acc, fmaxf(sc.x, sc.z), fmaxf(sc.y, sc.w), fabsf(vs));
+      uint32_t bh[2], bl[2];
+      tile_probs<DW>(acc, sc, vs, vs, bh, bl);
+      tile_pv<DW, VCVT>(acc, sv, voff, bh, bl, tok0, t0, t1, page_ok, full, qd);
+    }
+  } else {
 #pragma unroll 1
   for (int j = (PAIRS && !TOK) ? (my_tiles & ~1) : 0; ok_all && j < my_tiles;
-       ++j, tok0 += C::NW * kTileTokens) {
+       ++j, tok0 += C::NLW * kTileTokens) {
     if (!mbar_wait(wbar + 8 * stage, phase, p.wait_polls)) {
       if (lane == 0) raise_flag(FP8PD_FLAG_TIMEOUT);
       ok_all = false;
@@ -1952,7 +2025,8 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
                                  t0, t1, page_ok, full, grp, qd, hf);
     }
   }
-  if constexpr (KM != 3) lazy_finish<D>(acc);
+  }
+  if constexpr (KM != 3) lazy_finish<DW>(acc);
   if (!ok_all) {
     // A copy never completed: leave this warp's result out (its flag is set)
     // and wait, again bounded, for whatever this warp still has in flight.
@@ -1973,27 +2047,27 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
     acc.l1 += __shfl_xor_sync(0xffffffffu, acc.l1, o);
   }
   __syncthreads();  // every warp is done with its ring
-  float* Os = reinterpret_cast<float*>(pipe);  // [NW][8][D], already times fold
-  float* ml = misc;                            // [NW][8][2]
+  float* Os = reinterpret_cast<float*>(pipe);  // [NLW][8][D], already times fold
+  float* ml = misc;                            // [NLW][8][2]
   // f16 offset of the decoded V (bit assembly only), times the V reference scale
   const float fold = !ok_all ? 0.f : KM == 3 ? acc.vref * (1.f / 256.f)
                                               : (VCVT ? 1.f : 256.f) * acc.vref;
 #pragma unroll
-  for (int jb = 0; jb < D / 32; ++jb) {
-    const int d = 32 * jb + 2 * grp;
+  for (int jb = 0; jb < DW / 32; ++jb) {
+    const int d = half * DW + 32 * jb + 2 * grp;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      *reinterpret_cast<float2*>(Os + (warp * 8 + 2 * qd) * D + d + 16 * h) =
+      *reinterpret_cast<float2*>(Os + (lw * 8 + 2 * qd) * D + d + 16 * h) =
           make_float2(acc.O[jb][h][0] * fold, acc.O[jb][h][2] * fold);
-      *reinterpret_cast<float2*>(Os + (warp * 8 + 2 * qd + 1) * D + d + 16 * h) =
+      *reinterpret_cast<float2*>(Os + (lw * 8 + 2 * qd + 1) * D + d + 16 * h) =
           make_float2(acc.O[jb][h][1] * fold, acc.O[jb][h][3] * fold);
     }
   }
-  if (grp == 0) {
-    ml[(warp * 8 + 2 * qd) * 2 + 0] = acc.m0;
-    ml[(warp * 8 + 2 * qd) * 2 + 1] = acc.l0;
-    ml[(warp * 8 + 2 * qd + 1) * 2 + 0] = acc.m1;
-    ml[(warp * 8 + 2 * qd + 1) * 2 + 1] = acc.l1;
+  if (grp == 0 && half == 0) {  // (m, l) are the same in every warp of a stream
+    ml[(lw * 8 + 2 * qd) * 2 + 0] = acc.m0;
+    ml[(lw * 8 + 2 * qd) * 2 + 1] = acc.l0;
+    ml[(lw * 8 + 2 * qd + 1) * 2 + 0] = acc.m1;
+    ml[(lw * 8 + 2 * qd + 1) * 2 + 1] = acc.l1;
   }
   __syncthreads();
 
@@ -2020,12 +2094,12 @@ __global__ void __launch_bounds__(Cfg<D>::NT, Cfg<D>::MIN_BLOCKS)
     if (n >= nheads) continue;
     float M = -CUDART_INF_F;
 #pragma unroll
-    for (int w = 0; w < C::NW; ++w) M = fmaxf(M, ml[(w * 8 + n) * 2]);
+    for (int w = 0; w < C::NLW; ++w) M = fmaxf(M, ml[(w * 8 + n) * 2]);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float l = 0.f;
     if (M != -CUDART_INF_F) {
 #pragma unroll
-      for (int w = 0; w < C::NW; ++w) {
+      for (int w = 0; w < C::NLW; ++w) {
         const float mw = ml[(w * 8 + n) * 2];
         const float f = (mw == -CUDART_INF_F) ? 0.f : fast_exp2(mw - M);
         const float4 o = *reinterpret_cast<const float4*>(Os + (w * 8 + n) * D + d);
@@ -2932,26 +3006,26 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
 // ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
-template <int D, int KM, bool VCVT, int SC>
+template <int D, int KM, bool VCVT, int SC, int DS = 1>
 static cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap& tmk,
                                    const CUtensorMap& tmv, cudaStream_t s) {
   // The shared-memory opt-in is a per-device function attribute: set it once
   // per device (an idempotent call, so a race only repeats it).
   static std::atomic<uint64_t> configured{0};
-  const int smem = Cfg<D>::SMEM;
+  const int smem = Cfg<D, DS>::SMEM;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
   if (!bit || !(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(decode_tma_kernel<D, KM, VCVT, SC>,
+    e = cudaFuncSetAttribute(decode_tma_kernel<D, KM, VCVT, SC, DS>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
   const dim3 grid = p.prop ? dim3(p.Hkv * p.head_groups, p.nbx, 1)
                            : dim3(p.Hkv * p.head_groups, p.B, p.num_splits);
-  decode_tma_kernel<D, KM, VCVT, SC><<<grid, Cfg<D>::NT, smem, s>>>(p, tmk, tmv);
+  decode_tma_kernel<D, KM, VCVT, SC, DS><<<grid, Cfg<D, DS>::NT, smem, s>>>(p, tmk, tmv);
   return cudaGetLastError();
 }
 
@@ -2969,6 +3043,13 @@ static cudaError_t launch_decode_kv(const DecodeParams& p, const CUtensorMap& tm
     return launch_decode_d<D, 1, true, 2>(p, tmk, tmv, s);
   } else {
     if constexpr (SC == 0) {
+      if constexpr (D == 512) {
+        // the head-dim split (the host chose it and built half-width tensor maps)
+        if (p.dsplit == 2) {
+          if (k_mode != 1 || !v_cvt) return cudaErrorInvalidValue;
+          return launch_decode_d<D, 1, true, 0, 2>(p, tmk, tmv, s);
+        }
+      }
       if (k_mode == 3) return launch_decode_d<D, 3, true, 0>(p, tmk, tmv, s);
       if (k_mode == 2 && v_cvt) return launch_decode_d<D, 2, true, 0>(p, tmk, tmv, s);
     } else {
@@ -3026,18 +3107,18 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmk, const C
   }
 }
 
-template <int D>
+template <int D, int DS = 1>
 static int blocks_per_sm_d() {
   static std::atomic<int> cached{-1};
   int c = cached.load();
   if (c >= 0) return c;
   int n = 0;
-  if (cudaFuncSetAttribute(decode_tma_kernel<D, 1, true, 0>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tma_kernel<D, 1, true, 0>, Cfg<D>::NT,
-                                                    Cfg<D>::SMEM) != cudaSuccess) {
+  if (cudaFuncSetAttribute(decode_tma_kernel<D, 1, true, 0, DS>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, DS>::SMEM) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tma_kernel<D, 1, true, 0, DS>,
+                                                    Cfg<D, DS>::NT, Cfg<D, DS>::SMEM) != cudaSuccess) {
     cudaGetLastError();
-    return Cfg<D>::MIN_BLOCKS;  // no device: do not cache the guess
+    return Cfg<D, DS>::MIN_BLOCKS;  // no device: do not cache the guess
   }
   c = n > 0 ? n : 1;
   cached.store(c);
@@ -3070,32 +3151,32 @@ int decode_umma_blocks_per_sm(int D) {
   }
 }
 
-int decode_blocks_per_sm(int D) {
+int decode_blocks_per_sm(int D, int dsplit) {
   switch (D) {
     case 64: return blocks_per_sm_d<64>();
     case 128: return blocks_per_sm_d<128>();
     case 256: return blocks_per_sm_d<256>();
-    case 512: return blocks_per_sm_d<512>();
+    case 512: return dsplit == 2 ? blocks_per_sm_d<512, 2>() : blocks_per_sm_d<512>();
     default: return 1;
   }
 }
 
-int decode_warps_per_block(int D) {
+int decode_warps_per_block(int D, int dsplit) {
   switch (D) {
     case 64: return Cfg<64>::NW;
     case 128: return Cfg<128>::NW;
     case 256: return Cfg<256>::NW;
-    case 512: return Cfg<512>::NW;
+    case 512: return dsplit == 2 ? Cfg<512, 2>::NW : Cfg<512>::NW;
     default: return 4;
   }
 }
 
-int decode_smem_bytes(int D) {
+int decode_smem_bytes(int D, int dsplit) {
   switch (D) {
     case 64: return Cfg<64>::SMEM;
     case 128: return Cfg<128>::SMEM;
     case 256: return Cfg<256>::SMEM;
-    case 512: return Cfg<512>::SMEM;
+    case 512: return dsplit == 2 ? Cfg<512, 2>::SMEM : Cfg<512>::SMEM;
     default: return 0;
   }
 }

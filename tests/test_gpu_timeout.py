@@ -33,17 +33,21 @@ def F(cuda_device):
     F.fp8pd_check_errors()
 
 
-def _case(cuda_device, seq_len=64):
-    spec = W.Spec("stall", B=2, ps=16, layers=(W.LayerSpec(8, 1, 64, 0, 0.125),),
+def _case(cuda_device, seq_len=64, D=64):
+    spec = W.Spec("stall", B=2, ps=16, layers=(W.LayerSpec(8, 1, D, 0, 0.125),),
                   seq_len=seq_len, scale_mode="page", seed=91)
     return W.make_case(spec, cuda_device)
 
 
-def test_a_wait_that_runs_out_drops_that_warps_keys_and_sets_the_flag(F, cuda_device):
-    """One block per sequence (one split), 64 keys: warp w attends tile w, so
-    the stalled warp 0 of sequence 0's block drops keys 0..15. Sequence 0's
-    output is then attention over its last 48 keys; sequence 1 is untouched."""
-    case = _case(cuda_device)
+@pytest.mark.parametrize("D", [64, 512])
+def test_a_wait_that_runs_out_drops_that_warps_keys_and_sets_the_flag(F, cuda_device, D):
+    """One block per sequence (one split), 64 keys: tile stream w attends tile
+    w, so the stalled warp 0 of sequence 0's block drops keys 0..15. Sequence
+    0's output is then attention over its last 48 keys; sequence 1 is
+    untouched. At D = 512 stream 0 is two warps, each on half of the head dim:
+    the stalled warp's partner learns of the lost copy when the score halves
+    meet, and both leave the tile stream."""
+    case = _case(cuda_device, D=D)
     layer = case.layers[0]
     F.fp8pd_set_option(F.OPT_NUM_SPLITS, 1)
     F.fp8pd_set_option(F.OPT_SCHEDULE, 1)
@@ -56,6 +60,7 @@ def test_a_wait_that_runs_out_drops_that_warps_keys_and_sets_the_flag(F, cuda_de
     assert flags & ~F.FLAG_TIMEOUT == 0
     run = F.fp8pd_last_run_info()
     assert run["num_splits"] == 1 and run["schedule"] == 1
+    assert run["dim_split"] == (2 if D == 512 else 1)
     full = oracle_attention(layer, case.attend_lens)
     last48 = dataclasses.replace(layer, window=48)
     want0 = oracle_attention(last48, case.attend_lens)[0]
