@@ -220,13 +220,18 @@ bool use_umma(int D, bool tok, bool mx, int k_groups) {
   return k == 2 || kUmmaByDefault;
 }
 
-// Whether the split kernel runs a call with two warps per tile stream, each
-// on half of the head dim: D = 512 with page or head scales, f32 compute with
-// the hardware-cvt decodes and no fused append (at D = 512 a block of four
-// whole-width streams fills the SM's shared memory with four warps).
-bool use_dsplit(int D, bool tok, bool mx, int k_groups, bool append, bool umma) {
-  if (D != 512 || umma || tok || mx || k_groups > 1 || append) return false;
-  return g_opt_compute.load() == 0 && g_opt_k_decode.load() == 1 && g_opt_v_decode.load() == 1;
+// Warps per tile stream of the split kernel, each on its part of the head
+// dim: FP8PD_DSPLIT_D512 at D = 512 with page or head scales, f32 compute
+// with the hardware-cvt decodes and no fused append (at D = 512 a block of
+// four whole-width streams fills the SM's shared memory with four warps);
+// otherwise 1.
+int use_dsplit(int D, bool tok, bool mx, int k_groups, bool append, bool umma) {
+  static_assert(FP8PD_DSPLIT_D512 == 1 || FP8PD_DSPLIT_D512 == 2 || FP8PD_DSPLIT_D512 == 4,
+                "FP8PD_DSPLIT_D512: 1, 2 or 4");
+  if (D != 512 || umma || tok || mx || k_groups > 1 || append) return 1;
+  if (g_opt_compute.load() != 0 || g_opt_k_decode.load() != 1 || g_opt_v_decode.load() != 1)
+    return 1;
+  return FP8PD_DSPLIT_D512;
 }
 
 // Thread blocks one SM holds for the kernel that will run.
@@ -385,9 +390,10 @@ std::mutex g_map_mutex;
 std::vector<MapEntry> g_maps;  // small most-recently-used cache
 
 // The box is one 16-token tile of one KV head: whole rows, or with dsplit = 2
-// the first half of each row (the kernel moves the start to the second half).
+// or 4 the first half or quarter of each row (the kernel moves the start to
+// its own part).
 int make_pool_map(const fp8pd_tensor* pool, CUtensorMap* out, int dsplit = 1) {
-  if (dsplit != 2) dsplit = 1;
+  if (dsplit != 2 && dsplit != 4) dsplit = 1;
   MapKey key{pool->data, {}, {}, dsplit};
   for (int i = 0; i < 4; ++i) {
     key.shape[i] = pool->shape[i];
@@ -684,8 +690,7 @@ int run_decode(DecodeParams& p, const DecodeArgs& a, const fp8pd_tensor* k_pages
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   apply_plan(plan, &p);
   p.umma = um ? 1 : 0;
-  p.dsplit = use_dsplit(a.D, p.k_tok || p.v_tok, p.k_mx || p.v_mx, p.k_groups, p.append != 0, um)
-                 ? 2 : 1;
+  p.dsplit = use_dsplit(a.D, p.k_tok || p.v_tok, p.k_mx || p.v_mx, p.k_groups, p.append != 0, um);
   if (plan.combine) {
     void *ctr = nullptr, *part = nullptr;
     r = get_workspace(plan.counters_bytes, plan.workspace - plan.counters_bytes, s, &ctr, &part);
@@ -865,7 +870,7 @@ int fp8pd_plan(const fp8pd_tensor* q, const fp8pd_tensor* k_pages, const fp8pd_t
   info->workspace_bytes = plan.workspace;
   info->schedule = plan.schedule;
   // the tensor-memory kernel: 8 compute warps and the QK and PV issuing warps
-  const int ds = use_dsplit(static_cast<int>(D), false, false, 1, false, um) ? 2 : 1;
+  const int ds = use_dsplit(static_cast<int>(D), false, false, 1, false, um);
   info->warps = plan.grid_blocks * (um ? 10 : fp8pd::decode_warps_per_block(static_cast<int>(D), ds));
   return FP8PD_OK;
 }
@@ -1159,8 +1164,7 @@ extern "C" int fp8_paged_decode_attention_noalloc(
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   apply_plan(plan, &p);
   p.umma = um ? 1 : 0;
-  p.dsplit = use_dsplit(a.D, p.k_tok || p.v_tok, p.k_mx || p.v_mx, p.k_groups, p.append != 0, um)
-                 ? 2 : 1;
+  p.dsplit = use_dsplit(a.D, p.k_tok || p.v_tok, p.k_mx || p.v_mx, p.k_groups, p.append != 0, um);
   if (plan.combine) {
     void* ws = nullptr;
     r = noalloc_scratch(&ws);

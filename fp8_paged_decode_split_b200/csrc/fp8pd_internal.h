@@ -81,8 +81,9 @@ struct DecodeParams {
   // compute) runs this call
   int umma;
   // Warps sharing each tile stream of the split kernel, each on its part of
-  // the head dim: 1, or 2 at D = 512 (page or head scales, f32 compute with
-  // the cvt decodes, no fused append), where the tensor maps copy half rows.
+  // the head dim: 1, or 2 / 4 at D = 512 (page or head scales, f32 compute
+  // with the cvt decodes, no fused append), where the tensor maps copy half
+  // or quarter rows.
   int dsplit;
 };
 
@@ -129,8 +130,15 @@ cudaError_t launch_combine(const float* po, const float* pml, int R, int B, int 
 cudaError_t launch_encode(const float* x, int64_t xs, uint8_t* c, int64_t cs, int64_t n,
                           cudaStream_t s);
 
+// Warps per tile stream of the split kernel at D = 512 (1, 2 or 4) where a
+// call allows the head-dim split; a compile-time setting for tuning builds.
+// Two measured fastest: four repeat the softmax in every warp of a stream.
+#ifndef FP8PD_DSPLIT_D512
+#define FP8PD_DSPLIT_D512 2
+#endif
+
 // Thread blocks of the split kernel one SM holds for head dim D (dsplit: the
-// warps sharing each tile stream, 1 or 2).
+// warps sharing each tile stream, 1, 2 or 4).
 int decode_blocks_per_sm(int D, int dsplit = 1);
 // Thread blocks of the tensor-memory kernel one SM holds (D = 64 / 128; else 0).
 int decode_umma_blocks_per_sm(int D);

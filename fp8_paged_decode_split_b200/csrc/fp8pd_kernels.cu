@@ -358,13 +358,14 @@ __device__ __forceinline__ uint32_t tile_off(int r, int b) {
 
 // DS (head-dim split): each tile stream of a block is shared by DS warps,
 // warp h of the stream copying and contracting head-dim entries
-// [h * D / DS, (h + 1) * D / DS) of every tile (its own ring of half-width
+// [h * D / DS, (h + 1) * D / DS) of every tile (its own ring of part-width
 // tiles), the partial scores summed through shared memory once per tile.
-// DS = 2 is built for D = 512 only, where a block of four whole-width
+// DS = 2 and 4 are built for D = 512 only, where a block of four whole-width
 // streams fills the SM's shared memory with four warps.
 template <int D, int DS = 1>
 struct Cfg {
-  static_assert(DS == 1 || (DS == 2 && D == 512), "head-dim split: D = 512, two warps");
+  static_assert(DS == 1 || (D == 512 && (DS == 2 || DS == 4)),
+                "head-dim split: D = 512, two or four warps per stream");
   static constexpr int DW = D / DS;                                    // head-dim entries per warp
   static constexpr int NLW = (D == 64) ? FP8PD_NW_D64 : (D == 128) ? FP8PD_NW_D128 : (D == 256) ? FP8PD_NW_D256 : FP8PD_NW_D512;  // tile streams per block
   static constexpr int NW = NLW * DS;                                  // warps per block
@@ -377,7 +378,7 @@ struct Cfg {
   static constexpr int PIPE_BYTES = NW * WARP_BYTES;                  // multiple of 1024
   static constexpr bool Q_IN_SMEM = (D > 256);                        // q fragments in smem
   static constexpr int QFRAG_BYTES = Q_IN_SMEM ? (D / 16) * 32 * 8 : 0;
-  // per stream, two buffers of the DS warps' score fragments (float4 per lane) and their flags
+  // per stream, two buffers of the DS warps' score parts (float4 per lane) and their flags
   static constexpr int XCH_BYTES = DS > 1 ? NLW * 2 * DS * (32 * 16 + 16) : 0;
   static constexpr int LIST_BYTES = NLW * kMaxWarpTiles * 12;         // tile entry, k / v scale
   static constexpr int BAR_BYTES = NW * NS * 8;
@@ -1867,12 +1868,12 @@ __global__ void __launch_bounds__(Cfg<D, DS>::NT, Cfg<D, DS>::MIN_BLOCKS)
     }
   }
   if constexpr (DS > 1) {
-    // Head-dim split: each warp of the stream waits for its own half-width
-    // tile, contracts its part of S, and the two parts (and whether each
-    // copy arrived) meet in shared memory, so both warps run the same
+    // Head-dim split: each warp of the stream waits for its own part-width
+    // tile, contracts its part of S, and the parts (and whether each copy
+    // arrived) meet in shared memory, so all the stream's warps run the same
     // softmax on the same scores and leave the loop together; then each
     // accumulates its own head-dim part of O. The copy into the previous
-    // stage is issued once both have decided to go on.
+    // stage is issued once all have decided to go on.
     int* s_xok = reinterpret_cast<int*>(s_xch + C::NLW * 2 * DS * 32);
 #pragma unroll 1
     for (int j = 0; ok_all && j < my_tiles; ++j, tok0 += C::NLW * kTileTokens) {
@@ -1890,13 +1891,24 @@ __global__ void __launch_bounds__(Cfg<D, DS>::NT, Cfg<D, DS>::MIN_BLOCKS)
       s_xch[(xb + half) * 32 + lane] = sc;
       if (lane == 0) s_xok[xb + half] = got ? 1 : 0;
       stream_sync();
-      const float4 o = s_xch[(xb + (half ^ 1)) * 32 + lane];
-      if (!got || s_xok[xb + (half ^ 1)] == 0) {
+      bool all_got = true;
+#pragma unroll
+      for (int h = 0; h < DS; ++h) all_got = all_got && s_xok[xb + h] != 0;
+      if (!all_got) {
         ok_all = false;
         break;
       }
-      // a + b == b + a: both warps hold the same sums
-      sc = make_float4(sc.x + o.x, sc.y + o.y, sc.z + o.z, sc.w + o.w);
+      // the parts summed in the same order by every warp of the stream, so
+      // all of them hold the same scores (masked entries are -inf in every part)
+      {
+        float4 t = (half == 0) ? sc : s_xch[xb * 32 + lane];
+#pragma unroll
+        for (int h = 1; h < DS; ++h) {
+          const float4 o = (h == half) ? sc : s_xch[(xb + h) * 32 + lane];
+          t = make_float4(t.x + o.x, t.y + o.y, t.z + o.z, t.w + o.w);
+        }
+        sc = t;
+      }
       {
         const int nj = j + C::NS - 1;
         if (nj < my_tiles) issue(went[nj], stage == 0 ? C::NS - 1 : stage - 1);
@@ -3043,11 +3055,11 @@ static cudaError_t launch_decode_kv(const DecodeParams& p, const CUtensorMap& tm
     return launch_decode_d<D, 1, true, 2>(p, tmk, tmv, s);
   } else {
     if constexpr (SC == 0) {
-      if constexpr (D == 512) {
-        // the head-dim split (the host chose it and built half-width tensor maps)
-        if (p.dsplit == 2) {
-          if (k_mode != 1 || !v_cvt) return cudaErrorInvalidValue;
-          return launch_decode_d<D, 1, true, 0, 2>(p, tmk, tmv, s);
+      if constexpr (D == 512 && FP8PD_DSPLIT_D512 > 1) {
+        // the head-dim split (the host chose it and built part-width tensor maps)
+        if (p.dsplit > 1) {
+          if (p.dsplit != FP8PD_DSPLIT_D512 || k_mode != 1 || !v_cvt) return cudaErrorInvalidValue;
+          return launch_decode_d<D, 1, true, 0, FP8PD_DSPLIT_D512>(p, tmk, tmv, s);
         }
       }
       if (k_mode == 3) return launch_decode_d<D, 3, true, 0>(p, tmk, tmv, s);
@@ -3156,7 +3168,7 @@ int decode_blocks_per_sm(int D, int dsplit) {
     case 64: return blocks_per_sm_d<64>();
     case 128: return blocks_per_sm_d<128>();
     case 256: return blocks_per_sm_d<256>();
-    case 512: return dsplit == 2 ? blocks_per_sm_d<512, 2>() : blocks_per_sm_d<512>();
+    case 512: return dsplit > 1 ? blocks_per_sm_d<512, FP8PD_DSPLIT_D512>() : blocks_per_sm_d<512>();
     default: return 1;
   }
 }
@@ -3166,7 +3178,7 @@ int decode_warps_per_block(int D, int dsplit) {
     case 64: return Cfg<64>::NW;
     case 128: return Cfg<128>::NW;
     case 256: return Cfg<256>::NW;
-    case 512: return dsplit == 2 ? Cfg<512, 2>::NW : Cfg<512>::NW;
+    case 512: return dsplit > 1 ? Cfg<512, FP8PD_DSPLIT_D512>::NW : Cfg<512>::NW;
     default: return 4;
   }
 }
@@ -3176,7 +3188,7 @@ int decode_smem_bytes(int D, int dsplit) {
     case 64: return Cfg<64>::SMEM;
     case 128: return Cfg<128>::SMEM;
     case 256: return Cfg<256>::SMEM;
-    case 512: return dsplit == 2 ? Cfg<512, 2>::SMEM : Cfg<512>::SMEM;
+    case 512: return dsplit > 1 ? Cfg<512, FP8PD_DSPLIT_D512>::SMEM : Cfg<512>::SMEM;
     default: return 0;
   }
 }

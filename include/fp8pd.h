@@ -436,8 +436,9 @@ typedef struct fp8pd_run_info {
   int32_t compute;           /* FP8PD_OPT_COMPUTE of the last attention call (0 f32, 1 fp8) */
   int32_t kernel;            /* kernel of the last attention call: 1 split, 2 tensor-memory */
   int32_t dim_split;         /* warps sharing each tile stream of the split kernel, each on its
-                                part of the head dim: 1, or 2 at head_dim 512 with page or head
-                                scales, f32 compute, the cvt decodes and no fused append */
+                                part of the head dim: 1, or (a build setting, 2 or 4) at
+                                head_dim 512 with page or head scales, f32 compute, the cvt
+                                decodes and no fused append */
 } fp8pd_run_info;
 int fp8pd_last_run_info(fp8pd_run_info* info);
 
