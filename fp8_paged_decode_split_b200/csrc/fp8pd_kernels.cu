@@ -338,6 +338,14 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
 #ifndef FP8PD_NW_D512
 #define FP8PD_NW_D512 4
 #endif
+// Tile streams and ring stages of the D = 512 head-dim split (its warps are
+// streams x split; the rings hold the same 192 KiB as the whole-width shape).
+#ifndef FP8PD_NW_D512_SPLIT
+#define FP8PD_NW_D512_SPLIT 6
+#endif
+#ifndef FP8PD_NS_D512_SPLIT
+#define FP8PD_NS_D512_SPLIT 2
+#endif
 
 // ---------------------------------------------------------------------------
 // Shared-memory tile layout. The TMA writes one 16-token tile of one KV head
@@ -367,10 +375,10 @@ struct Cfg {
   static_assert(DS == 1 || (D == 512 && (DS == 2 || DS == 4)),
                 "head-dim split: D = 512, two or four warps per stream");
   static constexpr int DW = D / DS;                                    // head-dim entries per warp
-  static constexpr int NLW = (D == 64) ? FP8PD_NW_D64 : (D == 128) ? FP8PD_NW_D128 : (D == 256) ? FP8PD_NW_D256 : FP8PD_NW_D512;  // tile streams per block
+  static constexpr int NLW = (D == 64) ? FP8PD_NW_D64 : (D == 128) ? FP8PD_NW_D128 : (D == 256) ? FP8PD_NW_D256 : (DS > 1) ? FP8PD_NW_D512_SPLIT : FP8PD_NW_D512;  // tile streams per block
   static constexpr int NW = NLW * DS;                                  // warps per block
   static constexpr int NT = NW * 32;                                  // threads per block
-  static constexpr int NS = (D == 64) ? FP8PD_NS_D64 : (D == 128) ? FP8PD_NS_D128 : (D == 256) ? FP8PD_NS_D256 : FP8PD_NS_D512;  // ring stages per warp
+  static constexpr int NS = (D == 64) ? FP8PD_NS_D64 : (D == 128) ? FP8PD_NS_D128 : (D == 256) ? FP8PD_NS_D256 : (DS > 1) ? FP8PD_NS_D512_SPLIT : FP8PD_NS_D512;  // ring stages per warp
   static constexpr bool PAIR = (D == 64) && FP8PD_PAIR_D64;           // two tiles per softmax step
   static constexpr int TILE = kTileTokens * DW;                       // bytes of a warp's K or V tile
   static constexpr int STAGE = 2 * TILE;
@@ -389,6 +397,7 @@ struct Cfg {
   static_assert(PIPE_BYTES % 1024 == 0, "tiles must stay 1024-byte aligned for the swizzle");
   static_assert(DW % 128 == 0 || DS == 1, "a warp's part of a row is whole 128-byte blocks");
   static_assert(NLW * 8 * D * 4 <= PIPE_BYTES, "merge scratch must fit in the ring");
+  static_assert(NLW * kMaxWarpTiles >= kMaxSplitTiles, "a split's tiles fit the streams' lists");
   static_assert(8 * 32 * 4 <= PIPE_BYTES, "merge weights must fit in the ring");
   static_assert(SMEM <= 232448, "shared memory per block");
 };
