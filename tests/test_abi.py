@@ -335,6 +335,19 @@ def test_planner_plans_for_the_kernel_that_runs(F):
         F.fp8pd_set_option(F.OPT_KERNEL, 0)
 
 
+def test_planner_counts_the_head_dim_split_warps(F):
+    """At head dim 512 (page or head scales, the default f32 compute and
+    decodes) a tile stream is two warps, each on half of the head dim: the
+    plan's warps are a multiple of twice its blocks and more than the four
+    whole-width warps per block; other head dims keep four warps per block."""
+    d512 = _plan(F, 16, 16, 2, 512, 32, 513)
+    wpb, rem = divmod(d512["warps"], d512["grid_blocks"])
+    assert rem == 0 and wpb % 2 == 0 and wpb > 4
+    for D in (64, 128, 256):
+        p = _plan(F, 8, 16, 2, D, 32, 200)
+        assert p["warps"] == p["grid_blocks"] * 4, D
+
+
 def test_partial_and_combine_validation(F):
     """The context-parallel entry points refuse bad arguments before any
     launch: the partial call as the attention call plus its own outputs and
