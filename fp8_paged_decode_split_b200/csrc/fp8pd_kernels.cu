@@ -14,13 +14,13 @@
 //
 // Design on B200:
 // * One thread block = one (sequence b, KV head h, group of <= 8 query
-//   heads, split of the key range). Its 4 warps take 16-token tiles of the
-//   split round robin; each warp streams its tiles HBM -> shared memory with
-//   TMA (one cp.async.bulk.tensor per K or V tile, issued by one lane, no
-//   multicast) into a private multi-stage ring completed on mbarriers (no
-//   block-wide barrier in the main loop) and keeps its own online-softmax
-//   state (at head dim 64, two tiles per softmax step). The warps are
-//   merged once at the end; when the keys are split over several blocks the
+//   heads, split of the key range). Its tile streams (4 warps; at D = 512 6
+//   pairs, each warp on half the head dim) take 16-token tiles round robin;
+//   each warp copies its tiles with TMA (one cp.async.bulk.tensor per K or V
+//   tile, one lane, no multicast) into a private ring on mbarriers (no
+//   block-wide barrier in the main loop); a stream keeps its own online-
+//   softmax state (at head dim 64, two tiles per softmax step). The streams
+//   are merged once at the end; when the keys are split over several blocks the
 //   last block of a (sequence, KV head, head group) to finish merges the
 //   splits (a ticket counter, never a wait), so one launch does the call.
 // * QK and PV are tensor-core contractions (mma.sync m16n8k16, f16 inputs,
@@ -800,14 +800,20 @@ __device__ __forceinline__ void tile_pv(Acc<D>& a, uint32_t sv, const uint32_t (
                                         bool vmx = false, const uint32_t* vmw = nullptr,
                                         int E = 0) {
   uint32_t wa0 = 0u, wa1 = 0u, wb0 = 0u, wb1 = 0u;
-  uint32_t vmask_lo = ~0u, vmask_hi = ~0u;
+  // Byte permutes of the transposed words into token pairs per column
+  // (0x3120). With the hardware cvt a masked row must be zeroed (a NaN byte
+  // times P = 0 would still be NaN): its bytes (0-1: token 2q, 2-3: token
+  // 2q+1 of the word) are taken from the zero word instead (selector 4).
+  uint32_t sel_lo = 0x3120u, sel_hi = 0x3120u;
   if (VCVT && !full) {
-    // with the hardware cvt a masked row must be zeroed (a NaN byte times
-    // P = 0 would still be NaN); bytes 0-1 / 2-3 are tokens 2q / 2q+1
     const int r = tok0 + 2 * qd;
     auto in = [&](int t) { return page_ok && t >= t0 && t < t1; };
-    vmask_lo = (in(r) ? 0x0000FFFFu : 0u) | (in(r + 1) ? 0xFFFF0000u : 0u);
-    vmask_hi = (in(r + 8) ? 0x0000FFFFu : 0u) | (in(r + 9) ? 0xFFFF0000u : 0u);
+    auto sel = [](bool a, bool b) -> uint32_t {
+      return (a ? 0x0u : 0x4u) | ((b ? 0x2u : 0x4u) << 4) | ((a ? 0x1u : 0x4u) << 8) |
+             ((b ? 0x3u : 0x4u) << 12);
+    };
+    sel_lo = sel(in(r), in(r + 1));
+    sel_hi = sel(in(r + 8), in(r + 9));
   }
 #pragma unroll
   for (int jb = 0; jb < D / 32; ++jb) {
@@ -815,8 +821,8 @@ __device__ __forceinline__ void tile_pv(Acc<D>& a, uint32_t sv, const uint32_t (
     uint32_t a0, a1, a2, a3, e0, e1, e2, e3;
     if constexpr (VCVT) {
       // [t.d, t'.d, t.d+1, t'.d+1]: each 16-bit half is one column's token pair
-      const uint32_t z0 = prmt(vw.x & vmask_lo, 0, 0x3120), z1 = prmt(vw.y & vmask_lo, 0, 0x3120);
-      const uint32_t z2 = prmt(vw.z & vmask_hi, 0, 0x3120), z3 = prmt(vw.w & vmask_hi, 0, 0x3120);
+      const uint32_t z0 = prmt(vw.x, 0, sel_lo), z1 = prmt(vw.y, 0, sel_lo);
+      const uint32_t z2 = prmt(vw.z, 0, sel_hi), z3 = prmt(vw.w, 0, sel_hi);
       a0 = e4m3x2_lo16_to_f16x2(z0);
       a1 = e4m3x2_hi16_to_f16x2(z0);
       a2 = e4m3x2_lo16_to_f16x2(z2);
