@@ -158,3 +158,27 @@ def test_both_arms_state_the_same_config():
     ours = bench._config_dict(Args, "llama", nbytes=bench._step_bytes(case))
     ref = bench._config_dict(Args, "llama")
     assert ours == ref
+
+
+def test_traffic_is_reported_only_for_the_current_kernel_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu summary only while its
+    line carries the current kernel source hash; a layer index selects the
+    workload's per-layer line; anything else reads as unmeasured (None)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    h = bench._kernel_source_hash()
+    assert len(h) == 16 and int(h, 16) >= 0
+    f = tmp_path / "traffic.txt"
+    f.write_text("# comment line\n"
+                 f"long_b8 {h} 2163911936\n"
+                 f"mixed {h} 69356288\n"
+                 f"mixed:1 {h} 360100864\n"
+                 "llama 0000000000000000 153228288\n")
+    monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(f))
+    assert bench._traffic("long_b8") == 2163911936
+    assert bench._traffic("mixed") == 69356288
+    assert bench._traffic("mixed", 1) == 360100864
+    assert bench._traffic("llama") is None            # taken on another source
+    assert bench._traffic("gptoss_full") is None      # never taken
+    monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(tmp_path / "missing.txt"))
+    assert bench._traffic("long_b8") is None
